@@ -1,0 +1,167 @@
+"""CPU fp64 oracle for Kimi Delta Attention (KDA).
+
+TEST INFRASTRUCTURE ONLY. The tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` are the only callers allowed; the product
+library never imports this package and this package never imports the
+product library.
+
+Two independently written C implementations back it (compiled on first use
+with the host C compiler, or ahead of time by ``build()``):
+
+* ``recurrent`` -- form R, the token-by-token recurrence of page
+  "atlas_core/kimi_k3/kda.rs" (module doc and ``kda_recurrent_step``): the
+  definition, written out.
+* ``chunkwise`` -- form C, the chunk-at-a-time WY/UT form that the
+  ``chunk_kda`` boundary of page "K3/kda/ops/api.py" computes, derived here
+  from the same recurrence. It exists to cross-check form R.
+
+Both take packed inputs: q, k, g of shape [T_total, H, d_k], v of shape
+[T_total, H, d_v], beta logits [T_total, H], ``cu_seqlens`` int offsets
+[N+1] (sequence n is tokens cu_seqlens[n]..cu_seqlens[n+1]), and optional
+initial states [N, H, d_k, d_v] (row = key channel). Inputs of any float
+dtype are widened exactly to fp64; results come back as fp64 numpy arrays.
+A [B, T, H, D] batch is the same thing with cu_seqlens = [0, T, 2T, ...].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SOURCES = ("kda_recurrent.c", "kda_chunkwise.c")
+_LIB_PATH = os.path.join(_HERE, "libkda_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle's C sources into ``oracle/libkda_oracle.so``."""
+    srcs = [os.path.join(_HERE, s) for s in _SOURCES]
+    if not force and os.path.exists(_LIB_PATH):
+        newest = max(os.path.getmtime(s) for s in srcs)
+        if os.path.getmtime(_LIB_PATH) >= newest:
+            return _LIB_PATH
+    tmp = _LIB_PATH + ".tmp%d" % os.getpid()
+    # IEEE semantics are part of the definition (sigmoid(-inf) = 0, exp(-inf) = 0),
+    # so no fast-math.
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+           "-Wall", "-Wextra", "-o", tmp, *srcs, "-lm", "-lpthread"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            dp = ctypes.POINTER(ctypes.c_double)
+            i64p = ctypes.POINTER(ctypes.c_int64)
+            common = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, i64p,
+                      dp, dp, dp, dp, dp, ctypes.c_double, dp, dp, dp,
+                      ctypes.c_int, ctypes.c_int, ctypes.c_double]
+            lib.kda_oracle_recurrent.argtypes = common + [ctypes.c_int]
+            lib.kda_oracle_recurrent.restype = ctypes.c_int
+            lib.kda_oracle_chunkwise.argtypes = common + [ctypes.c_int, ctypes.c_int]
+            lib.kda_oracle_chunkwise.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # a torch tensor; bf16 -> fp64 is exact
+        import torch
+        x = x.detach().to("cpu", torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _prep(q, k, v, g, beta, cu_seqlens, initial_state):
+    q, k, v, g, beta = (_f64(t) for t in (q, k, v, g, beta))
+    if q.ndim == 4:  # [B, T, H, D] -> packed
+        B, T = q.shape[:2]
+        if cu_seqlens is not None and B != 1:
+            raise ValueError("cu_seqlens needs B == 1")
+        if cu_seqlens is None:
+            cu_seqlens = np.arange(B + 1, dtype=np.int64) * T
+        q, k, v, g = (t.reshape(B * T, *t.shape[2:]) for t in (q, k, v, g))
+        beta = beta.reshape(B * T, -1)
+    Ttot, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if cu_seqlens is None:
+        cu_seqlens = np.array([0, Ttot], dtype=np.int64)
+    if hasattr(cu_seqlens, "detach"):
+        cu_seqlens = cu_seqlens.detach().cpu().numpy()
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    N = cu.size - 1
+    if cu[0] != 0 or cu[-1] != Ttot or np.any(np.diff(cu) < 0):
+        raise ValueError("cu_seqlens must start at 0, be non-decreasing and end at T_total")
+    for name, t, shp in (("k", k, (Ttot, H, Dk)), ("v", v, (Ttot, H, Dv)),
+                         ("g", g, (Ttot, H, Dk)), ("beta", beta, (Ttot, H))):
+        if t.shape != shp:
+            raise ValueError(f"{name} has shape {t.shape}, expected {shp}")
+    S0 = _f64(initial_state)
+    if S0 is not None and S0.shape != (N, H, Dk, Dv):
+        raise ValueError(f"initial_state has shape {S0.shape}, expected {(N, H, Dk, Dv)}")
+    return q, k, v, g, beta, cu, S0, N, H, Dk, Dv
+
+
+def _threads(nthreads):
+    if nthreads and nthreads > 0:
+        return int(nthreads)
+    return os.cpu_count() or 1
+
+
+def recurrent(q, k, v, g, beta, *, scale=None, initial_state=None, cu_seqlens=None,
+              use_qk_l2norm=True, lower_bound=None, nthreads=0):
+    """Form R (the definition). Returns (o [T_total,H,d_v], final_state [N,H,d_k,d_v]).
+
+    ``beta`` holds logits (sigmoid applied per token), ``g`` holds per-channel
+    log-decays, ``lower_bound`` clamps g from below, ``scale`` defaults to
+    1/sqrt(d_k).
+    """
+    q, k, v, g, beta, cu, S0, N, H, Dk, Dv = _prep(q, k, v, g, beta, cu_seqlens, initial_state)
+    if scale is None:
+        scale = 1.0 / np.sqrt(Dk)
+    o = np.zeros((q.shape[0], H, Dv))
+    S = np.zeros((N, H, Dk, Dv))
+    rc = _load().kda_oracle_recurrent(
+        N, H, Dk, Dv, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(S0), _ptr(o), _ptr(S),
+        int(bool(use_qk_l2norm)), int(lower_bound is not None),
+        float(lower_bound if lower_bound is not None else 0.0), _threads(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"kda_oracle_recurrent failed ({rc})")
+    return o, S
+
+
+def chunkwise(q, k, v, g, beta, *, scale=None, initial_state=None, cu_seqlens=None,
+              use_qk_l2norm=True, lower_bound=None, chunk_size=64, nthreads=0):
+    """Form C (chunkwise WY/UT). Same arguments and results as ``recurrent``."""
+    q, k, v, g, beta, cu, S0, N, H, Dk, Dv = _prep(q, k, v, g, beta, cu_seqlens, initial_state)
+    if scale is None:
+        scale = 1.0 / np.sqrt(Dk)
+    o = np.zeros((q.shape[0], H, Dv))
+    S = np.zeros((N, H, Dk, Dv))
+    rc = _load().kda_oracle_chunkwise(
+        N, H, Dk, Dv, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(S0), _ptr(o), _ptr(S),
+        int(bool(use_qk_l2norm)), int(lower_bound is not None),
+        float(lower_bound if lower_bound is not None else 0.0), int(chunk_size),
+        _threads(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"kda_oracle_chunkwise failed ({rc})")
+    return o, S
