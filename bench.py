@@ -1,0 +1,415 @@
+"""Benchmark: KDA chunk forward tokens/s and decode steps/s on B200, with the
+roofline fraction of the dominant kernel and the CPU oracle beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
+
+One timed step = one `chunk_kda` forward over the varlen workload (4 packed
+sequences of 4096/8192/12288/7168 tokens, H = 96, d_k = d_v = 128, bf16
+inputs, fp32 states, lower bound -5, per-sequence initial states, final
+states out). The decode step workload (64 sequences x 96 heads x 128 x 128
+fp32 state, bf16 token vectors, one fresh token per step) is timed in the
+same run, K' = 256 steps per timed pass, and reported under "decode".
+Inputs are resident in HBM and larger than L2 (3.9 GB chunk inputs, 384 MiB
+decode state), so no L2 flush runs between iterations.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own replica of
+the workload (no data-path collective; weak scaling); the timed region is
+bracketed by barriers and the slowest rank's device time is reported.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workload on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "chunk_kda fwd tokens/s & decode steps/s on 1 B200; % of tensor/HBM roofline"
+CHUNK_WL = 4
+DECODE_WL = 3
+DECODE_STEPS_PER_PASS = 256
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def chunk_algorithmic(wl):
+    """Algorithmic bytes and flops of one chunk forward launch.
+
+    Per token-head: q, k, v, g, o (5 x 128 x 2 B) + beta (2 B) = 1282 B; plus
+    one read of the initial and one write of the final fp32 state per
+    (sequence, head). Flops per token-head (triangles exploited): A_kk, A_qk,
+    W, U, A_qk.Delta = 3 C d_k + 2 C d_v, state terms W.S, Q.S, K^T.Delta =
+    6 d_k d_v.
+    """
+    th = wl.tokens * wl.H
+    esz = 2
+    per_th = (3 * wl.Dk + 2 * wl.Dv) * esz + esz
+    states = wl.n_seqs * wl.H * wl.Dk * wl.Dv * 4 * (int(wl.init_state) + int(wl.final_state))
+    C = wl.chunk_size
+    flops = th * (3 * C * wl.Dk + 2 * C * wl.Dv + 6 * wl.Dk * wl.Dv)
+    return th * per_th + states, flops
+
+
+def decode_algorithmic(wl):
+    """Bytes and flops of one decode step: fp32 state read + write, q/k/g/v/o
+    vectors and one beta per head; 7 d_k d_v flops per head."""
+    heads = wl.N * wl.H
+    per_head = 2 * wl.Dk * wl.Dv * 4 + (3 * wl.Dk + 2 * wl.Dv) * 2 + 2
+    return heads * per_head, heads * 7 * wl.Dk * wl.Dv
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def source_sha(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "kimi_delta_attention_20_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(key, sha):
+    """DRAM bytes per launch recorded from an ncu capture of this exact kernel
+    source (profiles/ncu_traffic.json), else None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+            rec = json.load(f)[key]
+        return rec["bytes_per_launch"] if rec.get("source_sha") == sha else None
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def run_kda(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import kda_inputs as KI
+    import kimi_delta_attention_20_b200 as kda
+    from kimi_delta_attention_20_b200 import _abi
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    hbm_peak, tc_peak, peak_kind = load_peaks()
+
+    wl = KI.CHUNK_WORKLOADS[CHUNK_WL]
+    inp = KI.chunk_inputs(wl, device=dev)
+    q, k, v, g, beta = (inp[n] for n in ("q", "k", "v", "g", "beta"))
+    S0, cu = inp["initial_state"], inp["cu_seqlens"]
+    o = torch.empty_like(v)
+    S_out = torch.empty_like(S0)
+    ws_bytes = kda.chunk_workspace_bytes(1, wl.T, wl.H, wl.Dk, wl.Dv, N=wl.n_seqs, varlen=True)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+
+    def chunk_step():
+        kda.chunk_kda(q, k, v, g, beta, initial_state=S0, output_final_state=True,
+                      use_qk_l2norm_in_kernel=True, lower_bound=wl.lower_bound,
+                      cu_seqlens=cu, out=o, final_state_out=S_out, workspace=ws)
+
+    dwl = KI.DECODE_WORKLOADS[DECODE_WL]
+    dinp = KI.decode_inputs(dwl, device=dev)
+    state = dinp["state"].clone()
+    od = torch.empty(dwl.N, dwl.H, dwl.Dv, dtype=dwl.dtype, device=dev)
+
+    def decode_step(t):
+        kda.recurrent_step(dinp["q"][t], dinp["k"][t], dinp["v"][t], dinp["g"][t],
+                           dinp["beta"][t], state, out=od)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    stream = torch.cuda.current_stream(dev)
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[local_rank]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local_rank
+
+    # warm-up (untimed)
+    for _ in range(args.warmup):
+        chunk_step()
+    for t in range(min(args.warmup, dwl.steps)):
+        decode_step(t)
+    torch.cuda.synchronize(dev)
+
+    with ClockSampler(gpu_index) as clocks:
+        # chunk forward: K timed steps
+        barrier(); torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            chunk_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev); barrier()
+        chunk_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+
+        # decode: K passes of 256 steps each
+        state.copy_(dinp["state"])
+        barrier(); torch.cuda.synchronize(dev)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        nsteps = 0
+        for _ in range(args.steps):
+            for t in range(DECODE_STEPS_PER_PASS):
+                decode_step(t % dwl.steps)
+                nsteps += 1
+        d1.record(stream)
+        torch.cuda.synchronize(dev); barrier()
+        dec_ms = max_over_ranks(d0.elapsed_time(d1)) / nsteps
+    clk = clocks.summary()
+
+    # end to end through the public API with host buffers: pinned host inputs
+    # copied in, the chunk forward, outputs copied back, every step
+    host = {n: inp[n].cpu().pin_memory() for n in ("q", "k", "v", "g", "beta", "initial_state")}
+    h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    h_S = torch.empty(S_out.shape, dtype=S_out.dtype).pin_memory()
+    cu_host = cu.cpu()
+    h2d = sum(t.numel() * t.element_size() for t in host.values()) + cu_host.numel() * 4
+    d2h = o.numel() * o.element_size() + S_out.numel() * 4
+    dbuf = {n: torch.empty_like(inp[n]) for n in host}
+
+    def e2e_step():
+        for n in host:
+            dbuf[n].copy_(host[n], non_blocking=True)
+        cu_d = cu_host.to(dev, non_blocking=True)
+        oo, ss = kda.chunk_kda(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"],
+                               initial_state=dbuf["initial_state"], output_final_state=True,
+                               use_qk_l2norm_in_kernel=True, lower_bound=wl.lower_bound,
+                               cu_seqlens=cu_d, workspace=ws)
+        h_o.copy_(oo, non_blocking=True)
+        h_S.copy_(ss, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e2e_steps = max(1, min(args.steps, 3))
+    barrier(); torch.cuda.synchronize(dev)
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    x1.record(stream)
+    torch.cuda.synchronize(dev); barrier()
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1)) / e2e_steps
+
+    chunk_bytes, chunk_flops = chunk_algorithmic(wl)
+    dec_bytes, dec_flops = decode_algorithmic(dwl)
+    chunk_gbs = chunk_bytes / (chunk_ms * 1e-3) / 1e9
+    chunk_tflops = chunk_flops / (chunk_ms * 1e-3) / 1e12
+    dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
+    tc_used = os.path.exists(os.path.join(ROOT, "kimi_delta_attention_20_b200", "csrc",
+                                          "kda_chunk_tc.cu"))
+    chunk_sha = source_sha("kda_chunk_tc.cu", "kda_chunk_simt.cu", "kda_common.cuh") if tc_used else None
+    result = {
+        "metric": METRIC,
+        "value": world * wl.tokens / (chunk_ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": chunk_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; shapes and distributions of the varlen chunk and decode workloads)",
+        "config": {
+            "workload": "chunk_kda fwd: varlen 4096/8192/12288/7168 (T=31744), H=96, d_k=d_v=128, "
+                        "bf16, lower_bound=-5, chunk 64, initial+final states; decode: N=64, H=96, "
+                        "d=128, fp32 state, 256 steps per pass",
+            "tokens_per_step": wl.tokens, "heads": wl.H, "d_k": wl.Dk, "d_v": wl.Dv,
+            "chunk_size": wl.chunk_size, "parallelism": f"replica per GPU x{world} (no collective)",
+            "l2": "inputs larger than L2 (3.9 GB chunk inputs, 384 MiB decode state); no flush",
+        },
+        "roofline": {
+            "bound": "hbm", "achieved": chunk_gbs, "peak": hbm_peak, "unit": "GB/s",
+            "frac": chunk_gbs / hbm_peak, "peak_kind": peak_kind,
+            "algorithmic_bytes_per_launch": chunk_bytes,
+            "traffic": ncu_traffic("chunk", chunk_sha),
+            "tensor": {"achieved_tflops": chunk_tflops, "peak_tflops": tc_peak,
+                       "frac": chunk_tflops / tc_peak},
+        },
+        "decode": {
+            "value": world / (dec_ms * 1e-3), "unit": "steps/s",
+            "tokens_per_s": world * dwl.N / (dec_ms * 1e-3), "ms_per_step": dec_ms,
+            "steps_timed": nsteps,
+            "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": dec_gbs / hbm_peak, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": dec_bytes,
+                         "traffic": ncu_traffic("decode", source_sha("kda_decode.cu",
+                                                                     "kda_common.cuh"))},
+        },
+        "e2e": {"value": world * wl.tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps * (1 + DECODE_STEPS_PER_PASS),
+        "clocks": clk,
+        "library": os.path.relpath(_abi.LIB_PATH, ROOT),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(inp, wl)
+    return result
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(inp, wl, heads=24):
+    """Time the fp64 oracle (form R, as it stands) on a bounded sample of the
+    chunk workload: all four sequences, the first `heads` heads."""
+    import oracle
+    nthreads = os.cpu_count() or 1
+    sl = lambda x: x[0][:, :heads].cpu()
+    q, k, v, g, beta = (sl(inp[n]) for n in ("q", "k", "v", "g", "beta"))
+    S0 = inp["initial_state"][:, :heads].cpu()
+    cu = inp["cu_seqlens"].cpu()
+    t0 = time.perf_counter()
+    oracle.recurrent(q, k, v, g, beta, initial_state=S0, cu_seqlens=cu,
+                     lower_bound=wl.lower_bound, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    tok_heads = wl.tokens * heads
+    return {"value": tok_heads / wl.H / dt, "unit": "tokens/s", "cores": nthreads,
+            "kind": "oracle",
+            "sample": f"fp64 form R on all {wl.n_seqs} sequences ({wl.tokens} tokens) x {heads} of "
+                      f"{wl.H} heads; {tok_heads} token-heads in {dt:.1f} s, scaled to tokens of "
+                      f"all {wl.H} heads"}
+
+
+def run_reference(args):
+    import kda_inputs as KI
+    wl = KI.CHUNK_WORKLOADS[CHUNK_WL]
+    heads = 4
+    # the same recipe (lengths, dims, dtype, distributions) drawn for `heads` heads only,
+    # so the host does not materialise the 96-head tensors
+    inp = KI.draw_chunk(1, wl.T, heads, wl.Dk, wl.Dv, dtype=wl.dtype, seed=wl.seed,
+                        seqlens=wl.seqlens, init_state=True)
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state; warm-up steps are no-ops
+    vals = []
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(inp, wl, heads=heads))
+    v = statistics.median(x["value"] for x in vals)
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": wl.tokens / v * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "chunk_kda fwd: varlen 4096/8192/12288/7168, H=96, d=128, "
+                               "lower_bound=-5 (CPU oracle on a 4-head sample per step)"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["cores"],
+                         "kind": "oracle", "sample": vals[0]["sample"]},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "kda":
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_kda(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,140 @@
+/*
+ * kda.h -- C ABI of the Kimi Delta Attention (KDA) library for NVIDIA B200
+ * (sm_100a). Plain pointers and sizes only; no C++ or framework types.
+ *
+ * The operator (page "atlas_core/kimi_k3/kda.rs", module doc and
+ * `kda_recurrent_step`): per sequence and head, a state S of d_k x d_v fp32
+ * values (row = key channel) evolves token by token as
+ *     S     <- diag(exp(g_t)) S                 (decay on the key axis)
+ *     delta <- sigmoid(beta_t) (v_t - S^T k_t)  (beta_t is a logit)
+ *     S     <- S + k_t delta^T
+ *     o_t   <- scale S^T q_t
+ * with q_t, k_t optionally L2-normalised first as x / sqrt(sum x^2 + 1e-6)
+ * (same page, `l2norm_rows`, `KDA_L2_EPS`) and g_t optionally clamped from
+ * below, g_t <- max(g_t, lower_bound).
+ *
+ * Conventions shared by every entry point:
+ *  - Every buffer is caller-owned DEVICE memory, except the fields whose
+ *    names end in `_host`. The library allocates nothing, frees nothing and
+ *    never synchronises; work is queued on the caller's stream (a
+ *    cudaStream_t passed as `void *`; NULL is the legacy default stream).
+ *  - Tensors are dense, row-major, in the layouts given per field. Data
+ *    pointers must be 16-byte aligned (beta: 2-byte aligned for bf16,
+ *    4-byte for fp32). Outputs must not alias inputs (except where stated).
+ *  - Errors: every call validates its arguments on the host first and
+ *    returns a status without launching anything if they are bad. A launch
+ *    failure returns KDA_ERR_CUDA; kda_last_cuda_error() then gives the CUDA
+ *    error code. Nothing aborts, traps or prints.
+ *  - q/k L2 normalisation uses eps = 1e-6 inside the square root; states are
+ *    always fp32; inputs and the output share one dtype.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARGUMENT = 1, /* null/misaligned pointer, bad size, bad cu_seqlens ... */
+    KDA_ERR_UNSUPPORTED = 2,      /* valid request this build has no kernel for */
+    KDA_ERR_CUDA = 3,             /* a CUDA call or launch failed */
+    KDA_ERR_TIMEOUT = 4,          /* a bounded device-side wait gave up */
+    KDA_ERR_WORKSPACE = 5         /* workspace missing or smaller than required */
+} kda_status;
+
+typedef enum {
+    KDA_DTYPE_F32 = 0,
+    KDA_DTYPE_BF16 = 1
+} kda_dtype;
+
+/*
+ * Chunkwise forward: the `chunk_kda` boundary of page "K3/kda/ops/api.py"
+ * (signature and preprocessing: q/k L2 norm, sigmoid of beta, lower bound,
+ * initial_state, output_final_state, chunk_size), minus its backend dispatch
+ * and in-kernel gate. The result equals the token recurrence above run
+ * over each sequence; internally tokens are processed chunk_size at a time.
+ */
+typedef struct {
+    kda_dtype dtype;      /* dtype of q, k, v, g, beta and o */
+    int B, T, H, Dk, Dv;  /* q,k,g: [B,T,H,Dk]; v,o: [B,T,H,Dv]; beta: [B,T,H] */
+    const void *q, *k, *v;
+    const void *g;        /* per-channel log-decay, expected <= 0 */
+    const void *beta;     /* LOGITS; sigmoid is applied in the kernel */
+    void *o;              /* output [B,T,H,Dv] */
+    float scale;          /* <= 0 or NaN selects 1/sqrt(Dk) */
+    const float *initial_state; /* [N,H,Dk,Dv] fp32, NULL = zeros */
+    float *final_state;         /* [N,H,Dk,Dv] fp32 out, NULL = not wanted; may alias initial_state */
+    /* Varlen packing: when cu_seqlens != NULL, B must be 1 and the T tokens
+     * hold N sequences back to back; sequence n is tokens
+     * cu_seqlens[n] .. cu_seqlens[n+1]-1 (int32, device, N+1 entries,
+     * cu_seqlens[0] = 0, non-decreasing, cu_seqlens[N] = T). States never
+     * cross a sequence boundary. cu_seqlens_host, when given, is a host copy
+     * that is validated; without it the device copy is trusted. When
+     * cu_seqlens == NULL, N must equal B (each batch row is a sequence). */
+    const int32_t *cu_seqlens;
+    const int32_t *cu_seqlens_host;
+    int N;
+    int use_qk_l2norm;    /* 1: q,k <- x / sqrt(sum x^2 + 1e-6) in the kernel */
+    int has_lower_bound;  /* 1: g <- max(g, lower_bound); lower_bound must be < 0 */
+    float lower_bound;
+    int chunk_size;       /* 0 (default) or 64 */
+    void *workspace;      /* device scratch of kda_chunk_fwd_workspace_size() bytes */
+    size_t workspace_bytes;
+} kda_chunk_args;
+
+/* Bytes of device workspace kda_chunk_fwd needs for these arguments (may be
+ * 0). Only shapes, dtype and flags are read; pointers may be NULL. */
+KDA_API kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args *args, size_t *bytes);
+
+/* Queue the chunkwise forward on `stream`. Returns KDA_OK once queued. */
+KDA_API kda_status kda_chunk_fwd(const kda_chunk_args *args, void *stream);
+
+/*
+ * One recurrent decode step for N sequences at once: the recurrence above
+ * applied to one token per sequence (page "atlas_core/kimi_k3/kda.rs",
+ * `kda_recurrent_step`), with the state read, updated and written back IN
+ * PLACE (a read-modify-write of [N,H,Dk,Dv] fp32).
+ */
+typedef struct {
+    kda_dtype dtype;      /* dtype of q, k, v, g, beta and o */
+    int N, H, Dk, Dv;
+    const void *q, *k;    /* [N,H,Dk] */
+    const void *v;        /* [N,H,Dv] */
+    const void *g;        /* [N,H,Dk] log-decay */
+    const void *beta;     /* [N,H] logits */
+    float *state;         /* [N,H,Dk,Dv] fp32, updated in place */
+    void *o;              /* [N,H,Dv] out */
+    float scale;          /* <= 0 or NaN selects 1/sqrt(Dk) */
+    int use_qk_l2norm;
+    int has_lower_bound;
+    float lower_bound;
+} kda_step_args;
+
+KDA_API kda_status kda_recurrent_step(const kda_step_args *args, void *stream);
+
+/* Static, human-readable name of a status. */
+KDA_API const char *kda_status_string(kda_status status);
+
+/* CUDA error code (cudaError_t as int) of the last KDA_ERR_CUDA returned on
+ * this host thread, 0 if none. */
+KDA_API int kda_last_cuda_error(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+KDA_API int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

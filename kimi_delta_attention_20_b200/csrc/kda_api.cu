@@ -1,0 +1,159 @@
+// Host side of the C ABI declared in include/kda.h: argument validation,
+// kernel selection and launch. No allocation, no synchronisation.
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+#include "kda_common.cuh"
+
+namespace kda {
+cudaError_t launch_decode(const StepParams &p, bool bf16, int Dk, int Dv, cudaStream_t st);
+cudaError_t launch_chunk_simt(const ChunkParams &p, bool bf16, int Dk, int Dv, cudaStream_t st);
+bool chunk_tc_supported(bool bf16, int Dk, int Dv, int chunk_size);
+size_t chunk_tc_workspace_bytes(int N, int H, int Dk, int Dv);
+cudaError_t launch_chunk_tc(const ChunkParams &p, int Dk, int Dv, void *workspace,
+                            size_t workspace_bytes, const int32_t *cu_host, cudaStream_t st);
+}  // namespace kda
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+kda_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return KDA_OK;
+    g_last_cuda_error = (int)e;
+    return KDA_ERR_CUDA;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+float resolve_scale(float s, int Dk) {
+    if (!(s > 0.f)) return 1.0f / sqrtf((float)Dk);  // also catches NaN
+    return s;
+}
+
+// Shapes and flags only (shared by the workspace query and the launch).
+kda_status check_chunk_shape(const kda_chunk_args *a, int *N_out) {
+    if (!a) return KDA_ERR_INVALID_ARGUMENT;
+    if (a->dtype != KDA_DTYPE_F32 && a->dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARGUMENT;
+    if (a->B < 1 || a->T < 0 || a->H < 1 || a->Dk < 1 || a->Dv < 1) return KDA_ERR_INVALID_ARGUMENT;
+    if (!head_dim_ok(a->Dk) || !head_dim_ok(a->Dv)) return KDA_ERR_UNSUPPORTED;
+    if (a->chunk_size != 0 && a->chunk_size != 64) return KDA_ERR_UNSUPPORTED;
+    if (a->has_lower_bound && !(a->lower_bound < 0.f)) return KDA_ERR_INVALID_ARGUMENT;
+    if ((long long)a->B * a->T * a->H * (a->Dk > a->Dv ? a->Dk : a->Dv) >= (1LL << 40))
+        return KDA_ERR_INVALID_ARGUMENT;
+    int N = a->N;
+    if (a->cu_seqlens) {
+        if (a->B != 1 || N < 1) return KDA_ERR_INVALID_ARGUMENT;
+    } else {
+        if (N == 0) N = a->B;
+        if (N != a->B) return KDA_ERR_INVALID_ARGUMENT;
+    }
+    if ((long long)N * a->H * 4 >= 0x7fffffffLL) return KDA_ERR_INVALID_ARGUMENT;
+    *N_out = N;
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_status_string(kda_status s) {
+    switch (s) {
+    case KDA_OK: return "ok";
+    case KDA_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KDA_ERR_CUDA: return "CUDA error";
+    case KDA_ERR_TIMEOUT: return "device-side wait timed out";
+    case KDA_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+int kda_last_cuda_error(void) { return g_last_cuda_error; }
+
+int kda_version(void) { return 100; }
+
+kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args *a, size_t *bytes) {
+    if (!bytes) return KDA_ERR_INVALID_ARGUMENT;
+    int N = 0;
+    kda_status s = check_chunk_shape(a, &N);
+    if (s != KDA_OK) return s;
+    *bytes = 0;
+    if (kda::chunk_tc_supported(a->dtype == KDA_DTYPE_BF16, a->Dk, a->Dv, a->chunk_size))
+        *bytes = kda::chunk_tc_workspace_bytes(N, a->H, a->Dk, a->Dv);
+    return KDA_OK;
+}
+
+kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
+    int N = 0;
+    kda_status s = check_chunk_shape(a, &N);
+    if (s != KDA_OK) return s;
+    const bool bf16 = a->dtype == KDA_DTYPE_BF16;
+    const size_t esz = bf16 ? 2 : 4;
+    const long long ntok = (long long)a->B * a->T;
+    if (ntok > 0) {
+        if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->o) return KDA_ERR_INVALID_ARGUMENT;
+        if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->g, 16) ||
+            !aligned(a->o, 16) || !aligned(a->beta, esz))
+            return KDA_ERR_INVALID_ARGUMENT;
+    }
+    if ((a->initial_state && !aligned(a->initial_state, 16)) ||
+        (a->final_state && !aligned(a->final_state, 16)))
+        return KDA_ERR_INVALID_ARGUMENT;
+    if (a->cu_seqlens_host) {
+        const int32_t *cu = a->cu_seqlens_host;
+        if (cu[0] != 0 || cu[N] != a->T) return KDA_ERR_INVALID_ARGUMENT;
+        for (int n = 0; n < N; ++n)
+            if (cu[n + 1] < cu[n]) return KDA_ERR_INVALID_ARGUMENT;
+    }
+    if (!a->cu_seqlens && a->cu_seqlens_host) return KDA_ERR_INVALID_ARGUMENT;
+
+    kda::ChunkParams p;
+    p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta; p.o = a->o;
+    p.S0 = a->initial_state; p.S_out = a->final_state;
+    p.cu_seqlens = a->cu_seqlens; p.T = a->T; p.N = N; p.H = a->H;
+    p.scale = resolve_scale(a->scale, a->Dk);
+    p.use_l2 = a->use_qk_l2norm ? 1 : 0;
+    p.has_lb = a->has_lower_bound ? 1 : 0;
+    p.lb = a->lower_bound;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    if (kda::chunk_tc_supported(bf16, a->Dk, a->Dv, a->chunk_size)) {
+        const size_t need = kda::chunk_tc_workspace_bytes(N, a->H, a->Dk, a->Dv);
+        if (need > 0 && (!a->workspace || a->workspace_bytes < need || !aligned(a->workspace, 256)))
+            return KDA_ERR_WORKSPACE;
+        return cuda_status(kda::launch_chunk_tc(p, a->Dk, a->Dv, a->workspace, a->workspace_bytes,
+                                                a->cu_seqlens_host, st));
+    }
+    return cuda_status(kda::launch_chunk_simt(p, bf16, a->Dk, a->Dv, st));
+}
+
+kda_status kda_recurrent_step(const kda_step_args *a, void *stream) {
+    if (!a) return KDA_ERR_INVALID_ARGUMENT;
+    if (a->dtype != KDA_DTYPE_F32 && a->dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARGUMENT;
+    if (a->N < 0 || a->H < 1 || a->Dk < 1 || a->Dv < 1) return KDA_ERR_INVALID_ARGUMENT;
+    if (!head_dim_ok(a->Dk) || !head_dim_ok(a->Dv)) return KDA_ERR_UNSUPPORTED;
+    if (a->has_lower_bound && !(a->lower_bound < 0.f)) return KDA_ERR_INVALID_ARGUMENT;
+    if ((long long)a->N * a->H * 4 >= 0x7fffffffLL) return KDA_ERR_INVALID_ARGUMENT;
+    if (a->N == 0) return KDA_OK;
+    const bool bf16 = a->dtype == KDA_DTYPE_BF16;
+    const size_t esz = bf16 ? 2 : 4;
+    if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->state || !a->o)
+        return KDA_ERR_INVALID_ARGUMENT;
+    if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->g, 16) ||
+        !aligned(a->o, 16) || !aligned(a->state, 16) || !aligned(a->beta, esz))
+        return KDA_ERR_INVALID_ARGUMENT;
+    kda::StepParams p;
+    p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
+    p.state = a->state; p.o = a->o; p.N = a->N; p.H = a->H;
+    p.scale = resolve_scale(a->scale, a->Dk);
+    p.use_l2 = a->use_qk_l2norm ? 1 : 0;
+    p.has_lb = a->has_lower_bound ? 1 : 0;
+    p.lb = a->lower_bound;
+    return cuda_status(kda::launch_decode(p, bf16, a->Dk, a->Dv, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,253 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Every input is drawn by the seeded generators of kda_inputs and the same
+(cast) tensors feed both sides. The named workloads run at their full sizes
+and launch configuration; where the oracle would take too long on all heads
+it checks a sample of (sequence, head) pairs, which is exact because pairs
+are independent. Boundary lengths 1/7/63/64/65/130, decode-after-prefill
+(t0, steps) pairs and split points come from page
+"memra-engine tests/kda_fixture_gpu.rs" (gates 1-3).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import kda_inputs as KI
+import oracle
+from kda_check import check, oracle_chunk
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def kda_mod():
+    import kimi_delta_attention_20_b200 as kda
+    return kda
+
+
+def run_chunk(inp, wl=None, *, scale=None, lower_bound=None, final=True, l2=True, **kw):
+    kda = kda_mod()
+    d = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    return kda.chunk_kda(d["q"], d["k"], d["v"], d["g"], d["beta"], scale=scale,
+                         initial_state=d.get("initial_state"), output_final_state=final,
+                         use_qk_l2norm_in_kernel=l2, lower_bound=lower_bound,
+                         cu_seqlens=d.get("cu_seqlens"), **kw)
+
+
+def compare_chunk(inp, o, S, dtype, *, heads=None, seqs=None, scale=None, lower_bound=None,
+                  l2=True, tag=""):
+    ref = oracle_chunk({k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()},
+                       heads=heads, seqs=seqs, scale=scale, lower_bound=lower_bound, l2=l2)
+    H = inp["q"].shape[2]
+    hs = list(range(H)) if heads is None else list(heads)
+    ns = list(range(len(ref))) if seqs is None else list(seqs)
+    B, T = inp["q"].shape[:2]
+    o_flat = o.reshape(B * T, H, -1)
+    for (a, b, o_ref, S_ref), n in zip(ref, ns):
+        if b > a:
+            check(f"{tag} o seq{n}", o_flat[a:b][:, hs], o_ref, dtype)
+        if S is not None:
+            check(f"{tag} S seq{n}", S[n, hs], S_ref, dtype)
+
+
+# --- the named workloads, full size ------------------------------------------
+
+def test_workload_tiny_fp32():
+    wl = KI.CHUNK_WORKLOADS[0]
+    inp = KI.chunk_inputs(wl, device="cpu")
+    o, S = run_chunk(inp, scale=wl.scale)
+    compare_chunk(inp, o, S, wl.dtype, scale=wl.scale, tag="tiny-fp32")
+
+
+def test_workload_twin_d32():
+    wl = KI.CHUNK_WORKLOADS[1]
+    inp = KI.chunk_inputs(wl, device="cpu")
+    o, S = run_chunk(inp)
+    compare_chunk(inp, o, S, wl.dtype, tag="twin")
+
+
+def test_workload_d128_T8192_clamped():
+    wl = KI.CHUNK_WORKLOADS[2]
+    inp = KI.chunk_inputs(wl, device=DEV)
+    o, S = run_chunk(inp, lower_bound=wl.lower_bound)
+    compare_chunk(inp, o, S, wl.dtype, heads=[0, 5, 11, 15], lower_bound=wl.lower_bound,
+                  tag="d128")
+
+
+def test_workload_varlen_H96():
+    wl = KI.CHUNK_WORKLOADS[4]
+    inp = KI.chunk_inputs(wl, device=DEV)
+    o, S = run_chunk(inp, lower_bound=wl.lower_bound)
+    rng = np.random.default_rng(0)
+    heads = sorted(rng.choice(96, size=3, replace=False).tolist())
+    compare_chunk(inp, o, S, wl.dtype, heads=heads, lower_bound=wl.lower_bound, tag="varlen")
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+
+
+def test_workload_decode_256_steps():
+    wl = KI.DECODE_WORKLOADS[3]
+    kda = kda_mod()
+    inp = KI.decode_inputs(wl, device=DEV)
+    state = inp["state"].clone()
+    outs = []
+    for t in range(wl.steps):
+        outs.append(kda.recurrent_step(inp["q"][t], inp["k"][t], inp["v"][t], inp["g"][t],
+                                       inp["beta"][t], state))
+    o = torch.stack(outs)  # [steps, N, H, Dv]
+    rng = np.random.default_rng(1)
+    for n, h in zip(rng.choice(wl.N, 4, replace=False), rng.choice(wl.H, 4, replace=False)):
+        sl = lambda x: x[:, n, h:h + 1].cpu()
+        o_ref, S_ref = oracle.recurrent(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["g"]),
+                                        inp["beta"][:, n, h:h + 1].cpu(),
+                                        initial_state=inp["state"][n:n + 1, h:h + 1].cpu())
+        check(f"decode o n{n} h{h}", o[:, n, h:h + 1], o_ref, wl.dtype)
+        check(f"decode S n{n} h{h}", state[n, h], S_ref[0, 0], wl.dtype)
+
+
+# --- boundaries, shapes, flags ------------------------------------------------
+
+DIMS = [(32, 32), (64, 64), (128, 128), (32, 128), (128, 64)]
+
+
+@pytest.mark.parametrize("T", [1, 7, 63, 64, 65, 130])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dims", DIMS)
+def test_chunk_boundary_lengths(T, dtype, dims):
+    Dk, Dv = dims
+    inp = KI.draw_chunk(2, T, 3, Dk, Dv, dtype=dtype, seed=T * 31 + Dk + Dv, init_state=True)
+    o, S = run_chunk(inp)
+    compare_chunk(inp, o, S, dtype, tag=f"T{T}")
+
+
+@pytest.mark.parametrize("lb", [None, -5.0, -0.5])
+def test_chunk_lower_bound(lb):
+    inp = KI.draw_chunk(1, 200, 2, 128, 128, dtype=torch.bfloat16, seed=5, init_state=True)
+    o, S = run_chunk(inp, lower_bound=lb)
+    compare_chunk(inp, o, S, torch.bfloat16, lower_bound=lb, tag=f"lb{lb}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_chunk_scale_and_no_l2norm(dtype):
+    inp = KI.draw_chunk(1, 130, 2, 64, 64, dtype=dtype, seed=6)
+    # keep unnormalised keys short so the delta rule stays contractive
+    inp["k"] = (inp["k"].float() / 8.0).to(dtype)
+    with pytest.warns(RuntimeWarning):
+        o, S = run_chunk(inp, scale=0.37, l2=False)
+    compare_chunk(inp, o, S, dtype, scale=0.37, l2=False, tag="nol2")
+
+
+def test_chunk_varlen_ragged():
+    lens = [0, 1, 64, 65, 130, 7, 0, 200]
+    inp = KI.draw_chunk(1, sum(lens), 3, 128, 128, dtype=torch.bfloat16, seed=7,
+                        seqlens=lens, init_state=True)
+    o, S = run_chunk(inp, lower_bound=-5.0)
+    compare_chunk(inp, o, S, torch.bfloat16, lower_bound=-5.0, tag="ragged")
+    # zero-length sequences hand their initial state through unchanged
+    for n in (0, 6):
+        assert torch.equal(S[n].cpu(), inp["initial_state"][n])
+
+
+def test_chunk_empty_sequence_batch():
+    inp = KI.draw_chunk(2, 0, 2, 32, 32, dtype=torch.bfloat16, seed=8, init_state=True)
+    o, S = run_chunk(inp)
+    assert o.shape == (2, 0, 2, 32)
+    assert torch.equal(S.cpu(), inp["initial_state"])
+
+
+def test_chunk_final_state_in_place():
+    inp = KI.draw_chunk(2, 97, 2, 128, 128, dtype=torch.bfloat16, seed=9, init_state=True)
+    kda = kda_mod()
+    d = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    st = d["initial_state"].clone()
+    o, S = kda.chunk_kda(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=st,
+                         output_final_state=True, final_state_out=st,
+                         use_qk_l2norm_in_kernel=True)
+    assert S.data_ptr() == st.data_ptr()
+    compare_chunk(inp, o, S, torch.bfloat16, tag="inplace")
+
+
+def test_chunk_without_final_state():
+    inp = KI.draw_chunk(1, 70, 2, 32, 32, dtype=torch.bfloat16, seed=10, init_state=True)
+    o, S = run_chunk(inp, final=False)
+    assert S is None
+    compare_chunk(inp, o, None, torch.bfloat16, tag="nofinal")
+
+
+@pytest.mark.parametrize("split", [1, 2, 3, 63, 64, 65, 127])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_split_composition(split, dtype):
+    """Two calls threaded through the state equal one call over T = 130."""
+    inp = KI.draw_chunk(1, 130, 2, 128, 128, dtype=dtype, seed=11, init_state=True)
+    o, S = run_chunk(inp)
+    first = {k: (v[:, :split] if k in ("q", "k", "v", "g", "beta") else v) for k, v in inp.items()}
+    second = {k: (v[:, split:] if k in ("q", "k", "v", "g", "beta") else v) for k, v in inp.items()}
+    o1, S1 = run_chunk(first)
+    second["initial_state"] = S1
+    o2, S2 = run_chunk(second)
+    check("split o", torch.cat([o1, o2], 1), o, dtype)
+    check("split S", S2, S, dtype)
+    compare_chunk(inp, torch.cat([o1, o2], 1), S2, dtype, tag=f"split{split}")
+
+
+@pytest.mark.parametrize("t0,steps", [(1, 4), (7, 3), (63, 5), (64, 4), (65, 3)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_after_prefill(t0, steps, dtype):
+    kda = kda_mod()
+    T = t0 + steps
+    inp = KI.draw_chunk(2, T, 3, 128, 128, dtype=dtype, seed=12 + t0, init_state=True)
+    pre = {k: (v[:, :t0] if k in ("q", "k", "v", "g", "beta") else v) for k, v in inp.items()}
+    o_pre, S = run_chunk(pre, lower_bound=-5.0)
+    outs = [o_pre]
+    for t in range(t0, T):
+        x = {n: inp[n][:, t].to(DEV) for n in ("q", "k", "v", "g", "beta")}
+        outs.append(kda.recurrent_step(x["q"], x["k"], x["v"], x["g"], x["beta"], S,
+                                       lower_bound=-5.0)[:, None])
+    compare_chunk(inp, torch.cat(outs, 1), S, dtype, lower_bound=-5.0, tag="prefill+decode")
+
+
+@pytest.mark.parametrize("dims", DIMS)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_shapes(dims, dtype):
+    kda = kda_mod()
+    Dk, Dv = dims
+    inp = KI.draw_decode(5, 3, Dk, Dv, 6, dtype=dtype, seed=13)
+    state = inp["state"].to(DEV)
+    outs = []
+    for t in range(6):
+        outs.append(kda.recurrent_step(*(inp[n][t].to(DEV) for n in ("q", "k", "v", "g", "beta")),
+                                       state, scale=0.25))
+    o = torch.stack(outs)
+    for n in range(5):
+        o_ref, S_ref = oracle.recurrent(inp["q"][:, n], inp["k"][:, n], inp["v"][:, n],
+                                        inp["g"][:, n], inp["beta"][:, n], scale=0.25,
+                                        initial_state=inp["state"][n:n + 1])
+        check(f"dec o n{n}", o[:, n], o_ref, dtype)
+        check(f"dec S n{n}", state[n], S_ref[0], dtype)
+
+
+def test_decode_noop_and_reset_tokens():
+    """beta logit -inf with g = 0 leaves the state bit-identical; g = -inf with
+    beta logit +inf replaces it by k^ v^T (oracle invariants, on the GPU)."""
+    kda = kda_mod()
+    N, H, D = 3, 2, 128
+    S0 = torch.randn(N, H, D, D, device=DEV) * 0.1
+    q = torch.randn(N, H, D, device=DEV)
+    k = torch.randn(N, H, D, device=DEV)
+    v = torch.randn(N, H, D, device=DEV)
+    S = S0.clone()
+    kda.recurrent_step(q, k, v, torch.zeros_like(q), torch.full((N, H), -math.inf, device=DEV), S)
+    assert torch.equal(S, S0)
+    kda.recurrent_step(q, k, v, torch.full_like(q, -math.inf), torch.full((N, H), math.inf,
+                                                                          device=DEV), S)
+    kh = k / torch.sqrt((k * k).sum(-1, keepdim=True) + 1e-6)
+    torch.testing.assert_close(S, kh[..., :, None] * v[..., None, :], rtol=1e-5, atol=1e-6)
+
+
+def test_decode_empty_batch():
+    kda = kda_mod()
+    z = torch.zeros(0, 2, 32, device=DEV)
+    o = kda.recurrent_step(z, z, z, z, torch.zeros(0, 2, device=DEV), torch.zeros(0, 2, 32, 32, device=DEV))
+    assert o.shape == (0, 2, 32)
