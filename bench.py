@@ -198,6 +198,21 @@ def run_kda(args, rank, world, local_rank):
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[local_rank]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else local_rank
 
+    if args.only:
+        # one kernel, few launches: the shape profiler captures use
+        one = chunk_step if args.only == "chunk" else (lambda: decode_step(0))
+        for _ in range(args.warmup):
+            one()
+        torch.cuda.synchronize(dev)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.steps):
+            one()
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        return {"only": args.only, "ms_per_launch": a0.elapsed_time(a1) / args.steps,
+                "launches": args.steps}
+
     # warm-up (untimed)
     for _ in range(args.warmup):
         chunk_step()
@@ -379,6 +394,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["chunk", "decode"], default=None,
+                    help="run one leg only and print its timing (for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "kda":
         ap.error("--warmup must be >= 3")
