@@ -121,7 +121,7 @@ kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
     p.lb = a->lower_bound;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    if (kda::chunk_tc_supported(bf16, a->Dk, a->Dv, a->chunk_size)) {
+    if (ntok > 0 && kda::chunk_tc_supported(bf16, a->Dk, a->Dv, a->chunk_size)) {
         const size_t need = kda::chunk_tc_workspace_bytes(N, a->H, a->Dk, a->Dv);
         if (need > 0 && (!a->workspace || a->workspace_bytes < need || !aligned(a->workspace, 256)))
             return KDA_ERR_WORKSPACE;

@@ -251,3 +251,26 @@ def test_decode_empty_batch():
     z = torch.zeros(0, 2, 32, device=DEV)
     o = kda.recurrent_step(z, z, z, z, torch.zeros(0, 2, device=DEV), torch.zeros(0, 2, 32, 32, device=DEV))
     assert o.shape == (0, 2, 32)
+
+
+def test_chunk_steep_gates_take_exact_path():
+    """A chunk whose gate drops by more than the tensor-core split allows
+    (here 9 per token over a whole chunk) is computed exactly for that chunk;
+    its neighbours use the tensor-core split. Both must match the oracle."""
+    inp = KI.draw_chunk(1, 200, 2, 128, 128, dtype=torch.bfloat16, seed=21, init_state=True)
+    g = inp["g"].float()
+    g[:, 64:128] = -9.0
+    g[:, 150:160] = -9.5
+    inp["g"] = g.to(torch.bfloat16)
+    o, S = run_chunk(inp, lower_bound=-10.0)
+    compare_chunk(inp, o, S, torch.bfloat16, lower_bound=-10.0, tag="steep")
+
+
+def test_chunk_status_word_is_cleared():
+    """The tensor-core path reports device-side timeouts in the first word of
+    the workspace; a normal call leaves it zero."""
+    inp = KI.draw_chunk(1, 130, 2, 128, 128, dtype=torch.bfloat16, seed=22)
+    ws = torch.full((256,), 7, dtype=torch.uint8, device=DEV)
+    run_chunk(inp, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
