@@ -160,13 +160,14 @@ def run_kda(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     hbm_peak, tc_peak, peak_kind = load_peaks()
 
-    wl = KI.CHUNK_WORKLOADS[CHUNK_WL]
+    wl = KI.CHUNK_WORKLOADS[args.workload if (args.only and args.workload is not None) else CHUNK_WL]
     inp = KI.chunk_inputs(wl, device=dev)
     q, k, v, g, beta = (inp[n] for n in ("q", "k", "v", "g", "beta"))
     S0, cu = inp["initial_state"], inp["cu_seqlens"]
     o = torch.empty_like(v)
-    S_out = torch.empty_like(S0)
-    ws_bytes = kda.chunk_workspace_bytes(1, wl.T, wl.H, wl.Dk, wl.Dv, N=wl.n_seqs, varlen=True)
+    S_out = torch.empty(wl.n_seqs, wl.H, wl.Dk, wl.Dv, dtype=torch.float32, device=dev)
+    ws_bytes = kda.chunk_workspace_bytes(wl.B, wl.T, wl.H, wl.Dk, wl.Dv, N=wl.n_seqs,
+                                         varlen=wl.seqlens is not None)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
 
     def chunk_step():
@@ -175,9 +176,10 @@ def run_kda(args, rank, world, local_rank):
                       cu_seqlens=cu, out=o, final_state_out=S_out, workspace=ws)
 
     dwl = KI.DECODE_WORKLOADS[DECODE_WL]
-    dinp = KI.decode_inputs(dwl, device=dev)
-    state = dinp["state"].clone()
-    od = torch.empty(dwl.N, dwl.H, dwl.Dv, dtype=dwl.dtype, device=dev)
+    if args.only != "chunk":
+        dinp = KI.decode_inputs(dwl, device=dev)
+        state = dinp["state"].clone()
+        od = torch.empty(dwl.N, dwl.H, dwl.Dv, dtype=dwl.dtype, device=dev)
 
     def decode_step(t):
         kda.recurrent_step(dinp["q"][t], dinp["k"][t], dinp["v"][t], dinp["g"][t],
@@ -396,6 +398,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["chunk", "decode"], default=None,
                     help="run one leg only and print its timing (for profiler captures)")
+    ap.add_argument("--workload", type=int, default=None,
+                    help="with --only chunk: chunk workload index (default: the varlen H=96 one)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "kda":
         ap.error("--warmup must be >= 3")

@@ -41,28 +41,33 @@ using namespace sm100;
 
 constexpr int C = 64;
 constexpr int D = 128;
-constexpr int NT = 256;
-constexpr float kSpanMax = 80.f;           // e^80 = 5.5e34 stays finite in bf16 and fp32
+constexpr int NT = 512;                      // 16 warps
+constexpr float kSpanMax = 80.f;             // e^80 = 5.5e34 stays finite in bf16 and fp32
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 
 // ---- shared memory map (bytes from the 1024-aligned base) ----
 constexpr uint32_t STG_Q = 0, STG_K = 16384, STG_G = 32768, STG_V = 49152;  // TMA staging, [64][128]
 constexpr uint32_t AOPS = 65536;                                            // 72 KiB, two views:
 // view 1, operands of the A_kk / A_qk products
-constexpr uint32_t XKQO_H0 = AOPS + 0, YD_H0 = AOPS + 8192, XKQO_H1 = AOPS + 16384, YD_H1 = AOPS + 24576;
-constexpr uint32_t YO_H0 = AOPS + 32768, YO_H1 = AOPS + 36864, XKQD = AOPS + 40960;  // XKQD: 2 x 16 KiB
-// view 2, after those products: fp32 solve buffers, then W^T and D^T tiles
-constexpr int LDS = 65;  // padded fp32 row stride of the 64x64 solve buffers
-constexpr uint32_t LF = AOPS + 0, TF = AOPS + 16896, MF = AOPS + 33792, AQK = AOPS + 40960, TP = AOPS + 49152;
-constexpr uint32_t WT = AOPS + 0, DT = AOPS + 16384;
+constexpr uint32_t YD_H0 = AOPS + 0, YD_H1 = AOPS + 8192, YO_H0 = AOPS + 16384, YO_H1 = AOPS + 20480;
+constexpr uint32_t XKQD = AOPS + 40960;  // 2 halves x [128 rows][128 B]: rows 0..63 k, 64..127 q
+// view 2, after those products: fp32 solve buffers, T' tiles, then W^T, D^T and the output tile
+constexpr int LDS = 65;  // padded fp32 row stride of L (64x64)
+constexpr int LDT = 68;  // fp32 row stride of T (64x64)
+constexpr int LDR = 52;  // fp32 row stride of the 16x48 block-row buffer
+constexpr uint32_t LF = AOPS + 0, TF = AOPS + 16896, RF = AOPS + 34304, AQK = AOPS + 40960;
+constexpr uint32_t TPU = AOPS + 49152, TPW = AOPS + 57344;  // T diag(beta), T diag(beta / |k|)
+constexpr uint32_t WT = AOPS + 0, DT = AOPS + 16384, OT = AOPS + 57344;  // OT: [64][128] bf16, plain
 constexpr uint32_t QT = AOPS + 73728, KT = QT + 16384, KH = KT + 16384, ST = KH + 16384;  // ST: 32 KiB
 constexpr uint32_t MISC = ST + 32768;
-constexpr uint32_t M_BETA = MISC, M_INVQ = MISC + 256, M_INVK = MISC + 512, M_G31 = MISC + 768,
-                   M_G63 = MISC + 1280, M_GAM = MISC + 1792, M_BAR = MISC + 2304, M_TMEM = MISC + 2336;
-constexpr uint32_t SMEM_BYTES = MISC + 2560;
+constexpr uint32_t M_BETA = MISC, M_INVQ = MISC + 256, M_INVK = MISC + 512, M_GAM = MISC + 768,
+                   M_BAR = MISC + 1280, M_TMEM = MISC + 1312, M_RED = MISC + 1536,  // [q|k][half][64] f32
+                   M_SEG = MISC + 2560;                                             // [8][128] f32
+constexpr uint32_t SMEM_BYTES = M_SEG + 4096;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
-static_assert(LF + 64 * LDS * 4 <= TF && TF + 64 * LDS * 4 <= MF && MF + 32 * 33 * 4 <= AQK, "view 2");
-static_assert(TP + 8192 <= AOPS + 73728 && DT + 16384 <= AQK, "view 2 tiles");
+static_assert(YO_H1 + 4096 <= XKQD, "view 1");
+static_assert(LF + 64 * LDS * 4 <= TF && TF + 64 * LDT * 4 <= RF && RF + 16 * LDR * 4 <= AQK, "view 2");
+static_assert(TPW + 8192 <= AOPS + 73728 && DT + 16384 <= AQK && OT + 16384 <= AOPS + 73728, "view 2 tiles");
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
 // ---- tensor memory columns ----
@@ -86,13 +91,46 @@ struct TcParams {
     int perm[kMaxPerm];
 };
 
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
+    const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 t = __bfloat1622float2(b[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+__device__ __forceinline__ uint4 pack8(const float *f) {
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                      pack_bf16x2(f[6], f[7]));
+}
+__device__ __forceinline__ void sts128(uint8_t *base, uint32_t off, const uint4 &v) {
+    *reinterpret_cast<uint4 *>(base + off) = v;
+}
+__device__ __forceinline__ uint4 lds128(const uint8_t *base, uint32_t off) {
+    return *reinterpret_cast<const uint4 *>(base + off);
+}
 __device__ __forceinline__ float bf(const uint8_t *base, uint32_t off) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(base + off));
 }
 __device__ __forceinline__ void st_bf(uint8_t *base, uint32_t off, float x) {
     *reinterpret_cast<__nv_bfloat16 *>(base + off) = __float2bfloat16_rn(x);
 }
+// 16 fp32 values of one TMEM row to two 16-byte chunks of a swizzled bf16 tile row
+__device__ __forceinline__ void row16_to_tile(uint8_t *sm, uint32_t tile, int row, int col0, int rows,
+                                              const float (&x)[16]) {
+    sts128(sm, tile + sw128_chunk(row, col0, rows), pack8(x));
+    sts128(sm, tile + sw128_chunk(row, col0 + 8, rows), pack8(x + 8));
+}
 
+// Normalisation of q and k is deferred: the products use the raw rows and the
+// per-row factors 1/|q_r|, 1/|k_r| are applied where they act linearly --
+//   L[r,s]  = beta_r |k_r|^-1 |k_s|^-1 A_kk,raw[r,s]
+//   W       = T diag(beta_s |k_s|^-1) (k e^G)_raw            (second T' tile)
+//   D~      = D with column s scaled by |k_s|^-1, which feeds O += A_qk,raw D~ and
+//             S += Khat_raw^T D~
+//   o_r     = scale |q_r|^-1 (Qtil_raw S + A_qk,raw D~)_r
+// which is algebraically identical to normalising first.
 __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_constant__ TcParams P) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -112,12 +150,12 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     float *sbeta = reinterpret_cast<float *>(sm + M_BETA);
     float *sinvq = reinterpret_cast<float *>(sm + M_INVQ);
     float *sinvk = reinterpret_cast<float *>(sm + M_INVK);
-    float *sG31 = reinterpret_cast<float *>(sm + M_G31);
-    float *sG63 = reinterpret_cast<float *>(sm + M_G63);
     float *sGam = reinterpret_cast<float *>(sm + M_GAM);
+    float *sred = reinterpret_cast<float *>(sm + M_RED);
+    float *ssegt = reinterpret_cast<float *>(sm + M_SEG);
     float *Lf = reinterpret_cast<float *>(sm + LF);
     float *Tf = reinterpret_cast<float *>(sm + TF);
-    float *Mf = reinterpret_cast<float *>(sm + MF);
+    float *Rf = reinterpret_cast<float *>(sm + RF);
 
     if (warp == 0) { tmem_alloc(s_tmem, TM_COLS); tmem_relinquish(); }
     if (tid == 32) {
@@ -130,7 +168,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     tc_fence_after();
     const uint32_t tb = *s_tmem;
     const uint32_t sb = smem_u32(sm);
-    const uint32_t lane_sel = (uint32_t)(32 * (warp & 3)) << 16;  // this warp's TMEM lane quarter
+    const int quarter = warp & 3;                               // TMEM lanes 32*quarter .. +31
+    const uint32_t lane_sel = (uint32_t)(32 * quarter) << 16;
+    const int cgrp = warp >> 2;                                  // column group of TMEM phases
 
     auto issue_qkg = [&](long long t) {
         mbar_arrive_expect_tx(bar_qkg, 3 * 16384);
@@ -144,127 +184,208 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         mbar_arrive_expect_tx(bar_v, 16384);
         for (int hf = 0; hf < 2; ++hf) tma_load_3d(sm + STG_V + hf * 8192, &P.tv, bar_v, hf * 64, h, (int)t);
     };
+    // a bounded wait on an mbarrier phase by every thread; true if the CTA must stop
+    auto wait_all = [&](uint64_t *bar, uint32_t &ph) -> bool {
+        const bool ok = mbar_wait(bar, ph, kWaitLimitNs);
+        ph ^= 1;
+        return __syncthreads_or(!ok) != 0;
+    };
 
+    // thread kMma issues the MMAs, thread kTma (another warp) the TMA loads
+    constexpr int kMma = 0, kTma = NT - 32;
     uint32_t ph_qkg = 0, ph_v = 0, ph_mma = 0;
-    bool qkg_out = false, v_out = false, mma_out = false;  // thread 0's outstanding async work
+    bool qkg_out = false, v_out = false, mma_out = false;  // outstanding async work of this thread
     bool aborted = false;
-    if (tid == 0 && nchunks > 0) { issue_qkg(bos); issue_v(bos); qkg_out = v_out = true; }
+    if (tid == kTma && nchunks > 0) { issue_qkg(bos); issue_v(bos); qkg_out = v_out = true; }
 
     const long long sbase_state = ((long long)n * H + h) * D * D;
+    const __nv_bfloat16 *bt = static_cast<const __nv_bfloat16 *>(p.beta);
+    // beta logits run one chunk ahead in registers of threads 0..63
+    float beta_next = 0.f;
+    if (tid < C && bos + tid < eos) beta_next = __bfloat162float(bt[(bos + tid) * H + h]);
+
+    // thread -> (16-byte chunk of 8 channels, 2 consecutive rows) for the row-layout phases.
+    // Warp w owns channel half (w & 1) and the 8-row segment (w >> 1); the 8 lanes of each
+    // 128-bit access phase share their rows and take 8 different chunks, so the 128-byte
+    // swizzle spreads them over all banks.
+    const int seg = warp >> 1;
+    const int jch = 8 * (warp & 1) + (lane & 7);   // channels 8*jch .. 8*jch+7
+    const int rq = lane >> 3;
+    const int row0 = 8 * seg + 2 * rq;             // rows row0, row0 + 1
+    const int blk = seg >> 2;                      // 32-row block of those rows
 
     for (int ci = 0; ci < nchunks && !aborted; ++ci) {
         const long long t0 = bos + (long long)ci * C;
         const int L = (int)((eos - t0) < C ? (eos - t0) : C);
         const bool has_next = ci + 1 < nchunks;
 
+        if (tid < C) {
+            sbeta[tid] = tid < L ? sigmoidf_(beta_next) : 0.f;
+            beta_next = 0.f;
+            if (has_next && t0 + C + tid < eos) beta_next = __bfloat162float(bt[(t0 + C + tid) * H + h]);
+        }
+
         // ---------------- inputs of this chunk
         {
-            bool ok = mbar_wait(bar_qkg, ph_qkg, kWaitLimitNs) && mbar_wait(bar_v, ph_v, kWaitLimitNs);
+            const bool ok = mbar_wait(bar_qkg, ph_qkg, kWaitLimitNs) && mbar_wait(bar_v, ph_v, kWaitLimitNs);
             ph_qkg ^= 1; ph_v ^= 1;
-            if (tid == 0) qkg_out = v_out = false;
+            if (tid == kTma) qkg_out = v_out = false;
             if (__syncthreads_or(!ok)) { aborted = true; break; }
         }
 
-        // ---------------- P1: beta, row norms of q and k (warp per row)
-        if (tid < C) {
-            const __nv_bfloat16 *bt = static_cast<const __nv_bfloat16 *>(p.beta);
-            sbeta[tid] = tid < L ? sigmoidf_(__bfloat162float(bt[(t0 + tid) * H + h])) : 0.f;
-        }
-        for (int r = warp; r < C; r += NT / 32) {
-            const int hf = lane >> 4, cc = (lane & 15) * 4;
-            const uint32_t off = hf * 8192 + r * 128 + ((((cc >> 3) ^ (r & 7)) << 4) | ((cc & 7) << 1));
-            const uint2 qv = *reinterpret_cast<const uint2 *>(sm + STG_Q + off);
-            const uint2 kv = *reinterpret_cast<const uint2 *>(sm + STG_K + off);
-            const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qv);
-            const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kv);
-            float sq = 0.f, sk = 0.f;
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const float2 a = __bfloat1622float2(q2[e]), b = __bfloat1622float2(k2[e]);
-                sq += a.x * a.x + a.y * a.y;
-                sk += b.x * b.x + b.y * b.y;
-            }
-            sq = warp_sum(sq); sk = warp_sum(sk);
-            if (lane == 0) {
-                sinvq[r] = r < L ? (p.use_l2 ? rsqrtf(sq + kL2Eps) : 1.f) : 0.f;
-                sinvk[r] = r < L ? (p.use_l2 ? rsqrtf(sk + kL2Eps) : 1.f) : 0.f;
-            }
-        }
-
-        // ---------------- P2: in-chunk cumsum of the gate, thread per (channel, 32-row block)
-        const int c = tid & 127, blk = tid >> 7;
-        float Gl[32];
+        // ---------------- P1: gate cumsum and row norms
+        float G[2][8], Gm[8], G47[8], G63[8];
+        bool span_bad = false;
         {
-            float acc = 0.f;
+            float tot[8], sq[2], sk[2];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int r = 32 * blk + i;
-                float gv = 0.f;
-                if (r < L) {
-                    gv = bf(sm + STG_G, sw128(r, c, 64));
+            for (int e = 0; e < 8; ++e) tot[e] = 0.f;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int r = row0 + u;
+                const uint32_t off = sw128_chunk(r, 8 * jch, 64);
+                float gg[8], qq[8], kk[8];
+                unpack8(lds128(sm + STG_G, off), gg);
+                unpack8(lds128(sm + STG_Q, off), qq);
+                unpack8(lds128(sm + STG_K, off), kk);
+                sq[u] = 0.f; sk[u] = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float gv = r < L ? gg[e] : 0.f;
                     if (p.has_lb) gv = fmaxf(gv, p.lb);
+                    tot[e] += gv;
+                    G[u][e] = tot[e];
+                    sq[u] = fmaf(qq[e], qq[e], sq[u]);
+                    sk[u] = fmaf(kk[e], kk[e], sk[u]);
                 }
-                acc += gv;
-                Gl[i] = acc;
+            }
+            // scan of the 2-row totals over the 4 row pairs of this segment (lane bits 3, 4)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                float inc = tot[e];
+                float y = __shfl_up_sync(0xffffffffu, inc, 8);
+                if (rq >= 1) inc += y;
+                y = __shfl_up_sync(0xffffffffu, inc, 16);
+                if (rq >= 2) inc += y;
+                G[0][e] += inc - tot[e];
+                G[1][e] += inc - tot[e];
+                if (rq == 3) ssegt[seg * 128 + 8 * jch + e] = inc;
+            }
+            // row norms over this warp's 64 channels (lane bits 0..2), then per half
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+#pragma unroll
+                for (int o = 1; o < 8; o <<= 1) {
+                    sq[u] += __shfl_xor_sync(0xffffffffu, sq[u], o);
+                    sk[u] += __shfl_xor_sync(0xffffffffu, sk[u], o);
+                }
+            }
+            if ((lane & 7) == 0) {
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    sred[(warp & 1) * 64 + row0 + u] = sq[u];
+                    sred[128 + (warp & 1) * 64 + row0 + u] = sk[u];
+                }
             }
         }
-        if (blk == 0) sG31[c] = Gl[31];
         __syncthreads();
-        if (blk == 1) {
-            const float b = sG31[c];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) Gl[i] += b;
-            sG63[c] = Gl[31];
-            sGam[c] = expf(Gl[31]);
+        if (tid < 128) {
+            const int r = tid & 63, which = tid >> 6;
+            const float ssum = sred[which * 128 + r] + sred[which * 128 + 64 + r];
+            const float inv = r < L ? (p.use_l2 ? rsqrtf(ssum + kL2Eps) : 1.f) : 0.f;
+            (which ? sinvk : sinvq)[r] = inv;
         }
-        const float Gm = Gl[15];
-        const int span_bad = fmaxf(Gl[0] - Gm, Gm - Gl[31]) > kSpanMax;
-        const bool fb = __syncthreads_or(span_bad) != 0;  // also publishes sG63 / sGam
-
-        // ---------------- P3: bf16 operand tiles
         {
-            const float G31 = blk == 0 ? Gl[31] : sG31[c];
-            const float G63 = sG63[c];
-            const int hf = c >> 6, cc = c & 63;
-            if (!fb) {
-                const float Emid = __expf(Gm);
-                const float Fkh = __expf(G63 - Gm);
-                const float Foff = blk == 0 ? __expf(G31 - Gm) : __expf(Gm - G31);
-                const uint32_t yd = hf ? YD_H1 : YD_H0, yo = hf ? YO_H1 : YO_H0, xo = hf ? XKQO_H1 : XKQO_H0;
+            // carries from earlier segments; block references G_15, G_47 and G_63
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int r = 32 * blk + i;
-                    const uint32_t o64 = sw128(r, c, 64);
-                    const float kh = bf(sm + STG_K, o64) * sinvk[r];
-                    const float qh = bf(sm + STG_Q, o64) * sinvq[r];
-                    const float a = Gl[i] - Gm;
-                    const float ed = __expf(a), ydf = __expf(-a);
-                    const float xk = kh * ed, xq = qh * ed, y = kh * ydf;
-                    st_bf(sm, XKQD + sw128(r, c, 128), xk);
-                    st_bf(sm, XKQD + sw128(64 + r, c, 128), xq);
-                    st_bf(sm, yd + sw128(r, cc, 64), y);
-                    st_bf(sm, QT + o64, xq * Emid);
-                    st_bf(sm, KT + o64, xk * Emid);
-                    st_bf(sm, KH + o64, y * Fkh);
-                    if (blk == 0) {
-                        st_bf(sm, yo + sw128(r, cc, 32), y * Foff);
-                    } else {
-                        st_bf(sm, xo + sw128(i, cc, 64), xk * Foff);
-                        st_bf(sm, xo + sw128(32 + i, cc, 64), xq * Foff);
+            for (int e8 = 0; e8 < 2; ++e8) {
+                float cum[4] = {0.f, 0.f, 0.f, 0.f}, carry[4] = {0.f, 0.f, 0.f, 0.f}, g15[4], g47[4];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    if (q == seg) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) carry[e] = cum[e];
+                    }
+                    const float4 a = *reinterpret_cast<const float4 *>(ssegt + q * 128 + 8 * jch + 4 * e8);
+                    cum[0] += a.x; cum[1] += a.y; cum[2] += a.z; cum[3] += a.w;
+                    if (q == 1) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) g15[e] = cum[e];
+                    }
+                    if (q == 5) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) g47[e] = cum[e];
                     }
                 }
-            } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int r = 32 * blk + i;
-                    const uint32_t o64 = sw128(r, c, 64);
-                    const float kh = bf(sm + STG_K, o64) * sinvk[r];
-                    const float qh = bf(sm + STG_Q, o64) * sinvq[r];
-                    const float eg = expf(Gl[i]);
-                    st_bf(sm, QT + o64, qh * eg);
-                    st_bf(sm, KT + o64, kh * eg);
-                    st_bf(sm, KH + o64, kh * expf(G63 - Gl[i]));
+                for (int e = 0; e < 4; ++e) {
+                    const int ee = 4 * e8 + e;
+                    G[0][ee] += carry[e];
+                    G[1][ee] += carry[e];
+                    Gm[ee] = blk ? g47[e] : g15[e];
+                    G47[ee] = g47[e];
+                    G63[ee] = cum[e];
+                    span_bad |= fabsf(G[0][ee] - Gm[ee]) > kSpanMax;
+                    span_bad |= fabsf(G[1][ee] - Gm[ee]) > kSpanMax;
                 }
+            }
+            if (seg == 7 && rq == 3) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) sGam[8 * jch + e] = expf(G63[e]);
+            }
+        }
+        const bool fb = __syncthreads_or(span_bad) != 0;
+
+        // ---------------- P2: bf16 operand tiles from the raw rows
+        {
+            const int hf = jch >> 3, jc = 8 * (jch & 7);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int r = row0 + u;
+                const uint32_t off = sw128_chunk(r, 8 * jch, 64);
+                float qq[8], kk[8];
+                unpack8(lds128(sm + STG_Q, off), qq);
+                unpack8(lds128(sm + STG_K, off), kk);
+                if (r >= L) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) { qq[e] = 0.f; kk[e] = 0.f; }
+                }
+                float t1[8], t2[8], t3[8];
+                if (!fb) {
+                    float xk[8], xq[8], y[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float a = G[u][e] - Gm[e];
+                        const float ed = __expf(a), ydf = __expf(-a);
+                        const float emid = __expf(Gm[e]);
+                        xk[e] = kk[e] * ed;
+                        xq[e] = qq[e] * ed;
+                        y[e] = kk[e] * ydf;
+                        t1[e] = xq[e] * emid;
+                        t2[e] = xk[e] * emid;
+                        t3[e] = y[e] * __expf(G63[e] - Gm[e]);
+                    }
+                    sts128(sm, XKQD + sw128_chunk(r, 8 * jch, 128), pack8(xk));
+                    sts128(sm, XKQD + sw128_chunk(64 + r, 8 * jch, 128), pack8(xq));
+                    sts128(sm, (hf ? YD_H1 : YD_H0) + sw128_chunk(r, jc, 64), pack8(y));
+                    if (blk == 0) {
+                        // off-diagonal column operand k_s e^{G_47 - G_s}, paired with the block-1 rows
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) y[e] *= __expf(G47[e] - Gm[e]);
+                        sts128(sm, (hf ? YO_H1 : YO_H0) + sw128_chunk(r, jc, 32), pack8(y));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float eg = expf(G[u][e]);
+                        t1[e] = qq[e] * eg;
+                        t2[e] = kk[e] * eg;
+                        t3[e] = kk[e] * expf(G63[e] - G[u][e]);
+                    }
+                }
+                sts128(sm, QT + off, pack8(t1));
+                sts128(sm, KT + off, pack8(t2));
+                sts128(sm, KH + off, pack8(t3));
             }
         }
         fence_proxy_async_smem();
@@ -273,15 +394,18 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         tc_fence_after();
 
         // ---------------- A_kk / A_qk products; next chunk's q, k, g loads
-        if (tid == 0 && !fb) {
-            if (has_next) { issue_qkg(t0 + C); qkg_out = true; }
+        // D1 (cols 0..63): rows 0..63 = A_kk, rows 64..127 = A_qk (diagonal 32-blocks valid).
+        // D2 (cols 64..95): A rows start at row 32, so lanes 0..31 = A_kk[32+i][0..31] and
+        // lanes 64..95 = A_qk[32+i][0..31]; the other lanes are unused.
+        if (tid == kTma && !fb && has_next) { issue_qkg(t0 + C); qkg_out = true; }
+        if (tid == kMma && !fb) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
                 const uint32_t yb = (kk >> 2) ? YD_H1 : YD_H0, ob = (kk >> 2) ? YO_H1 : YO_H0;
                 mma_bf16(tb + TM_A, sdesc_sw128(sb + XKQD + ko, 16, 1024),
                          sdesc_sw128(sb + yb + (kk & 3) * 32, 16, 1024), ID_A1, kk > 0);
-                mma_bf16(tb + TM_A + 64, sdesc_sw128(sb + XKQO_H0 + ko, 16, 1024),
+                mma_bf16(tb + TM_A + 64, sdesc_sw128(sb + XKQD + ko + 32 * 128, 16, 1024),
                          sdesc_sw128(sb + ob + (kk & 3) * 32, 16, 1024), ID_A2, kk > 0);
             }
             mma_commit(bar_mma);
@@ -291,101 +415,92 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         // ---------------- state refresh (overlaps the products above):
         // bf16 copy of S^T for this chunk's MMAs, and S^T diag(e^{G_last}) back into TMEM
         {
-            const int v = 32 * (warp & 3) + lane;
-            const int cb = (warp >> 2) * 64;
+            const int v = 32 * quarter + lane;
+            const int c0 = 32 * cgrp;
+            float x[32];
+            if (ci == 0) {
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                const int c0 = cb + 32 * b;
-                float x[32];
-                if (ci == 0) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        x[j] = p.S0 ? p.S0[sbase_state + (long long)(c0 + j) * D + v] : 0.f;
-                } else {
-                    tmem_ld32(tb + TM_S + lane_sel + c0, x);
-                    tmem_ld_wait();
-                }
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint4 pk;
-                    pk.x = pack_bf16x2(x[8 * q4 + 0], x[8 * q4 + 1]);
-                    pk.y = pack_bf16x2(x[8 * q4 + 2], x[8 * q4 + 3]);
-                    pk.z = pack_bf16x2(x[8 * q4 + 4], x[8 * q4 + 5]);
-                    pk.w = pack_bf16x2(x[8 * q4 + 6], x[8 * q4 + 7]);
-                    *reinterpret_cast<uint4 *>(sm + ST + sw128_chunk(v, c0 + 8 * q4, 128)) = pk;
-                }
-#pragma unroll
-                for (int j = 0; j < 32; ++j) x[j] *= sGam[c0 + j];
-                tmem_st32(tb + TM_S + lane_sel + c0, x);
+                for (int j = 0; j < 32; ++j) x[j] = p.S0 ? p.S0[sbase_state + (long long)(c0 + j) * D + v] : 0.f;
+            } else {
+                tmem_ld32(tb + TM_S + lane_sel + c0, x);
+                tmem_ld_wait();
             }
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) sts128(sm, ST + sw128_chunk(v, c0 + 8 * q4, 128), pack8(x + 8 * q4));
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] *= sGam[c0 + j];
+            tmem_st32(tb + TM_S + lane_sel + c0, x);
             tmem_st_wait();
         }
 
-        // ---------------- A results -> beta-scaled L (fp32) and A_qk (bf16 tile)
+        // ---------------- A results -> L (fp32, beta and key norms applied) and raw A_qk (bf16 tile)
         if (!fb) {
-            bool ok = mbar_wait(bar_mma, ph_mma, kWaitLimitNs);
-            ph_mma ^= 1;
-            if (tid == 0) mma_out = false;
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
+            if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
+            if (tid == kMma) mma_out = false;
             tc_fence_after();
-            if (warp < 4) {
-                const int i = lane;
-                float va[32], vb[32];
-                if (warp == 0 || warp == 2) tmem_ld32(tb + TM_A + lane_sel + 0, va);
-                else tmem_ld32(tb + TM_A + lane_sel + 32, va);
-                if (warp < 2) tmem_ld32(tb + TM_A + lane_sel + 64, vb);
+            const int i = lane;
+            // (quarter, column group) -> a 32-row x 16-column piece of D1 / D2
+            const bool has = (quarter & 1) == 0 || cgrp < 2;
+            const int col = (quarter & 1) ? 32 + 16 * cgrp : (cgrp < 2 ? 16 * cgrp : 64 + 16 * (cgrp - 2));
+            float va[16];
+            if (has) {
+                tmem_ld16(tb + TM_A + lane_sel + col, va);
                 tmem_ld_wait();
-                if (warp == 0) {
-                    const float b0 = sbeta[i], b1 = sbeta[32 + i];
+            }
+            if (quarter == 0) {
+                if (cgrp < 2) {  // A_kk rows 0..31, cols 16*cgrp..: s < i
+                    const float f = sbeta[i] * sinvk[i];
 #pragma unroll
-                    for (int s = 0; s < 32; ++s) {
-                        Lf[i * LDS + s] = s < i ? b0 * va[s] : 0.f;
-                        Lf[i * LDS + 32 + s] = 0.f;
-                        Lf[(32 + i) * LDS + s] = b1 * vb[s];
+                    for (int j = 0; j < 16; ++j) {
+                        const int s = 16 * cgrp + j;
+                        Lf[i * LDS + s] = s < i ? f * sinvk[s] * va[j] : 0.f;
                     }
-                } else if (warp == 1) {
-                    const float b1 = sbeta[32 + i];
+                } else {         // A_kk rows 32..63, cols 0..31 (all below the diagonal)
+                    const float f = sbeta[32 + i] * sinvk[32 + i];
 #pragma unroll
-                    for (int s = 0; s < 32; ++s) Lf[(32 + i) * LDS + 32 + s] = s < i ? b1 * va[s] : 0.f;
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4 pk;
-                        pk.x = pack_bf16x2(vb[8 * q4 + 0], vb[8 * q4 + 1]);
-                        pk.y = pack_bf16x2(vb[8 * q4 + 2], vb[8 * q4 + 3]);
-                        pk.z = pack_bf16x2(vb[8 * q4 + 4], vb[8 * q4 + 5]);
-                        pk.w = pack_bf16x2(vb[8 * q4 + 6], vb[8 * q4 + 7]);
-                        *reinterpret_cast<uint4 *>(sm + AQK + sw128_chunk(32 + i, 8 * q4, 64)) = pk;
+                    for (int j = 0; j < 16; ++j) {
+                        const int s = 16 * (cgrp - 2) + j;
+                        Lf[(32 + i) * LDS + s] = f * sinvk[s] * va[j];
                     }
-                } else {
-                    const int row = warp == 2 ? i : 32 + i;
-                    const int col0 = warp == 2 ? 0 : 32;
-                    float m[32];
+                }
+            } else if (quarter == 1) {
+                if (cgrp < 2) {  // A_kk rows 32..63, cols 32..63: s < i
+                    const float f = sbeta[32 + i] * sinvk[32 + i];
 #pragma unroll
-                    for (int s = 0; s < 32; ++s) m[s] = s <= i ? va[s] : 0.f;
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4 pk;
-                        pk.x = pack_bf16x2(m[8 * q4 + 0], m[8 * q4 + 1]);
-                        pk.y = pack_bf16x2(m[8 * q4 + 2], m[8 * q4 + 3]);
-                        pk.z = pack_bf16x2(m[8 * q4 + 4], m[8 * q4 + 5]);
-                        pk.w = pack_bf16x2(m[8 * q4 + 6], m[8 * q4 + 7]);
-                        *reinterpret_cast<uint4 *>(sm + AQK + sw128_chunk(row, col0 + 8 * q4, 64)) = pk;
-                        if (warp == 2)
-                            *reinterpret_cast<uint4 *>(sm + AQK + sw128_chunk(row, 32 + 8 * q4, 64)) =
-                                make_uint4(0u, 0u, 0u, 0u);
+                    for (int j = 0; j < 16; ++j) {
+                        const int s = 16 * cgrp + j;
+                        Lf[(32 + i) * LDS + 32 + s] = s < i ? f * sinvk[32 + s] * va[j] : 0.f;
                     }
+                }
+            } else if (quarter == 2) {
+                if (cgrp < 2) {  // A_qk rows 0..31, cols 0..31: s <= i
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) va[j] = 16 * cgrp + j <= i ? va[j] : 0.f;
+                    row16_to_tile(sm, AQK, i, 16 * cgrp, 64, va);
+                } else {         // A_qk rows 32..63, cols 0..31
+                    row16_to_tile(sm, AQK, 32 + i, 16 * (cgrp - 2), 64, va);
+                }
+            } else {
+                if (cgrp < 2) {  // A_qk rows 32..63, cols 32..63: s <= i
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) va[j] = 16 * cgrp + j <= i ? va[j] : 0.f;
+                    row16_to_tile(sm, AQK, 32 + i, 32 + 16 * cgrp, 64, va);
+                } else {         // A_qk rows 0..31, cols 32..63 are zero
+                    const int c0 = 32 + 16 * (cgrp - 2);
+                    sts128(sm, AQK + sw128_chunk(i, c0, 64), make_uint4(0u, 0u, 0u, 0u));
+                    sts128(sm, AQK + sw128_chunk(i, c0 + 8, 64), make_uint4(0u, 0u, 0u, 0u));
                 }
             }
         } else {
-            // exact A_kk / A_qk on CUDA cores: warp per row r, lanes over channels,
+            // exact A_kk / A_qk on CUDA cores (raw rows): warp per row r, lanes over channels,
             // walking s downwards while accumulating the gate between s and r
             for (int r = warp; r < C; r += NT / 32) {
                 float kr[4], qr[4], dg[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const uint32_t o = sw128(r, lane + 32 * u, 64);
-                    kr[u] = bf(sm + STG_K, o) * sinvk[r];
-                    qr[u] = bf(sm + STG_Q, o) * sinvq[r];
+                    kr[u] = r < L ? bf(sm + STG_K, o) : 0.f;
+                    qr[u] = r < L ? bf(sm + STG_Q, o) : 0.f;
                     dg[u] = 0.f;
                 }
                 for (int s = r; s >= 0; --s) {
@@ -393,7 +508,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const uint32_t o = sw128(s, lane + 32 * u, 64);
-                        const float e = expf(dg[u]) * bf(sm + STG_K, o) * sinvk[s];
+                        const float e = expf(dg[u]) * (s < L ? bf(sm + STG_K, o) : 0.f);
                         akk = fmaf(kr[u], e, akk);
                         aqk = fmaf(qr[u], e, aqk);
                         float gv = 0.f;
@@ -405,112 +520,127 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                     }
                     akk = warp_sum(akk); aqk = warp_sum(aqk);
                     if (lane == 0) {
-                        Lf[r * LDS + s] = s < r ? sbeta[r] * akk : 0.f;
+                        Lf[r * LDS + s] = s < r ? sbeta[r] * sinvk[r] * sinvk[s] * akk : 0.f;
                         st_bf(sm, AQK + sw128(r, s, 64), aqk);
                     }
                 }
-                for (int s = r + 1 + lane; s < C; s += 32) {
-                    Lf[r * LDS + s] = 0.f;
-                    st_bf(sm, AQK + sw128(r, s, 64), 0.f);
-                }
+                for (int s = r + 1 + lane; s < C; s += 32) st_bf(sm, AQK + sw128(r, s, 64), 0.f);
             }
             fence_proxy_async_smem();
             __syncthreads();
-            if (tid == 0 && has_next) { issue_qkg(t0 + C); qkg_out = true; }
+            if (tid == kTma && has_next) { issue_qkg(t0 + C); qkg_out = true; }
         }
         __syncthreads();
 
-        // ---------------- T = (I + L)^-1 by blocks: diagonal 32x32 by forward substitution
-        if (warp < 2) {
+        // ---------------- T = (I + L)^-1 on 16x16 blocks
+        // diagonal blocks by a column sweep (lane j = column j): once t[k] is final it
+        // updates every later row, so the dependent chain is 16 steps long
+        if (warp < 4 && lane < 16) {
             const int b = warp, j = lane;
-            float t[32];
+            float t[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                float s = i == j ? 1.f : 0.f;
-                const float *Lrow = Lf + (32 * b + i) * LDS + 32 * b;
+            for (int i = 0; i < 16; ++i) t[i] = i == j ? 1.f : 0.f;
 #pragma unroll
-                for (int k = 0; k < i; ++k) s = fmaf(-Lrow[k], t[k], s);
-                t[i] = s;
+            for (int k = 0; k < 15; ++k) {
+#pragma unroll
+                for (int i = k + 1; i < 16; ++i) t[i] = fmaf(-Lf[(16 * b + i) * LDS + 16 * b + k], t[k], t[i]);
             }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) Tf[(32 * b + i) * LDS + 32 * b + j] = t[i];
-        }
-        __syncthreads();
-        {   // M1 = L10 T00
-            const int j = lane;
-#pragma unroll
-            for (int ii = 0; ii < 4; ++ii) {
-                const int i = warp * 4 + ii;
-                float acc = 0.f;
-#pragma unroll 8
-                for (int k = 0; k < 32; ++k) acc = fmaf(Lf[(32 + i) * LDS + k], Tf[k * LDS + j], acc);
-                Mf[i * 33 + j] = acc;
+            for (int i = 0; i < 16; ++i) Tf[(16 * b + i) * LDT + 16 * b + j] = t[i];
+        } else if (warp >= 4) {
+            // zero the blocks above the diagonal, which the block products read
+            for (int e = tid - 128; e < 6 * 256; e += NT - 128) {
+                const int bid = e >> 8, i = (e >> 4) & 15, j = e & 15;
+                const int bi = bid < 3 ? 0 : bid < 5 ? 1 : 2;
+                const int bj = bid < 3 ? bid + 1 : bid < 5 ? bid - 1 : 3;
+                Tf[(16 * bi + i) * LDT + 16 * bj + j] = 0.f;
             }
         }
         __syncthreads();
-        {   // T10 = -T11 M1
-            const int j = lane;
+        // block rows I = 1..3:  T[I, J<I] = -T_II sum_{K<I} L_IK T_KJ, on warp-level tf32
+        // MMAs; warp w < 2I owns the 8 output columns 8w .. 8w+7
+        {
+            const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
-            for (int ii = 0; ii < 4; ++ii) {
-                const int i = warp * 4 + ii;
-                float acc = 0.f;
-#pragma unroll 8
-                for (int k = 0; k < 32; ++k) acc = fmaf(Tf[(32 + i) * LDS + 32 + k], Mf[k * 33 + j], acc);
-                Tf[(32 + i) * LDS + j] = -acc;
+            for (int I = 1; I < 4; ++I) {
+                const bool act = warp < 2 * I;
+                const int n0 = 8 * warp;
+                if (act) {
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    const float *La = Lf + (16 * I + g) * LDS, *Lb = Lf + (16 * I + g + 8) * LDS;
+#pragma unroll
+                    for (int ks = 0; ks < 2 * I; ++ks) {
+                        const int k0 = 8 * ks;
+                        const uint32_t a[4] = {to_tf32(La[k0 + t4]), to_tf32(Lb[k0 + t4]), to_tf32(La[k0 + t4 + 4]),
+                                               to_tf32(Lb[k0 + t4 + 4])};
+                        const uint32_t b[2] = {to_tf32(Tf[(k0 + t4) * LDT + n0 + g]),
+                                               to_tf32(Tf[(k0 + t4 + 4) * LDT + n0 + g])};
+                        mma_tf32_16x8x8(d, a, b);
+                    }
+                    Rf[g * LDR + n0 + 2 * t4] = d[0];
+                    Rf[g * LDR + n0 + 2 * t4 + 1] = d[1];
+                    Rf[(g + 8) * LDR + n0 + 2 * t4] = d[2];
+                    Rf[(g + 8) * LDR + n0 + 2 * t4 + 1] = d[3];
+                }
+                __syncthreads();
+                if (act) {
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    const float *Ta = Tf + (16 * I + g) * LDT + 16 * I, *Tb = Tf + (16 * I + g + 8) * LDT + 16 * I;
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        const int k0 = 8 * ks;
+                        const uint32_t a[4] = {to_tf32(Ta[k0 + t4]), to_tf32(Tb[k0 + t4]), to_tf32(Ta[k0 + t4 + 4]),
+                                               to_tf32(Tb[k0 + t4 + 4])};
+                        const uint32_t b[2] = {to_tf32(Rf[(k0 + t4) * LDR + n0 + g]),
+                                               to_tf32(Rf[(k0 + t4 + 4) * LDR + n0 + g])};
+                        mma_tf32_16x8x8(d, a, b);
+                    }
+                    Tf[(16 * I + g) * LDT + n0 + 2 * t4] = -d[0];
+                    Tf[(16 * I + g) * LDT + n0 + 2 * t4 + 1] = -d[1];
+                    Tf[(16 * I + g + 8) * LDT + n0 + 2 * t4] = -d[2];
+                    Tf[(16 * I + g + 8) * LDT + n0 + 2 * t4 + 1] = -d[3];
+                }
+                __syncthreads();
             }
         }
-        __syncthreads();
-        // T' = T diag(beta) as a bf16 tile [r][s]
-        for (int q = tid; q < 512; q += NT) {
-            const int r = q >> 3, s0 = (q & 7) * 8;
-            float m[8];
+        // T' tiles: T diag(beta) for U and T diag(beta / |k|) for W (one chunk of each per thread)
+        {
+            const int r = tid >> 3, s0 = (tid & 7) * 8;
+            float mu[8], mw[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int s = s0 + e;
-                m[e] = s <= r ? Tf[r * LDS + s] * sbeta[s] : 0.f;
+                mu[e] = s <= r ? Tf[r * LDT + s] * sbeta[s] : 0.f;
+                mw[e] = mu[e] * sinvk[s];
             }
-            uint4 pk;
-            pk.x = pack_bf16x2(m[0], m[1]); pk.y = pack_bf16x2(m[2], m[3]);
-            pk.z = pack_bf16x2(m[4], m[5]); pk.w = pack_bf16x2(m[6], m[7]);
-            *reinterpret_cast<uint4 *>(sm + TP + sw128_chunk(r, s0, 64)) = pk;
+            sts128(sm, TPU + sw128_chunk(r, s0, 64), pack8(mu));
+            sts128(sm, TPW + sw128_chunk(r, s0, 64), pack8(mw));
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
 
-        // ---------------- U^T = V^T T'^T, W^T = Ktil^T T'^T
-        if (tid == 0) {
+        // ---------------- U^T = V^T T_u^T, W^T = Ktil^T T_w^T
+        if (tid == kMma) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t bdesc = sdesc_sw128(sb + TP + kk * 32, 16, 1024);
-                mma_bf16(tb + TM_U, sdesc_sw128(sb + STG_V + kk * 2048, 8192, 1024), bdesc, ID_UW, kk > 0);
-                mma_bf16(tb + TM_W, sdesc_sw128(sb + KT + kk * 2048, 8192, 1024), bdesc, ID_UW, kk > 0);
+                mma_bf16(tb + TM_U, sdesc_sw128(sb + STG_V + kk * 2048, 8192, 1024),
+                         sdesc_sw128(sb + TPU + kk * 32, 16, 1024), ID_UW, kk > 0);
+                mma_bf16(tb + TM_W, sdesc_sw128(sb + KT + kk * 2048, 8192, 1024),
+                         sdesc_sw128(sb + TPW + kk * 32, 16, 1024), ID_UW, kk > 0);
             }
             mma_commit(bar_mma);
             mma_out = true;
         }
-        {
-            bool ok = mbar_wait(bar_mma, ph_mma, kWaitLimitNs);
-            ph_mma ^= 1;
-            if (tid == 0) mma_out = false;
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-        }
+        if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
+        if (tid == kMma) mma_out = false;
         tc_fence_after();
         {   // W^T (lane c, columns r) -> bf16 tile [c][r]
-            const int cr = 32 * (warp & 3) + lane, r0 = (warp >> 2) * 32;
-            float x[32];
-            tmem_ld32(tb + TM_W + lane_sel + r0, x);
+            float x[16];
+            tmem_ld16(tb + TM_W + lane_sel + 16 * cgrp, x);
             tmem_ld_wait();
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint4 pk;
-                pk.x = pack_bf16x2(x[8 * q4 + 0], x[8 * q4 + 1]);
-                pk.y = pack_bf16x2(x[8 * q4 + 2], x[8 * q4 + 3]);
-                pk.z = pack_bf16x2(x[8 * q4 + 4], x[8 * q4 + 5]);
-                pk.w = pack_bf16x2(x[8 * q4 + 6], x[8 * q4 + 7]);
-                *reinterpret_cast<uint4 *>(sm + WT + sw128_chunk(cr, r0 + 8 * q4, 128)) = pk;
-            }
+            row16_to_tile(sm, WT, 32 * quarter + lane, 16 * cgrp, 128, x);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -518,8 +648,8 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         tc_fence_after();
 
         // ---------------- D^T = U^T - S^T W^T ; O^T = S^T Qtil^T ; next chunk's v load
-        if (tid == 0) {
-            if (has_next) { issue_v(t0 + C); v_out = true; }
+        if (tid == kTma && has_next) { issue_v(t0 + C); v_out = true; }
+        if (tid == kMma) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
                 const uint64_t adesc = sdesc_sw128(sb + ST + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
@@ -530,35 +660,25 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
             mma_commit(bar_mma);
             mma_out = true;
         }
-        {
-            bool ok = mbar_wait(bar_mma, ph_mma, kWaitLimitNs);
-            ph_mma ^= 1;
-            if (tid == 0) mma_out = false;
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-        }
+        if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
+        if (tid == kMma) mma_out = false;
         tc_fence_after();
-        {   // D^T (lane v, columns s) -> bf16 tile [v][s]
-            const int v = 32 * (warp & 3) + lane, s0 = (warp >> 2) * 32;
-            float x[32];
-            tmem_ld32(tb + TM_U + lane_sel + s0, x);
+        {   // D^T (lane v, columns s), times |k_s|^-1 -> bf16 tile [v][s]
+            float x[16];
+            const int s0 = 16 * cgrp;
+            tmem_ld16(tb + TM_U + lane_sel + s0, x);
             tmem_ld_wait();
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                uint4 pk;
-                pk.x = pack_bf16x2(x[8 * q4 + 0], x[8 * q4 + 1]);
-                pk.y = pack_bf16x2(x[8 * q4 + 2], x[8 * q4 + 3]);
-                pk.z = pack_bf16x2(x[8 * q4 + 4], x[8 * q4 + 5]);
-                pk.w = pack_bf16x2(x[8 * q4 + 6], x[8 * q4 + 7]);
-                *reinterpret_cast<uint4 *>(sm + DT + sw128_chunk(v, s0 + 8 * q4, 128)) = pk;
-            }
+            for (int j = 0; j < 16; ++j) x[j] *= sinvk[s0 + j];
+            row16_to_tile(sm, DT, 32 * quarter + lane, s0, 128, x);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
 
-        // ---------------- O^T += D^T A_qk^T ; S^T += D^T Khat
-        if (tid == 0) {
+        // ---------------- O^T += D~^T A_qk^T ; S^T += D~^T Khat
+        if (tid == kMma) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t adesc = sdesc_sw128(sb + DT + kk * 32, 16, 1024);
@@ -568,23 +688,31 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
             mma_commit(bar_mma);
             mma_out = true;
         }
-        {
-            bool ok = mbar_wait(bar_mma, ph_mma, kWaitLimitNs);
-            ph_mma ^= 1;
-            if (tid == 0) mma_out = false;
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-        }
+        if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
+        if (tid == kMma) mma_out = false;
         tc_fence_after();
-        {   // O^T (lane v, columns r) -> o[t0 + r, h, v]
-            const int v = 32 * (warp & 3) + lane, r0 = (warp >> 2) * 32;
-            float x[32];
-            tmem_ld32(tb + TM_O + lane_sel + r0, x);
+        {   // O^T (lane v, columns r) -> plain [r][v] tile, scale and 1/|q_r| applied
+            float x[16];
+            const int v = 32 * quarter + lane, r0 = 16 * cgrp;
+            tmem_ld16(tb + TM_O + lane_sel + r0, x);
             tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int r = r0 + j;
+                *reinterpret_cast<__nv_bfloat16 *>(sm + OT + r * 256 + v * 2) =
+                    __float2bfloat16_rn(p.scale * sinvq[r] * x[j]);
+            }
+        }
+        __syncthreads();
+        {   // coalesced 16-byte stores of the rows that belong to this sequence
             __nv_bfloat16 *O = static_cast<__nv_bfloat16 *>(p.o);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int r = r0 + j;
-                if (r < L) O[((t0 + r) * H + h) * D + v] = __float2bfloat16_rn(p.scale * x[j]);
+            for (int m = 0; m < 2; ++m) {
+                const int qd = tid + NT * m, r = qd >> 4, c16 = qd & 15;
+                if (r < L) {
+                    const uint4 val = lds128(sm + OT, r * 256 + c16 * 16);
+                    *reinterpret_cast<uint4 *>(O + ((t0 + r) * H + h) * D + c16 * 8) = val;
+                }
             }
         }
         tc_fence_before();
@@ -593,30 +721,26 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     }
 
     if (!aborted && p.S_out) {
-        const int v = 32 * (warp & 3) + lane;
-        const int cb = (warp >> 2) * 64;
+        const int v = 32 * quarter + lane;
+        const int c0 = 32 * cgrp;
+        float x[32];
+        if (nchunks == 0) {
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
-            const int c0 = cb + 32 * b;
-            float x[32];
-            if (nchunks == 0) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) x[j] = p.S0 ? p.S0[sbase_state + (long long)(c0 + j) * D + v] : 0.f;
-            } else {
-                tmem_ld32(tb + TM_S + lane_sel + c0, x);
-                tmem_ld_wait();
-            }
-#pragma unroll
-            for (int j = 0; j < 32; ++j) p.S_out[sbase_state + (long long)(c0 + j) * D + v] = x[j];
+            for (int j = 0; j < 32; ++j) x[j] = p.S0 ? p.S0[sbase_state + (long long)(c0 + j) * D + v] : 0.f;
+        } else {
+            tmem_ld32(tb + TM_S + lane_sel + c0, x);
+            tmem_ld_wait();
         }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) p.S_out[sbase_state + (long long)(c0 + j) * D + v] = x[j];
     }
 
-    if (aborted && tid == 0) {
+    if (aborted && (tid == kMma || tid == kTma)) {
         // let copies and products already in flight land before the CTA leaves
         if (qkg_out) mbar_wait(bar_qkg, ph_qkg, kWaitLimitNs);
         if (v_out) mbar_wait(bar_v, ph_v, kWaitLimitNs);
         if (mma_out) mbar_wait(bar_mma, ph_mma, kWaitLimitNs);
-        if (P.status) atomicOr(P.status, 1);
+        if (P.status && tid == kMma) atomicOr(P.status, 1);
     }
     tc_fence_before();
     __syncthreads();
