@@ -62,8 +62,9 @@ constexpr uint32_t QT = AOPS + 73728, KT = QT + 16384, KH = KT + 16384, ST = KH 
 constexpr uint32_t MISC = ST + 32768;
 constexpr uint32_t M_BETA = MISC, M_INVQ = MISC + 256, M_INVK = MISC + 512, M_GAM = MISC + 768,
                    M_BAR = MISC + 1280, M_TMEM = MISC + 1312, M_RED = MISC + 1536,  // [q|k][half][64] f32
-                   M_SEG = MISC + 2560;                                             // [8][128] f32
-constexpr uint32_t SMEM_BYTES = M_SEG + 4096;
+                   M_SEG = MISC + 2560,   // [8][128] f32: segment totals, then exclusive carries
+                   M_REF = MISC + 6656;   // [3][128] f32: G_15, G_47, G_63 per channel
+constexpr uint32_t SMEM_BYTES = M_REF + 1536;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
 static_assert(YO_H1 + 4096 <= XKQD, "view 1");
 static_assert(LF + 64 * LDS * 4 <= TF && TF + 64 * LDT * 4 <= RF && RF + 16 * LDR * 4 <= AQK, "view 2");
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     float *sGam = reinterpret_cast<float *>(sm + M_GAM);
     float *sred = reinterpret_cast<float *>(sm + M_RED);
     float *ssegt = reinterpret_cast<float *>(sm + M_SEG);
+    float *sref = reinterpret_cast<float *>(sm + M_REF);
     float *Lf = reinterpret_cast<float *>(sm + LF);
     float *Tf = reinterpret_cast<float *>(sm + TF);
     float *Rf = reinterpret_cast<float *>(sm + RF);
@@ -290,48 +292,43 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         }
         __syncthreads();
         if (tid < 128) {
-            const int r = tid & 63, which = tid >> 6;
+            // one thread per channel: exclusive carries over the 8 segments, block references
+            float cum = 0.f;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float tq = ssegt[q * 128 + tid];
+                ssegt[q * 128 + tid] = cum;
+                cum += tq;
+                if (q == 1) sref[tid] = cum;        // G_15
+                if (q == 5) sref[128 + tid] = cum;  // G_47
+            }
+            sref[256 + tid] = cum;                  // G_63
+            sGam[tid] = expf(cum);
+        } else if (tid < 256) {
+            const int r = tid & 63, which = (tid >> 6) & 1;
             const float ssum = sred[which * 128 + r] + sred[which * 128 + 64 + r];
             const float inv = r < L ? (p.use_l2 ? rsqrtf(ssum + kL2Eps) : 1.f) : 0.f;
             (which ? sinvk : sinvq)[r] = inv;
         }
+        __syncthreads();
         {
-            // carries from earlier segments; block references G_15, G_47 and G_63
+            auto ld8 = [&](const float *src, float (&dst)[8]) {
+                const float4 a = *reinterpret_cast<const float4 *>(src + 8 * jch);
+                const float4 b = *reinterpret_cast<const float4 *>(src + 8 * jch + 4);
+                dst[0] = a.x; dst[1] = a.y; dst[2] = a.z; dst[3] = a.w;
+                dst[4] = b.x; dst[5] = b.y; dst[6] = b.z; dst[7] = b.w;
+            };
+            float carry[8];
+            ld8(ssegt + seg * 128, carry);
+            ld8(sref + (blk ? 128 : 0), Gm);
+            ld8(sref + 128, G47);
+            ld8(sref + 256, G63);
 #pragma unroll
-            for (int e8 = 0; e8 < 2; ++e8) {
-                float cum[4] = {0.f, 0.f, 0.f, 0.f}, carry[4] = {0.f, 0.f, 0.f, 0.f}, g15[4], g47[4];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    if (q == seg) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) carry[e] = cum[e];
-                    }
-                    const float4 a = *reinterpret_cast<const float4 *>(ssegt + q * 128 + 8 * jch + 4 * e8);
-                    cum[0] += a.x; cum[1] += a.y; cum[2] += a.z; cum[3] += a.w;
-                    if (q == 1) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) g15[e] = cum[e];
-                    }
-                    if (q == 5) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) g47[e] = cum[e];
-                    }
-                }
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int ee = 4 * e8 + e;
-                    G[0][ee] += carry[e];
-                    G[1][ee] += carry[e];
-                    Gm[ee] = blk ? g47[e] : g15[e];
-                    G47[ee] = g47[e];
-                    G63[ee] = cum[e];
-                    span_bad |= fabsf(G[0][ee] - Gm[ee]) > kSpanMax;
-                    span_bad |= fabsf(G[1][ee] - Gm[ee]) > kSpanMax;
-                }
-            }
-            if (seg == 7 && rq == 3) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) sGam[8 * jch + e] = expf(G63[e]);
+            for (int e = 0; e < 8; ++e) {
+                G[0][e] += carry[e];
+                G[1][e] += carry[e];
+                span_bad |= fabsf(G[0][e] - Gm[e]) > kSpanMax;
+                span_bad |= fabsf(G[1][e] - Gm[e]) > kSpanMax;
             }
         }
         const bool fb = __syncthreads_or(span_bad) != 0;
