@@ -51,28 +51,29 @@ constexpr uint32_t AOPS = 65536;                                            // 7
 // view 1, operands of the A_kk / A_qk products
 constexpr uint32_t YD_H0 = AOPS + 0, YD_H1 = AOPS + 8192, YO_H0 = AOPS + 16384, YO_H1 = AOPS + 20480;
 constexpr uint32_t XKQD = AOPS + 40960;  // 2 halves x [128 rows][128 B]: rows 0..63 k, 64..127 q
+constexpr uint32_t NRM = AOPS + 24576;   // [q|k][16 warps][64 rows] f32 partial squared norms
 // view 2, after those products: fp32 solve buffers, T' tiles, then W^T, D^T and the output tile
 constexpr int LDS = 65;  // padded fp32 row stride of L (64x64)
 constexpr int LDT = 68;  // fp32 row stride of T (64x64)
 constexpr int LDR = 52;  // fp32 row stride of the 16x48 block-row buffer
-constexpr uint32_t LF = AOPS + 0, TF = AOPS + 16896, RF = AOPS + 34304, AQK = AOPS + 40960;
-constexpr uint32_t TPU = AOPS + 49152, TPW = AOPS + 57344;  // T diag(beta), T diag(beta / |k|)
+// (the k rows of XKQD, 40960..49152 and 57344..65536, stay live until the W products)
+constexpr uint32_t LF = AOPS + 0, TF = AOPS + 16896, RF = AOPS + 34304, AQK = AOPS + 49152;
 constexpr uint32_t WT = AOPS + 0, DT = AOPS + 16384, OT = AOPS + 57344;  // OT: [64][128] bf16, plain
-constexpr uint32_t QT = AOPS + 73728, KT = QT + 16384, KH = KT + 16384, ST = KH + 16384;  // ST: 32 KiB
+constexpr uint32_t QT = AOPS + 73728, TPU = QT + 16384, TPW = TPU + 8192;  // T diag(beta), T diag(beta/|k|)
+constexpr uint32_t KH = TPW + 8192, ST = KH + 16384;                       // ST: 32 KiB
 constexpr uint32_t MISC = ST + 32768;
 constexpr uint32_t M_BETA = MISC, M_INVQ = MISC + 256, M_INVK = MISC + 512, M_GAM = MISC + 768,
-                   M_BAR = MISC + 1280, M_TMEM = MISC + 1312, M_RED = MISC + 1536,  // [q|k][half][64] f32
-                   M_SEG = MISC + 2560,   // [8][128] f32: segment totals, then exclusive carries
-                   M_REF = MISC + 6656;   // [3][128] f32: G_15, G_47, G_63 per channel
-constexpr uint32_t SMEM_BYTES = M_REF + 1536;
+                   M_BAR = MISC + 1280, M_TMEM = MISC + 1312,
+                   M_EW = MISC + 1536;    // [2][128] f32: e^{G_15}, e^{G_47} per channel
+constexpr uint32_t SMEM_BYTES = M_EW + 1024;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
-static_assert(YO_H1 + 4096 <= XKQD, "view 1");
-static_assert(LF + 64 * LDS * 4 <= TF && TF + 64 * LDT * 4 <= RF && RF + 16 * LDR * 4 <= AQK, "view 2");
-static_assert(TPW + 8192 <= AOPS + 73728 && DT + 16384 <= AQK && OT + 16384 <= AOPS + 73728, "view 2 tiles");
+static_assert(YO_H1 + 4096 <= NRM && NRM + 8192 <= XKQD, "view 1");
+static_assert(LF + 64 * LDS * 4 <= TF && TF + 64 * LDT * 4 <= RF && RF + 16 * LDR * 4 <= XKQD, "view 2");
+static_assert(AQK + 8192 <= XKQD + 16384 + 8192 && DT + 16384 <= XKQD && OT + 16384 <= AOPS + 73728, "view 2 tiles");
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
 // ---- tensor memory columns ----
-constexpr uint32_t TM_S = 0, TM_U = 128, TM_W = 192, TM_O = 256, TM_A = 320, TM_COLS = 512;
+constexpr uint32_t TM_S = 0, TM_U = 128, TM_W = 192, TM_O = 256, TM_A = 320, TM_W1 = 416, TM_COLS = 512;
 
 // ---- instruction descriptors ----
 constexpr uint32_t ID_A1 = idesc_bf16(128, 64, false, false);
@@ -117,6 +118,36 @@ __device__ __forceinline__ float bf(const uint8_t *base, uint32_t off) {
 __device__ __forceinline__ void st_bf(uint8_t *base, uint32_t off, float x) {
     *reinterpret_cast<__nv_bfloat16 *>(base + off) = __float2bfloat16_rn(x);
 }
+__device__ __forceinline__ uint32_t pack2(float2 v) {
+    __nv_bfloat162 b = __float22bfloat162_rn(v);
+    return *reinterpret_cast<uint32_t *>(&b);
+}
+__device__ __forceinline__ void unpack8x2(const uint4 &u, float2 (&f)[4]) {
+    const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = __bfloat1622float2(b[i]);
+}
+__device__ __forceinline__ uint4 pack8x2(const float2 (&f)[4]) {
+    return make_uint4(pack2(f[0]), pack2(f[1]), pack2(f[2]), pack2(f[3]));
+}
+// 2^x on the special-function unit (the approximate exp2 instruction)
+__device__ __forceinline__ float ex2a(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// 1/x for normal positive x on the FMA pipe: a bit-pattern first estimate
+// (reciprocal ~ 2^(2*127) / x read off the exponent/mantissa bits) refined by two
+// Newton-Raphson steps y <- y (2 - x y); relative error ~1e-5.
+__device__ __forceinline__ float2 rcp2_nr(float2 x) {
+    float2 y = make_float2(__int_as_float(0x7EF311C3 - __float_as_int(x.x)),
+                           __int_as_float(0x7EF311C3 - __float_as_int(x.y)));
+    const float2 nx = make_float2(-x.x, -x.y), two = make_float2(2.f, 2.f);
+    y = __fmul2_rn(y, __ffma2_rn(nx, y, two));
+    y = __fmul2_rn(y, __ffma2_rn(nx, y, two));
+    return y;
+}
+
 // 16 fp32 values of one TMEM row to two 16-byte chunks of a swizzled bf16 tile row
 __device__ __forceinline__ void row16_to_tile(uint8_t *sm, uint32_t tile, int row, int col0, int rows,
                                               const float (&x)[16]) {
@@ -152,12 +183,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     float *sinvq = reinterpret_cast<float *>(sm + M_INVQ);
     float *sinvk = reinterpret_cast<float *>(sm + M_INVK);
     float *sGam = reinterpret_cast<float *>(sm + M_GAM);
-    float *sred = reinterpret_cast<float *>(sm + M_RED);
-    float *ssegt = reinterpret_cast<float *>(sm + M_SEG);
-    float *sref = reinterpret_cast<float *>(sm + M_REF);
+    float *sEw = reinterpret_cast<float *>(sm + M_EW);
     float *Lf = reinterpret_cast<float *>(sm + LF);
     float *Tf = reinterpret_cast<float *>(sm + TF);
-    float *Rf = reinterpret_cast<float *>(sm + RF);
 
     if (warp == 0) { tmem_alloc(s_tmem, TM_COLS); tmem_relinquish(); }
     if (tid == 32) {
@@ -170,6 +198,14 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     tc_fence_after();
     const uint32_t tb = *s_tmem;
     const uint32_t sb = smem_u32(sm);
+    // descriptor of byte offset `off` from the tile base: the start-address field is the
+    // only one that changes, so each descriptor is one add on a precomputed base
+    const uint64_t dK = sdesc_sw128(sb, 16, 1024);    // K-major operands
+    const uint64_t dM = sdesc_sw128(sb, 8192, 1024);  // MN-major operands (atoms 8 KiB apart)
+    const uint64_t dX = sdesc_sw128(sb, 16384, 1024); // MN-major view of XKQD (halves 16 KiB apart)
+    auto dk = [&](uint32_t off) { return dK + (uint64_t)(off >> 4); };
+    auto dm = [&](uint32_t off) { return dM + (uint64_t)(off >> 4); };
+    auto dx = [&](uint32_t off) { return dX + (uint64_t)(off >> 4); };
     const int quarter = warp & 3;                               // TMEM lanes 32*quarter .. +31
     const uint32_t lane_sel = (uint32_t)(32 * quarter) << 16;
     const int cgrp = warp >> 2;                                  // column group of TMEM phases
@@ -186,9 +222,11 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         mbar_arrive_expect_tx(bar_v, 16384);
         for (int hf = 0; hf < 2; ++hf) tma_load_3d(sm + STG_V + hf * 8192, &P.tv, bar_v, hf * 64, h, (int)t);
     };
-    // a bounded wait on an mbarrier phase by every thread; true if the CTA must stop
+    // a bounded wait on an mbarrier phase: one warp polls, the others park in the
+    // CTA barrier (no issue slots spent polling); true if the CTA must stop
     auto wait_all = [&](uint64_t *bar, uint32_t &ph) -> bool {
-        const bool ok = mbar_wait(bar, ph, kWaitLimitNs);
+        bool ok = true;
+        if (warp == 0) ok = mbar_wait(bar, ph, kWaitLimitNs);
         ph ^= 1;
         return __syncthreads_or(!ok) != 0;
     };
@@ -206,15 +244,12 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     float beta_next = 0.f;
     if (tid < C && bos + tid < eos) beta_next = __bfloat162float(bt[(bos + tid) * H + h]);
 
-    // thread -> (16-byte chunk of 8 channels, 2 consecutive rows) for the row-layout phases.
-    // Warp w owns channel half (w & 1) and the 8-row segment (w >> 1); the 8 lanes of each
-    // 128-bit access phase share their rows and take 8 different chunks, so the 128-byte
-    // swizzle spreads them over all banks.
-    const int seg = warp >> 1;
-    const int jch = 8 * (warp & 1) + (lane & 7);   // channels 8*jch .. 8*jch+7
-    const int rq = lane >> 3;
-    const int row0 = 8 * seg + 2 * rq;             // rows row0, row0 + 1
-    const int blk = seg >> 2;                      // 32-row block of those rows
+    // thread -> (16-byte chunk of 8 channels, 2 consecutive rows) for the row-layout phases:
+    // warp w owns channels 8w .. 8w+7 for all 64 rows, lane l rows 2l and 2l+1, so the
+    // in-chunk cumsum is a scan across the lanes of one warp.
+    const int jch = warp;
+    const int row0 = 2 * lane;
+    const int blk = lane >> 4;                     // 32-row block of those rows
 
     for (int ci = 0; ci < nchunks && !aborted; ++ci) {
         const long long t0 = bos + (long long)ci * C;
@@ -229,106 +264,65 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
 
         // ---------------- inputs of this chunk
         {
-            const bool ok = mbar_wait(bar_qkg, ph_qkg, kWaitLimitNs) && mbar_wait(bar_v, ph_v, kWaitLimitNs);
+            bool ok = true;
+            if (warp == 0) ok = mbar_wait(bar_qkg, ph_qkg, kWaitLimitNs) && mbar_wait(bar_v, ph_v, kWaitLimitNs);
             ph_qkg ^= 1; ph_v ^= 1;
             if (tid == kTma) qkg_out = v_out = false;
             if (__syncthreads_or(!ok)) { aborted = true; break; }
         }
 
-        // ---------------- P1: gate cumsum and row norms
+        // ---------------- P1: gate cumsum, in-warp scan over the 64 rows
         float G[2][8], Gm[8], G47[8], G63[8];
         bool span_bad = false;
         {
-            float tot[8], sq[2], sk[2];
+            float tot[8];
+            {
+                float2 tt[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) tot[e] = 0.f;
+                for (int e = 0; e < 4; ++e) tt[e] = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int r = row0 + u;
-                const uint32_t off = sw128_chunk(r, 8 * jch, 64);
-                float gg[8], qq[8], kk[8];
-                unpack8(lds128(sm + STG_G, off), gg);
-                unpack8(lds128(sm + STG_Q, off), qq);
-                unpack8(lds128(sm + STG_K, off), kk);
-                sq[u] = 0.f; sk[u] = 0.f;
+                for (int u = 0; u < 2; ++u) {
+                    const int r = row0 + u;
+                    float2 gg[4];
+                    unpack8x2(lds128(sm + STG_G, sw128_chunk(r, 8 * jch, 64)), gg);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float gv = r < L ? gg[e] : 0.f;
-                    if (p.has_lb) gv = fmaxf(gv, p.lb);
-                    tot[e] += gv;
-                    G[u][e] = tot[e];
-                    sq[u] = fmaf(qq[e], qq[e], sq[u]);
-                    sk[u] = fmaf(kk[e], kk[e], sk[u]);
+                    for (int e = 0; e < 4; ++e) {
+                        float2 gv = r < L ? gg[e] : make_float2(0.f, 0.f);
+                        if (p.has_lb) gv = make_float2(fmaxf(gv.x, p.lb), fmaxf(gv.y, p.lb));
+                        tt[e] = __fadd2_rn(tt[e], gv);
+                        G[u][2 * e] = tt[e].x;
+                        G[u][2 * e + 1] = tt[e].y;
+                    }
                 }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) { tot[2 * e] = tt[e].x; tot[2 * e + 1] = tt[e].y; }
             }
-            // scan of the 2-row totals over the 4 row pairs of this segment (lane bits 3, 4)
+            float G15[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 float inc = tot[e];
-                float y = __shfl_up_sync(0xffffffffu, inc, 8);
-                if (rq >= 1) inc += y;
-                y = __shfl_up_sync(0xffffffffu, inc, 16);
-                if (rq >= 2) inc += y;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, inc, d);
+                    if (lane >= d) inc += y;
+                }
                 G[0][e] += inc - tot[e];
                 G[1][e] += inc - tot[e];
-                if (rq == 3) ssegt[seg * 128 + 8 * jch + e] = inc;
-            }
-            // row norms over this warp's 64 channels (lane bits 0..2), then per half
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-#pragma unroll
-                for (int o = 1; o < 8; o <<= 1) {
-                    sq[u] += __shfl_xor_sync(0xffffffffu, sq[u], o);
-                    sk[u] += __shfl_xor_sync(0xffffffffu, sk[u], o);
-                }
-            }
-            if ((lane & 7) == 0) {
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    sred[(warp & 1) * 64 + row0 + u] = sq[u];
-                    sred[128 + (warp & 1) * 64 + row0 + u] = sk[u];
-                }
-            }
-        }
-        __syncthreads();
-        if (tid < 128) {
-            // one thread per channel: exclusive carries over the 8 segments, block references
-            float cum = 0.f;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const float tq = ssegt[q * 128 + tid];
-                ssegt[q * 128 + tid] = cum;
-                cum += tq;
-                if (q == 1) sref[tid] = cum;        // G_15
-                if (q == 5) sref[128 + tid] = cum;  // G_47
-            }
-            sref[256 + tid] = cum;                  // G_63
-            sGam[tid] = expf(cum);
-        } else if (tid < 256) {
-            const int r = tid & 63, which = (tid >> 6) & 1;
-            const float ssum = sred[which * 128 + r] + sred[which * 128 + 64 + r];
-            const float inv = r < L ? (p.use_l2 ? rsqrtf(ssum + kL2Eps) : 1.f) : 0.f;
-            (which ? sinvk : sinvq)[r] = inv;
-        }
-        __syncthreads();
-        {
-            auto ld8 = [&](const float *src, float (&dst)[8]) {
-                const float4 a = *reinterpret_cast<const float4 *>(src + 8 * jch);
-                const float4 b = *reinterpret_cast<const float4 *>(src + 8 * jch + 4);
-                dst[0] = a.x; dst[1] = a.y; dst[2] = a.z; dst[3] = a.w;
-                dst[4] = b.x; dst[5] = b.y; dst[6] = b.z; dst[7] = b.w;
-            };
-            float carry[8];
-            ld8(ssegt + seg * 128, carry);
-            ld8(sref + (blk ? 128 : 0), Gm);
-            ld8(sref + 128, G47);
-            ld8(sref + 256, G63);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                G[0][e] += carry[e];
-                G[1][e] += carry[e];
+                G15[e] = __shfl_sync(0xffffffffu, inc, 7);
+                G47[e] = __shfl_sync(0xffffffffu, inc, 23);
+                G63[e] = __shfl_sync(0xffffffffu, inc, 31);
+                Gm[e] = blk ? G47[e] : G15[e];
                 span_bad |= fabsf(G[0][e] - Gm[e]) > kSpanMax;
                 span_bad |= fabsf(G[1][e] - Gm[e]) > kSpanMax;
+            }
+            if (lane < 8) {  // lane e writes channel 8*jch + e
+                float a = G63[0], b = G15[0], c = G47[0];
+#pragma unroll
+                for (int e = 1; e < 8; ++e)
+                    if (lane == e) { a = G63[e]; b = G15[e]; c = G47[e]; }
+                sGam[8 * jch + lane] = expf(a);
+                sEw[8 * jch + lane] = expf(b);
+                sEw[128 + 8 * jch + lane] = expf(c);
             }
         }
         const bool fb = __syncthreads_or(span_bad) != 0;
@@ -336,53 +330,77 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         // ---------------- P2: bf16 operand tiles from the raw rows
         {
             const int hf = jch >> 3, jc = 8 * (jch & 7);
+            constexpr float kLog2e = 1.4426950408889634f;
+            float2 ngm[4], emid[4], fkh[4], foff[4];
+            if (!fb) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float m0 = Gm[2 * e], m1 = Gm[2 * e + 1];
+                    ngm[e] = make_float2(-m0, -m1);
+                    emid[e] = make_float2(__expf(m0), __expf(m1));
+                    fkh[e] = make_float2(__expf(G63[2 * e] - m0), __expf(G63[2 * e + 1] - m1));
+                    foff[e] = make_float2(__expf(G47[2 * e] - m0), __expf(G47[2 * e + 1] - m1));
+                }
+            }
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int r = row0 + u;
                 const uint32_t off = sw128_chunk(r, 8 * jch, 64);
-                float qq[8], kk[8];
-                unpack8(lds128(sm + STG_Q, off), qq);
-                unpack8(lds128(sm + STG_K, off), kk);
+                float2 qq[4], kk[4];
+                unpack8x2(lds128(sm + STG_Q, off), qq);
+                unpack8x2(lds128(sm + STG_K, off), kk);
                 if (r >= L) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) { qq[e] = 0.f; kk[e] = 0.f; }
+                    for (int e = 0; e < 4; ++e) { qq[e] = make_float2(0.f, 0.f); kk[e] = qq[e]; }
                 }
-                float t1[8], t2[8], t3[8];
-                if (!fb) {
-                    float xk[8], xq[8], y[8];
+                {   // this thread's 8 channels of |q_r|^2 and |k_r|^2
+                    float2 a = __fmul2_rn(qq[0], qq[0]), b = __fmul2_rn(kk[0], kk[0]);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float a = G[u][e] - Gm[e];
-                        const float ed = __expf(a), ydf = __expf(-a);
-                        const float emid = __expf(Gm[e]);
-                        xk[e] = kk[e] * ed;
-                        xq[e] = qq[e] * ed;
-                        y[e] = kk[e] * ydf;
-                        t1[e] = xq[e] * emid;
-                        t2[e] = xk[e] * emid;
-                        t3[e] = y[e] * __expf(G63[e] - Gm[e]);
+                    for (int e = 1; e < 4; ++e) { a = __ffma2_rn(qq[e], qq[e], a); b = __ffma2_rn(kk[e], kk[e], b); }
+                    float *nrm = reinterpret_cast<float *>(sm + NRM);
+                    nrm[jch * 64 + r] = a.x + a.y;
+                    nrm[1024 + jch * 64 + r] = b.x + b.y;
+                }
+                float2 t1[4], t3[4];
+                if (!fb) {
+                    float2 xk[4], xq[4], y[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        // a = G - G_m; ed = e^a (SFU), yd = e^-a = 1/ed (FMA pipe)
+                        const float2 a = __fmul2_rn(__fadd2_rn(make_float2(G[u][2 * e], G[u][2 * e + 1]), ngm[e]),
+                                                    make_float2(kLog2e, kLog2e));
+                        const float2 ed = make_float2(ex2a(a.x), ex2a(a.y));
+                        const float2 yd = rcp2_nr(ed);
+                        xk[e] = __fmul2_rn(kk[e], ed);
+                        xq[e] = __fmul2_rn(qq[e], ed);
+                        y[e] = __fmul2_rn(kk[e], yd);
+                        t1[e] = __fmul2_rn(xq[e], emid[e]);
+                        t3[e] = __fmul2_rn(y[e], fkh[e]);
                     }
-                    sts128(sm, XKQD + sw128_chunk(r, 8 * jch, 128), pack8(xk));
-                    sts128(sm, XKQD + sw128_chunk(64 + r, 8 * jch, 128), pack8(xq));
-                    sts128(sm, (hf ? YD_H1 : YD_H0) + sw128_chunk(r, jc, 64), pack8(y));
+                    sts128(sm, XKQD + sw128_chunk(r, 8 * jch, 128), pack8x2(xk));
+                    sts128(sm, XKQD + sw128_chunk(64 + r, 8 * jch, 128), pack8x2(xq));
+                    sts128(sm, (hf ? YD_H1 : YD_H0) + sw128_chunk(r, jc, 64), pack8x2(y));
                     if (blk == 0) {
                         // off-diagonal column operand k_s e^{G_47 - G_s}, paired with the block-1 rows
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) y[e] *= __expf(G47[e] - Gm[e]);
-                        sts128(sm, (hf ? YO_H1 : YO_H0) + sw128_chunk(r, jc, 32), pack8(y));
+                        for (int e = 0; e < 4; ++e) y[e] = __fmul2_rn(y[e], foff[e]);
+                        sts128(sm, (hf ? YO_H1 : YO_H0) + sw128_chunk(r, jc, 32), pack8x2(y));
                     }
                 } else {
+                    // exact path: no block reference, the k rows of XKQD hold k e^G (<= 1)
+                    float2 t2[4];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float eg = expf(G[u][e]);
-                        t1[e] = qq[e] * eg;
-                        t2[e] = kk[e] * eg;
-                        t3[e] = kk[e] * expf(G63[e] - G[u][e]);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 eg = make_float2(expf(G[u][2 * e]), expf(G[u][2 * e + 1]));
+                        const float2 ek = make_float2(expf(G63[2 * e] - G[u][2 * e]), expf(G63[2 * e + 1] - G[u][2 * e + 1]));
+                        t1[e] = __fmul2_rn(qq[e], eg);
+                        t2[e] = __fmul2_rn(kk[e], eg);
+                        t3[e] = __fmul2_rn(kk[e], ek);
                     }
+                    sts128(sm, XKQD + sw128_chunk(r, 8 * jch, 128), pack8x2(t2));
                 }
-                sts128(sm, QT + off, pack8(t1));
-                sts128(sm, KT + off, pack8(t2));
-                sts128(sm, KH + off, pack8(t3));
+                sts128(sm, QT + off, pack8x2(t1));
+                sts128(sm, KH + off, pack8x2(t3));
             }
         }
         fence_proxy_async_smem();
@@ -400,13 +418,23 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
             for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t ko = (kk >> 2) * 16384 + (kk & 3) * 32;
                 const uint32_t yb = (kk >> 2) ? YD_H1 : YD_H0, ob = (kk >> 2) ? YO_H1 : YO_H0;
-                mma_bf16(tb + TM_A, sdesc_sw128(sb + XKQD + ko, 16, 1024),
-                         sdesc_sw128(sb + yb + (kk & 3) * 32, 16, 1024), ID_A1, kk > 0);
-                mma_bf16(tb + TM_A + 64, sdesc_sw128(sb + XKQD + ko + 32 * 128, 16, 1024),
-                         sdesc_sw128(sb + ob + (kk & 3) * 32, 16, 1024), ID_A2, kk > 0);
+                mma_bf16(tb + TM_A, dk(XKQD + ko),
+                         dk(yb + (kk & 3) * 32), ID_A1, kk > 0);
+                mma_bf16(tb + TM_A + 64, dk(XKQD + ko + 32 * 128),
+                         dk(ob + (kk & 3) * 32), ID_A2, kk > 0);
             }
             mma_commit(bar_mma);
             mma_out = true;
+        }
+
+        if (tid < 128) {  // row norms from the 16 per-warp partials
+            const int r = tid & 63, which = tid >> 6;
+            const float *nrm = reinterpret_cast<const float *>(sm + NRM) + which * 1024 + r;
+            float ssum = 0.f;
+#pragma unroll
+            for (int w = 0; w < 16; ++w) ssum += nrm[w * 64];
+            const float inv = r < L ? (p.use_l2 ? rsqrtf(ssum + kL2Eps) : 1.f) : 0.f;
+            (which ? sinvk : sinvq)[r] = inv;
         }
 
         // ---------------- state refresh (overlaps the products above):
@@ -425,7 +453,11 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) sts128(sm, ST + sw128_chunk(v, c0 + 8 * q4, 128), pack8(x + 8 * q4));
 #pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] *= sGam[c0 + j];
+            for (int j = 0; j < 32; j += 2) {
+                const float2 v2 = __fmul2_rn(make_float2(x[j], x[j + 1]),
+                                             *reinterpret_cast<const float2 *>(sGam + c0 + j));
+                x[j] = v2.x; x[j + 1] = v2.y;
+            }
             tmem_st32(tb + TM_S + lane_sel + c0, x);
             tmem_st_wait();
         }
@@ -489,6 +521,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                 }
             }
         } else {
+            __syncthreads();  // the row norms above are read below
             // exact A_kk / A_qk on CUDA cores (raw rows): warp per row r, lanes over channels,
             // walking s downwards while accumulating the gate between s and r
             for (int r = warp; r < C; r += NT / 32) {
@@ -529,40 +562,67 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         }
         __syncthreads();
 
-        // ---------------- T = (I + L)^-1 on 16x16 blocks
-        // diagonal blocks by a column sweep (lane j = column j): once t[k] is final it
-        // updates every later row, so the dependent chain is 16 steps long
-        if (warp < 4 && lane < 16) {
-            const int b = warp, j = lane;
-            float t[16];
+        // ---------------- T = (I + L)^-1 on 16x16 blocks, written straight into the bf16
+        // tiles T_u = T diag(beta) and T_w = T diag(beta / |k|) (rows r, columns s <= r)
+        if (warp < 4) {
+            // diagonal blocks by a column sweep (lane j = column j): once t[k] is final it
+            // updates every later row, so the dependent chain is 16 steps long
+            if (lane < 16) {
+                const int b = warp, j = lane;
+                float t[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) t[i] = i == j ? 1.f : 0.f;
+                for (int i = 0; i < 16; ++i) t[i] = i == j ? 1.f : 0.f;
 #pragma unroll
-            for (int k = 0; k < 15; ++k) {
+                for (int k = 0; k < 15; ++k) {
 #pragma unroll
-                for (int i = k + 1; i < 16; ++i) t[i] = fmaf(-Lf[(16 * b + i) * LDS + 16 * b + k], t[k], t[i]);
+                    for (int i = k + 1; i < 16; ++i) t[i] = fmaf(-Lf[(16 * b + i) * LDS + 16 * b + k], t[k], t[i]);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) Tf[(16 * b + i) * LDT + 16 * b + j] = t[i];
             }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) Tf[(16 * b + i) * LDT + 16 * b + j] = t[i];
-        } else if (warp >= 4) {
-            // zero the blocks above the diagonal, which the block products read
-            for (int e = tid - 128; e < 6 * 256; e += NT - 128) {
-                const int bid = e >> 8, i = (e >> 4) & 15, j = e & 15;
+        } else {
+            // blocks above the block diagonal: zero in T (read by the block products) and in
+            // both bf16 tiles
+            // 6 blocks x 16 rows x 2 chunks of 8 columns = 192 items for 384 threads
+            const int e = tid - 128;
+            if (e < 192) {
+                const int bid = e >> 5, i = (e >> 1) & 15, half = e & 1;
                 const int bi = bid < 3 ? 0 : bid < 5 ? 1 : 2;
                 const int bj = bid < 3 ? bid + 1 : bid < 5 ? bid - 1 : 3;
-                Tf[(16 * bi + i) * LDT + 16 * bj + j] = 0.f;
+                const int r = 16 * bi + i, c = 16 * bj + 8 * half;
+                *reinterpret_cast<float4 *>(Tf + r * LDT + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4 *>(Tf + r * LDT + c + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+                sts128(sm, TPU + sw128_chunk(r, c, 64), make_uint4(0u, 0u, 0u, 0u));
+                sts128(sm, TPW + sw128_chunk(r, c, 64), make_uint4(0u, 0u, 0u, 0u));
             }
         }
         __syncthreads();
-        // block rows I = 1..3:  T[I, J<I] = -T_II sum_{K<I} L_IK T_KJ, on warp-level tf32
-        // MMAs; warp w < 2I owns the 8 output columns 8w .. 8w+7
+        // block rows I = 1..3:  T[I, J<I] = -T_II sum_{K<I} L_IK T_KJ on warp-level tf32 MMAs;
+        // warp w < 2I owns output columns 8w .. 8w+7; the step-1 accumulator is transposed
+        // into the step-2 operand with shuffles inside the warp
+        if (warp >= 8) {
+            // diagonal blocks of T -> both bf16 tiles (s <= r), 4 blocks x 16 rows x 2 chunks
+            const int e = tid - 256;
+            if (e < 128) {
+                const int b = e >> 5, i = (e >> 1) & 15, half = e & 1;
+                const int r = 16 * b + i, c = 16 * b + 8 * half;
+                float mu[8], mw[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int s_ = c + q;
+                    mu[q] = s_ <= r ? Tf[r * LDT + s_] * sbeta[s_] : 0.f;
+                    mw[q] = mu[q] * sinvk[s_];
+                }
+                sts128(sm, TPU + sw128_chunk(r, c, 64), pack8(mu));
+                sts128(sm, TPW + sw128_chunk(r, c, 64), pack8(mw));
+            }
+        }
         {
             const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
             for (int I = 1; I < 4; ++I) {
-                const bool act = warp < 2 * I;
-                const int n0 = 8 * warp;
-                if (act) {
+                if (warp < 2 * I) {
+                    const int n0 = 8 * warp;
                     float d[4] = {0.f, 0.f, 0.f, 0.f};
                     const float *La = Lf + (16 * I + g) * LDS, *Lb = Lf + (16 * I + g + 8) * LDS;
 #pragma unroll
@@ -574,44 +634,46 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                                                to_tf32(Tf[(k0 + t4 + 4) * LDT + n0 + g])};
                         mma_tf32_16x8x8(d, a, b);
                     }
-                    Rf[g * LDR + n0 + 2 * t4] = d[0];
-                    Rf[g * LDR + n0 + 2 * t4 + 1] = d[1];
-                    Rf[(g + 8) * LDR + n0 + 2 * t4] = d[2];
-                    Rf[(g + 8) * LDR + n0 + 2 * t4 + 1] = d[3];
-                }
-                __syncthreads();
-                if (act) {
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-                    const float *Ta = Tf + (16 * I + g) * LDT + 16 * I, *Tb = Tf + (16 * I + g + 8) * LDT + 16 * I;
+                    // R[row][col] sits in lane 4*(row % 8) + col/2, component (row >= 8) * 2 + col % 2
+                    const int srcA = 4 * t4 + (g >> 1), srcB = 4 * (t4 + 4) + (g >> 1);
+                    const bool odd = g & 1;
+                    float v[8];
 #pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {
-                        const int k0 = 8 * ks;
-                        const uint32_t a[4] = {to_tf32(Ta[k0 + t4]), to_tf32(Tb[k0 + t4]), to_tf32(Ta[k0 + t4 + 4]),
-                                               to_tf32(Tb[k0 + t4 + 4])};
-                        const uint32_t b[2] = {to_tf32(Rf[(k0 + t4) * LDR + n0 + g]),
-                                               to_tf32(Rf[(k0 + t4 + 4) * LDR + n0 + g])};
-                        mma_tf32_16x8x8(d, a, b);
+                    for (int c = 0; c < 4; ++c) {
+                        v[c] = __shfl_sync(0xffffffffu, d[c], srcA);
+                        v[4 + c] = __shfl_sync(0xffffffffu, d[c], srcB);
                     }
-                    Tf[(16 * I + g) * LDT + n0 + 2 * t4] = -d[0];
-                    Tf[(16 * I + g) * LDT + n0 + 2 * t4 + 1] = -d[1];
-                    Tf[(16 * I + g + 8) * LDT + n0 + 2 * t4] = -d[2];
-                    Tf[(16 * I + g + 8) * LDT + n0 + 2 * t4 + 1] = -d[3];
+                    const uint32_t b0[2] = {to_tf32(odd ? v[1] : v[0]), to_tf32(odd ? v[5] : v[4])};  // rows t, t+4
+                    const uint32_t b1[2] = {to_tf32(odd ? v[3] : v[2]), to_tf32(odd ? v[7] : v[6])};  // rows 8+t, 12+t
+                    float e[4] = {0.f, 0.f, 0.f, 0.f};
+                    const float *Ta = Tf + (16 * I + g) * LDT + 16 * I, *Tb = Tf + (16 * I + g + 8) * LDT + 16 * I;
+                    {
+                        const uint32_t a[4] = {to_tf32(Ta[t4]), to_tf32(Tb[t4]), to_tf32(Ta[t4 + 4]), to_tf32(Tb[t4 + 4])};
+                        mma_tf32_16x8x8(e, a, b0);
+                    }
+                    {
+                        const uint32_t a[4] = {to_tf32(Ta[8 + t4]), to_tf32(Tb[8 + t4]), to_tf32(Ta[12 + t4]),
+                                               to_tf32(Tb[12 + t4])};
+                        mma_tf32_16x8x8(e, a, b1);
+                    }
+                    const int r0 = 16 * I + g, c0 = n0 + 2 * t4;
+                    Tf[r0 * LDT + c0] = -e[0];
+                    Tf[r0 * LDT + c0 + 1] = -e[1];
+                    Tf[(r0 + 8) * LDT + c0] = -e[2];
+                    Tf[(r0 + 8) * LDT + c0 + 1] = -e[3];
+                    const float b0s = sbeta[c0], b1s = sbeta[c0 + 1];
+                    const float w0s = b0s * sinvk[c0], w1s = b1s * sinvk[c0 + 1];
+                    *reinterpret_cast<uint32_t *>(sm + TPU + sw128(r0, c0, 64)) =
+                        pack_bf16x2(-e[0] * b0s, -e[1] * b1s);
+                    *reinterpret_cast<uint32_t *>(sm + TPU + sw128(r0 + 8, c0, 64)) =
+                        pack_bf16x2(-e[2] * b0s, -e[3] * b1s);
+                    *reinterpret_cast<uint32_t *>(sm + TPW + sw128(r0, c0, 64)) =
+                        pack_bf16x2(-e[0] * w0s, -e[1] * w1s);
+                    *reinterpret_cast<uint32_t *>(sm + TPW + sw128(r0 + 8, c0, 64)) =
+                        pack_bf16x2(-e[2] * w0s, -e[3] * w1s);
                 }
-                __syncthreads();
+                if (I < 3) __syncthreads();
             }
-        }
-        // T' tiles: T diag(beta) for U and T diag(beta / |k|) for W (one chunk of each per thread)
-        {
-            const int r = tid >> 3, s0 = (tid & 7) * 8;
-            float mu[8], mw[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int s = s0 + e;
-                mu[e] = s <= r ? Tf[r * LDT + s] * sbeta[s] : 0.f;
-                mw[e] = mu[e] * sinvk[s];
-            }
-            sts128(sm, TPU + sw128_chunk(r, s0, 64), pack8(mu));
-            sts128(sm, TPW + sw128_chunk(r, s0, 64), pack8(mw));
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -622,10 +684,11 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         if (tid == kMma) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                mma_bf16(tb + TM_U, sdesc_sw128(sb + STG_V + kk * 2048, 8192, 1024),
-                         sdesc_sw128(sb + TPU + kk * 32, 16, 1024), ID_UW, kk > 0);
-                mma_bf16(tb + TM_W, sdesc_sw128(sb + KT + kk * 2048, 8192, 1024),
-                         sdesc_sw128(sb + TPW + kk * 32, 16, 1024), ID_UW, kk > 0);
+                mma_bf16(tb + TM_U, dm(STG_V + kk * 2048), dk(TPU + kk * 32), ID_UW, kk > 0);
+                // W in two K halves (token blocks 0..31 and 32..63), each with its own
+                // block reference; recombined per key channel when W is read back
+                mma_bf16(tb + (kk < 2 ? TM_W : TM_W1), dx(XKQD + kk * 2048), dk(TPW + kk * 32), ID_UW,
+                         (kk & 1) != 0);
             }
             mma_commit(bar_mma);
             mma_out = true;
@@ -633,11 +696,16 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
         if (tid == kMma) mma_out = false;
         tc_fence_after();
-        {   // W^T (lane c, columns r) -> bf16 tile [c][r]
-            float x[16];
+        {   // W^T (lane c, columns r) = e^{G_15[c]} W0 + e^{G_47[c]} W1 -> bf16 tile [c][r]
+            float x[16], x1[16];
+            const int c = 32 * quarter + lane;
             tmem_ld16(tb + TM_W + lane_sel + 16 * cgrp, x);
+            tmem_ld16(tb + TM_W1 + lane_sel + 16 * cgrp, x1);
             tmem_ld_wait();
-            row16_to_tile(sm, WT, 32 * quarter + lane, 16 * cgrp, 128, x);
+            const float e0 = fb ? 1.f : sEw[c], e1 = fb ? 1.f : sEw[128 + c];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) x[j] = fmaf(e0, x[j], e1 * x1[j]);
+            row16_to_tile(sm, WT, c, 16 * cgrp, 128, x);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -649,9 +717,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         if (tid == kMma) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t adesc = sdesc_sw128(sb + ST + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                mma_bf16(tb + TM_U, adesc, sdesc_sw128(sb + WT + kk * 2048, 8192, 1024), ID_DL, 1);
-                mma_bf16(tb + TM_O, adesc, sdesc_sw128(sb + QT + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                const uint64_t adesc = dk(ST + (kk >> 2) * 16384 + (kk & 3) * 32);
+                mma_bf16(tb + TM_U, adesc, dm(WT + kk * 2048), ID_DL, 1);
+                mma_bf16(tb + TM_O, adesc, dk(QT + (kk >> 2) * 8192 + (kk & 3) * 32),
                          ID_O, kk > 0);
             }
             mma_commit(bar_mma);
@@ -678,9 +746,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         if (tid == kMma) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t adesc = sdesc_sw128(sb + DT + kk * 32, 16, 1024);
-                mma_bf16(tb + TM_O, adesc, sdesc_sw128(sb + AQK + kk * 32, 16, 1024), ID_O, 1);
-                mma_bf16(tb + TM_S, adesc, sdesc_sw128(sb + KH + kk * 2048, 8192, 1024), ID_S, 1);
+                const uint64_t adesc = dk(DT + kk * 32);
+                mma_bf16(tb + TM_O, adesc, dk(AQK + kk * 32), ID_O, 1);
+                mma_bf16(tb + TM_S, adesc, dm(KH + kk * 2048), ID_S, 1);
             }
             mma_commit(bar_mma);
             mma_out = true;
