@@ -123,6 +123,29 @@ typedef struct {
 
 KDA_API kda_status kda_recurrent_step(const kda_step_args *args, void *stream);
 
+/*
+ * Chunkwise forward for callers that cannot allocate device memory. This entry
+ * point has no counterpart in the pages; it exists for callers that run under a
+ * fixed device-memory plan and may not allocate once running (an inference
+ * engine that reserves its memory at start-up, a plug-in whose host application
+ * owns every device buffer, a C host with no allocator at the call site), for
+ * whom kda_chunk_fwd's workspace is out of reach.
+ *
+ * Same arguments and result as kda_chunk_fwd; `workspace` and `workspace_bytes`
+ * are ignored. The scratch it needs comes from a fixed 4096-byte array in the
+ * library's own device memory (one per device, held from library load until
+ * process exit); requests needing more than that return KDA_ERR_WORKSPACE (none
+ * do today: the chunk kernels need at most 256 bytes). Nothing is allocated or
+ * freed.
+ *  - The first call on a device looks up that array's device address (a
+ *    cudaGetSymbolAddress with the device current); make that first call before
+ *    any stream capture.
+ *  - Every call on a device shares the one array, which keeps the last call's
+ *    contents; the library clears what must start at zero. Calls whose work
+ *    overlaps on the GPU (different streams, no ordering) race on it: order them.
+ */
+KDA_API kda_status kda_chunk_fwd_noalloc(const kda_chunk_args *args, void *stream);
+
 /* Static, human-readable name of a status. */
 KDA_API const char *kda_status_string(kda_status status);
 

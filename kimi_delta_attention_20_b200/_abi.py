@@ -57,8 +57,8 @@ class StepArgs(ctypes.Structure):
 
 
 # every symbol include/kda.h declares
-EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_recurrent_step",
-           "kda_status_string", "kda_last_cuda_error", "kda_version")
+EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_noalloc",
+           "kda_recurrent_step", "kda_status_string", "kda_last_cuda_error", "kda_version")
 
 _lib = None
 
@@ -77,6 +77,8 @@ def load():
     lib.kda_chunk_fwd_workspace_size.restype = ctypes.c_int
     lib.kda_chunk_fwd.argtypes = [ctypes.POINTER(ChunkArgs), _vp]
     lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(ChunkArgs), _vp]
+    lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
     lib.kda_recurrent_step.argtypes = [ctypes.POINTER(StepArgs), _vp]
     lib.kda_recurrent_step.restype = ctypes.c_int
     lib.kda_status_string.argtypes = [ctypes.c_int]

@@ -58,6 +58,10 @@ kda_status check_chunk_shape(const kda_chunk_args *a, int *N_out) {
 
 }  // namespace
 
+namespace kda {
+void record_cuda_error(int e) { g_last_cuda_error = e; }
+}  // namespace kda
+
 extern "C" {
 
 const char *kda_status_string(kda_status s) {

@@ -1,0 +1,72 @@
+// kda_chunk_fwd_noalloc: the chunkwise forward for callers that cannot allocate
+// device memory.
+//
+// Some callers run under a fixed device-memory plan and may not allocate once
+// they are running: an inference engine that reserves all of its memory at start-
+// up, a plug-in whose host application owns every device buffer, or a C host
+// that has no allocator handle at the call site. kda_chunk_fwd asks such callers
+// for a workspace they have no way to obtain. This entry point instead uses a
+// small scratch array that lives in the library's own device memory (a
+// file-scope __device__ array, created when the library is loaded on a device
+// and held until the process exits). Inputs and outputs are still the caller's.
+//
+// The array's name, seen from host code, is only a host-side stand-in and not a
+// device address; its device address is looked up once per device with
+// cudaGetSymbolAddress (with that device current) and that address is what the
+// kernels receive.
+#include <mutex>
+
+#include "../../include/kda.h"
+#include "kda_common.cuh"
+
+// Scratch of the no-allocation entry point: the tensor-core chunk kernel keeps
+// its device status word here (it needs 256 bytes whatever the problem size).
+static constexpr size_t kScratchBytes = 4096;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void *g_scratch_addr[kMaxDevices] = {};
+
+}  // namespace
+
+namespace kda {
+void record_cuda_error(int e);  // kda_api.cu: value returned by kda_last_cuda_error()
+}  // namespace kda
+
+extern "C" {
+
+KDA_API kda_status kda_chunk_fwd_noalloc(const kda_chunk_args *args, void *stream) {
+    if (!args) return KDA_ERR_INVALID_ARGUMENT;
+    size_t need = 0;
+    kda_status s = kda_chunk_fwd_workspace_size(args, &need);
+    if (s != KDA_OK) return s;
+    if (need > kScratchBytes) return KDA_ERR_WORKSPACE;  // beyond the fixed scratch size
+
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) { kda::record_cuda_error((int)e); return KDA_ERR_CUDA; }
+    if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!g_scratch_addr[dev]) {
+            void *p = nullptr;
+            e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+            if (e != cudaSuccess || !p) {
+                kda::record_cuda_error((int)e);
+                return KDA_ERR_CUDA;
+            }
+            g_scratch_addr[dev] = p;
+        }
+        scratch = g_scratch_addr[dev];
+    }
+    kda_chunk_args a = *args;
+    a.workspace = need ? scratch : nullptr;
+    a.workspace_bytes = need ? kScratchBytes : 0;
+    return kda_chunk_fwd(&a, stream);
+}
+
+}  // extern "C"
