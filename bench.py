@@ -146,6 +146,32 @@ def ncu_traffic(key, sha):
         return None
 
 
+# --------------------------------------------------------------------------- ranks
+
+def rank_barrier(world):
+    """Barrier across ranks (no-op for a single process)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks_value(x, world, device):
+    """Slowest rank's value: an all-reduce MAX of one float (NCCL on GPUs, gloo on CPU)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, units_per_rank, ms_max):
+    """Weak scaling: every rank processes `units_per_rank`; the job takes the slowest
+    rank's time, so the whole-job rate is world * units / that time."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
 # --------------------------------------------------------------------------- GPU arm
 
 def run_kda(args, rank, world, local_rank):
@@ -186,15 +212,10 @@ def run_kda(args, rank, world, local_rank):
                            dinp["beta"][t], state, out=od)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        rank_barrier(world)
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks_value(x, world, dev)
 
     stream = torch.cuda.current_stream(dev)
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[local_rank]) \
@@ -291,7 +312,7 @@ def run_kda(args, rank, world, local_rank):
     chunk_sha = source_sha("kda_chunk_tc.cu", "kda_chunk_simt.cu", "kda_common.cuh") if tc_used else None
     result = {
         "metric": METRIC,
-        "value": world * wl.tokens / (chunk_ms * 1e-3),
+        "value": whole_job_rate(world, wl.tokens, chunk_ms),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -319,8 +340,8 @@ def run_kda(args, rank, world, local_rank):
                        "frac": chunk_tflops / tc_peak},
         },
         "decode": {
-            "value": world / (dec_ms * 1e-3), "unit": "steps/s",
-            "tokens_per_s": world * dwl.N / (dec_ms * 1e-3), "ms_per_step": dec_ms,
+            "value": whole_job_rate(world, 1, dec_ms), "unit": "steps/s",
+            "tokens_per_s": whole_job_rate(world, dwl.N, dec_ms), "ms_per_step": dec_ms,
             "steps_timed": nsteps,
             "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": dec_gbs / hbm_peak, "peak_kind": peak_kind,
@@ -328,7 +349,7 @@ def run_kda(args, rank, world, local_rank):
                          "traffic": ncu_traffic("decode", source_sha("kda_decode.cu",
                                                                      "kda_common.cuh"))},
         },
-        "e2e": {"value": world * wl.tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_rate(world, wl.tokens, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": args.steps * (1 + DECODE_STEPS_PER_PASS),
         "clocks": clk,
