@@ -11,7 +11,9 @@
  *     o_t   <- scale S^T q_t
  * with q_t, k_t optionally L2-normalised first as x / sqrt(sum x^2 + 1e-6)
  * (same page, `l2norm_rows`, `KDA_L2_EPS`) and g_t optionally clamped from
- * below, g_t <- max(g_t, lower_bound).
+ * below, g_t <- max(g_t, lower_bound). Optionally the kernel forms g_t itself
+ * from the gate input (kda_gate_mode) and takes beta_t as a probability
+ * instead of a logit (`beta_is_prob`).
  *
  * Conventions shared by every entry point:
  *  - Every buffer is caller-owned DEVICE memory, except the fields whose
@@ -59,18 +61,39 @@ typedef enum {
 } kda_dtype;
 
 /*
+ * How the kernel obtains the log-decay g from the `g` input: page
+ * "atlas_core/kimi_k3/kda.rs", `bounded_gate`, and page "K3/kda/ops/api.py",
+ * `use_gate_in_kernel` / `safe_gate`. With x = g_in + dt_bias[h, c] and
+ * rate = exp(A_log[h]), all in fp32:
+ *   KDA_GATE_LOG       g = g_in, then max(g, lower_bound) if has_lower_bound
+ *   KDA_GATE_SOFTPLUS  g = -rate * softplus(x)        (has_lower_bound must be 0:
+ *                                                      the unbounded form has none)
+ *   KDA_GATE_SAFE      g = lower_bound * sigmoid(rate * x)  (has_lower_bound must
+ *                                                      be 1, lower_bound < 0)
+ * A_log: [H] fp32 device, required by the two in-kernel forms. dt_bias:
+ * [H, Dk] fp32 device, NULL = zeros. Both are ignored by KDA_GATE_LOG.
+ */
+typedef enum {
+    KDA_GATE_LOG = 0,
+    KDA_GATE_SOFTPLUS = 1,
+    KDA_GATE_SAFE = 2
+} kda_gate_mode;
+
+/*
  * Chunkwise forward: the `chunk_kda` boundary of page "K3/kda/ops/api.py"
- * (signature and preprocessing: q/k L2 norm, sigmoid of beta, lower bound,
- * initial_state, output_final_state, chunk_size), minus its backend dispatch
- * and in-kernel gate. The result equals the token recurrence above run
+ * (signature and preprocessing: q/k L2 norm, sigmoid of beta, in-kernel
+ * gate, lower bound, initial_state, output_final_state, chunk_size), minus
+ * its backend dispatch. The result equals the token recurrence above run
  * over each sequence; internally tokens are processed chunk_size at a time.
+ * The fields after `workspace_bytes` default to the plain operator when
+ * zero-initialised.
  */
 typedef struct {
     kda_dtype dtype;      /* dtype of q, k, v, g, beta and o */
     int B, T, H, Dk, Dv;  /* q,k,g: [B,T,H,Dk]; v,o: [B,T,H,Dv]; beta: [B,T,H] */
     const void *q, *k, *v;
-    const void *g;        /* per-channel log-decay, expected <= 0 */
-    const void *beta;     /* LOGITS; sigmoid is applied in the kernel */
+    const void *g;        /* per-channel log-decay (<= 0), or the gate input (gate_mode) */
+    const void *beta;     /* logits, sigmoid applied in the kernel (or see beta_is_prob) */
     void *o;              /* output [B,T,H,Dv] */
     float scale;          /* <= 0 or NaN selects 1/sqrt(Dk) */
     const float *initial_state; /* [N,H,Dk,Dv] fp32, NULL = zeros */
@@ -91,6 +114,10 @@ typedef struct {
     int chunk_size;       /* 0 (default) or 64 */
     void *workspace;      /* device scratch of kda_chunk_fwd_workspace_size() bytes */
     size_t workspace_bytes;
+    kda_gate_mode gate_mode;   /* KDA_GATE_LOG (0): g is the log-decay */
+    const float *A_log;        /* [H] fp32, in-kernel gate forms only */
+    const float *dt_bias;      /* [H,Dk] fp32 or NULL, in-kernel gate forms only */
+    int beta_is_prob;          /* 1: beta is used as given (no sigmoid) */
 } kda_chunk_args;
 
 /* Bytes of device workspace kda_chunk_fwd needs for these arguments (may be
@@ -111,14 +138,18 @@ typedef struct {
     int N, H, Dk, Dv;
     const void *q, *k;    /* [N,H,Dk] */
     const void *v;        /* [N,H,Dv] */
-    const void *g;        /* [N,H,Dk] log-decay */
-    const void *beta;     /* [N,H] logits */
+    const void *g;        /* [N,H,Dk] log-decay, or the gate input (gate_mode) */
+    const void *beta;     /* [N,H] logits (or see beta_is_prob) */
     float *state;         /* [N,H,Dk,Dv] fp32, updated in place */
     void *o;              /* [N,H,Dv] out */
     float scale;          /* <= 0 or NaN selects 1/sqrt(Dk) */
     int use_qk_l2norm;
     int has_lower_bound;
     float lower_bound;
+    kda_gate_mode gate_mode;   /* as in kda_chunk_args */
+    const float *A_log;        /* [H] fp32 */
+    const float *dt_bias;      /* [H,Dk] fp32 or NULL */
+    int beta_is_prob;
 } kda_step_args;
 
 KDA_API kda_status kda_recurrent_step(const kda_step_args *args, void *stream);

@@ -13,7 +13,12 @@ three geometries plus a tiny fp32 case, and a batched decode step):
   here only to draw realistic log-decays); clamped workloads pass
   lower_bound = -5 to the operator, which applies the clamp.
 * decode: g = -5 * sigmoid(N(0, 1)).
-* beta logits ~ N(0, 1).
+* in-kernel gate cases: the raw gate input z ~ N(0, 1) is passed as g, with
+  A_log = log(U(1, 16)) per head and dt_bias = the inverse softplus of
+  dt = exp(U(log 1e-3, log 1e-1)) per channel (the initialisation page
+  "Kimi Delta Attention on AMD MI300X" names as FLA's, `draw_gate_params`).
+* beta logits ~ N(0, 1); beta probabilities (cases that pass beta as given)
+  ~ U(0, 1).
 * initial states ~ N(0, 1) * 0.1, fp32.
 
 Everything is drawn in fp32 with one ``torch.Generator`` seeded with the
@@ -97,12 +102,14 @@ def _gen(device, seed):
 
 
 def draw_chunk(B, T, H, Dk, Dv, *, dtype=torch.bfloat16, seed=0, device="cpu",
-               seqlens=None, init_state=False, gate="unbounded"):
+               seqlens=None, init_state=False, gate="unbounded", beta="logit"):
     """Draw one chunk-forward input set.
 
-    Returns a dict with q, k, g [B,T,H,Dk], v [B,T,H,Dv], beta [B,T,H] (logits),
+    Returns a dict with q, k, g [B,T,H,Dk], v [B,T,H,Dv], beta [B,T,H],
     initial_state [N,H,Dk,Dv] fp32 or None, cu_seqlens int32 [N+1] or None.
-    ``gate`` is "unbounded" (-exp(a_h) softplus(z)) or "decode" (-5 sigmoid(z)).
+    ``gate`` is "unbounded" (-exp(a_h) softplus(z)), "decode" (-5 sigmoid(z))
+    or "input" (z itself, for the in-kernel gate). ``beta`` is "logit"
+    (N(0, 1)) or "prob" (U(0, 1)).
     """
     gen = _gen(device, seed)
     f32 = dict(dtype=torch.float32, device=device, generator=gen)
@@ -111,11 +118,17 @@ def draw_chunk(B, T, H, Dk, Dv, *, dtype=torch.bfloat16, seed=0, device="cpu",
     v = torch.randn(B, T, H, Dv, **f32)
     z = torch.randn(B, T, H, Dk, **f32)
     a_h = torch.rand(H, **f32) * 2.5 - 2.0
-    beta = torch.randn(B, T, H, **f32)
+    beta_t = torch.randn(B, T, H, **f32)
+    if beta == "prob":
+        beta_t = torch.rand(B, T, H, **f32)
+    elif beta != "logit":
+        raise ValueError(beta)
     if gate == "unbounded":
         g = -torch.exp(a_h).view(1, 1, H, 1) * F.softplus(z)
     elif gate == "decode":
         g = -5.0 * torch.sigmoid(z)
+    elif gate == "input":
+        g = z
     else:
         raise ValueError(gate)
     del z
@@ -130,8 +143,21 @@ def draw_chunk(B, T, H, Dk, Dv, *, dtype=torch.bfloat16, seed=0, device="cpu",
         cu = cu.to(device)
     S0 = torch.randn(N, H, Dk, Dv, **f32) * 0.1 if init_state else None
     out = dict(q=q.to(dtype), k=k.to(dtype), v=v.to(dtype), g=g.to(dtype),
-               beta=beta.to(dtype), initial_state=S0, cu_seqlens=cu)
+               beta=beta_t.to(dtype), initial_state=S0, cu_seqlens=cu)
     return out
+
+
+def draw_gate_params(H, Dk, *, seed=0, device="cpu"):
+    """Parameters of the in-kernel gate, fp32: A_log [H] = log(U(1, 16)) and
+    dt_bias [H, Dk] = inverse softplus of dt = exp(U(log 1e-3, log 1e-1))
+    (dt floored at 1e-4), the initialisation named for FLA's KDA layer."""
+    gen = _gen(device, 1000 + int(seed))
+    f32 = dict(dtype=torch.float32, device=device, generator=gen)
+    A_log = torch.log(torch.rand(H, **f32) * 15.0 + 1.0)
+    lo, hi = math.log(1e-3), math.log(1e-1)
+    dt = torch.exp(torch.rand(H, Dk, **f32) * (hi - lo) + lo).clamp_min(1e-4)
+    dt_bias = dt + torch.log(-torch.expm1(-dt))
+    return dict(A_log=A_log, dt_bias=dt_bias)
 
 
 def chunk_inputs(idx_or_wl, device="cpu"):
@@ -141,19 +167,31 @@ def chunk_inputs(idx_or_wl, device="cpu"):
                       device=device, seqlens=wl.seqlens, init_state=wl.init_state)
 
 
-def draw_decode(N, H, Dk, Dv, steps, *, dtype=torch.bfloat16, seed=3, device="cpu"):
+def draw_decode(N, H, Dk, Dv, steps, *, dtype=torch.bfloat16, seed=3, device="cpu",
+                gate="decode", beta="logit"):
     """Decode inputs: initial state [N,H,Dk,Dv] fp32 ~ 0.1 N(0,1), then per step
-    q, k [steps,N,H,Dk], v [steps,N,H,Dv], g = -5 sigmoid(z) [steps,N,H,Dk],
-    beta logits [steps,N,H]."""
+    q, k [steps,N,H,Dk], v [steps,N,H,Dv], g = -5 sigmoid(z) [steps,N,H,Dk]
+    (or z itself with gate="input"), beta [steps,N,H] logits (or U(0, 1)
+    probabilities with beta="prob")."""
     gen = _gen(device, seed)
     f32 = dict(dtype=torch.float32, device=device, generator=gen)
     S0 = torch.randn(N, H, Dk, Dv, **f32) * 0.1
     q = torch.randn(steps, N, H, Dk, **f32).to(dtype)
     k = torch.randn(steps, N, H, Dk, **f32).to(dtype)
     v = torch.randn(steps, N, H, Dv, **f32).to(dtype)
-    g = (-5.0 * torch.sigmoid(torch.randn(steps, N, H, Dk, **f32))).to(dtype)
-    beta = torch.randn(steps, N, H, **f32).to(dtype)
-    return dict(state=S0, q=q, k=k, v=v, g=g, beta=beta)
+    z = torch.randn(steps, N, H, Dk, **f32)
+    if gate == "decode":
+        g = (-5.0 * torch.sigmoid(z)).to(dtype)
+    elif gate == "input":
+        g = z.to(dtype)
+    else:
+        raise ValueError(gate)
+    beta_t = torch.randn(steps, N, H, **f32)
+    if beta == "prob":
+        beta_t = torch.rand(steps, N, H, **f32)
+    elif beta != "logit":
+        raise ValueError(beta)
+    return dict(state=S0, q=q, k=k, v=v, g=g, beta=beta_t.to(dtype))
 
 
 def decode_inputs(idx_or_wl, device="cpu", steps=None):

@@ -21,6 +21,10 @@ KDA_ERR_WORKSPACE = 5
 KDA_DTYPE_F32 = 0
 KDA_DTYPE_BF16 = 1
 
+KDA_GATE_LOG = 0
+KDA_GATE_SOFTPLUS = 1
+KDA_GATE_SAFE = 2
+
 _vp = ctypes.c_void_p
 _fp = ctypes.POINTER(ctypes.c_float)
 _i32p = ctypes.POINTER(ctypes.c_int32)
@@ -41,6 +45,8 @@ class ChunkArgs(ctypes.Structure):
         ("has_lower_bound", ctypes.c_int), ("lower_bound", ctypes.c_float),
         ("chunk_size", ctypes.c_int),
         ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+        ("gate_mode", ctypes.c_int), ("A_log", _vp), ("dt_bias", _vp),
+        ("beta_is_prob", ctypes.c_int),
     ]
 
 
@@ -53,6 +59,8 @@ class StepArgs(ctypes.Structure):
         ("scale", ctypes.c_float),
         ("use_qk_l2norm", ctypes.c_int),
         ("has_lower_bound", ctypes.c_int), ("lower_bound", ctypes.c_float),
+        ("gate_mode", ctypes.c_int), ("A_log", _vp), ("dt_bias", _vp),
+        ("beta_is_prob", ctypes.c_int),
     ]
 
 

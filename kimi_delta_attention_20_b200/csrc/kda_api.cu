@@ -34,6 +34,22 @@ float resolve_scale(float s, int Dk) {
     return s;
 }
 
+// Gate mode against the lower-bound flag: the unbounded in-kernel form has no
+// lower bound and the safe form needs one.
+kda_status check_gate_mode(int mode, int has_lb) {
+    if (mode == KDA_GATE_LOG) return KDA_OK;
+    if (mode == KDA_GATE_SOFTPLUS) return has_lb ? KDA_ERR_INVALID_ARGUMENT : KDA_OK;
+    if (mode == KDA_GATE_SAFE) return has_lb ? KDA_OK : KDA_ERR_INVALID_ARGUMENT;
+    return KDA_ERR_INVALID_ARGUMENT;
+}
+
+// Gate parameter pointers, when the in-kernel gate will read them.
+kda_status check_gate_ptrs(int mode, const float *A_log, const float *dt_bias) {
+    if (mode == KDA_GATE_LOG) return KDA_OK;
+    if (!A_log || !aligned(A_log, 4) || (dt_bias && !aligned(dt_bias, 4))) return KDA_ERR_INVALID_ARGUMENT;
+    return KDA_OK;
+}
+
 // Shapes and flags only (shared by the workspace query and the launch).
 kda_status check_chunk_shape(const kda_chunk_args *a, int *N_out) {
     if (!a) return KDA_ERR_INVALID_ARGUMENT;
@@ -42,6 +58,7 @@ kda_status check_chunk_shape(const kda_chunk_args *a, int *N_out) {
     if (!head_dim_ok(a->Dk) || !head_dim_ok(a->Dv)) return KDA_ERR_UNSUPPORTED;
     if (a->chunk_size != 0 && a->chunk_size != 64) return KDA_ERR_UNSUPPORTED;
     if (a->has_lower_bound && !(a->lower_bound < 0.f)) return KDA_ERR_INVALID_ARGUMENT;
+    if (check_gate_mode(a->gate_mode, a->has_lower_bound) != KDA_OK) return KDA_ERR_INVALID_ARGUMENT;
     if ((long long)a->B * a->T * a->H * (a->Dk > a->Dv ? a->Dk : a->Dv) >= (1LL << 40))
         return KDA_ERR_INVALID_ARGUMENT;
     int N = a->N;
@@ -103,6 +120,7 @@ kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
         if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->g, 16) ||
             !aligned(a->o, 16) || !aligned(a->beta, esz))
             return KDA_ERR_INVALID_ARGUMENT;
+        if (check_gate_ptrs(a->gate_mode, a->A_log, a->dt_bias) != KDA_OK) return KDA_ERR_INVALID_ARGUMENT;
     }
     if ((a->initial_state && !aligned(a->initial_state, 16)) ||
         (a->final_state && !aligned(a->final_state, 16)))
@@ -123,6 +141,10 @@ kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
     p.use_l2 = a->use_qk_l2norm ? 1 : 0;
     p.has_lb = a->has_lower_bound ? 1 : 0;
     p.lb = a->lower_bound;
+    p.gate_mode = a->gate_mode;
+    p.A_log = a->A_log;
+    p.dt_bias = a->dt_bias;
+    p.beta_prob = a->beta_is_prob ? 1 : 0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     if (ntok > 0 && kda::chunk_tc_supported(bf16, a->Dk, a->Dv, a->chunk_size)) {
@@ -141,6 +163,7 @@ kda_status kda_recurrent_step(const kda_step_args *a, void *stream) {
     if (a->N < 0 || a->H < 1 || a->Dk < 1 || a->Dv < 1) return KDA_ERR_INVALID_ARGUMENT;
     if (!head_dim_ok(a->Dk) || !head_dim_ok(a->Dv)) return KDA_ERR_UNSUPPORTED;
     if (a->has_lower_bound && !(a->lower_bound < 0.f)) return KDA_ERR_INVALID_ARGUMENT;
+    if (check_gate_mode(a->gate_mode, a->has_lower_bound) != KDA_OK) return KDA_ERR_INVALID_ARGUMENT;
     if ((long long)a->N * a->H * 4 >= 0x7fffffffLL) return KDA_ERR_INVALID_ARGUMENT;
     if (a->N == 0) return KDA_OK;
     const bool bf16 = a->dtype == KDA_DTYPE_BF16;
@@ -150,6 +173,7 @@ kda_status kda_recurrent_step(const kda_step_args *a, void *stream) {
     if (!aligned(a->q, 16) || !aligned(a->k, 16) || !aligned(a->v, 16) || !aligned(a->g, 16) ||
         !aligned(a->o, 16) || !aligned(a->state, 16) || !aligned(a->beta, esz))
         return KDA_ERR_INVALID_ARGUMENT;
+    if (check_gate_ptrs(a->gate_mode, a->A_log, a->dt_bias) != KDA_OK) return KDA_ERR_INVALID_ARGUMENT;
     kda::StepParams p;
     p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
     p.state = a->state; p.o = a->o; p.N = a->N; p.H = a->H;
@@ -157,6 +181,10 @@ kda_status kda_recurrent_step(const kda_step_args *a, void *stream) {
     p.use_l2 = a->use_qk_l2norm ? 1 : 0;
     p.has_lb = a->has_lower_bound ? 1 : 0;
     p.lb = a->lower_bound;
+    p.gate_mode = a->gate_mode;
+    p.A_log = a->A_log;
+    p.dt_bias = a->dt_bias;
+    p.beta_prob = a->beta_is_prob ? 1 : 0;
     return cuda_status(kda::launch_decode(p, bf16, a->Dk, a->Dv, static_cast<cudaStream_t>(stream)));
 }
 

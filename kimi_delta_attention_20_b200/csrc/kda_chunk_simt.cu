@@ -6,7 +6,8 @@
 // 64-column slab of d_v) and walks the sequence one chunk of C = 64 tokens
 // at a time, with the state slab S (d_k x 64, fp32) resident in shared
 // memory across chunks. Per chunk, with G the inclusive in-chunk cumsum of
-// the (clamped) gate and beta = sigmoid(logit):
+// the gate (clamped, or formed in the kernel from A_log and dt_bias) and
+// beta = sigmoid(logit) (or a given probability):
 //
 //   A_kk[r,s] = sum_c k_r k_s exp(G_r - G_s)       (s < r)
 //   A_qk[r,s] = sum_c q_r k_s exp(G_r - G_s)       (s <= r)
@@ -71,6 +72,9 @@ __global__ void __launch_bounds__(256, 1) kda_chunk_simt_kernel(ChunkParams p) {
     const Tin *Bt = static_cast<const Tin *>(p.beta);
     Tin *O = static_cast<Tin *>(p.o);
 
+    const float rate = p.gate_mode != kGateLog ? expf(p.A_log[h]) : 0.f;
+    const float *dtb = p.gate_mode != kGateLog && p.dt_bias ? p.dt_bias + (long long)h * DK : nullptr;
+
     for (long long t0 = bos; t0 < eos; t0 += C) {
         const int L = (int)((eos - t0) < C ? (eos - t0) : C);
         __syncthreads();  // previous chunk done with every buffer
@@ -80,8 +84,8 @@ __global__ void __launch_bounds__(256, 1) kda_chunk_simt_kernel(ChunkParams p) {
             float qv = 0.f, kv = 0.f, gv = 0.f;
             if (r < L) {
                 const long long off = ((t0 + r) * H + h) * DK + c;
-                qv = to_f32(Q[off]); kv = to_f32(K[off]); gv = to_f32(Gg[off]);
-                if (p.has_lb) gv = fmaxf(gv, p.lb);
+                qv = to_f32(Q[off]); kv = to_f32(K[off]);
+                gv = gate_value(to_f32(Gg[off]), dtb ? dtb[c] : 0.f, rate, p.gate_mode, p.has_lb, p.lb);
             }
             qs[i] = qv; ks[i] = kv; Gs[i] = gv;
         }
@@ -90,7 +94,7 @@ __global__ void __launch_bounds__(256, 1) kda_chunk_simt_kernel(ChunkParams p) {
             vs[i] = r < L ? to_f32(Vv[((t0 + r) * H + h) * DV + col0 + j]) : 0.f;
         }
         for (int r = tid; r < C; r += NT)
-            sb[r] = r < L ? sigmoidf_(to_f32(Bt[(t0 + r) * H + h])) : 0.f;
+            sb[r] = r < L ? beta_value(to_f32(Bt[(t0 + r) * H + h]), p.beta_prob) : 0.f;
         __syncthreads();
 
         // 2. row L2 norms of q and k (warp per row), cumsum of g (thread per channel)

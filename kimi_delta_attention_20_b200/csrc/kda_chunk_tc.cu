@@ -8,8 +8,9 @@
 // in tensor memory for the whole sequence, so every state contraction is an
 // M = 128 MMA whose accumulator row is a value channel:
 //
-//   per chunk, with G the inclusive in-chunk cumsum of the clamped gate,
-//   beta = sigmoid(logit), k^/q^ the L2-normalised rows and T' = T diag(beta),
+//   per chunk, with G the inclusive in-chunk cumsum of the gate (clamped, or
+//   formed in the kernel from A_log and dt_bias), beta = sigmoid(logit) (or a
+//   given probability), k^/q^ the L2-normalised rows and T' = T diag(beta),
 //   T = (I + diag(beta) A_kk)^-1:
 //     A_kk[r,s] = sum_c k^_r k^_s e^{G_r-G_s} (s<r), A_qk likewise with q^_r (s<=r)
 //     U^T   = V^T T'^T                   (MMA, M=v)
@@ -64,8 +65,9 @@ constexpr uint32_t KH = TPW + 8192, ST = KH + 16384;                       // ST
 constexpr uint32_t MISC = ST + 32768;
 constexpr uint32_t M_BETA = MISC, M_INVQ = MISC + 256, M_INVK = MISC + 512, M_GAM = MISC + 768,
                    M_BAR = MISC + 1280, M_TMEM = MISC + 1312,
-                   M_EW = MISC + 1536;    // [2][128] f32: e^{G_15}, e^{G_47} per channel
-constexpr uint32_t SMEM_BYTES = M_EW + 1024;
+                   M_EW = MISC + 1536,    // [2][128] f32: e^{G_15}, e^{G_47} per channel
+                   M_DTB = M_EW + 1024;   // [128] f32: dt_bias of this head (in-kernel gate)
+constexpr uint32_t SMEM_BYTES = M_DTB + 512;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // slack for 1024-byte alignment
 static_assert(YO_H1 + 4096 <= NRM && NRM + 8192 <= XKQD, "view 1");
 static_assert(LF + 64 * LDS * 4 <= TF && TF + 64 * LDT * 4 <= RF && RF + 16 * LDR * 4 <= XKQD, "view 2");
@@ -136,6 +138,29 @@ __device__ __forceinline__ float ex2a(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// log2(x) on the special-function unit (the approximate log2 instruction)
+__device__ __forceinline__ float lg2a(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// In-kernel gate (page "atlas_core/kimi_k3/kda.rs", `bounded_gate`) for this bf16
+// path, on the special-function unit: with x = x_in + bias,
+//   kGateSoftplus: -rate (max(x, 0) + ln 2 * log2(1 + 2^(-|x| log2 e)))
+//   kGateSafe:     lb / (1 + 2^(-rate x log2 e)), exponent capped at 64 so the
+//                  denominator stays finite (the capped tail is below 1e-19 |lb|)
+// The absolute error of g is a few 1e-7 * rate, far inside bf16 input rounding.
+__device__ __forceinline__ float gate_fast(float x_in, float bias, float rate, int mode, float lb) {
+    constexpr float kL2e = 1.4426950408889634f, kLn2 = 0.6931471805599453f;
+    const float x = x_in + bias;
+    if (mode == kGateSoftplus) {
+        const float e = ex2a(-fabsf(x) * kL2e);
+        return -rate * fmaf(lg2a(1.f + e), kLn2, fmaxf(x, 0.f));
+    }
+    return __fdividef(lb, 1.f + ex2a(fminf(-rate * x * kL2e, 64.f)));
+}
+
 // 1/x for normal positive x on the FMA pipe: a bit-pattern first estimate
 // (reciprocal ~ 2^(2*127) / x read off the exponent/mantissa bits) refined by two
 // Newton-Raphson steps y <- y (2 - x y); relative error ~1e-5.
@@ -184,6 +209,10 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     float *sinvk = reinterpret_cast<float *>(sm + M_INVK);
     float *sGam = reinterpret_cast<float *>(sm + M_GAM);
     float *sEw = reinterpret_cast<float *>(sm + M_EW);
+    float *sDtb = reinterpret_cast<float *>(sm + M_DTB);
+    const int gmode = p.gate_mode;
+    const float rate = gmode != kGateLog ? expf(p.A_log[h]) : 0.f;
+    if (tid < D) sDtb[tid] = gmode != kGateLog && p.dt_bias ? p.dt_bias[h * D + tid] : 0.f;
     float *Lf = reinterpret_cast<float *>(sm + LF);
     float *Tf = reinterpret_cast<float *>(sm + TF);
 
@@ -257,7 +286,7 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         const bool has_next = ci + 1 < nchunks;
 
         if (tid < C) {
-            sbeta[tid] = tid < L ? sigmoidf_(beta_next) : 0.f;
+            sbeta[tid] = tid < L ? beta_value(beta_next, p.beta_prob) : 0.f;
             beta_next = 0.f;
             if (has_next && t0 + C + tid < eos) beta_next = __bfloat162float(bt[(t0 + C + tid) * H + h]);
         }
@@ -285,10 +314,20 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                     const int r = row0 + u;
                     float2 gg[4];
                     unpack8x2(lds128(sm + STG_G, sw128_chunk(r, 8 * jch, 64)), gg);
+                    if (gmode != kGateLog) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 b = *reinterpret_cast<const float2 *>(sDtb + 8 * jch + 2 * e);
+                            gg[e] = make_float2(gate_fast(gg[e].x, b.x, rate, gmode, p.lb),
+                                                gate_fast(gg[e].y, b.y, rate, gmode, p.lb));
+                        }
+                    } else if (p.has_lb) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) gg[e] = make_float2(fmaxf(gg[e].x, p.lb), fmaxf(gg[e].y, p.lb));
+                    }
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        float2 gv = r < L ? gg[e] : make_float2(0.f, 0.f);
-                        if (p.has_lb) gv = make_float2(fmaxf(gv.x, p.lb), fmaxf(gv.y, p.lb));
+                        const float2 gv = r < L ? gg[e] : make_float2(0.f, 0.f);
                         tt[e] = __fadd2_rn(tt[e], gv);
                         G[u][2 * e] = tt[e].x;
                         G[u][2 * e + 1] = tt[e].y;
@@ -544,7 +583,8 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
                         float gv = 0.f;
                         if (s < L) {
                             gv = bf(sm + STG_G, o);
-                            if (p.has_lb) gv = fmaxf(gv, p.lb);
+                            if (gmode != kGateLog) gv = gate_fast(gv, sDtb[lane + 32 * u], rate, gmode, p.lb);
+                            else if (p.has_lb) gv = fmaxf(gv, p.lb);
                         }
                         dg[u] += gv;
                     }

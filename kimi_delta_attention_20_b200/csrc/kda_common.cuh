@@ -20,6 +20,27 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
 
+// How g is obtained from the g input (kda_gate_mode of the C ABI).
+enum : int { kGateLog = 0, kGateSoftplus = 1, kGateSafe = 2 };
+
+// The per-channel log-decay from the g input x_in (page "atlas_core/kimi_k3/kda.rs",
+// `bounded_gate`): rate = exp(A_log[h]) and bias = dt_bias[h, c].
+//   kGateLog:      x_in, clamped below by lb when has_lb
+//   kGateSoftplus: -rate * log(1 + e^x), x = x_in + bias (overflow-free split)
+//   kGateSafe:     lb * sigmoid(rate * x)
+__device__ __forceinline__ float gate_value(float x_in, float bias, float rate, int mode, int has_lb,
+                                            float lb) {
+    if (mode == kGateSoftplus) {
+        const float x = x_in + bias;
+        return -rate * (fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))));
+    }
+    if (mode == kGateSafe) return lb / (1.f + expf(-rate * (x_in + bias)));
+    return has_lb ? fmaxf(x_in, lb) : x_in;
+}
+
+// beta as the recurrence uses it: sigmoid of a logit, or the probability as given.
+__device__ __forceinline__ float beta_value(float b, int is_prob) { return is_prob ? b : sigmoidf_(b); }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -43,6 +64,10 @@ struct ChunkParams {
     int use_l2;
     int has_lb;
     float lb;
+    int gate_mode;              // kGate*
+    const float *A_log;         // [H], in-kernel gate forms
+    const float *dt_bias;       // [H, Dk] or null
+    int beta_prob;              // 1: beta is a probability
 };
 
 // Launch parameters of the recurrent decode step.
@@ -55,6 +80,10 @@ struct StepParams {
     int use_l2;
     int has_lb;
     float lb;
+    int gate_mode;
+    const float *A_log;
+    const float *dt_bias;
+    int beta_prob;
 };
 
 }  // namespace kda

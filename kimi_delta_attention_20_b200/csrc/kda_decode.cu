@@ -7,7 +7,8 @@
 // every key row, read and written back as float4 with streaming cache hints,
 // kept in registers between the read and the write (one pass over HBM).
 //
-// Per head, with S' = diag(exp g) S, the two column reductions over the key
+// g is the log-decay as given (clamped) or formed from the gate input in the
+// kernel; beta a logit or a given probability. Per head, with S' = diag(exp g) S, the two column reductions over the key
 // axis r_k = S'^T k and r_q = S'^T q are taken in the same pass; then
 //   delta = sigmoid(beta) (v - r_k),
 //   S     = S' + k delta^T,
@@ -57,12 +58,13 @@ __global__ void __launch_bounds__(256) kda_decode_kernel(StepParams p) {
     const Tin *qp = static_cast<const Tin *>(p.q) + nh * DK;
     const Tin *kp = static_cast<const Tin *>(p.k) + nh * DK;
     const Tin *gp = static_cast<const Tin *>(p.g) + nh * DK;
+    const int h = nh % p.H;
+    const float rate = p.gate_mode != kGateLog ? expf(p.A_log[h]) : 0.f;
     for (int c = tid; c < DK; c += Cfg::kThreads) {
         sq[c] = to_f32(qp[c]);
         sk[c] = to_f32(kp[c]);
-        float gv = to_f32(gp[c]);
-        if (p.has_lb) gv = fmaxf(gv, p.lb);
-        sa[c] = expf(gv);
+        const float bias = p.gate_mode != kGateLog && p.dt_bias ? p.dt_bias[h * DK + c] : 0.f;
+        sa[c] = expf(gate_value(to_f32(gp[c]), bias, rate, p.gate_mode, p.has_lb, p.lb));
     }
     __syncthreads();
     if (warp == 0) {
@@ -110,7 +112,7 @@ __global__ void __launch_bounds__(256) kda_decode_kernel(StepParams p) {
 #pragma unroll
         for (int w = 0; w < NW; ++w) { a += rk_part[w][lane]; b += rq_part[w][lane]; }
         const int col = slab * Cfg::kCols + lane;
-        const float bsig = sigmoidf_(to_f32(static_cast<const Tin *>(p.beta)[nh]));
+        const float bsig = beta_value(to_f32(static_cast<const Tin *>(p.beta)[nh]), p.beta_prob);
         const float vj = to_f32(static_cast<const Tin *>(p.v)[nh * DV + col]);
         const float delta = bsig * (vj - inv_k * a);
         sdelta[lane] = delta;

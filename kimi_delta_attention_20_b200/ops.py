@@ -33,20 +33,65 @@ def _stream(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+def _gate_fields(a, device, H, Dk, A_log, dt_bias, use_gate_in_kernel, safe_gate,
+                 lower_bound, use_beta_sigmoid_in_kernel):
+    """Gate and beta fields of the C argument struct (page "K3/kda/ops/api.py",
+    `use_gate_in_kernel`, `safe_gate`, `use_beta_sigmoid_in_kernel`)."""
+    if lower_bound is not None and not lower_bound < 0:
+        raise ValueError("lower_bound must be negative")
+    a.beta_is_prob = int(not use_beta_sigmoid_in_kernel)
+    if not use_gate_in_kernel:
+        a.gate_mode = _abi.KDA_GATE_LOG
+        a.has_lower_bound = int(lower_bound is not None)
+        a.lower_bound = float(lower_bound) if lower_bound is not None else 0.0
+        return
+    if A_log is None:
+        raise ValueError("A_log is required when use_gate_in_kernel=True")
+    _need_cuda("A_log", A_log)
+    if A_log.dtype != torch.float32 or A_log.numel() != H or A_log.device != device:
+        raise ValueError(f"A_log must be float32 with {H} elements on {device}")
+    if dt_bias is not None:
+        _need_cuda("dt_bias", dt_bias)
+        if dt_bias.dtype != torch.float32 or dt_bias.numel() != H * Dk or dt_bias.device != device:
+            raise ValueError(f"dt_bias must be float32 with {H}x{Dk} elements on {device}")
+    a.A_log = _ptr(A_log)
+    a.dt_bias = _ptr(dt_bias)
+    if safe_gate:
+        if lower_bound is None:
+            raise ValueError("lower_bound is required when safe_gate=True")
+        a.gate_mode = _abi.KDA_GATE_SAFE
+        a.has_lower_bound = 1
+        a.lower_bound = float(lower_bound)
+    else:  # the unbounded form takes no lower bound
+        a.gate_mode = _abi.KDA_GATE_SOFTPLUS
+        a.has_lower_bound = 0
+        a.lower_bound = 0.0
+
+
 def chunk_kda(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
-              beta: torch.Tensor, *, scale: Optional[float] = None,
+              beta: torch.Tensor, *, A_log: Optional[torch.Tensor] = None,
+              dt_bias: Optional[torch.Tensor] = None, scale: Optional[float] = None,
               initial_state: Optional[torch.Tensor] = None, output_final_state: bool = False,
-              use_qk_l2norm_in_kernel: bool = False, lower_bound: Optional[float] = None,
+              use_qk_l2norm_in_kernel: bool = False, use_gate_in_kernel: bool = False,
+              use_beta_sigmoid_in_kernel: bool = True, safe_gate: bool = False,
+              lower_bound: Optional[float] = None,
               chunk_size: int = 64, cu_seqlens: Optional[torch.Tensor] = None,
               out: Optional[torch.Tensor] = None, final_state_out: Optional[torch.Tensor] = None,
               workspace: Optional[torch.Tensor] = None
               ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunkwise KDA forward (the `chunk_kda` boundary of page
-    "K3/kda/ops/api.py", without backend dispatch or in-kernel gate).
+    "K3/kda/ops/api.py", without backend dispatch).
 
-    q, k, g: [B, T, H, Dk]; v: [B, T, H, Dv]; beta: [B, T, H] LOGITS.
-    g is the per-channel log-decay (<= 0); ``lower_bound`` clamps it from
-    below. ``cu_seqlens`` (int32, [N+1], B == 1) packs N sequences.
+    q, k, g: [B, T, H, Dk]; v: [B, T, H, Dv]; beta: [B, T, H].
+    beta holds LOGITS (sigmoid in the kernel) unless use_beta_sigmoid_in_kernel
+    is False, when it holds probabilities used as given. Note the default: the
+    logit form is this operator's boundary, where api.py defaults to False.
+    g is the per-channel log-decay (<= 0), clamped below by ``lower_bound``;
+    with use_gate_in_kernel it is the gate input instead and the kernel forms
+    -exp(A_log) softplus(g + dt_bias), or with safe_gate
+    lower_bound * sigmoid(exp(A_log) (g + dt_bias)) (A_log: [H] fp32,
+    dt_bias: [H, Dk] fp32 or None; the unbounded form ignores lower_bound).
+    ``cu_seqlens`` (int32, [N+1], B == 1) packs N sequences.
     Returns (o [B, T, H, Dv], final_state [N, H, Dk, Dv] fp32 or None).
     """
     lib = _abi.load()
@@ -65,8 +110,6 @@ def chunk_kda(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
             "use_qk_l2norm_in_kernel=False: the chunkwise form relies on unit-norm keys; "
             "unnormalised keys can make the output grow without bound.",
             RuntimeWarning, stacklevel=2)
-    if lower_bound is not None and not lower_bound < 0:
-        raise ValueError("lower_bound must be negative")
     if chunk_size not in (0, 64):
         raise ValueError("chunk_size must be 64")
     cu_host = None
@@ -99,8 +142,8 @@ def chunk_kda(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
     a.cu_seqlens_host = _ptr(cu_host)
     a.N = N
     a.use_qk_l2norm = int(bool(use_qk_l2norm_in_kernel))
-    a.has_lower_bound = int(lower_bound is not None)
-    a.lower_bound = float(lower_bound) if lower_bound is not None else 0.0
+    _gate_fields(a, q.device, H, Dk, A_log, dt_bias, use_gate_in_kernel, safe_gate, lower_bound,
+                 use_beta_sigmoid_in_kernel)
     a.chunk_size = int(chunk_size)
     nbytes = ctypes.c_size_t(0)
     _abi.check(lib.kda_chunk_fwd_workspace_size(ctypes.byref(a), ctypes.byref(nbytes)),
@@ -130,14 +173,18 @@ def chunk_workspace_bytes(B, T, H, Dk, Dv, *, dtype=torch.bfloat16, N=None, varl
 
 
 def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
-                   beta: torch.Tensor, state: torch.Tensor, *, scale: Optional[float] = None,
-                   use_qk_l2norm_in_kernel: bool = True, lower_bound: Optional[float] = None,
+                   beta: torch.Tensor, state: torch.Tensor, *, A_log: Optional[torch.Tensor] = None,
+                   dt_bias: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                   use_qk_l2norm_in_kernel: bool = True, use_gate_in_kernel: bool = False,
+                   use_beta_sigmoid_in_kernel: bool = True, safe_gate: bool = False,
+                   lower_bound: Optional[float] = None,
                    out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """One decode token per sequence (page "atlas_core/kimi_k3/kda.rs",
     `kda_recurrent_step`, which always normalises q and k).
 
-    q, k, g: [N, H, Dk]; v: [N, H, Dv]; beta: [N, H] logits; state:
-    [N, H, Dk, Dv] fp32, updated IN PLACE. Returns o [N, H, Dv].
+    q, k, g: [N, H, Dk]; v: [N, H, Dv]; beta: [N, H] logits (or probabilities
+    with use_beta_sigmoid_in_kernel=False); state: [N, H, Dk, Dv] fp32, updated
+    IN PLACE. Gate arguments as in ``chunk_kda``. Returns o [N, H, Dv].
     """
     lib = _abi.load()
     for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta), ("state", state)):
@@ -150,8 +197,6 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
         raise ValueError("shape mismatch among q, k, v, g, beta")
     if state.dtype != torch.float32 or state.shape != (N, H, Dk, Dv):
         raise ValueError(f"state must be float32 [{N}, {H}, {Dk}, {Dv}]")
-    if lower_bound is not None and not lower_bound < 0:
-        raise ValueError("lower_bound must be negative")
     o = out if out is not None else torch.empty(N, H, Dv, dtype=q.dtype, device=q.device)
     a = _abi.StepArgs()
     a.dtype = _DTYPES[q.dtype]
@@ -159,8 +204,8 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
     a.q, a.k, a.v, a.g, a.beta, a.state, a.o = (_ptr(t) for t in (q, k, v, g, beta, state, o))
     a.scale = float("nan") if scale is None else float(scale)
     a.use_qk_l2norm = int(bool(use_qk_l2norm_in_kernel))
-    a.has_lower_bound = int(lower_bound is not None)
-    a.lower_bound = float(lower_bound) if lower_bound is not None else 0.0
+    _gate_fields(a, q.device, H, Dk, A_log, dt_bias, use_gate_in_kernel, safe_gate, lower_bound,
+                 use_beta_sigmoid_in_kernel)
     with torch.cuda.device(q.device):
         _abi.check(lib.kda_recurrent_step(ctypes.byref(a), _stream(q.device)), "kda_recurrent_step")
     return o

@@ -14,6 +14,9 @@ with the host C compiler, or ahead of time by ``build()``):
 * ``chunkwise`` -- form C, the chunk-at-a-time WY/UT form that the
   ``chunk_kda`` boundary of page "K3/kda/ops/api.py" computes, derived here
   from the same recurrence. It exists to cross-check form R.
+* ``gate`` -- the in-kernel forget gate of the same boundary (``A_log``,
+  ``dt_bias``, unbounded or safe form), in fp64 numpy, as page
+  "atlas_core/kimi_k3/kda.rs" writes it in ``bounded_gate``.
 
 Both take packed inputs: q, k, g of shape [T_total, H, d_k], v of shape
 [T_total, H, d_v], beta logits [T_total, H], ``cu_seqlens`` int offsets
@@ -66,9 +69,9 @@ def _load():
             common = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, i64p,
                       dp, dp, dp, dp, dp, ctypes.c_double, dp, dp, dp,
                       ctypes.c_int, ctypes.c_int, ctypes.c_double]
-            lib.kda_oracle_recurrent.argtypes = common + [ctypes.c_int]
+            lib.kda_oracle_recurrent.argtypes = common + [ctypes.c_int, ctypes.c_int]
             lib.kda_oracle_recurrent.restype = ctypes.c_int
-            lib.kda_oracle_chunkwise.argtypes = common + [ctypes.c_int, ctypes.c_int]
+            lib.kda_oracle_chunkwise.argtypes = common + [ctypes.c_int, ctypes.c_int, ctypes.c_int]
             lib.kda_oracle_chunkwise.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -125,14 +128,65 @@ def _threads(nthreads):
     return os.cpu_count() or 1
 
 
+def softplus(x):
+    """log(1 + e^x) in the overflow-free split max(x, 0) + log1p(e^-|x|)
+    (page "atlas_core/kimi_k3/kda.rs", `softplus`)."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x)))
+
+
+def gate(g_in, A_log, dt_bias=None, lower_bound=None):
+    """In-kernel forget gate in log space for inputs g_in [..., H, Dk].
+
+    With x = g_in + dt_bias (dt_bias [H, Dk] or None) and rate = exp(A_log[h]):
+      lower_bound None: g = -rate * softplus(x)                (unbounded form)
+      lower_bound lb:   g = lb * sigmoid(rate * x)             (safe form)
+    (page "atlas_core/kimi_k3/kda.rs", `bounded_gate`; page "K3/kda/ops/api.py",
+    `use_gate_in_kernel` / `safe_gate`).
+    """
+    x = _f64(g_in)
+    if dt_bias is not None:
+        x = x + _f64(dt_bias)
+    rate = np.exp(_f64(A_log)).reshape(-1, 1)
+    if lower_bound is None:
+        return -rate * softplus(x)
+    return float(lower_bound) / (1.0 + np.exp(-rate * x))
+
+
+def _gate_prep(g, gate_form, A_log, dt_bias, lower_bound):
+    """The log-decay the recurrence uses, and the lower bound left to clamp it.
+
+    gate_form None: g is the log-decay (clamped by lower_bound inside the recurrence).
+    gate_form "softplus" / "safe": g is the gate input, turned into the log-decay by
+    ``gate`` above (page "K3/kda/ops/api.py", ``use_gate_in_kernel``; the
+    unbounded form takes no lower bound, the safe form needs one).
+    """
+    if gate_form is None:
+        return g, lower_bound
+    if gate_form not in ("softplus", "safe"):
+        raise ValueError("gate_form must be None, 'softplus' or 'safe'")
+    if A_log is None:
+        raise ValueError("the in-kernel gate needs A_log")
+    if gate_form == "safe" and lower_bound is None:
+        raise ValueError("the safe gate needs lower_bound")
+    g = _f64(g)
+    H, Dk = g.shape[-2], g.shape[-1]
+    dt = None if dt_bias is None else _f64(dt_bias).reshape(H, Dk)
+    return gate(g, _f64(A_log).reshape(H), dt, lower_bound if gate_form == "safe" else None), None
+
+
 def recurrent(q, k, v, g, beta, *, scale=None, initial_state=None, cu_seqlens=None,
-              use_qk_l2norm=True, lower_bound=None, nthreads=0):
+              use_qk_l2norm=True, lower_bound=None, beta_is_logit=True,
+              gate_form=None, A_log=None, dt_bias=None, nthreads=0):
     """Form R (the definition). Returns (o [T_total,H,d_v], final_state [N,H,d_k,d_v]).
 
-    ``beta`` holds logits (sigmoid applied per token), ``g`` holds per-channel
-    log-decays, ``lower_bound`` clamps g from below, ``scale`` defaults to
-    1/sqrt(d_k).
+    ``beta`` holds logits (sigmoid applied per token) unless ``beta_is_logit`` is
+    False (then probabilities, used as given); ``g`` holds per-channel log-decays,
+    ``lower_bound`` clamps g from below, ``scale`` defaults to 1/sqrt(d_k). With
+    ``gate_form`` = "softplus" or "safe", ``g`` is the gate input instead (see
+    ``_gate_prep``).
     """
+    g, lower_bound = _gate_prep(g, gate_form, A_log, dt_bias, lower_bound)
     q, k, v, g, beta, cu, S0, N, H, Dk, Dv = _prep(q, k, v, g, beta, cu_seqlens, initial_state)
     if scale is None:
         scale = 1.0 / np.sqrt(Dk)
@@ -142,15 +196,18 @@ def recurrent(q, k, v, g, beta, *, scale=None, initial_state=None, cu_seqlens=No
         N, H, Dk, Dv, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(S0), _ptr(o), _ptr(S),
         int(bool(use_qk_l2norm)), int(lower_bound is not None),
-        float(lower_bound if lower_bound is not None else 0.0), _threads(nthreads))
+        float(lower_bound if lower_bound is not None else 0.0), int(bool(beta_is_logit)),
+        _threads(nthreads))
     if rc != 0:
         raise RuntimeError(f"kda_oracle_recurrent failed ({rc})")
     return o, S
 
 
 def chunkwise(q, k, v, g, beta, *, scale=None, initial_state=None, cu_seqlens=None,
-              use_qk_l2norm=True, lower_bound=None, chunk_size=64, nthreads=0):
+              use_qk_l2norm=True, lower_bound=None, beta_is_logit=True,
+              gate_form=None, A_log=None, dt_bias=None, chunk_size=64, nthreads=0):
     """Form C (chunkwise WY/UT). Same arguments and results as ``recurrent``."""
+    g, lower_bound = _gate_prep(g, gate_form, A_log, dt_bias, lower_bound)
     q, k, v, g, beta, cu, S0, N, H, Dk, Dv = _prep(q, k, v, g, beta, cu_seqlens, initial_state)
     if scale is None:
         scale = 1.0 / np.sqrt(Dk)
@@ -160,8 +217,8 @@ def chunkwise(q, k, v, g, beta, *, scale=None, initial_state=None, cu_seqlens=No
         N, H, Dk, Dv, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(S0), _ptr(o), _ptr(S),
         int(bool(use_qk_l2norm)), int(lower_bound is not None),
-        float(lower_bound if lower_bound is not None else 0.0), int(chunk_size),
-        _threads(nthreads))
+        float(lower_bound if lower_bound is not None else 0.0), int(bool(beta_is_logit)),
+        int(chunk_size), _threads(nthreads))
     if rc != 0:
         raise RuntimeError(f"kda_oracle_chunkwise failed ({rc})")
     return o, S

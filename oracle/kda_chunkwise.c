@@ -41,6 +41,7 @@ typedef struct {
     double *o, *S_out;
     int l2, has_lb;
     double lb;
+    int beta_logit; /* 1: beta holds logits (sigmoid applied); 0: probabilities */
     int next, npairs, failed;
     pthread_mutex_t mu;
 } chk_job;
@@ -103,7 +104,7 @@ static void chk_chunk(chk_job *J, chk_buf *B, int h, int64_t t0, int L)
             B->G[(size_t)r * Dk + c] = (r ? B->G[(size_t)(r - 1) * Dk + c] : 0.0) + gc;
         }
         memcpy(B->vv + (size_t)r * Dv, J->v + row * Dv, sizeof(double) * Dv);
-        B->b[r] = 1.0 / (1.0 + exp(-J->beta[row]));
+        B->b[r] = J->beta_logit ? 1.0 / (1.0 + exp(-J->beta[row])) : J->beta[row];
     }
     /* gated key-key and query-key blocks, lower triangle only */
     for (int r = 0; r < L; ++r)
@@ -216,7 +217,7 @@ int kda_oracle_chunkwise(int N, int H, int Dk, int Dv, const int64_t *cu_seqlens
                          const double *q, const double *k, const double *v, const double *g,
                          const double *beta, double scale, const double *initial_state,
                          double *o, double *final_state, int use_qk_l2norm, int has_lower_bound,
-                         double lower_bound, int chunk_size, int nthreads)
+                         double lower_bound, int beta_is_logit, int chunk_size, int nthreads)
 {
     if (N < 0 || H <= 0 || Dk <= 0 || Dv <= 0 || chunk_size <= 0 || !cu_seqlens) return -1;
     if (cu_seqlens[0] != 0) return -1;
@@ -225,6 +226,7 @@ int kda_oracle_chunkwise(int N, int H, int Dk, int Dv, const int64_t *cu_seqlens
     chk_job J;
     J.N = N; J.H = H; J.Dk = Dk; J.Dv = Dv; J.C = chunk_size; J.cu = cu_seqlens;
     J.q = q; J.k = k; J.v = v; J.g = g; J.beta = beta; J.scale = scale;
+    J.beta_logit = beta_is_logit;
     J.S0 = initial_state; J.o = o; J.S_out = final_state;
     J.l2 = use_qk_l2norm; J.has_lb = has_lower_bound; J.lb = lower_bound;
     J.next = 0; J.npairs = N * H; J.failed = 0;

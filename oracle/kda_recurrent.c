@@ -14,12 +14,14 @@
  *     g  = max(g_t, lower_bound)                          (if a bound is given)
  *     S  = diag(exp(g)) S            decay on the key axis, per channel
  *     d  = sigmoid(beta_t) (v_t - S^T k^)                 read of the decayed S
+ *          (beta_t as given when it holds probabilities: api.py's
+ *          use_beta_sigmoid_in_kernel = False)
  *     S  = S + k^ d^T                                     rank-1 write
  *     o_t = scale S^T q^                                  read of the updated S
  *   final_state[n,h] = S.
  *
  * Layout: q,k,g are [T_total, H, d_k], v and o are [T_total, H, d_v], beta is
- * [T_total, H] (logits), states are [N, H, d_k, d_v] with element (c, j) of a
+ * [T_total, H] (logits, or probabilities), states are [N, H, d_k, d_v] with element (c, j) of a
  * head at c*d_v + j. Sequence n covers tokens cu_seqlens[n] .. cu_seqlens[n+1].
  * Every pair (n, h) is independent; pairs are spread over POSIX threads.
  */
@@ -37,6 +39,7 @@ typedef struct {
     const double *S0;
     double *o, *S_out;
     int use_qk_l2norm, has_lb;
+    int beta_logit; /* 1: beta holds logits (sigmoid applied); 0: probabilities */
     double lb;
     int next_pair, npairs;
     pthread_mutex_t lock;
@@ -92,7 +95,8 @@ static int rec_pair(rec_job *J, int n, int h)
             for (int j = 0; j < Dv; ++j) S[(size_t)c * Dv + j] *= a;
         }
         /* delta = sigmoid(beta) (v - S^T k^) */
-        double b = rec_sigmoid(J->beta[(size_t)t * H + h]);
+        double b = J->beta[(size_t)t * H + h];
+        if (J->beta_logit) b = rec_sigmoid(b);
         for (int j = 0; j < Dv; ++j) {
             double kv = 0.0;
             for (int c = 0; c < Dk; ++c) kv += S[(size_t)c * Dv + j] * kh[c];
@@ -136,7 +140,7 @@ int kda_oracle_recurrent(int N, int H, int Dk, int Dv, const int64_t *cu_seqlens
                          const double *q, const double *k, const double *v, const double *g,
                          const double *beta, double scale, const double *initial_state,
                          double *o, double *final_state, int use_qk_l2norm, int has_lower_bound,
-                         double lower_bound, int nthreads)
+                         double lower_bound, int beta_is_logit, int nthreads)
 {
     if (N < 0 || H <= 0 || Dk <= 0 || Dv <= 0 || !cu_seqlens) return -1;
     if (cu_seqlens[0] != 0) return -1;
@@ -145,6 +149,7 @@ int kda_oracle_recurrent(int N, int H, int Dk, int Dv, const int64_t *cu_seqlens
     rec_job J;
     J.N = N; J.H = H; J.Dk = Dk; J.Dv = Dv; J.cu_seqlens = cu_seqlens;
     J.q = q; J.k = k; J.v = v; J.g = g; J.beta = beta; J.scale = scale;
+    J.beta_logit = beta_is_logit;
     J.S0 = initial_state; J.o = o; J.S_out = final_state;
     J.use_qk_l2norm = use_qk_l2norm; J.has_lb = has_lower_bound; J.lb = lower_bound;
     J.next_pair = 0; J.npairs = N * H; J.failed = 0;

@@ -40,9 +40,12 @@ def check(name, got, want, dtype):
     return rel
 
 
-def oracle_chunk(inp, *, heads=None, seqs=None, scale=None, lower_bound=None, l2=True):
+def oracle_chunk(inp, *, heads=None, seqs=None, scale=None, lower_bound=None, l2=True,
+                 beta_is_logit=True, gate_form=None, A_log=None, dt_bias=None):
     """Form R on (a subset of) a chunk-forward input dict; returns per-sequence
-    (o [T_n, h, Dv], S [h, Dk, Dv]) lists over the chosen sequences and heads."""
+    (o [T_n, h, Dv], S [h, Dk, Dv]) lists over the chosen sequences and heads.
+    The gate arguments are those of ``oracle.recurrent`` (A_log [H], dt_bias
+    [H, Dk] over all heads; the chosen heads are taken from them)."""
     q, k, v, g, beta = (inp[n] for n in ("q", "k", "v", "g", "beta"))
     B, T, H, _ = q.shape
     cu = inp.get("cu_seqlens")
@@ -56,12 +59,18 @@ def oracle_chunk(inp, *, heads=None, seqs=None, scale=None, lower_bound=None, l2
     hs = list(range(H)) if heads is None else list(heads)
     ns = list(range(len(bounds))) if seqs is None else list(seqs)
     S0 = inp.get("initial_state")
+    if A_log is not None:
+        A_log = _np(A_log).reshape(H)[hs]
+    if dt_bias is not None:
+        dt_bias = _np(dt_bias).reshape(H, -1)[hs]
     out = []
     for n in ns:
         a, b = bounds[n]
         sl = lambda x: flat(x)[a:b][:, hs]
         s0 = None if S0 is None else S0[n:n + 1, hs]
         o, S = oracle.recurrent(sl(q), sl(k), sl(v), sl(g), flat(beta)[a:b][:, hs], scale=scale,
-                                initial_state=s0, use_qk_l2norm=l2, lower_bound=lower_bound)
+                                initial_state=s0, use_qk_l2norm=l2, lower_bound=lower_bound,
+                                beta_is_logit=beta_is_logit, gate_form=gate_form, A_log=A_log,
+                                dt_bias=dt_bias)
         out.append((a, b, o, S[0]))
     return out

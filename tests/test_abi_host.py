@@ -85,6 +85,16 @@ def step_args(**over):
     (dict(B=2, N=3), _abi.KDA_ERR_INVALID_ARGUMENT),
     (dict(B=2, cu_seqlens=FAKE, N=2), _abi.KDA_ERR_INVALID_ARGUMENT),
     (dict(cu_seqlens=FAKE, N=0), _abi.KDA_ERR_INVALID_ARGUMENT),
+    # in-kernel gate: unknown mode, missing A_log, misaligned pointers, bound rules
+    (dict(gate_mode=3, A_log=FAKE), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(gate_mode=_abi.KDA_GATE_SOFTPLUS), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(gate_mode=_abi.KDA_GATE_SOFTPLUS, A_log=FAKE + 2), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(gate_mode=_abi.KDA_GATE_SOFTPLUS, A_log=FAKE, dt_bias=FAKE + 1), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(gate_mode=_abi.KDA_GATE_SOFTPLUS, A_log=FAKE, has_lower_bound=1, lower_bound=-5.0),
+     _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(gate_mode=_abi.KDA_GATE_SAFE, A_log=FAKE), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(gate_mode=_abi.KDA_GATE_SAFE, A_log=FAKE, has_lower_bound=1, lower_bound=1.0),
+     _abi.KDA_ERR_INVALID_ARGUMENT),
 ])
 def test_chunk_fwd_rejects(over, want):
     lib = _abi.load()
@@ -152,3 +162,63 @@ def test_python_binding_refuses_cpu_tensors():
         kda.chunk_kda(x, x, x, x, torch.zeros(1, 4, 1), use_qk_l2norm_in_kernel=True)
     with pytest.raises(ValueError):
         kda.recurrent_step(x[0], x[0], x[0], x[0], torch.zeros(4, 1), torch.zeros(4, 1, 32, 32))
+
+
+@pytest.mark.parametrize("over", [
+    dict(gate_mode=_abi.KDA_GATE_SOFTPLUS, A_log=FAKE, q=None),
+    dict(gate_mode=_abi.KDA_GATE_SAFE, A_log=FAKE, has_lower_bound=1, lower_bound=-5.0, o=None),
+])
+def test_valid_gate_modes_pass_gate_checks(over):
+    """A request whose gate fields are valid fails only on the pointer planted as bad."""
+    lib = _abi.load()
+    a = chunk_args(**over)
+    assert lib.kda_chunk_fwd(ctypes.byref(a), None) == _abi.KDA_ERR_INVALID_ARGUMENT
+    n = ctypes.c_size_t(0)
+    assert lib.kda_chunk_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == _abi.KDA_OK
+
+
+@pytest.mark.parametrize("over,want", [
+    (dict(gate_mode=_abi.KDA_GATE_SOFTPLUS), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(gate_mode=_abi.KDA_GATE_SAFE, A_log=FAKE), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(gate_mode=-1), _abi.KDA_ERR_INVALID_ARGUMENT),
+])
+def test_step_rejects_bad_gate(over, want):
+    lib = _abi.load()
+    a = step_args(**over)
+    assert lib.kda_recurrent_step(ctypes.byref(a), None) == want
+
+
+_LAYOUT_C = r"""
+#include <stdio.h>
+#include <stddef.h>
+#include "kda.h"
+#define F(S, m) printf(#S " " #m " %zu\n", offsetof(S, m));
+int main(void) {
+    printf("kda_chunk_args sizeof %zu\n", sizeof(kda_chunk_args));
+    printf("kda_step_args sizeof %zu\n", sizeof(kda_step_args));
+    CHUNK_FIELDS
+    STEP_FIELDS
+    return 0;
+}
+"""
+
+
+def test_ctypes_structs_match_header_layout(tmp_path):
+    """Every field of the ctypes mirrors sits at the offset the C compiler gives it."""
+    import subprocess
+    chunk = "".join(f"F(kda_chunk_args, {n})" for n, _ in _abi.ChunkArgs._fields_)
+    step = "".join(f"F(kda_step_args, {n})" for n, _ in _abi.StepArgs._fields_)
+    src = tmp_path / "layout.c"
+    src.write_text(_LAYOUT_C.replace("CHUNK_FIELDS", chunk).replace("STEP_FIELDS", step))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)],
+                   check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines():
+        struct, field, val = line.split()
+        got[(struct, field)] = int(val)
+    assert got[("kda_chunk_args", "sizeof")] == ctypes.sizeof(_abi.ChunkArgs)
+    assert got[("kda_step_args", "sizeof")] == ctypes.sizeof(_abi.StepArgs)
+    for cls, name in ((_abi.ChunkArgs, "kda_chunk_args"), (_abi.StepArgs, "kda_step_args")):
+        for field, _ in cls._fields_:
+            assert got[(name, field)] == getattr(cls, field).offset, (name, field)

@@ -38,9 +38,9 @@ def run_chunk(inp, wl=None, *, scale=None, lower_bound=None, final=True, l2=True
 
 
 def compare_chunk(inp, o, S, dtype, *, heads=None, seqs=None, scale=None, lower_bound=None,
-                  l2=True, tag=""):
+                  l2=True, tag="", **okw):
     ref = oracle_chunk({k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()},
-                       heads=heads, seqs=seqs, scale=scale, lower_bound=lower_bound, l2=l2)
+                       heads=heads, seqs=seqs, scale=scale, lower_bound=lower_bound, l2=l2, **okw)
     H = inp["q"].shape[2]
     hs = list(range(H)) if heads is None else list(heads)
     ns = list(range(len(ref))) if seqs is None else list(seqs)

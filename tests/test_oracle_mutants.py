@@ -23,8 +23,12 @@ MUTANTS = {
     # form R
     "R: no decay": ("kda_recurrent.c", "S[(size_t)c * Dv + j] *= a;", "S[(size_t)c * Dv + j] *= 1.0;"),
     "R: delta sign": ("kda_recurrent.c", "delta[j] = b * (vt[j] - kv);", "delta[j] = b * (vt[j] + kv);"),
-    "R: beta not squashed": ("kda_recurrent.c", "double b = rec_sigmoid(J->beta[(size_t)t * H + h]);",
-                             "double b = J->beta[(size_t)t * H + h];"),
+    "R: beta not squashed": ("kda_recurrent.c", "if (J->beta_logit) b = rec_sigmoid(b);", ""),
+    "R: beta always squashed": ("kda_recurrent.c", "if (J->beta_logit) b = rec_sigmoid(b);",
+                                "b = rec_sigmoid(b);"),
+    "C: beta always squashed": ("kda_chunkwise.c",
+                                "B->b[r] = J->beta_logit ? 1.0 / (1.0 + exp(-J->beta[row])) : J->beta[row];",
+                                "B->b[r] = 1.0 / (1.0 + exp(-J->beta[row]));"),
     "R: output reads k": ("kda_recurrent.c", "acc += S[(size_t)c * Dv + j] * qh[c];",
                           "acc += S[(size_t)c * Dv + j] * kh[c];"),
     "R: eps outside root": ("kda_recurrent.c", "double inv = 1.0 / sqrt(ss + 1e-6);",
@@ -74,6 +78,8 @@ PIN_CALLS = [
     lambda: pins.test_beta_zero_is_half_not_skip("recurrent"),
     lambda: pins.test_forms_agree(65, 16, (4, 3)),
     lambda: pins.test_forms_agree_varlen_and_steep_gates(),
+    lambda: pins.test_beta_probability_matches_logit_form(),
+    lambda: pins.test_beta_probability_special_values(),
 ]
 
 
@@ -126,3 +132,56 @@ def test_unmutated_copy_passes_every_pin(tmp_path, monkeypatch):
     monkeypatch.setattr(oracle, "_lib", lib)
     for call in PIN_CALLS:
         call()
+
+
+# Mistakes planted in the in-kernel gate (numpy side of the oracle): each must
+# fail one of the gate pins.
+def _sig(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def _x(g, dt):
+    return np.asarray(g, float) + (0.0 if dt is None else np.asarray(dt, float))
+
+
+def _rate(a):
+    return np.exp(np.asarray(a, float)).reshape(-1, 1)
+
+
+GATE_MUTANTS = {
+    "dt_bias dropped": lambda g, a, dt=None, lb=None: (
+        -_rate(a) * oracle.softplus(np.asarray(g, float)) if lb is None
+        else lb * _sig(_rate(a) * np.asarray(g, float))),
+    "rate not exponentiated": lambda g, a, dt=None, lb=None: (
+        -np.asarray(a, float).reshape(-1, 1) * oracle.softplus(_x(g, dt)) if lb is None
+        else lb * _sig(np.asarray(a, float).reshape(-1, 1) * _x(g, dt))),
+    "softplus sign": lambda g, a, dt=None, lb=None: (
+        _rate(a) * oracle.softplus(_x(g, dt)) if lb is None else lb * _sig(_rate(a) * _x(g, dt))),
+    "safe rate outside": lambda g, a, dt=None, lb=None: (
+        -_rate(a) * oracle.softplus(_x(g, dt)) if lb is None else _rate(a) * lb * _sig(_x(g, dt))),
+    "safe sigmoid of -x": lambda g, a, dt=None, lb=None: (
+        -_rate(a) * oracle.softplus(_x(g, dt)) if lb is None else lb * _sig(-_rate(a) * _x(g, dt))),
+    "softplus as relu": lambda g, a, dt=None, lb=None: (
+        -_rate(a) * np.maximum(_x(g, dt), 0) if lb is None else lb * _sig(_rate(a) * _x(g, dt))),
+}
+
+GATE_PINS = [
+    lambda: pins.test_gate_printed_example(),
+    lambda: pins.test_gate_closed_forms(),
+    lambda: pins.test_gate_dt_bias_is_per_head_channel(),
+    lambda: pins.test_in_kernel_gate_forms_agree_and_safe_bound_holds(),
+]
+
+
+@pytest.mark.parametrize("name", sorted(GATE_MUTANTS))
+def test_gate_pins_kill_mutant(name, monkeypatch):
+    mut = GATE_MUTANTS[name]
+    monkeypatch.setattr(oracle, "gate", lambda g, a, dt=None, lower_bound=None: mut(g, a, dt, lower_bound))
+    killed = []
+    with np.errstate(all="ignore"):
+        for i, call in enumerate(GATE_PINS):
+            try:
+                call()
+            except AssertionError:
+                killed.append(i)
+    assert killed, f"no gate pin caught the planted mistake '{name}'"

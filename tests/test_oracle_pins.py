@@ -360,3 +360,110 @@ def test_batched_layout_equals_packed():
         on, Sn = oracle.recurrent(q[n], k[n], v[n], g[n], b[n])
         np.testing.assert_allclose(o[n * T:(n + 1) * T], on, atol=1e-14)
         np.testing.assert_allclose(S[n], Sn[0], atol=1e-14)
+
+
+# --- in-kernel gate -----------------------------------------------------------
+
+def test_gate_printed_example():
+    """tests/golden/gate_rs_test.json: the values kda.rs's own gate test fixes."""
+    fx = json.load(open(os.path.join(GOLDEN, "gate_rs_test.json")))
+    z = np.array([fx["z"]]); dt = np.array([fx["dt_bias"]]); a = np.array(fx["A_log"])
+    g = oracle.gate(z, a, dt)[0]
+    sp = lambda x: math.log1p(math.exp(x))  # plain softplus, fine at these arguments
+    assert abs(g[0] - (-sp(0.6))) < 1e-6 and abs(g[1] - (-sp(-0.25))) < 1e-6
+    g5 = oracle.gate(z, a, dt, lower_bound=fx["safe_lower_bound"])[0]
+    assert abs(g5[0] - g[0]) > fx["safe_differs_from_unbounded_by_more_than"]
+
+
+def test_gate_closed_forms():
+    """Safe form: lb * sigmoid(0) = lb / 2 at x = 0, range (lb, 0), monotone in x;
+    unbounded form: -rate * x for large x, -rate * e^x for very negative x, never positive."""
+    a = np.log(np.array([0.5, 2.0]))            # rates 0.5 and 2
+    x = np.zeros((2, 3))
+    np.testing.assert_allclose(oracle.gate(x, a, lower_bound=-5.0), -2.5)
+    xs = np.linspace(-10, 10, 41)[None, :].repeat(2, 0)
+    gs = oracle.gate(xs, a, lower_bound=-5.0)
+    assert np.all(gs < 0) and np.all(gs > -5.0) and np.all(np.diff(gs, axis=1) < 0)
+    ends = oracle.gate(np.array([[-40.0], [40.0]]), np.zeros(2), lower_bound=-5.0)
+    assert -1e-15 < ends[0, 0] <= 0.0 and -5.0 <= ends[1, 0] < -5.0 + 1e-15
+    big = oracle.gate(np.full((2, 1), 50.0), a)
+    np.testing.assert_allclose(big[:, 0], -np.exp(a) * 50.0, rtol=1e-12)
+    tiny = oracle.gate(np.full((2, 1), -40.0), a)
+    np.testing.assert_allclose(tiny[:, 0], -np.exp(a) * math.exp(-40.0), rtol=1e-9)
+    assert np.all(oracle.gate(np.random.default_rng(0).normal(size=(2, 50)) * 10, a) <= 0)
+
+
+def test_gate_dt_bias_is_per_head_channel():
+    a = np.array([0.0, np.log(3.0)])
+    dt = np.array([[0.2, -0.1], [0.0, 0.5]])
+    x = np.zeros((4, 2, 2))
+    g = oracle.gate(x, a, dt)
+    np.testing.assert_allclose(g[1, 0], -oracle.softplus(dt[0]))
+    np.testing.assert_allclose(g[3, 1], -3.0 * oracle.softplus(dt[1]))
+
+
+def test_beta_probability_matches_logit_form():
+    """beta given as a probability p (api.py, use_beta_sigmoid_in_kernel=False) is the
+    same recurrence as the logit log(p / (1 - p)); forms R and C agree on it."""
+    rng = np.random.default_rng(7)
+    T, H, D = 37, 2, 4
+    q, k, v = (rng.normal(size=(T, H, D)) for _ in range(3))
+    g = -np.abs(rng.normal(size=(T, H, D))) * 0.3
+    p = rng.uniform(0.05, 0.95, size=(T, H))
+    o1, s1 = oracle.recurrent(q, k, v, g, p, beta_is_logit=False)
+    o2, s2 = oracle.recurrent(q, k, v, g, np.log(p / (1 - p)))
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(s1, s2, rtol=1e-12, atol=1e-13)
+    o3, s3 = oracle.chunkwise(q, k, v, g, p, beta_is_logit=False, chunk_size=16)
+    np.testing.assert_allclose(o3, o1, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(s3, s1, rtol=1e-10, atol=1e-11)
+
+
+def test_beta_probability_special_values():
+    """p = 0 writes nothing (the state only decays); p = 1 from a zero state with a unit
+    key stores exactly k v^T (the write replaces the key's read-out by v)."""
+    rng = np.random.default_rng(8)
+    H, D = 1, 3
+    q, k, v = (rng.normal(size=(1, H, D)) for _ in range(3))
+    g = np.full((1, H, D), -0.5)
+    S0 = rng.normal(size=(1, H, D, D))
+    _, s = oracle.recurrent(q, k, v, g, np.zeros((1, H)), beta_is_logit=False, initial_state=S0)
+    np.testing.assert_allclose(s, S0 * math.exp(-0.5), rtol=1e-14)
+    kh = k / np.sqrt((k ** 2).sum(-1, keepdims=True) + 1e-6)
+    _, s = oracle.recurrent(q, k, v, np.zeros((1, H, D)), np.ones((1, H)), beta_is_logit=False)
+    np.testing.assert_allclose(s[0, 0], np.outer(kh[0, 0], v[0, 0]), rtol=1e-13)
+
+
+def test_in_kernel_gate_forms_agree_and_safe_bound_holds():
+    """With gate_form the g input is the gate's argument: forms R and C agree, and the
+    safe form keeps every per-token decay above e^lb (state norm shrinks at most by it)."""
+    rng = np.random.default_rng(9)
+    T, H, D = 70, 3, 8
+    q, k, v = (rng.normal(size=(T, H, D)) for _ in range(3))
+    z = rng.normal(size=(T, H, D)) * 2
+    beta = rng.normal(size=(T, H))
+    A_log = rng.uniform(-1, 1, size=H)
+    dt = rng.normal(size=(H, D)) * 0.5
+    for form, lb in (("softplus", None), ("safe", -5.0)):
+        oR, sR = oracle.recurrent(q, k, v, z, beta, gate_form=form, A_log=A_log, dt_bias=dt,
+                                  lower_bound=lb)
+        oC, sC = oracle.chunkwise(q, k, v, z, beta, gate_form=form, A_log=A_log, dt_bias=dt,
+                                  lower_bound=lb, chunk_size=32)
+        np.testing.assert_allclose(oC, oR, rtol=1e-9, atol=1e-10)
+        np.testing.assert_allclose(sC, sR, rtol=1e-9, atol=1e-10)
+    # a single token with zero beta: the state is the decayed initial state, decay = e^gate
+    S0 = rng.normal(size=(1, H, D, D))
+    _, s = oracle.recurrent(q[:1], k[:1], v[:1], z[:1], np.full((1, H), -np.inf),
+                            gate_form="safe", A_log=A_log, dt_bias=dt, lower_bound=-5.0,
+                            initial_state=S0)
+    gg = -5.0 / (1 + np.exp(-np.exp(A_log)[:, None] * (z[0] + dt)))
+    np.testing.assert_allclose(s[0], S0[0] * np.exp(gg)[:, :, None], rtol=1e-12)
+    assert np.all(np.exp(gg) > math.exp(-5.0))
+
+
+def test_gate_form_argument_rules():
+    z = np.zeros((2, 1, 2))
+    with pytest.raises(ValueError):
+        oracle.recurrent(z, z, z, z, np.zeros((2, 1)), gate_form="softplus")   # no A_log
+    with pytest.raises(ValueError):
+        oracle.recurrent(z, z, z, z, np.zeros((2, 1)), gate_form="safe", A_log=[0.0])  # no lb
