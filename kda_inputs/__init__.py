@@ -16,7 +16,8 @@ three geometries plus a tiny fp32 case, and a batched decode step):
 * in-kernel gate cases: the raw gate input z ~ N(0, 1) is passed as g, with
   A_log = log(U(1, 16)) per head and dt_bias = the inverse softplus of
   dt = exp(U(log 1e-3, log 1e-1)) per channel (the initialisation page
-  "Kimi Delta Attention on AMD MI300X" names as FLA's, `draw_gate_params`).
+  "KDA ⇄ FLA Parity in Primus", section "What changed and why" (A), names
+  as FLA's; `draw_gate_params`).
 * beta logits ~ N(0, 1); beta probabilities (cases that pass beta as given)
   ~ U(0, 1).
 * initial states ~ N(0, 1) * 0.1, fp32.
