@@ -67,6 +67,18 @@ def chunk_algorithmic(wl):
     return th * per_th + states, flops
 
 
+def chunk_options(wl, inp):
+    """chunk_kda keyword arguments of a chunk workload: L2 norm in the kernel,
+    its lower bound, chunk size, in-kernel gate and beta form."""
+    kw = dict(use_qk_l2norm_in_kernel=True, lower_bound=wl.lower_bound, chunk_size=wl.chunk_size)
+    if wl.gate_in_kernel:
+        kw.update(use_gate_in_kernel=True, A_log=inp["A_log"], dt_bias=inp["dt_bias"],
+                  safe_gate=wl.lower_bound is not None)
+    if wl.beta_prob:
+        kw["use_beta_sigmoid_in_kernel"] = False
+    return kw
+
+
 def decode_algorithmic(wl):
     """Bytes and flops of one decode step: fp32 state read + write, q/k/g/v/o
     vectors and one beta per head; 7 d_k d_v flops per head."""
@@ -191,15 +203,16 @@ def run_kda(args, rank, world, local_rank):
     q, k, v, g, beta = (inp[n] for n in ("q", "k", "v", "g", "beta"))
     S0, cu = inp["initial_state"], inp["cu_seqlens"]
     o = torch.empty_like(v)
-    S_out = torch.empty(wl.n_seqs, wl.H, wl.Dk, wl.Dv, dtype=torch.float32, device=dev)
+    S_out = torch.empty(wl.n_seqs, wl.H, wl.Dk, wl.Dv, dtype=torch.float32, device=dev) \
+        if wl.final_state else None
+    opts = chunk_options(wl, inp)
     ws_bytes = kda.chunk_workspace_bytes(wl.B, wl.T, wl.H, wl.Dk, wl.Dv, N=wl.n_seqs,
                                          varlen=wl.seqlens is not None)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
 
     def chunk_step():
-        kda.chunk_kda(q, k, v, g, beta, initial_state=S0, output_final_state=True,
-                      use_qk_l2norm_in_kernel=True, lower_bound=wl.lower_bound,
-                      cu_seqlens=cu, out=o, final_state_out=S_out, workspace=ws)
+        kda.chunk_kda(q, k, v, g, beta, initial_state=S0, output_final_state=wl.final_state,
+                      cu_seqlens=cu, out=o, final_state_out=S_out, workspace=ws, **opts)
 
     dwl = KI.DECODE_WORKLOADS[DECODE_WL]
     if args.only != "chunk":
@@ -233,8 +246,16 @@ def run_kda(args, rank, world, local_rank):
             one()
         a1.record(stream)
         torch.cuda.synchronize(dev)
-        return {"only": args.only, "ms_per_launch": a0.elapsed_time(a1) / args.steps,
-                "launches": args.steps}
+        ms = a0.elapsed_time(a1) / args.steps
+        out = {"only": args.only, "ms_per_launch": ms, "launches": args.steps}
+        if args.only == "chunk":
+            nbytes, nflops = chunk_algorithmic(wl)
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            out.update({"workload": wl.name, "tokens_per_s": wl.tokens / (ms * 1e-3),
+                        "algorithmic_bytes_per_launch": nbytes, "achieved_gbs": gbs,
+                        "hbm_frac": gbs / hbm_peak, "peak_kind": peak_kind,
+                        "achieved_tflops": nflops / (ms * 1e-3) / 1e12})
+        return out
 
     # warm-up (untimed)
     for _ in range(args.warmup):
@@ -285,8 +306,7 @@ def run_kda(args, rank, world, local_rank):
         cu_d = cu_host.to(dev, non_blocking=True)
         oo, ss = kda.chunk_kda(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"],
                                initial_state=dbuf["initial_state"], output_final_state=True,
-                               use_qk_l2norm_in_kernel=True, lower_bound=wl.lower_bound,
-                               cu_seqlens=cu_d, workspace=ws)
+                               cu_seqlens=cu_d, workspace=ws, **opts)
         h_o.copy_(oo, non_blocking=True)
         h_S.copy_(ss, non_blocking=True)
 
@@ -309,7 +329,8 @@ def run_kda(args, rank, world, local_rank):
     dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
     tc_used = os.path.exists(os.path.join(ROOT, "kimi_delta_attention_20_b200", "csrc",
                                           "kda_chunk_tc.cu"))
-    chunk_sha = source_sha("kda_chunk_tc.cu", "kda_chunk_simt.cu", "kda_common.cuh") if tc_used else None
+    chunk_sha = source_sha("kda_chunk_tc.cu", "kda_chunk_simt.cu", "kda_common.cuh",
+                           "kda_sm100.cuh") if tc_used else None
     result = {
         "metric": METRIC,
         "value": whole_job_rate(world, wl.tokens, chunk_ms),

@@ -111,7 +111,8 @@ typedef struct {
     int use_qk_l2norm;    /* 1: q,k <- x / sqrt(sum x^2 + 1e-6) in the kernel */
     int has_lower_bound;  /* 1: g <- max(g, lower_bound); lower_bound must be < 0 */
     float lower_bound;
-    int chunk_size;       /* 0 (default) or 64 */
+    int chunk_size;       /* 0 (default, = 64), 32 or 64 tokens per chunk; the result does
+                           * not depend on it (up to rounding). 32 runs on CUDA cores only */
     void *workspace;      /* device scratch of kda_chunk_fwd_workspace_size() bytes */
     size_t workspace_bytes;
     kda_gate_mode gate_mode;   /* KDA_GATE_LOG (0): g is the log-decay */

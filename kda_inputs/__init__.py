@@ -55,6 +55,8 @@ class ChunkWorkload:
     seqlens: Optional[Sequence[int]] = None  # varlen packing (B must be 1)
     scale: Optional[float] = None
     chunk_size: int = 64
+    gate_in_kernel: bool = False   # g holds the gate input; A_log / dt_bias drawn too
+    beta_prob: bool = False        # beta holds probabilities instead of logits
 
     @property
     def tokens(self) -> int:
@@ -89,6 +91,11 @@ CHUNK_WORKLOADS = {
     4: ChunkWorkload("varlen 4096/8192/12288/7168 H96 d128 lb-5", 1, 31744, 96, 128, 128,
                      torch.bfloat16, 4, init_state=True, final_state=True, lower_bound=-5.0,
                      seqlens=(4096, 8192, 12288, 7168)),
+    # one KDA layer of the 300M pure-KDA model in training: micro-batch 128 x 2048 tokens,
+    # 8 heads, d_k 32, d_v 64, in-kernel unbounded gate, beta already a probability
+    5: ChunkWorkload("300M layer B128 T2048 H8 dk32 dv64 gate-in-kernel", 128, 2048, 8, 32, 64,
+                     torch.bfloat16, 5, init_state=False, final_state=False, lower_bound=None,
+                     gate_in_kernel=True, beta_prob=True),
 }
 
 DECODE_WORKLOADS = {
@@ -164,8 +171,13 @@ def draw_gate_params(H, Dk, *, seed=0, device="cpu"):
 def chunk_inputs(idx_or_wl, device="cpu"):
     """Inputs of a named chunk-forward workload (see CHUNK_WORKLOADS)."""
     wl = CHUNK_WORKLOADS[idx_or_wl] if isinstance(idx_or_wl, int) else idx_or_wl
-    return draw_chunk(wl.B, wl.T, wl.H, wl.Dk, wl.Dv, dtype=wl.dtype, seed=wl.seed,
-                      device=device, seqlens=wl.seqlens, init_state=wl.init_state)
+    out = draw_chunk(wl.B, wl.T, wl.H, wl.Dk, wl.Dv, dtype=wl.dtype, seed=wl.seed,
+                     device=device, seqlens=wl.seqlens, init_state=wl.init_state,
+                     gate="input" if wl.gate_in_kernel else "unbounded",
+                     beta="prob" if wl.beta_prob else "logit")
+    if wl.gate_in_kernel:
+        out.update(draw_gate_params(wl.H, wl.Dk, seed=wl.seed, device=device))
+    return out
 
 
 def draw_decode(N, H, Dk, Dv, steps, *, dtype=torch.bfloat16, seed=3, device="cpu",

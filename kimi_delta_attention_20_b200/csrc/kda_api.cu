@@ -8,7 +8,7 @@
 
 namespace kda {
 cudaError_t launch_decode(const StepParams &p, bool bf16, int Dk, int Dv, cudaStream_t st);
-cudaError_t launch_chunk_simt(const ChunkParams &p, bool bf16, int Dk, int Dv, cudaStream_t st);
+cudaError_t launch_chunk_simt(const ChunkParams &p, bool bf16, int Dk, int Dv, int chunk, cudaStream_t st);
 bool chunk_tc_supported(bool bf16, int Dk, int Dv, int chunk_size);
 size_t chunk_tc_workspace_bytes(int N, int H, int Dk, int Dv);
 cudaError_t launch_chunk_tc(const ChunkParams &p, int Dk, int Dv, void *workspace,
@@ -56,7 +56,7 @@ kda_status check_chunk_shape(const kda_chunk_args *a, int *N_out) {
     if (a->dtype != KDA_DTYPE_F32 && a->dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARGUMENT;
     if (a->B < 1 || a->T < 0 || a->H < 1 || a->Dk < 1 || a->Dv < 1) return KDA_ERR_INVALID_ARGUMENT;
     if (!head_dim_ok(a->Dk) || !head_dim_ok(a->Dv)) return KDA_ERR_UNSUPPORTED;
-    if (a->chunk_size != 0 && a->chunk_size != 64) return KDA_ERR_UNSUPPORTED;
+    if (a->chunk_size != 0 && a->chunk_size != 32 && a->chunk_size != 64) return KDA_ERR_UNSUPPORTED;
     if (a->has_lower_bound && !(a->lower_bound < 0.f)) return KDA_ERR_INVALID_ARGUMENT;
     if (check_gate_mode(a->gate_mode, a->has_lower_bound) != KDA_OK) return KDA_ERR_INVALID_ARGUMENT;
     if ((long long)a->B * a->T * a->H * (a->Dk > a->Dv ? a->Dk : a->Dv) >= (1LL << 40))
@@ -154,7 +154,7 @@ kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
         return cuda_status(kda::launch_chunk_tc(p, a->Dk, a->Dv, a->workspace, a->workspace_bytes,
                                                 a->cu_seqlens_host, st));
     }
-    return cuda_status(kda::launch_chunk_simt(p, bf16, a->Dk, a->Dv, st));
+    return cuda_status(kda::launch_chunk_simt(p, bf16, a->Dk, a->Dv, a->chunk_size == 32 ? 32 : 64, st));
 }
 
 kda_status kda_recurrent_step(const kda_step_args *a, void *stream) {

@@ -5,7 +5,8 @@
 // algorithm the tensor-core path follows. One CTA owns one (sequence, head,
 // 64-column slab of d_v) and walks the sequence one chunk of C = 64 tokens
 // at a time, with the state slab S (d_k x 64, fp32) resident in shared
-// memory across chunks. Per chunk, with G the inclusive in-chunk cumsum of
+// memory across chunks (C = 64, or 32 when the caller asks for 32-token
+// chunks). Per chunk, with G the inclusive in-chunk cumsum of
 // the gate (clamped, or formed in the kernel from A_log and dt_bias) and
 // beta = sigmoid(logit) (or a given probability):
 //
@@ -26,9 +27,9 @@
 
 namespace kda {
 
-template <int DK, int DV>
+template <int DK, int DV, int CC>
 struct SimtCfg {
-    static constexpr int C = 64;
+    static constexpr int C = CC;                  // tokens per chunk: 32 or 64
     static constexpr int VS = DV < 64 ? DV : 64;  // state columns per CTA
     static constexpr int kSlabs = DV / VS;
     static constexpr int kThreads = 256;
@@ -40,9 +41,9 @@ struct SimtCfg {
     static constexpr size_t kSmemBytes = sizeof(float) * kFloats;
 };
 
-template <typename Tin, int DK, int DV>
+template <typename Tin, int DK, int DV, int CC>
 __global__ void __launch_bounds__(256, 1) kda_chunk_simt_kernel(ChunkParams p) {
-    using Cfg = SimtCfg<DK, DV>;
+    using Cfg = SimtCfg<DK, DV, CC>;
     constexpr int C = Cfg::C, VS = Cfg::VS, NT = Cfg::kThreads, NW = Cfg::kWarps;
     extern __shared__ float smem[];
     float *qs = smem + Cfg::oQ, *ks = smem + Cfg::oK, *Gs = smem + Cfg::oG;
@@ -210,13 +211,13 @@ __global__ void __launch_bounds__(256, 1) kda_chunk_simt_kernel(ChunkParams p) {
     }
 }
 
-template <typename Tin, int DK, int DV>
+template <typename Tin, int DK, int DV, int CC>
 cudaError_t launch_simt_t(const ChunkParams &p, cudaStream_t st) {
-    using Cfg = SimtCfg<DK, DV>;
+    using Cfg = SimtCfg<DK, DV, CC>;
     const long long blocks = (long long)p.N * p.H * Cfg::kSlabs;
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    auto kern = kda_chunk_simt_kernel<Tin, DK, DV>;
+    auto kern = kda_chunk_simt_kernel<Tin, DK, DV, CC>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -224,10 +225,10 @@ cudaError_t launch_simt_t(const ChunkParams &p, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-template <typename Tin>
+template <typename Tin, int CC>
 cudaError_t launch_simt_dt(const ChunkParams &p, int Dk, int Dv, cudaStream_t st) {
 #define KDA_SIMT_CASE(DK_, DV_) \
-    if (Dk == DK_ && Dv == DV_) return launch_simt_t<Tin, DK_, DV_>(p, st);
+    if (Dk == DK_ && Dv == DV_) return launch_simt_t<Tin, DK_, DV_, CC>(p, st);
     KDA_SIMT_CASE(32, 32) KDA_SIMT_CASE(32, 64) KDA_SIMT_CASE(32, 128)
     KDA_SIMT_CASE(64, 32) KDA_SIMT_CASE(64, 64) KDA_SIMT_CASE(64, 128)
     KDA_SIMT_CASE(128, 32) KDA_SIMT_CASE(128, 64) KDA_SIMT_CASE(128, 128)
@@ -235,8 +236,10 @@ cudaError_t launch_simt_dt(const ChunkParams &p, int Dk, int Dv, cudaStream_t st
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_chunk_simt(const ChunkParams &p, bool bf16, int Dk, int Dv, cudaStream_t st) {
-    return bf16 ? launch_simt_dt<__nv_bfloat16>(p, Dk, Dv, st) : launch_simt_dt<float>(p, Dk, Dv, st);
+cudaError_t launch_chunk_simt(const ChunkParams &p, bool bf16, int Dk, int Dv, int chunk, cudaStream_t st) {
+    if (chunk == 32)
+        return bf16 ? launch_simt_dt<__nv_bfloat16, 32>(p, Dk, Dv, st) : launch_simt_dt<float, 32>(p, Dk, Dv, st);
+    return bf16 ? launch_simt_dt<__nv_bfloat16, 64>(p, Dk, Dv, st) : launch_simt_dt<float, 64>(p, Dk, Dv, st);
 }
 
 }  // namespace kda

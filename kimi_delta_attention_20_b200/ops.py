@@ -91,7 +91,8 @@ def chunk_kda(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
     -exp(A_log) softplus(g + dt_bias), or with safe_gate
     lower_bound * sigmoid(exp(A_log) (g + dt_bias)) (A_log: [H] fp32,
     dt_bias: [H, Dk] fp32 or None; the unbounded form ignores lower_bound).
-    ``cu_seqlens`` (int32, [N+1], B == 1) packs N sequences.
+    ``cu_seqlens`` (int32, [N+1], B == 1) packs N sequences. ``chunk_size``
+    <= 32 selects 32-token chunks (CUDA-core kernel), anything else 64.
     Returns (o [B, T, H, Dv], final_state [N, H, Dk, Dv] fp32 or None).
     """
     lib = _abi.load()
@@ -110,8 +111,9 @@ def chunk_kda(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
             "use_qk_l2norm_in_kernel=False: the chunkwise form relies on unit-norm keys; "
             "unnormalised keys can make the output grow without bound.",
             RuntimeWarning, stacklevel=2)
-    if chunk_size not in (0, 64):
-        raise ValueError("chunk_size must be 64")
+    if not isinstance(chunk_size, int) or chunk_size < 0:
+        raise ValueError("chunk_size must be a non-negative int")
+    chunk_size = 32 if 0 < chunk_size <= 32 else 64  # api.py's 32-or-64 rule
     cu_host = None
     if cu_seqlens is not None:
         if B != 1:

@@ -73,7 +73,7 @@ def step_args(**over):
     (dict(H=0), _abi.KDA_ERR_INVALID_ARGUMENT),
     (dict(Dk=96), _abi.KDA_ERR_UNSUPPORTED),
     (dict(Dv=256), _abi.KDA_ERR_UNSUPPORTED),
-    (dict(chunk_size=32), _abi.KDA_ERR_UNSUPPORTED),
+    (dict(chunk_size=48), _abi.KDA_ERR_UNSUPPORTED),
     (dict(q=None), _abi.KDA_ERR_INVALID_ARGUMENT),
     (dict(o=None), _abi.KDA_ERR_INVALID_ARGUMENT),
     (dict(beta=None), _abi.KDA_ERR_INVALID_ARGUMENT),

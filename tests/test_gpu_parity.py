@@ -87,6 +87,23 @@ def test_workload_varlen_H96():
     assert torch.isfinite(o).all() and torch.isfinite(S).all()
 
 
+def test_workload_300m_layer():
+    """One layer of the 300M pure-KDA model (d_k 32, d_v 64, in-kernel gate, beta as a
+    probability), full size; 6 of the 128 sequences checked on all 8 heads."""
+    wl = KI.CHUNK_WORKLOADS[5]
+    inp = KI.chunk_inputs(wl, device=DEV)
+    kda = kda_mod()
+    o, S = kda.chunk_kda(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                         A_log=inp["A_log"], dt_bias=inp["dt_bias"], use_qk_l2norm_in_kernel=True,
+                         use_gate_in_kernel=True, use_beta_sigmoid_in_kernel=False)
+    assert S is None and torch.isfinite(o).all()
+    sub = {n: inp[n][[0, 17, 63, 64, 100, 127]].cpu() for n in ("q", "k", "v", "g", "beta")}
+    sub["initial_state"] = None
+    compare_chunk(sub, o[[0, 17, 63, 64, 100, 127]], None, wl.dtype, tag="300m",
+                  gate_form="softplus", A_log=inp["A_log"].cpu(), dt_bias=inp["dt_bias"].cpu(),
+                  beta_is_logit=False)
+
+
 def test_workload_decode_256_steps():
     wl = KI.DECODE_WORKLOADS[3]
     kda = kda_mod()
@@ -109,7 +126,7 @@ def test_workload_decode_256_steps():
 
 # --- boundaries, shapes, flags ------------------------------------------------
 
-DIMS = [(32, 32), (64, 64), (128, 128), (32, 128), (128, 64)]
+DIMS = [(32, 32), (64, 64), (128, 128), (32, 64), (32, 128), (128, 64)]
 
 
 @pytest.mark.parametrize("T", [1, 7, 63, 64, 65, 130])
@@ -120,6 +137,29 @@ def test_chunk_boundary_lengths(T, dtype, dims):
     inp = KI.draw_chunk(2, T, 3, Dk, Dv, dtype=dtype, seed=T * 31 + Dk + Dv, init_state=True)
     o, S = run_chunk(inp)
     compare_chunk(inp, o, S, dtype, tag=f"T{T}")
+
+
+@pytest.mark.parametrize("T", [1, 31, 32, 33, 100])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dims", [(32, 64), (64, 32), (128, 128)])
+def test_chunk_size_32(T, dtype, dims):
+    """32-token chunks (api.py's chunk_size 32) give the same operator result."""
+    Dk, Dv = dims
+    inp = KI.draw_chunk(2, T, 3, Dk, Dv, dtype=dtype, seed=T * 17 + Dk, init_state=True)
+    o, S = run_chunk(inp, chunk_size=32, lower_bound=-5.0)
+    compare_chunk(inp, o, S, dtype, lower_bound=-5.0, tag=f"C32 T{T}")
+
+
+def test_chunk_size_rule():
+    """chunk sizes <= 32 select 32-token chunks, larger ones 64 (api.py's rule); both
+    agree with each other to rounding on the same input."""
+    inp = KI.draw_chunk(1, 150, 2, 32, 64, dtype=torch.float32, seed=77, init_state=True)
+    o16, S16 = run_chunk(inp, chunk_size=16)
+    o32, S32 = run_chunk(inp, chunk_size=32)
+    o64, S64 = run_chunk(inp, chunk_size=100)
+    assert torch.equal(o16, o32) and torch.equal(S16, S32)
+    torch.testing.assert_close(o32, o64, rtol=1e-5, atol=1e-5)
+    torch.testing.assert_close(S32, S64, rtol=1e-5, atol=1e-5)
 
 
 @pytest.mark.parametrize("lb", [None, -5.0, -0.5])
