@@ -113,7 +113,7 @@ typedef struct {
     float lower_bound;
     int chunk_size;       /* 0 (default, = 64), 32 or 64 tokens per chunk; the result does
                            * not depend on it (up to rounding). 32 runs on CUDA cores only */
-    void *workspace;      /* device scratch of kda_chunk_fwd_workspace_size() bytes */
+    void *workspace;      /* device scratch, 256-byte aligned; see kda_chunk_fwd_workspace_size */
     size_t workspace_bytes;
     kda_gate_mode gate_mode;   /* KDA_GATE_LOG (0): g is the log-decay */
     const float *A_log;        /* [H] fp32, in-kernel gate forms only */
@@ -121,8 +121,13 @@ typedef struct {
     int beta_is_prob;          /* 1: beta is used as given (no sigmoid) */
 } kda_chunk_args;
 
-/* Bytes of device workspace kda_chunk_fwd needs for these arguments (may be
- * 0). Only shapes, dtype and flags are read; pointers may be NULL. */
+/* Bytes of device workspace with which kda_chunk_fwd runs its fastest kernel
+ * for these arguments (may be 0). Only shapes, dtype and flags are read;
+ * pointers may be NULL. For bf16 with d_k = d_v = 128 this is the two-pass
+ * tensor-core kernel, whose workspace holds one 65 KiB record per (chunk, head)
+ * (about 1.04 bytes per input byte of q, k, g and v); a smaller workspace of at
+ * least 256 bytes runs the single-pass tensor-core kernel instead (same result
+ * up to rounding), and less than that returns KDA_ERR_WORKSPACE. */
 KDA_API kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args *args, size_t *bytes);
 
 /* Queue the chunkwise forward on `stream`. Returns KDA_OK once queued. */

@@ -13,6 +13,8 @@ bool chunk_tc_supported(bool bf16, int Dk, int Dv, int chunk_size);
 size_t chunk_tc_workspace_bytes(int N, int H, int Dk, int Dv);
 cudaError_t launch_chunk_tc(const ChunkParams &p, int Dk, int Dv, void *workspace,
                             size_t workspace_bytes, const int32_t *cu_host, cudaStream_t st);
+size_t chunk_2pass_workspace_bytes(const ChunkParams &p);
+cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int32_t *cu_host, cudaStream_t st);
 }  // namespace kda
 
 namespace {
@@ -79,6 +81,21 @@ namespace kda {
 void record_cuda_error(int e) { g_last_cuda_error = e; }
 }  // namespace kda
 
+namespace kda {
+// Smallest workspace kda_chunk_fwd accepts for these arguments (the single-pass
+// tensor-core kernel's status word, or 0 where no kernel needs scratch).
+kda_status chunk_workspace_min_bytes(const kda_chunk_args *a, size_t *bytes) {
+    int N = 0;
+    kda_status s = check_chunk_shape(a, &N);
+    if (s != KDA_OK) return s;
+    *bytes = 0;
+    if (chunk_tc_supported(a->dtype == KDA_DTYPE_BF16, a->Dk, a->Dv, a->chunk_size) &&
+        (long long)a->B * a->T > 0)
+        *bytes = chunk_tc_workspace_bytes(N, a->H, a->Dk, a->Dv);
+    return KDA_OK;
+}
+}  // namespace kda
+
 extern "C" {
 
 const char *kda_status_string(kda_status s) {
@@ -103,10 +120,16 @@ kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args *a, size_t *bytes) 
     kda_status s = check_chunk_shape(a, &N);
     if (s != KDA_OK) return s;
     *bytes = 0;
-    if (kda::chunk_tc_supported(a->dtype == KDA_DTYPE_BF16, a->Dk, a->Dv, a->chunk_size))
-        *bytes = kda::chunk_tc_workspace_bytes(N, a->H, a->Dk, a->Dv);
+    if (kda::chunk_tc_supported(a->dtype == KDA_DTYPE_BF16, a->Dk, a->Dv, a->chunk_size) &&
+        (long long)a->B * a->T > 0) {
+        kda::ChunkParams p{};
+        p.cu_seqlens = a->cu_seqlens;  // only its presence is read
+        p.T = a->T; p.N = N; p.H = a->H;
+        *bytes = kda::chunk_2pass_workspace_bytes(p);
+    }
     return KDA_OK;
 }
+
 
 kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
     int N = 0;
@@ -148,6 +171,10 @@ kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     if (ntok > 0 && kda::chunk_tc_supported(bf16, a->Dk, a->Dv, a->chunk_size)) {
+        // two passes when the workspace holds the per-chunk records, else the single-pass kernel
+        if (a->workspace && aligned(a->workspace, 256) &&
+            a->workspace_bytes >= kda::chunk_2pass_workspace_bytes(p))
+            return cuda_status(kda::launch_chunk_2pass(p, a->workspace, a->cu_seqlens_host, st));
         const size_t need = kda::chunk_tc_workspace_bytes(N, a->H, a->Dk, a->Dv);
         if (need > 0 && (!a->workspace || a->workspace_bytes < need || !aligned(a->workspace, 256)))
             return KDA_ERR_WORKSPACE;

@@ -34,6 +34,8 @@ void *g_scratch_addr[kMaxDevices] = {};
 
 namespace kda {
 void record_cuda_error(int e);  // kda_api.cu: value returned by kda_last_cuda_error()
+// kda_api.cu: the smallest workspace kda_chunk_fwd accepts for these arguments
+kda_status chunk_workspace_min_bytes(const kda_chunk_args *a, size_t *bytes);
 }  // namespace kda
 
 extern "C" {
@@ -41,7 +43,9 @@ extern "C" {
 KDA_API kda_status kda_chunk_fwd_noalloc(const kda_chunk_args *args, void *stream) {
     if (!args) return KDA_ERR_INVALID_ARGUMENT;
     size_t need = 0;
-    kda_status s = kda_chunk_fwd_workspace_size(args, &need);
+    // the smallest workspace the forward accepts: with it, kda_chunk_fwd runs the
+    // single-pass kernel, which keeps only a status word in scratch
+    kda_status s = kda::chunk_workspace_min_bytes(args, &need);
     if (s != KDA_OK) return s;
     if (need > kScratchBytes) return KDA_ERR_WORKSPACE;  // beyond the fixed scratch size
 

@@ -151,10 +151,14 @@ def chunk_kda(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
     _abi.check(lib.kda_chunk_fwd_workspace_size(ctypes.byref(a), ctypes.byref(nbytes)),
                "kda_chunk_fwd_workspace_size")
     if nbytes.value:
-        if workspace is None or workspace.numel() * workspace.element_size() < nbytes.value:
+        # a caller's workspace is passed as is: the library runs the fastest kernel it
+        # allows (the per-chunk records of the two-pass kernel need the full size, the
+        # single-pass kernel 256 bytes) and rejects one too small for any
+        if workspace is None:
             workspace = torch.empty(nbytes.value, dtype=torch.uint8, device=q.device)
+        _need_cuda("workspace", workspace)
         a.workspace = _ptr(workspace)
-        a.workspace_bytes = nbytes.value
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
     with torch.cuda.device(q.device):
         _abi.check(lib.kda_chunk_fwd(ctypes.byref(a), _stream(q.device)), "kda_chunk_fwd")
     return o, fs

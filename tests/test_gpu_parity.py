@@ -314,3 +314,38 @@ def test_chunk_status_word_is_cleared():
     run_chunk(inp, workspace=ws)
     torch.cuda.synchronize()
     assert int(ws[:4].view(torch.int32).item()) == 0
+
+
+# --- the single-pass tensor-core kernel ----------------------------------------
+# kda_chunk_fwd runs the two-pass kernel when the workspace holds its per-chunk
+# records and the single-pass kernel when only the 256-byte minimum is given;
+# both must match the oracle on their own.
+
+@pytest.mark.parametrize("lens", [(1,), (63,), (64,), (65,), (130,), (0, 1, 64, 65, 130, 7, 0, 200)])
+def test_single_pass_kernel_lengths(lens):
+    inp = KI.draw_chunk(1, sum(lens), 3, 128, 128, dtype=torch.bfloat16, seed=40 + sum(lens),
+                        seqlens=lens, init_state=True)
+    ws = torch.empty(256, dtype=torch.uint8, device=DEV)
+    o, S = run_chunk(inp, lower_bound=-5.0, workspace=ws)
+    compare_chunk(inp, o, S, torch.bfloat16, lower_bound=-5.0, tag=f"1pass {lens}")
+
+
+def test_single_pass_kernel_steep_gates_and_gate_forms():
+    inp = KI.draw_chunk(1, 200, 2, 128, 128, dtype=torch.bfloat16, seed=41, init_state=True)
+    g = inp["g"].float()
+    g[:, 64:128] = -9.0
+    inp["g"] = g.to(torch.bfloat16)
+    ws = torch.empty(256, dtype=torch.uint8, device=DEV)
+    o, S = run_chunk(inp, lower_bound=-10.0, workspace=ws)
+    compare_chunk(inp, o, S, torch.bfloat16, lower_bound=-10.0, tag="1pass steep")
+
+
+def test_two_pass_and_single_pass_agree():
+    """Both tensor-core kernels on one input: equal up to bf16 output rounding."""
+    inp = KI.draw_chunk(1, 1000, 4, 128, 128, dtype=torch.bfloat16, seed=42,
+                        seqlens=(300, 1, 699), init_state=True)
+    o2, S2 = run_chunk(inp, lower_bound=-5.0)
+    ws = torch.empty(256, dtype=torch.uint8, device=DEV)
+    o1, S1 = run_chunk(inp, lower_bound=-5.0, workspace=ws)
+    check("2pass vs 1pass o", o2, o1.double().cpu().numpy(), torch.bfloat16)
+    check("2pass vs 1pass S", S2, S1.double().cpu().numpy(), torch.bfloat16)
