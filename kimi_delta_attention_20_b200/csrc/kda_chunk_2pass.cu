@@ -11,24 +11,29 @@
 // and only four products carry the state from chunk to chunk:
 //   D = T'V - W S,  O = Qtil S + A_qk D,  S <- diag(e^{G_last}) S + Khat^T D.
 //
-// Pass 1 (`kda_tp_intra_kernel`) computes the chunk-local part for every
-// (chunk, head) at once -- all chunks of all sequences are independent, so the
-// pass runs two 256-thread CTAs per SM over a flat list of work items -- and
-// writes one record per (chunk, head) to the workspace: W^T, Qtil, Khat, T' and
-// A_qk as bf16 tiles already laid out as the 128-byte-swizzled shared-memory
-// images the tensor cores read, plus e^{G_last} and the row norms.
+// Pass 1 (`kda_tp_intra_kernel`) computes the chunk-local part of every
+// (chunk, head) at once -- all chunks of all sequences are independent -- with
+// two 256-thread CTAs per SM walking a flat list of work items, and writes one
+// record per (chunk, head): W^T, Qtil^T, Khat^T, T' and A_qk as bf16 tiles
+// already laid out as the 128-byte-swizzled shared-memory images the tensor
+// cores read, plus e^{G_last} and the row norms. Its layout is by key channel:
+// three tensor-core products against constant tiles put the in-chunk cumsum
+// G^T = g^T Tri^T and the transposes k^T, q^T into tensor memory (lane = key
+// channel), so each thread holds one channel for a run of rows, takes its block
+// references from its own registers and writes every operand tile as whole
+// 128-byte rows; the tiles go to the record with bulk copies.
 // Pass 2 (`kda_tp_state_kernel`) walks each (sequence, head) through its
 // chunks with the fp32 state S^T resident in tensor memory; per chunk it
-// bulk-copies the record (one untiled copy) and the v tile (TMA) into a
-// double-buffered stage and issues the four state products, so the sequential
-// part of the work is short.
+// bulk-copies the record and the v tile (TMA) into a double-buffered stage and
+// issues the four state products, so the sequential part of the work is short.
 //
-// Normalisation of q and k is deferred exactly as in the single-pass kernel:
-// the products use raw rows, and 1/|k_s| scales the columns of D, 1/|q_r| the
-// output rows, beta/|k_s| the columns of the W factor (all algebraically
-// identical to normalising first). The in-chunk factorisation of the gated
-// products uses 32-row blocks with middle references; a chunk whose gate span
-// exceeds kSpanMax in some channel computes A_kk and A_qk exactly on CUDA cores.
+// Normalisation of q and k is deferred: the products use raw rows, and 1/|k_s|
+// scales the columns of D, 1/|q_r| the output rows, beta/|k_s| the columns of
+// the W factor (all algebraically identical to normalising first). The gated
+// products use 32-row blocks with middle references (factors up to e^{span});
+// a chunk whose gate moves by more than kSpanMax inside a block is queued and
+// its record is rewritten by `kda_tp_exact_kernel`, which computes every
+// product on CUDA cores from exponent differences alone (any gate).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -51,9 +56,10 @@ constexpr float kSpanMax = 80.f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 
 // ---- record of one (chunk, head), bytes; every tile is a shared-memory image
-constexpr uint32_t R_WT = 0;        // W^T   [128 c][64 r], MN-major B operand (128 rows per half)
-constexpr uint32_t R_QT = 16384;    // Qtil  [64 r][128 c] as two 64-column halves, K-major B
-constexpr uint32_t R_KH = 32768;    // Khat  [64 s][128 c] as two halves, MN-major B
+// with the 128-byte swizzle (16-byte chunk index XOR row % 8, rows of 128 B)
+constexpr uint32_t R_WT = 0;        // W^T    [128 c][64 r]: B of S^T W^T, N = r contiguous (MN-major)
+constexpr uint32_t R_QT = 16384;    // Qtil^T [128 c][64 r]: B of S^T Qtil^T, MN-major
+constexpr uint32_t R_KH = 32768;    // Khat^T [128 c][64 s]: B of D~^T Khat, K = s contiguous (K-major)
 constexpr uint32_t R_TPU = 49152;   // T' = T diag(beta) [64 r][64 s], K-major B
 constexpr uint32_t R_AQK = 57344;   // A_qk (raw rows) [64 r][64 s], K-major B
 constexpr uint32_t R_MISC = 65536;  // f32: e^{G_last}[128], 1/|q_r|[64], 1/|k_s|[64]
@@ -63,87 +69,89 @@ static_assert(REC_BYTES % 1024 == 0, "records stay 1024-byte aligned");
 
 // ============================================================== pass 1
 constexpr int NT1 = 256;  // 8 warps, two CTAs per SM
-// shared memory, view 1 (inputs and the operands of the A_kk / A_qk products)
-constexpr uint32_t STG_Q = 0, STG_K = 16384, STG_G = 32768;      // TMA staging, [64][128] bf16
-constexpr uint32_t XKQD = 49152;                                  // 2 halves x [128 rows][128 B]
-constexpr uint32_t YD_H0 = 81920, YD_H1 = 90112, YO_H0 = 98304, YO_H1 = 102400;
-constexpr uint32_t NRM = 106496;                                  // [q|k][8 warps][64 rows] f32
-// view 2 (after the products): fp32 L and T, the T' tiles and the A_qk tile
+// Shared memory (bytes from a 1024-aligned base). Phases reuse regions:
+//   inputs      KQ: 2 channel halves x [128 rows: k tokens 0..63, q tokens 0..63][128 B]
+//               GS: 2 channel halves x [64 tokens][128 B] (the gate)
+//               TRI, IDT: [64][64] bf16 constant tiles; GLO: low part of a split gate
+//   operands    XK, XQ: X^T images [128 c][64 r] of k e^{G-G_m}, q e^{G-G_m}
+//               YT: Y^T [128 c][64 s] of k e^{G_m-G};  YP: Y'^T of k e^{G_47-G} (s < 32)
+//               QT, KH: the record's Qtil^T and Khat^T images
+//   inverse     LF: fp32 L [64][65];  TF: fp32 T [64][68];  TW: bf16 T diag(beta/|k|)
+//               AQK, TPU: the record's A_qk and T' images;  WT: the record's W^T image
+constexpr uint32_t KQ = 0, GS = 32768;
+constexpr uint32_t XK = 0, XQ = 16384, YT = 32768;
+constexpr uint32_t R2 = 49152;
+constexpr uint32_t TRI = R2, IDT = R2 + 8192, GLO = R2 + 16384;
+constexpr uint32_t QT = R2, KH = R2 + 16384, YP = R2 + 32768;
 constexpr int LDS = 65, LDT = 68;
-constexpr uint32_t TF = 0, TPU = 24576, TPW = 32768;              // in the dead staging area
-constexpr uint32_t AQK = XKQD + 8192;                             // the dead q rows of half 0
-constexpr uint32_t LF = YD_H0;                                    // the dead Y tiles
-constexpr uint32_t MISC1 = 110592;
-constexpr uint32_t M1_BETA = MISC1, M1_INVQ = MISC1 + 256, M1_INVK = MISC1 + 512,
-                   M1_G = MISC1 + 768,      // [3][128] f32: G_15, G_47, G_63 per channel
-                   M1_DTB = MISC1 + 2304,   // [128] f32: dt_bias of the item's head
-                   M1_BAR = MISC1 + 2816, M1_TMEM = MISC1 + 2848;
-constexpr uint32_t SMEM1_BYTES = MISC1 + 2864;
+constexpr uint32_t LF = 16384, TF = 33792, TW = 51200;
+constexpr uint32_t AQK = YP, TPU = YP + 8192, WT = KH;
+constexpr uint32_t MISC1 = 98304;
+constexpr uint32_t M1_REC = MISC1,           // record misc image: gamma[128], invq[64], invk[64]
+    M1_GAM = MISC1, M1_INVQ = MISC1 + 512, M1_INVK = MISC1 + 768,
+                   M1_BETA = MISC1 + 1024,   // [64] f32
+                   M1_GX = MISC1 + 1280,     // [128] f32: gate totals of rows 0..31 (gate forms)
+                   M1_DTB = MISC1 + 1792,    // [128] f32: dt_bias of the item's head
+                   M1_BAR = MISC1 + 2304, M1_TMEM = MISC1 + 2336;
+constexpr uint32_t SMEM1_BYTES = MISC1 + 2368;
 constexpr uint32_t SMEM1_ALLOC = SMEM1_BYTES + 1024;
-static_assert(TF + 64 * LDT * 4 <= TPU && TPW + 8192 <= XKQD, "view 2 in the staging area");
-static_assert(LF + 64 * LDS * 4 <= NRM && AQK + 8192 <= XKQD + 16384, "view 2 in the operand area");
+static_assert(LF + 64 * LDS * 4 <= TF && TF + 64 * LDT * 4 <= TW && TW + 8192 <= KH, "inverse scratch");
+static_assert(TW % 1024 == 0 && AQK % 1024 == 0 && TPU % 1024 == 0 && TPU + 8192 == MISC1, "tile alignment");
 static_assert(2 * (SMEM1_ALLOC + 1024) <= 233472, "two CTAs per SM");
 
-// tensor memory: A products (D1 cols 0..63, D2 cols 64..95), W halves
-constexpr uint32_t TM1_A = 0, TM1_W = 128, TM1_W1 = 192, TM1_COLS = 256;
+// tensor memory (256 columns): G^T, k^T, q^T; then the A products; then W in two K halves
+constexpr uint32_t TM_G = 0, TM_K = 64, TM_Q = 128;
+constexpr uint32_t TM_A1 = 0, TM_A2 = 64, TM_W0 = 128, TM_W1 = 192, TM1_COLS = 256;
 
-constexpr uint32_t ID_A1 = idesc_bf16(128, 64, false, false);
-constexpr uint32_t ID_A2 = idesc_bf16(128, 32, false, false);
-constexpr uint32_t ID_UW = idesc_bf16(128, 64, true, false);
-constexpr uint32_t ID_DL = idesc_bf16(128, 64, false, true, /*neg_b=*/true);
-constexpr uint32_t ID_O = idesc_bf16(128, 64, false, false);
-constexpr uint32_t ID_S = idesc_bf16(128, 128, false, true);
+constexpr uint32_t ID_T = idesc_bf16(128, 64, true, false);   // g^T Tri^T, k^T I, q^T I
+constexpr uint32_t ID_A = idesc_bf16(128, 64, true, true);    // [X_k; X_q] Y^T and Y'^T
+constexpr uint32_t ID_W = idesc_bf16(128, 64, false, false);  // X_k^T T_w^T
 
 struct IntraParams {
     CUtensorMap tq, tk, tg;
     ChunkParams p;
-    uint8_t *rec;           // records, index (global chunk) * H + head
-    const int *chunk_off;   // varlen: [N+1] first global chunk of each sequence
-    int cpr;                // batch: chunks per batch row
-    long long n_items;      // upper bound of (global chunk, head) items
+    uint8_t *rec;            // records, index (global chunk) * H + head
+    const int2 *chunk_tok;   // varlen: per global chunk (first token, valid rows)
+    const int *n_chunks;     // varlen: device count of global chunks
+    int cpr;                 // batch: chunks per batch row
+    long long n_items;       // upper bound of (global chunk, head) items
+    int split_gate;          // the clamped gate needs a low bf16 part (bound not a bf16 value)
+    int *fix_count;          // items whose gate span needs the exact kernel
+    int *fix_list;
     int *status;
 };
 
 struct Item {
     int h;
-    long long t0;  // first token of the chunk
+    int t0;        // first token of the chunk
     int L;         // valid rows
     long long gc;  // global chunk index
 };
 
 // (global chunk, head) of flat item index `item` -> the chunk's tokens; false past the end
-__device__ __forceinline__ bool decode_item(const IntraParams &P, long long item, Item &it) {
+__device__ __forceinline__ bool decode_item(const IntraParams &P, long long item, int nch, Item &it) {
     const ChunkParams &p = P.p;
     if (item >= P.n_items) return false;
     const long long gc = item / p.H;
     it.h = (int)(item % p.H);
     it.gc = gc;
-    long long bos, eos, ci;
-    if (P.chunk_off) {
-        if (gc >= P.chunk_off[p.N]) return false;
-        int lo = 0, hi = p.N - 1;  // last n with chunk_off[n] <= gc
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (P.chunk_off[mid] <= gc) lo = mid; else hi = mid - 1;
-        }
-        bos = p.cu_seqlens[lo];
-        eos = p.cu_seqlens[lo + 1];
-        ci = gc - P.chunk_off[lo];
+    if (P.chunk_tok) {
+        if (gc >= nch) return false;
+        const int2 e = P.chunk_tok[gc];
+        it.t0 = e.x;
+        it.L = e.y;
     } else {
         const long long n = gc / P.cpr;
         if (n >= p.N) return false;
-        ci = gc % P.cpr;
-        bos = n * p.T;
-        eos = bos + p.T;
+        const int ci = (int)(gc % P.cpr);
+        it.t0 = (int)(n * p.T) + ci * C;
+        it.L = min(C, p.T - ci * C);
     }
-    it.t0 = bos + ci * C;
-    it.L = (int)((eos - it.t0) < C ? (eos - it.t0) : C);
     return it.L > 0;
 }
 
-__device__ __forceinline__ void stg128(uint8_t *base, uint32_t off, const uint4 &v) {
-    *reinterpret_cast<uint4 *>(base + off) = v;
-}
+// 8 bf16 of an unpacked register pair set -> one 16-byte chunk
+__device__ __forceinline__ uint4 pack16B(const float2 (&f)[4]) { return pack8x2(f); }
 
 __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_constant__ IntraParams P) {
     extern __shared__ uint8_t smem_raw[];
@@ -152,6 +160,7 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = p.H;
     constexpr int kMma = 0, kTma = NT1 - 32;
+    constexpr float kL2e = 1.4426950408889634f;
 
     uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + M1_BAR);
     uint64_t *bar_mma = bar_in + 1;
@@ -159,7 +168,8 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
     float *sbeta = reinterpret_cast<float *>(sm + M1_BETA);
     float *sinvq = reinterpret_cast<float *>(sm + M1_INVQ);
     float *sinvk = reinterpret_cast<float *>(sm + M1_INVK);
-    float *sG = reinterpret_cast<float *>(sm + M1_G);
+    float *sgam = reinterpret_cast<float *>(sm + M1_GAM);
+    float *sGX = reinterpret_cast<float *>(sm + M1_GX);
     float *sDtb = reinterpret_cast<float *>(sm + M1_DTB);
     float *Lf = reinterpret_cast<float *>(sm + LF);
     float *Tf = reinterpret_cast<float *>(sm + TF);
@@ -175,17 +185,17 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
     tc_fence_after();
     const uint32_t tb = *s_tmem;
     const uint32_t sb = smem_u32(sm);
-    const uint64_t dK = sdesc_sw128(sb, 16, 1024);     // K-major operands
-    const uint64_t dX = sdesc_sw128(sb, 16384, 1024);  // MN-major view of XKQD (halves 16 KiB apart)
-    auto dk = [&](uint32_t off) { return dK + (uint64_t)(off >> 4); };
-    auto dx = [&](uint32_t off) { return dX + (uint64_t)(off >> 4); };
-    const int quarter = warp & 3;                      // TMEM lanes 32*quarter .. +31
+    // 128-byte-swizzled operand at `off`: K-major (lbo unused) or MN-major (lbo = step
+    // between 64-element groups along M/N); 8-row groups 1024 bytes apart
+    auto desc = [&](uint32_t off, uint32_t lbo) { return sdesc_sw128(sb + off, lbo, 1024); };
+    // channel layout: thread (quarter, hw) owns key channel c (tensor-memory lane c)
+    // and rows 32 hw .. 32 hw + 31; hw also splits columns in the row-layout phases
+    const int quarter = warp & 3, hw = warp >> 2;
+    const int c = 32 * quarter + lane;
     const uint32_t lane_sel = (uint32_t)(32 * quarter) << 16;
-    const int cgrp = warp >> 2;                        // 0..1
-    const int row0 = 2 * lane;                         // row-layout phases: rows 2l, 2l+1
-    const int blk = lane >> 4;                         // their 32-row block
     const int gmode = p.gate_mode;
     const __nv_bfloat16 *bt = static_cast<const __nv_bfloat16 *>(p.beta);
+    const int nch = P.chunk_tok ? *P.n_chunks : 0;
 
     uint32_t ph_in = 0, ph_mma = 0;
     bool in_out = false, mma_out = false, aborted = false;
@@ -198,318 +208,307 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
     auto issue_in = [&](const Item &it) {
         mbar_arrive_expect_tx(bar_in, 3 * 16384);
         for (int hf = 0; hf < 2; ++hf) {
-            tma_load_3d(sm + STG_Q + hf * 8192, &P.tq, bar_in, hf * 64, it.h, (int)it.t0);
-            tma_load_3d(sm + STG_K + hf * 8192, &P.tk, bar_in, hf * 64, it.h, (int)it.t0);
-            tma_load_3d(sm + STG_G + hf * 8192, &P.tg, bar_in, hf * 64, it.h, (int)it.t0);
+            tma_load_3d(sm + KQ + hf * 16384, &P.tk, bar_in, hf * 64, it.h, it.t0);
+            tma_load_3d(sm + KQ + hf * 16384 + 8192, &P.tq, bar_in, hf * 64, it.h, it.t0);
+            tma_load_3d(sm + GS + hf * 8192, &P.tg, bar_in, hf * 64, it.h, it.t0);
         }
     };
 
     long long item = blockIdx.x;
     Item cur;
-    bool have = decode_item(P, item, cur);
+    bool have = decode_item(P, item, nch, cur);
     if (have && tid == kTma) { issue_in(cur); in_out = true; }
 
     while (have) {
         const long long nitem = item + gridDim.x;
         Item nxt;
-        const bool have_next = decode_item(P, nitem, nxt);
-        const int h = cur.h, L = cur.L;
-        const long long t0 = cur.t0;
+        const bool have_next = decode_item(P, nitem, nch, nxt);
+        const int h = cur.h, L = cur.L, t0 = cur.t0;
         uint8_t *rec = P.rec + (cur.gc * H + h) * (long long)REC_BYTES;
 
-        // ---------------- per-item scalars: beta, gate parameters
+        // ---------------- per-item scalars and the constant tiles Tri (s <= r) and I
         if (tid < C) {
-            const float b = tid < L ? __bfloat162float(bt[(t0 + tid) * H + h]) : 0.f;
+            const float b = tid < L ? __bfloat162float(bt[((long long)t0 + tid) * H + h]) : 0.f;
             sbeta[tid] = tid < L ? beta_value(b, p.beta_prob) : 0.f;
         }
         const float rate = gmode != kGateLog ? expf(p.A_log[h]) : 0.f;
         if (gmode != kGateLog && tid < D) sDtb[tid] = p.dt_bias ? p.dt_bias[h * D + tid] : 0.f;
+        // the previous item's record stores must have read their sources (GLO, misc)
+        if (tid == kTma) bulk_wait_read_all();
+        for (int e = tid; e < 2 * 64 * 8; e += NT1) {
+            const int tile = e >> 9, r = (e >> 3) & 63, j = e & 7;
+            float v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int s = 8 * j + q;
+                v[q] = tile ? (s == r ? 1.f : 0.f) : (s <= r ? 1.f : 0.f);
+            }
+            sts128(sm, (tile ? IDT : TRI) + sw128_chunk(r, 8 * j, 64), pack8(v));
+        }
         if (wait_all(bar_in, ph_in)) { aborted = true; break; }
         if (tid == kTma) in_out = false;
 
-        // ---------------- P1: gate (clamp or in-kernel form) and its in-chunk cumsum;
-        // warp w owns the 8-channel chunks 2w and 2w+1 for all 64 rows, lane l rows 2l, 2l+1
-        float G[2][2][8];
-        bool span_bad = false;
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-            const int jch = 2 * warp + jj;
-            float2 tt[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) tt[e] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int r = row0 + u;
-                float2 gg[4];
-                unpack8x2(lds128(sm + STG_G, sw128_chunk(r, 8 * jch, 64)), gg);
-                if (gmode != kGateLog) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 b = *reinterpret_cast<const float2 *>(sDtb + 8 * jch + 2 * e);
-                        gg[e] = make_float2(gate_fast(gg[e].x, b.x, rate, gmode, p.lb),
-                                            gate_fast(gg[e].y, b.y, rate, gmode, p.lb));
-                    }
-                } else if (p.has_lb) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) gg[e] = make_float2(fmaxf(gg[e].x, p.lb), fmaxf(gg[e].y, p.lb));
+        // ---------------- rows past the sequence end: zero k, q and the gate input
+        if (L < C) {
+            for (int e = tid; e < 3072; e += NT1) {
+                uint32_t off;
+                int tok;
+                if (e < 2048) {
+                    const int row = (e >> 3) & 127;
+                    tok = row & 63;
+                    off = KQ + (e >> 10) * 16384 + row * 128 + (e & 7) * 16;
+                } else {
+                    const int e2 = e - 2048, row = (e2 >> 3) & 63;
+                    tok = row;
+                    off = GS + (e2 >> 9) * 8192 + row * 128 + (e2 & 7) * 16;
                 }
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 gv = r < L ? gg[e] : make_float2(0.f, 0.f);
-                    tt[e] = __fadd2_rn(tt[e], gv);
-                    G[jj][u][2 * e] = tt[e].x;
-                    G[jj][u][2 * e + 1] = tt[e].y;
-                }
+                if (tok >= L) sts128(sm, off, make_uint4(0u, 0u, 0u, 0u));
             }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float tot = (e & 1) ? tt[e >> 1].y : tt[e >> 1].x;
-                float inc = tot;
-#pragma unroll
-                for (int d = 1; d < 32; d <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, inc, d);
-                    if (lane >= d) inc += y;
-                }
-                G[jj][0][e] += inc - tot;
-                G[jj][1][e] += inc - tot;
-                const float g15 = __shfl_sync(0xffffffffu, inc, 7);
-                const float g47 = __shfl_sync(0xffffffffu, inc, 23);
-                const float g63 = __shfl_sync(0xffffffffu, inc, 31);
-                const float gm = blk ? g47 : g15;
-                span_bad |= fabsf(G[jj][0][e] - gm) > kSpanMax;
-                span_bad |= fabsf(G[jj][1][e] - gm) > kSpanMax;
-                if (lane == e) {
-                    sG[8 * jch + e] = g15;
-                    sG[128 + 8 * jch + e] = g47;
-                    sG[256 + 8 * jch + e] = g63;
-                }
-            }
+            __syncthreads();
         }
-        const bool fb = __syncthreads_or(span_bad) != 0;
 
-        // ---------------- P2: bf16 operand tiles (shared memory) and Qtil, Khat (record)
-        {
-            constexpr float kLog2e = 1.4426950408889634f;
-            float2 nrm_q = make_float2(0.f, 0.f), nrm_k = nrm_q;  // partial squared norms, rows row0 + u
+        // ---------------- the gate: clamp in place for the tensor-core cumsum (a low bf16
+        // part when the bound is not a bf16 value), or the in-kernel gate forms summed in
+        // fp32 on the CUDA cores straight into tensor memory
+        if (gmode == kGateLog) {
+            if (p.has_lb) {
+                for (int e = tid; e < 1024; e += NT1) {
+                    float2 f[4], hi[4], lo[4];
+                    unpack8x2(lds128(sm + GS, e * 16), f);
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int jch = 2 * warp + jj;
-                const int hf = jch >> 3, jc = 8 * (jch & 7);
-                float2 ngm[4], emid[4], fkh[4], foff[4];
-                if (!fb) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int c = 8 * jch + 2 * e;
-                        const float2 m = blk ? make_float2(sG[128 + c], sG[128 + c + 1])
-                                             : make_float2(sG[c], sG[c + 1]);
-                        const float2 g63 = make_float2(sG[256 + c], sG[256 + c + 1]);
-                        const float2 g47 = make_float2(sG[128 + c], sG[128 + c + 1]);
-                        ngm[e] = make_float2(-m.x, -m.y);
-                        emid[e] = make_float2(__expf(m.x), __expf(m.y));
-                        fkh[e] = make_float2(__expf(g63.x - m.x), __expf(g63.y - m.y));
-                        foff[e] = make_float2(__expf(g47.x - m.x), __expf(g47.y - m.y));
+                    for (int q = 0; q < 4; ++q) {
+                        const float2 v = make_float2(fmaxf(f[q].x, p.lb), fmaxf(f[q].y, p.lb));
+                        const __nv_bfloat162 hb = __float22bfloat162_rn(v);
+                        hi[q] = __bfloat1622float2(hb);
+                        lo[q] = make_float2(v.x - hi[q].x, v.y - hi[q].y);
                     }
-                }
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int r = row0 + u;
-                    const uint32_t off = sw128_chunk(r, 8 * jch, 64);
-                    float2 qq[4], kk[4];
-                    unpack8x2(lds128(sm + STG_Q, off), qq);
-                    unpack8x2(lds128(sm + STG_K, off), kk);
-                    if (r >= L) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) { qq[e] = make_float2(0.f, 0.f); kk[e] = qq[e]; }
-                    }
-                    {
-                        float2 a = __fmul2_rn(qq[0], qq[0]), b = __fmul2_rn(kk[0], kk[0]);
-#pragma unroll
-                        for (int e = 1; e < 4; ++e) { a = __ffma2_rn(qq[e], qq[e], a); b = __ffma2_rn(kk[e], kk[e], b); }
-                        if (u == 0) { nrm_q.x += a.x + a.y; nrm_k.x += b.x + b.y; }
-                        else { nrm_q.y += a.x + a.y; nrm_k.y += b.x + b.y; }
-                    }
-                    float2 t1[4], t3[4];
-                    if (!fb) {
-                        float2 xk[4], xq[4], y[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            // a = G - G_m; ed = e^a (SFU), yd = e^-a = 1/ed (FMA pipe)
-                            const float2 a = __fmul2_rn(__fadd2_rn(make_float2(G[jj][u][2 * e], G[jj][u][2 * e + 1]), ngm[e]),
-                                                        make_float2(kLog2e, kLog2e));
-                            const float2 ed = make_float2(ex2a(a.x), ex2a(a.y));
-                            const float2 yd = rcp2_nr(ed);
-                            xk[e] = __fmul2_rn(kk[e], ed);
-                            xq[e] = __fmul2_rn(qq[e], ed);
-                            y[e] = __fmul2_rn(kk[e], yd);
-                            t1[e] = __fmul2_rn(xq[e], emid[e]);
-                            t3[e] = __fmul2_rn(y[e], fkh[e]);
-                        }
-                        sts128(sm, XKQD + sw128_chunk(r, 8 * jch, 128), pack8x2(xk));
-                        sts128(sm, XKQD + sw128_chunk(64 + r, 8 * jch, 128), pack8x2(xq));
-                        sts128(sm, (hf ? YD_H1 : YD_H0) + sw128_chunk(r, jc, 64), pack8x2(y));
-                        if (blk == 0) {
-                            // off-diagonal column operand k_s e^{G_47 - G_s}, paired with the block-1 rows
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) y[e] = __fmul2_rn(y[e], foff[e]);
-                            sts128(sm, (hf ? YO_H1 : YO_H0) + sw128_chunk(r, jc, 32), pack8x2(y));
-                        }
-                    } else {
-                        // exact path: no block reference, the k rows of XKQD hold k e^G (<= 1)
-                        float2 t2[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int c = 8 * jch + 2 * e;
-                            const float2 g = make_float2(G[jj][u][2 * e], G[jj][u][2 * e + 1]);
-                            const float2 eg = make_float2(expf(g.x), expf(g.y));
-                            const float2 ek = make_float2(expf(sG[256 + c] - g.x), expf(sG[256 + c + 1] - g.y));
-                            t1[e] = __fmul2_rn(qq[e], eg);
-                            t2[e] = __fmul2_rn(kk[e], eg);
-                            t3[e] = __fmul2_rn(kk[e], ek);
-                        }
-                        sts128(sm, XKQD + sw128_chunk(r, 8 * jch, 128), pack8x2(t2));
-                    }
-                    stg128(rec, R_QT + off, pack8x2(t1));
-                    stg128(rec, R_KH + off, pack8x2(t3));
+                    sts128(sm, GS + e * 16, pack8x2(hi));
+                    if (P.split_gate) sts128(sm, GLO + e * 16, pack8x2(lo));
                 }
             }
-            float *nrm = reinterpret_cast<float *>(sm + NRM);
-            nrm[warp * 64 + row0] = nrm_q.x;
-            nrm[warp * 64 + row0 + 1] = nrm_q.y;
-            nrm[512 + warp * 64 + row0] = nrm_k.x;
-            nrm[512 + warp * 64 + row0 + 1] = nrm_k.y;
+        } else {
+            const float bias = sDtb[c];
+            float Gv[32];
+            float run = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int r = 32 * hw + j;
+                const float x = bf(sm + GS, sw128(r, c, 64));
+                run += r < L ? gate_fast(x, bias, rate, gmode, p.lb) : 0.f;
+                Gv[j] = run;
+            }
+            if (hw == 0) sGX[c] = run;
+            __syncthreads();
+            if (hw == 1) {
+                const float off = sGX[c];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) Gv[j] += off;
+            }
+            tmem_st32(tb + lane_sel + TM_G + 32 * hw, Gv);
+            tmem_st_wait();
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
 
-        // ---------------- A_kk / A_qk products
-        // D1 (cols 0..63): rows 0..63 = A_kk, rows 64..127 = A_qk (diagonal 32-blocks valid).
-        // D2 (cols 64..95): lanes 0..31 = A_kk[32+i][0..31], lanes 64..95 = A_qk[32+i][0..31].
-        if (tid == kMma && !fb) {
+        // ---------------- tensor core: G^T = g^T Tri^T, k^T = k^T I, q^T = q^T I (lane = channel)
+        if (tid == kMma) {
+            if (gmode == kGateLog) {
+#pragma unroll
+                for (int kq = 0; kq < 4; ++kq)
+                    mma_bf16(tb + TM_G, desc(GS + kq * 2048, 8192), desc(TRI + kq * 32, 16), ID_T, kq > 0);
+                if (p.has_lb && P.split_gate) {
+#pragma unroll
+                    for (int kq = 0; kq < 4; ++kq)
+                        mma_bf16(tb + TM_G, desc(GLO + kq * 2048, 8192), desc(TRI + kq * 32, 16), ID_T, 1);
+                }
+            }
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)
+                mma_bf16(tb + TM_K, desc(KQ + kq * 2048, 16384), desc(IDT + kq * 32, 16), ID_T, kq > 0);
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq)
+                mma_bf16(tb + TM_Q, desc(KQ + 8192 + kq * 2048, 16384), desc(IDT + kq * 32, 16), ID_T, kq > 0);
+            mma_commit(bar_mma);
+            mma_out = true;
+        }
+        // row norms of k and q from the staged rows while the products run: four
+        // threads per row, 32 channels each
+        {
+            const int r = tid >> 2, part = tid & 3, half = part >> 1, cb = (part & 1) * 4;
+            float2 ak = make_float2(0.f, 0.f), aq = ak;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t off = KQ + half * 16384 + r * 128 + ((((cb + j) ^ (r & 7))) << 4);
+                float2 fk[4], fq[4];
+                unpack8x2(lds128(sm, off), fk);
+                unpack8x2(lds128(sm, off + 8192), fq);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) { ak = __ffma2_rn(fk[e], fk[e], ak); aq = __ffma2_rn(fq[e], fq[e], aq); }
+            }
+            float sk = ak.x + ak.y, sq = aq.x + aq.y;
+            sk += __shfl_xor_sync(0xffffffffu, sk, 1);
+            sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+            sk += __shfl_xor_sync(0xffffffffu, sk, 2);
+            sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+            if (part == 0) {
+                sinvk[r] = r < L ? (p.use_l2 ? rsqrtf(sk + kL2Eps) : 1.f) : 0.f;
+                sinvq[r] = r < L ? (p.use_l2 ? rsqrtf(sq + kL2Eps) : 1.f) : 0.f;
+            }
+        }
+        if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
+        if (tid == kMma) mma_out = false;
+        tc_fence_after();
+
+        // ---------------- operands, channel layout: thread (c, hw) turns its 32 rows of
+        // G, k, q into the bf16 rows c of X_k^T, X_q^T, Y^T (block reference G_m = G_15
+        // or G_47 by hw), Y'^T (reference G_47, hw = 0), Qtil^T and Khat^T
+        float e15, e47;
+        bool span_bad;
+        {
+            const float g15 = tmem_ld1(tb + lane_sel + TM_G + 15);
+            const float g47 = tmem_ld1(tb + lane_sel + TM_G + 47);
+            const float g63 = tmem_ld1(tb + lane_sel + TM_G + 63);
+            tmem_ld_wait();
+            const float gm = hw ? g47 : g15;
+            e15 = ex2a(g15 * kL2e);
+            e47 = ex2a(g47 * kL2e);
+            if (hw == 0) sgam[c] = ex2a(g63 * kL2e);
+            const float2 l2e2 = make_float2(kL2e, kL2e), nb = make_float2(-gm * kL2e, -gm * kL2e);
+            const float em = ex2a(gm * kL2e), fk = ex2a((g63 - gm) * kL2e);
+            const float2 em2 = make_float2(em, em), fk2 = make_float2(fk, fk);
+            // Y' takes its own exponent G_47 - G_s (>= -80 - |g_32| next to the block
+            // boundary, where it matters): a factor e^{G_47 - G_15} spans 32 tokens and
+            // would leave the fp32 range for steep gates
+            const float2 nl2e2 = make_float2(-kL2e, -kL2e), b47 = make_float2(g47 * kL2e, g47 * kL2e);
+            float amax = 0.f;  // largest |G - G_m| in log2 units
+#pragma unroll
+            for (int sb2 = 0; sb2 < 2; ++sb2) {
+                const int r0 = 32 * hw + 16 * sb2;
+                float Gv[16], Kv[16], Qv[16];
+                tmem_ld16(tb + lane_sel + TM_G + r0, Gv);
+                tmem_ld16(tb + lane_sel + TM_K + r0, Kv);
+                tmem_ld16(tb + lane_sel + TM_Q + r0, Qv);
+                tmem_ld_wait();
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    float2 xk[4], xq[4], y[4], qt[4], kh[4], yo[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int i = 8 * u + 2 * j;
+                        const float2 g2 = make_float2(Gv[i], Gv[i + 1]);
+                        const float2 k2 = make_float2(Kv[i], Kv[i + 1]);
+                        const float2 q2 = make_float2(Qv[i], Qv[i + 1]);
+                        const float2 a = __ffma2_rn(g2, l2e2, nb);
+                        amax = fmaxf(amax, fmaxf(fabsf(a.x), fabsf(a.y)));
+                        const float2 ed = make_float2(ex2a(a.x), ex2a(a.y));
+                        const float2 yd = make_float2(ex2a(-a.x), ex2a(-a.y));
+                        xk[j] = __fmul2_rn(k2, ed);
+                        xq[j] = __fmul2_rn(q2, ed);
+                        y[j] = __fmul2_rn(k2, yd);
+                        qt[j] = __fmul2_rn(xq[j], em2);
+                        kh[j] = __fmul2_rn(y[j], fk2);
+                        if (hw == 0) {
+                            const float2 a47 = __ffma2_rn(g2, nl2e2, b47);
+                            yo[j] = __fmul2_rn(k2, make_float2(ex2a(a47.x), ex2a(a47.y)));
+                        }
+                    }
+                    const uint32_t off = c * 128 + ((((r0 >> 3) + u) ^ (c & 7)) << 4);
+                    sts128(sm, XK + off, pack8x2(xk));
+                    sts128(sm, XQ + off, pack8x2(xq));
+                    sts128(sm, YT + off, pack8x2(y));
+                    sts128(sm, QT + off, pack8x2(qt));
+                    sts128(sm, KH + off, pack8x2(kh));
+                    if (hw == 0) sts128(sm, YP + off, pack8x2(yo));
+                }
+            }
+            span_bad = !(amax <= kSpanMax * kL2e);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        const bool fb = __syncthreads_or(span_bad) != 0;
+        tc_fence_after();
+        // a chunk whose gate moves too far inside a block: its record is rewritten exactly
+        if (fb && tid == kMma) P.fix_list[atomicAdd(P.fix_count, 1)] = (int)item;
+        if (tid == kTma) {
+            bulk_store(rec + R_QT, sm + QT, 16384);
+            bulk_store(rec + R_KH, sm + KH, 16384);
+            bulk_commit();
+        }
+
+        // ---------------- A products: D1 = [X_k; X_q] Y^T (diagonal 32-blocks valid),
+        // D2 = [X_k; X_q] Y'^T (rows 32..63 against columns 0..31 valid)
+        if (tid == kMma) {
 #pragma unroll
             for (int kq = 0; kq < 8; ++kq) {
-                const uint32_t ko = (kq >> 2) * 16384 + (kq & 3) * 32;
-                const uint32_t yb = (kq >> 2) ? YD_H1 : YD_H0, ob = (kq >> 2) ? YO_H1 : YO_H0;
-                mma_bf16(tb + TM1_A, dk(XKQD + ko), dk(yb + (kq & 3) * 32), ID_A1, kq > 0);
-                mma_bf16(tb + TM1_A + 64, dk(XKQD + ko + 32 * 128), dk(ob + (kq & 3) * 32), ID_A2, kq > 0);
+                const uint64_t a = desc(XK + kq * 2048, 16384);
+                mma_bf16(tb + TM_A1, a, desc(YT + kq * 2048, 8192), ID_A, kq > 0);
+                mma_bf16(tb + TM_A2, a, desc(YP + kq * 2048, 8192), ID_A, kq > 0);
             }
             mma_commit(bar_mma);
             mma_out = true;
         }
-        if (tid < 128) {  // row norms from the 8 per-warp partials
-            const int r = tid & 63, which = tid >> 6;
-            const float *nrm = reinterpret_cast<const float *>(sm + NRM) + which * 512 + r;
-            float ssum = 0.f;
-#pragma unroll
-            for (int w = 0; w < 8; ++w) ssum += nrm[w * 64];
-            const float inv = r < L ? (p.use_l2 ? rsqrtf(ssum + kL2Eps) : 1.f) : 0.f;
-            (which ? sinvk : sinvq)[r] = inv;
-        }
+        if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
+        if (tid == kMma) mma_out = false;
+        tc_fence_after();
 
-        // ---------------- A results -> L (fp32, beta and key norms applied) and raw A_qk tile
-        if (!fb) {
-            if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
-            if (tid == kMma) mma_out = false;
-            tc_fence_after();
+        // ---------------- read-back, row layout (lane = row): L = beta_r |k_r|^-1 |k_s|^-1 A_kk
+        // (fp32, strictly lower part) and the raw A_qk tile (bf16, s <= r)
+        {
             const int i = lane;
-#pragma unroll
-            for (int it = 0; it < 2; ++it) {
-                const int cg4 = 2 * cgrp + it;
-                const bool has = (quarter & 1) == 0 || cg4 < 2;
-                const int col = (quarter & 1) ? 32 + 16 * cg4 : (cg4 < 2 ? 16 * cg4 : 64 + 16 * (cg4 - 2));
+            if (quarter == 0) {  // A_kk rows 0..31, columns 16 hw ..: s < i
                 float va[16];
-                if (has) {
-                    tmem_ld16(tb + TM1_A + lane_sel + col, va);
-                    tmem_ld_wait();
+                tmem_ld16(tb + lane_sel + TM_A1 + 16 * hw, va);
+                tmem_ld_wait();
+                const float f = sbeta[i] * sinvk[i];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int s = 16 * hw + j;
+                    if (s < i) Lf[i * LDS + s] = f * sinvk[s] * va[j];
                 }
-                if (quarter == 0) {
-                    if (cg4 < 2) {  // A_kk rows 0..31, cols 16*cg4..: s < i
-                        const float f = sbeta[i] * sinvk[i];
+            } else if (quarter == 1) {  // A_kk rows 32..63: hw 0 the diagonal block, hw 1 columns 0..31
+                float va[32];
+                tmem_ld32(tb + lane_sel + (hw ? TM_A2 : TM_A1 + 32), va);
+                tmem_ld_wait();
+                const float f = sbeta[32 + i] * sinvk[32 + i];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int s = 16 * cg4 + j;
-                            Lf[i * LDS + s] = s < i ? f * sinvk[s] * va[j] : 0.f;
-                        }
-                    } else {        // A_kk rows 32..63, cols 0..31 (all below the diagonal)
-                        const float f = sbeta[32 + i] * sinvk[32 + i];
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int s = 16 * (cg4 - 2) + j;
-                            Lf[(32 + i) * LDS + s] = f * sinvk[s] * va[j];
-                        }
-                    }
-                } else if (quarter == 1) {
-                    if (cg4 < 2) {  // A_kk rows 32..63, cols 32..63: s < i
-                        const float f = sbeta[32 + i] * sinvk[32 + i];
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const int s = 16 * cg4 + j;
-                            Lf[(32 + i) * LDS + 32 + s] = s < i ? f * sinvk[32 + s] * va[j] : 0.f;
-                        }
-                    }
-                } else if (quarter == 2) {
-                    if (cg4 < 2) {  // A_qk rows 0..31, cols 0..31: s <= i
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) va[j] = 16 * cg4 + j <= i ? va[j] : 0.f;
-                        row16_to_tile(sm, AQK, i, 16 * cg4, 64, va);
-                    } else {        // A_qk rows 32..63, cols 0..31
-                        row16_to_tile(sm, AQK, 32 + i, 16 * (cg4 - 2), 64, va);
-                    }
-                } else {
-                    if (cg4 < 2) {  // A_qk rows 32..63, cols 32..63: s <= i
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) va[j] = 16 * cg4 + j <= i ? va[j] : 0.f;
-                        row16_to_tile(sm, AQK, 32 + i, 32 + 16 * cg4, 64, va);
-                    } else {        // A_qk rows 0..31, cols 32..63 are zero
-                        const int c0 = 32 + 16 * (cg4 - 2);
-                        sts128(sm, AQK + sw128_chunk(i, c0, 64), make_uint4(0u, 0u, 0u, 0u));
-                        sts128(sm, AQK + sw128_chunk(i, c0 + 8, 64), make_uint4(0u, 0u, 0u, 0u));
-                    }
+                for (int j = 0; j < 32; ++j) {
+                    const int s = (hw ? 0 : 32) + j;
+                    if (hw || j < i) Lf[(32 + i) * LDS + s] = f * sinvk[s] * va[j];
                 }
-            }
-        } else {
-            __syncthreads();  // the row norms above are read below
-            // exact A_kk / A_qk on CUDA cores (raw rows): warp per row r, lanes over channels,
-            // walking s downwards while accumulating the gate between s and r
-            for (int r = warp; r < C; r += NT1 / 32) {
-                float kr[4], qr[4], dg[4];
+            } else if (quarter == 2) {  // A_qk rows 0..31: columns 16 hw .. (s <= i), zeros right of 32
+                float va[16];
+                tmem_ld16(tb + lane_sel + TM_A1 + 16 * hw, va);
+                tmem_ld_wait();
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const uint32_t o = sw128(r, lane + 32 * u, 64);
-                    kr[u] = r < L ? bf(sm + STG_K, o) : 0.f;
-                    qr[u] = r < L ? bf(sm + STG_Q, o) : 0.f;
-                    dg[u] = 0.f;
-                }
-                for (int s = r; s >= 0; --s) {
-                    float akk = 0.f, aqk = 0.f;
+                for (int j = 0; j < 16; ++j) va[j] = 16 * hw + j <= i ? va[j] : 0.f;
+                row16_to_tile(sm, AQK, i, 16 * hw, 64, va);
+                sts128(sm, AQK + sw128_chunk(i, 32 + 16 * hw, 64), make_uint4(0u, 0u, 0u, 0u));
+                sts128(sm, AQK + sw128_chunk(i, 40 + 16 * hw, 64), make_uint4(0u, 0u, 0u, 0u));
+            } else {  // A_qk rows 32..63: hw 0 the diagonal block (s <= i), hw 1 columns 0..31
+                float va[32];
+                tmem_ld32(tb + lane_sel + (hw ? TM_A2 : TM_A1 + 32), va);
+                tmem_ld_wait();
+                if (!hw) {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint32_t o = sw128(s, lane + 32 * u, 64);
-                        const float e = expf(dg[u]) * (s < L ? bf(sm + STG_K, o) : 0.f);
-                        akk = fmaf(kr[u], e, akk);
-                        aqk = fmaf(qr[u], e, aqk);
-                        float gv = 0.f;
-                        if (s < L) {
-                            gv = bf(sm + STG_G, o);
-                            if (gmode != kGateLog) gv = gate_fast(gv, sDtb[lane + 32 * u], rate, gmode, p.lb);
-                            else if (p.has_lb) gv = fmaxf(gv, p.lb);
-                        }
-                        dg[u] += gv;
-                    }
-                    akk = warp_sum(akk); aqk = warp_sum(aqk);
-                    if (lane == 0) {
-                        Lf[r * LDS + s] = s < r ? sbeta[r] * sinvk[r] * sinvk[s] * akk : 0.f;
-                        st_bf(sm, AQK + sw128(r, s, 64), aqk);
-                    }
+                    for (int j = 0; j < 32; ++j) va[j] = j <= i ? va[j] : 0.f;
                 }
-                for (int s = r + 1 + lane; s < C; s += 32) st_bf(sm, AQK + sw128(r, s, 64), 0.f);
+                float v16[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v16[j] = va[j];
+                row16_to_tile(sm, AQK, 32 + i, hw ? 0 : 32, 64, v16);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v16[j] = va[16 + j];
+                row16_to_tile(sm, AQK, 32 + i, hw ? 16 : 48, 64, v16);
             }
         }
+        // the Qtil^T / Khat^T stores must have read their sources before T and T_w overwrite them
+        if (tid == kTma) bulk_wait_read_all();
         __syncthreads();
 
         // ---------------- T = (I + L)^-1 on 16x16 blocks, written straight into the bf16
-        // tiles T_u = T diag(beta) and T_w = T diag(beta / |k|) (rows r, columns s <= r)
+        // tiles T' = T diag(beta) (record) and T_w = T diag(beta / |k|) (rows r, columns s <= r)
         if (warp < 4) {
             // diagonal blocks by a column sweep (lane j = column j)
             if (lane < 16) {
@@ -532,11 +531,11 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
                 const int bid = e >> 5, i = (e >> 1) & 15, half = e & 1;
                 const int bi = bid < 3 ? 0 : bid < 5 ? 1 : 2;
                 const int bj = bid < 3 ? bid + 1 : bid < 5 ? bid - 1 : 3;
-                const int r = 16 * bi + i, c = 16 * bj + 8 * half;
-                *reinterpret_cast<float4 *>(Tf + r * LDT + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-                *reinterpret_cast<float4 *>(Tf + r * LDT + c + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
-                sts128(sm, TPU + sw128_chunk(r, c, 64), make_uint4(0u, 0u, 0u, 0u));
-                sts128(sm, TPW + sw128_chunk(r, c, 64), make_uint4(0u, 0u, 0u, 0u));
+                const int r = 16 * bi + i, cc = 16 * bj + 8 * half;
+                *reinterpret_cast<float4 *>(Tf + r * LDT + cc) = make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4 *>(Tf + r * LDT + cc + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+                sts128(sm, TPU + sw128_chunk(r, cc, 64), make_uint4(0u, 0u, 0u, 0u));
+                sts128(sm, TW + sw128_chunk(r, cc, 64), make_uint4(0u, 0u, 0u, 0u));
             }
         }
         __syncthreads();
@@ -546,16 +545,16 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
         if (warp >= 6) {
             for (int e = tid - 192; e < 128; e += 64) {
                 const int b = e >> 5, i = (e >> 1) & 15, half = e & 1;
-                const int r = 16 * b + i, c = 16 * b + 8 * half;
+                const int r = 16 * b + i, cc = 16 * b + 8 * half;
                 float mu[8], mw[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    const int s_ = c + q;
+                    const int s_ = cc + q;
                     mu[q] = s_ <= r ? Tf[r * LDT + s_] * sbeta[s_] : 0.f;
                     mw[q] = mu[q] * sinvk[s_];
                 }
-                sts128(sm, TPU + sw128_chunk(r, c, 64), pack8(mu));
-                sts128(sm, TPW + sw128_chunk(r, c, 64), pack8(mw));
+                sts128(sm, TPU + sw128_chunk(r, cc, 64), pack8(mu));
+                sts128(sm, TW + sw128_chunk(r, cc, 64), pack8(mw));
             }
         }
         {
@@ -580,34 +579,34 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
                     const bool odd = g & 1;
                     float v[8];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        v[c] = __shfl_sync(0xffffffffu, d[c], srcA);
-                        v[4 + c] = __shfl_sync(0xffffffffu, d[c], srcB);
+                    for (int cq = 0; cq < 4; ++cq) {
+                        v[cq] = __shfl_sync(0xffffffffu, d[cq], srcA);
+                        v[4 + cq] = __shfl_sync(0xffffffffu, d[cq], srcB);
                     }
                     const uint32_t b0[2] = {to_tf32(odd ? v[1] : v[0]), to_tf32(odd ? v[5] : v[4])};
                     const uint32_t b1[2] = {to_tf32(odd ? v[3] : v[2]), to_tf32(odd ? v[7] : v[6])};
-                    float e[4] = {0.f, 0.f, 0.f, 0.f};
+                    float e4[4] = {0.f, 0.f, 0.f, 0.f};
                     const float *Ta = Tf + (16 * I + g) * LDT + 16 * I, *Tb = Tf + (16 * I + g + 8) * LDT + 16 * I;
                     {
                         const uint32_t a[4] = {to_tf32(Ta[t4]), to_tf32(Tb[t4]), to_tf32(Ta[t4 + 4]), to_tf32(Tb[t4 + 4])};
-                        mma_tf32_16x8x8(e, a, b0);
+                        mma_tf32_16x8x8(e4, a, b0);
                     }
                     {
                         const uint32_t a[4] = {to_tf32(Ta[8 + t4]), to_tf32(Tb[8 + t4]), to_tf32(Ta[12 + t4]),
                                                to_tf32(Tb[12 + t4])};
-                        mma_tf32_16x8x8(e, a, b1);
+                        mma_tf32_16x8x8(e4, a, b1);
                     }
                     const int r0 = 16 * I + g, c0 = n0 + 2 * t4;
-                    Tf[r0 * LDT + c0] = -e[0];
-                    Tf[r0 * LDT + c0 + 1] = -e[1];
-                    Tf[(r0 + 8) * LDT + c0] = -e[2];
-                    Tf[(r0 + 8) * LDT + c0 + 1] = -e[3];
+                    Tf[r0 * LDT + c0] = -e4[0];
+                    Tf[r0 * LDT + c0 + 1] = -e4[1];
+                    Tf[(r0 + 8) * LDT + c0] = -e4[2];
+                    Tf[(r0 + 8) * LDT + c0 + 1] = -e4[3];
                     const float b0s = sbeta[c0], b1s = sbeta[c0 + 1];
                     const float w0s = b0s * sinvk[c0], w1s = b1s * sinvk[c0 + 1];
-                    *reinterpret_cast<uint32_t *>(sm + TPU + sw128(r0, c0, 64)) = pack_bf16x2(-e[0] * b0s, -e[1] * b1s);
-                    *reinterpret_cast<uint32_t *>(sm + TPU + sw128(r0 + 8, c0, 64)) = pack_bf16x2(-e[2] * b0s, -e[3] * b1s);
-                    *reinterpret_cast<uint32_t *>(sm + TPW + sw128(r0, c0, 64)) = pack_bf16x2(-e[0] * w0s, -e[1] * w1s);
-                    *reinterpret_cast<uint32_t *>(sm + TPW + sw128(r0 + 8, c0, 64)) = pack_bf16x2(-e[2] * w0s, -e[3] * w1s);
+                    *reinterpret_cast<uint32_t *>(sm + TPU + sw128(r0, c0, 64)) = pack_bf16x2(-e4[0] * b0s, -e4[1] * b1s);
+                    *reinterpret_cast<uint32_t *>(sm + TPU + sw128(r0 + 8, c0, 64)) = pack_bf16x2(-e4[2] * b0s, -e4[3] * b1s);
+                    *reinterpret_cast<uint32_t *>(sm + TW + sw128(r0, c0, 64)) = pack_bf16x2(-e4[0] * w0s, -e4[1] * w1s);
+                    *reinterpret_cast<uint32_t *>(sm + TW + sw128(r0 + 8, c0, 64)) = pack_bf16x2(-e4[2] * w0s, -e4[3] * w1s);
                 }
                 if (I < 3) __syncthreads();
             }
@@ -617,56 +616,49 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
         __syncthreads();
         tc_fence_after();
 
-        // ---------------- W^T = Ktil^T T_w^T in two K halves (token blocks 0..31, 32..63), each
-        // with its own block reference, recombined per key channel at read-back
+        // ---------------- W^T = X_k^T T_w^T in two K halves (token blocks 0..31, 32..63, each
+        // with its own block reference), recombined per key channel at read-back
         if (tid == kMma) {
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq)
-                mma_bf16(tb + (kq < 2 ? TM1_W : TM1_W1), dx(XKQD + kq * 2048), dk(TPW + kq * 32), ID_UW,
+                mma_bf16(tb + (kq < 2 ? TM_W0 : TM_W1), desc(XK + kq * 32, 16), desc(TW + kq * 32, 16), ID_W,
                          (kq & 1) != 0);
             mma_commit(bar_mma);
             mma_out = true;
         }
-        // T', A_qk and the per-row / per-channel scalars to the record while the product runs
-        {
-            const uint4 *src_u = reinterpret_cast<const uint4 *>(sm + TPU);
-            const uint4 *src_a = reinterpret_cast<const uint4 *>(sm + AQK);
-            uint4 *dst_u = reinterpret_cast<uint4 *>(rec + R_TPU);
-            uint4 *dst_a = reinterpret_cast<uint4 *>(rec + R_AQK);
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                dst_u[tid + NT1 * m] = src_u[tid + NT1 * m];
-                dst_a[tid + NT1 * m] = src_a[tid + NT1 * m];
-            }
-            float *misc = reinterpret_cast<float *>(rec + R_MISC);
-            if (tid < D) misc[tid] = fb ? expf(sG[256 + tid]) : __expf(sG[256 + tid]);
-            else if (tid < D + 64) misc[128 + (tid - D)] = sinvq[tid - D];
-            else misc[192 + (tid - D - 64)] = sinvk[tid - D - 64];
+        if (tid == kTma) {
+            bulk_store(rec + R_AQK, sm + AQK, 8192);
+            bulk_store(rec + R_TPU, sm + TPU, 8192);
+            bulk_commit();
         }
         if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
         if (tid == kMma) mma_out = false;
         tc_fence_after();
-        // the staging area is free again: the next item's inputs load during the read-back
+        // the input area is free again: the next item's inputs load during the read-back
         if (tid == kTma && have_next) { issue_in(nxt); in_out = true; }
-        {   // W^T (lane c, columns r) = e^{G_15[c]} W0 + e^{G_47[c]} W1 -> record image [c][r]
-            const int c = 32 * quarter + lane;
-            const float e0 = fb ? 1.f : __expf(sG[c]), e1 = fb ? 1.f : __expf(sG[128 + c]);
+        {   // thread (c, hw): W^T[c][r], r = 32 hw .., = e^{G_15} W0 + e^{G_47} W1
 #pragma unroll
-            for (int it = 0; it < 2; ++it) {
-                const int col = 32 * cgrp + 16 * it;
-                float x[16], x1[16];
-                tmem_ld16(tb + TM1_W + lane_sel + col, x);
-                tmem_ld16(tb + TM1_W1 + lane_sel + col, x1);
+            for (int u = 0; u < 2; ++u) {
+                const int r0 = 32 * hw + 16 * u;
+                float w0[16], w1[16];
+                tmem_ld16(tb + lane_sel + TM_W0 + r0, w0);
+                tmem_ld16(tb + lane_sel + TM_W1 + r0, w1);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) x[j] = fmaf(e0, x[j], e1 * x1[j]);
-                stg128(rec, R_WT + sw128_chunk(c, col, 128), pack8(x));
-                stg128(rec, R_WT + sw128_chunk(c, col + 8, 128), pack8(x + 8));
+                for (int j = 0; j < 16; ++j) w0[j] = fmaf(e15, w0[j], e47 * w1[j]);
+                sts128(sm, WT + c * 128 + (((r0 >> 3) ^ (c & 7)) << 4), pack8(w0));
+                sts128(sm, WT + c * 128 + ((((r0 >> 3) + 1) ^ (c & 7)) << 4), pack8(w0 + 8));
             }
         }
+        fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
+        if (tid == kTma) {
+            bulk_store(rec + R_WT, sm + WT, 16384);
+            bulk_store(rec + R_MISC, sm + M1_REC, 1024);
+            bulk_commit();
+        }
 
         item = nitem;
         cur = nxt;
@@ -678,11 +670,148 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
         if (mma_out) mbar_wait(bar_mma, ph_mma, kWaitLimitNs);
         if (P.status && tid == kMma) atomicOr(P.status, 1);
     }
+    if (tid == kTma) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tb, TM1_COLS);
+    }
+}
+
+// ============================================================== exact records
+// Rewrites the record of every queued (chunk, head) on CUDA cores in fp32 from
+// exponent differences that are never positive (gate <= 0), so no factor can
+// overflow whatever the gate: A_kk and A_qk term by term, T by row-wise forward
+// substitution, W = T diag(beta/|k|) (k e^G), Qtil = q e^G, Khat = k e^{G_last-G}.
+constexpr int NTX = 256;
+constexpr int LDX = 65;
+constexpr uint32_t X_Q = 0, X_K = 32768, X_G = 65536;           // fp32 [64][128]
+constexpr uint32_t X_AKK = 98304, X_AQK = X_AKK + 64 * LDX * 4;  // fp32 [64][65]
+constexpr uint32_t X_T = X_AQK + 64 * LDX * 4;
+constexpr uint32_t X_MISC = X_T + 64 * LDX * 4;                  // beta, invq, invk [64] each
+constexpr uint32_t SMEMX_BYTES = X_MISC + 768;
+
+__global__ void __launch_bounds__(NTX, 1) kda_tp_exact_kernel(const __grid_constant__ IntraParams P) {
+    extern __shared__ uint8_t smx[];
+    const ChunkParams &p = P.p;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = p.H;
+    float *qf = reinterpret_cast<float *>(smx + X_Q), *kf = reinterpret_cast<float *>(smx + X_K);
+    float *Gf = reinterpret_cast<float *>(smx + X_G);
+    float *Akk = reinterpret_cast<float *>(smx + X_AKK), *Aqk = reinterpret_cast<float *>(smx + X_AQK);
+    float *Tm = reinterpret_cast<float *>(smx + X_T);
+    float *sbeta = reinterpret_cast<float *>(smx + X_MISC), *sinvq = sbeta + 64, *sinvk = sbeta + 128;
+    const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(p.q), *kb = static_cast<const __nv_bfloat16 *>(p.k);
+    const __nv_bfloat16 *gb = static_cast<const __nv_bfloat16 *>(p.g), *bt = static_cast<const __nv_bfloat16 *>(p.beta);
+    const int nch = P.chunk_tok ? *P.n_chunks : 0;
+    const int count = *P.fix_count;
+
+    for (int idx = blockIdx.x; idx < count; idx += gridDim.x) {
+        Item it;
+        if (!decode_item(P, P.fix_list[idx], nch, it)) continue;
+        const int h = it.h, L = it.L;
+        const long long t0 = it.t0;
+        uint8_t *rec = P.rec + (it.gc * H + h) * (long long)REC_BYTES;
+        const float rate = p.gate_mode != kGateLog ? expf(p.A_log[h]) : 0.f;
+
+        __syncthreads();  // the previous item's shared data is no longer read
+        for (int e = tid; e < C * D; e += NTX) {
+            const int r = e >> 7, cc = e & 127;
+            const long long gi = ((t0 + r) * H + h) * D + cc;
+            float x = 0.f, y = 0.f, gv = 0.f;
+            if (r < L) {
+                x = __bfloat162float(qb[gi]);
+                y = __bfloat162float(kb[gi]);
+                const float bias = (p.gate_mode != kGateLog && p.dt_bias) ? p.dt_bias[h * D + cc] : 0.f;
+                gv = gate_value(__bfloat162float(gb[gi]), bias, rate, p.gate_mode, p.has_lb, p.lb);
+            }
+            qf[e] = x;
+            kf[e] = y;
+            Gf[e] = gv;
+        }
+        if (tid < C) {
+            const float b = tid < L ? __bfloat162float(bt[(t0 + tid) * H + h]) : 0.f;
+            sbeta[tid] = tid < L ? beta_value(b, p.beta_prob) : 0.f;
+        }
+        __syncthreads();
+        if (tid < D) {  // inclusive cumsum per channel
+            float run = 0.f;
+            for (int r = 0; r < C; ++r) { run += Gf[r * D + tid]; Gf[r * D + tid] = run; }
+        }
+        for (int r = warp; r < C; r += NTX / 32) {  // row norms
+            float sq = 0.f, sk = 0.f;
+            for (int cc = lane; cc < D; cc += 32) {
+                sq = fmaf(qf[r * D + cc], qf[r * D + cc], sq);
+                sk = fmaf(kf[r * D + cc], kf[r * D + cc], sk);
+            }
+            sq = warp_sum(sq);
+            sk = warp_sum(sk);
+            if (lane == 0) {
+                sinvq[r] = r < L ? (p.use_l2 ? rsqrtf(sq + kL2Eps) : 1.f) : 0.f;
+                sinvk[r] = r < L ? (p.use_l2 ? rsqrtf(sk + kL2Eps) : 1.f) : 0.f;
+            }
+        }
+        __syncthreads();
+        // raw A_kk[r][s] and A_qk[r][s] for s <= r: warp per pair, lanes over channels
+        for (int pr = warp; pr < C * (C + 1) / 2; pr += NTX / 32) {
+            int r = (int)((sqrtf(8.f * pr + 1.f) - 1.f) * 0.5f);
+            while ((r + 1) * (r + 2) / 2 <= pr) ++r;
+            while (r * (r + 1) / 2 > pr) --r;
+            const int s = pr - r * (r + 1) / 2;
+            float akk = 0.f, aqk = 0.f;
+            for (int cc = lane; cc < D; cc += 32) {
+                const float e = expf(Gf[r * D + cc] - Gf[s * D + cc]) * kf[s * D + cc];
+                akk = fmaf(kf[r * D + cc], e, akk);
+                aqk = fmaf(qf[r * D + cc], e, aqk);
+            }
+            akk = warp_sum(akk);
+            aqk = warp_sum(aqk);
+            if (lane == 0) {
+                Akk[r * LDX + s] = s < r ? sbeta[r] * sinvk[r] * sinvk[s] * akk : 0.f;  // L
+                Aqk[r * LDX + s] = aqk;
+            }
+        }
+        __syncthreads();
+        // T = (I + L)^-1, row by row: T[i][j] = delta_ij - sum_{j<=k<i} L[i][k] T[k][j]
+        for (int i = 0; i < C; ++i) {
+            if (tid <= i) {
+                float t = tid == i ? 1.f : 0.f;
+                for (int k = tid; k < i; ++k) t = fmaf(-Akk[i * LDX + k], Tm[k * LDX + tid], t);
+                Tm[i * LDX + tid] = t;
+            }
+            __syncthreads();
+        }
+        // record: A_qk, T' tiles (bf16 images, zero above the diagonal)
+        for (int e = tid; e < C * C; e += NTX) {
+            const int r = e >> 6, s = e & 63;
+            const float aq = s <= r ? Aqk[r * LDX + s] : 0.f;
+            const float tp = s <= r ? Tm[r * LDX + s] * sbeta[s] : 0.f;
+            *reinterpret_cast<__nv_bfloat16 *>(rec + R_AQK + sw128(r, s, 64)) = __float2bfloat16_rn(aq);
+            *reinterpret_cast<__nv_bfloat16 *>(rec + R_TPU + sw128(r, s, 64)) = __float2bfloat16_rn(tp);
+        }
+        // Qtil^T, Khat^T, then k e^G in place of k
+        for (int e = tid; e < C * D; e += NTX) {
+            const int r = e >> 7, cc = e & 127;
+            const float g = Gf[e], gl = Gf[(C - 1) * D + cc];
+            *reinterpret_cast<__nv_bfloat16 *>(rec + R_QT + sw128(cc, r, 128)) = __float2bfloat16_rn(qf[e] * expf(g));
+            *reinterpret_cast<__nv_bfloat16 *>(rec + R_KH + sw128(cc, r, 128)) =
+                __float2bfloat16_rn(kf[e] * expf(gl - g));
+        }
+        __syncthreads();
+        for (int e = tid; e < C * D; e += NTX) kf[e] *= expf(Gf[e]);
+        __syncthreads();
+        // W^T[c][r] = sum_{s<=r} T[r][s] beta_s |k_s|^-1 (k e^G)[s][c]
+        for (int e = tid; e < C * D; e += NTX) {
+            const int cc = e & 127, r = e >> 7;
+            float w = 0.f;
+            for (int s = 0; s <= r; ++s) w = fmaf(Tm[r * LDX + s] * sbeta[s] * sinvk[s], kf[s * D + cc], w);
+            *reinterpret_cast<__nv_bfloat16 *>(rec + R_WT + sw128(cc, r, 128)) = __float2bfloat16_rn(w);
+        }
+        float *misc = reinterpret_cast<float *>(rec + R_MISC);
+        if (tid < D) misc[tid] = expf(Gf[(C - 1) * D + tid]);
+        else if (tid < D + C) misc[128 + tid - D] = sinvq[tid - D];
+        else misc[192 + tid - D - C] = sinvk[tid - D - C];
     }
 }
 
@@ -699,6 +828,11 @@ constexpr uint32_t SMEM2_ALLOC = SMEM2_BYTES + 1024;
 static_assert(STAGE_BYTES % 1024 == 0 && SMEM2_ALLOC <= 232448, "pass 2 shared memory");
 
 constexpr uint32_t TM2_S = 0, TM2_D = 128, TM2_O = 192, TM2_COLS = 256;
+constexpr uint32_t ID2_UW = idesc_bf16(128, 64, true, false);           // V^T T'^T
+constexpr uint32_t ID2_DL = idesc_bf16(128, 64, false, true, true);     // - S^T W^T
+constexpr uint32_t ID2_OQ = idesc_bf16(128, 64, false, true);           // S^T Qtil^T
+constexpr uint32_t ID2_OA = idesc_bf16(128, 64, false, false);          // D~^T A_qk^T
+constexpr uint32_t ID2_S = idesc_bf16(128, 128, false, false);          // D~^T Khat
 constexpr int kMaxPerm = 256;
 
 struct StateParams {
@@ -823,12 +957,12 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
         if (tid == kMma) {
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq)
-                mma_bf16(tb + TM2_D, dm(so + S_V + kq * 2048), dk(so + R_TPU + kq * 32), ID_UW, kq > 0);
+                mma_bf16(tb + TM2_D, dm(so + S_V + kq * 2048), dk(so + R_TPU + kq * 32), ID2_UW, kq > 0);
 #pragma unroll
             for (int kq = 0; kq < 8; ++kq) {
                 const uint64_t adesc = dk(ST2 + (kq >> 2) * 16384 + (kq & 3) * 32);
-                mma_bf16(tb + TM2_D, adesc, dm(so + R_WT + kq * 2048), ID_DL, 1);
-                mma_bf16(tb + TM2_O, adesc, dk(so + R_QT + (kq >> 2) * 8192 + (kq & 3) * 32), ID_O, kq > 0);
+                mma_bf16(tb + TM2_D, adesc, dm(so + R_WT + kq * 2048), ID2_DL, 1);
+                mma_bf16(tb + TM2_O, adesc, dm(so + R_QT + kq * 2048), ID2_OQ, kq > 0);
             }
             mma_commit(bar_mma);
             mma_out = true;
@@ -850,13 +984,13 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
         __syncthreads();
         tc_fence_after();
 
-        // ---------------- O^T += D~^T A_qk^T ; S^T += D~^T Khat
+        // ---------------- O^T += D~^T A_qk^T ; S^T += D~^T Khat (Khat^T rows = key channel)
         if (tid == kMma) {
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq) {
                 const uint64_t adesc = dk(DT2 + kq * 32);
-                mma_bf16(tb + TM2_O, adesc, dk(so + R_AQK + kq * 32), ID_O, 1);
-                mma_bf16(tb + TM2_S, adesc, dm(so + R_KH + kq * 2048), ID_S, 1);
+                mma_bf16(tb + TM2_O, adesc, dk(so + R_AQK + kq * 32), ID2_OA, 1);
+                mma_bf16(tb + TM2_S, adesc, dk(so + R_KH + kq * 32), ID2_S, 1);
             }
             mma_commit(bar_mma);
             mma_out = true;
@@ -864,7 +998,7 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
         if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
         if (tid == kMma) mma_out = false;
         tc_fence_after();
-        {   // O^T (lane v, columns r) -> plain [r][v] tile over the consumed Qtil image
+        {   // O^T (lane v, columns r) -> plain [r][v] tile over the consumed Qtil^T image
             float x[16];
             const int v = 32 * quarter + lane, r0 = 16 * cgrp;
             tmem_ld16(tb + TM2_O + lane_sel + r0, x);
@@ -929,9 +1063,10 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
     }
 }
 
-// First global chunk of every sequence: chunk_off[n] = sum_{m<n} ceil(len_m / C),
-// chunk_off[N] = the total. One block; sequences in tiles of its size.
-__global__ void kda_tp_chunk_offsets(const int32_t *cu, int N, int *chunk_off) {
+// Chunk table of a varlen batch: chunk_off[n] = sum_{m<n} ceil(len_m / C) (the first
+// global chunk of sequence n; chunk_off[N] = the total) and, per global chunk, its
+// first token and number of valid rows. One block; sequences in tiles of its size.
+__global__ void kda_tp_chunk_table(const int32_t *cu, int N, int *chunk_off, int2 *chunk_tok) {
     __shared__ int warp_tot[32];
     __shared__ int carry;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
@@ -961,30 +1096,45 @@ __global__ void kda_tp_chunk_offsets(const int32_t *cu, int N, int *chunk_off) {
         }
         __syncthreads();
     }
+    // chunk_off is complete (written by this block before the barriers above)
+    for (int n = warp; n < N; n += nw) {
+        const int first = chunk_off[n], bos = cu[n], len = cu[n + 1] - bos;
+        const int nc = (len + C - 1) / C;
+        for (int ci = lane; ci < nc; ci += 32) chunk_tok[first + ci] = make_int2(bos + ci * C, min(C, len - ci * C));
+    }
 }
 
-// ---- workspace: [status 256 B][chunk offsets, 1024-aligned][records]
+// ---- workspace: [header 256 B: status word, exact-queue count][chunk offsets]
+// [chunk table][exact queue][records], every part 1024-aligned after the header
 long long max_chunks(const ChunkParams &p) {
     if (p.cu_seqlens) return ((long long)p.T + C - 1) / C + p.N;
     return (long long)p.N * (((long long)p.T + C - 1) / C);
 }
-size_t offsets_bytes(int N) { return (((size_t)(N + 1) * 4 + 1023) / 1024) * 1024; }
+size_t round1k(size_t b) { return (b + 1023) / 1024 * 1024; }
+size_t offsets_bytes(const ChunkParams &p) { return p.cu_seqlens ? round1k((size_t)(p.N + 1) * 4) : 0; }
+size_t table_bytes(const ChunkParams &p) { return p.cu_seqlens ? round1k((size_t)max_chunks(p) * 8) : 0; }
+size_t queue_bytes(const ChunkParams &p) { return round1k((size_t)max_chunks(p) * p.H * 4); }
 
 }  // namespace tp
 
 size_t chunk_2pass_workspace_bytes(const ChunkParams &p) {
     using namespace tp;
-    return 256 + offsets_bytes(p.N) + (size_t)max_chunks(p) * p.H * REC_BYTES;
+    return 256 + offsets_bytes(p) + table_bytes(p) + queue_bytes(p) + (size_t)max_chunks(p) * p.H * REC_BYTES;
 }
 
 cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int32_t *cu_host, cudaStream_t st) {
     using namespace tp;
     const long long total = p.cu_seqlens ? (long long)p.T : (long long)p.N * p.T;
     if (total <= 0) return cudaErrorInvalidValue;
+    const long long n_items = max_chunks(p) * p.H;
+    if (n_items >= (1LL << 31) || total >= (1LL << 31)) return cudaErrorInvalidValue;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *status = reinterpret_cast<int *>(ws);
+    int *fix_count = reinterpret_cast<int *>(ws + 64);
     int *chunk_off = reinterpret_cast<int *>(ws + 256);
-    uint8_t *rec = ws + 256 + offsets_bytes(p.N);
+    int2 *chunk_tok = reinterpret_cast<int2 *>(ws + 256 + offsets_bytes(p));
+    int *fix_list = reinterpret_cast<int *>(ws + 256 + offsets_bytes(p) + table_bytes(p));
+    uint8_t *rec = ws + 256 + offsets_bytes(p) + table_bytes(p) + queue_bytes(p);
     const int cpr = (int)(((long long)p.T + C - 1) / C);
 
     static_assert(sizeof(IntraParams) <= 4096 && sizeof(StateParams) <= 4096, "kernel parameter blocks");
@@ -992,9 +1142,14 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     memset(&A, 0, sizeof(A));
     A.p = p;
     A.rec = rec;
-    A.chunk_off = p.cu_seqlens ? chunk_off : nullptr;
+    A.chunk_tok = p.cu_seqlens ? chunk_tok : nullptr;
+    A.n_chunks = p.cu_seqlens ? chunk_off + p.N : nullptr;
     A.cpr = cpr;
-    A.n_items = max_chunks(p) * p.H;
+    A.n_items = n_items;
+    A.split_gate = (p.gate_mode == kGateLog && p.has_lb &&
+                    __bfloat162float(__float2bfloat16_rn(p.lb)) != p.lb) ? 1 : 0;
+    A.fix_count = fix_count;
+    A.fix_list = fix_list;
     A.status = status;
     if (!make_map(&A.tq, p.q, total, p.H) || !make_map(&A.tk, p.k, total, p.H) ||
         !make_map(&A.tg, p.g, total, p.H))
@@ -1004,7 +1159,7 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     memset(&B, 0, sizeof(B));
     B.p = p;
     B.rec = rec;
-    B.chunk_off = A.chunk_off;
+    B.chunk_off = p.cu_seqlens ? chunk_off : nullptr;
     B.cpr = cpr;
     B.status = status;
     if (!make_map(&B.tv, p.v, total, p.H)) return cudaErrorInvalidValue;
@@ -1019,10 +1174,10 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
         B.nperm = p.N;
     }
 
-    cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), st);
+    cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
     if (e != cudaSuccess) return e;
     if (p.cu_seqlens) {
-        kda_tp_chunk_offsets<<<1, 1024, 0, st>>>(p.cu_seqlens, p.N, chunk_off);
+        kda_tp_chunk_table<<<1, 1024, 0, st>>>(p.cu_seqlens, p.N, chunk_off, chunk_tok);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     int dev = 0, nsm = 148;
@@ -1030,8 +1185,12 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_tp_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM1_ALLOC);
     if (e != cudaSuccess) return e;
-    const long long grid1 = std::min<long long>(A.n_items, 2LL * nsm);
+    const long long grid1 = std::min<long long>(n_items, 2LL * nsm);
     kda_tp_intra_kernel<<<(unsigned)grid1, NT1, SMEM1_ALLOC, st>>>(A);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kda_tp_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEMX_BYTES);
+    if (e != cudaSuccess) return e;
+    kda_tp_exact_kernel<<<(unsigned)std::min<long long>(n_items, nsm), NTX, SMEMX_BYTES, st>>>(A);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_tp_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2_ALLOC);
     if (e != cudaSuccess) return e;

@@ -162,8 +162,10 @@ def test_chunk_size_rule():
     torch.testing.assert_close(S32, S64, rtol=1e-5, atol=1e-5)
 
 
-@pytest.mark.parametrize("lb", [None, -5.0, -0.5])
+@pytest.mark.parametrize("lb", [None, -5.0, -0.5, -0.3, -2.7])
 def test_chunk_lower_bound(lb):
+    """Bounds that are bf16 values and bounds that are not (-0.3, -2.7: the clamped
+    gate then carries a low-order part into the in-chunk sum)."""
     inp = KI.draw_chunk(1, 200, 2, 128, 128, dtype=torch.bfloat16, seed=5, init_state=True)
     o, S = run_chunk(inp, lower_bound=lb)
     compare_chunk(inp, o, S, torch.bfloat16, lower_bound=lb, tag=f"lb{lb}")
