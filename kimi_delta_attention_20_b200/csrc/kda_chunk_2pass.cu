@@ -57,11 +57,14 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 
 // ---- record of one (chunk, head), bytes; every tile is a shared-memory image
 // with the 128-byte swizzle (16-byte chunk index XOR row % 8, rows of 128 B)
-constexpr uint32_t R_WT = 0;        // W^T    [128 c][64 r]: B of S^T W^T, N = r contiguous (MN-major)
-constexpr uint32_t R_QT = 16384;    // Qtil^T [128 c][64 r]: B of S^T Qtil^T, MN-major
+// Pass 2 reads [Qtil^T | -W^T] as one N = 128 operand and [Khat^T ; A_qk] as one
+// N = 192 operand, so those tiles are adjacent.
+constexpr uint32_t R_QT = 0;        // Qtil^T [128 c][64 r]: B of S^T Qtil^T, N = r contiguous (MN-major)
+constexpr uint32_t R_WT = 16384;    // -W^T   [128 c][64 r]: B of S^T (-W^T), MN-major
 constexpr uint32_t R_KH = 32768;    // Khat^T [128 c][64 s]: B of D~^T Khat, K = s contiguous (K-major)
-constexpr uint32_t R_TPU = 49152;   // T' = T diag(beta) [64 r][64 s], K-major B
-constexpr uint32_t R_AQK = 57344;   // A_qk (raw rows) [64 r][64 s], K-major B
+constexpr uint32_t R_AQK = 49152;   // A_qk (raw rows) [64 r][64 s], K-major B
+constexpr uint32_t R_TPU = 57344;   // T' = T diag(beta) [64 r][64 s], K-major B
+static_assert(R_WT - R_QT == 16384 && R_AQK == R_KH + 16384, "operand groups of pass 2 are adjacent");
 constexpr uint32_t R_MISC = 65536;  // f32: e^{G_last}[128], 1/|q_r|[64], 1/|k_s|[64]
 constexpr uint32_t R_GAM = R_MISC, R_INVQ = R_MISC + 512, R_INVK = R_MISC + 768;
 constexpr uint32_t REC_BYTES = R_MISC + 1024;
@@ -72,19 +75,20 @@ constexpr int NT1 = 256;  // 8 warps, two CTAs per SM
 // Shared memory (bytes from a 1024-aligned base). Phases reuse regions:
 //   inputs      KQ: 2 channel halves x [128 rows: k tokens 0..63, q tokens 0..63][128 B]
 //               GS: 2 channel halves x [64 tokens][128 B] (the gate)
-//               TRI, IDT: [64][64] bf16 constant tiles; GLO: low part of a split gate
+//               TRI, IDT: [64][64] bf16 constant tiles (bulk-copied with the inputs);
+//               GLO: low part of a split gate
 //   operands    XK, XQ: X^T images [128 c][64 r] of k e^{G-G_m}, q e^{G-G_m}
 //               YT: Y^T [128 c][64 s] of k e^{G_m-G};  YP: Y'^T of k e^{G_47-G} (s < 32)
 //               QT, KH: the record's Qtil^T and Khat^T images
-//   inverse     LF: fp32 L [64][65];  TF: fp32 T [64][68];  TW: bf16 T diag(beta/|k|)
+//   inverse     LF: fp32 L [64][68];  TF: fp32 T [64][72];  TW: bf16 T diag(beta/|k|)
 //               AQK, TPU: the record's A_qk and T' images;  WT: the record's W^T image
 constexpr uint32_t KQ = 0, GS = 32768;
 constexpr uint32_t XK = 0, XQ = 16384, YT = 32768;
 constexpr uint32_t R2 = 49152;
 constexpr uint32_t TRI = R2, IDT = R2 + 8192, GLO = R2 + 16384;
 constexpr uint32_t QT = R2, KH = R2 + 16384, YP = R2 + 32768;
-constexpr int LDS = 65, LDT = 68;
-constexpr uint32_t LF = 16384, TF = 33792, TW = 51200;
+constexpr int LDS = 68, LDT = 72;  // row strides (floats) of L and T: 16-byte rows, fragment loads conflict-free
+constexpr uint32_t LF = 16384, TF = 33792, TW = 53248;
 constexpr uint32_t AQK = YP, TPU = YP + 8192, WT = KH;
 constexpr uint32_t MISC1 = 98304;
 constexpr uint32_t M1_REC = MISC1,           // record misc image: gamma[128], invq[64], invk[64]
@@ -99,12 +103,14 @@ static_assert(LF + 64 * LDS * 4 <= TF && TF + 64 * LDT * 4 <= TW && TW + 8192 <=
 static_assert(TW % 1024 == 0 && AQK % 1024 == 0 && TPU % 1024 == 0 && TPU + 8192 == MISC1, "tile alignment");
 static_assert(2 * (SMEM1_ALLOC + 1024) <= 233472, "two CTAs per SM");
 
-// tensor memory (256 columns): G^T, k^T, q^T; then the A products; then W in two K halves
+// tensor memory (256 columns): G^T, k^T, q^T; then the A products (one N = 128 product
+// against [Y | Y']: D1 in columns 0..63, D2 in 64..127); then W in two K halves
 constexpr uint32_t TM_G = 0, TM_K = 64, TM_Q = 128;
 constexpr uint32_t TM_A1 = 0, TM_A2 = 64, TM_W0 = 128, TM_W1 = 192, TM1_COLS = 256;
+static_assert(YP - YT == 49152, "Y and Y' are the two N groups of one operand (LBO 48 KB)");
 
 constexpr uint32_t ID_T = idesc_bf16(128, 64, true, false);   // g^T Tri^T, k^T I, q^T I
-constexpr uint32_t ID_A = idesc_bf16(128, 64, true, true);    // [X_k; X_q] Y^T and Y'^T
+constexpr uint32_t ID_A = idesc_bf16(128, 128, true, true);   // [X_k; X_q] [Y | Y']^T
 constexpr uint32_t ID_W = idesc_bf16(128, 64, false, false);  // X_k^T T_w^T
 
 struct IntraParams {
@@ -116,6 +122,7 @@ struct IntraParams {
     int cpr;                 // batch: chunks per batch row
     long long n_items;       // upper bound of (global chunk, head) items
     int split_gate;          // the clamped gate needs a low bf16 part (bound not a bf16 value)
+    const uint8_t *consts;   // the Tri and I tile images (16 KB, written by kda_tp_prep)
     int *fix_count;          // items whose gate span needs the exact kernel
     int *fix_list;
     int *status;
@@ -128,26 +135,29 @@ struct Item {
     long long gc;  // global chunk index
 };
 
-// (global chunk, head) of flat item index `item` -> the chunk's tokens; false past the end
-__device__ __forceinline__ bool decode_item(const IntraParams &P, long long item, int nch, Item &it) {
+// The chunk's tokens of work item (global chunk gc, head h); false past the end
+__device__ __forceinline__ bool decode_chunk(const IntraParams &P, long long gc, int h, int nch, Item &it) {
     const ChunkParams &p = P.p;
-    if (item >= P.n_items) return false;
-    const long long gc = item / p.H;
-    it.h = (int)(item % p.H);
+    it.h = h;
     it.gc = gc;
     if (P.chunk_tok) {
         if (gc >= nch) return false;
         const int2 e = P.chunk_tok[gc];
         it.t0 = e.x;
         it.L = e.y;
-    } else {
-        const long long n = gc / P.cpr;
-        if (n >= p.N) return false;
-        const int ci = (int)(gc % P.cpr);
-        it.t0 = (int)(n * p.T) + ci * C;
+    } else {  // gc < 2^31 (checked on the host): 32-bit division
+        const unsigned n = (unsigned)gc / (unsigned)P.cpr;
+        if ((int)n >= p.N) return false;
+        const int ci = (int)((unsigned)gc - n * (unsigned)P.cpr);
+        it.t0 = (int)n * p.T + ci * C;
         it.L = min(C, p.T - ci * C);
     }
     return it.L > 0;
+}
+// (global chunk, head) of flat item index `item` (= gc * H + h)
+__device__ __forceinline__ bool decode_item(const IntraParams &P, long long item, int nch, Item &it) {
+    if (item >= P.n_items) return false;
+    return decode_chunk(P, item / P.p.H, (int)(item % P.p.H), nch, it);
 }
 
 // 8 bf16 of an unpacked register pair set -> one 16-byte chunk
@@ -157,9 +167,10 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const ChunkParams &p = P.p;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);  // warp-uniform by construction
     const int H = p.H;
-    constexpr int kMma = 0, kTma = NT1 - 32;
+    constexpr int kMma = 0, kTma = NT1 - 32;  // warp 0 issues the MMAs, thread kTma the copies
     constexpr float kL2e = 1.4426950408889634f;
 
     uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + M1_BAR);
@@ -187,14 +198,17 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
     const uint32_t sb = smem_u32(sm);
     // 128-byte-swizzled operand at `off`: K-major (lbo unused) or MN-major (lbo = step
     // between 64-element groups along M/N); 8-row groups 1024 bytes apart
-    auto desc = [&](uint32_t off, uint32_t lbo) { return sdesc_sw128(sb + off, lbo, 1024); };
+    const uint64_t dK = sdesc_sw128(sb, 16, 1024), dA8 = sdesc_sw128(sb, 8192, 1024),
+                   dA16 = sdesc_sw128(sb, 16384, 1024), dYY = sdesc_sw128(sb, YP - YT, 1024);
+    auto desc = [&](uint32_t off, uint32_t lbo) {
+        return (lbo == 16 ? dK : lbo == 8192 ? dA8 : dA16) + (uint64_t)(off >> 4);
+    };
     // channel layout: thread (quarter, hw) owns key channel c (tensor-memory lane c)
     // and rows 32 hw .. 32 hw + 31; hw also splits columns in the row-layout phases
     const int quarter = warp & 3, hw = warp >> 2;
     const int c = 32 * quarter + lane;
     const uint32_t lane_sel = (uint32_t)(32 * quarter) << 16;
     const int gmode = p.gate_mode;
-    const __nv_bfloat16 *bt = static_cast<const __nv_bfloat16 *>(p.beta);
     const int nch = P.chunk_tok ? *P.n_chunks : 0;
 
     uint32_t ph_in = 0, ph_mma = 0;
@@ -206,7 +220,8 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
         return __syncthreads_or(!ok) != 0;
     };
     auto issue_in = [&](const Item &it) {
-        mbar_arrive_expect_tx(bar_in, 3 * 16384);
+        mbar_arrive_expect_tx(bar_in, 4 * 16384);
+        bulk_load(sm + TRI, P.consts, 16384, bar_in);
         for (int hf = 0; hf < 2; ++hf) {
             tma_load_3d(sm + KQ + hf * 16384, &P.tk, bar_in, hf * 64, it.h, it.t0);
             tma_load_3d(sm + KQ + hf * 16384 + 8192, &P.tq, bar_in, hf * 64, it.h, it.t0);
@@ -214,37 +229,40 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
         }
     };
 
+    // raw bits: the load is consumed (converted) only when the item starts
+    const unsigned short *bt16 = reinterpret_cast<const unsigned short *>(p.beta);
+    auto load_beta = [&](const Item &it) -> unsigned short {
+        return tid < it.L ? bt16[((long long)it.t0 + tid) * H + it.h] : (unsigned short)0;
+    };
+
+    // items blockIdx.x + k gridDim.x, walked as (global chunk, head) with the stride split once
+    const int step_h = (int)(gridDim.x % H);
+    const long long step_c = gridDim.x / H;
     long long item = blockIdx.x;
     Item cur;
     bool have = decode_item(P, item, nch, cur);
     if (have && tid == kTma) { issue_in(cur); in_out = true; }
+    unsigned short beta_raw = (have && tid < C) ? load_beta(cur) : (unsigned short)0;
 
     while (have) {
         const long long nitem = item + gridDim.x;
         Item nxt;
-        const bool have_next = decode_item(P, nitem, nch, nxt);
-        const int h = cur.h, L = cur.L, t0 = cur.t0;
+        bool have_next = false;
+        if (nitem < P.n_items) {
+            int nh = cur.h + step_h;
+            long long ngc = cur.gc + step_c;
+            if (nh >= H) { nh -= H; ++ngc; }
+            have_next = decode_chunk(P, ngc, nh, nch, nxt);
+        }
+        const int h = cur.h, L = cur.L;
         uint8_t *rec = P.rec + (cur.gc * H + h) * (long long)REC_BYTES;
 
-        // ---------------- per-item scalars and the constant tiles Tri (s <= r) and I
-        if (tid < C) {
-            const float b = tid < L ? __bfloat162float(bt[((long long)t0 + tid) * H + h]) : 0.f;
-            sbeta[tid] = tid < L ? beta_value(b, p.beta_prob) : 0.f;
-        }
+        // ---------------- per-item scalars (beta was loaded one item ahead)
+        if (tid < C) sbeta[tid] = tid < L ? beta_value(__uint_as_float((uint32_t)beta_raw << 16), p.beta_prob) : 0.f;
         const float rate = gmode != kGateLog ? expf(p.A_log[h]) : 0.f;
         if (gmode != kGateLog && tid < D) sDtb[tid] = p.dt_bias ? p.dt_bias[h * D + tid] : 0.f;
         // the previous item's record stores must have read their sources (GLO, misc)
         if (tid == kTma) bulk_wait_read_all();
-        for (int e = tid; e < 2 * 64 * 8; e += NT1) {
-            const int tile = e >> 9, r = (e >> 3) & 63, j = e & 7;
-            float v[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int s = 8 * j + q;
-                v[q] = tile ? (s == r ? 1.f : 0.f) : (s <= r ? 1.f : 0.f);
-            }
-            sts128(sm, (tile ? IDT : TRI) + sw128_chunk(r, 8 * j, 64), pack8(v));
-        }
         if (wait_all(bar_in, ph_in)) { aborted = true; break; }
         if (tid == kTma) in_out = false;
 
@@ -271,7 +289,17 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
         // part when the bound is not a bf16 value), or the in-kernel gate forms summed in
         // fp32 on the CUDA cores straight into tensor memory
         if (gmode == kGateLog) {
-            if (p.has_lb) {
+            if (p.has_lb && !P.split_gate) {
+                const __nv_bfloat162 lb2 = __float2bfloat162_rn(p.lb);
+#pragma unroll
+                for (int e = tid; e < 1024; e += NT1) {
+                    uint4 u = lds128(sm + GS, e * 16);
+                    __nv_bfloat162 *b2 = reinterpret_cast<__nv_bfloat162 *>(&u);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) b2[q] = __hmax2(b2[q], lb2);
+                    sts128(sm, GS + e * 16, u);
+                }
+            } else if (p.has_lb) {
                 for (int e = tid; e < 1024; e += NT1) {
                     float2 f[4], hi[4], lo[4];
                     unpack8x2(lds128(sm + GS, e * 16), f);
@@ -283,7 +311,7 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
                         lo[q] = make_float2(v.x - hi[q].x, v.y - hi[q].y);
                     }
                     sts128(sm, GS + e * 16, pack8x2(hi));
-                    if (P.split_gate) sts128(sm, GLO + e * 16, pack8x2(lo));
+                    sts128(sm, GLO + e * 16, pack8x2(lo));
                 }
             }
         } else {
@@ -313,24 +341,25 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
         tc_fence_after();
 
         // ---------------- tensor core: G^T = g^T Tri^T, k^T = k^T I, q^T = q^T I (lane = channel)
-        if (tid == kMma) {
+        if (warp == 0) {
+            const uint32_t ld = elect_one();
             if (gmode == kGateLog) {
 #pragma unroll
                 for (int kq = 0; kq < 4; ++kq)
-                    mma_bf16(tb + TM_G, desc(GS + kq * 2048, 8192), desc(TRI + kq * 32, 16), ID_T, kq > 0);
+                    mma_bf16_by(ld, tb + TM_G, desc(GS + kq * 2048, 8192), desc(TRI + kq * 32, 16), ID_T, kq > 0);
                 if (p.has_lb && P.split_gate) {
 #pragma unroll
                     for (int kq = 0; kq < 4; ++kq)
-                        mma_bf16(tb + TM_G, desc(GLO + kq * 2048, 8192), desc(TRI + kq * 32, 16), ID_T, 1);
+                        mma_bf16_by(ld, tb + TM_G, desc(GLO + kq * 2048, 8192), desc(TRI + kq * 32, 16), ID_T, 1);
                 }
             }
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq)
-                mma_bf16(tb + TM_K, desc(KQ + kq * 2048, 16384), desc(IDT + kq * 32, 16), ID_T, kq > 0);
+                mma_bf16_by(ld, tb + TM_K, desc(KQ + kq * 2048, 16384), desc(IDT + kq * 32, 16), ID_T, kq > 0);
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq)
-                mma_bf16(tb + TM_Q, desc(KQ + 8192 + kq * 2048, 16384), desc(IDT + kq * 32, 16), ID_T, kq > 0);
-            mma_commit(bar_mma);
+                mma_bf16_by(ld, tb + TM_Q, desc(KQ + 8192 + kq * 2048, 16384), desc(IDT + kq * 32, 16), ID_T, kq > 0);
+            mma_commit_by(ld, bar_mma);
             mma_out = true;
         }
         // row norms of k and q from the staged rows while the products run: four
@@ -358,7 +387,7 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
             }
         }
         if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
-        if (tid == kMma) mma_out = false;
+        if (warp == 0) mma_out = false;
         tc_fence_after();
 
         // ---------------- operands, channel layout: thread (c, hw) turns its 32 rows of
@@ -403,7 +432,7 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
                         const float2 a = __ffma2_rn(g2, l2e2, nb);
                         amax = fmaxf(amax, fmaxf(fabsf(a.x), fabsf(a.y)));
                         const float2 ed = make_float2(ex2a(a.x), ex2a(a.y));
-                        const float2 yd = make_float2(ex2a(-a.x), ex2a(-a.y));
+                        const float2 yd = rcp2_nr(ed);  // e^{G_m - G} on the FMA pipe (ed >= 2^-116 here)
                         xk[j] = __fmul2_rn(k2, ed);
                         xq[j] = __fmul2_rn(q2, ed);
                         y[j] = __fmul2_rn(k2, yd);
@@ -439,18 +468,17 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
 
         // ---------------- A products: D1 = [X_k; X_q] Y^T (diagonal 32-blocks valid),
         // D2 = [X_k; X_q] Y'^T (rows 32..63 against columns 0..31 valid)
-        if (tid == kMma) {
+        if (warp == 0) {
+            const uint32_t ld = elect_one();
 #pragma unroll
-            for (int kq = 0; kq < 8; ++kq) {
-                const uint64_t a = desc(XK + kq * 2048, 16384);
-                mma_bf16(tb + TM_A1, a, desc(YT + kq * 2048, 8192), ID_A, kq > 0);
-                mma_bf16(tb + TM_A2, a, desc(YP + kq * 2048, 8192), ID_A, kq > 0);
-            }
-            mma_commit(bar_mma);
+            for (int kq = 0; kq < 8; ++kq)
+                mma_bf16_by(ld, tb + TM_A1, desc(XK + kq * 2048, 16384), dYY + (uint64_t)((YT + kq * 2048) >> 4), ID_A,
+                            kq > 0);
+            mma_commit_by(ld, bar_mma);
             mma_out = true;
         }
         if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
-        if (tid == kMma) mma_out = false;
+        if (warp == 0) mma_out = false;
         tc_fence_after();
 
         // ---------------- read-back, row layout (lane = row): L = beta_r |k_r|^-1 |k_s|^-1 A_kk
@@ -517,9 +545,16 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
 #pragma unroll
                 for (int i = 0; i < 16; ++i) t[i] = i == j ? 1.f : 0.f;
 #pragma unroll
-                for (int k = 0; k < 15; ++k) {
+                for (int i = 1; i < 16; ++i) {  // row i of the block: t[i] -= sum_{k<i} L[i][k] t[k]
+                    const float *Lr = Lf + (16 * b + i) * LDS + 16 * b;
 #pragma unroll
-                    for (int i = k + 1; i < 16; ++i) t[i] = fmaf(-Lf[(16 * b + i) * LDS + 16 * b + k], t[k], t[i]);
+                    for (int k4 = 0; k4 < i; k4 += 4) {
+                        const float4 l4 = *reinterpret_cast<const float4 *>(Lr + k4);
+                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            if (k4 + u < i) t[i] = fmaf(-lv[u], t[k4 + u], t[i]);
+                    }
                 }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) Tf[(16 * b + i) * LDT + 16 * b + j] = t[i];
@@ -618,12 +653,13 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
 
         // ---------------- W^T = X_k^T T_w^T in two K halves (token blocks 0..31, 32..63, each
         // with its own block reference), recombined per key channel at read-back
-        if (tid == kMma) {
+        if (warp == 0) {
+            const uint32_t ld = elect_one();
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq)
-                mma_bf16(tb + (kq < 2 ? TM_W0 : TM_W1), desc(XK + kq * 32, 16), desc(TW + kq * 32, 16), ID_W,
-                         (kq & 1) != 0);
-            mma_commit(bar_mma);
+                mma_bf16_by(ld, tb + (kq < 2 ? TM_W0 : TM_W1), desc(XK + kq * 32, 16), desc(TW + kq * 32, 16), ID_W,
+                            (kq & 1) != 0);
+            mma_commit_by(ld, bar_mma);
             mma_out = true;
         }
         if (tid == kTma) {
@@ -631,12 +667,13 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
             bulk_store(rec + R_TPU, sm + TPU, 8192);
             bulk_commit();
         }
+        if (tid < C) beta_raw = have_next ? load_beta(nxt) : (unsigned short)0;  // consumed by the next item
         if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
-        if (tid == kMma) mma_out = false;
+        if (warp == 0) mma_out = false;
         tc_fence_after();
         // the input area is free again: the next item's inputs load during the read-back
         if (tid == kTma && have_next) { issue_in(nxt); in_out = true; }
-        {   // thread (c, hw): W^T[c][r], r = 32 hw .., = e^{G_15} W0 + e^{G_47} W1
+        {   // thread (c, hw): -W^T[c][r], r = 32 hw .., = -(e^{G_15} W0 + e^{G_47} W1)
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int r0 = 32 * hw + 16 * u;
@@ -645,7 +682,7 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
                 tmem_ld16(tb + lane_sel + TM_W1 + r0, w1);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) w0[j] = fmaf(e15, w0[j], e47 * w1[j]);
+                for (int j = 0; j < 16; ++j) w0[j] = -fmaf(e15, w0[j], e47 * w1[j]);
                 sts128(sm, WT + c * 128 + (((r0 >> 3) ^ (c & 7)) << 4), pack8(w0));
                 sts128(sm, WT + c * 128 + ((((r0 >> 3) + 1) ^ (c & 7)) << 4), pack8(w0 + 8));
             }
@@ -683,7 +720,8 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
 // Rewrites the record of every queued (chunk, head) on CUDA cores in fp32 from
 // exponent differences that are never positive (gate <= 0), so no factor can
 // overflow whatever the gate: A_kk and A_qk term by term, T by row-wise forward
-// substitution, W = T diag(beta/|k|) (k e^G), Qtil = q e^G, Khat = k e^{G_last-G}.
+// substitution, W = T diag(beta/|k|) (k e^G) (stored negated), Qtil = q e^G,
+// Khat = k e^{G_last-G}.
 constexpr int NTX = 256;
 constexpr int LDX = 65;
 constexpr uint32_t X_Q = 0, X_K = 32768, X_G = 65536;           // fp32 [64][128]
@@ -806,7 +844,7 @@ __global__ void __launch_bounds__(NTX, 1) kda_tp_exact_kernel(const __grid_const
             const int cc = e & 127, r = e >> 7;
             float w = 0.f;
             for (int s = 0; s <= r; ++s) w = fmaf(Tm[r * LDX + s] * sbeta[s] * sinvk[s], kf[s * D + cc], w);
-            *reinterpret_cast<__nv_bfloat16 *>(rec + R_WT + sw128(cc, r, 128)) = __float2bfloat16_rn(w);
+            *reinterpret_cast<__nv_bfloat16 *>(rec + R_WT + sw128(cc, r, 128)) = __float2bfloat16_rn(-w);
         }
         float *misc = reinterpret_cast<float *>(rec + R_MISC);
         if (tid < D) misc[tid] = expf(Gf[(C - 1) * D + tid]);
@@ -816,23 +854,36 @@ __global__ void __launch_bounds__(NTX, 1) kda_tp_exact_kernel(const __grid_const
 }
 
 // ============================================================== pass 2
-constexpr int NT2 = 512;  // 16 warps, one CTA per SM
+// One CTA per (sequence, head), 16 warps in two groups:
+//   warps 0..7 (the state chain): per chunk, a bf16 copy of S^T for the products
+//     and the decayed state written back; [O^T | D^T] = S^T [Qtil^T | -W^T] and
+//     D^T += V^T T'^T; D~^T = D^T diag(|k|^-1) to shared memory; S^T += D~^T Khat
+//     (its own commit, which the next chunk waits for) and O^T += D~^T A_qk^T;
+//   warps 8..15 (output): one chunk behind, read O^T, let the consumed stage be
+//     refilled two chunks ahead, and write the output rows.
+// O^T and D^T are double-buffered in tensor memory, so the output work of chunk i
+// overlaps the state chain of chunk i + 1.
+constexpr int NT2 = 512;
+constexpr int kGroup = 256;  // threads per warp group
 constexpr uint32_t STAGE_BYTES = REC_BYTES + 16384;  // record image + v tile
 constexpr uint32_t S_V = REC_BYTES;                  // v tile [64 r][128 v] as two halves (MN-major A)
 constexpr uint32_t ST2 = 2 * STAGE_BYTES;            // bf16 S^T [128 v][128 c], K-major A (halves 16 KiB apart)
 constexpr uint32_t DT2 = ST2 + 32768;                // bf16 D~^T [128 v][64 s], K-major A
 constexpr uint32_t MISC2 = DT2 + 16384;
-constexpr uint32_t M2_BAR = MISC2, M2_TMEM = MISC2 + 32;
-constexpr uint32_t SMEM2_BYTES = MISC2 + 64;
+constexpr uint32_t M2_BAR = MISC2, M2_TMEM = MISC2 + 96;
+constexpr uint32_t SMEM2_BYTES = MISC2 + 128;
 constexpr uint32_t SMEM2_ALLOC = SMEM2_BYTES + 1024;
 static_assert(STAGE_BYTES % 1024 == 0 && SMEM2_ALLOC <= 232448, "pass 2 shared memory");
 
-constexpr uint32_t TM2_S = 0, TM2_D = 128, TM2_O = 192, TM2_COLS = 256;
-constexpr uint32_t ID2_UW = idesc_bf16(128, 64, true, false);           // V^T T'^T
-constexpr uint32_t ID2_DL = idesc_bf16(128, 64, false, true, true);     // - S^T W^T
-constexpr uint32_t ID2_OQ = idesc_bf16(128, 64, false, true);           // S^T Qtil^T
-constexpr uint32_t ID2_OA = idesc_bf16(128, 64, false, false);          // D~^T A_qk^T
-constexpr uint32_t ID2_S = idesc_bf16(128, 128, false, false);          // D~^T Khat
+// tensor memory (512 columns): S^T, then per buffer b: O^T at 128 + 128 b and D^T
+// right after it, so [O^T | D^T] is the accumulator of one N = 128 product
+constexpr uint32_t TM2_S = 0, TM2_COLS = 512;
+__host__ __device__ constexpr uint32_t tm2_o(int b) { return 128 + 128 * b; }
+__host__ __device__ constexpr uint32_t tm2_d(int b) { return 192 + 128 * b; }
+constexpr uint32_t ID2_QW = idesc_bf16(128, 128, false, true);  // S^T [Qtil^T | -W^T]
+constexpr uint32_t ID2_UW = idesc_bf16(128, 64, true, false);   // + V^T T'^T
+constexpr uint32_t ID2_KS = idesc_bf16(128, 128, false, false); // D~^T Khat
+constexpr uint32_t ID2_KA = idesc_bf16(128, 64, false, false);  // D~^T A_qk^T
 constexpr int kMaxPerm = 256;
 
 struct StateParams {
@@ -850,7 +901,8 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const ChunkParams &p = P.p;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);  // warp-uniform by construction
     const int H = p.H;
     const int rank = blockIdx.x / H, h = blockIdx.x % H;
     const int n = rank < P.nperm ? P.perm[rank] : rank;
@@ -858,15 +910,19 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
     if (p.cu_seqlens) { bos = p.cu_seqlens[n]; eos = p.cu_seqlens[n + 1]; c_first = P.chunk_off[n]; }
     else { bos = (long long)n * p.T; eos = bos + p.T; c_first = (long long)n * P.cpr; }
     const int nchunks = (int)((eos - bos + C - 1) / C);
-    constexpr int kMma = 0, kTma = NT2 - 32;
+    constexpr int kTma = kGroup;  // first thread of the output group issues the stage copies
 
-    uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + M2_BAR);  // [2]
-    uint64_t *bar_mma = bar_full + 2;
+    uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + M2_BAR);  // [2] stage s loaded
+    uint64_t *bar_m1 = bar_full + 2;                                 // first products done
+    uint64_t *bar_s = bar_full + 3;                                  // state update done
+    uint64_t *bar_o = bar_full + 4;                                  // [2] O^T buffer b complete
+    uint64_t *bar_of = bar_full + 6;                                 // [2] O^T buffer b read
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + M2_TMEM);
 
     if (warp == 0) { tmem_alloc(s_tmem, TM2_COLS); tmem_relinquish(); }
     if (tid == 32) {
-        mbar_init(bar_full, 1); mbar_init(bar_full + 1, 1); mbar_init(bar_mma, 1);
+        for (int i = 0; i < 6; ++i) mbar_init(bar_full + i, 1);
+        mbar_init(bar_of, kGroup); mbar_init(bar_of + 1, kGroup);
         fence_mbar_init();
         tma_prefetch_desc(&P.tv);
     }
@@ -877,21 +933,16 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
     const uint32_t sb = smem_u32(sm);
     const uint64_t dK = sdesc_sw128(sb, 16, 1024);    // K-major operands
     const uint64_t dM = sdesc_sw128(sb, 8192, 1024);  // MN-major operands (atoms 8 KiB apart)
+    const uint64_t dQW = sdesc_sw128(sb, R_WT - R_QT, 1024);  // [Qtil^T | -W^T], groups 16 KiB apart
     auto dk = [&](uint32_t off) { return dK + (uint64_t)(off >> 4); };
     auto dm = [&](uint32_t off) { return dM + (uint64_t)(off >> 4); };
     const int quarter = warp & 3;
     const uint32_t lane_sel = (uint32_t)(32 * quarter) << 16;
-    const int cgrp = warp >> 2;  // 0..3
+    const int v = 32 * quarter + lane;   // value channel = tensor-memory lane of this thread
+    const int half = (warp >> 2) & 1;    // column half within the group
 
-    uint32_t ph_full = 0, ph_mma = 0;  // bit s: parity of stage s's next phase
-    uint32_t full_out = 0;             // bit s: stage s has copies in flight
-    bool mma_out = false, aborted = false;
-    auto wait_all = [&](uint64_t *bar, uint32_t &ph) -> bool {
-        bool ok = true;
-        if (warp == 0) ok = mbar_wait(bar, ph, kWaitLimitNs);
-        ph ^= 1;
-        return __syncthreads_or(!ok) != 0;
-    };
+    uint32_t full_out = 0;  // stage copies in flight (thread kTma)
+    bool aborted = false;
     auto issue_stage = [&](int ci) {
         const int s = ci & 1;
         uint8_t *dst = sm + s * STAGE_BYTES;
@@ -906,154 +957,176 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
         if (nchunks > 0) issue_stage(0);
         if (nchunks > 1) issue_stage(1);
     }
-
     const long long sbase_state = ((long long)n * H + h) * D * D;
-    for (int ci = 0; ci < nchunks && !aborted; ++ci) {
-        const int s = ci & 1;
-        uint8_t *stg = sm + s * STAGE_BYTES;
-        const float *gam = reinterpret_cast<const float *>(stg + R_GAM);
-        const float *invq = reinterpret_cast<const float *>(stg + R_INVQ);
-        const float *invk = reinterpret_cast<const float *>(stg + R_INVK);
-        const long long t0 = bos + (long long)ci * C;
-        const int L = (int)((eos - t0) < C ? (eos - t0) : C);
-        {
-            uint32_t ph = (ph_full >> s) & 1u;
-            ph_full ^= 1u << s;
-            if (wait_all(bar_full + s, ph)) { aborted = true; break; }
-        }
-        if (tid == kTma) full_out &= ~(1u << s);
 
-        // ---------------- state refresh: bf16 copy of S^T for this chunk's products, and
-        // S^T diag(e^{G_last}) back into tensor memory for the update product
-        {
-            const int v = 32 * quarter + lane;
-            const int c0 = 32 * cgrp;
-            float x[32];
-            if (ci == 0) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) x[j] = p.S0 ? p.S0[sbase_state + (long long)(c0 + j) * D + v] : 0.f;
-            } else {
-                tmem_ld32(tb + TM2_S + lane_sel + c0, x);
-                tmem_ld_wait();
+    if (warp < 8) {
+        // ================= the state chain
+        int issued = -1;  // last chunk whose products were issued (warp 0)
+        for (int ci = 0; ci < nchunks; ++ci) {
+            const int s = ci & 1, b = ci & 1;
+            uint8_t *stg = sm + s * STAGE_BYTES;
+            const uint32_t so = s * STAGE_BYTES;
+            {
+                bool ok = true;
+                if (warp == 0) {
+                    ok = mbar_wait(bar_full + s, (ci >> 1) & 1, kWaitLimitNs);
+                    if (ok && ci > 0) ok = mbar_wait(bar_s, (ci - 1) & 1, kWaitLimitNs);
+                }
+                if (bar_or(1, kGroup, !ok)) { aborted = true; break; }
             }
+            tc_fence_after();
+            // bf16 copy of S^T for the products; the decayed S^T diag(e^{G_last}) back into
+            // tensor memory (the update product accumulates onto it)
+            const float *gam = reinterpret_cast<const float *>(stg + R_GAM);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) sts128(sm, ST2 + sw128_chunk(v, c0 + 8 * q4, 128), pack8(x + 8 * q4));
+            for (int jc = 0; jc < 2; ++jc) {
+                const int c0 = 64 * half + 32 * jc;
+                float x[32];
+                if (ci == 0) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                const float2 v2 = __fmul2_rn(make_float2(x[j], x[j + 1]),
-                                             *reinterpret_cast<const float2 *>(gam + c0 + j));
-                x[j] = v2.x; x[j + 1] = v2.y;
+                    for (int j = 0; j < 32; ++j) x[j] = p.S0 ? p.S0[sbase_state + (long long)(c0 + j) * D + v] : 0.f;
+                } else {
+                    tmem_ld32(tb + TM2_S + lane_sel + c0, x);
+                    tmem_ld_wait();
+                }
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) sts128(sm, ST2 + sw128_chunk(v, c0 + 8 * q4, 128), pack8(x + 8 * q4));
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    const float2 v2 = __fmul2_rn(make_float2(x[j], x[j + 1]),
+                                                 *reinterpret_cast<const float2 *>(gam + c0 + j));
+                    x[j] = v2.x; x[j + 1] = v2.y;
+                }
+                tmem_st32(tb + TM2_S + lane_sel + c0, x);
             }
-            tmem_st32(tb + TM2_S + lane_sel + c0, x);
             tmem_st_wait();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            bar_sync(1, kGroup);
+            tc_fence_after();
 
-        // ---------------- D^T = V^T T'^T - S^T W^T ; O^T = S^T Qtil^T
-        const uint32_t so = s * STAGE_BYTES;
-        if (tid == kMma) {
+            // [O^T | D^T] = S^T [Qtil^T | -W^T], then D^T += V^T T'^T
+            if (warp == 0) {
+                bool ok = true;
+                if (ci >= 2) ok = mbar_wait(bar_of + b, ((ci - 2) >> 1) & 1, kWaitLimitNs);  // O^T buffer read
+                if (ok) {
+                    const uint32_t ld = elect_one();
 #pragma unroll
-            for (int kq = 0; kq < 4; ++kq)
-                mma_bf16(tb + TM2_D, dm(so + S_V + kq * 2048), dk(so + R_TPU + kq * 32), ID2_UW, kq > 0);
+                    for (int kq = 0; kq < 8; ++kq)
+                        mma_bf16_by(ld, tb + tm2_o(b), dk(ST2 + (kq >> 2) * 16384 + (kq & 3) * 32),
+                                    dQW + (uint64_t)((so + R_QT + kq * 2048) >> 4), ID2_QW, kq > 0);
 #pragma unroll
-            for (int kq = 0; kq < 8; ++kq) {
-                const uint64_t adesc = dk(ST2 + (kq >> 2) * 16384 + (kq & 3) * 32);
-                mma_bf16(tb + TM2_D, adesc, dm(so + R_WT + kq * 2048), ID2_DL, 1);
-                mma_bf16(tb + TM2_O, adesc, dm(so + R_QT + kq * 2048), ID2_OQ, kq > 0);
+                    for (int kq = 0; kq < 4; ++kq)
+                        mma_bf16_by(ld, tb + tm2_d(b), dm(so + S_V + kq * 2048), dk(so + R_TPU + kq * 32), ID2_UW, 1);
+                    mma_commit_by(ld, bar_m1);
+                    ok = mbar_wait(bar_m1, ci & 1, kWaitLimitNs);
+                }
+                if (!ok) aborted = true;
             }
-            mma_commit(bar_mma);
-            mma_out = true;
-        }
-        if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
-        if (tid == kMma) mma_out = false;
-        tc_fence_after();
-        {   // D^T (lane v, columns s), times |k_s|^-1 -> bf16 tile [v][s]
-            float x[16];
-            const int s0 = 16 * cgrp;
-            tmem_ld16(tb + TM2_D + lane_sel + s0, x);
-            tmem_ld_wait();
+            if (bar_or(1, kGroup, aborted)) { aborted = true; break; }
+            tc_fence_after();
+            {   // D^T (lane v, columns s), times |k_s|^-1 -> bf16 tile [v][s]
+                const float *invk = reinterpret_cast<const float *>(stg + R_INVK);
+                float x[32];
+                const int s0 = 32 * half;
+                tmem_ld32(tb + tm2_d(b) + lane_sel + s0, x);
+                tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) x[j] *= invk[s0 + j];
-            row16_to_tile(sm, DT2, 32 * quarter + lane, s0, 128, x);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 f = *reinterpret_cast<const float4 *>(invk + s0 + j);
+                    x[j] *= f.x; x[j + 1] *= f.y; x[j + 2] *= f.z; x[j + 3] *= f.w;
+                }
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) sts128(sm, DT2 + sw128_chunk(v, s0 + 8 * q4, 128), pack8(x + 8 * q4));
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            bar_sync(1, kGroup);
+            tc_fence_after();
 
-        // ---------------- O^T += D~^T A_qk^T ; S^T += D~^T Khat (Khat^T rows = key channel)
-        if (tid == kMma) {
+            // S^T += D~^T Khat (committed on its own: the next chunk waits for it), then
+            // O^T += D~^T A_qk^T (the output group waits for that one)
+            if (warp == 0) {
+                const uint32_t ld = elect_one();
 #pragma unroll
-            for (int kq = 0; kq < 4; ++kq) {
-                const uint64_t adesc = dk(DT2 + kq * 32);
-                mma_bf16(tb + TM2_O, adesc, dk(so + R_AQK + kq * 32), ID2_OA, 1);
-                mma_bf16(tb + TM2_S, adesc, dk(so + R_KH + kq * 32), ID2_S, 1);
-            }
-            mma_commit(bar_mma);
-            mma_out = true;
-        }
-        if (wait_all(bar_mma, ph_mma)) { aborted = true; break; }
-        if (tid == kMma) mma_out = false;
-        tc_fence_after();
-        {   // O^T (lane v, columns r) -> plain [r][v] tile over the consumed Qtil^T image
-            float x[16];
-            const int v = 32 * quarter + lane, r0 = 16 * cgrp;
-            tmem_ld16(tb + TM2_O + lane_sel + r0, x);
-            tmem_ld_wait();
+                for (int kq = 0; kq < 4; ++kq)
+                    mma_bf16_by(ld, tb + TM2_S, dk(DT2 + kq * 32), dk(so + R_KH + kq * 32), ID2_KS, 1);
+                mma_commit_by(ld, bar_s);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int r = r0 + j;
-                *reinterpret_cast<__nv_bfloat16 *>(stg + R_QT + r * 256 + v * 2) =
-                    __float2bfloat16_rn(p.scale * invq[r] * x[j]);
+                for (int kq = 0; kq < 4; ++kq)
+                    mma_bf16_by(ld, tb + tm2_o(b), dk(DT2 + kq * 32), dk(so + R_AQK + kq * 32), ID2_KA, 1);
+                mma_commit_by(ld, bar_o + b);
+                issued = ci;
             }
         }
-        __syncthreads();
-        {   // coalesced 16-byte stores of the rows that belong to this sequence
-            __nv_bfloat16 *O = static_cast<__nv_bfloat16 *>(p.o);
+        if (!aborted && p.S_out) {
+            bool ok = true;
+            if (warp == 0 && nchunks > 0) ok = mbar_wait(bar_s, (nchunks - 1) & 1, kWaitLimitNs);
+            if (bar_or(1, kGroup, !ok)) aborted = true;
+            tc_fence_after();
+            if (!aborted) {
 #pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const int qd = tid + NT2 * m, r = qd >> 4, c16 = qd & 15;
-                if (r < L) {
-                    const uint4 val = lds128(stg + R_QT, r * 256 + c16 * 16);
-                    *reinterpret_cast<uint4 *>(O + ((t0 + r) * H + h) * D + c16 * 8) = val;
+                for (int jc = 0; jc < 2; ++jc) {
+                    const int c0 = 64 * half + 32 * jc;
+                    float x[32];
+                    if (nchunks == 0) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) x[j] = p.S0 ? p.S0[sbase_state + (long long)(c0 + j) * D + v] : 0.f;
+                    } else {
+                        tmem_ld32(tb + TM2_S + lane_sel + c0, x);
+                        tmem_ld_wait();
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) p.S_out[sbase_state + (long long)(c0 + j) * D + v] = x[j];
                 }
             }
         }
-        // the output staging was written through the generic proxy; the refill below
-        // writes the same bytes through the async proxy
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // the stage is consumed: refill it with chunk ci + 2
-        if (tid == kTma && ci + 2 < nchunks) issue_stage(ci + 2);
-    }
-
-    if (!aborted && p.S_out) {
-        const int v = 32 * quarter + lane;
-        const int c0 = 32 * cgrp;
-        float x[32];
-        if (nchunks == 0) {
+        if (aborted && warp == 0 && issued >= 0) {  // let the issued products finish before exit
+            mbar_wait(bar_o + (issued & 1), (issued >> 1) & 1, kWaitLimitNs);
+            if (P.status && lane == 0) atomicOr(P.status, 1);
+        }
+    } else {
+        // ================= output rows, one chunk behind
+        __nv_bfloat16 *O = static_cast<__nv_bfloat16 *>(p.o);
+        for (int ci = 0; ci < nchunks; ++ci) {
+            const int s = ci & 1, b = ci & 1;
+            const uint8_t *stg = sm + s * STAGE_BYTES;
+            {
+                bool ok = true;
+                if (warp == 8) ok = mbar_wait(bar_o + b, (ci >> 1) & 1, kWaitLimitNs);
+                if (bar_or(2, kGroup, !ok)) { aborted = true; break; }
+            }
+            tc_fence_after();
+            const int r0 = 32 * half;
+            float x[32], iq[32];
+            tmem_ld32(tb + tm2_o(b) + lane_sel + r0, x);
+            const float *invq = reinterpret_cast<const float *>(stg + R_INVQ);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] = p.S0 ? p.S0[sbase_state + (long long)(c0 + j) * D + v] : 0.f;
-        } else {
-            tmem_ld32(tb + TM2_S + lane_sel + c0, x);
+            for (int j = 0; j < 32; j += 4) {
+                const float4 f = *reinterpret_cast<const float4 *>(invq + r0 + j);
+                iq[j] = f.x; iq[j + 1] = f.y; iq[j + 2] = f.z; iq[j + 3] = f.w;
+            }
             tmem_ld_wait();
-        }
+            tc_fence_before();
+            bar_sync(2, kGroup);  // O^T buffer and the stage are no longer read by this group
+            if (tid == kTma) {
+                if ((full_out >> s) & 1u) full_out &= ~(1u << s);  // chunk ci's copies completed (waited above)
+                if (ci + 2 < nchunks) issue_stage(ci + 2);
+            }
+            mbar_arrive(bar_of + b);
+            const long long t0 = bos + (long long)ci * C;
+            const int L = (int)((eos - t0) < C ? (eos - t0) : C);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) p.S_out[sbase_state + (long long)(c0 + j) * D + v] = x[j];
-    }
-
-    if (aborted && (tid == kMma || tid == kTma)) {
-        if (tid == kTma) {
-            for (int s = 0; s < 2; ++s)
-                if ((full_out >> s) & 1u) mbar_wait(bar_full + s, (ph_full >> s) & 1u, kWaitLimitNs);
+            for (int j = 0; j < 32; ++j) {
+                const int r = r0 + j;
+                if (r < L) O[((t0 + r) * H + h) * D + v] = __float2bfloat16_rn(p.scale * iq[j] * x[j]);
+            }
         }
-        if (mma_out) mbar_wait(bar_mma, ph_mma, kWaitLimitNs);
-        if (P.status && tid == kMma) atomicOr(P.status, 1);
+        if (aborted && tid == kTma) {  // copies still in flight finish before exit
+            for (int s = 0; s < 2; ++s)
+                if ((full_out >> s) & 1u) mbar_wait(bar_full + s, 0, kWaitLimitNs), mbar_wait(bar_full + s, 1, kWaitLimitNs);
+            if (P.status) atomicOr(P.status, 1);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -1063,13 +1136,28 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
     }
 }
 
-// Chunk table of a varlen batch: chunk_off[n] = sum_{m<n} ceil(len_m / C) (the first
-// global chunk of sequence n; chunk_off[N] = the total) and, per global chunk, its
-// first token and number of valid rows. One block; sequences in tiles of its size.
-__global__ void kda_tp_chunk_table(const int32_t *cu, int N, int *chunk_off, int2 *chunk_tok) {
+// Set-up of a forward call, one block of 1024 threads:
+//  * the constant tile images of pass 1 (bf16, 128-byte swizzle): Tri[r][s] = 1 for
+//    s <= r (B operand of the in-chunk cumsum) and the identity (the transposes);
+//  * for a varlen batch, the chunk table: chunk_off[n] = sum_{m<n} ceil(len_m / C)
+//    (the first global chunk of sequence n; chunk_off[N] = the total) and, per global
+//    chunk, its first token and number of valid rows (sequences in tiles of 1024).
+__global__ void __launch_bounds__(1024) kda_tp_prep(uint8_t *consts, const int32_t *cu, int N, int *chunk_off,
+                                                    int2 *chunk_tok) {
     __shared__ int warp_tot[32];
     __shared__ int carry;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    {
+        const int tile = tid >> 9, r = (tid >> 3) & 63, j = tid & 7;
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int s_ = 8 * j + q;
+            v[q] = tile ? (s_ == r ? 1.f : 0.f) : (s_ <= r ? 1.f : 0.f);
+        }
+        *reinterpret_cast<uint4 *>(consts + tile * 8192 + sw128_chunk(r, 8 * j, 64)) = pack8(v);
+    }
+    if (!cu) return;
     if (tid == 0) { carry = 0; chunk_off[0] = 0; }
     __syncthreads();
     for (int base = 0; base < N; base += blockDim.x) {
@@ -1104,8 +1192,8 @@ __global__ void kda_tp_chunk_table(const int32_t *cu, int N, int *chunk_off, int
     }
 }
 
-// ---- workspace: [header 256 B: status word, exact-queue count][chunk offsets]
-// [chunk table][exact queue][records], every part 1024-aligned after the header
+// ---- workspace: [header 1 KB: status word, exact-queue count][constant tiles 16 KB]
+// [chunk offsets][chunk table][exact queue][records], every part 1024-aligned
 long long max_chunks(const ChunkParams &p) {
     if (p.cu_seqlens) return ((long long)p.T + C - 1) / C + p.N;
     return (long long)p.N * (((long long)p.T + C - 1) / C);
@@ -1119,7 +1207,7 @@ size_t queue_bytes(const ChunkParams &p) { return round1k((size_t)max_chunks(p) 
 
 size_t chunk_2pass_workspace_bytes(const ChunkParams &p) {
     using namespace tp;
-    return 256 + offsets_bytes(p) + table_bytes(p) + queue_bytes(p) + (size_t)max_chunks(p) * p.H * REC_BYTES;
+    return 1024 + 16384 + offsets_bytes(p) + table_bytes(p) + queue_bytes(p) + (size_t)max_chunks(p) * p.H * REC_BYTES;
 }
 
 cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int32_t *cu_host, cudaStream_t st) {
@@ -1131,10 +1219,12 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *status = reinterpret_cast<int *>(ws);
     int *fix_count = reinterpret_cast<int *>(ws + 64);
-    int *chunk_off = reinterpret_cast<int *>(ws + 256);
-    int2 *chunk_tok = reinterpret_cast<int2 *>(ws + 256 + offsets_bytes(p));
-    int *fix_list = reinterpret_cast<int *>(ws + 256 + offsets_bytes(p) + table_bytes(p));
-    uint8_t *rec = ws + 256 + offsets_bytes(p) + table_bytes(p) + queue_bytes(p);
+    uint8_t *consts = ws + 1024;
+    const size_t base = 1024 + 16384;
+    int *chunk_off = reinterpret_cast<int *>(ws + base);
+    int2 *chunk_tok = reinterpret_cast<int2 *>(ws + base + offsets_bytes(p));
+    int *fix_list = reinterpret_cast<int *>(ws + base + offsets_bytes(p) + table_bytes(p));
+    uint8_t *rec = ws + base + offsets_bytes(p) + table_bytes(p) + queue_bytes(p);
     const int cpr = (int)(((long long)p.T + C - 1) / C);
 
     static_assert(sizeof(IntraParams) <= 4096 && sizeof(StateParams) <= 4096, "kernel parameter blocks");
@@ -1148,6 +1238,7 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     A.n_items = n_items;
     A.split_gate = (p.gate_mode == kGateLog && p.has_lb &&
                     __bfloat162float(__float2bfloat16_rn(p.lb)) != p.lb) ? 1 : 0;
+    A.consts = consts;
     A.fix_count = fix_count;
     A.fix_list = fix_list;
     A.status = status;
@@ -1176,10 +1267,8 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
 
     cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
     if (e != cudaSuccess) return e;
-    if (p.cu_seqlens) {
-        kda_tp_chunk_table<<<1, 1024, 0, st>>>(p.cu_seqlens, p.N, chunk_off, chunk_tok);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
+    kda_tp_prep<<<1, 1024, 0, st>>>(consts, p.cu_seqlens, p.N, chunk_off, chunk_tok);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     int dev = 0, nsm = 148;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
