@@ -96,8 +96,10 @@ constexpr uint32_t M1_REC = MISC1,           // record misc image: gamma[128], i
                    M1_BETA = MISC1 + 1024,   // [64] f32
                    M1_GX = MISC1 + 1280,     // [128] f32: gate totals of rows 0..31 (gate forms)
                    M1_DTB = MISC1 + 1792,    // [128] f32: dt_bias of the item's head
-                   M1_BAR = MISC1 + 2304, M1_TMEM = MISC1 + 2336;
-constexpr uint32_t SMEM1_BYTES = MISC1 + 2368;
+                   M1_BAR = MISC1 + 2304, M1_TMEM = MISC1 + 2336,
+                   M1_XS = MISC1 + 2432;     // fp32 X [32][LDX] of the inverse's last step
+constexpr int LDXS = 40;  // row stride (floats) of X: fragment loads conflict-free
+constexpr uint32_t SMEM1_BYTES = M1_XS + 32 * LDXS * 4;
 constexpr uint32_t SMEM1_ALLOC = SMEM1_BYTES + 1024;
 static_assert(LF + 64 * LDS * 4 <= TF && TF + 64 * LDT * 4 <= TW && TW + 8192 <= KH, "inverse scratch");
 static_assert(TW % 1024 == 0 && AQK % 1024 == 0 && TPU % 1024 == 0 && TPU + 8192 == MISC1, "tile alignment");
@@ -140,11 +142,12 @@ __device__ __forceinline__ bool decode_chunk(const IntraParams &P, long long gc,
     const ChunkParams &p = P.p;
     it.h = h;
     it.gc = gc;
-    if (P.chunk_tok) {
+    if (P.chunk_tok) {  // every table entry has rows: the result does not wait for the load
         if (gc >= nch) return false;
         const int2 e = P.chunk_tok[gc];
         it.t0 = e.x;
         it.L = e.y;
+        return true;
     } else {  // gc < 2^31 (checked on the host): 32-bit division
         const unsigned n = (unsigned)gc / (unsigned)P.cpr;
         if ((int)n >= p.N) return false;
@@ -184,6 +187,7 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
     float *sDtb = reinterpret_cast<float *>(sm + M1_DTB);
     float *Lf = reinterpret_cast<float *>(sm + LF);
     float *Tf = reinterpret_cast<float *>(sm + TF);
+    float *Xs = reinterpret_cast<float *>(sm + M1_XS);
 
     if (warp == 0) { tmem_alloc(s_tmem, TM1_COLS); tmem_relinquish(); }
     if (tid == 32) {
@@ -482,28 +486,36 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
         tc_fence_after();
 
         // ---------------- read-back, row layout (lane = row): L = beta_r |k_r|^-1 |k_s|^-1 A_kk
-        // (fp32, strictly lower part) and the raw A_qk tile (bf16, s <= r)
+        // (fp32 rows of 16-byte groups; only its strictly lower part is read later) and the
+        // raw A_qk tile (bf16, zero above the diagonal)
         {
             const int i = lane;
-            if (quarter == 0) {  // A_kk rows 0..31, columns 16 hw ..: s < i
-                float va[16];
-                tmem_ld16(tb + lane_sel + TM_A1 + 16 * hw, va);
-                tmem_ld_wait();
-                const float f = sbeta[i] * sinvk[i];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int s = 16 * hw + j;
-                    if (s < i) Lf[i * LDS + s] = f * sinvk[s] * va[j];
-                }
-            } else if (quarter == 1) {  // A_kk rows 32..63: hw 0 the diagonal block, hw 1 columns 0..31
+            if (quarter < 2) {  // A_kk rows 32 quarter + i
+                const int r = 32 * quarter + i;
+                const float f = sbeta[r] * sinvk[r];
                 float va[32];
-                tmem_ld32(tb + lane_sel + (hw ? TM_A2 : TM_A1 + 32), va);
-                tmem_ld_wait();
-                const float f = sbeta[32 + i] * sinvk[32 + i];
+                int s0, nv;
+                if (quarter == 0) {  // block 0: columns 16 hw ..
+                    float v16[16];
+                    tmem_ld16(tb + lane_sel + TM_A1 + 16 * hw, v16);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int s = (hw ? 0 : 32) + j;
-                    if (hw || j < i) Lf[(32 + i) * LDS + s] = f * sinvk[s] * va[j];
+                    for (int j = 0; j < 16; ++j) va[j] = v16[j];
+                    s0 = 16 * hw;
+                    nv = 16;
+                } else {  // hw 0: the diagonal block (columns 32..63), hw 1: columns 0..31
+                    tmem_ld32(tb + lane_sel + (hw ? TM_A2 : TM_A1 + 32), va);
+                    tmem_ld_wait();
+                    s0 = hw ? 0 : 32;
+                    nv = 32;
+                }
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    if (j < nv) {
+                        const float4 ik = *reinterpret_cast<const float4 *>(sinvk + s0 + j);
+                        *reinterpret_cast<float4 *>(Lf + r * LDS + s0 + j) =
+                            make_float4(f * ik.x * va[j], f * ik.y * va[j + 1], f * ik.z * va[j + 2], f * ik.w * va[j + 3]);
+                    }
                 }
             } else if (quarter == 2) {  // A_qk rows 0..31: columns 16 hw .. (s <= i), zeros right of 32
                 float va[16];
@@ -535,25 +547,33 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
         if (tid == kTma) bulk_wait_read_all();
         __syncthreads();
 
-        // ---------------- T = (I + L)^-1 on 16x16 blocks, written straight into the bf16
-        // tiles T' = T diag(beta) (record) and T_w = T diag(beta / |k|) (rows r, columns s <= r)
+        // ---------------- T = (I + L)^-1, written straight into the bf16 tiles T' = T diag(beta)
+        // (record) and T_w = T diag(beta / |k|) (rows r, columns s <= r):
+        //   1. the four 16x16 diagonal blocks by forward substitution (lane j = column j, the
+        //      updates of step k applied to all later rows at once);
+        //   2. T_10 = -T_11 L_10 T_00 and T_32 = -T_33 L_32 T_22;
+        //   3. X = L_[23][01] T_[01][01], then T_[23][01] = -T_[23][23] X  (32x32 blocks).
+        // Steps 2 and 3 run on warp-level tf32 MMAs.
         if (warp < 4) {
-            // diagonal blocks by a column sweep (lane j = column j)
             if (lane < 16) {
                 const int b = warp, j = lane;
                 float t[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) t[i] = i == j ? 1.f : 0.f;
+                const float *Lb = Lf + 16 * b * LDS + 16 * b;
 #pragma unroll
-                for (int i = 1; i < 16; ++i) {  // row i of the block: t[i] -= sum_{k<i} L[i][k] t[k]
-                    const float *Lr = Lf + (16 * b + i) * LDS + 16 * b;
+                for (int kg = 0; kg < 4; ++kg) {
+                    float lv[16][4];
 #pragma unroll
-                    for (int k4 = 0; k4 < i; k4 += 4) {
-                        const float4 l4 = *reinterpret_cast<const float4 *>(Lr + k4);
-                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    for (int i = 4 * kg + 1; i < 16; ++i) {
+                        const float4 l4 = *reinterpret_cast<const float4 *>(Lb + i * LDS + 4 * kg);
+                        lv[i][0] = l4.x; lv[i][1] = l4.y; lv[i][2] = l4.z; lv[i][3] = l4.w;
+                    }
 #pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            if (k4 + u < i) t[i] = fmaf(-lv[u], t[k4 + u], t[i]);
+                    for (int u = 0; u < 4; ++u) {
+                        const int k = 4 * kg + u;
+#pragma unroll
+                        for (int i = k + 1; i < 16; ++i) t[i] = fmaf(-lv[i][u], t[k], t[i]);
                     }
                 }
 #pragma unroll
@@ -563,10 +583,10 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
             // blocks above the block diagonal: zero in T and in both bf16 tiles
             // (6 blocks x 16 rows x 2 chunks of 8 columns = 192 items for 128 threads)
             for (int e = tid - 128; e < 192; e += 128) {
-                const int bid = e >> 5, i = (e >> 1) & 15, half = e & 1;
+                const int bid = e >> 5, i = (e >> 1) & 15, hf = e & 1;
                 const int bi = bid < 3 ? 0 : bid < 5 ? 1 : 2;
                 const int bj = bid < 3 ? bid + 1 : bid < 5 ? bid - 1 : 3;
-                const int r = 16 * bi + i, cc = 16 * bj + 8 * half;
+                const int r = 16 * bi + i, cc = 16 * bj + 8 * hf;
                 *reinterpret_cast<float4 *>(Tf + r * LDT + cc) = make_float4(0.f, 0.f, 0.f, 0.f);
                 *reinterpret_cast<float4 *>(Tf + r * LDT + cc + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
                 sts128(sm, TPU + sw128_chunk(r, cc, 64), make_uint4(0u, 0u, 0u, 0u));
@@ -574,13 +594,58 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
             }
         }
         __syncthreads();
-        // block rows I = 1..3:  T[I, J<I] = -T_II sum_{K<I} L_IK T_KJ on warp-level tf32 MMAs;
-        // warp w < 2I owns output columns 8w .. 8w+7; warps 6 and 7 meanwhile convert the
-        // diagonal blocks into both bf16 tiles
-        if (warp >= 6) {
+        const int g8 = lane >> 2, t4 = lane & 3;
+        // -T[r][c], -T[r][c+1] of an MMA output pair into T and both bf16 tiles
+        auto put_pair = [&](int r, int c0, float e0, float e1) {
+            Tf[r * LDT + c0] = -e0;
+            Tf[r * LDT + c0 + 1] = -e1;
+            const float b0s = sbeta[c0], b1s = sbeta[c0 + 1];
+            *reinterpret_cast<uint32_t *>(sm + TPU + sw128(r, c0, 64)) = pack_bf16x2(-e0 * b0s, -e1 * b1s);
+            *reinterpret_cast<uint32_t *>(sm + TW + sw128(r, c0, 64)) =
+                pack_bf16x2(-e0 * b0s * sinvk[c0], -e1 * b1s * sinvk[c0 + 1]);
+        };
+        if (warp < 4) {
+            // step 2: block row I (1 or 3) against block column J = I - 1; warp w owns
+            // output columns n0 .. n0 + 7
+            const int I = warp < 2 ? 1 : 3, jb = 16 * (I - 1), n0 = jb + 8 * (warp & 1);
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            const float *La = Lf + (16 * I + g8) * LDS, *Lb2 = Lf + (16 * I + g8 + 8) * LDS;
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+                const int k0 = jb + 8 * ks;
+                const uint32_t a[4] = {to_tf32(La[k0 + t4]), to_tf32(Lb2[k0 + t4]), to_tf32(La[k0 + t4 + 4]),
+                                       to_tf32(Lb2[k0 + t4 + 4])};
+                const uint32_t b[2] = {to_tf32(Tf[(k0 + t4) * LDT + n0 + g8]), to_tf32(Tf[(k0 + t4 + 4) * LDT + n0 + g8])};
+                mma_tf32_16x8x8(d, a, b);
+            }
+            // R[row][col] sits in lane 4*(row % 8) + col/2, component (row >= 8) * 2 + col % 2
+            const int srcA = 4 * t4 + (g8 >> 1), srcB = 4 * (t4 + 4) + (g8 >> 1);
+            const bool odd = g8 & 1;
+            float vv[8];
+#pragma unroll
+            for (int cq = 0; cq < 4; ++cq) {
+                vv[cq] = __shfl_sync(0xffffffffu, d[cq], srcA);
+                vv[4 + cq] = __shfl_sync(0xffffffffu, d[cq], srcB);
+            }
+            const uint32_t b0[2] = {to_tf32(odd ? vv[1] : vv[0]), to_tf32(odd ? vv[5] : vv[4])};
+            const uint32_t b1[2] = {to_tf32(odd ? vv[3] : vv[2]), to_tf32(odd ? vv[7] : vv[6])};
+            float e4[4] = {0.f, 0.f, 0.f, 0.f};
+            const float *Ta = Tf + (16 * I + g8) * LDT + 16 * I, *Tb = Tf + (16 * I + g8 + 8) * LDT + 16 * I;
+            {
+                const uint32_t a[4] = {to_tf32(Ta[t4]), to_tf32(Tb[t4]), to_tf32(Ta[t4 + 4]), to_tf32(Tb[t4 + 4])};
+                mma_tf32_16x8x8(e4, a, b0);
+            }
+            {
+                const uint32_t a[4] = {to_tf32(Ta[8 + t4]), to_tf32(Tb[8 + t4]), to_tf32(Ta[12 + t4]), to_tf32(Tb[12 + t4])};
+                mma_tf32_16x8x8(e4, a, b1);
+            }
+            put_pair(16 * I + g8, n0 + 2 * t4, e4[0], e4[1]);
+            put_pair(16 * I + g8 + 8, n0 + 2 * t4, e4[2], e4[3]);
+        } else if (warp >= 6) {
+            // meanwhile: the diagonal blocks into both bf16 tiles
             for (int e = tid - 192; e < 128; e += 64) {
-                const int b = e >> 5, i = (e >> 1) & 15, half = e & 1;
-                const int r = 16 * b + i, cc = 16 * b + 8 * half;
+                const int b = e >> 5, i = (e >> 1) & 15, hf = e & 1;
+                const int r = 16 * b + i, cc = 16 * b + 8 * hf;
                 float mu[8], mw[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
@@ -592,59 +657,41 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
                 sts128(sm, TW + sw128_chunk(r, cc, 64), pack8(mw));
             }
         }
+        __syncthreads();
+        // step 3: warp w owns rows 32 + 16 mt .. (mt = w / 4) and columns 8 nt .. (nt = w % 4)
+        const int mt = warp >> 2, n0 = 8 * (warp & 3);
         {
-            const int g = lane >> 2, t4 = lane & 3;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            const float *La = Lf + (32 + 16 * mt + g8) * LDS, *Lb2 = Lf + (32 + 16 * mt + g8 + 8) * LDS;
 #pragma unroll
-            for (int I = 1; I < 4; ++I) {
-                if (warp < 2 * I) {
-                    const int n0 = 8 * warp;
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-                    const float *La = Lf + (16 * I + g) * LDS, *Lb = Lf + (16 * I + g + 8) * LDS;
-#pragma unroll
-                    for (int ks = 0; ks < 2 * I; ++ks) {
-                        const int k0 = 8 * ks;
-                        const uint32_t a[4] = {to_tf32(La[k0 + t4]), to_tf32(Lb[k0 + t4]), to_tf32(La[k0 + t4 + 4]),
-                                               to_tf32(Lb[k0 + t4 + 4])};
-                        const uint32_t b[2] = {to_tf32(Tf[(k0 + t4) * LDT + n0 + g]),
-                                               to_tf32(Tf[(k0 + t4 + 4) * LDT + n0 + g])};
-                        mma_tf32_16x8x8(d, a, b);
-                    }
-                    // R[row][col] sits in lane 4*(row % 8) + col/2, component (row >= 8) * 2 + col % 2
-                    const int srcA = 4 * t4 + (g >> 1), srcB = 4 * (t4 + 4) + (g >> 1);
-                    const bool odd = g & 1;
-                    float v[8];
-#pragma unroll
-                    for (int cq = 0; cq < 4; ++cq) {
-                        v[cq] = __shfl_sync(0xffffffffu, d[cq], srcA);
-                        v[4 + cq] = __shfl_sync(0xffffffffu, d[cq], srcB);
-                    }
-                    const uint32_t b0[2] = {to_tf32(odd ? v[1] : v[0]), to_tf32(odd ? v[5] : v[4])};
-                    const uint32_t b1[2] = {to_tf32(odd ? v[3] : v[2]), to_tf32(odd ? v[7] : v[6])};
-                    float e4[4] = {0.f, 0.f, 0.f, 0.f};
-                    const float *Ta = Tf + (16 * I + g) * LDT + 16 * I, *Tb = Tf + (16 * I + g + 8) * LDT + 16 * I;
-                    {
-                        const uint32_t a[4] = {to_tf32(Ta[t4]), to_tf32(Tb[t4]), to_tf32(Ta[t4 + 4]), to_tf32(Tb[t4 + 4])};
-                        mma_tf32_16x8x8(e4, a, b0);
-                    }
-                    {
-                        const uint32_t a[4] = {to_tf32(Ta[8 + t4]), to_tf32(Tb[8 + t4]), to_tf32(Ta[12 + t4]),
-                                               to_tf32(Tb[12 + t4])};
-                        mma_tf32_16x8x8(e4, a, b1);
-                    }
-                    const int r0 = 16 * I + g, c0 = n0 + 2 * t4;
-                    Tf[r0 * LDT + c0] = -e4[0];
-                    Tf[r0 * LDT + c0 + 1] = -e4[1];
-                    Tf[(r0 + 8) * LDT + c0] = -e4[2];
-                    Tf[(r0 + 8) * LDT + c0 + 1] = -e4[3];
-                    const float b0s = sbeta[c0], b1s = sbeta[c0 + 1];
-                    const float w0s = b0s * sinvk[c0], w1s = b1s * sinvk[c0 + 1];
-                    *reinterpret_cast<uint32_t *>(sm + TPU + sw128(r0, c0, 64)) = pack_bf16x2(-e4[0] * b0s, -e4[1] * b1s);
-                    *reinterpret_cast<uint32_t *>(sm + TPU + sw128(r0 + 8, c0, 64)) = pack_bf16x2(-e4[2] * b0s, -e4[3] * b1s);
-                    *reinterpret_cast<uint32_t *>(sm + TW + sw128(r0, c0, 64)) = pack_bf16x2(-e4[0] * w0s, -e4[1] * w1s);
-                    *reinterpret_cast<uint32_t *>(sm + TW + sw128(r0 + 8, c0, 64)) = pack_bf16x2(-e4[2] * w0s, -e4[3] * w1s);
-                }
-                if (I < 3) __syncthreads();
+            for (int ks = 0; ks < 4; ++ks) {
+                const int k0 = 8 * ks;
+                const uint32_t a[4] = {to_tf32(La[k0 + t4]), to_tf32(Lb2[k0 + t4]), to_tf32(La[k0 + t4 + 4]),
+                                       to_tf32(Lb2[k0 + t4 + 4])};
+                const uint32_t b[2] = {to_tf32(Tf[(k0 + t4) * LDT + n0 + g8]), to_tf32(Tf[(k0 + t4 + 4) * LDT + n0 + g8])};
+                mma_tf32_16x8x8(d, a, b);
             }
+            float *xr = Xs + (16 * mt + g8) * LDXS + n0 + 2 * t4;
+            xr[0] = d[0]; xr[1] = d[1];
+            xr[8 * LDXS] = d[2]; xr[8 * LDXS + 1] = d[3];
+        }
+        __syncthreads();
+        {
+            float e4[4] = {0.f, 0.f, 0.f, 0.f};
+            const float *Ta = Tf + (32 + 16 * mt + g8) * LDT, *Tb = Tf + (32 + 16 * mt + g8 + 8) * LDT;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                if (ks < 2 + 2 * mt) {  // T_[23][23] is zero right of its block diagonal
+                    const int k0 = 32 + 8 * ks;
+                    const uint32_t a[4] = {to_tf32(Ta[k0 + t4]), to_tf32(Tb[k0 + t4]), to_tf32(Ta[k0 + t4 + 4]),
+                                           to_tf32(Tb[k0 + t4 + 4])};
+                    const uint32_t b[2] = {to_tf32(Xs[(k0 - 32 + t4) * LDXS + n0 + g8]),
+                                           to_tf32(Xs[(k0 - 32 + t4 + 4) * LDXS + n0 + g8])};
+                    mma_tf32_16x8x8(e4, a, b);
+                }
+            }
+            put_pair(32 + 16 * mt + g8, n0 + 2 * t4, e4[0], e4[1]);
+            put_pair(32 + 16 * mt + g8 + 8, n0 + 2 * t4, e4[2], e4[3]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
