@@ -1,5 +1,5 @@
 """Benchmark: KDA chunk forward tokens/s and decode steps/s on B200, with the
-roofline fraction of the dominant kernel and the CPU oracle beside it.
+roofline fraction of the chunk forward and the CPU oracle beside it.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
 
@@ -11,6 +11,11 @@ fp32 state, bf16 token vectors, one fresh token per step) is timed in the
 same run, K' = 256 steps per timed pass, and reported under "decode".
 Inputs are resident in HBM and larger than L2 (3.9 GB chunk inputs, 384 MiB
 decode state), so no L2 flush runs between iterations.
+
+The chunk forward is one `kda_chunk_fwd` call that launches four kernels (set-up,
+the intra-chunk pass, the exact-record pass for steep gates, the state pass);
+its roofline entry divides the operator's algorithmic bytes by the time of the
+whole call, and `traffic` is the DRAM traffic of those four launches.
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own replica of
 the workload (no data-path collective; weak scaling); the timed region is
@@ -37,6 +42,10 @@ METRIC = "chunk_kda fwd tokens/s & decode steps/s on 1 B200; % of tensor/HBM roo
 CHUNK_WL = 4
 DECODE_WL = 3
 DECODE_STEPS_PER_PASS = 256
+# kernels one chunk forward launches on the bench workload (set-up, intra-chunk
+# records, exact records, state pass) and the sources they are built from
+CHUNK_LAUNCHES = 4
+CHUNK_SOURCES = ("kda_chunk_2pass.cu", "kda_tc_util.cuh", "kda_sm100.cuh", "kda_common.cuh")
 
 
 def load_peaks():
@@ -327,10 +336,7 @@ def run_kda(args, rank, world, local_rank):
     chunk_gbs = chunk_bytes / (chunk_ms * 1e-3) / 1e9
     chunk_tflops = chunk_flops / (chunk_ms * 1e-3) / 1e12
     dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
-    tc_used = os.path.exists(os.path.join(ROOT, "kimi_delta_attention_20_b200", "csrc",
-                                          "kda_chunk_tc.cu"))
-    chunk_sha = source_sha("kda_chunk_tc.cu", "kda_chunk_simt.cu", "kda_common.cuh",
-                           "kda_sm100.cuh") if tc_used else None
+    chunk_sha = source_sha(*CHUNK_SOURCES)
     result = {
         "metric": METRIC,
         "value": whole_job_rate(world, wl.tokens, chunk_ms),
@@ -372,7 +378,7 @@ def run_kda(args, rank, world, local_rank):
         },
         "e2e": {"value": whole_job_rate(world, wl.tokens, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": args.steps * (1 + DECODE_STEPS_PER_PASS),
+        "gpu_launches": args.steps * (CHUNK_LAUNCHES + DECODE_STEPS_PER_PASS),
         "clocks": clk,
         "library": os.path.relpath(_abi.LIB_PATH, ROOT),
     }
