@@ -17,6 +17,10 @@ with the host C compiler, or ahead of time by ``build()``):
 * ``gate`` -- the in-kernel forget gate of the same boundary (``A_log``,
   ``dt_bias``, unbounded or safe form), in fp64 numpy, as page
   "atlas_core/kimi_k3/kda.rs" writes it in ``bounded_gate``.
+* ``conv_update``, ``output_gate``, ``decode_token`` -- the serving decode token
+  of the same page (``conv_update``, ``kda_decode_token``,
+  ``full_rank_output_gate``): causal depthwise conv + SiLU, then form R for one
+  token, then sigmoid(gate) * RMSNorm, in fp64 numpy.
 
 Both take packed inputs: q, k, g of shape [T_total, H, d_k], v of shape
 [T_total, H, d_v], beta logits [T_total, H], ``cu_seqlens`` int offsets
@@ -222,3 +226,70 @@ def chunkwise(q, k, v, g, beta, *, scale=None, initial_state=None, cu_seqlens=No
     if rc != 0:
         raise RuntimeError(f"kda_oracle_chunkwise failed ({rc})")
     return o, S
+
+
+# --------------------------------------------------------------------------- decode token
+
+def silu(x):
+    """x * sigmoid(x) in fp64 (page "atlas_core/kimi_k3/kda.rs", `conv_update`)."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / (1.0 + np.exp(-x))
+
+
+def conv_update(state, x, w):
+    """Causal depthwise convolution + SiLU over one new sample per channel.
+
+    ``state`` [..., C, K] holds each channel's last K inputs, oldest first; it is
+    shifted one slot towards the start, ``x`` [..., C] is written into the last
+    slot, and y[c] = silu(sum_k w[c, k] state[c, k]) with ``w`` [C, K]
+    (page "atlas_core/kimi_k3/kda.rs", `conv_update`). Returns (y, new_state) in
+    fp64; the input state is not modified.
+    """
+    st = _f64(state).copy()
+    xs = _f64(x)
+    ww = _f64(w)
+    st[..., :-1] = st[..., 1:]
+    st[..., -1] = xs
+    return silu(np.sum(ww * st, axis=-1)), st
+
+
+def output_gate(core, g, head_dim, eps):
+    """Full-rank output gate: sigmoid(g) * RMSNorm(core) per head of ``head_dim``
+    channels, RMSNorm(x) = x / sqrt(mean(x^2) + eps), no weight (page
+    "atlas_core/kimi_k3/kda.rs", `full_rank_output_gate`)."""
+    c = _f64(core)
+    gg = _f64(g)
+    shp = c.shape
+    c = c.reshape(*shp[:-1], -1, head_dim)
+    gg = gg.reshape(*shp[:-1], -1, head_dim)
+    inv = 1.0 / np.sqrt(np.mean(c * c, axis=-1, keepdims=True) + float(eps))
+    return (c * inv / (1.0 + np.exp(-gg))).reshape(shp)
+
+
+def decode_token(x, conv_w, conv_state, g, beta, state, *, H, Dk, Dv, scale=None,
+                 use_qk_l2norm=True, lower_bound=None, beta_is_logit=True, gate_form=None,
+                 A_log=None, dt_bias=None, g_out=None, norm_eps=1e-6):
+    """One decode token for N sequences (page "atlas_core/kimi_k3/kda.rs",
+    `kda_decode_token`, with `full_rank_output_gate` when ``g_out`` is given):
+    the conv update + SiLU over the pre-conv projections ``x`` [N, H*(2Dk+Dv)]
+    laid out q | k | v, then the recurrent step (form R) on that token from
+    ``state`` [N, H, Dk, Dv], then, with ``g_out`` [N, H*Dv], the output gate.
+
+    ``conv_w`` [H*(2Dk+Dv), K], ``conv_state`` [N, H*(2Dk+Dv), K]; ``g`` [N, H, Dk]
+    and ``beta`` [N, H] as in ``recurrent``. Returns (o [N, H, Dv],
+    new_conv_state, new_state), fp64.
+    """
+    y, cs = conv_update(conv_state, x, conv_w)
+    N = y.shape[0]
+    qd, vd = H * Dk, H * Dv
+    q = y[:, :qd].reshape(N, H, Dk)
+    k = y[:, qd:2 * qd].reshape(N, H, Dk)
+    v = y[:, 2 * qd:2 * qd + vd].reshape(N, H, Dv)
+    cu = np.arange(N + 1, dtype=np.int64)  # one token per sequence
+    o, S = recurrent(q, k, v, _f64(g).reshape(N, H, Dk), _f64(beta).reshape(N, H), scale=scale,
+                     initial_state=state, cu_seqlens=cu, use_qk_l2norm=use_qk_l2norm,
+                     lower_bound=lower_bound, beta_is_logit=beta_is_logit, gate_form=gate_form,
+                     A_log=A_log, dt_bias=dt_bias)
+    if g_out is not None:
+        o = output_gate(o.reshape(N, H * Dv), _f64(g_out).reshape(N, H * Dv), Dv, norm_eps).reshape(N, H, Dv)
+    return o, cs, S
