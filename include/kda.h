@@ -161,6 +161,45 @@ typedef struct {
 KDA_API kda_status kda_recurrent_step(const kda_step_args *args, void *stream);
 
 /*
+ * One serving decode token for N sequences (page "atlas_core/kimi_k3/kda.rs",
+ * `kda_decode_token` followed by `full_rank_output_gate`), fused in one launch:
+ *   1. causal depthwise convolution + SiLU over the pre-conv projections x,
+ *      channels laid out q | k | v (H*Dk, H*Dk, H*Dv): each channel's window of
+ *      the last conv_kernel inputs (oldest first) shifts one slot, x enters the
+ *      last slot, y = silu(sum_t conv_w[c][t] * window[c][t]); the windows are
+ *      updated IN PLACE;
+ *   2. the recurrent step of kda_recurrent_step on q, k, v = y (same gate,
+ *      beta, scale and L2-norm options), state updated IN PLACE;
+ *   3. when g_out is given, o = sigmoid(g_out) * core / sqrt(mean(core^2) + norm_eps)
+ *      per head (RMSNorm without a weight); otherwise o = core.
+ * Host-side validation as for kda_recurrent_step; conv_kernel in 1..8.
+ */
+typedef struct {
+    kda_dtype dtype;      /* dtype of x, g, beta, g_out and o */
+    int N, H, Dk, Dv;     /* Dk, Dv in {32, 64, 128} */
+    int conv_kernel;      /* window length K, 1..8 */
+    const void *x;        /* [N, H*(2*Dk+Dv)] pre-conv q | k | v */
+    const float *conv_w;  /* [H*(2*Dk+Dv), K] fp32 */
+    float *conv_state;    /* [N, H*(2*Dk+Dv), K] fp32, oldest input first, updated in place */
+    const void *g;        /* [N,H,Dk] log-decay, or the gate input (gate_mode) */
+    const void *beta;     /* [N,H] logits (or see beta_is_prob) */
+    float *state;         /* [N,H,Dk,Dv] fp32, updated in place */
+    const void *g_out;    /* [N,H,Dv] output-gate input, or NULL for the ungated core output */
+    float norm_eps;       /* RMSNorm epsilon of the output gate (>= 0) */
+    void *o;              /* [N,H,Dv] out */
+    float scale;          /* <= 0 or NaN selects 1/sqrt(Dk) */
+    int use_qk_l2norm;
+    int has_lower_bound;
+    float lower_bound;
+    kda_gate_mode gate_mode;
+    const float *A_log;   /* [H] fp32, in-kernel gate forms only */
+    const float *dt_bias; /* [H,Dk] fp32 or NULL */
+    int beta_is_prob;
+} kda_token_args;
+
+KDA_API kda_status kda_decode_token(const kda_token_args *args, void *stream);
+
+/*
  * Chunkwise forward for callers that cannot allocate device memory. This entry
  * point has no counterpart in the pages; it exists for callers that run under a
  * fixed device-memory plan and may not allocate once running (an inference

@@ -64,9 +64,25 @@ class StepArgs(ctypes.Structure):
     ]
 
 
+class TokenArgs(ctypes.Structure):
+    _fields_ = [
+        ("dtype", ctypes.c_int),
+        ("N", ctypes.c_int), ("H", ctypes.c_int), ("Dk", ctypes.c_int), ("Dv", ctypes.c_int),
+        ("conv_kernel", ctypes.c_int),
+        ("x", _vp), ("conv_w", _vp), ("conv_state", _vp), ("g", _vp), ("beta", _vp),
+        ("state", _vp), ("g_out", _vp), ("norm_eps", ctypes.c_float), ("o", _vp),
+        ("scale", ctypes.c_float),
+        ("use_qk_l2norm", ctypes.c_int),
+        ("has_lower_bound", ctypes.c_int), ("lower_bound", ctypes.c_float),
+        ("gate_mode", ctypes.c_int), ("A_log", _vp), ("dt_bias", _vp),
+        ("beta_is_prob", ctypes.c_int),
+    ]
+
+
 # every symbol include/kda.h declares
 EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_noalloc",
-           "kda_recurrent_step", "kda_status_string", "kda_last_cuda_error", "kda_version")
+           "kda_recurrent_step", "kda_decode_token", "kda_status_string", "kda_last_cuda_error",
+           "kda_version")
 
 _lib = None
 
@@ -89,6 +105,8 @@ def load():
     lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
     lib.kda_recurrent_step.argtypes = [ctypes.POINTER(StepArgs), _vp]
     lib.kda_recurrent_step.restype = ctypes.c_int
+    lib.kda_decode_token.argtypes = [ctypes.POINTER(TokenArgs), _vp]
+    lib.kda_decode_token.restype = ctypes.c_int
     lib.kda_status_string.argtypes = [ctypes.c_int]
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_last_cuda_error.argtypes = []

@@ -15,6 +15,8 @@ cudaError_t launch_chunk_tc(const ChunkParams &p, int Dk, int Dv, void *workspac
                             size_t workspace_bytes, const int32_t *cu_host, cudaStream_t st);
 size_t chunk_2pass_workspace_bytes(const ChunkParams &p);
 cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int32_t *cu_host, cudaStream_t st);
+bool token_conv_supported(int K);
+cudaError_t launch_token(const TokenParams &tp, bool bf16, int Dk, int Dv, cudaStream_t st);
 }  // namespace kda
 
 namespace {
@@ -213,6 +215,48 @@ kda_status kda_recurrent_step(const kda_step_args *a, void *stream) {
     p.dt_bias = a->dt_bias;
     p.beta_prob = a->beta_is_prob ? 1 : 0;
     return cuda_status(kda::launch_decode(p, bf16, a->Dk, a->Dv, static_cast<cudaStream_t>(stream)));
+}
+
+kda_status kda_decode_token(const kda_token_args *a, void *stream) {
+    if (!a) return KDA_ERR_INVALID_ARGUMENT;
+    if (a->dtype != KDA_DTYPE_F32 && a->dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARGUMENT;
+    if (a->N < 0 || a->H < 1 || a->Dk < 1 || a->Dv < 1) return KDA_ERR_INVALID_ARGUMENT;
+    if (!head_dim_ok(a->Dk) || !head_dim_ok(a->Dv)) return KDA_ERR_UNSUPPORTED;
+    if (!kda::token_conv_supported(a->conv_kernel)) return KDA_ERR_UNSUPPORTED;
+    if (a->has_lower_bound && !(a->lower_bound < 0.f)) return KDA_ERR_INVALID_ARGUMENT;
+    if (check_gate_mode(a->gate_mode, a->has_lower_bound) != KDA_OK) return KDA_ERR_INVALID_ARGUMENT;
+    if (!(a->norm_eps >= 0.f)) return KDA_ERR_INVALID_ARGUMENT;
+    if ((long long)a->N * a->H * 4 >= 0x7fffffffLL) return KDA_ERR_INVALID_ARGUMENT;
+    if (a->N == 0) return KDA_OK;
+    const bool bf16 = a->dtype == KDA_DTYPE_BF16;
+    const size_t esz = bf16 ? 2 : 4;
+    if (!a->x || !a->conv_w || !a->conv_state || !a->g || !a->beta || !a->state || !a->o)
+        return KDA_ERR_INVALID_ARGUMENT;
+    if (!aligned(a->x, esz) || !aligned(a->g, esz) || !aligned(a->beta, esz) || !aligned(a->o, esz) ||
+        (a->g_out && !aligned(a->g_out, esz)) || !aligned(a->conv_w, 4) || !aligned(a->conv_state, 4) ||
+        !aligned(a->state, 16))
+        return KDA_ERR_INVALID_ARGUMENT;
+    if (check_gate_ptrs(a->gate_mode, a->A_log, a->dt_bias) != KDA_OK) return KDA_ERR_INVALID_ARGUMENT;
+    kda::TokenParams tp;
+    kda::StepParams &p = tp.step;
+    p.q = p.k = p.v = nullptr;
+    p.g = a->g; p.beta = a->beta;
+    p.state = a->state; p.o = a->o; p.N = a->N; p.H = a->H;
+    p.scale = resolve_scale(a->scale, a->Dk);
+    p.use_l2 = a->use_qk_l2norm ? 1 : 0;
+    p.has_lb = a->has_lower_bound ? 1 : 0;
+    p.lb = a->lower_bound;
+    p.gate_mode = a->gate_mode;
+    p.A_log = a->A_log;
+    p.dt_bias = a->dt_bias;
+    p.beta_prob = a->beta_is_prob ? 1 : 0;
+    tp.x = a->x;
+    tp.conv_w = a->conv_w;
+    tp.conv_state = a->conv_state;
+    tp.K = a->conv_kernel;
+    tp.g_out = a->g_out;
+    tp.norm_eps = a->norm_eps;
+    return cuda_status(kda::launch_token(tp, bf16, a->Dk, a->Dv, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

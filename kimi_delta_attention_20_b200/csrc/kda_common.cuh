@@ -86,4 +86,15 @@ struct StepParams {
     int beta_prob;
 };
 
+// Launch parameters of the fused decode token (conv + SiLU, recurrent step, output gate).
+struct TokenParams {
+    StepParams step;            // q, k, v unused: they come from the convolution
+    const void *x;              // [N, H*(2Dk+Dv)]
+    const float *conv_w;        // [H*(2Dk+Dv), K]
+    float *conv_state;          // [N, H*(2Dk+Dv), K]
+    int K;
+    const void *g_out;          // [N, H, Dv] or null
+    float norm_eps;
+};
+
 }  // namespace kda

@@ -215,3 +215,69 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
     with torch.cuda.device(q.device):
         _abi.check(lib.kda_recurrent_step(ctypes.byref(a), _stream(q.device)), "kda_recurrent_step")
     return o
+
+
+def decode_token(x: torch.Tensor, conv_w: torch.Tensor, conv_state: torch.Tensor, g: torch.Tensor,
+                 beta: torch.Tensor, state: torch.Tensor, *, g_out: Optional[torch.Tensor] = None,
+                 norm_eps: float = 1e-6, A_log: Optional[torch.Tensor] = None,
+                 dt_bias: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                 use_qk_l2norm_in_kernel: bool = True, use_gate_in_kernel: bool = False,
+                 use_beta_sigmoid_in_kernel: bool = True, safe_gate: bool = False,
+                 lower_bound: Optional[float] = None,
+                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One serving decode token per sequence in one launch (page
+    "atlas_core/kimi_k3/kda.rs": `conv_update` + SiLU, `kda_recurrent_step`, and
+    `full_rank_output_gate` when ``g_out`` is given).
+
+    x: [N, H*(2 Dk + Dv)] pre-conv projections q | k | v; conv_w: [H*(2 Dk + Dv), K]
+    fp32; conv_state: [N, H*(2 Dk + Dv), K] fp32, oldest input first, updated IN
+    PLACE; g: [N, H, Dk]; beta: [N, H]; state: [N, H, Dk, Dv] fp32, updated IN PLACE;
+    g_out: [N, H, Dv] or None. ``norm_eps`` is the RMSNorm epsilon of the output
+    gate (1e-6 by default, the norm epsilon of the KDA model configs). Gate and beta
+    arguments as in ``recurrent_step``. Returns o [N, H, Dv]: the gated, normalised
+    output with ``g_out``, else the recurrent step's output.
+    """
+    lib = _abi.load()
+    for name, t in (("x", x), ("conv_w", conv_w), ("conv_state", conv_state), ("g", g), ("beta", beta),
+                    ("state", state)):
+        _need_cuda(name, t)
+    if x.dtype not in _DTYPES or any(t.dtype != x.dtype for t in (g, beta)):
+        raise ValueError("x, g, beta must share one dtype: float32 or bfloat16")
+    if g_out is not None:
+        _need_cuda("g_out", g_out)
+        if g_out.dtype != x.dtype:
+            raise ValueError("g_out must have the dtype of x")
+    if state.dtype != torch.float32 or state.dim() != 4:
+        raise ValueError("state must be float32 [N, H, Dk, Dv]")
+    N, H, Dk, Dv = state.shape
+    C = H * (2 * Dk + Dv)
+    if x.shape != (N, C):
+        raise ValueError(f"x must be [{N}, {C}] (q | k | v of H={H}, Dk={Dk}, Dv={Dv})")
+    if conv_w.dtype != torch.float32 or conv_w.dim() != 2 or conv_w.shape[0] != C:
+        raise ValueError(f"conv_w must be float32 [{C}, K]")
+    K = conv_w.shape[1]
+    if conv_state.dtype != torch.float32 or conv_state.shape != (N, C, K):
+        raise ValueError(f"conv_state must be float32 [{N}, {C}, {K}]")
+    if g.shape != (N, H, Dk) or beta.shape != (N, H):
+        raise ValueError("g must be [N, H, Dk] and beta [N, H]")
+    if g_out is not None and g_out.shape != (N, H, Dv):
+        raise ValueError(f"g_out must be [{N}, {H}, {Dv}]")
+    for name, t in (("x", x), ("conv_w", conv_w), ("conv_state", conv_state), ("g", g), ("beta", beta),
+                    ("state", state)) + ((("g_out", g_out),) if g_out is not None else ()):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    o = out if out is not None else torch.empty(N, H, Dv, dtype=x.dtype, device=x.device)
+    a = _abi.TokenArgs()
+    a.dtype = _DTYPES[x.dtype]
+    a.N, a.H, a.Dk, a.Dv, a.conv_kernel = N, H, Dk, Dv, K
+    a.x, a.conv_w, a.conv_state, a.g, a.beta, a.state, a.o = (
+        _ptr(t) for t in (x, conv_w, conv_state, g, beta, state, o))
+    a.g_out = _ptr(g_out) if g_out is not None else None
+    a.norm_eps = float(norm_eps)
+    a.scale = float("nan") if scale is None else float(scale)
+    a.use_qk_l2norm = int(bool(use_qk_l2norm_in_kernel))
+    _gate_fields(a, x.device, H, Dk, A_log, dt_bias, use_gate_in_kernel, safe_gate, lower_bound,
+                 use_beta_sigmoid_in_kernel)
+    with torch.cuda.device(x.device):
+        _abi.check(lib.kda_decode_token(ctypes.byref(a), _stream(x.device)), "kda_decode_token")
+    return o

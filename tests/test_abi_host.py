@@ -154,6 +154,48 @@ def test_recurrent_step_empty_batch_is_a_noop():
     assert lib.kda_recurrent_step(ctypes.byref(a), None) == _abi.KDA_OK
 
 
+def token_args(**over):
+    a = _abi.TokenArgs()
+    a.dtype = _abi.KDA_DTYPE_BF16
+    a.N, a.H, a.Dk, a.Dv, a.conv_kernel = 2, 2, 128, 128, 4
+    for f in ("x", "conv_w", "conv_state", "g", "beta", "state", "o"):
+        setattr(a, f, FAKE)
+    a.norm_eps = 1e-6
+    a.use_qk_l2norm = 1
+    for kk, vv in over.items():
+        setattr(a, kk, vv)
+    return a
+
+
+@pytest.mark.parametrize("over,want", [
+    (dict(dtype=3), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(N=-1), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(H=0), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(Dv=48), _abi.KDA_ERR_UNSUPPORTED),
+    (dict(conv_kernel=0), _abi.KDA_ERR_UNSUPPORTED),
+    (dict(conv_kernel=9), _abi.KDA_ERR_UNSUPPORTED),
+    (dict(norm_eps=-1.0), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(norm_eps=float("nan")), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(conv_state=None), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(x=FAKE + 1), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(state=FAKE + 4), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(conv_w=FAKE + 2), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(g_out=FAKE + 1), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(has_lower_bound=1, lower_bound=0.5), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(gate_mode=_abi.KDA_GATE_SOFTPLUS), _abi.KDA_ERR_INVALID_ARGUMENT),
+])
+def test_decode_token_rejects(over, want):
+    lib = _abi.load()
+    a = token_args(**over)
+    assert lib.kda_decode_token(ctypes.byref(a), None) == want
+
+
+def test_decode_token_empty_batch_is_a_noop():
+    lib = _abi.load()
+    a = token_args(N=0, x=None, conv_w=None, conv_state=None, g=None, beta=None, state=None, o=None)
+    assert lib.kda_decode_token(ctypes.byref(a), None) == _abi.KDA_OK
+
+
 def test_python_binding_refuses_cpu_tensors():
     import torch
     import kimi_delta_attention_20_b200 as kda
@@ -196,8 +238,10 @@ _LAYOUT_C = r"""
 int main(void) {
     printf("kda_chunk_args sizeof %zu\n", sizeof(kda_chunk_args));
     printf("kda_step_args sizeof %zu\n", sizeof(kda_step_args));
+    printf("kda_token_args sizeof %zu\n", sizeof(kda_token_args));
     CHUNK_FIELDS
     STEP_FIELDS
+    TOKEN_FIELDS
     return 0;
 }
 """
@@ -208,8 +252,10 @@ def test_ctypes_structs_match_header_layout(tmp_path):
     import subprocess
     chunk = "".join(f"F(kda_chunk_args, {n})" for n, _ in _abi.ChunkArgs._fields_)
     step = "".join(f"F(kda_step_args, {n})" for n, _ in _abi.StepArgs._fields_)
+    token = "".join(f"F(kda_token_args, {n})" for n, _ in _abi.TokenArgs._fields_)
     src = tmp_path / "layout.c"
-    src.write_text(_LAYOUT_C.replace("CHUNK_FIELDS", chunk).replace("STEP_FIELDS", step))
+    src.write_text(_LAYOUT_C.replace("CHUNK_FIELDS", chunk).replace("STEP_FIELDS", step)
+                   .replace("TOKEN_FIELDS", token))
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)],
                    check=True)
@@ -219,6 +265,8 @@ def test_ctypes_structs_match_header_layout(tmp_path):
         got[(struct, field)] = int(val)
     assert got[("kda_chunk_args", "sizeof")] == ctypes.sizeof(_abi.ChunkArgs)
     assert got[("kda_step_args", "sizeof")] == ctypes.sizeof(_abi.StepArgs)
-    for cls, name in ((_abi.ChunkArgs, "kda_chunk_args"), (_abi.StepArgs, "kda_step_args")):
+    assert got[("kda_token_args", "sizeof")] == ctypes.sizeof(_abi.TokenArgs)
+    for cls, name in ((_abi.ChunkArgs, "kda_chunk_args"), (_abi.StepArgs, "kda_step_args"),
+                      (_abi.TokenArgs, "kda_token_args")):
         for field, _ in cls._fields_:
             assert got[(name, field)] == getattr(cls, field).offset, (name, field)
