@@ -8,7 +8,9 @@ sequences of 4096/8192/12288/7168 tokens, H = 96, d_k = d_v = 128, bf16
 inputs, fp32 states, lower bound -5, per-sequence initial states, final
 states out). The decode step workload (64 sequences x 96 heads x 128 x 128
 fp32 state, bf16 token vectors, one fresh token per step) is timed in the
-same run, K' = 256 steps per timed pass, and reported under "decode".
+same run, K' = 256 steps per timed pass, and reported under "decode"; so is the
+serving decode token (conv window 4 + SiLU, the recurrent step and the output
+gate fused, same geometry) under "decode_token".
 Inputs are resident in HBM and larger than L2 (3.9 GB chunk inputs, 384 MiB
 decode state), so no L2 flush runs between iterations.
 
@@ -86,6 +88,20 @@ def chunk_options(wl, inp):
     if wl.beta_prob:
         kw["use_beta_sigmoid_in_kernel"] = False
     return kw
+
+
+# serving decode token (conv + SiLU, recurrent step, output gate): the production
+# layer (H 96, d 128, conv window 4, lower bound -5) for 64 sequences
+TOKEN_WL = dict(N=64, H=96, D=128, K=4, distinct_steps=32)
+
+
+def token_algorithmic(N, H, D, K):
+    """Bytes of one decode token: fp32 state read + write, fp32 conv windows read +
+    write (3 D channels x K per head), the bf16 token vectors (x of 3 D channels, g,
+    g_out, o) and one beta per head, plus one read of the shared conv weights."""
+    heads = N * H
+    per_head = 2 * D * D * 4 + 2 * 3 * D * K * 4 + (3 * D + 3 * D) * 2 + 2
+    return heads * per_head + H * 3 * D * K * 4
 
 
 def decode_algorithmic(wl):
@@ -208,23 +224,34 @@ def run_kda(args, rank, world, local_rank):
     hbm_peak, tc_peak, peak_kind = load_peaks()
 
     wl = KI.CHUNK_WORKLOADS[args.workload if (args.only and args.workload is not None) else CHUNK_WL]
-    inp = KI.chunk_inputs(wl, device=dev)
-    q, k, v, g, beta = (inp[n] for n in ("q", "k", "v", "g", "beta"))
-    S0, cu = inp["initial_state"], inp["cu_seqlens"]
-    o = torch.empty_like(v)
-    S_out = torch.empty(wl.n_seqs, wl.H, wl.Dk, wl.Dv, dtype=torch.float32, device=dev) \
-        if wl.final_state else None
-    opts = chunk_options(wl, inp)
-    ws_bytes = kda.chunk_workspace_bytes(wl.B, wl.T, wl.H, wl.Dk, wl.Dv, N=wl.n_seqs,
-                                         varlen=wl.seqlens is not None)
-    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    if args.only in (None, "chunk"):  # the single-leg profiler runs allocate only their own leg
+        inp = KI.chunk_inputs(wl, device=dev)
+        q, k, v, g, beta = (inp[n] for n in ("q", "k", "v", "g", "beta"))
+        S0, cu = inp["initial_state"], inp["cu_seqlens"]
+        o = torch.empty_like(v)
+        S_out = torch.empty(wl.n_seqs, wl.H, wl.Dk, wl.Dv, dtype=torch.float32, device=dev) \
+            if wl.final_state else None
+        opts = chunk_options(wl, inp)
+        ws_bytes = kda.chunk_workspace_bytes(wl.B, wl.T, wl.H, wl.Dk, wl.Dv, N=wl.n_seqs,
+                                             varlen=wl.seqlens is not None)
+        ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
 
     def chunk_step():
         kda.chunk_kda(q, k, v, g, beta, initial_state=S0, output_final_state=wl.final_state,
                       cu_seqlens=cu, out=o, final_state_out=S_out, workspace=ws, **opts)
 
     dwl = KI.DECODE_WORKLOADS[DECODE_WL]
-    if args.only != "chunk":
+    if args.only in (None, "token"):
+        tk = KI.draw_token(TOKEN_WL["N"], TOKEN_WL["H"], TOKEN_WL["D"], TOKEN_WL["D"], TOKEN_WL["K"],
+                           TOKEN_WL["distinct_steps"], dtype=torch.bfloat16, seed=9, device=dev)
+        tk_o = torch.empty(TOKEN_WL["N"], TOKEN_WL["H"], TOKEN_WL["D"], dtype=torch.bfloat16, device=dev)
+
+    def token_step(t):
+        i = t % TOKEN_WL["distinct_steps"]
+        kda.decode_token(tk["x"][i], tk["w"], tk["cs"], tk["g"][i], tk["beta"][i], tk["S0"],
+                         g_out=tk["g_out"][i], lower_bound=-5.0, out=tk_o)
+
+    if args.only in (None, "decode"):
         dinp = KI.decode_inputs(dwl, device=dev)
         state = dinp["state"].clone()
         od = torch.empty(dwl.N, dwl.H, dwl.Dv, dtype=dwl.dtype, device=dev)
@@ -245,7 +272,7 @@ def run_kda(args, rank, world, local_rank):
 
     if args.only:
         # one kernel, few launches: the shape profiler captures use
-        one = chunk_step if args.only == "chunk" else (lambda: decode_step(0))
+        one = {"chunk": chunk_step, "decode": lambda: decode_step(0), "token": lambda: token_step(0)}[args.only]
         for _ in range(args.warmup):
             one()
         torch.cuda.synchronize(dev)
@@ -297,6 +324,20 @@ def run_kda(args, rank, world, local_rank):
         d1.record(stream)
         torch.cuda.synchronize(dev); barrier()
         dec_ms = max_over_ranks(d0.elapsed_time(d1)) / nsteps
+        # serving decode token: K passes of 256 tokens (cycling over the drawn inputs)
+        for t in range(args.warmup):
+            token_step(t)
+        barrier(); torch.cuda.synchronize(dev)
+        k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        k0.record(stream)
+        ntok = 0
+        for _ in range(args.steps):
+            for t in range(DECODE_STEPS_PER_PASS):
+                token_step(t)
+                ntok += 1
+        k1.record(stream)
+        torch.cuda.synchronize(dev); barrier()
+        tok_ms = max_over_ranks(k0.elapsed_time(k1)) / ntok
     clk = clocks.summary()
 
     # end to end through the public API with host buffers: pinned host inputs
@@ -336,6 +377,8 @@ def run_kda(args, rank, world, local_rank):
     chunk_gbs = chunk_bytes / (chunk_ms * 1e-3) / 1e9
     chunk_tflops = chunk_flops / (chunk_ms * 1e-3) / 1e12
     dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
+    tok_bytes = token_algorithmic(TOKEN_WL["N"], TOKEN_WL["H"], TOKEN_WL["D"], TOKEN_WL["K"])
+    tok_gbs = tok_bytes / (tok_ms * 1e-3) / 1e9
     chunk_sha = source_sha(*CHUNK_SOURCES)
     result = {
         "metric": METRIC,
@@ -376,9 +419,19 @@ def run_kda(args, rank, world, local_rank):
                          "traffic": ncu_traffic("decode", source_sha("kda_decode.cu",
                                                                      "kda_common.cuh"))},
         },
+        "decode_token": {
+            "value": whole_job_rate(world, 1, tok_ms), "unit": "steps/s",
+            "tokens_per_s": whole_job_rate(world, TOKEN_WL["N"], tok_ms), "ms_per_step": tok_ms,
+            "steps_timed": ntok,
+            "workload": "serving decode token: conv window 4 + SiLU, recurrent step, output gate; "
+                        "N=64, H=96, d=128, bf16 vectors, fp32 state and windows, lower_bound=-5",
+            "roofline": {"bound": "hbm", "achieved": tok_gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": tok_gbs / hbm_peak, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": tok_bytes},
+        },
         "e2e": {"value": whole_job_rate(world, wl.tokens, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": args.steps * (CHUNK_LAUNCHES + DECODE_STEPS_PER_PASS),
+        "gpu_launches": args.steps * (CHUNK_LAUNCHES + 2 * DECODE_STEPS_PER_PASS),
         "clocks": clk,
         "library": os.path.relpath(_abi.LIB_PATH, ROOT),
     }
@@ -444,7 +497,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["chunk", "decode"], default=None,
+    ap.add_argument("--only", choices=["chunk", "decode", "token"], default=None,
                     help="run one leg only and print its timing (for profiler captures)")
     ap.add_argument("--workload", type=int, default=None,
                     help="with --only chunk: chunk workload index (default: the varlen H=96 one)")

@@ -211,3 +211,24 @@ def decode_inputs(idx_or_wl, device="cpu", steps=None):
     wl = DECODE_WORKLOADS[idx_or_wl] if isinstance(idx_or_wl, int) else idx_or_wl
     return draw_decode(wl.N, wl.H, wl.Dk, wl.Dv, wl.steps if steps is None else steps,
                        dtype=wl.dtype, seed=wl.seed, device=device)
+
+
+def draw_token(N, H, Dk, Dv, K, steps, *, dtype=torch.bfloat16, seed=0, device="cpu", gate="decode"):
+    """Serving decode-token inputs: pre-conv projections x [steps, N, H*(2Dk+Dv)] ~ N(0,1),
+    conv weights [H*(2Dk+Dv), K] ~ N(0, 1/K), conv windows [N, H*(2Dk+Dv), K] ~ N(0,1),
+    gates [steps, N, H, Dk] = -5 sigmoid(z) (or z itself with gate="input"), beta
+    logits [steps, N, H], output-gate inputs [steps, N, H, Dv] ~ N(0,1), and the
+    initial state [N, H, Dk, Dv] ~ 0.1 N(0,1) fp32. Drawn in that order with one
+    generator seeded with ``seed``, on ``device``; token tensors cast to ``dtype``."""
+    gen = torch.Generator(device=device).manual_seed(seed)
+    C = H * (2 * Dk + Dv)
+    rn = lambda *shape: torch.randn(*shape, generator=gen, device=device)
+    x = rn(steps, N, C).to(dtype)
+    w = rn(C, K) / K ** 0.5
+    cs = rn(N, C, K)
+    z = rn(steps, N, H, Dk)
+    g = (z if gate == "input" else -5.0 * torch.sigmoid(z)).to(dtype)
+    beta = rn(steps, N, H).to(dtype)
+    g_out = rn(steps, N, H, Dv).to(dtype)
+    S0 = rn(N, H, Dk, Dv) * 0.1
+    return dict(x=x, w=w, cs=cs, g=g, beta=beta, g_out=g_out, S0=S0)

@@ -17,20 +17,7 @@ DEV = "cuda"
 
 
 def draw(N, H, Dk, Dv, K, steps, dtype, seed, gate="decode"):
-    """Seeded token inputs: pre-conv projections ~N(0,1), conv weights ~N(0, 1/K), conv
-    windows ~N(0,1), decode gates (-5 sigmoid(z)) or gate inputs, beta logits,
-    output-gate inputs ~N(0,1), states 0.1 N(0,1)."""
-    gen = torch.Generator().manual_seed(seed)
-    C = H * (2 * Dk + Dv)
-    x = torch.randn(steps, N, C, generator=gen).to(dtype)
-    w = torch.randn(C, K, generator=gen) / K ** 0.5
-    cs = torch.randn(N, C, K, generator=gen)
-    z = torch.randn(steps, N, H, Dk, generator=gen)
-    g = (z if gate == "input" else -5.0 * torch.sigmoid(z)).to(dtype)
-    beta = torch.randn(steps, N, H, generator=gen).to(dtype)
-    g_out = torch.randn(steps, N, H, Dv, generator=gen).to(dtype)
-    S0 = torch.randn(N, H, Dk, Dv, generator=gen) * 0.1
-    return dict(x=x, w=w, cs=cs, g=g, beta=beta, g_out=g_out, S0=S0)
+    return KI.draw_token(N, H, Dk, Dv, K, steps, dtype=dtype, seed=seed, gate=gate)
 
 
 def run_tokens(inp, steps, *, gated, oracle_kw=None, gpu_kw=None, eps=1e-6):
