@@ -21,6 +21,10 @@ with the host C compiler, or ahead of time by ``build()``):
   of the same page (``conv_update``, ``kda_decode_token``,
   ``full_rank_output_gate``): causal depthwise conv + SiLU, then form R for one
   token, then sigmoid(gate) * RMSNorm, in fp64 numpy.
+* ``backward`` -- the gradients of the forward (dq, dk, dv, dg, dbeta and the
+  initial-state gradient) for an output cotangent and an optional final-state
+  cotangent: reverse-mode differentiation (torch autograd) of an fp64 torch
+  restatement of the same recurrence; small cases only.
 
 Both take packed inputs: q, k, g of shape [T_total, H, d_k], v of shape
 [T_total, H, d_v], beta logits [T_total, H], ``cu_seqlens`` int offsets
@@ -293,3 +297,60 @@ def decode_token(x, conv_w, conv_state, g, beta, state, *, H, Dk, Dv, scale=None
     if g_out is not None:
         o = output_gate(o.reshape(N, H * Dv), _f64(g_out).reshape(N, H * Dv), Dv, norm_eps).reshape(N, H, Dv)
     return o, cs, S
+
+
+# --------------------------------------------------------------------------- backward
+
+def backward(q, k, v, g, beta, do, *, dS_final=None, scale=None, initial_state=None, cu_seqlens=None,
+             use_qk_l2norm=True, lower_bound=None, beta_is_logit=True):
+    """Gradients of the chunkwise forward: given the output cotangent ``do``
+    [T_total, H, d_v] (and optionally ``dS_final`` [N, H, d_k, d_v] for the final
+    states), returns (dq, dk, dv, dg, dbeta, dS0) as fp64 numpy arrays, dS0 of the
+    initial states [N, H, d_k, d_v] (zeros when none are given).
+
+    The forward is the recurrence of page "atlas_core/kimi_k3/kda.rs" (module doc,
+    `l2norm_rows`, `kda_recurrent_step`) written out token by token in fp64 torch
+    operations, with the clamp g <- max(g, lower_bound) and beta a logit (sigmoid)
+    or a probability as in ``recurrent``; the gradients are its reverse-mode
+    derivatives (torch autograd: the definition differentiated, no other form).
+    Python loops over tokens: small cases only.
+    """
+    import torch
+
+    def t64(x, grad=False):
+        if x is None:
+            return None
+        a = torch.from_numpy(_f64(x).copy())
+        return a.requires_grad_(grad)
+
+    q, k, v, g, beta, cu, S0, N, H, Dk, Dv = _prep(q, k, v, g, beta, cu_seqlens, initial_state)
+    dO = _f64(do).reshape(q.shape[0], H, Dv)
+    tq, tk, tv, tg, tb = (t64(x, True) for x in (q, k, v, g, beta))
+    tS0 = t64(S0 if S0 is not None else np.zeros((N, H, Dk, Dv)), True)
+    if scale is None:
+        scale = 1.0 / np.sqrt(Dk)
+    outs, finals = [], []
+    for n in range(N):
+        S = tS0[n]
+        for t in range(int(cu[n]), int(cu[n + 1])):
+            qt, kt = tq[t], tk[t]
+            if use_qk_l2norm:
+                qt = qt / torch.sqrt((qt * qt).sum(-1, keepdim=True) + 1e-6)
+                kt = kt / torch.sqrt((kt * kt).sum(-1, keepdim=True) + 1e-6)
+            gt = tg[t] if lower_bound is None else torch.clamp(tg[t], min=float(lower_bound))
+            b = torch.sigmoid(tb[t]) if beta_is_logit else tb[t]
+            S = torch.exp(gt)[..., :, None] * S                      # decay along the key axis
+            delta = b[:, None] * (tv[t] - torch.einsum("hkv,hk->hv", S, kt))
+            S = S + kt[..., :, None] * delta[..., None, :]
+            outs.append((t, scale * torch.einsum("hkv,hk->hv", S, qt)))
+        finals.append(S)
+    loss = sum((o * torch.from_numpy(dO[t])).sum() for t, o in outs)
+    if dS_final is not None:
+        dSf = _f64(dS_final).reshape(N, H, Dk, Dv)
+        loss = loss + sum((finals[n] * torch.from_numpy(dSf[n])).sum() for n in range(N))
+    if not torch.is_tensor(loss):  # no tokens and no final-state cotangent
+        z = lambda a: np.zeros(a.shape)
+        return z(q), z(k), z(v), z(g), z(beta), np.zeros((N, H, Dk, Dv))
+    grads = torch.autograd.grad(loss, (tq, tk, tv, tg, tb, tS0), allow_unused=True)
+    return tuple(np.zeros(x.shape) if gr is None else gr.detach().numpy()
+                 for gr, x in zip(grads, (tq, tk, tv, tg, tb, tS0)))
