@@ -200,6 +200,46 @@ typedef struct {
 KDA_API kda_status kda_decode_token(const kda_token_args *args, void *stream);
 
 /*
+ * Gradients of the chunkwise forward (the operator above with gate_mode
+ * KDA_GATE_LOG): given the output cotangent `dout` and optionally a final-state
+ * cotangent, returns dq, dk, dv, dg, dbeta and the initial-state gradient. The
+ * pages give no backward formulas: these are the derivatives of the token
+ * recurrence of page "atlas_core/kimi_k3/kda.rs" (through the L2 norm, the clamp
+ * g <- max(g, lower_bound), whose gradient is zero where the bound is taken, and
+ * the sigmoid of beta). First implementation: a recompute of the forward that
+ * stores the state every 16 tokens, then a reverse sweep per (sequence, head)
+ * that rebuilds each token's entering state from its checkpoint; CUDA cores,
+ * fp32. Validation as kda_chunk_fwd; in-kernel gate forms return UNSUPPORTED.
+ */
+typedef struct {
+    kda_dtype dtype;            /* of q, k, v, g, beta, dout and dq, dk, dv, dg, dbeta */
+    int B, T, H, Dk, Dv;        /* as kda_chunk_args */
+    const void *q, *k, *v, *g, *beta;
+    const void *dout;           /* [B,T,H,Dv] cotangent of o */
+    float scale;                /* <= 0 or NaN selects 1/sqrt(Dk) */
+    const float *initial_state; /* [N,H,Dk,Dv] or NULL (zeros) */
+    const float *dfinal_state;  /* [N,H,Dk,Dv] cotangent of the final state, or NULL */
+    void *dq, *dk, *dv, *dg;    /* out, layouts of q, k, v, g */
+    void *dbeta;                /* out, [B,T,H] */
+    float *dinitial_state;      /* out [N,H,Dk,Dv], or NULL when not wanted */
+    const int32_t *cu_seqlens;  /* as kda_chunk_args */
+    const int32_t *cu_seqlens_host;
+    int N;
+    int use_qk_l2norm;
+    int has_lower_bound;
+    float lower_bound;
+    int beta_is_prob;           /* 1: beta is a probability (dbeta is then d/dprob) */
+    void *workspace;            /* device scratch of kda_chunk_bwd_workspace_size() bytes, 16-byte aligned */
+    size_t workspace_bytes;
+} kda_chunk_bwd_args;
+
+/* Bytes of workspace kda_chunk_bwd needs (the state checkpoints: one d_k x d_v
+ * fp32 state per 16 tokens per head, plus a small header). Only shapes are read. */
+KDA_API kda_status kda_chunk_bwd_workspace_size(const kda_chunk_bwd_args *args, size_t *bytes);
+
+KDA_API kda_status kda_chunk_bwd(const kda_chunk_bwd_args *args, void *stream);
+
+/*
  * Chunkwise forward for callers that cannot allocate device memory. This entry
  * point has no counterpart in the pages; it exists for callers that run under a
  * fixed device-memory plan and may not allocate once running (an inference

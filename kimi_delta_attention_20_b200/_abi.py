@@ -79,10 +79,30 @@ class TokenArgs(ctypes.Structure):
     ]
 
 
+class BwdArgs(ctypes.Structure):
+    _fields_ = [
+        ("dtype", ctypes.c_int),
+        ("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
+        ("Dk", ctypes.c_int), ("Dv", ctypes.c_int),
+        ("q", _vp), ("k", _vp), ("v", _vp), ("g", _vp), ("beta", _vp),
+        ("dout", _vp),
+        ("scale", ctypes.c_float),
+        ("initial_state", _vp), ("dfinal_state", _vp),
+        ("dq", _vp), ("dk", _vp), ("dv", _vp), ("dg", _vp), ("dbeta", _vp),
+        ("dinitial_state", _vp),
+        ("cu_seqlens", _vp), ("cu_seqlens_host", _vp),
+        ("N", ctypes.c_int),
+        ("use_qk_l2norm", ctypes.c_int),
+        ("has_lower_bound", ctypes.c_int), ("lower_bound", ctypes.c_float),
+        ("beta_is_prob", ctypes.c_int),
+        ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 # every symbol include/kda.h declares
 EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_noalloc",
-           "kda_recurrent_step", "kda_decode_token", "kda_status_string", "kda_last_cuda_error",
-           "kda_version")
+           "kda_recurrent_step", "kda_decode_token", "kda_chunk_bwd_workspace_size", "kda_chunk_bwd",
+           "kda_status_string", "kda_last_cuda_error", "kda_version")
 
 _lib = None
 
@@ -107,6 +127,10 @@ def load():
     lib.kda_recurrent_step.restype = ctypes.c_int
     lib.kda_decode_token.argtypes = [ctypes.POINTER(TokenArgs), _vp]
     lib.kda_decode_token.restype = ctypes.c_int
+    lib.kda_chunk_bwd_workspace_size.argtypes = [ctypes.POINTER(BwdArgs), ctypes.POINTER(ctypes.c_size_t)]
+    lib.kda_chunk_bwd_workspace_size.restype = ctypes.c_int
+    lib.kda_chunk_bwd.argtypes = [ctypes.POINTER(BwdArgs), _vp]
+    lib.kda_chunk_bwd.restype = ctypes.c_int
     lib.kda_status_string.argtypes = [ctypes.c_int]
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_last_cuda_error.argtypes = []

@@ -16,6 +16,8 @@ cudaError_t launch_chunk_tc(const ChunkParams &p, int Dk, int Dv, void *workspac
 size_t chunk_2pass_workspace_bytes(const ChunkParams &p);
 cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int32_t *cu_host, cudaStream_t st);
 bool token_conv_supported(int K);
+size_t bwd_workspace_bytes(bool varlen, long long T, int N, int H, int Dk, int Dv);
+cudaError_t launch_bwd(BwdParams p, bool bf16, int Dk, int Dv, void *workspace, cudaStream_t st);
 cudaError_t launch_token(const TokenParams &tp, bool bf16, int Dk, int Dv, cudaStream_t st);
 }  // namespace kda
 
@@ -82,6 +84,19 @@ kda_status check_chunk_shape(const kda_chunk_args *a, int *N_out) {
 namespace kda {
 void record_cuda_error(int e) { g_last_cuda_error = e; }
 }  // namespace kda
+
+namespace {
+// The forward's shape view of backward arguments (shared validation).
+kda_chunk_args fwd_view(const kda_chunk_bwd_args *a) {
+    kda_chunk_args f{};
+    f.dtype = a->dtype;
+    f.B = a->B; f.T = a->T; f.H = a->H; f.Dk = a->Dk; f.Dv = a->Dv;
+    f.cu_seqlens = a->cu_seqlens; f.cu_seqlens_host = a->cu_seqlens_host; f.N = a->N;
+    f.has_lower_bound = a->has_lower_bound; f.lower_bound = a->lower_bound;
+    f.gate_mode = KDA_GATE_LOG;
+    return f;
+}
+}  // namespace
 
 namespace kda {
 // Smallest workspace kda_chunk_fwd accepts for these arguments (the single-pass
@@ -257,6 +272,55 @@ kda_status kda_decode_token(const kda_token_args *a, void *stream) {
     tp.g_out = a->g_out;
     tp.norm_eps = a->norm_eps;
     return cuda_status(kda::launch_token(tp, bf16, a->Dk, a->Dv, static_cast<cudaStream_t>(stream)));
+}
+
+kda_status kda_chunk_bwd_workspace_size(const kda_chunk_bwd_args *a, size_t *bytes) {
+    if (!a || !bytes) return KDA_ERR_INVALID_ARGUMENT;
+    const kda_chunk_args f = fwd_view(a);
+    int N = 0;
+    kda_status s = check_chunk_shape(&f, &N);
+    if (s != KDA_OK) return s;
+    *bytes = kda::bwd_workspace_bytes(a->cu_seqlens != nullptr, a->T, N, a->H, a->Dk, a->Dv);
+    return KDA_OK;
+}
+
+kda_status kda_chunk_bwd(const kda_chunk_bwd_args *a, void *stream) {
+    if (!a) return KDA_ERR_INVALID_ARGUMENT;
+    const kda_chunk_args f = fwd_view(a);
+    int N = 0;
+    kda_status s = check_chunk_shape(&f, &N);
+    if (s != KDA_OK) return s;
+    const bool bf16 = a->dtype == KDA_DTYPE_BF16;
+    const size_t esz = bf16 ? 2 : 4;
+    const long long ntok = (long long)a->B * a->T;
+    if (ntok > 0) {
+        const void *need[] = {a->q, a->k, a->v, a->g, a->beta, a->dout, a->dq, a->dk, a->dv, a->dg, a->dbeta};
+        for (const void *ptr : need)
+            if (!ptr || !aligned(ptr, esz)) return KDA_ERR_INVALID_ARGUMENT;
+    }
+    if ((a->initial_state && !aligned(a->initial_state, 16)) || (a->dfinal_state && !aligned(a->dfinal_state, 16)) ||
+        (a->dinitial_state && !aligned(a->dinitial_state, 16)))
+        return KDA_ERR_INVALID_ARGUMENT;
+    if (a->cu_seqlens_host) {
+        const int32_t *cu = a->cu_seqlens_host;
+        if (cu[0] != 0 || cu[N] != a->T) return KDA_ERR_INVALID_ARGUMENT;
+        for (int n = 0; n < N; ++n)
+            if (cu[n + 1] < cu[n]) return KDA_ERR_INVALID_ARGUMENT;
+    }
+    if (!a->cu_seqlens && a->cu_seqlens_host) return KDA_ERR_INVALID_ARGUMENT;
+    const size_t need_ws = kda::bwd_workspace_bytes(a->cu_seqlens != nullptr, a->T, N, a->H, a->Dk, a->Dv);
+    if (!a->workspace || a->workspace_bytes < need_ws || !aligned(a->workspace, 16)) return KDA_ERR_WORKSPACE;
+    kda::BwdParams p{};
+    p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta; p.dout = a->dout;
+    p.S0 = a->initial_state; p.dSf = a->dfinal_state;
+    p.dq = a->dq; p.dk = a->dk; p.dv = a->dv; p.dg = a->dg; p.dbeta = a->dbeta; p.dS0 = a->dinitial_state;
+    p.cu_seqlens = a->cu_seqlens; p.T = a->T; p.N = N; p.H = a->H;
+    p.scale = resolve_scale(a->scale, a->Dk);
+    p.use_l2 = a->use_qk_l2norm ? 1 : 0;
+    p.has_lb = a->has_lower_bound ? 1 : 0;
+    p.lb = a->lower_bound;
+    p.beta_prob = a->beta_is_prob ? 1 : 0;
+    return cuda_status(kda::launch_bwd(p, bf16, a->Dk, a->Dv, a->workspace, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

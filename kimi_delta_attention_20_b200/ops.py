@@ -68,7 +68,7 @@ def _gate_fields(a, device, H, Dk, A_log, dt_bias, use_gate_in_kernel, safe_gate
         a.lower_bound = 0.0
 
 
-def chunk_kda(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+def _chunk_kda_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
               beta: torch.Tensor, *, A_log: Optional[torch.Tensor] = None,
               dt_bias: Optional[torch.Tensor] = None, scale: Optional[float] = None,
               initial_state: Optional[torch.Tensor] = None, output_final_state: bool = False,
@@ -94,6 +94,10 @@ def chunk_kda(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor
     ``cu_seqlens`` (int32, [N+1], B == 1) packs N sequences. ``chunk_size``
     <= 32 selects 32-token chunks (CUDA-core kernel), anything else 64.
     Returns (o [B, T, H, Dv], final_state [N, H, Dk, Dv] fp32 or None).
+
+    When autograd is on and q, k, v, g, beta or initial_state requires grad, the
+    call is recorded for the backward (``chunk_kda_bwd``): gradients flow to
+    those inputs (the log-decay form; in-kernel gate forms raise).
     """
     lib = _abi.load()
     for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta)):
@@ -281,3 +285,112 @@ def decode_token(x: torch.Tensor, conv_w: torch.Tensor, conv_state: torch.Tensor
     with torch.cuda.device(x.device):
         _abi.check(lib.kda_decode_token(ctypes.byref(a), _stream(x.device)), "kda_decode_token")
     return o
+
+
+def chunk_kda_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor, beta: torch.Tensor,
+                  dout: torch.Tensor, *, dfinal_state: Optional[torch.Tensor] = None,
+                  initial_state: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                  use_qk_l2norm_in_kernel: bool = False, use_beta_sigmoid_in_kernel: bool = True,
+                  lower_bound: Optional[float] = None, cu_seqlens: Optional[torch.Tensor] = None,
+                  want_dinitial_state: bool = True, workspace: Optional[torch.Tensor] = None):
+    """Gradients of ``chunk_kda`` (log-decay gate, the derivatives of the token
+    recurrence of page "atlas_core/kimi_k3/kda.rs"; the pages give no backward
+    formulas). Arguments as ``chunk_kda`` plus ``dout`` [B, T, H, Dv] (cotangent of
+    o) and ``dfinal_state`` [N, H, Dk, Dv] fp32 (cotangent of the final state) or
+    None. Returns (dq, dk, dv, dg, dbeta, dinitial_state or None); gradients have
+    the dtype of q, dinitial_state is fp32. The gradient of g is zero where the
+    lower bound is taken (g < lower_bound).
+    """
+    lib = _abi.load()
+    for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta), ("dout", dout)):
+        _need_cuda(name, t)
+    if q.dtype not in _DTYPES or any(t.dtype != q.dtype for t in (k, v, g, beta)):
+        raise ValueError("q, k, v, g, beta must share one dtype: float32 or bfloat16")
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    if k.shape != q.shape or g.shape != q.shape or v.shape != (B, T, H, Dv) or beta.shape != (B, T, H):
+        raise ValueError("shape mismatch among q, k, v, g, beta")
+    dout = dout.to(q.dtype).contiguous()
+    if dout.shape != v.shape:
+        raise ValueError("dout must have the shape of v")
+    cu_host = cu_dev = None
+    N = B
+    if cu_seqlens is not None:
+        if B != 1:
+            raise ValueError("cu_seqlens requires B == 1")
+        cu_host = cu_seqlens.detach().to("cpu", torch.int32).contiguous()
+        cu_dev = cu_seqlens.to(q.device, torch.int32).contiguous()
+        N = cu_host.numel() - 1
+    for name, t in (("initial_state", initial_state), ("dfinal_state", dfinal_state)):
+        if t is not None:
+            _need_cuda(name, t)
+            if t.dtype != torch.float32 or t.shape != (N, H, Dk, Dv):
+                raise ValueError(f"{name} must be float32 [{N}, {H}, {Dk}, {Dv}]")
+    if dfinal_state is not None:
+        dfinal_state = dfinal_state.contiguous()
+    grads = [torch.empty_like(t) for t in (q, k, v, g, beta)]
+    dS0 = torch.empty(N, H, Dk, Dv, dtype=torch.float32, device=q.device) if want_dinitial_state else None
+    a = _abi.BwdArgs()
+    a.dtype = _DTYPES[q.dtype]
+    a.B, a.T, a.H, a.Dk, a.Dv = B, T, H, Dk, Dv
+    a.q, a.k, a.v, a.g, a.beta, a.dout = (_ptr(t) for t in (q, k, v, g, beta, dout))
+    a.scale = float("nan") if scale is None else float(scale)
+    a.initial_state, a.dfinal_state = _ptr(initial_state), _ptr(dfinal_state)
+    a.dq, a.dk, a.dv, a.dg, a.dbeta = (_ptr(t) for t in grads)
+    a.dinitial_state = _ptr(dS0)
+    a.cu_seqlens, a.cu_seqlens_host, a.N = _ptr(cu_dev), _ptr(cu_host), N
+    a.use_qk_l2norm = int(bool(use_qk_l2norm_in_kernel))
+    a.has_lower_bound = int(lower_bound is not None)
+    a.lower_bound = float(lower_bound) if lower_bound is not None else 0.0
+    a.beta_is_prob = int(not use_beta_sigmoid_in_kernel)
+    nbytes = ctypes.c_size_t(0)
+    _abi.check(lib.kda_chunk_bwd_workspace_size(ctypes.byref(a), ctypes.byref(nbytes)), "kda_chunk_bwd_workspace_size")
+    if workspace is None or workspace.numel() * workspace.element_size() < nbytes.value:
+        workspace = torch.empty(max(nbytes.value, 16), dtype=torch.uint8, device=q.device)
+    a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    with torch.cuda.device(q.device):
+        _abi.check(lib.kda_chunk_bwd(ctypes.byref(a), _stream(q.device)), "kda_chunk_bwd")
+    return (*grads, dS0)
+
+
+class _ChunkKDA(torch.autograd.Function):
+    """chunk_kda recorded for autograd: forward by kda_chunk_fwd, backward by kda_chunk_bwd."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, g, beta, initial_state, kw):
+        o, fs = _chunk_kda_fwd(q, k, v, g, beta, initial_state=initial_state, output_final_state=True, **kw)
+        ctx.save_for_backward(q, k, v, g, beta, initial_state)
+        ctx.kw = kw
+        return o, fs
+
+    @staticmethod
+    def backward(ctx, do, dfs):
+        q, k, v, g, beta, S0 = ctx.saved_tensors
+        kw = ctx.kw
+        if do is None:
+            do = torch.zeros(v.shape, dtype=v.dtype, device=v.device)
+        dq, dk, dv, dg, db, dS0 = chunk_kda_bwd(
+            q, k, v, g, beta, do, dfinal_state=dfs, initial_state=S0, scale=kw.get("scale"),
+            use_qk_l2norm_in_kernel=kw.get("use_qk_l2norm_in_kernel", False),
+            use_beta_sigmoid_in_kernel=kw.get("use_beta_sigmoid_in_kernel", True),
+            lower_bound=kw.get("lower_bound"), cu_seqlens=kw.get("cu_seqlens"),
+            want_dinitial_state=S0 is not None and ctx.needs_input_grad[5])
+        return dq, dk, dv, dg, db, dS0, None
+
+
+def chunk_kda(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+              beta: torch.Tensor, *, initial_state: Optional[torch.Tensor] = None,
+              output_final_state: bool = False, **kw) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    tensors = (q, k, v, g, beta, initial_state)
+    if torch.is_grad_enabled() and any(t is not None and t.requires_grad for t in tensors):
+        if kw.get("use_gate_in_kernel") or kw.get("A_log") is not None:
+            raise NotImplementedError("gradients of the in-kernel gate forms are not provided; pass the log-decay g")
+        for name in ("out", "final_state_out"):
+            if kw.get(name) is not None:
+                raise ValueError(f"{name} cannot be used when gradients are recorded")
+        o, fs = _ChunkKDA.apply(q, k, v, g, beta, initial_state, kw)
+        return o, (fs if output_final_state else None)
+    return _chunk_kda_fwd(q, k, v, g, beta, initial_state=initial_state, output_final_state=output_final_state, **kw)
+
+
+chunk_kda.__doc__ = _chunk_kda_fwd.__doc__

@@ -1,0 +1,101 @@
+"""GPU parity of the chunk_kda backward (kda_chunk_bwd) against the fp64 oracle
+(`oracle.backward`, the derivatives of the token recurrence of page
+"atlas_core/kimi_k3/kda.rs", pinned by finite differences), and of the autograd
+route through `chunk_kda`. Lengths straddle the 16-token checkpoints of the
+reverse sweep.
+"""
+import numpy as np
+import pytest
+import torch
+
+import kda_inputs as KI
+import oracle
+from kda_check import check
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+NAMES = ("dq", "dk", "dv", "dg", "dbeta", "dS0")
+
+
+def draw(lens, H, Dk, Dv, dtype, seed, **kw):
+    inp = KI.draw_chunk(1, sum(lens), H, Dk, Dv, dtype=dtype, seed=seed, seqlens=lens, init_state=True, **kw)
+    gen = torch.Generator().manual_seed(seed + 1000)
+    inp["do"] = torch.randn(inp["v"].shape, generator=gen).to(dtype)
+    inp["dSf"] = torch.randn(inp["initial_state"].shape, generator=gen) * 0.5
+    return inp
+
+
+def run_and_compare(inp, dtype, *, lower_bound=None, l2=True, prob=False, final=True, tag=""):
+    import kimi_delta_attention_20_b200 as kda
+    d = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    got = kda.chunk_kda_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["do"],
+                            dfinal_state=d["dSf"] if final else None, initial_state=d["initial_state"],
+                            use_qk_l2norm_in_kernel=l2, use_beta_sigmoid_in_kernel=not prob,
+                            lower_bound=lower_bound, cu_seqlens=d["cu_seqlens"])
+    torch.cuda.synchronize()
+    want = oracle.backward(inp["q"][0], inp["k"][0], inp["v"][0], inp["g"][0], inp["beta"][0], inp["do"][0],
+                           dS_final=inp["dSf"] if final else None, initial_state=inp["initial_state"],
+                           cu_seqlens=inp["cu_seqlens"], use_qk_l2norm=l2, lower_bound=lower_bound,
+                           beta_is_logit=not prob)
+    for name, gt, wt in zip(NAMES, got, want):
+        if name != "dS0":
+            gt = gt[0]
+        check(f"{tag} {name}", gt, wt, dtype)
+    return got
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dims", [(32, 32), (64, 64), (128, 128), (32, 64), (128, 32)])
+def test_backward_matches_oracle(dims, dtype):
+    Dk, Dv = dims
+    inp = draw((15, 16, 17, 1, 33), 2, Dk, Dv, dtype, seed=Dk + Dv)
+    run_and_compare(inp, dtype, lower_bound=-5.0, tag=f"{dims}")
+
+
+@pytest.mark.parametrize("case", ["no_final", "no_l2", "prob", "clamp_active", "empty_seqs"])
+def test_backward_options(case):
+    dtype = torch.float32
+    lens = (0, 20, 0, 9) if case == "empty_seqs" else (20, 9)
+    inp = draw(lens, 2, 64, 64, dtype, seed=90 + len(case))
+    kw = dict(lower_bound=-5.0)
+    if case == "no_final":
+        kw["final"] = False
+    elif case == "no_l2":
+        inp["k"] = (inp["k"].float() / 8.0).to(dtype)
+        kw["l2"] = False
+    elif case == "prob":
+        inp["beta"] = torch.sigmoid(inp["beta"].float()).to(dtype)
+        kw["prob"] = True
+    elif case == "clamp_active":
+        inp["g"] = (inp["g"].float() * 4.0).to(dtype)  # many gates below the bound
+        kw["lower_bound"] = -1.0
+    run_and_compare(inp, dtype, tag=case, **kw)
+
+
+def test_autograd_through_chunk_kda():
+    """loss.backward() through chunk_kda gives kda_chunk_bwd's gradients, which match the oracle."""
+    import kimi_delta_attention_20_b200 as kda
+    inp = draw((24, 40), 2, 32, 64, torch.float32, seed=95)
+    leaves = {n: inp[n].to(DEV).requires_grad_(True) for n in ("q", "k", "v", "g", "beta", "initial_state")}
+    o, S = kda.chunk_kda(leaves["q"], leaves["k"], leaves["v"], leaves["g"], leaves["beta"],
+                         initial_state=leaves["initial_state"], output_final_state=True,
+                         use_qk_l2norm_in_kernel=True, lower_bound=-5.0, cu_seqlens=inp["cu_seqlens"].to(DEV))
+    loss = (o * inp["do"].to(DEV)).sum() + (S * inp["dSf"].to(DEV)).sum()
+    loss.backward()
+    want = oracle.backward(inp["q"][0], inp["k"][0], inp["v"][0], inp["g"][0], inp["beta"][0], inp["do"][0],
+                           dS_final=inp["dSf"], initial_state=inp["initial_state"], cu_seqlens=inp["cu_seqlens"],
+                           lower_bound=-5.0)
+    for name, leaf, wt in zip(NAMES, ("q", "k", "v", "g", "beta", "initial_state"), want):
+        gt = leaves[leaf].grad
+        check(f"autograd {name}", gt if leaf == "initial_state" else gt[0], wt, torch.float32)
+
+
+def test_autograd_rejects_in_kernel_gate():
+    import kimi_delta_attention_20_b200 as kda
+    inp = KI.draw_chunk(1, 8, 2, 32, 32, seed=96, device=DEV, gate="input")
+    q = inp["q"].requires_grad_(True)
+    params = KI.draw_gate_params(2, 32, seed=96, device=DEV)
+    with pytest.raises(NotImplementedError):
+        kda.chunk_kda(q, inp["k"], inp["v"], inp["g"], inp["beta"], use_gate_in_kernel=True,
+                      A_log=params["A_log"], use_qk_l2norm_in_kernel=True)
