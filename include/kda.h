@@ -208,8 +208,9 @@ KDA_API kda_status kda_decode_token(const kda_token_args *args, void *stream);
  * g <- max(g, lower_bound), whose gradient is zero where the bound is taken, and
  * the sigmoid of beta). First implementation: a recompute of the forward that
  * stores the state every 16 tokens, then a reverse sweep per (sequence, head)
- * that rebuilds each token's entering state from its checkpoint; CUDA cores,
- * fp32. Validation as kda_chunk_fwd; in-kernel gate forms return UNSUPPORTED.
+ * that reruns each 16-token stretch forward from its checkpoint (keeping the
+ * entering states) and walks it back; CUDA cores, fp32. Validation as
+ * kda_chunk_fwd; g is the log-decay (the in-kernel gate forms are not covered).
  */
 typedef struct {
     kda_dtype dtype;            /* of q, k, v, g, beta, dout and dq, dk, dv, dg, dbeta */
@@ -233,8 +234,9 @@ typedef struct {
     size_t workspace_bytes;
 } kda_chunk_bwd_args;
 
-/* Bytes of workspace kda_chunk_bwd needs (the state checkpoints: one d_k x d_v
- * fp32 state per 16 tokens per head, plus a small header). Only shapes are read. */
+/* Bytes of workspace kda_chunk_bwd needs: the state checkpoints (one d_k x d_v fp32
+ * state per 16 tokens per head), a scratch of 16 states per (sequence, head) and a
+ * small header. Only shapes are read. */
 KDA_API kda_status kda_chunk_bwd_workspace_size(const kda_chunk_bwd_args *args, size_t *bytes);
 
 KDA_API kda_status kda_chunk_bwd(const kda_chunk_bwd_args *args, void *stream);

@@ -16,10 +16,11 @@
 //   dg_c     = a_c sum_j dS'_cj S_cj = sum_j dS'_cj S'_cj   (zero where g_c < lb)
 //   dS      <- diag(a) dS'          (the cotangent of the previous token's state)
 //   dq       = r_q (dq^ - q^ (q^ . dq^)) for q^ = r_q q, likewise dk.
-// The entering state of every token is rebuilt from a checkpoint written every
-// kCB tokens by a recompute of the forward (`kda_bwd_ckpt_kernel`), so the
-// reverse sweep (`kda_bwd_kernel`) repeats at most kCB - 1 forward steps per
-// token and stores nothing per token.
+// The entering state of every token comes from a checkpoint written every kCB
+// tokens by a recompute of the forward (`kda_bwd_ckpt_kernel`): per sub-chunk of
+// kCB tokens the reverse sweep (`kda_bwd_kernel`) runs the forward once from the
+// checkpoint, keeping each token's entering state in a per-head scratch (each
+// thread stores and later reloads only its own tile), then walks the tokens back.
 //
 // One CTA of 256 threads per (sequence, head). Thread (kg, vg) keeps rows
 // kg*RP .. kg*RP+RP-1, columns 4 vg .. 4 vg+3 of S and of dS as float4 in
@@ -189,6 +190,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) kda_bwd_kernel(BwdParams p) {
     const int H = p.H;
     const long long bos = seq_begin(p, n), eos = seq_end(p, n);
     const long long c0 = first_ckpt(p, n);
+    float *scr = p.scratch + nh * (long long)kCB * DK * DV;  // this head's per-token states
 
     float4 ds[RP], s[RP];
 #pragma unroll
@@ -202,12 +204,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) kda_bwd_kernel(BwdParams p) {
         const int cnt = (int)min((long long)kCB, eos - t0);
         const float *ck = p.ckpt + ((c0 + cs) * H + h) * DK * DV;
         load_tokens<Tin, DK, DV>(p, sm, t0, cnt, h, true);
-        for (int i = cnt - 1; i >= 0; --i) {
-            // the entering state of token i: checkpoint, then tokens 0 .. i-1 forward
+        // forward from the checkpoint, keeping every token's entering state
 #pragma unroll
-            for (int r = 0; r < RP; ++r) s[r] = *reinterpret_cast<const float4 *>(tile_ptr<DK, DV>(const_cast<float *>(ck),
+        for (int r = 0; r < RP; ++r)
+            s[r] = *reinterpret_cast<const float4 *>(tile_ptr<DK, DV>(const_cast<float *>(ck), kg * RP + r, vg));
+        for (int i = 0; i < cnt; ++i) {
+#pragma unroll
+            for (int r = 0; r < RP; ++r) *reinterpret_cast<float4 *>(tile_ptr<DK, DV>(scr + (long long)i * DK * DV, kg * RP + r, vg)) = s[r];
+            if (i + 1 < cnt) fwd_step<DK, DV>(sm, i, s);
+        }
+        for (int i = cnt - 1; i >= 0; --i) {
+            // the entering state of token i, stored by the forward pass over this sub-chunk
+#pragma unroll
+            for (int r = 0; r < RP; ++r) s[r] = *reinterpret_cast<const float4 *>(tile_ptr<DK, DV>(scr + (long long)i * DK * DV,
                                                                                                     kg * RP + r, vg));
-            for (int j = 0; j < i; ++j) fwd_step<DK, DV>(sm, j, s);
 
             // ---- token i: S', u = S'^T k^, dS += scale q^ do^T, ddelta = dS^T k^
             const float b = sm.b[i];
@@ -373,17 +383,18 @@ cudaError_t launch_bwd_dt(const BwdParams &p, int Dk, int Dv, cudaStream_t st) {
 
 }  // namespace
 
-// Workspace: [ckpt_off: N+1 ints, 256-byte block][checkpoints]
+// Workspace: [ckpt_off: N+1 ints, 256-byte block][per-head scratch: kCB states][checkpoints]
 size_t bwd_workspace_bytes(bool varlen, long long T, int N, int H, int Dk, int Dv) {
     const long long nck = varlen ? (T + kCB - 1) / kCB + N : (long long)N * ((T + kCB - 1) / kCB);
     const size_t head = (((size_t)(N + 1) * 4 + 255) / 256) * 256;
-    return head + (size_t)nck * H * Dk * Dv * 4;
+    return head + (size_t)N * H * kCB * Dk * Dv * 4 + (size_t)nck * H * Dk * Dv * 4;
 }
 
 cudaError_t launch_bwd(BwdParams p, bool bf16, int Dk, int Dv, void *workspace, cudaStream_t st) {
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     p.ckpt_off = reinterpret_cast<int *>(ws);
-    p.ckpt = reinterpret_cast<float *>(ws + (((size_t)(p.N + 1) * 4 + 255) / 256) * 256);
+    p.scratch = reinterpret_cast<float *>(ws + (((size_t)(p.N + 1) * 4 + 255) / 256) * 256);
+    p.ckpt = p.scratch + (size_t)p.N * p.H * kCB * Dk * Dv;
     return bf16 ? launch_bwd_dt<__nv_bfloat16>(p, Dk, Dv, st) : launch_bwd_dt<float>(p, Dk, Dv, st);
 }
 
