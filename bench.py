@@ -10,7 +10,8 @@ states out). The decode step workload (64 sequences x 96 heads x 128 x 128
 fp32 state, bf16 token vectors, one fresh token per step) is timed in the
 same run, K' = 256 steps per timed pass, and reported under "decode"; so is the
 serving decode token (conv window 4 + SiLU, the recurrent step and the output
-gate fused, same geometry) under "decode_token".
+gate fused, same geometry) under "decode_token", and the chunk_kda backward on the
+B1 T8192 H16 d128 chunk workload under "backward".
 Inputs are resident in HBM and larger than L2 (3.9 GB chunk inputs, 384 MiB
 decode state), so no L2 flush runs between iterations.
 
@@ -102,6 +103,31 @@ def token_algorithmic(N, H, D, K):
     heads = N * H
     per_head = 2 * D * D * 4 + 2 * 3 * D * K * 4 + (3 * D + 3 * D) * 2 + 2
     return heads * per_head + H * 3 * D * K * 4
+
+
+# chunk_kda backward: the B1 T8192 H16 d128 lb-5 chunk workload with an output and a
+# final-state cotangent; two kernels per call (checkpoints, reverse sweep)
+BWD_WL = 2
+BWD_LAUNCHES = 2
+# FP32 FMA peak of the part: 148 SMs x 128 FP32 lanes x 2 flops x 1965 MHz
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def bwd_algorithmic(wl):
+    """Flops and bytes of one chunk_kda backward call on workload wl.
+
+    Flops per token-head (fp32, the token recurrence): one forward step to rebuild
+    the entering state (S' = a S, u = S'^T k, S += k delta^T: 5 d_k d_v) and the
+    reverse step (S', u, dS += q do^T, ddelta = dS^T k, the four row sums S' do,
+    dS delta, S' ddelta, dS . S', dS - b k ddelta^T and the decay of dS:
+    18 d_k d_v). Bytes: q, k, v, g, do, beta read, dq, dk, dv, dg, dbeta written,
+    the final-state cotangent read and the initial-state gradient written.
+    """
+    th = wl.tokens * wl.H
+    esz = 2
+    per_th = 2 * (3 * wl.Dk + 2 * wl.Dv) * esz + 2 * esz
+    states = 2 * wl.n_seqs * wl.H * wl.Dk * wl.Dv * 4
+    return th * 23 * wl.Dk * wl.Dv, th * per_th + states
 
 
 def decode_algorithmic(wl):
@@ -251,6 +277,21 @@ def run_kda(args, rank, world, local_rank):
         kda.decode_token(tk["x"][i], tk["w"], tk["cs"], tk["g"][i], tk["beta"][i], tk["S0"],
                          g_out=tk["g_out"][i], lower_bound=-5.0, out=tk_o)
 
+    bwl = KI.CHUNK_WORKLOADS[BWD_WL]
+    if args.only in (None, "bwd"):
+        binp = KI.chunk_inputs(bwl, device=dev)
+        bgen = torch.Generator(device=dev)
+        bgen.manual_seed(bwl.seed + 1000)
+        b_do = torch.randn(binp["v"].shape, generator=bgen, device=dev).to(bwl.dtype)
+        b_dSf = torch.randn(bwl.n_seqs, bwl.H, bwl.Dk, bwl.Dv, generator=bgen, device=dev) * 0.5
+        b_ws = torch.empty(kda.chunk_bwd_workspace_bytes(bwl.B, bwl.T, bwl.H, bwl.Dk, bwl.Dv, N=bwl.n_seqs),
+                           dtype=torch.uint8, device=dev)
+
+    def bwd_step():
+        return kda.chunk_kda_bwd(binp["q"], binp["k"], binp["v"], binp["g"], binp["beta"], b_do,
+                                 dfinal_state=b_dSf, use_qk_l2norm_in_kernel=True,
+                                 lower_bound=bwl.lower_bound, workspace=b_ws)
+
     if args.only in (None, "decode"):
         dinp = KI.decode_inputs(dwl, device=dev)
         state = dinp["state"].clone()
@@ -272,7 +313,8 @@ def run_kda(args, rank, world, local_rank):
 
     if args.only:
         # one kernel, few launches: the shape profiler captures use
-        one = {"chunk": chunk_step, "decode": lambda: decode_step(0), "token": lambda: token_step(0)}[args.only]
+        one = {"chunk": chunk_step, "decode": lambda: decode_step(0), "token": lambda: token_step(0),
+               "bwd": bwd_step}[args.only]
         for _ in range(args.warmup):
             one()
         torch.cuda.synchronize(dev)
@@ -338,6 +380,17 @@ def run_kda(args, rank, world, local_rank):
         k1.record(stream)
         torch.cuda.synchronize(dev); barrier()
         tok_ms = max_over_ranks(k0.elapsed_time(k1)) / ntok
+        # chunk_kda backward: K timed calls
+        for _ in range(args.warmup):
+            bwd_step()
+        barrier(); torch.cuda.synchronize(dev)
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(args.steps):
+            bwd_step()
+        b1.record(stream)
+        torch.cuda.synchronize(dev); barrier()
+        bwd_ms = max_over_ranks(b0.elapsed_time(b1)) / args.steps
     clk = clocks.summary()
 
     # end to end through the public API with host buffers: pinned host inputs
@@ -379,6 +432,7 @@ def run_kda(args, rank, world, local_rank):
     dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
     tok_bytes = token_algorithmic(TOKEN_WL["N"], TOKEN_WL["H"], TOKEN_WL["D"], TOKEN_WL["K"])
     tok_gbs = tok_bytes / (tok_ms * 1e-3) / 1e9
+    bwd_flops, bwd_bytes = bwd_algorithmic(bwl)
     chunk_sha = source_sha(*CHUNK_SOURCES)
     result = {
         "metric": METRIC,
@@ -429,9 +483,22 @@ def run_kda(args, rank, world, local_rank):
                          "frac": tok_gbs / hbm_peak, "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": tok_bytes},
         },
+        "backward": {
+            "value": whole_job_rate(world, bwl.tokens, bwd_ms), "unit": "tokens/s", "ms_per_step": bwd_ms,
+            "steps_timed": args.steps,
+            "workload": "chunk_kda backward: B1 T8192 H16 d128, bf16, lower_bound=-5, output and "
+                        "final-state cotangents, initial-state gradient out",
+            "roofline": {"bound": "alu", "achieved": bwd_flops / (bwd_ms * 1e-3) / 1e12,
+                         "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                         "frac": bwd_flops / (bwd_ms * 1e-3) / 1e12 / FP32_PEAK_TFLOPS,
+                         "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 x 1965 MHz",
+                         "algorithmic_flops_per_launch": bwd_flops,
+                         "hbm": {"algorithmic_bytes_per_launch": bwd_bytes,
+                                 "achieved_gbs": bwd_bytes / (bwd_ms * 1e-3) / 1e9}},
+        },
         "e2e": {"value": whole_job_rate(world, wl.tokens, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": args.steps * (CHUNK_LAUNCHES + 2 * DECODE_STEPS_PER_PASS),
+        "gpu_launches": args.steps * (CHUNK_LAUNCHES + 2 * DECODE_STEPS_PER_PASS + BWD_LAUNCHES),
         "clocks": clk,
         "library": os.path.relpath(_abi.LIB_PATH, ROOT),
     }
@@ -497,7 +564,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["chunk", "decode", "token"], default=None,
+    ap.add_argument("--only", choices=["chunk", "decode", "token", "bwd"], default=None,
                     help="run one leg only and print its timing (for profiler captures)")
     ap.add_argument("--workload", type=int, default=None,
                     help="with --only chunk: chunk workload index (default: the varlen H=96 one)")

@@ -6,6 +6,7 @@ update + SiLU, the recurrent step and the output gate in one launch) call the
 C-ABI library libkda.so built from csrc/
 (`python -m kimi_delta_attention_20_b200.build`).
 """
-from .ops import chunk_kda, chunk_kda_bwd, chunk_workspace_bytes, decode_token, recurrent_step  # noqa: F401
+from .ops import chunk_bwd_workspace_bytes, chunk_kda, chunk_kda_bwd, chunk_workspace_bytes, decode_token, recurrent_step  # noqa: F401
 
-__all__ = ["chunk_kda", "chunk_kda_bwd", "recurrent_step", "decode_token", "chunk_workspace_bytes"]
+__all__ = ["chunk_kda", "chunk_kda_bwd", "recurrent_step", "decode_token", "chunk_workspace_bytes",
+           "chunk_bwd_workspace_bytes"]

@@ -294,9 +294,10 @@ kda_status kda_chunk_bwd(const kda_chunk_bwd_args *a, void *stream) {
     const size_t esz = bf16 ? 2 : 4;
     const long long ntok = (long long)a->B * a->T;
     if (ntok > 0) {
-        const void *need[] = {a->q, a->k, a->v, a->g, a->beta, a->dout, a->dq, a->dk, a->dv, a->dg, a->dbeta};
-        for (const void *ptr : need)
-            if (!ptr || !aligned(ptr, esz)) return KDA_ERR_INVALID_ARGUMENT;
+        const void *rows[] = {a->q, a->k, a->v, a->g, a->dout, a->dq, a->dk, a->dv, a->dg};
+        for (const void *ptr : rows)
+            if (!ptr || !aligned(ptr, 16)) return KDA_ERR_INVALID_ARGUMENT;
+        if (!a->beta || !aligned(a->beta, esz) || !a->dbeta || !aligned(a->dbeta, esz)) return KDA_ERR_INVALID_ARGUMENT;
     }
     if ((a->initial_state && !aligned(a->initial_state, 16)) || (a->dfinal_state && !aligned(a->dfinal_state, 16)) ||
         (a->dinitial_state && !aligned(a->dinitial_state, 16)))

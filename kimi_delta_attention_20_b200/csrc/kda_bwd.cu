@@ -59,10 +59,18 @@ struct BwdTile {
     static_assert(VG == 4 && KG == 32 && RP * KG == DK && RP >= 1 && NS >= 1 && NS <= 8, "state tiling");
 };
 
+// Raw inputs of one stretch, copied in by cp.async while the previous stretch runs.
+template <typename Tin, int DK>
+struct Stage {
+    Tin k[kCB][DK], g[kCB][DK], q[kCB][DK];  // q: reverse sweep only
+    Tin v[kCB][kDVC], dout[kCB][kDVC];       // this CTA's value columns; dout: reverse sweep only
+};
+
 // Token vectors of one stretch (fp32; k^ normalised) and the key-axis reduction
 // buffers: what the forward recompute needs.
-template <int DK>
+template <typename Tin, int DK>
 struct FwdSmem {
+    Stage<Tin, DK> st;
     float kh[kCB][DK], al[kCB][DK];
     float v[kCB][kDVC];
     float b[kCB], rk[kCB];
@@ -72,8 +80,8 @@ struct FwdSmem {
 // The reverse sweep adds q^, the raw gate (for the clamp mask), the output
 // cotangent, and the per-slice terms of dq^, dk^, dg and db, double-buffered
 // across stretches so that one cluster barrier per stretch suffices.
-template <int DK>
-struct BwdSmem : FwdSmem<DK> {
+template <typename Tin, int DK>
+struct BwdSmem : FwdSmem<Tin, DK> {
     float qh[kCB][DK], graw[kCB][DK];
     float dout[kCB][kDVC];
     float rq[kCB];
@@ -125,34 +133,66 @@ __device__ __forceinline__ float colgroup_sum(float x) {
     return x;
 }
 
-// Load tokens [t0, t0 + cnt) of head h into shared memory: k^ (and q^ for the
-// reverse sweep; normalised when use_l2), the decay a = exp(max(g, lb)), this
-// CTA's columns of v (and of the output cotangent) and the write strength b.
-// Barriers on both sides: the previous stretch's readers are done before the
-// first write, and the vectors are complete on return.
-template <typename Tin, int DK, int DV, bool kRev, typename Sm>
-__device__ void load_tokens(const BwdParams &p, Sm &sm, long long t0, int cnt, int h, int col0) {
+__device__ __forceinline__ void cp_async16(void *sdst, const void *gsrc) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(sdst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Start the copy of tokens [t0, t0 + cnt) of head h into the stage: k, g (and q
+// for the reverse sweep) rows, and this CTA's columns of v (and of the output
+// cotangent), in 16-byte pieces. Returns this thread's raw beta (thread i < cnt
+// holds token i's); the load completes in the background like the copies.
+template <typename Tin, int DK, int DV, bool kRev>
+__device__ __forceinline__ float issue_stretch(const BwdParams &p, Stage<Tin, DK> &st, long long t0, int cnt, int h,
+                                               int col0) {
+    constexpr int EP = 16 / (int)sizeof(Tin);  // elements per piece
+    constexpr int RK = DK / EP, RV = kDVC / EP;
+    const int tid = threadIdx.x, H = p.H;
+    for (int e = tid; e < cnt * RK; e += kBwdThreads) {
+        const int i = e / RK, c = (e % RK) * EP;
+        const long long gi = ((t0 + i) * H + h) * DK + c;
+        cp_async16(&st.k[i][c], static_cast<const Tin *>(p.k) + gi);
+        cp_async16(&st.g[i][c], static_cast<const Tin *>(p.g) + gi);
+        if constexpr (kRev) cp_async16(&st.q[i][c], static_cast<const Tin *>(p.q) + gi);
+    }
+    for (int e = tid; e < cnt * RV; e += kBwdThreads) {
+        const int i = e / RV, c = (e % RV) * EP;
+        const long long gi = ((t0 + i) * H + h) * DV + col0 + c;
+        cp_async16(&st.v[i][c], static_cast<const Tin *>(p.v) + gi);
+        if constexpr (kRev) cp_async16(&st.dout[i][c], static_cast<const Tin *>(p.dout) + gi);
+    }
+    cp_async_commit();
+    return tid < cnt ? to_f32(static_cast<const Tin *>(p.beta)[(t0 + tid) * H + h]) : 0.f;
+}
+
+// Turn the staged stretch into the fp32 token vectors: k^ (and q^; normalised
+// when use_l2), the decay a = exp(max(g, lb)), v (and the output cotangent), the
+// write strength b. The first barrier publishes the copies and also separates
+// these writes from the previous stretch's last readers; on return the vectors
+// are complete and the stage is free for the next copy.
+template <typename Tin, int DK, bool kRev, typename Sm>
+__device__ void take_stretch(const BwdParams &p, Sm &sm, int cnt, float beta_raw) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int H = p.H;
+    cp_async_wait_all();
     __syncthreads();
     for (int e = tid; e < cnt * DK; e += kBwdThreads) {
         const int i = e / DK, c = e % DK;
-        const long long gi = ((t0 + i) * H + h) * DK + c;
-        sm.kh[i][c] = to_f32(static_cast<const Tin *>(p.k)[gi]);
-        const float gr = to_f32(static_cast<const Tin *>(p.g)[gi]);
+        sm.kh[i][c] = to_f32(sm.st.k[i][c]);
+        const float gr = to_f32(sm.st.g[i][c]);
         sm.al[i][c] = expf(p.has_lb ? fmaxf(gr, p.lb) : gr);
         if constexpr (kRev) {
-            sm.qh[i][c] = to_f32(static_cast<const Tin *>(p.q)[gi]);
+            sm.qh[i][c] = to_f32(sm.st.q[i][c]);
             sm.graw[i][c] = gr;
         }
     }
     for (int e = tid; e < cnt * kDVC; e += kBwdThreads) {
         const int i = e / kDVC, c = e % kDVC;
-        const long long gi = ((t0 + i) * H + h) * DV + col0 + c;
-        sm.v[i][c] = to_f32(static_cast<const Tin *>(p.v)[gi]);
-        if constexpr (kRev) sm.dout[i][c] = to_f32(static_cast<const Tin *>(p.dout)[gi]);
+        sm.v[i][c] = to_f32(sm.st.v[i][c]);
+        if constexpr (kRev) sm.dout[i][c] = to_f32(sm.st.dout[i][c]);
     }
-    if (tid < cnt) sm.b[tid] = beta_value(to_f32(static_cast<const Tin *>(p.beta)[(t0 + tid) * H + h]), p.beta_prob);
+    if (tid < cnt) sm.b[tid] = beta_value(beta_raw, p.beta_prob);
     __syncthreads();
     for (int i = warp; i < cnt; i += kWarps) {
         float kk = 0.f, qq = 0.f;
@@ -176,8 +216,8 @@ __device__ void load_tokens(const BwdParams &p, Sm &sm, long long t0, int cnt, i
 
 // One forward step of token i of the loaded stretch on the register tile s; ph
 // selects the reduction buffer (alternating between consecutive steps).
-template <int DK, int DV>
-__device__ __forceinline__ void fwd_step(FwdSmem<DK> &sm, int i, int ph, float4 (&s)[BwdTile<DK, DV>::RP]) {
+template <typename Tin, int DK, int DV>
+__device__ __forceinline__ void fwd_step(FwdSmem<Tin, DK> &sm, int i, int ph, float4 (&s)[BwdTile<DK, DV>::RP]) {
     constexpr int RP = BwdTile<DK, DV>::RP;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, vg = tid & 3, kg = tid >> 2;
     float kr[RP], ar[RP];
@@ -219,7 +259,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_ckpt_kernel(BwdParams p) 
     using Tl = BwdTile<DK, DV>;
     constexpr int RP = Tl::RP, NS = Tl::NS;
     extern __shared__ __align__(16) uint8_t smraw[];
-    FwdSmem<DK> &sm = *reinterpret_cast<FwdSmem<DK> *>(smraw);
+    FwdSmem<Tin, DK> &sm = *reinterpret_cast<FwdSmem<Tin, DK> *>(smraw);
     const int tid = threadIdx.x, vg = tid & 3, kg = tid >> 2;
     const long long nh = blockIdx.x / NS;
     const int col0 = (int)(blockIdx.x % NS) * kDVC;
@@ -232,13 +272,15 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_ckpt_kernel(BwdParams p) 
                     : make_float4(0.f, 0.f, 0.f, 0.f);
     const long long c0 = first_ckpt(p, n);
     int ph = 0;
+    float braw = bos < eos ? issue_stretch<Tin, DK, DV, false>(p, sm.st, bos, (int)min((long long)kCB, eos - bos), h, col0) : 0.f;
     for (long long t0 = bos; t0 < eos; t0 += kCB) {
         const int cnt = (int)min((long long)kCB, eos - t0);
         float *ck = p.ckpt + ((c0 + (t0 - bos) / kCB) * p.H + h) * DK * DV;
 #pragma unroll
         for (int r = 0; r < RP; ++r) *state_ptr<DV>(ck, kg * RP + r, col0, vg) = s[r];
-        load_tokens<Tin, DK, DV, false>(p, sm, t0, cnt, h, col0);
-        for (int i = 0; i < cnt; ++i, ph ^= 1) fwd_step<DK, DV>(sm, i, ph, s);
+        take_stretch<Tin, DK, false>(p, sm, cnt, braw);
+        if (t0 + kCB < eos) braw = issue_stretch<Tin, DK, DV, false>(p, sm.st, t0 + kCB, (int)min((long long)kCB, eos - t0 - kCB), h, col0);
+        for (int i = 0; i < cnt; ++i, ph ^= 1) fwd_step<Tin, DK, DV>(sm, i, ph, s);
     }
 }
 
@@ -249,7 +291,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
     using Tl = BwdTile<DK, DV>;
     constexpr int RP = Tl::RP, NS = Tl::NS;
     extern __shared__ __align__(16) uint8_t smraw[];
-    BwdSmem<DK> &sm = *reinterpret_cast<BwdSmem<DK> *>(smraw);
+    BwdSmem<Tin, DK> &sm = *reinterpret_cast<BwdSmem<Tin, DK> *>(smraw);
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, vg = tid & 3, kg = tid >> 2;
@@ -269,12 +311,16 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
                       : make_float4(0.f, 0.f, 0.f, 0.f);
     int ph = 0;
     const long long len = eos - bos;
-    for (long long cs = (len + kCB - 1) / kCB - 1; cs >= 0; --cs) {
+    const long long nst = (len + kCB - 1) / kCB;
+    float braw = nst > 0 ? issue_stretch<Tin, DK, DV, true>(p, sm.st, bos + (nst - 1) * kCB,
+                                                            (int)(len - (nst - 1) * kCB), h, col0) : 0.f;
+    for (long long cs = nst - 1; cs >= 0; --cs) {
         const long long t0 = bos + cs * kCB;
         const int cnt = (int)min((long long)kCB, eos - t0);
         const int pb = (int)(cs & 1);
         const float *ck = p.ckpt + ((c0 + cs) * H + h) * DK * DV;
-        load_tokens<Tin, DK, DV, true>(p, sm, t0, cnt, h, col0);
+        take_stretch<Tin, DK, true>(p, sm, cnt, braw);
+        if (cs > 0) braw = issue_stretch<Tin, DK, DV, true>(p, sm.st, t0 - kCB, kCB, h, col0);
         // forward from the checkpoint, keeping every token's entering state; the
         // last one stays in s
 #pragma unroll
@@ -282,7 +328,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
         for (int i = 0; i + 1 < cnt; ++i, ph ^= 1) {
 #pragma unroll
             for (int r = 0; r < RP; ++r) scr[(i * RP + r) * kBwdThreads + tid] = s[r];
-            fwd_step<DK, DV>(sm, i, ph, s);
+            fwd_step<Tin, DK, DV>(sm, i, ph, s);
         }
         for (int i = cnt - 1; i >= 0; --i, ph ^= 1) {
             // the previous token's entering state, fetched while this token runs
@@ -377,7 +423,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
                 sq[j] = 0.f; sk[j] = 0.f; sg[j] = 0.f;
 #pragma unroll
                 for (int q = 0; q < NS; ++q) {
-                    const BwdSmem<DK> *rs = cluster.map_shared_rank(&sm, q);
+                    const BwdSmem<Tin, DK> *rs = cluster.map_shared_rank(&sm, q);
                     sq[j] += rs->pdq[pb][i][c];
                     sk[j] += rs->pdk[pb][i][c];
                     sg[j] += rs->pdg[pb][i][c];
@@ -430,7 +476,7 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st) {
     constexpr int NS = BwdTile<DK, DV>::NS;
     const long long heads = (long long)p.N * p.H;
     if (heads == 0) return cudaSuccess;
-    const int smem_f = (int)sizeof(FwdSmem<DK>), smem_b = (int)sizeof(BwdSmem<DK>);
+    const int smem_f = (int)sizeof(FwdSmem<Tin, DK>), smem_b = (int)sizeof(BwdSmem<Tin, DK>);
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(kda_bwd_ckpt_kernel<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_f)) != cudaSuccess)
         return e;

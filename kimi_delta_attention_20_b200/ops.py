@@ -182,6 +182,20 @@ def chunk_workspace_bytes(B, T, H, Dk, Dv, *, dtype=torch.bfloat16, N=None, varl
     return nbytes.value
 
 
+def chunk_bwd_workspace_bytes(B, T, H, Dk, Dv, *, dtype=torch.bfloat16, N=None, varlen=False):
+    """Workspace bytes kda_chunk_bwd needs for this geometry."""
+    lib = _abi.load()
+    a = _abi.BwdArgs()
+    a.dtype = _DTYPES[dtype]
+    a.B, a.T, a.H, a.Dk, a.Dv = B, T, H, Dk, Dv
+    a.N = N if N is not None else B
+    a.cu_seqlens = ctypes.c_void_p(1) if varlen else None  # only its presence is read
+    nbytes = ctypes.c_size_t(0)
+    _abi.check(lib.kda_chunk_bwd_workspace_size(ctypes.byref(a), ctypes.byref(nbytes)),
+               "kda_chunk_bwd_workspace_size")
+    return nbytes.value
+
+
 def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                    beta: torch.Tensor, state: torch.Tensor, *, A_log: Optional[torch.Tensor] = None,
                    dt_bias: Optional[torch.Tensor] = None, scale: Optional[float] = None,
