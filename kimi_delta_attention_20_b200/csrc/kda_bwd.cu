@@ -19,25 +19,25 @@
 //
 // Column split. The value columns of S and of dS evolve independently (u, delta,
 // ddelta and the decay act column by column), so each (sequence, head) runs as a
-// cluster of Dv/16 CTAs, one per 16-column slice. What sums over the value axis
-// (dq^, dk^, dg, db) is linear in the per-slice terms: every CTA keeps its slice's
-// terms for the kCB tokens of a stretch in shared memory, and after the stretch
-// the cluster adds them across its CTAs through distributed shared memory (a
-// fixed rank order, so the result is deterministic) and applies the L2-norm and
-// sigmoid chain rules once per token.
+// cluster of Dv/16 CTAs, one per 16-column slice, and inside a CTA each warp owns
+// 4 columns over all Dk rows: lane l keeps rows l*RP .. l*RP+RP-1 of those
+// columns of S and of dS as float4 in registers. Key-axis sums (u, ddelta) are
+// warp reductions (no block barrier; the forward recompute needs none at all);
+// value-axis sums over a warp's columns are lane-local. What sums over the value
+// axis across warps and CTAs (dq^, dk^, dg, db) is linear in the per-warp terms:
+// the 4 warps' terms of a token meet in shared memory (one block barrier per
+// token), every CTA keeps its slice's terms for the kCB tokens of a stretch, and
+// after the stretch the cluster adds them across its CTAs through distributed
+// shared memory (a fixed rank order, so the result is deterministic) and applies
+// the L2-norm and sigmoid chain rules once per token.
 //
 // The entering state of every token comes from a checkpoint written every kCB
 // tokens by a recompute of the forward (`kda_bwd_ckpt_kernel`): per stretch of kCB
 // tokens the reverse sweep (`kda_bwd_kernel`) runs the forward once from the
-// checkpoint, keeping each token's entering state in a per-CTA scratch (each
-// thread stores and later reloads only its own tile), then walks the tokens back.
-//
-// 128 threads per CTA. Thread (kg, vg) = (tid / 4, tid % 4) keeps rows
-// kg*RP .. kg*RP+RP-1 and slice columns 4 vg .. 4 vg+3 of S and of dS as float4
-// in registers. Key-axis sums go through shuffles among the 8 row groups of a
-// warp, then shared memory across the 4 warps (one block barrier per token, the
-// buffers alternating between tokens); value-axis sums within the slice go
-// through shuffles among the 4 lanes of a row group.
+// checkpoint, keeping each token's decayed state S' = diag(a) S in a per-CTA
+// scratch (each thread stores and later reloads only its own tile; it stays in
+// L2) and u = S'^T k^ in shared memory, then walks the tokens back. Checkpoints
+// and scratch are thread-major per CTA (coalesced).
 #include <cooperative_groups.h>
 
 #include "kda_common.cuh"
@@ -55,8 +55,8 @@ constexpr int kDVC = 16;  // value columns per CTA
 
 template <int DK, int DV>
 struct BwdTile {
-    static constexpr int VG = kDVC / 4, KG = kBwdThreads / VG, RP = DK / KG, NS = DV / kDVC;
-    static_assert(VG == 4 && KG == 32 && RP * KG == DK && RP >= 1 && NS >= 1 && NS <= 8, "state tiling");
+    static constexpr int RP = DK / 32, NS = DV / kDVC;
+    static_assert(kWarps * 4 == kDVC && RP * 32 == DK && RP >= 1 && RP <= 4 && NS >= 1 && NS <= 8, "state tiling");
 };
 
 // Raw inputs of one stretch, copied in by cp.async while the previous stretch runs.
@@ -66,27 +66,31 @@ struct Stage {
     Tin v[kCB][kDVC], dout[kCB][kDVC];       // this CTA's value columns; dout: reverse sweep only
 };
 
-// Token vectors of one stretch (fp32; k^ normalised) and the key-axis reduction
-// buffers: what the forward recompute needs.
+// Token vectors of one stretch (fp32; k^ normalised): what the forward recompute
+// needs. al holds the decay a = exp(max(g, lb)), negated where g < lb (the clamp
+// is taken there and the gate gets no gradient).
 template <typename Tin, int DK>
 struct FwdSmem {
     Stage<Tin, DK> st;
     float kh[kCB][DK], al[kCB][DK];
     float v[kCB][kDVC];
     float b[kCB], rk[kCB];
-    float4 red[2][kWarps][2][4];  // [token parity][warp][u or ddelta][column group]
 };
 
-// The reverse sweep adds q^, the raw gate (for the clamp mask), the output
-// cotangent, and the per-slice terms of dq^, dk^, dg and db, double-buffered
-// across stretches so that one cluster barrier per stretch suffices.
+// The reverse sweep adds q^, the output cotangent, u = S'^T k^ of every token of
+// the stretch (from its forward recompute), the per-warp terms of the current
+// token (alternating between tokens) and the per-CTA terms of dq^, dk^, dg
+// ([0], [1], [2]) and db of the stretch.
 template <typename Tin, int DK>
 struct BwdSmem : FwdSmem<Tin, DK> {
-    float qh[kCB][DK], graw[kCB][DK];
+    float qh[kCB][DK];
     float dout[kCB][kDVC];
+    float u[kCB][kDVC];
     float rq[kCB];
-    float pdq[2][kCB][DK], pdk[2][kCB][DK], pdg[2][kCB][DK];
-    float pdb[2][kCB];
+    float wp[2][kWarps][3][DK];
+    float wdb[2][kWarps];
+    float pd[3][kCB][DK];
+    float pdb[kCB];
 };
 
 __device__ __forceinline__ long long seq_begin(const BwdParams &p, int n) {
@@ -112,25 +116,66 @@ __device__ __forceinline__ void load_rows(const float *src, float (&out)[RP]) {
     }
 }
 
-__device__ __forceinline__ float4 f4_add(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+template <int RP>
+__device__ __forceinline__ void store_rows(float *dst, const float (&x)[RP]) {
+    if constexpr (RP == 4) {
+        *reinterpret_cast<float4 *>(dst) = make_float4(x[0], x[1], x[2], x[3]);
+    } else if constexpr (RP == 2) {
+        *reinterpret_cast<float2 *>(dst) = make_float2(x[0], x[1]);
+    } else {
+        dst[0] = x[0];
+    }
+}
+
 __device__ __forceinline__ float dot4(float4 a, float4 b) { return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w; }
 
-// Sum over the 8 row groups of a warp (lane bits 2..4).
-__device__ __forceinline__ float4 rowgroup_sum(float4 x) {
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-        x.x += __shfl_xor_sync(0xffffffffu, x.x, o);
-        x.y += __shfl_xor_sync(0xffffffffu, x.y, o);
-        x.z += __shfl_xor_sync(0xffffffffu, x.z, o);
-        x.w += __shfl_xor_sync(0xffffffffu, x.w, o);
-    }
-    return x;
+// Warp all-reduce of 4 values: reduce-scatter over lane bits 4 and 3 (each lane
+// keeps half of its values at each step), butterfly over bits 2..0, then each
+// sum is gathered from the lanes that hold it (value v sits in lanes with
+// bits 4..3 = v). 10 shuffles instead of 20.
+__device__ __forceinline__ float4 warp_allreduce4(float4 x) {
+    const int lane = threadIdx.x & 31;
+    const bool h4 = lane & 16, h3 = lane & 8;
+    // bit 4: keep (z, w) or (x, y)
+    float a0 = h4 ? x.z : x.x, a1 = h4 ? x.w : x.y;
+    const float s0 = h4 ? x.x : x.z, s1 = h4 ? x.y : x.w;
+    a0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+    a1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+    // bit 3: keep one of the two
+    float m = h3 ? a1 : a0;
+    m += __shfl_xor_sync(0xffffffffu, h3 ? a0 : a1, 8);
+    m += __shfl_xor_sync(0xffffffffu, m, 4);
+    m += __shfl_xor_sync(0xffffffffu, m, 2);
+    m += __shfl_xor_sync(0xffffffffu, m, 1);
+    return make_float4(__shfl_sync(0xffffffffu, m, 0), __shfl_sync(0xffffffffu, m, 8),
+                       __shfl_sync(0xffffffffu, m, 16), __shfl_sync(0xffffffffu, m, 24));
 }
-// Sum over the 4 column groups of a row group (lane bits 0..1).
-__device__ __forceinline__ float colgroup_sum(float x) {
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    x += __shfl_xor_sync(0xffffffffu, x, 2);
-    return x;
+
+// Warp all-reduce of 8 values (x then y): reduce-scatter over lane bits 4, 3, 2,
+// butterfly over bits 1, 0, gather (value v sits in lanes with bits 4..2 = v).
+// 17 shuffles instead of 40.
+__device__ __forceinline__ void warp_allreduce8(float4 &x, float4 &y) {
+    const int lane = threadIdx.x & 31;
+    const bool h4 = lane & 16, h3 = lane & 8, h2 = lane & 4;
+    // bit 4: keep y (values 4..7) or x (values 0..3)
+    float a0 = h4 ? y.x : x.x, a1 = h4 ? y.y : x.y, a2 = h4 ? y.z : x.z, a3 = h4 ? y.w : x.w;
+    a0 += __shfl_xor_sync(0xffffffffu, h4 ? x.x : y.x, 16);
+    a1 += __shfl_xor_sync(0xffffffffu, h4 ? x.y : y.y, 16);
+    a2 += __shfl_xor_sync(0xffffffffu, h4 ? x.z : y.z, 16);
+    a3 += __shfl_xor_sync(0xffffffffu, h4 ? x.w : y.w, 16);
+    // bit 3: keep (a2, a3) or (a0, a1)
+    float b0 = h3 ? a2 : a0, b1 = h3 ? a3 : a1;
+    b0 += __shfl_xor_sync(0xffffffffu, h3 ? a0 : a2, 8);
+    b1 += __shfl_xor_sync(0xffffffffu, h3 ? a1 : a3, 8);
+    // bit 2: keep b1 or b0
+    float m = h2 ? b1 : b0;
+    m += __shfl_xor_sync(0xffffffffu, h2 ? b0 : b1, 4);
+    m += __shfl_xor_sync(0xffffffffu, m, 2);
+    m += __shfl_xor_sync(0xffffffffu, m, 1);
+    x = make_float4(__shfl_sync(0xffffffffu, m, 0), __shfl_sync(0xffffffffu, m, 4),
+                    __shfl_sync(0xffffffffu, m, 8), __shfl_sync(0xffffffffu, m, 12));
+    y = make_float4(__shfl_sync(0xffffffffu, m, 16), __shfl_sync(0xffffffffu, m, 20),
+                    __shfl_sync(0xffffffffu, m, 24), __shfl_sync(0xffffffffu, m, 28));
 }
 
 __device__ __forceinline__ void cp_async16(void *sdst, const void *gsrc) {
@@ -143,10 +188,11 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // Start the copy of tokens [t0, t0 + cnt) of head h into the stage: k, g (and q
 // for the reverse sweep) rows, and this CTA's columns of v (and of the output
 // cotangent), in 16-byte pieces. Returns this thread's raw beta (thread i < cnt
-// holds token i's); the load completes in the background like the copies.
+// holds token i's), left unconverted so that its load completes in the
+// background like the copies.
 template <typename Tin, int DK, int DV, bool kRev>
-__device__ __forceinline__ float issue_stretch(const BwdParams &p, Stage<Tin, DK> &st, long long t0, int cnt, int h,
-                                               int col0) {
+__device__ __forceinline__ Tin issue_stretch(const BwdParams &p, Stage<Tin, DK> &st, long long t0, int cnt, int h,
+                                             int col0) {
     constexpr int EP = 16 / (int)sizeof(Tin);  // elements per piece
     constexpr int RK = DK / EP, RV = kDVC / EP;
     const int tid = threadIdx.x, H = p.H;
@@ -164,65 +210,134 @@ __device__ __forceinline__ float issue_stretch(const BwdParams &p, Stage<Tin, DK
         if constexpr (kRev) cp_async16(&st.dout[i][c], static_cast<const Tin *>(p.dout) + gi);
     }
     cp_async_commit();
-    return tid < cnt ? to_f32(static_cast<const Tin *>(p.beta)[(t0 + tid) * H + h]) : 0.f;
+    return tid < cnt ? static_cast<const Tin *>(p.beta)[(t0 + tid) * H + h] : Tin(0.f);
+}
+
+// E consecutive staged elements to fp32, with vector shared loads (bf16 widens exactly).
+template <int E>
+__device__ __forceinline__ void stage_cvt(const float *src, float (&out)[E]) {
+#pragma unroll
+    for (int j = 0; j < E; j += 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(src + j);
+        out[j] = x.x; out[j + 1] = x.y; out[j + 2] = x.z; out[j + 3] = x.w;
+    }
+}
+template <int E>
+__device__ __forceinline__ void stage_cvt(const __nv_bfloat16 *src, float (&out)[E]) {
+    static_assert(E % 2 == 0, "pairs");
+    if constexpr (E % 8 == 0) {
+#pragma unroll
+        for (int j = 0; j < E; j += 8) {
+            const uint4 x = *reinterpret_cast<const uint4 *>(src + j);
+            const unsigned w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                out[j + 2 * e] = __uint_as_float(w[e] << 16);
+                out[j + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < E; j += 2) {
+            const unsigned w = *reinterpret_cast<const unsigned *>(src + j);
+            out[j] = __uint_as_float(w << 16);
+            out[j + 1] = __uint_as_float(w & 0xffff0000u);
+        }
+    }
+}
+template <int E>
+__device__ __forceinline__ void store_vec(float *dst, const float (&x)[E]) {
+    if constexpr (E % 4 == 0) {
+#pragma unroll
+        for (int j = 0; j < E; j += 4) *reinterpret_cast<float4 *>(dst + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+    } else {
+#pragma unroll
+        for (int j = 0; j < E; j += 2) *reinterpret_cast<float2 *>(dst + j) = make_float2(x[j], x[j + 1]);
+    }
 }
 
 // Turn the staged stretch into the fp32 token vectors: k^ (and q^; normalised
-// when use_l2), the decay a = exp(max(g, lb)), v (and the output cotangent), the
-// write strength b. The first barrier publishes the copies and also separates
-// these writes from the previous stretch's last readers; on return the vectors
-// are complete and the stage is free for the next copy.
+// when use_l2), the signed decay al, v (and the output cotangent), the write
+// strength b. Each key row is taken by 16 threads (DK / 16 elements each) that
+// form its squared norm with shuffles. The first barrier publishes the copies
+// and separates these writes from the previous stretch's last readers; on return
+// the vectors are complete and the stage is free for the next copy.
 template <typename Tin, int DK, bool kRev, typename Sm>
-__device__ void take_stretch(const BwdParams &p, Sm &sm, int cnt, float beta_raw) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+__device__ void take_stretch(const BwdParams &p, Sm &sm, int cnt, Tin beta_raw) {
+    constexpr int TPR = 16, E = DK / TPR;
+    const int tid = threadIdx.x;
     cp_async_wait_all();
     __syncthreads();
-    for (int e = tid; e < cnt * DK; e += kBwdThreads) {
-        const int i = e / DK, c = e % DK;
-        sm.kh[i][c] = to_f32(sm.st.k[i][c]);
-        const float gr = to_f32(sm.st.g[i][c]);
-        sm.al[i][c] = expf(p.has_lb ? fmaxf(gr, p.lb) : gr);
+    const int c = (tid % TPR) * E;
+    // uniform trip count: every lane joins the shuffles; rows past cnt read row 0
+    // and store nothing
+    for (int i0 = 0; i0 < cnt; i0 += kBwdThreads / TPR) {
+        const int i = i0 + tid / TPR;
+        const bool live = i < cnt;
+        const int ir = live ? i : 0;
+        float kx[E], gx[E];
+        stage_cvt<E>(&sm.st.k[ir][c], kx);
+        stage_cvt<E>(&sm.st.g[ir][c], gx);
+        float kk = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) kk = fmaf(kx[e], kx[e], kk);
+#pragma unroll
+        for (int o = TPR / 2; o > 0; o >>= 1) kk += __shfl_xor_sync(0xffffffffu, kk, o);
+        const float rk = p.use_l2 ? rsqrtf(kk + kL2Eps) : 1.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            kx[e] *= rk;
+            const bool pass = !p.has_lb || gx[e] >= p.lb;
+            const float a = expf(pass ? gx[e] : p.lb);
+            gx[e] = pass ? a : -a;
+        }
+        if (live) {
+            store_vec<E>(&sm.kh[i][c], kx);
+            store_vec<E>(&sm.al[i][c], gx);
+            if (tid % TPR == 0) sm.rk[i] = rk;
+        }
         if constexpr (kRev) {
-            sm.qh[i][c] = to_f32(sm.st.q[i][c]);
-            sm.graw[i][c] = gr;
+            float qx[E];
+            stage_cvt<E>(&sm.st.q[ir][c], qx);
+            float qq = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) qq = fmaf(qx[e], qx[e], qq);
+#pragma unroll
+            for (int o = TPR / 2; o > 0; o >>= 1) qq += __shfl_xor_sync(0xffffffffu, qq, o);
+            const float rq = p.use_l2 ? rsqrtf(qq + kL2Eps) : 1.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) qx[e] *= rq;
+            if (live) {
+                store_vec<E>(&sm.qh[i][c], qx);
+                if (tid % TPR == 0) sm.rq[i] = rq;
+            }
         }
     }
     for (int e = tid; e < cnt * kDVC; e += kBwdThreads) {
-        const int i = e / kDVC, c = e % kDVC;
-        sm.v[i][c] = to_f32(sm.st.v[i][c]);
-        if constexpr (kRev) sm.dout[i][c] = to_f32(sm.st.dout[i][c]);
+        const int i = e / kDVC, cc = e % kDVC;
+        sm.v[i][cc] = to_f32(sm.st.v[i][cc]);
+        if constexpr (kRev) sm.dout[i][cc] = to_f32(sm.st.dout[i][cc]);
     }
-    if (tid < cnt) sm.b[tid] = beta_value(beta_raw, p.beta_prob);
-    __syncthreads();
-    for (int i = warp; i < cnt; i += kWarps) {
-        float kk = 0.f, qq = 0.f;
-        for (int c = lane; c < DK; c += 32) {
-            kk = fmaf(sm.kh[i][c], sm.kh[i][c], kk);
-            if constexpr (kRev) qq = fmaf(sm.qh[i][c], sm.qh[i][c], qq);
-        }
-        kk = warp_sum(kk);
-        const float rk = p.use_l2 ? rsqrtf(kk + kL2Eps) : 1.f;
-        for (int c = lane; c < DK; c += 32) sm.kh[i][c] *= rk;
-        if (lane == 0) sm.rk[i] = rk;
-        if constexpr (kRev) {
-            qq = warp_sum(qq);
-            const float rq = p.use_l2 ? rsqrtf(qq + kL2Eps) : 1.f;
-            for (int c = lane; c < DK; c += 32) sm.qh[i][c] *= rq;
-            if (lane == 0) sm.rq[i] = rq;
-        }
-    }
+    if (tid < cnt) sm.b[tid] = beta_value(to_f32(beta_raw), p.beta_prob);
     __syncthreads();
 }
 
-// One forward step of token i of the loaded stretch on the register tile s; ph
-// selects the reduction buffer (alternating between consecutive steps).
+// One forward step of token i of the loaded stretch on this warp's register tile
+// s (rows lane*RP.., columns 4 warp .. 4 warp + 3 of the slice). Warp-local. With
+// keep_s, the decayed state S' = diag(a) S goes to keep_s[r * 128] (this thread's
+// slots) and u = S'^T k^ of the warp's columns to keep_u.
 template <typename Tin, int DK, int DV>
-__device__ __forceinline__ void fwd_step(FwdSmem<Tin, DK> &sm, int i, int ph, float4 (&s)[BwdTile<DK, DV>::RP]) {
+__device__ __forceinline__ void fwd_step(const FwdSmem<Tin, DK> &sm, int i, float4 (&s)[BwdTile<DK, DV>::RP],
+                                         float4 *keep_s = nullptr, float *keep_u = nullptr) {
     constexpr int RP = BwdTile<DK, DV>::RP;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, vg = tid & 3, kg = tid >> 2;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float kr[RP], ar[RP];
-    load_rows<RP>(&sm.kh[i][kg * RP], kr);
-    load_rows<RP>(&sm.al[i][kg * RP], ar);
+    load_rows<RP>(&sm.kh[i][lane * RP], kr);
+    load_rows<RP>(&sm.al[i][lane * RP], ar);
+#pragma unroll
+    for (int r = 0; r < RP; ++r) ar[r] = fabsf(ar[r]);
+    const float b = sm.b[i];
+    const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][4 * warp]);
     float4 pu = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < RP; ++r) {
@@ -230,14 +345,12 @@ __device__ __forceinline__ void fwd_step(FwdSmem<Tin, DK> &sm, int i, int ph, fl
         pu.x = fmaf(s[r].x, kr[r], pu.x); pu.y = fmaf(s[r].y, kr[r], pu.y);
         pu.z = fmaf(s[r].z, kr[r], pu.z); pu.w = fmaf(s[r].w, kr[r], pu.w);
     }
-    pu = rowgroup_sum(pu);
-    if (lane < 4) sm.red[ph][warp][0][vg] = pu;
-    __syncthreads();
-    float4 u = sm.red[ph][0][0][vg];
+    if (keep_s) {
 #pragma unroll
-    for (int w = 1; w < kWarps; ++w) u = f4_add(u, sm.red[ph][w][0][vg]);
-    const float b = sm.b[i];
-    const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][4 * vg]);
+        for (int r = 0; r < RP; ++r) keep_s[r * kBwdThreads] = s[r];
+    }
+    const float4 u = warp_allreduce4(pu);
+    if (keep_u && lane == 0) *reinterpret_cast<float4 *>(keep_u) = u;
     const float4 d = make_float4(b * (vv.x - u.x), b * (vv.y - u.y), b * (vv.z - u.z), b * (vv.w - u.w));
 #pragma unroll
     for (int r = 0; r < RP; ++r) {
@@ -246,13 +359,14 @@ __device__ __forceinline__ void fwd_step(FwdSmem<Tin, DK> &sm, int i, int ph, fl
     }
 }
 
-// Row `row`, slice column 4 vg of a [DK, DV] state tile whose slice starts at col0.
+// Element (row, slice column 4 warp) of a user [DK, DV] state whose slice starts at col0.
 template <int DV>
-__device__ __forceinline__ float4 *state_ptr(float *base, int row, int col0, int vg) {
-    return reinterpret_cast<float4 *>(base + (long long)row * DV + col0 + 4 * vg);
+__device__ __forceinline__ float4 *state_ptr(float *base, int row, int col0, int warp) {
+    return reinterpret_cast<float4 *>(base + (long long)row * DV + col0 + 4 * warp);
 }
 
 // Recompute of the forward, storing the entering state of tokens 0, kCB, 2 kCB, ...
+// (thread-major: checkpoint j of CTA slice r at ((j H + h) NS + r) RP 128 float4).
 // One CTA per (sequence, head, 16-column slice); no cross-CTA traffic.
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kBwdThreads) kda_bwd_ckpt_kernel(BwdParams p) {
@@ -260,32 +374,42 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_ckpt_kernel(BwdParams p) 
     constexpr int RP = Tl::RP, NS = Tl::NS;
     extern __shared__ __align__(16) uint8_t smraw[];
     FwdSmem<Tin, DK> &sm = *reinterpret_cast<FwdSmem<Tin, DK> *>(smraw);
-    const int tid = threadIdx.x, vg = tid & 3, kg = tid >> 2;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long nh = blockIdx.x / NS;
-    const int col0 = (int)(blockIdx.x % NS) * kDVC;
+    const int rank = (int)(blockIdx.x % NS), col0 = rank * kDVC;
     const int n = (int)(nh / p.H), h = (int)(nh % p.H);
     const long long bos = seq_begin(p, n), eos = seq_end(p, n);
     float4 s[RP];
 #pragma unroll
     for (int r = 0; r < RP; ++r)
-        s[r] = p.S0 ? *state_ptr<DV>(const_cast<float *>(p.S0) + nh * DK * DV, kg * RP + r, col0, vg)
+        s[r] = p.S0 ? *state_ptr<DV>(const_cast<float *>(p.S0) + nh * DK * DV, lane * RP + r, col0, warp)
                     : make_float4(0.f, 0.f, 0.f, 0.f);
     const long long c0 = first_ckpt(p, n);
-    int ph = 0;
-    float braw = bos < eos ? issue_stretch<Tin, DK, DV, false>(p, sm.st, bos, (int)min((long long)kCB, eos - bos), h, col0) : 0.f;
+    float4 *ckb = reinterpret_cast<float4 *>(p.ckpt);
+    Tin braw = bos < eos ? issue_stretch<Tin, DK, DV, false>(p, sm.st, bos, (int)min((long long)kCB, eos - bos), h, col0)
+                         : Tin(0.f);
     for (long long t0 = bos; t0 < eos; t0 += kCB) {
         const int cnt = (int)min((long long)kCB, eos - t0);
-        float *ck = p.ckpt + ((c0 + (t0 - bos) / kCB) * p.H + h) * DK * DV;
+        float4 *ck = ckb + (((c0 + (t0 - bos) / kCB) * p.H + h) * NS + rank) * (RP * kBwdThreads);
 #pragma unroll
-        for (int r = 0; r < RP; ++r) *state_ptr<DV>(ck, kg * RP + r, col0, vg) = s[r];
+        for (int r = 0; r < RP; ++r) ck[r * kBwdThreads + tid] = s[r];
         take_stretch<Tin, DK, false>(p, sm, cnt, braw);
         if (t0 + kCB < eos) braw = issue_stretch<Tin, DK, DV, false>(p, sm.st, t0 + kCB, (int)min((long long)kCB, eos - t0 - kCB), h, col0);
-        for (int i = 0; i < cnt; ++i, ph ^= 1) fwd_step<Tin, DK, DV>(sm, i, ph, s);
+        for (int i = 0; i < cnt; ++i) fwd_step<Tin, DK, DV>(sm, i, s);
     }
 }
 
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
 // Reverse sweep: one cluster of NS CTAs per (sequence, head), CTA rank r owning
-// value columns 16 r .. 16 r + 15.
+// value columns 16 r .. 16 r + 15, warp w of it columns 16 r + 4 w .. 16 r + 4 w + 3.
+// Per stretch: take the staged tokens, start the copy of the stretch before,
+// rerun the stretch forward from its checkpoint keeping every token's decayed
+// state S' (in this CTA's scratch, thread-major) and u = S'^T k^, walk it back,
+// then the cluster adds the slice terms. The cluster barrier that frees the
+// slice-term buffers for the next stretch is split: arrive after the adding,
+// wait just before the next walk writes them.
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
     using Tl = BwdTile<DK, DV>;
@@ -294,125 +418,122 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
     BwdSmem<Tin, DK> &sm = *reinterpret_cast<BwdSmem<Tin, DK> *>(smraw);
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, vg = tid & 3, kg = tid >> 2;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long nh = blockIdx.x / NS;
     const int col0 = rank * kDVC;
     const int n = (int)(nh / p.H), h = (int)(nh % p.H);
     const int H = p.H;
     const long long bos = seq_begin(p, n), eos = seq_end(p, n);
     const long long c0 = first_ckpt(p, n);
-    // this CTA's per-token entering states, thread-major: slot i, row part r at ((i RP + r) 128 + tid)
-    float4 *scr = reinterpret_cast<float4 *>(p.scratch) + (long long)blockIdx.x * kCB * RP * kBwdThreads;
+    const float4 *ckb = reinterpret_cast<const float4 *>(p.ckpt);
+    // slot i, row part r of thread t at scr[(i RP + r) 128 + t]
+    float4 *scr = reinterpret_cast<float4 *>(p.scratch) + (long long)blockIdx.x * kCB * RP * kBwdThreads + tid;
 
     float4 ds[RP], s[RP];
 #pragma unroll
     for (int r = 0; r < RP; ++r)
-        ds[r] = p.dSf ? *state_ptr<DV>(const_cast<float *>(p.dSf) + nh * DK * DV, kg * RP + r, col0, vg)
+        ds[r] = p.dSf ? *state_ptr<DV>(const_cast<float *>(p.dSf) + nh * DK * DV, lane * RP + r, col0, warp)
                       : make_float4(0.f, 0.f, 0.f, 0.f);
     int ph = 0;
     const long long len = eos - bos;
     const long long nst = (len + kCB - 1) / kCB;
-    float braw = nst > 0 ? issue_stretch<Tin, DK, DV, true>(p, sm.st, bos + (nst - 1) * kCB,
-                                                            (int)(len - (nst - 1) * kCB), h, col0) : 0.f;
+    Tin braw = nst > 0 ? issue_stretch<Tin, DK, DV, true>(p, sm.st, bos + (nst - 1) * kCB, (int)(len - (nst - 1) * kCB),
+                                                          h, col0)
+                       : Tin(0.f);
     for (long long cs = nst - 1; cs >= 0; --cs) {
         const long long t0 = bos + cs * kCB;
         const int cnt = (int)min((long long)kCB, eos - t0);
-        const int pb = (int)(cs & 1);
-        const float *ck = p.ckpt + ((c0 + cs) * H + h) * DK * DV;
+        const float4 *ck = ckb + (((c0 + cs) * H + h) * NS + rank) * (RP * kBwdThreads);
         take_stretch<Tin, DK, true>(p, sm, cnt, braw);
         if (cs > 0) braw = issue_stretch<Tin, DK, DV, true>(p, sm.st, t0 - kCB, kCB, h, col0);
-        // forward from the checkpoint, keeping every token's entering state; the
-        // last one stays in s
+        // forward from the checkpoint, keeping S' and u of every token
 #pragma unroll
-        for (int r = 0; r < RP; ++r) s[r] = *state_ptr<DV>(const_cast<float *>(ck), kg * RP + r, col0, vg);
-        for (int i = 0; i + 1 < cnt; ++i, ph ^= 1) {
+        for (int r = 0; r < RP; ++r) s[r] = ck[r * kBwdThreads + tid];
+        for (int i = 0; i < cnt; ++i) fwd_step<Tin, DK, DV>(sm, i, s, scr + i * RP * kBwdThreads, &sm.u[i][4 * warp]);
+        __syncwarp();  // u of the warp's columns, written by lane 0, is read by all lanes
+        if (cs != nst - 1) cluster_wait();  // every rank has added the previous stretch's terms
+        float4 sp[RP];  // S' of the current token, fetched one token ahead
 #pragma unroll
-            for (int r = 0; r < RP; ++r) scr[(i * RP + r) * kBwdThreads + tid] = s[r];
-            fwd_step<Tin, DK, DV>(sm, i, ph, s);
-        }
+        for (int r = 0; r < RP; ++r) sp[r] = scr[((cnt - 1) * RP + r) * kBwdThreads];
         for (int i = cnt - 1; i >= 0; --i, ph ^= 1) {
-            // the previous token's entering state, fetched while this token runs
-            float4 sn[RP];
+#pragma unroll
+            for (int r = 0; r < RP; ++r) s[r] = sp[r];
             if (i > 0) {
 #pragma unroll
-                for (int r = 0; r < RP; ++r) sn[r] = scr[((i - 1) * RP + r) * kBwdThreads + tid];
+                for (int r = 0; r < RP; ++r) sp[r] = scr[((i - 1) * RP + r) * kBwdThreads];
             }
             float kr[RP], ar[RP], qr[RP];
-            load_rows<RP>(&sm.kh[i][kg * RP], kr);
-            load_rows<RP>(&sm.al[i][kg * RP], ar);
-            load_rows<RP>(&sm.qh[i][kg * RP], qr);
+            load_rows<RP>(&sm.kh[i][lane * RP], kr);
+            load_rows<RP>(&sm.al[i][lane * RP], ar);
+            load_rows<RP>(&sm.qh[i][lane * RP], qr);
             const float b = sm.b[i];
-            const float4 dov = *reinterpret_cast<const float4 *>(&sm.dout[i][4 * vg]);
+            const float4 dov = *reinterpret_cast<const float4 *>(&sm.dout[i][4 * warp]);
+            const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][4 * warp]);
+            const float4 u = *reinterpret_cast<const float4 *>(&sm.u[i][4 * warp]);
 
-            // ---- S', u = S'^T k^, dS += scale q^ do^T, ddelta = dS^T k^
-            float4 pu = make_float4(0.f, 0.f, 0.f, 0.f), pd = pu;
+            // ---- dS += scale q^ do^T, then ddelta = dS^T k^ (warp sum)
+            float4 dd = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
                 const float qs = p.scale * qr[r];
-                s[r].x *= ar[r]; s[r].y *= ar[r]; s[r].z *= ar[r]; s[r].w *= ar[r];
-                pu.x = fmaf(s[r].x, kr[r], pu.x); pu.y = fmaf(s[r].y, kr[r], pu.y);
-                pu.z = fmaf(s[r].z, kr[r], pu.z); pu.w = fmaf(s[r].w, kr[r], pu.w);
                 ds[r].x = fmaf(qs, dov.x, ds[r].x); ds[r].y = fmaf(qs, dov.y, ds[r].y);
                 ds[r].z = fmaf(qs, dov.z, ds[r].z); ds[r].w = fmaf(qs, dov.w, ds[r].w);
-                pd.x = fmaf(ds[r].x, kr[r], pd.x); pd.y = fmaf(ds[r].y, kr[r], pd.y);
-                pd.z = fmaf(ds[r].z, kr[r], pd.z); pd.w = fmaf(ds[r].w, kr[r], pd.w);
+                dd.x = fmaf(ds[r].x, kr[r], dd.x); dd.y = fmaf(ds[r].y, kr[r], dd.y);
+                dd.z = fmaf(ds[r].z, kr[r], dd.z); dd.w = fmaf(ds[r].w, kr[r], dd.w);
             }
-            pu = rowgroup_sum(pu);
-            pd = rowgroup_sum(pd);
-            if (lane < 4) { sm.red[ph][warp][0][vg] = pu; sm.red[ph][warp][1][vg] = pd; }
-            __syncthreads();
-            float4 u = sm.red[ph][0][0][vg], dd = sm.red[ph][0][1][vg];
-#pragma unroll
-            for (int w = 1; w < kWarps; ++w) { u = f4_add(u, sm.red[ph][w][0][vg]); dd = f4_add(dd, sm.red[ph][w][1][vg]); }
-            const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][4 * vg]);
+            dd = warp_allreduce4(dd);
             const float4 vu = make_float4(vv.x - u.x, vv.y - u.y, vv.z - u.z, vv.w - u.w);
             const float4 dl = make_float4(b * vu.x, b * vu.y, b * vu.z, b * vu.w);
-            if (tid < 4) {  // dv = b ddelta for this slice
-                Tin *dv = static_cast<Tin *>(p.dv) + ((t0 + i) * H + h) * DV + col0 + 4 * tid;
-                dv[0] = from_f32<Tin>(b * dd.x); dv[1] = from_f32<Tin>(b * dd.y);
-                dv[2] = from_f32<Tin>(b * dd.z); dv[3] = from_f32<Tin>(b * dd.w);
+            if (lane < 4) {  // dv = b ddelta for this warp's columns, one per lane
+                const float x = lane == 0 ? dd.x : lane == 1 ? dd.y : lane == 2 ? dd.z : dd.w;
+                static_cast<Tin *>(p.dv)[((t0 + i) * H + h) * DV + col0 + 4 * warp + lane] = from_f32<Tin>(b * x);
             }
-            // slice terms of delta . do and ddelta . (v - u)
-            const float ddo = colgroup_sum(dot4(dl, dov));
-            const float db = colgroup_sum(dot4(dd, vu));
+            // this warp's terms of delta . do and ddelta . (v - u)
+            const float ddo = dot4(dl, dov), db = dot4(dd, vu);
 
-            // ---- slice terms of the row sums: S' do, dS delta, S' ddelta, dS (.) S'
-            float ra[RP], rb[RP], re[RP], rh[RP];
+            // ---- this warp's terms of the row sums S' do, dS delta, S' ddelta, dS (.) S'
+            float tq[RP], tk[RP], tg[RP];
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
-                ra[r] = colgroup_sum(dot4(s[r], dov));
-                rb[r] = colgroup_sum(dot4(ds[r], dl));
-                re[r] = colgroup_sum(dot4(s[r], dd));
-                rh[r] = colgroup_sum(dot4(ds[r], s[r]));
+                const float ra = dot4(s[r], dov), rb = dot4(ds[r], dl), re = dot4(s[r], dd), rh = dot4(ds[r], s[r]);
+                tq[r] = p.scale * fmaf(kr[r], ddo, ra);
+                tk[r] = fmaf(-b, re, rb);
+                tg[r] = ar[r] > 0.f ? fmaf(-b * kr[r], re, rh) : 0.f;
             }
-            if (vg == 0) {
-                float g4[RP];
-                load_rows<RP>(&sm.graw[i][kg * RP], g4);
-#pragma unroll
-                for (int r = 0; r < RP; ++r) {
-                    const int c = kg * RP + r;
-                    sm.pdq[pb][i][c] = p.scale * fmaf(kr[r], ddo, ra[r]);
-                    sm.pdk[pb][i][c] = fmaf(-b, re[r], rb[r]);
-                    const bool pass = !p.has_lb || g4[r] >= p.lb;
-                    sm.pdg[pb][i][c] = pass ? fmaf(-b * kr[r], re[r], rh[r]) : 0.f;
-                }
-            }
-            if (tid == 0) sm.pdb[pb][i] = db;
+            store_rows<RP>(&sm.wp[ph][warp][0][lane * RP], tq);
+            store_rows<RP>(&sm.wp[ph][warp][1][lane * RP], tk);
+            store_rows<RP>(&sm.wp[ph][warp][2][lane * RP], tg);
+            if (lane == 0) sm.wdb[ph][warp] = db;
             // ---- dS <- diag(a) (dS - b k^ ddelta^T), the cotangent of the entering state
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
-                const float bk = b * kr[r];
-                ds[r].x = ar[r] * fmaf(-bk, dd.x, ds[r].x); ds[r].y = ar[r] * fmaf(-bk, dd.y, ds[r].y);
-                ds[r].z = ar[r] * fmaf(-bk, dd.z, ds[r].z); ds[r].w = ar[r] * fmaf(-bk, dd.w, ds[r].w);
+                const float bk = b * kr[r], a = fabsf(ar[r]);
+                ds[r].x = a * fmaf(-bk, dd.x, ds[r].x); ds[r].y = a * fmaf(-bk, dd.y, ds[r].y);
+                ds[r].z = a * fmaf(-bk, dd.z, ds[r].z); ds[r].w = a * fmaf(-bk, dd.w, ds[r].w);
             }
-            if (i > 0) {
+            // ---- the CTA's terms of token i: the 4 warps' terms added in a fixed order
+            __syncthreads();
+            constexpr int Q4 = DK / 4;  // float4 per quantity row
+            if (tid < 3 * Q4) {
+                const int qn = tid / Q4, c = (tid % Q4) * 4;
+                float4 acc = *reinterpret_cast<const float4 *>(&sm.wp[ph][0][qn][c]);
 #pragma unroll
-                for (int r = 0; r < RP; ++r) s[r] = sn[r];
+                for (int w = 1; w < kWarps; ++w) {
+                    const float4 x = *reinterpret_cast<const float4 *>(&sm.wp[ph][w][qn][c]);
+                    acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+                }
+                *reinterpret_cast<float4 *>(&sm.pd[qn][i][c]) = acc;
+            } else if (tid == kBwdThreads - 1) {
+                float acc = sm.wdb[ph][0];
+#pragma unroll
+                for (int w = 1; w < kWarps; ++w) acc += sm.wdb[ph][w];
+                sm.pdb[i] = acc;
             }
         }
         // ---- the stretch's slice terms are complete in every CTA of the cluster:
         // rank r finishes tokens r, r + NS, ... (warp w takes every kWarps-th of them)
-        cluster.sync();
+        cluster_arrive();
+        cluster_wait();
         for (int i = rank + NS * warp; i < cnt; i += NS * kWarps) {
             constexpr int CP = DK / 32;
             float sq[CP], sk[CP], sg[CP];
@@ -424,9 +545,9 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
 #pragma unroll
                 for (int q = 0; q < NS; ++q) {
                     const BwdSmem<Tin, DK> *rs = cluster.map_shared_rank(&sm, q);
-                    sq[j] += rs->pdq[pb][i][c];
-                    sk[j] += rs->pdk[pb][i][c];
-                    sg[j] += rs->pdg[pb][i][c];
+                    sq[j] += rs->pd[0][i][c];
+                    sk[j] += rs->pd[1][i][c];
+                    sg[j] += rs->pd[2][i][c];
                 }
                 qd = fmaf(sm.qh[i][c], sq[j], qd);
                 kd = fmaf(sm.kh[i][c], sk[j], kd);
@@ -445,17 +566,18 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
             if (lane == 0) {
                 float db = 0.f;
 #pragma unroll
-                for (int q = 0; q < NS; ++q) db += cluster.map_shared_rank(&sm, q)->pdb[pb][i];
+                for (int q = 0; q < NS; ++q) db += cluster.map_shared_rank(&sm, q)->pdb[i];
                 const float b = sm.b[i];
                 static_cast<Tin *>(p.dbeta)[(t0 + i) * H + h] = from_f32<Tin>(p.beta_prob ? db : db * b * (1.f - b));
             }
         }
+        cluster_arrive();  // this rank has read every rank's terms of the stretch
     }
     // no CTA leaves while another rank may still read its shared memory
-    cluster.sync();
+    if (nst > 0) cluster_wait();
     if (p.dS0) {
 #pragma unroll
-        for (int r = 0; r < RP; ++r) *state_ptr<DV>(p.dS0 + nh * DK * DV, kg * RP + r, col0, vg) = ds[r];
+        for (int r = 0; r < RP; ++r) *state_ptr<DV>(p.dS0 + nh * DK * DV, lane * RP + r, col0, warp) = ds[r];
     }
 }
 
@@ -477,6 +599,7 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st) {
     const long long heads = (long long)p.N * p.H;
     if (heads == 0) return cudaSuccess;
     const int smem_f = (int)sizeof(FwdSmem<Tin, DK>), smem_b = (int)sizeof(BwdSmem<Tin, DK>);
+    static_assert(sizeof(BwdSmem<Tin, DK>) <= 232448, "shared memory of the reverse sweep");
     cudaError_t e;
     if ((e = cudaFuncSetAttribute(kda_bwd_ckpt_kernel<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_f)) != cudaSuccess)
         return e;

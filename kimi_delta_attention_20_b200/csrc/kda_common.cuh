@@ -110,7 +110,7 @@ struct BwdParams {
     float lb;
     int beta_prob;
     float *ckpt;                // state checkpoints
-    float *scratch;             // per (sequence, head): the entering states of one sub-chunk
+    float *scratch;             // per CTA of the reverse sweep: the decayed states of one stretch
     int *ckpt_off;              // varlen: [N+1] first checkpoint of each sequence (device-computed)
 };
 
