@@ -29,6 +29,7 @@ workload on the host cores (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -278,6 +279,8 @@ def run_kda(args, rank, world, local_rank):
                          g_out=tk["g_out"][i], lower_bound=-5.0, out=tk_o)
 
     bwl = KI.CHUNK_WORKLOADS[BWD_WL]
+    if args.only == "bwd" and args.bwd_tokens:  # shorter sequence for profiler captures
+        bwl = dataclasses.replace(bwl, T=args.bwd_tokens, name=f"{bwl.name} T{args.bwd_tokens}")
     if args.only in (None, "bwd"):
         binp = KI.chunk_inputs(bwl, device=dev)
         bgen = torch.Generator(device=dev)
@@ -566,6 +569,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=["chunk", "decode", "token", "bwd"], default=None,
                     help="run one leg only and print its timing (for profiler captures)")
+    ap.add_argument("--bwd-tokens", type=int, default=None,
+                    help="with --only bwd: sequence length of the backward workload (default 8192)")
     ap.add_argument("--workload", type=int, default=None,
                     help="with --only chunk: chunk workload index (default: the varlen H=96 one)")
     args = ap.parse_args()
