@@ -9,6 +9,7 @@
 namespace kda {
 cudaError_t launch_decode(const StepParams &p, bool bf16, int Dk, int Dv, cudaStream_t st);
 cudaError_t launch_chunk_simt(const ChunkParams &p, bool bf16, int Dk, int Dv, int chunk, cudaStream_t st);
+cudaError_t launch_chunk_rec(const ChunkParams &p, bool bf16, int Dk, int Dv, cudaStream_t st);
 bool chunk_tc_supported(bool bf16, int Dk, int Dv, int chunk_size);
 size_t chunk_tc_workspace_bytes(int N, int H, int Dk, int Dv);
 cudaError_t launch_chunk_tc(const ChunkParams &p, int Dk, int Dv, void *workspace,
@@ -198,7 +199,10 @@ kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
         return cuda_status(kda::launch_chunk_tc(p, a->Dk, a->Dv, a->workspace, a->workspace_bytes,
                                                 a->cu_seqlens_host, st));
     }
-    return cuda_status(kda::launch_chunk_simt(p, bf16, a->Dk, a->Dv, a->chunk_size == 32 ? 32 : 64, st));
+    // other shapes: the register-resident recurrence; an explicit 32-token chunk
+    // request runs the chunked CUDA-core kernel with C = 32 (same result)
+    if (a->chunk_size == 32) return cuda_status(kda::launch_chunk_simt(p, bf16, a->Dk, a->Dv, 32, st));
+    return cuda_status(kda::launch_chunk_rec(p, bf16, a->Dk, a->Dv, st));
 }
 
 kda_status kda_recurrent_step(const kda_step_args *a, void *stream) {

@@ -41,6 +41,7 @@
 #include <cooperative_groups.h>
 
 #include "kda_common.cuh"
+#include "kda_stage.cuh"
 
 namespace kda {
 
@@ -178,13 +179,6 @@ __device__ __forceinline__ void warp_allreduce8(float4 &x, float4 &y) {
                     __shfl_sync(0xffffffffu, m, 24), __shfl_sync(0xffffffffu, m, 28));
 }
 
-__device__ __forceinline__ void cp_async16(void *sdst, const void *gsrc) {
-    const unsigned d = (unsigned)__cvta_generic_to_shared(sdst);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
 // Start the copy of tokens [t0, t0 + cnt) of head h into the stage: k, g (and q
 // for the reverse sweep) rows, and this CTA's columns of v (and of the output
 // cotangent), in 16-byte pieces. Returns this thread's raw beta (thread i < cnt
@@ -211,49 +205,6 @@ __device__ __forceinline__ Tin issue_stretch(const BwdParams &p, Stage<Tin, DK> 
     }
     cp_async_commit();
     return tid < cnt ? static_cast<const Tin *>(p.beta)[(t0 + tid) * H + h] : Tin(0.f);
-}
-
-// E consecutive staged elements to fp32, with vector shared loads (bf16 widens exactly).
-template <int E>
-__device__ __forceinline__ void stage_cvt(const float *src, float (&out)[E]) {
-#pragma unroll
-    for (int j = 0; j < E; j += 4) {
-        const float4 x = *reinterpret_cast<const float4 *>(src + j);
-        out[j] = x.x; out[j + 1] = x.y; out[j + 2] = x.z; out[j + 3] = x.w;
-    }
-}
-template <int E>
-__device__ __forceinline__ void stage_cvt(const __nv_bfloat16 *src, float (&out)[E]) {
-    static_assert(E % 2 == 0, "pairs");
-    if constexpr (E % 8 == 0) {
-#pragma unroll
-        for (int j = 0; j < E; j += 8) {
-            const uint4 x = *reinterpret_cast<const uint4 *>(src + j);
-            const unsigned w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                out[j + 2 * e] = __uint_as_float(w[e] << 16);
-                out[j + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-            }
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < E; j += 2) {
-            const unsigned w = *reinterpret_cast<const unsigned *>(src + j);
-            out[j] = __uint_as_float(w << 16);
-            out[j + 1] = __uint_as_float(w & 0xffff0000u);
-        }
-    }
-}
-template <int E>
-__device__ __forceinline__ void store_vec(float *dst, const float (&x)[E]) {
-    if constexpr (E % 4 == 0) {
-#pragma unroll
-        for (int j = 0; j < E; j += 4) *reinterpret_cast<float4 *>(dst + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
-    } else {
-#pragma unroll
-        for (int j = 0; j < E; j += 2) *reinterpret_cast<float2 *>(dst + j) = make_float2(x[j], x[j + 1]);
-    }
 }
 
 // Turn the staged stretch into the fp32 token vectors: k^ (and q^; normalised

@@ -1,0 +1,253 @@
+// Chunk forward for the shapes the tensor-core path does not take (fp32 inputs,
+// d_k or d_v other than 128): the token recurrence of page
+// "atlas_core/kimi_k3/kda.rs" run directly, with the fp32 state in registers.
+//
+// Per token, with k^, q^ the normalised rows, a = exp(g) (g clamped, or formed
+// in the kernel from A_log and dt_bias) and b the write strength:
+//   S' = diag(a) S,  u = S'^T k^,  S = S' + k^ (b (v - u))^T,  o = scale S^T q^.
+// The result is that of `chunk_kda` (page "K3/kda/ops/api.py") for any chunk
+// size: regrouping the recurrence by chunks changes the order of the
+// arithmetic, not its value. For small head dims the recurrence also takes
+// fewer operations than the chunked form (no C x C blocks, no inverse).
+//
+// One CTA per (sequence, head), one warp per 16 value columns. Lane (rg, cg) =
+// (lane / 4, lane % 4) keeps rows rg*RP .. rg*RP+RP-1 (RP = d_k / 8) of columns
+// 4 cg .. 4 cg + 3 of its warp's block as float4 in registers. The key-axis sums
+// u and o are reductions over the 8 row groups of a warp (reduce-scatter, then
+// a gather for u: 8 shuffles); nothing else crosses lanes, and no barrier is
+// taken per token. Tokens arrive in stretches of CT: the raw rows of the next
+// stretch are copied by cp.async while the current one runs, turned into fp32
+// (L2 norms, gate, sigmoid) once per stretch, and the stretch's outputs leave
+// from shared memory as whole rows.
+#include "kda_common.cuh"
+#include "kda_stage.cuh"
+
+namespace kda {
+
+namespace {
+
+template <int DK, int DV>
+struct RecCfg {
+    static constexpr int NW = DV / 16, NT = NW * 32;
+    static constexpr int RP = DK / 8;               // rows per lane
+    static constexpr int CT = DK >= 128 ? 16 : 32;  // tokens per stretch
+    static constexpr int TPR = 8, E = DK / TPR;     // intake: threads per key row, elements each
+    static_assert(NW >= 2 && NW * 16 == DV && RP * 8 == DK && NT >= CT, "recurrent tiling");
+};
+
+template <typename Tin, int DK, int DV>
+struct RecSmem {
+    static constexpr int CT = RecCfg<DK, DV>::CT;
+    Tin rk[CT][DK], rq[CT][DK], rg[CT][DK], rv[CT][DV];  // raw rows, copied in by cp.async
+    float kh[CT][DK], qh[CT][DK], al[CT][DK];           // k^, q^, a = exp(g)
+    float v[CT][DV], o[CT][DV];
+    float b[CT];
+    float dtb[DK];                                       // dt_bias of the head (in-kernel gate)
+};
+
+// Start the copy of tokens [t0, t0 + cnt) of head h; returns this thread's raw
+// beta (thread i < cnt holds token i's), left unconverted so that the load
+// completes in the background.
+template <typename Tin, int DK, int DV>
+__device__ __forceinline__ Tin rec_issue(const ChunkParams &p, RecSmem<Tin, DK, DV> &sm, long long t0, int cnt, int h) {
+    constexpr int NT = RecCfg<DK, DV>::NT, EP = 16 / (int)sizeof(Tin);
+    constexpr int RK = DK / EP, RV = DV / EP;
+    const int tid = threadIdx.x, H = p.H;
+    for (int e = tid; e < cnt * RK; e += NT) {
+        const int i = e / RK, c = (e % RK) * EP;
+        const long long gi = ((t0 + i) * H + h) * DK + c;
+        cp_async16(&sm.rk[i][c], static_cast<const Tin *>(p.k) + gi);
+        cp_async16(&sm.rq[i][c], static_cast<const Tin *>(p.q) + gi);
+        cp_async16(&sm.rg[i][c], static_cast<const Tin *>(p.g) + gi);
+    }
+    for (int e = tid; e < cnt * RV; e += NT) {
+        const int i = e / RV, c = (e % RV) * EP;
+        cp_async16(&sm.rv[i][c], static_cast<const Tin *>(p.v) + ((t0 + i) * H + h) * DV + c);
+    }
+    cp_async_commit();
+    return tid < cnt ? static_cast<const Tin *>(p.beta)[(t0 + tid) * H + h] : Tin(0.f);
+}
+
+// The staged stretch as fp32 token vectors. Each key row is taken by TPR
+// threads that form its squared norms with shuffles (uniform trip count: rows
+// past cnt read row 0 and store nothing). Barriers on both sides.
+template <typename Tin, int DK, int DV>
+__device__ void rec_take(const ChunkParams &p, RecSmem<Tin, DK, DV> &sm, int cnt, Tin beta_raw, float rate) {
+    using Cfg = RecCfg<DK, DV>;
+    constexpr int NT = Cfg::NT, TPR = Cfg::TPR, E = Cfg::E;
+    const int tid = threadIdx.x;
+    cp_async_wait_all();
+    __syncthreads();
+    const int c = (tid % TPR) * E;
+    for (int i0 = 0; i0 < cnt; i0 += NT / TPR) {
+        const int i = i0 + tid / TPR;
+        const bool live = i < cnt;
+        const int ir = live ? i : 0;
+        float kx[E], qx[E], gx[E];
+        stage_cvt<E>(&sm.rk[ir][c], kx);
+        stage_cvt<E>(&sm.rq[ir][c], qx);
+        stage_cvt<E>(&sm.rg[ir][c], gx);
+        float kk = 0.f, qq = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) { kk = fmaf(kx[e], kx[e], kk); qq = fmaf(qx[e], qx[e], qq); }
+#pragma unroll
+        for (int o = TPR / 2; o > 0; o >>= 1) {
+            kk += __shfl_xor_sync(0xffffffffu, kk, o);
+            qq += __shfl_xor_sync(0xffffffffu, qq, o);
+        }
+        const float rk = p.use_l2 ? rsqrtf(kk + kL2Eps) : 1.f, rq = p.use_l2 ? rsqrtf(qq + kL2Eps) : 1.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            kx[e] *= rk;
+            qx[e] *= rq;
+            gx[e] = expf(gate_value(gx[e], sm.dtb[c + e], rate, p.gate_mode, p.has_lb, p.lb));
+        }
+        if (live) {
+            store_vec<E>(&sm.kh[i][c], kx);
+            store_vec<E>(&sm.qh[i][c], qx);
+            store_vec<E>(&sm.al[i][c], gx);
+        }
+    }
+    for (int e = tid; e < cnt * DV; e += NT) {
+        const int i = e / DV, cc = e % DV;
+        sm.v[i][cc] = to_f32(sm.rv[i][cc]);
+    }
+    if (tid < cnt) sm.b[tid] = beta_value(to_f32(beta_raw), p.beta_prob);
+    __syncthreads();
+}
+
+template <int RP>
+__device__ __forceinline__ void rows_in(const float *src, float (&out)[RP]) {
+#pragma unroll
+    for (int j = 0; j < RP; j += 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(src + j);
+        out[j] = x.x; out[j + 1] = x.y; out[j + 2] = x.z; out[j + 3] = x.w;
+    }
+}
+
+// Sum of 4 values over the 8 row groups of a warp (lane bits 4, 3, 2), by
+// reduce-scatter: bit 4 keeps (z, w) or (x, y), bit 3 one of the two, bit 2 adds
+// the partner. Returns the total of value (bit 4, bit 3) of this lane's column
+// group (lanes with bit 2 = 0 and 1 hold the same).
+__device__ __forceinline__ float rowgroup_scatter4(float4 x) {
+    const int lane = threadIdx.x & 31;
+    const bool h4 = lane & 16, h3 = lane & 8;
+    float a0 = h4 ? x.z : x.x, a1 = h4 ? x.w : x.y;
+    a0 += __shfl_xor_sync(0xffffffffu, h4 ? x.x : x.z, 16);
+    a1 += __shfl_xor_sync(0xffffffffu, h4 ? x.y : x.w, 16);
+    float m = h3 ? a1 : a0;
+    m += __shfl_xor_sync(0xffffffffu, h3 ? a0 : a1, 8);
+    m += __shfl_xor_sync(0xffffffffu, m, 4);
+    return m;
+}
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(ChunkParams p) {
+    using Cfg = RecCfg<DK, DV>;
+    constexpr int RP = Cfg::RP, CT = Cfg::CT, NT = Cfg::NT;
+    extern __shared__ __align__(16) uint8_t smraw[];
+    RecSmem<Tin, DK, DV> &sm = *reinterpret_cast<RecSmem<Tin, DK, DV> *>(smraw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int rg = lane >> 2, cg = lane & 3;
+    const int col = 16 * warp + 4 * cg;  // this lane's first value column
+    const long long nh = blockIdx.x;
+    const int n = (int)(nh / p.H), h = (int)(nh % p.H), H = p.H;
+    long long bos, eos;
+    if (p.cu_seqlens) { bos = p.cu_seqlens[n]; eos = p.cu_seqlens[n + 1]; }
+    else { bos = (long long)n * p.T; eos = bos + p.T; }
+
+    const float rate = p.gate_mode != kGateLog ? expf(p.A_log[h]) : 0.f;
+    for (int c = tid; c < DK; c += NT)
+        sm.dtb[c] = (p.gate_mode != kGateLog && p.dt_bias) ? p.dt_bias[(long long)h * DK + c] : 0.f;
+
+    float4 s[RP];
+#pragma unroll
+    for (int r = 0; r < RP; ++r)
+        s[r] = p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + (nh * DK + rg * RP + r) * DV + col)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+
+    Tin braw = bos < eos ? rec_issue<Tin, DK, DV>(p, sm, bos, (int)min((long long)CT, eos - bos), h) : Tin(0.f);
+    for (long long t0 = bos; t0 < eos; t0 += CT) {
+        const int cnt = (int)min((long long)CT, eos - t0);
+        rec_take<Tin, DK, DV>(p, sm, cnt, braw, rate);
+        if (t0 + CT < eos) braw = rec_issue<Tin, DK, DV>(p, sm, t0 + CT, (int)min((long long)CT, eos - t0 - CT), h);
+        for (int i = 0; i < cnt; ++i) {
+            float kr[RP], ar[RP], qr[RP];
+            rows_in<RP>(&sm.kh[i][rg * RP], kr);
+            rows_in<RP>(&sm.al[i][rg * RP], ar);
+            rows_in<RP>(&sm.qh[i][rg * RP], qr);
+            const float b = sm.b[i];
+            const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][col]);
+            // S' = diag(a) S and this lane's part of u = S'^T k^ (two chains)
+            float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+                s[r].x *= ar[r]; s[r].y *= ar[r]; s[r].z *= ar[r]; s[r].w *= ar[r];
+                float4 &acc = (r & 1) ? pb : pa;
+                acc.x = fmaf(s[r].x, kr[r], acc.x); acc.y = fmaf(s[r].y, kr[r], acc.y);
+                acc.z = fmaf(s[r].z, kr[r], acc.z); acc.w = fmaf(s[r].w, kr[r], acc.w);
+            }
+            const float m = rowgroup_scatter4(make_float4(pa.x + pb.x, pa.y + pb.y, pa.z + pb.z, pa.w + pb.w));
+            // gather u of the 4 columns from the lanes that hold them (bits 4, 3 = value index)
+            const float4 u = make_float4(__shfl_sync(0xffffffffu, m, cg), __shfl_sync(0xffffffffu, m, 8 + cg),
+                                         __shfl_sync(0xffffffffu, m, 16 + cg), __shfl_sync(0xffffffffu, m, 24 + cg));
+            const float4 d = make_float4(b * (vv.x - u.x), b * (vv.y - u.y), b * (vv.z - u.z), b * (vv.w - u.w));
+            // S = S' + k^ d^T and this lane's part of S^T q^
+            pa = make_float4(0.f, 0.f, 0.f, 0.f);
+            pb = pa;
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+                s[r].x = fmaf(kr[r], d.x, s[r].x); s[r].y = fmaf(kr[r], d.y, s[r].y);
+                s[r].z = fmaf(kr[r], d.z, s[r].z); s[r].w = fmaf(kr[r], d.w, s[r].w);
+                float4 &acc = (r & 1) ? pb : pa;
+                acc.x = fmaf(s[r].x, qr[r], acc.x); acc.y = fmaf(s[r].y, qr[r], acc.y);
+                acc.z = fmaf(s[r].z, qr[r], acc.z); acc.w = fmaf(s[r].w, qr[r], acc.w);
+            }
+            const float ov = rowgroup_scatter4(make_float4(pa.x + pb.x, pa.y + pb.y, pa.z + pb.z, pa.w + pb.w));
+            if ((lane & 4) == 0) sm.o[i][col + (lane >> 3)] = p.scale * ov;
+        }
+        // the stretch's output rows, from shared memory
+        __syncthreads();
+        for (int e = 4 * tid; e < cnt * DV; e += 4 * NT) {
+            const int i = e / DV, c = e % DV;
+            const float4 x = *reinterpret_cast<const float4 *>(&sm.o[i][c]);
+            Tin *dst = static_cast<Tin *>(p.o) + ((t0 + i) * H + h) * DV + c;
+            dst[0] = from_f32<Tin>(x.x); dst[1] = from_f32<Tin>(x.y);
+            dst[2] = from_f32<Tin>(x.z); dst[3] = from_f32<Tin>(x.w);
+        }
+    }
+    if (p.S_out) {
+#pragma unroll
+        for (int r = 0; r < RP; ++r) *reinterpret_cast<float4 *>(p.S_out + (nh * DK + rg * RP + r) * DV + col) = s[r];
+    }
+}
+
+template <typename Tin, int DK, int DV>
+cudaError_t launch_rec_t(const ChunkParams &p, cudaStream_t st) {
+    const long long blocks = (long long)p.N * p.H;
+    if (blocks == 0) return cudaSuccess;
+    const int smem = (int)sizeof(RecSmem<Tin, DK, DV>);
+    cudaError_t e = cudaFuncSetAttribute(kda_chunk_rec_kernel<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kda_chunk_rec_kernel<Tin, DK, DV><<<(unsigned)blocks, RecCfg<DK, DV>::NT, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t launch_rec_dt(const ChunkParams &p, int Dk, int Dv, cudaStream_t st) {
+#define KDA_REC_CASE(DK_, DV_) \
+    if (Dk == DK_ && Dv == DV_) return launch_rec_t<Tin, DK_, DV_>(p, st);
+    KDA_REC_CASE(32, 32) KDA_REC_CASE(32, 64) KDA_REC_CASE(32, 128)
+    KDA_REC_CASE(64, 32) KDA_REC_CASE(64, 64) KDA_REC_CASE(64, 128)
+    KDA_REC_CASE(128, 32) KDA_REC_CASE(128, 64) KDA_REC_CASE(128, 128)
+#undef KDA_REC_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_rec(const ChunkParams &p, bool bf16, int Dk, int Dv, cudaStream_t st) {
+    return bf16 ? launch_rec_dt<__nv_bfloat16>(p, Dk, Dv, st) : launch_rec_dt<float>(p, Dk, Dv, st);
+}
+
+}  // namespace kda
