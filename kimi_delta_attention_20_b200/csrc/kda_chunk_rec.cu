@@ -40,7 +40,8 @@ struct RecSmem {
     static constexpr int CT = RecCfg<DK, DV>::CT;
     Tin rk[CT][DK], rq[CT][DK], rg[CT][DK], rv[CT][DV];  // raw rows, copied in by cp.async
     float kh[CT][DK], qh[CT][DK], al[CT][DK];           // k^, q^, a = exp(g)
-    float v[CT][DV], o[CT][DV];
+    float vo[CT][DV];  // v of token i, then its output: a warp reads v[i] of its own columns
+                       // before its shuffles and writes o[i] of the same columns after them
     float b[CT];
     float dtb[DK];                                       // dt_bias of the head (in-kernel gate)
 };
@@ -110,7 +111,7 @@ __device__ void rec_take(const ChunkParams &p, RecSmem<Tin, DK, DV> &sm, int cnt
     }
     for (int e = tid; e < cnt * DV; e += NT) {
         const int i = e / DV, cc = e % DV;
-        sm.v[i][cc] = to_f32(sm.rv[i][cc]);
+        sm.vo[i][cc] = to_f32(sm.rv[i][cc]);
     }
     if (tid < cnt) sm.b[tid] = beta_value(to_f32(beta_raw), p.beta_prob);
     __syncthreads();
@@ -171,13 +172,14 @@ __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(Chunk
         const int cnt = (int)min((long long)CT, eos - t0);
         rec_take<Tin, DK, DV>(p, sm, cnt, braw, rate);
         if (t0 + CT < eos) braw = rec_issue<Tin, DK, DV>(p, sm, t0 + CT, (int)min((long long)CT, eos - t0 - CT), h);
+#pragma unroll 2
         for (int i = 0; i < cnt; ++i) {
             float kr[RP], ar[RP], qr[RP];
             rows_in<RP>(&sm.kh[i][rg * RP], kr);
             rows_in<RP>(&sm.al[i][rg * RP], ar);
             rows_in<RP>(&sm.qh[i][rg * RP], qr);
             const float b = sm.b[i];
-            const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][col]);
+            const float4 vv = *reinterpret_cast<const float4 *>(&sm.vo[i][col]);
             // S' = diag(a) S and this lane's part of u = S'^T k^ (two chains)
             float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
 #pragma unroll
@@ -204,13 +206,13 @@ __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(Chunk
                 acc.z = fmaf(s[r].z, qr[r], acc.z); acc.w = fmaf(s[r].w, qr[r], acc.w);
             }
             const float ov = rowgroup_scatter4(make_float4(pa.x + pb.x, pa.y + pb.y, pa.z + pb.z, pa.w + pb.w));
-            if ((lane & 4) == 0) sm.o[i][col + (lane >> 3)] = p.scale * ov;
+            if ((lane & 4) == 0) sm.vo[i][col + (lane >> 3)] = p.scale * ov;
         }
         // the stretch's output rows, from shared memory
         __syncthreads();
         for (int e = 4 * tid; e < cnt * DV; e += 4 * NT) {
             const int i = e / DV, c = e % DV;
-            const float4 x = *reinterpret_cast<const float4 *>(&sm.o[i][c]);
+            const float4 x = *reinterpret_cast<const float4 *>(&sm.vo[i][c]);
             Tin *dst = static_cast<Tin *>(p.o) + ((t0 + i) * H + h) * DV + c;
             dst[0] = from_f32<Tin>(x.x); dst[1] = from_f32<Tin>(x.y);
             dst[2] = from_f32<Tin>(x.z); dst[3] = from_f32<Tin>(x.w);
