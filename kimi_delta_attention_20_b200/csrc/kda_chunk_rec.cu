@@ -161,11 +161,16 @@ __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(Chunk
     for (int c = tid; c < DK; c += NT)
         sm.dtb[c] = (p.gate_mode != kGateLog && p.dt_bias) ? p.dt_bias[(long long)h * DK + c] : 0.f;
 
-    float4 s[RP];
+    // the state as column pairs (4 cg, 4 cg + 1) and (4 cg + 2, 4 cg + 3), for the
+    // paired fp32 FMA pipe
+    float2 s[RP][2];
 #pragma unroll
-    for (int r = 0; r < RP; ++r)
-        s[r] = p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + (nh * DK + rg * RP + r) * DV + col)
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = 0; r < RP; ++r) {
+        const float4 x = p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + (nh * DK + rg * RP + r) * DV + col)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        s[r][0] = make_float2(x.x, x.y);
+        s[r][1] = make_float2(x.z, x.w);
+    }
 
     Tin braw = bos < eos ? rec_issue<Tin, DK, DV>(p, sm, bos, (int)min((long long)CT, eos - bos), h) : Tin(0.f);
     for (long long t0 = bos; t0 < eos; t0 += CT) {
@@ -180,32 +185,39 @@ __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(Chunk
             rows_in<RP>(&sm.qh[i][rg * RP], qr);
             const float b = sm.b[i];
             const float4 vv = *reinterpret_cast<const float4 *>(&sm.vo[i][col]);
-            // S' = diag(a) S and this lane's part of u = S'^T k^ (two chains)
-            float4 pa = make_float4(0.f, 0.f, 0.f, 0.f), pb = pa;
+            // S' = diag(a) S and this lane's part of u = S'^T k^ (two chains per pair)
+            const float2 z2 = make_float2(0.f, 0.f);
+            float2 acc[2][2] = {{z2, z2}, {z2, z2}};
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
-                s[r].x *= ar[r]; s[r].y *= ar[r]; s[r].z *= ar[r]; s[r].w *= ar[r];
-                float4 &acc = (r & 1) ? pb : pa;
-                acc.x = fmaf(s[r].x, kr[r], acc.x); acc.y = fmaf(s[r].y, kr[r], acc.y);
-                acc.z = fmaf(s[r].z, kr[r], acc.z); acc.w = fmaf(s[r].w, kr[r], acc.w);
+                const float2 a2 = make_float2(ar[r], ar[r]), k2 = make_float2(kr[r], kr[r]);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    s[r][j] = __fmul2_rn(s[r][j], a2);
+                    acc[r & 1][j] = __ffma2_rn(s[r][j], k2, acc[r & 1][j]);
+                }
             }
-            const float m = rowgroup_scatter4(make_float4(pa.x + pb.x, pa.y + pb.y, pa.z + pb.z, pa.w + pb.w));
+            float2 u01 = __fadd2_rn(acc[0][0], acc[1][0]), u23 = __fadd2_rn(acc[0][1], acc[1][1]);
+            const float m = rowgroup_scatter4(make_float4(u01.x, u01.y, u23.x, u23.y));
             // gather u of the 4 columns from the lanes that hold them (bits 4, 3 = value index)
-            const float4 u = make_float4(__shfl_sync(0xffffffffu, m, cg), __shfl_sync(0xffffffffu, m, 8 + cg),
-                                         __shfl_sync(0xffffffffu, m, 16 + cg), __shfl_sync(0xffffffffu, m, 24 + cg));
-            const float4 d = make_float4(b * (vv.x - u.x), b * (vv.y - u.y), b * (vv.z - u.z), b * (vv.w - u.w));
+            u01 = make_float2(__shfl_sync(0xffffffffu, m, cg), __shfl_sync(0xffffffffu, m, 8 + cg));
+            u23 = make_float2(__shfl_sync(0xffffffffu, m, 16 + cg), __shfl_sync(0xffffffffu, m, 24 + cg));
+            const float2 b2 = make_float2(b, b);
+            const float2 d[2] = {__fmul2_rn(b2, __fadd2_rn(make_float2(vv.x, vv.y), make_float2(-u01.x, -u01.y))),
+                                 __fmul2_rn(b2, __fadd2_rn(make_float2(vv.z, vv.w), make_float2(-u23.x, -u23.y)))};
             // S = S' + k^ d^T and this lane's part of S^T q^
-            pa = make_float4(0.f, 0.f, 0.f, 0.f);
-            pb = pa;
+            float2 oc[2][2] = {{z2, z2}, {z2, z2}};
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
-                s[r].x = fmaf(kr[r], d.x, s[r].x); s[r].y = fmaf(kr[r], d.y, s[r].y);
-                s[r].z = fmaf(kr[r], d.z, s[r].z); s[r].w = fmaf(kr[r], d.w, s[r].w);
-                float4 &acc = (r & 1) ? pb : pa;
-                acc.x = fmaf(s[r].x, qr[r], acc.x); acc.y = fmaf(s[r].y, qr[r], acc.y);
-                acc.z = fmaf(s[r].z, qr[r], acc.z); acc.w = fmaf(s[r].w, qr[r], acc.w);
+                const float2 k2 = make_float2(kr[r], kr[r]), q2 = make_float2(qr[r], qr[r]);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    s[r][j] = __ffma2_rn(k2, d[j], s[r][j]);
+                    oc[r & 1][j] = __ffma2_rn(s[r][j], q2, oc[r & 1][j]);
+                }
             }
-            const float ov = rowgroup_scatter4(make_float4(pa.x + pb.x, pa.y + pb.y, pa.z + pb.z, pa.w + pb.w));
+            const float2 o01 = __fadd2_rn(oc[0][0], oc[1][0]), o23 = __fadd2_rn(oc[0][1], oc[1][1]);
+            const float ov = rowgroup_scatter4(make_float4(o01.x, o01.y, o23.x, o23.y));
             if ((lane & 4) == 0) sm.vo[i][col + (lane >> 3)] = p.scale * ov;
         }
         // the stretch's output rows, from shared memory
@@ -220,7 +232,9 @@ __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(Chunk
     }
     if (p.S_out) {
 #pragma unroll
-        for (int r = 0; r < RP; ++r) *reinterpret_cast<float4 *>(p.S_out + (nh * DK + rg * RP + r) * DV + col) = s[r];
+        for (int r = 0; r < RP; ++r)
+            *reinterpret_cast<float4 *>(p.S_out + (nh * DK + rg * RP + r) * DV + col) =
+                make_float4(s[r][0].x, s[r][0].y, s[r][1].x, s[r][1].y);
     }
 }
 
