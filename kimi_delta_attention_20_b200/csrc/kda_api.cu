@@ -5,6 +5,7 @@
 
 #include "../../include/kda.h"
 #include "kda_common.cuh"
+#include "kda_bwd.cuh"
 
 namespace kda {
 cudaError_t launch_decode(const StepParams &p, bool bf16, int Dk, int Dv, cudaStream_t st);

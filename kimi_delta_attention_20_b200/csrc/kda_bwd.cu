@@ -41,6 +41,7 @@
 #include <cooperative_groups.h>
 
 #include "kda_common.cuh"
+#include "kda_bwd.cuh"
 #include "kda_stage.cuh"
 
 namespace kda {
