@@ -290,24 +290,30 @@ __device__ __forceinline__ void fwd_step(const FwdSmem<Tin, DK> &sm, int i, floa
     for (int r = 0; r < RP; ++r) ar[r] = fabsf(ar[r]);
     const float b = sm.b[i];
     const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][4 * warp]);
-    float4 pu = make_float4(0.f, 0.f, 0.f, 0.f);
+    // decay and this lane's part of u on the paired fp32 FMA pipe
+    const float2 z2 = make_float2(0.f, 0.f);
+    float2 pu01 = z2, pu23 = z2;
 #pragma unroll
     for (int r = 0; r < RP; ++r) {
-        s[r].x *= ar[r]; s[r].y *= ar[r]; s[r].z *= ar[r]; s[r].w *= ar[r];
-        pu.x = fmaf(s[r].x, kr[r], pu.x); pu.y = fmaf(s[r].y, kr[r], pu.y);
-        pu.z = fmaf(s[r].z, kr[r], pu.z); pu.w = fmaf(s[r].w, kr[r], pu.w);
+        const float2 a2 = make_float2(ar[r], ar[r]), k2 = make_float2(kr[r], kr[r]);
+        float2 lo = __fmul2_rn(make_float2(s[r].x, s[r].y), a2), hi = __fmul2_rn(make_float2(s[r].z, s[r].w), a2);
+        s[r] = make_float4(lo.x, lo.y, hi.x, hi.y);
+        pu01 = __ffma2_rn(lo, k2, pu01);
+        pu23 = __ffma2_rn(hi, k2, pu23);
     }
     if (keep_s) {
 #pragma unroll
         for (int r = 0; r < RP; ++r) keep_s[r * kBwdThreads] = s[r];
     }
-    const float4 u = warp_allreduce4(pu);
+    const float4 u = warp_allreduce4(make_float4(pu01.x, pu01.y, pu23.x, pu23.y));
     if (keep_u && lane == 0) *reinterpret_cast<float4 *>(keep_u) = u;
-    const float4 d = make_float4(b * (vv.x - u.x), b * (vv.y - u.y), b * (vv.z - u.z), b * (vv.w - u.w));
+    const float2 d01 = make_float2(b * (vv.x - u.x), b * (vv.y - u.y)), d23 = make_float2(b * (vv.z - u.z), b * (vv.w - u.w));
 #pragma unroll
     for (int r = 0; r < RP; ++r) {
-        s[r].x = fmaf(kr[r], d.x, s[r].x); s[r].y = fmaf(kr[r], d.y, s[r].y);
-        s[r].z = fmaf(kr[r], d.z, s[r].z); s[r].w = fmaf(kr[r], d.w, s[r].w);
+        const float2 k2 = make_float2(kr[r], kr[r]);
+        const float2 lo = __ffma2_rn(k2, d01, make_float2(s[r].x, s[r].y));
+        const float2 hi = __ffma2_rn(k2, d23, make_float2(s[r].z, s[r].w));
+        s[r] = make_float4(lo.x, lo.y, hi.x, hi.y);
     }
 }
 
@@ -423,17 +429,21 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
             const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][4 * warp]);
             const float4 u = *reinterpret_cast<const float4 *>(&sm.u[i][4 * warp]);
 
-            // ---- dS += scale q^ do^T, then ddelta = dS^T k^ (warp sum)
-            float4 dd = make_float4(0.f, 0.f, 0.f, 0.f);
+            // ---- dS += scale q^ do^T, then ddelta = dS^T k^ (warp sum); column pairs
+            // on the paired fp32 FMA pipe
+            const float2 do01 = make_float2(dov.x, dov.y), do23 = make_float2(dov.z, dov.w);
+            float2 dd01 = make_float2(0.f, 0.f), dd23 = dd01;
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
                 const float qs = p.scale * qr[r];
-                ds[r].x = fmaf(qs, dov.x, ds[r].x); ds[r].y = fmaf(qs, dov.y, ds[r].y);
-                ds[r].z = fmaf(qs, dov.z, ds[r].z); ds[r].w = fmaf(qs, dov.w, ds[r].w);
-                dd.x = fmaf(ds[r].x, kr[r], dd.x); dd.y = fmaf(ds[r].y, kr[r], dd.y);
-                dd.z = fmaf(ds[r].z, kr[r], dd.z); dd.w = fmaf(ds[r].w, kr[r], dd.w);
+                const float2 qs2 = make_float2(qs, qs), k2 = make_float2(kr[r], kr[r]);
+                const float2 lo = __ffma2_rn(qs2, do01, make_float2(ds[r].x, ds[r].y));
+                const float2 hi = __ffma2_rn(qs2, do23, make_float2(ds[r].z, ds[r].w));
+                ds[r] = make_float4(lo.x, lo.y, hi.x, hi.y);
+                dd01 = __ffma2_rn(lo, k2, dd01);
+                dd23 = __ffma2_rn(hi, k2, dd23);
             }
-            dd = warp_allreduce4(dd);
+            const float4 dd = warp_allreduce4(make_float4(dd01.x, dd01.y, dd23.x, dd23.y));
             const float4 vu = make_float4(vv.x - u.x, vv.y - u.y, vv.z - u.z, vv.w - u.w);
             const float4 dl = make_float4(b * vu.x, b * vu.y, b * vu.z, b * vu.w);
             if (lane < 4) {  // dv = b ddelta for this warp's columns, one per lane
@@ -444,10 +454,18 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
             const float ddo = dot4(dl, dov), db = dot4(dd, vu);
 
             // ---- this warp's terms of the row sums S' do, dS delta, S' ddelta, dS (.) S'
+            const float2 dl01 = make_float2(dl.x, dl.y), dl23 = make_float2(dl.z, dl.w);
+            const float2 dd01r = make_float2(dd.x, dd.y), dd23r = make_float2(dd.z, dd.w);
             float tq[RP], tk[RP], tg[RP];
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
-                const float ra = dot4(s[r], dov), rb = dot4(ds[r], dl), re = dot4(s[r], dd), rh = dot4(ds[r], s[r]);
+                const float2 s01 = make_float2(s[r].x, s[r].y), s23 = make_float2(s[r].z, s[r].w);
+                const float2 g01 = make_float2(ds[r].x, ds[r].y), g23 = make_float2(ds[r].z, ds[r].w);
+                const float2 xa = __ffma2_rn(s23, do23, __fmul2_rn(s01, do01));
+                const float2 xb = __ffma2_rn(g23, dl23, __fmul2_rn(g01, dl01));
+                const float2 xe = __ffma2_rn(s23, dd23r, __fmul2_rn(s01, dd01r));
+                const float2 xh = __ffma2_rn(g23, s23, __fmul2_rn(g01, s01));
+                const float ra = xa.x + xa.y, rb = xb.x + xb.y, re = xe.x + xe.y, rh = xh.x + xh.y;
                 tq[r] = p.scale * fmaf(kr[r], ddo, ra);
                 tk[r] = fmaf(-b, re, rb);
                 tg[r] = ar[r] > 0.f ? fmaf(-b * kr[r], re, rh) : 0.f;
@@ -459,9 +477,11 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
             // ---- dS <- diag(a) (dS - b k^ ddelta^T), the cotangent of the entering state
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
-                const float bk = b * kr[r], a = fabsf(ar[r]);
-                ds[r].x = a * fmaf(-bk, dd.x, ds[r].x); ds[r].y = a * fmaf(-bk, dd.y, ds[r].y);
-                ds[r].z = a * fmaf(-bk, dd.z, ds[r].z); ds[r].w = a * fmaf(-bk, dd.w, ds[r].w);
+                const float nbk = -b * kr[r], a = fabsf(ar[r]);
+                const float2 nbk2 = make_float2(nbk, nbk), a2 = make_float2(a, a);
+                const float2 lo = __fmul2_rn(a2, __ffma2_rn(nbk2, dd01r, make_float2(ds[r].x, ds[r].y)));
+                const float2 hi = __fmul2_rn(a2, __ffma2_rn(nbk2, dd23r, make_float2(ds[r].z, ds[r].w)));
+                ds[r] = make_float4(lo.x, lo.y, hi.x, hi.y);
             }
             // ---- the CTA's terms of token i: the 4 warps' terms added in a fixed order
             __syncthreads();
@@ -487,33 +507,35 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
         cluster_arrive();
         cluster_wait();
         for (int i = rank + NS * warp; i < cnt; i += NS * kWarps) {
-            constexpr int CP = DK / 32;
-            float sq[CP], sk[CP], sg[CP];
+            constexpr int CP = DK / 32;  // channels per lane, contiguous: c0 .. c0 + CP - 1
+            const int c0 = CP * lane;
+            float sq[CP], sk[CP], sg[CP], qv[CP], kv[CP];
+#pragma unroll
+            for (int j = 0; j < CP; ++j) { sq[j] = 0.f; sk[j] = 0.f; sg[j] = 0.f; }
+#pragma unroll
+            for (int q = 0; q < NS; ++q) {
+                const BwdSmem<Tin, DK> *rs = cluster.map_shared_rank(&sm, q);
+                float x[CP], y[CP], z[CP];
+                load_rows<CP>(&rs->pd[0][i][c0], x);
+                load_rows<CP>(&rs->pd[1][i][c0], y);
+                load_rows<CP>(&rs->pd[2][i][c0], z);
+#pragma unroll
+                for (int j = 0; j < CP; ++j) { sq[j] += x[j]; sk[j] += y[j]; sg[j] += z[j]; }
+            }
+            load_rows<CP>(&sm.qh[i][c0], qv);
+            load_rows<CP>(&sm.kh[i][c0], kv);
             float qd = 0.f, kd = 0.f;
 #pragma unroll
-            for (int j = 0; j < CP; ++j) {
-                const int c = lane + 32 * j;
-                sq[j] = 0.f; sk[j] = 0.f; sg[j] = 0.f;
-#pragma unroll
-                for (int q = 0; q < NS; ++q) {
-                    const BwdSmem<Tin, DK> *rs = cluster.map_shared_rank(&sm, q);
-                    sq[j] += rs->pd[0][i][c];
-                    sk[j] += rs->pd[1][i][c];
-                    sg[j] += rs->pd[2][i][c];
-                }
-                qd = fmaf(sm.qh[i][c], sq[j], qd);
-                kd = fmaf(sm.kh[i][c], sk[j], kd);
-            }
+            for (int j = 0; j < CP; ++j) { qd = fmaf(qv[j], sq[j], qd); kd = fmaf(kv[j], sk[j], kd); }
             qd = p.use_l2 ? warp_sum(qd) : 0.f;
             kd = p.use_l2 ? warp_sum(kd) : 0.f;
             const float rq = sm.rq[i], rk = sm.rk[i];
+            const long long gi = ((t0 + i) * H + h) * DK + c0;
 #pragma unroll
             for (int j = 0; j < CP; ++j) {
-                const int c = lane + 32 * j;
-                const long long gi = ((t0 + i) * H + h) * DK + c;
-                static_cast<Tin *>(p.dq)[gi] = from_f32<Tin>(rq * fmaf(-sm.qh[i][c], qd, sq[j]));
-                static_cast<Tin *>(p.dk)[gi] = from_f32<Tin>(rk * fmaf(-sm.kh[i][c], kd, sk[j]));
-                static_cast<Tin *>(p.dg)[gi] = from_f32<Tin>(sg[j]);
+                static_cast<Tin *>(p.dq)[gi + j] = from_f32<Tin>(rq * fmaf(-qv[j], qd, sq[j]));
+                static_cast<Tin *>(p.dk)[gi + j] = from_f32<Tin>(rk * fmaf(-kv[j], kd, sk[j]));
+                static_cast<Tin *>(p.dg)[gi + j] = from_f32<Tin>(sg[j]);
             }
             if (lane == 0) {
                 float db = 0.f;
