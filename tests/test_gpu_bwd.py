@@ -99,3 +99,32 @@ def test_autograd_rejects_in_kernel_gate():
     with pytest.raises(NotImplementedError):
         kda.chunk_kda(q, inp["k"], inp["v"], inp["g"], inp["beta"], use_gate_in_kernel=True,
                       A_log=params["A_log"], use_qk_l2norm_in_kernel=True)
+
+
+def test_backward_full_size_sampled():
+    """The backward leg of bench.py at its full size (B1 T8192 H16 d128, bf16, lower bound
+    -5, output and final-state cotangents) in the launch configuration it times. The
+    gradients of a head's last 1024 tokens depend on the rest of the sequence only
+    through the state entering token 7168, so for heads 0 and 15 the oracle runs the
+    forward recurrence to that state (`oracle.recurrent`) and the backward from there
+    (`oracle.backward` with that initial state and the final-state cotangent)."""
+    import kimi_delta_attention_20_b200 as kda
+    wl = KI.CHUNK_WORKLOADS[2]
+    inp = KI.chunk_inputs(wl)
+    gen = torch.Generator().manual_seed(wl.seed + 1000)
+    do = torch.randn(inp["v"].shape, generator=gen).to(wl.dtype)
+    dSf = torch.randn(1, wl.H, wl.Dk, wl.Dv, generator=gen) * 0.5
+    d = {n: inp[n].to(DEV) for n in ("q", "k", "v", "g", "beta")}
+    got = kda.chunk_kda_bwd(d["q"], d["k"], d["v"], d["g"], d["beta"], do.to(DEV), dfinal_state=dSf.to(DEV),
+                            use_qk_l2norm_in_kernel=True, lower_bound=wl.lower_bound)
+    torch.cuda.synchronize()
+    t_split = wl.T - 1024
+    for h in (0, wl.H - 1):
+        sl = lambda x: x[0, :, h:h + 1]
+        pre = [sl(inp[n])[:t_split] for n in ("q", "k", "v", "g", "beta")]
+        _, S_mid = oracle.recurrent(*pre, lower_bound=wl.lower_bound)
+        post = [sl(inp[n])[t_split:] for n in ("q", "k", "v", "g", "beta")]
+        want = oracle.backward(*post, sl(do)[t_split:], dS_final=dSf[:, h:h + 1], initial_state=S_mid,
+                               lower_bound=wl.lower_bound)
+        for name, gt, wt in zip(NAMES[:5], got[:5], want[:5]):
+            check(f"full-size h{h} {name}", gt[0, t_split:, h:h + 1], wt, wl.dtype)
