@@ -10,12 +10,12 @@
 // arithmetic, not its value. For small head dims the recurrence also takes
 // fewer operations than the chunked form (no C x C blocks, no inverse).
 //
-// One CTA per (sequence, head), one warp per 16 value columns. Lane (rg, cg) =
-// (lane / 4, lane % 4) keeps rows rg*RP .. rg*RP+RP-1 (RP = d_k / 8) of columns
-// 4 cg .. 4 cg + 3 of its warp's block as float4 in registers. The key-axis sums
-// u and o are reductions over the 8 row groups of a warp (reduce-scatter, then
-// a gather for u: 8 shuffles); nothing else crosses lanes, and no barrier is
-// taken per token. Tokens arrive in stretches of CT: the raw rows of the next
+// One CTA per (sequence, head), one warp per 4 CG value columns (CG = 4). Lane (rg, cg) = (lane / 4, lane % 4) keeps rows
+// rg*RP .. rg*RP+RP-1 (RP = d_k / 8) of columns CG cg .. CG cg + CG - 1 of its
+// warp's block in registers, as column pairs for the paired fp32 FMA pipe. The
+// key-axis sums u and o are reductions over the 8 row groups of a warp (a
+// reduce-scatter, then a gather for u); nothing else crosses lanes, and no barrier
+// is taken per token. Tokens arrive in stretches of CT: the raw rows of the next
 // stretch are copied by cp.async while the current one runs, turned into fp32
 // (L2 norms, gate, sigmoid) once per stretch, and the stretch's outputs leave
 // from shared memory as whole rows.
@@ -28,11 +28,16 @@ namespace {
 
 template <int DK, int DV>
 struct RecCfg {
-    static constexpr int NW = DV / 16, NT = NW * 32;
+    // value columns per lane: 4. Eight halve the shuffles and loads per state element
+    // but also the warps per CTA; on the 300M layer (1024 CTAs, one wave) that was
+    // slower (1.59 ms against 1.44 ms), the kernel leaning on warps to hide latency.
+    static constexpr int CG = 4;
+    static constexpr int WC = 4 * CG;               // value columns per warp
+    static constexpr int NW = DV / WC, NT = NW * 32;
     static constexpr int RP = DK / 8;               // rows per lane
     static constexpr int CT = DK >= 128 ? 16 : 32;  // tokens per stretch
     static constexpr int TPR = 8, E = DK / TPR;     // intake: threads per key row, elements each
-    static_assert(NW >= 2 && NW * 16 == DV && RP * 8 == DK && NT >= CT, "recurrent tiling");
+    static_assert(NW >= 1 && NW * WC == DV && RP * 8 == DK && NT >= CT && NT >= 64, "recurrent tiling");
 };
 
 template <typename Tin, int DK, int DV>
@@ -126,31 +131,40 @@ __device__ __forceinline__ void rows_in(const float *src, float (&out)[RP]) {
     }
 }
 
-// Sum of 4 values over the 8 row groups of a warp (lane bits 4, 3, 2), by
-// reduce-scatter: bit 4 keeps (z, w) or (x, y), bit 3 one of the two, bit 2 adds
-// the partner. Returns the total of value (bit 4, bit 3) of this lane's column
-// group (lanes with bit 2 = 0 and 1 hold the same).
-__device__ __forceinline__ float rowgroup_scatter4(float4 x) {
+// Sum of CG values over the 8 row groups of a warp (lane bits 4, 3, 2) by
+// reduce-scatter: at lane bit 16, 8, ... each lane keeps the upper or lower half of
+// its values and adds the partner's copy of that half. Returns the total of value
+// v = lane / (32 / CG) of this lane's column group (for CG = 4, bit 2 is a plain
+// butterfly and lanes with bit 2 = 0 and 1 hold the same).
+template <int CG>
+__device__ __forceinline__ float rowgroup_scatter(const float (&x)[CG]) {
     const int lane = threadIdx.x & 31;
-    const bool h4 = lane & 16, h3 = lane & 8;
-    float a0 = h4 ? x.z : x.x, a1 = h4 ? x.w : x.y;
-    a0 += __shfl_xor_sync(0xffffffffu, h4 ? x.x : x.z, 16);
-    a1 += __shfl_xor_sync(0xffffffffu, h4 ? x.y : x.w, 16);
-    float m = h3 ? a1 : a0;
-    m += __shfl_xor_sync(0xffffffffu, h3 ? a0 : a1, 8);
-    m += __shfl_xor_sync(0xffffffffu, m, 4);
-    return m;
+    float a[CG];
+#pragma unroll
+    for (int j = 0; j < CG; ++j) a[j] = x[j];
+#pragma unroll
+    for (int n = CG, bit = 16; n > 1; n >>= 1, bit >>= 1) {
+        const bool hi = lane & bit;
+#pragma unroll
+        for (int j = 0; j < n / 2; ++j) {
+            const float keep = hi ? a[n / 2 + j] : a[j], send = hi ? a[j] : a[n / 2 + j];
+            a[j] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+        }
+    }
+    if constexpr (CG == 4) a[0] += __shfl_xor_sync(0xffffffffu, a[0], 4);
+    return a[0];
 }
 
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(ChunkParams p) {
     using Cfg = RecCfg<DK, DV>;
-    constexpr int RP = Cfg::RP, CT = Cfg::CT, NT = Cfg::NT;
+    constexpr int RP = Cfg::RP, CT = Cfg::CT, NT = Cfg::NT, CG = Cfg::CG, CP = CG / 2;
+    constexpr int VS = 32 / CG;  // lanes between the holders of consecutive reduced values
     extern __shared__ __align__(16) uint8_t smraw[];
     RecSmem<Tin, DK, DV> &sm = *reinterpret_cast<RecSmem<Tin, DK, DV> *>(smraw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int rg = lane >> 2, cg = lane & 3;
-    const int col = 16 * warp + 4 * cg;  // this lane's first value column
+    const int col = Cfg::WC * warp + CG * cg;  // this lane's first value column
     const long long nh = blockIdx.x;
     const int n = (int)(nh / p.H), h = (int)(nh % p.H), H = p.H;
     long long bos, eos;
@@ -161,16 +175,17 @@ __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(Chunk
     for (int c = tid; c < DK; c += NT)
         sm.dtb[c] = (p.gate_mode != kGateLog && p.dt_bias) ? p.dt_bias[(long long)h * DK + c] : 0.f;
 
-    // the state as column pairs (4 cg, 4 cg + 1) and (4 cg + 2, 4 cg + 3), for the
-    // paired fp32 FMA pipe
-    float2 s[RP][2];
+    // the state as column pairs (col + 2 j, col + 2 j + 1), for the paired fp32 FMA pipe
+    float2 s[RP][CP];
 #pragma unroll
-    for (int r = 0; r < RP; ++r) {
-        const float4 x = p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + (nh * DK + rg * RP + r) * DV + col)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-        s[r][0] = make_float2(x.x, x.y);
-        s[r][1] = make_float2(x.z, x.w);
-    }
+    for (int r = 0; r < RP; ++r)
+#pragma unroll
+        for (int j = 0; j < CP; j += 2) {
+            const float4 x = p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + (nh * DK + rg * RP + r) * DV + col + 2 * j)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            s[r][j] = make_float2(x.x, x.y);
+            s[r][j + 1] = make_float2(x.z, x.w);
+        }
 
     Tin braw = bos < eos ? rec_issue<Tin, DK, DV>(p, sm, bos, (int)min((long long)CT, eos - bos), h) : Tin(0.f);
     for (long long t0 = bos; t0 < eos; t0 += CT) {
@@ -184,41 +199,62 @@ __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(Chunk
             rows_in<RP>(&sm.al[i][rg * RP], ar);
             rows_in<RP>(&sm.qh[i][rg * RP], qr);
             const float b = sm.b[i];
-            const float4 vv = *reinterpret_cast<const float4 *>(&sm.vo[i][col]);
+            float2 vv[CP];
+#pragma unroll
+            for (int j = 0; j < CP; j += 2) {
+                const float4 x = *reinterpret_cast<const float4 *>(&sm.vo[i][col + 2 * j]);
+                vv[j] = make_float2(x.x, x.y);
+                vv[j + 1] = make_float2(x.z, x.w);
+            }
             // S' = diag(a) S and this lane's part of u = S'^T k^ (two chains per pair)
             const float2 z2 = make_float2(0.f, 0.f);
-            float2 acc[2][2] = {{z2, z2}, {z2, z2}};
+            float2 acc[2][CP];
+#pragma unroll
+            for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
                 const float2 a2 = make_float2(ar[r], ar[r]), k2 = make_float2(kr[r], kr[r]);
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
+                for (int j = 0; j < CP; ++j) {
                     s[r][j] = __fmul2_rn(s[r][j], a2);
                     acc[r & 1][j] = __ffma2_rn(s[r][j], k2, acc[r & 1][j]);
                 }
             }
-            float2 u01 = __fadd2_rn(acc[0][0], acc[1][0]), u23 = __fadd2_rn(acc[0][1], acc[1][1]);
-            const float m = rowgroup_scatter4(make_float4(u01.x, u01.y, u23.x, u23.y));
-            // gather u of the 4 columns from the lanes that hold them (bits 4, 3 = value index)
-            u01 = make_float2(__shfl_sync(0xffffffffu, m, cg), __shfl_sync(0xffffffffu, m, 8 + cg));
-            u23 = make_float2(__shfl_sync(0xffffffffu, m, 16 + cg), __shfl_sync(0xffffffffu, m, 24 + cg));
+            float part[CG];
+#pragma unroll
+            for (int j = 0; j < CP; ++j) {
+                const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
+                part[2 * j] = t.x; part[2 * j + 1] = t.y;
+            }
+            const float m = rowgroup_scatter<CG>(part);
+            // gather u of the lane's columns from the lanes that hold them
+            float2 d[CP];
             const float2 b2 = make_float2(b, b);
-            const float2 d[2] = {__fmul2_rn(b2, __fadd2_rn(make_float2(vv.x, vv.y), make_float2(-u01.x, -u01.y))),
-                                 __fmul2_rn(b2, __fadd2_rn(make_float2(vv.z, vv.w), make_float2(-u23.x, -u23.y)))};
+#pragma unroll
+            for (int j = 0; j < CP; ++j) {
+                const float2 u = make_float2(__shfl_sync(0xffffffffu, m, (2 * j) * VS + cg),
+                                             __shfl_sync(0xffffffffu, m, (2 * j + 1) * VS + cg));
+                d[j] = __fmul2_rn(b2, __fadd2_rn(vv[j], make_float2(-u.x, -u.y)));
+            }
             // S = S' + k^ d^T and this lane's part of S^T q^
-            float2 oc[2][2] = {{z2, z2}, {z2, z2}};
+#pragma unroll
+            for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
                 const float2 k2 = make_float2(kr[r], kr[r]), q2 = make_float2(qr[r], qr[r]);
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
+                for (int j = 0; j < CP; ++j) {
                     s[r][j] = __ffma2_rn(k2, d[j], s[r][j]);
-                    oc[r & 1][j] = __ffma2_rn(s[r][j], q2, oc[r & 1][j]);
+                    acc[r & 1][j] = __ffma2_rn(s[r][j], q2, acc[r & 1][j]);
                 }
             }
-            const float2 o01 = __fadd2_rn(oc[0][0], oc[1][0]), o23 = __fadd2_rn(oc[0][1], oc[1][1]);
-            const float ov = rowgroup_scatter4(make_float4(o01.x, o01.y, o23.x, o23.y));
-            if ((lane & 4) == 0) sm.vo[i][col + (lane >> 3)] = p.scale * ov;
+#pragma unroll
+            for (int j = 0; j < CP; ++j) {
+                const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
+                part[2 * j] = t.x; part[2 * j + 1] = t.y;
+            }
+            const float ov = rowgroup_scatter<CG>(part);
+            if (CG == 8 || (lane & 4) == 0) sm.vo[i][col + lane / VS] = p.scale * ov;
         }
         // the stretch's output rows, from shared memory
         __syncthreads();
@@ -233,8 +269,10 @@ __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(Chunk
     if (p.S_out) {
 #pragma unroll
         for (int r = 0; r < RP; ++r)
-            *reinterpret_cast<float4 *>(p.S_out + (nh * DK + rg * RP + r) * DV + col) =
-                make_float4(s[r][0].x, s[r][0].y, s[r][1].x, s[r][1].y);
+#pragma unroll
+            for (int j = 0; j < CP; j += 2)
+                *reinterpret_cast<float4 *>(p.S_out + (nh * DK + rg * RP + r) * DV + col + 2 * j) =
+                    make_float4(s[r][j].x, s[r][j].y, s[r][j + 1].x, s[r][j + 1].y);
     }
 }
 
