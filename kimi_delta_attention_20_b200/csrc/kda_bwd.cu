@@ -53,12 +53,14 @@ namespace cg = cooperative_groups;
 constexpr int kBwdThreads = 128;
 constexpr int kWarps = kBwdThreads / 32;
 constexpr int kCB = 16;   // tokens per checkpoint (one stretch)
-constexpr int kDVC = 16;  // value columns per CTA
+constexpr int kDVC = 32;  // value columns per CTA: 8 per warp
 
+// Lane (rg, cg) = (lane / 2, lane % 2) of warp w holds rows rg*RP .. rg*RP+RP-1 and
+// columns 8 w + 4 cg .. 8 w + 4 cg + 3 of its CTA's slice.
 template <int DK, int DV>
 struct BwdTile {
-    static constexpr int RP = DK / 32, NS = DV / kDVC;
-    static_assert(kWarps * 4 == kDVC && RP * 32 == DK && RP >= 1 && RP <= 4 && NS >= 1 && NS <= 8, "state tiling");
+    static constexpr int RP = DK / 16, NS = DV / kDVC;
+    static_assert(kWarps * 8 == kDVC && RP * 16 == DK && RP >= 2 && RP <= 8 && NS >= 1 && NS <= 8, "state tiling");
 };
 
 // Raw inputs of one stretch, copied in by cp.async while the previous stretch runs.
@@ -107,9 +109,12 @@ __device__ __forceinline__ long long first_ckpt(const BwdParams &p, int n) {
 
 template <int RP>
 __device__ __forceinline__ void load_rows(const float *src, float (&out)[RP]) {
-    if constexpr (RP == 4) {
-        const float4 x = *reinterpret_cast<const float4 *>(src);
-        out[0] = x.x; out[1] = x.y; out[2] = x.z; out[3] = x.w;
+    if constexpr (RP % 4 == 0) {
+#pragma unroll
+        for (int j = 0; j < RP; j += 4) {
+            const float4 x = *reinterpret_cast<const float4 *>(src + j);
+            out[j] = x.x; out[j + 1] = x.y; out[j + 2] = x.z; out[j + 3] = x.w;
+        }
     } else if constexpr (RP == 2) {
         const float2 x = *reinterpret_cast<const float2 *>(src);
         out[0] = x.x; out[1] = x.y;
@@ -131,53 +136,23 @@ __device__ __forceinline__ void store_rows(float *dst, const float (&x)[RP]) {
 
 __device__ __forceinline__ float dot4(float4 a, float4 b) { return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w; }
 
-// Warp all-reduce of 4 values: reduce-scatter over lane bits 4 and 3 (each lane
-// keeps half of its values at each step), butterfly over bits 2..0, then each
-// sum is gathered from the lanes that hold it (value v sits in lanes with
-// bits 4..3 = v). 10 shuffles instead of 20.
-__device__ __forceinline__ float4 warp_allreduce4(float4 x) {
-    const int lane = threadIdx.x & 31;
+// Sum of 4 column values over the 16 row groups of a warp (lane bits 4..1), returned
+// to every lane of the column group: reduce-scatter over bits 4 and 3 (each lane
+// keeps half of its values at each step), butterfly over bits 2 and 1, then each
+// sum is gathered from the lanes that hold it (value v sits in lanes with bits
+// 4..3 = v). 9 shuffles.
+__device__ __forceinline__ float4 colsum4(float4 x) {
+    const int lane = threadIdx.x & 31, cg = lane & 1;
     const bool h4 = lane & 16, h3 = lane & 8;
-    // bit 4: keep (z, w) or (x, y)
     float a0 = h4 ? x.z : x.x, a1 = h4 ? x.w : x.y;
-    const float s0 = h4 ? x.x : x.z, s1 = h4 ? x.y : x.w;
-    a0 += __shfl_xor_sync(0xffffffffu, s0, 16);
-    a1 += __shfl_xor_sync(0xffffffffu, s1, 16);
-    // bit 3: keep one of the two
+    a0 += __shfl_xor_sync(0xffffffffu, h4 ? x.x : x.z, 16);
+    a1 += __shfl_xor_sync(0xffffffffu, h4 ? x.y : x.w, 16);
     float m = h3 ? a1 : a0;
     m += __shfl_xor_sync(0xffffffffu, h3 ? a0 : a1, 8);
     m += __shfl_xor_sync(0xffffffffu, m, 4);
     m += __shfl_xor_sync(0xffffffffu, m, 2);
-    m += __shfl_xor_sync(0xffffffffu, m, 1);
-    return make_float4(__shfl_sync(0xffffffffu, m, 0), __shfl_sync(0xffffffffu, m, 8),
-                       __shfl_sync(0xffffffffu, m, 16), __shfl_sync(0xffffffffu, m, 24));
-}
-
-// Warp all-reduce of 8 values (x then y): reduce-scatter over lane bits 4, 3, 2,
-// butterfly over bits 1, 0, gather (value v sits in lanes with bits 4..2 = v).
-// 17 shuffles instead of 40.
-__device__ __forceinline__ void warp_allreduce8(float4 &x, float4 &y) {
-    const int lane = threadIdx.x & 31;
-    const bool h4 = lane & 16, h3 = lane & 8, h2 = lane & 4;
-    // bit 4: keep y (values 4..7) or x (values 0..3)
-    float a0 = h4 ? y.x : x.x, a1 = h4 ? y.y : x.y, a2 = h4 ? y.z : x.z, a3 = h4 ? y.w : x.w;
-    a0 += __shfl_xor_sync(0xffffffffu, h4 ? x.x : y.x, 16);
-    a1 += __shfl_xor_sync(0xffffffffu, h4 ? x.y : y.y, 16);
-    a2 += __shfl_xor_sync(0xffffffffu, h4 ? x.z : y.z, 16);
-    a3 += __shfl_xor_sync(0xffffffffu, h4 ? x.w : y.w, 16);
-    // bit 3: keep (a2, a3) or (a0, a1)
-    float b0 = h3 ? a2 : a0, b1 = h3 ? a3 : a1;
-    b0 += __shfl_xor_sync(0xffffffffu, h3 ? a0 : a2, 8);
-    b1 += __shfl_xor_sync(0xffffffffu, h3 ? a1 : a3, 8);
-    // bit 2: keep b1 or b0
-    float m = h2 ? b1 : b0;
-    m += __shfl_xor_sync(0xffffffffu, h2 ? b0 : b1, 4);
-    m += __shfl_xor_sync(0xffffffffu, m, 2);
-    m += __shfl_xor_sync(0xffffffffu, m, 1);
-    x = make_float4(__shfl_sync(0xffffffffu, m, 0), __shfl_sync(0xffffffffu, m, 4),
-                    __shfl_sync(0xffffffffu, m, 8), __shfl_sync(0xffffffffu, m, 12));
-    y = make_float4(__shfl_sync(0xffffffffu, m, 16), __shfl_sync(0xffffffffu, m, 20),
-                    __shfl_sync(0xffffffffu, m, 24), __shfl_sync(0xffffffffu, m, 28));
+    return make_float4(__shfl_sync(0xffffffffu, m, cg), __shfl_sync(0xffffffffu, m, 8 + cg),
+                       __shfl_sync(0xffffffffu, m, 16 + cg), __shfl_sync(0xffffffffu, m, 24 + cg));
 }
 
 // Start the copy of tokens [t0, t0 + cnt) of head h into the stage: k, g (and q
@@ -274,39 +249,39 @@ __device__ void take_stretch(const BwdParams &p, Sm &sm, int cnt, Tin beta_raw) 
     __syncthreads();
 }
 
-// One forward step of token i of the loaded stretch on this warp's register tile
-// s (rows lane*RP.., columns 4 warp .. 4 warp + 3 of the slice). Warp-local. With
-// keep_s, the decayed state S' = diag(a) S goes to keep_s[r * 128] (this thread's
-// slots) and u = S'^T k^ of the warp's columns to keep_u.
+// One forward step of token i of the loaded stretch on this lane's register tile s
+// (rows rg*RP.., slice columns 8 warp + 4 cg ..). Warp-local. With keep_s, the
+// decayed state S' = diag(a) S goes to keep_s[r * 128] (this thread's slots) and u =
+// S'^T k^ of the lane's columns to keep_u[0..3] (written by lanes 0 and 1).
 template <typename Tin, int DK, int DV>
 __device__ __forceinline__ void fwd_step(const FwdSmem<Tin, DK> &sm, int i, float4 (&s)[BwdTile<DK, DV>::RP],
                                          float4 *keep_s = nullptr, float *keep_u = nullptr) {
     constexpr int RP = BwdTile<DK, DV>::RP;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, rg = lane >> 1, cg = lane & 1;
     float kr[RP], ar[RP];
-    load_rows<RP>(&sm.kh[i][lane * RP], kr);
-    load_rows<RP>(&sm.al[i][lane * RP], ar);
-#pragma unroll
-    for (int r = 0; r < RP; ++r) ar[r] = fabsf(ar[r]);
+    load_rows<RP>(&sm.kh[i][rg * RP], kr);
+    load_rows<RP>(&sm.al[i][rg * RP], ar);
     const float b = sm.b[i];
-    const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][4 * warp]);
-    // decay and this lane's part of u on the paired fp32 FMA pipe
+    const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][8 * warp + 4 * cg]);
+    // decay and this lane's part of u on the paired fp32 FMA pipe (two chains)
     const float2 z2 = make_float2(0.f, 0.f);
-    float2 pu01 = z2, pu23 = z2;
+    float2 pu[2][2] = {{z2, z2}, {z2, z2}};
 #pragma unroll
     for (int r = 0; r < RP; ++r) {
-        const float2 a2 = make_float2(ar[r], ar[r]), k2 = make_float2(kr[r], kr[r]);
-        float2 lo = __fmul2_rn(make_float2(s[r].x, s[r].y), a2), hi = __fmul2_rn(make_float2(s[r].z, s[r].w), a2);
+        const float a = fabsf(ar[r]);
+        const float2 a2 = make_float2(a, a), k2 = make_float2(kr[r], kr[r]);
+        const float2 lo = __fmul2_rn(make_float2(s[r].x, s[r].y), a2), hi = __fmul2_rn(make_float2(s[r].z, s[r].w), a2);
         s[r] = make_float4(lo.x, lo.y, hi.x, hi.y);
-        pu01 = __ffma2_rn(lo, k2, pu01);
-        pu23 = __ffma2_rn(hi, k2, pu23);
+        pu[r & 1][0] = __ffma2_rn(lo, k2, pu[r & 1][0]);
+        pu[r & 1][1] = __ffma2_rn(hi, k2, pu[r & 1][1]);
     }
     if (keep_s) {
 #pragma unroll
         for (int r = 0; r < RP; ++r) keep_s[r * kBwdThreads] = s[r];
     }
-    const float4 u = warp_allreduce4(make_float4(pu01.x, pu01.y, pu23.x, pu23.y));
-    if (keep_u && lane == 0) *reinterpret_cast<float4 *>(keep_u) = u;
+    const float2 u01 = __fadd2_rn(pu[0][0], pu[1][0]), u23 = __fadd2_rn(pu[0][1], pu[1][1]);
+    const float4 u = colsum4(make_float4(u01.x, u01.y, u23.x, u23.y));
+    if (keep_u && lane < 2) *reinterpret_cast<float4 *>(keep_u + 4 * cg) = u;
     const float2 d01 = make_float2(b * (vv.x - u.x), b * (vv.y - u.y)), d23 = make_float2(b * (vv.z - u.z), b * (vv.w - u.w));
 #pragma unroll
     for (int r = 0; r < RP; ++r) {
@@ -317,22 +292,24 @@ __device__ __forceinline__ void fwd_step(const FwdSmem<Tin, DK> &sm, int i, floa
     }
 }
 
-// Element (row, slice column 4 warp) of a user [DK, DV] state whose slice starts at col0.
+// This lane's element (row, first of its 4 columns) of a user [DK, DV] state whose
+// CTA slice starts at col0.
 template <int DV>
-__device__ __forceinline__ float4 *state_ptr(float *base, int row, int col0, int warp) {
-    return reinterpret_cast<float4 *>(base + (long long)row * DV + col0 + 4 * warp);
+__device__ __forceinline__ float4 *state_ptr(float *base, int row, int col0) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    return reinterpret_cast<float4 *>(base + (long long)row * DV + col0 + 8 * warp + 4 * (lane & 1));
 }
 
 // Recompute of the forward, storing the entering state of tokens 0, kCB, 2 kCB, ...
 // (thread-major: checkpoint j of CTA slice r at ((j H + h) NS + r) RP 128 float4).
-// One CTA per (sequence, head, 16-column slice); no cross-CTA traffic.
+// One CTA per (sequence, head, 32-column slice); no cross-CTA traffic.
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kBwdThreads) kda_bwd_ckpt_kernel(BwdParams p) {
     using Tl = BwdTile<DK, DV>;
     constexpr int RP = Tl::RP, NS = Tl::NS;
     extern __shared__ __align__(16) uint8_t smraw[];
     FwdSmem<Tin, DK> &sm = *reinterpret_cast<FwdSmem<Tin, DK> *>(smraw);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, rg = (tid & 31) >> 1;
     const long long nh = blockIdx.x / NS;
     const int rank = (int)(blockIdx.x % NS), col0 = rank * kDVC;
     const int n = (int)(nh / p.H), h = (int)(nh % p.H);
@@ -340,7 +317,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_ckpt_kernel(BwdParams p) 
     float4 s[RP];
 #pragma unroll
     for (int r = 0; r < RP; ++r)
-        s[r] = p.S0 ? *state_ptr<DV>(const_cast<float *>(p.S0) + nh * DK * DV, lane * RP + r, col0, warp)
+        s[r] = p.S0 ? *state_ptr<DV>(const_cast<float *>(p.S0) + nh * DK * DV, rg * RP + r, col0)
                     : make_float4(0.f, 0.f, 0.f, 0.f);
     const long long c0 = first_ckpt(p, n);
     float4 *ckb = reinterpret_cast<float4 *>(p.ckpt);
@@ -361,7 +338,7 @@ __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 // Reverse sweep: one cluster of NS CTAs per (sequence, head), CTA rank r owning
-// value columns 16 r .. 16 r + 15, warp w of it columns 16 r + 4 w .. 16 r + 4 w + 3.
+// value columns 32 r .. 32 r + 31, warp w of it columns 32 r + 8 w .. 32 r + 8 w + 7.
 // Per stretch: take the staged tokens, start the copy of the stretch before,
 // rerun the stretch forward from its checkpoint keeping every token's decayed
 // state S' (in this CTA's scratch, thread-major) and u = S'^T k^, walk it back,
@@ -371,12 +348,13 @@ __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.w
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
     using Tl = BwdTile<DK, DV>;
-    constexpr int RP = Tl::RP, NS = Tl::NS;
+    constexpr int RP = Tl::RP, NS = Tl::NS, RH = RP / 2;
     extern __shared__ __align__(16) uint8_t smraw[];
     BwdSmem<Tin, DK> &sm = *reinterpret_cast<BwdSmem<Tin, DK> *>(smraw);
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, rg = lane >> 1, cgp = lane & 1;
+    const int cs0 = 8 * warp + 4 * cgp;  // this lane's first column within the CTA slice
     const long long nh = blockIdx.x / NS;
     const int col0 = rank * kDVC;
     const int n = (int)(nh / p.H), h = (int)(nh % p.H);
@@ -390,7 +368,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
     float4 ds[RP], s[RP];
 #pragma unroll
     for (int r = 0; r < RP; ++r)
-        ds[r] = p.dSf ? *state_ptr<DV>(const_cast<float *>(p.dSf) + nh * DK * DV, lane * RP + r, col0, warp)
+        ds[r] = p.dSf ? *state_ptr<DV>(const_cast<float *>(p.dSf) + nh * DK * DV, rg * RP + r, col0)
                       : make_float4(0.f, 0.f, 0.f, 0.f);
     int ph = 0;
     const long long len = eos - bos;
@@ -407,8 +385,8 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
         // forward from the checkpoint, keeping S' and u of every token
 #pragma unroll
         for (int r = 0; r < RP; ++r) s[r] = ck[r * kBwdThreads + tid];
-        for (int i = 0; i < cnt; ++i) fwd_step<Tin, DK, DV>(sm, i, s, scr + i * RP * kBwdThreads, &sm.u[i][4 * warp]);
-        __syncwarp();  // u of the warp's columns, written by lane 0, is read by all lanes
+        for (int i = 0; i < cnt; ++i) fwd_step<Tin, DK, DV>(sm, i, s, scr + i * RP * kBwdThreads, &sm.u[i][8 * warp]);
+        __syncwarp();  // u of the lane's columns, written by lanes 0 and 1, is read by all lanes
         if (cs != nst - 1) cluster_wait();  // every rank has added the previous stretch's terms
         float4 sp[RP];  // S' of the current token, fetched one token ahead
 #pragma unroll
@@ -421,18 +399,19 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
                 for (int r = 0; r < RP; ++r) sp[r] = scr[((i - 1) * RP + r) * kBwdThreads];
             }
             float kr[RP], ar[RP], qr[RP];
-            load_rows<RP>(&sm.kh[i][lane * RP], kr);
-            load_rows<RP>(&sm.al[i][lane * RP], ar);
-            load_rows<RP>(&sm.qh[i][lane * RP], qr);
+            load_rows<RP>(&sm.kh[i][rg * RP], kr);
+            load_rows<RP>(&sm.al[i][rg * RP], ar);
+            load_rows<RP>(&sm.qh[i][rg * RP], qr);
             const float b = sm.b[i];
-            const float4 dov = *reinterpret_cast<const float4 *>(&sm.dout[i][4 * warp]);
-            const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][4 * warp]);
-            const float4 u = *reinterpret_cast<const float4 *>(&sm.u[i][4 * warp]);
+            const float4 dov = *reinterpret_cast<const float4 *>(&sm.dout[i][cs0]);
+            const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][cs0]);
+            const float4 u = *reinterpret_cast<const float4 *>(&sm.u[i][cs0]);
 
-            // ---- dS += scale q^ do^T, then ddelta = dS^T k^ (warp sum); column pairs
-            // on the paired fp32 FMA pipe
+            // ---- dS += scale q^ do^T, then ddelta = dS^T k^ (column sums); column pairs on
+            // the paired fp32 FMA pipe, two chains
             const float2 do01 = make_float2(dov.x, dov.y), do23 = make_float2(dov.z, dov.w);
-            float2 dd01 = make_float2(0.f, 0.f), dd23 = dd01;
+            const float2 z2 = make_float2(0.f, 0.f);
+            float2 pd[2][2] = {{z2, z2}, {z2, z2}};
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
                 const float qs = p.scale * qr[r];
@@ -440,22 +419,25 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
                 const float2 lo = __ffma2_rn(qs2, do01, make_float2(ds[r].x, ds[r].y));
                 const float2 hi = __ffma2_rn(qs2, do23, make_float2(ds[r].z, ds[r].w));
                 ds[r] = make_float4(lo.x, lo.y, hi.x, hi.y);
-                dd01 = __ffma2_rn(lo, k2, dd01);
-                dd23 = __ffma2_rn(hi, k2, dd23);
+                pd[r & 1][0] = __ffma2_rn(lo, k2, pd[r & 1][0]);
+                pd[r & 1][1] = __ffma2_rn(hi, k2, pd[r & 1][1]);
             }
-            const float4 dd = warp_allreduce4(make_float4(dd01.x, dd01.y, dd23.x, dd23.y));
+            const float2 e01 = __fadd2_rn(pd[0][0], pd[1][0]), e23 = __fadd2_rn(pd[0][1], pd[1][1]);
+            const float4 dd = colsum4(make_float4(e01.x, e01.y, e23.x, e23.y));
             const float4 vu = make_float4(vv.x - u.x, vv.y - u.y, vv.z - u.z, vv.w - u.w);
             const float4 dl = make_float4(b * vu.x, b * vu.y, b * vu.z, b * vu.w);
-            if (lane < 4) {  // dv = b ddelta for this warp's columns, one per lane
-                const float x = lane == 0 ? dd.x : lane == 1 ? dd.y : lane == 2 ? dd.z : dd.w;
-                static_cast<Tin *>(p.dv)[((t0 + i) * H + h) * DV + col0 + 4 * warp + lane] = from_f32<Tin>(b * x);
+            if (lane < 2) {  // dv = b ddelta for this lane's columns
+                Tin *dv = static_cast<Tin *>(p.dv) + ((t0 + i) * H + h) * DV + col0 + cs0;
+                dv[0] = from_f32<Tin>(b * dd.x); dv[1] = from_f32<Tin>(b * dd.y);
+                dv[2] = from_f32<Tin>(b * dd.z); dv[3] = from_f32<Tin>(b * dd.w);
             }
-            // this warp's terms of delta . do and ddelta . (v - u)
-            const float ddo = dot4(dl, dov), db = dot4(dd, vu);
+            // this lane's terms of delta . do and ddelta . (v - u) (its 4 columns)
+            const float ddo = dot4(dl, dov);
+            float db = dot4(dd, vu);
 
-            // ---- this warp's terms of the row sums S' do, dS delta, S' ddelta, dS (.) S'
+            // ---- this lane's terms of the row sums S' do, dS delta, S' ddelta, dS (.) S'
             const float2 dl01 = make_float2(dl.x, dl.y), dl23 = make_float2(dl.z, dl.w);
-            const float2 dd01r = make_float2(dd.x, dd.y), dd23r = make_float2(dd.z, dd.w);
+            const float2 dd01 = make_float2(dd.x, dd.y), dd23 = make_float2(dd.z, dd.w);
             float tq[RP], tk[RP], tg[RP];
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
@@ -463,24 +445,38 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
                 const float2 g01 = make_float2(ds[r].x, ds[r].y), g23 = make_float2(ds[r].z, ds[r].w);
                 const float2 xa = __ffma2_rn(s23, do23, __fmul2_rn(s01, do01));
                 const float2 xb = __ffma2_rn(g23, dl23, __fmul2_rn(g01, dl01));
-                const float2 xe = __ffma2_rn(s23, dd23r, __fmul2_rn(s01, dd01r));
+                const float2 xe = __ffma2_rn(s23, dd23, __fmul2_rn(s01, dd01));
                 const float2 xh = __ffma2_rn(g23, s23, __fmul2_rn(g01, s01));
                 const float ra = xa.x + xa.y, rb = xb.x + xb.y, re = xe.x + xe.y, rh = xh.x + xh.y;
                 tq[r] = p.scale * fmaf(kr[r], ddo, ra);
                 tk[r] = fmaf(-b, re, rb);
                 tg[r] = ar[r] > 0.f ? fmaf(-b * kr[r], re, rh) : 0.f;
             }
-            store_rows<RP>(&sm.wp[ph][warp][0][lane * RP], tq);
-            store_rows<RP>(&sm.wp[ph][warp][1][lane * RP], tk);
-            store_rows<RP>(&sm.wp[ph][warp][2][lane * RP], tg);
+            // ---- the warp's terms: add the two column groups (lane bit 0), each lane keeping
+            // half of its rows (cg 0 the first RH, cg 1 the last RH)
+            float wq[RH], wk[RH], wg[RH];
+#pragma unroll
+            for (int j = 0; j < RH; ++j) {
+                const float kq = cgp ? tq[RH + j] : tq[j], sq = cgp ? tq[j] : tq[RH + j];
+                const float kk = cgp ? tk[RH + j] : tk[j], sk = cgp ? tk[j] : tk[RH + j];
+                const float kg = cgp ? tg[RH + j] : tg[j], sg = cgp ? tg[j] : tg[RH + j];
+                wq[j] = kq + __shfl_xor_sync(0xffffffffu, sq, 1);
+                wk[j] = kk + __shfl_xor_sync(0xffffffffu, sk, 1);
+                wg[j] = kg + __shfl_xor_sync(0xffffffffu, sg, 1);
+            }
+            db += __shfl_xor_sync(0xffffffffu, db, 1);
+            const int row0 = rg * RP + cgp * RH;
+            store_rows<RH>(&sm.wp[ph][warp][0][row0], wq);
+            store_rows<RH>(&sm.wp[ph][warp][1][row0], wk);
+            store_rows<RH>(&sm.wp[ph][warp][2][row0], wg);
             if (lane == 0) sm.wdb[ph][warp] = db;
             // ---- dS <- diag(a) (dS - b k^ ddelta^T), the cotangent of the entering state
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
                 const float nbk = -b * kr[r], a = fabsf(ar[r]);
                 const float2 nbk2 = make_float2(nbk, nbk), a2 = make_float2(a, a);
-                const float2 lo = __fmul2_rn(a2, __ffma2_rn(nbk2, dd01r, make_float2(ds[r].x, ds[r].y)));
-                const float2 hi = __fmul2_rn(a2, __ffma2_rn(nbk2, dd23r, make_float2(ds[r].z, ds[r].w)));
+                const float2 lo = __fmul2_rn(a2, __ffma2_rn(nbk2, dd01, make_float2(ds[r].x, ds[r].y)));
+                const float2 hi = __fmul2_rn(a2, __ffma2_rn(nbk2, dd23, make_float2(ds[r].z, ds[r].w)));
                 ds[r] = make_float4(lo.x, lo.y, hi.x, hi.y);
             }
             // ---- the CTA's terms of token i: the 4 warps' terms added in a fixed order
@@ -551,7 +547,7 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
     if (nst > 0) cluster_wait();
     if (p.dS0) {
 #pragma unroll
-        for (int r = 0; r < RP; ++r) *state_ptr<DV>(p.dS0 + nh * DK * DV, lane * RP + r, col0, warp) = ds[r];
+        for (int r = 0; r < RP; ++r) *state_ptr<DV>(p.dS0 + nh * DK * DV, rg * RP + r, col0) = ds[r];
     }
 }
 
