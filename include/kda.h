@@ -208,9 +208,9 @@ KDA_API kda_status kda_decode_token(const kda_token_args *args, void *stream);
  * g <- max(g, lower_bound), whose gradient is zero where the bound is taken, and
  * the sigmoid of beta). A recompute of the forward stores the state every 16
  * tokens; a reverse sweep then reruns each 16-token stretch forward from its
- * checkpoint (keeping the decayed states in an L2-resident scratch) and walks it back, each
- * (sequence, head) split by value columns over a cluster of Dv/16 CTAs; CUDA
- * cores, fp32. Validation as kda_chunk_fwd (q, k, v, g, dout and dq, dk, dv, dg
+ * checkpoint (keeping the decayed states in an L2-resident scratch) and walks it
+ * back, each (sequence, head) split by value columns over a cluster of Dv/32
+ * CTAs; CUDA cores, fp32. Validation as kda_chunk_fwd (q, k, v, g, dout and dq, dk, dv, dg
  * 16-byte aligned; beta and dbeta aligned to their element); g is the log-decay
  * (the in-kernel gate forms are not covered).
  */

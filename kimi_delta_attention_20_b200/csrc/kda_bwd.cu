@@ -19,17 +19,19 @@
 //
 // Column split. The value columns of S and of dS evolve independently (u, delta,
 // ddelta and the decay act column by column), so each (sequence, head) runs as a
-// cluster of Dv/16 CTAs, one per 16-column slice, and inside a CTA each warp owns
-// 4 columns over all Dk rows: lane l keeps rows l*RP .. l*RP+RP-1 of those
-// columns of S and of dS as float4 in registers. Key-axis sums (u, ddelta) are
-// warp reductions (no block barrier; the forward recompute needs none at all);
-// value-axis sums over a warp's columns are lane-local. What sums over the value
-// axis across warps and CTAs (dq^, dk^, dg, db) is linear in the per-warp terms:
-// the 4 warps' terms of a token meet in shared memory (one block barrier per
-// token), every CTA keeps its slice's terms for the kCB tokens of a stretch, and
-// after the stretch the cluster adds them across its CTAs through distributed
-// shared memory (a fixed rank order, so the result is deterministic) and applies
-// the L2-norm and sigmoid chain rules once per token.
+// cluster of Dv/32 CTAs, one per 32-column slice; inside a CTA each of the 4 warps
+// owns 8 columns over all Dk rows, and lane (rg, cg) = (lane / 2, lane % 2) keeps
+// rows rg*RP .. rg*RP+RP-1 (RP = Dk / 16) of columns 4 cg .. 4 cg + 3 of its warp's
+// block, of S and of dS, as column pairs for the paired fp32 FMA pipe. Key-axis
+// sums (u, ddelta) are reductions over the 16 row groups of a warp (no block
+// barrier; the forward recompute needs none at all); value-axis sums are lane-local
+// over 4 columns and then added across the 2 column groups of a warp. What sums
+// over the value axis across warps and CTAs (dq^, dk^, dg, db) is linear in the
+// per-warp terms: the 4 warps' terms of a token meet in shared memory (one block
+// barrier per token), every CTA keeps its slice's terms for the kCB tokens of a
+// stretch, and after the stretch the cluster adds them across its CTAs through
+// distributed shared memory (a fixed rank order, so the result is deterministic)
+// and applies the L2-norm and sigmoid chain rules once per token.
 //
 // The entering state of every token comes from a checkpoint written every kCB
 // tokens by a recompute of the forward (`kda_bwd_ckpt_kernel`): per stretch of kCB
