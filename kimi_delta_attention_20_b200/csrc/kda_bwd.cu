@@ -52,17 +52,18 @@ namespace {
 
 namespace cg = cooperative_groups;
 
-constexpr int kBwdThreads = 128;
-constexpr int kWarps = kBwdThreads / 32;
-constexpr int kCB = 16;   // tokens per checkpoint (one stretch)
-constexpr int kDVC = 32;  // value columns per CTA: 8 per warp
+constexpr int kGrp = 128;              // threads of one warp group; the checkpoint kernel is one group
+constexpr int kGW = kGrp / 32;         // warps per group
+constexpr int kRevThreads = 2 * kGrp;  // reverse sweep: a walking group and a preparing group
+constexpr int kCB = 16;                // tokens per checkpoint (one stretch)
+constexpr int kDVC = 32;               // value columns per CTA: 8 per warp of a group
 
-// Lane (rg, cg) = (lane / 2, lane % 2) of warp w holds rows rg*RP .. rg*RP+RP-1 and
-// columns 8 w + 4 cg .. 8 w + 4 cg + 3 of its CTA's slice.
+// Lane (rg, cg) = (lane / 2, lane % 2) of group warp w holds rows rg*RP .. rg*RP+RP-1
+// and columns 8 w + 4 cg .. 8 w + 4 cg + 3 of its CTA's slice.
 template <int DK, int DV>
 struct BwdTile {
     static constexpr int RP = DK / 16, NS = DV / kDVC;
-    static_assert(kWarps * 8 == kDVC && RP * 16 == DK && RP >= 2 && RP <= 8 && NS >= 1 && NS <= 8, "state tiling");
+    static_assert(kGW * 8 == kDVC && RP * 16 == DK && RP >= 2 && RP <= 8 && NS >= 1 && NS <= 8, "state tiling");
 };
 
 // Raw inputs of one stretch, copied in by cp.async while the previous stretch runs.
@@ -75,29 +76,51 @@ struct Stage {
 // Token vectors of one stretch (fp32; k^ normalised): what the forward recompute
 // needs. al holds the decay a = exp(max(g, lb)), negated where g < lb (the clamp
 // is taken there and the gate gets no gradient).
-template <typename Tin, int DK>
-struct FwdSmem {
-    Stage<Tin, DK> st;
+template <int DK>
+struct FwdVec {
     float kh[kCB][DK], al[kCB][DK];
     float v[kCB][kDVC];
     float b[kCB], rk[kCB];
 };
 
-// The reverse sweep adds q^, the output cotangent, u = S'^T k^ of every token of
-// the stretch (from its forward recompute), the per-warp terms of the current
-// token (alternating between tokens) and the per-CTA terms of dq^, dk^, dg
-// ([0], [1], [2]) and db of the stretch.
-template <typename Tin, int DK>
-struct BwdSmem : FwdSmem<Tin, DK> {
+// The reverse sweep adds q^, the output cotangent and u = S'^T k^ of every token
+// (from the stretch's forward recompute).
+template <int DK>
+struct RevVec : FwdVec<DK> {
     float qh[kCB][DK];
     float dout[kCB][kDVC];
     float u[kCB][kDVC];
     float rq[kCB];
-    float wp[2][kWarps][3][DK];
-    float wdb[2][kWarps];
+};
+
+template <typename Tin, int DK>
+struct CkptSmem {
+    Stage<Tin, DK> st;
+    FwdVec<DK> tv;
+};
+
+// Reverse sweep: two sets of token vectors (the walked stretch and the one being
+// prepared), the walking group's per-warp terms of the current token (alternating
+// between tokens), and the per-CTA terms of dq^, dk^, dg ([0], [1], [2]) and db of
+// the walked stretch.
+template <typename Tin, int DK>
+struct RevSmem {
+    Stage<Tin, DK> st;
+    RevVec<DK> tv[2];
+    float wp[2][kGW][3][DK];
+    float wdb[2][kGW];
     float pd[3][kCB][DK];
     float pdb[kCB];
 };
+
+// Thread and warp index within the thread's group of 128.
+__device__ __forceinline__ int gtid() { return threadIdx.x & (kGrp - 1); }
+__device__ __forceinline__ int gwarp() { return (threadIdx.x >> 5) & (kGW - 1); }
+// Barrier of the whole block (id 0) or of one group of 128 threads (named barrier id).
+__device__ __forceinline__ void grp_sync(int id) {
+    if (id == 0) __syncthreads();
+    else asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kGrp) : "memory");
+}
 
 __device__ __forceinline__ long long seq_begin(const BwdParams &p, int n) {
     return p.cu_seqlens ? (long long)p.cu_seqlens[n] : (long long)n * p.T;
@@ -159,23 +182,23 @@ __device__ __forceinline__ float4 colsum4(float4 x) {
 
 // Start the copy of tokens [t0, t0 + cnt) of head h into the stage: k, g (and q
 // for the reverse sweep) rows, and this CTA's columns of v (and of the output
-// cotangent), in 16-byte pieces. Returns this thread's raw beta (thread i < cnt
-// holds token i's), left unconverted so that its load completes in the
-// background like the copies.
+// cotangent), in 16-byte pieces, by the calling group. Returns this thread's raw
+// beta (thread i < cnt of the group holds token i's), left unconverted so that its
+// load completes in the background like the copies.
 template <typename Tin, int DK, int DV, bool kRev>
 __device__ __forceinline__ Tin issue_stretch(const BwdParams &p, Stage<Tin, DK> &st, long long t0, int cnt, int h,
                                              int col0) {
     constexpr int EP = 16 / (int)sizeof(Tin);  // elements per piece
     constexpr int RK = DK / EP, RV = kDVC / EP;
-    const int tid = threadIdx.x, H = p.H;
-    for (int e = tid; e < cnt * RK; e += kBwdThreads) {
+    const int tid = gtid(), H = p.H;
+    for (int e = tid; e < cnt * RK; e += kGrp) {
         const int i = e / RK, c = (e % RK) * EP;
         const long long gi = ((t0 + i) * H + h) * DK + c;
         cp_async16(&st.k[i][c], static_cast<const Tin *>(p.k) + gi);
         cp_async16(&st.g[i][c], static_cast<const Tin *>(p.g) + gi);
         if constexpr (kRev) cp_async16(&st.q[i][c], static_cast<const Tin *>(p.q) + gi);
     }
-    for (int e = tid; e < cnt * RV; e += kBwdThreads) {
+    for (int e = tid; e < cnt * RV; e += kGrp) {
         const int i = e / RV, c = (e % RV) * EP;
         const long long gi = ((t0 + i) * H + h) * DV + col0 + c;
         cp_async16(&st.v[i][c], static_cast<const Tin *>(p.v) + gi);
@@ -185,28 +208,28 @@ __device__ __forceinline__ Tin issue_stretch(const BwdParams &p, Stage<Tin, DK> 
     return tid < cnt ? static_cast<const Tin *>(p.beta)[(t0 + tid) * H + h] : Tin(0.f);
 }
 
-// Turn the staged stretch into the fp32 token vectors: k^ (and q^; normalised
+// Turn the staged stretch into the fp32 token vectors tv: k^ (and q^; normalised
 // when use_l2), the signed decay al, v (and the output cotangent), the write
-// strength b. Each key row is taken by 16 threads (DK / 16 elements each) that
-// form its squared norm with shuffles. The first barrier publishes the copies
-// and separates these writes from the previous stretch's last readers; on return
-// the vectors are complete and the stage is free for the next copy.
-template <typename Tin, int DK, bool kRev, typename Sm>
-__device__ void take_stretch(const BwdParams &p, Sm &sm, int cnt, Tin beta_raw) {
+// strength b. Each key row is taken by 16 threads (DK / 16 elements each) that form
+// its squared norm with shuffles. The first barrier (`bar`, the calling group's)
+// publishes the copies and separates these writes from earlier readers of tv; on
+// return the vectors are complete and the stage is free for the next copy.
+template <typename Tin, int DK, bool kRev, typename TV>
+__device__ void take_stretch(const BwdParams &p, Stage<Tin, DK> &st, TV &tv, int cnt, Tin beta_raw, int bar) {
     constexpr int TPR = 16, E = DK / TPR;
-    const int tid = threadIdx.x;
+    const int tid = gtid();
     cp_async_wait_all();
-    __syncthreads();
+    grp_sync(bar);
     const int c = (tid % TPR) * E;
     // uniform trip count: every lane joins the shuffles; rows past cnt read row 0
     // and store nothing
-    for (int i0 = 0; i0 < cnt; i0 += kBwdThreads / TPR) {
+    for (int i0 = 0; i0 < cnt; i0 += kGrp / TPR) {
         const int i = i0 + tid / TPR;
         const bool live = i < cnt;
         const int ir = live ? i : 0;
         float kx[E], gx[E];
-        stage_cvt<E>(&sm.st.k[ir][c], kx);
-        stage_cvt<E>(&sm.st.g[ir][c], gx);
+        stage_cvt<E>(&st.k[ir][c], kx);
+        stage_cvt<E>(&st.g[ir][c], gx);
         float kk = 0.f;
 #pragma unroll
         for (int e = 0; e < E; ++e) kk = fmaf(kx[e], kx[e], kk);
@@ -221,13 +244,13 @@ __device__ void take_stretch(const BwdParams &p, Sm &sm, int cnt, Tin beta_raw) 
             gx[e] = pass ? a : -a;
         }
         if (live) {
-            store_vec<E>(&sm.kh[i][c], kx);
-            store_vec<E>(&sm.al[i][c], gx);
-            if (tid % TPR == 0) sm.rk[i] = rk;
+            store_vec<E>(&tv.kh[i][c], kx);
+            store_vec<E>(&tv.al[i][c], gx);
+            if (tid % TPR == 0) tv.rk[i] = rk;
         }
         if constexpr (kRev) {
             float qx[E];
-            stage_cvt<E>(&sm.st.q[ir][c], qx);
+            stage_cvt<E>(&st.q[ir][c], qx);
             float qq = 0.f;
 #pragma unroll
             for (int e = 0; e < E; ++e) qq = fmaf(qx[e], qx[e], qq);
@@ -237,34 +260,34 @@ __device__ void take_stretch(const BwdParams &p, Sm &sm, int cnt, Tin beta_raw) 
 #pragma unroll
             for (int e = 0; e < E; ++e) qx[e] *= rq;
             if (live) {
-                store_vec<E>(&sm.qh[i][c], qx);
-                if (tid % TPR == 0) sm.rq[i] = rq;
+                store_vec<E>(&tv.qh[i][c], qx);
+                if (tid % TPR == 0) tv.rq[i] = rq;
             }
         }
     }
-    for (int e = tid; e < cnt * kDVC; e += kBwdThreads) {
+    for (int e = tid; e < cnt * kDVC; e += kGrp) {
         const int i = e / kDVC, cc = e % kDVC;
-        sm.v[i][cc] = to_f32(sm.st.v[i][cc]);
-        if constexpr (kRev) sm.dout[i][cc] = to_f32(sm.st.dout[i][cc]);
+        tv.v[i][cc] = to_f32(st.v[i][cc]);
+        if constexpr (kRev) tv.dout[i][cc] = to_f32(st.dout[i][cc]);
     }
-    if (tid < cnt) sm.b[tid] = beta_value(to_f32(beta_raw), p.beta_prob);
-    __syncthreads();
+    if (tid < cnt) tv.b[tid] = beta_value(to_f32(beta_raw), p.beta_prob);
+    grp_sync(bar);
 }
 
-// One forward step of token i of the loaded stretch on this lane's register tile s
-// (rows rg*RP.., slice columns 8 warp + 4 cg ..). Warp-local. With keep_s, the
-// decayed state S' = diag(a) S goes to keep_s[r * 128] (this thread's slots) and u =
-// S'^T k^ of the lane's columns to keep_u[0..3] (written by lanes 0 and 1).
-template <typename Tin, int DK, int DV>
-__device__ __forceinline__ void fwd_step(const FwdSmem<Tin, DK> &sm, int i, float4 (&s)[BwdTile<DK, DV>::RP],
+// One forward step of token i of the stretch in tv on this lane's register tile s
+// (rows rg*RP.., slice columns 8 w + 4 cg .. of group warp w). Warp-local. With
+// keep_s, the decayed state S' = diag(a) S goes to keep_s[r * 128] (this thread's
+// slots) and u = S'^T k^ of the lane's columns to keep_u[0..3] (lanes 0 and 1).
+template <typename Tin, int DK, int DV, typename TV>
+__device__ __forceinline__ void fwd_step(const TV &tv, int i, float4 (&s)[BwdTile<DK, DV>::RP],
                                          float4 *keep_s = nullptr, float *keep_u = nullptr) {
     constexpr int RP = BwdTile<DK, DV>::RP;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, rg = lane >> 1, cg = lane & 1;
+    const int lane = threadIdx.x & 31, warp = gwarp(), rg = lane >> 1, cg = lane & 1;
     float kr[RP], ar[RP];
-    load_rows<RP>(&sm.kh[i][rg * RP], kr);
-    load_rows<RP>(&sm.al[i][rg * RP], ar);
-    const float b = sm.b[i];
-    const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][8 * warp + 4 * cg]);
+    load_rows<RP>(&tv.kh[i][rg * RP], kr);
+    load_rows<RP>(&tv.al[i][rg * RP], ar);
+    const float b = tv.b[i];
+    const float4 vv = *reinterpret_cast<const float4 *>(&tv.v[i][8 * warp + 4 * cg]);
     // decay and this lane's part of u on the paired fp32 FMA pipe (two chains)
     const float2 z2 = make_float2(0.f, 0.f);
     float2 pu[2][2] = {{z2, z2}, {z2, z2}};
@@ -279,7 +302,7 @@ __device__ __forceinline__ void fwd_step(const FwdSmem<Tin, DK> &sm, int i, floa
     }
     if (keep_s) {
 #pragma unroll
-        for (int r = 0; r < RP; ++r) keep_s[r * kBwdThreads] = s[r];
+        for (int r = 0; r < RP; ++r) keep_s[r * kGrp] = s[r];
     }
     const float2 u01 = __fadd2_rn(pu[0][0], pu[1][0]), u23 = __fadd2_rn(pu[0][1], pu[1][1]);
     const float4 u = colsum4(make_float4(u01.x, u01.y, u23.x, u23.y));
@@ -298,19 +321,19 @@ __device__ __forceinline__ void fwd_step(const FwdSmem<Tin, DK> &sm, int i, floa
 // CTA slice starts at col0.
 template <int DV>
 __device__ __forceinline__ float4 *state_ptr(float *base, int row, int col0) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    return reinterpret_cast<float4 *>(base + (long long)row * DV + col0 + 8 * warp + 4 * (lane & 1));
+    const int lane = threadIdx.x & 31;
+    return reinterpret_cast<float4 *>(base + (long long)row * DV + col0 + 8 * gwarp() + 4 * (lane & 1));
 }
 
 // Recompute of the forward, storing the entering state of tokens 0, kCB, 2 kCB, ...
 // (thread-major: checkpoint j of CTA slice r at ((j H + h) NS + r) RP 128 float4).
-// One CTA per (sequence, head, 32-column slice); no cross-CTA traffic.
+// One CTA of 128 threads per (sequence, head, 32-column slice); no cross-CTA traffic.
 template <typename Tin, int DK, int DV>
-__global__ void __launch_bounds__(kBwdThreads) kda_bwd_ckpt_kernel(BwdParams p) {
+__global__ void __launch_bounds__(kGrp) kda_bwd_ckpt_kernel(BwdParams p) {
     using Tl = BwdTile<DK, DV>;
     constexpr int RP = Tl::RP, NS = Tl::NS;
     extern __shared__ __align__(16) uint8_t smraw[];
-    FwdSmem<Tin, DK> &sm = *reinterpret_cast<FwdSmem<Tin, DK> *>(smraw);
+    CkptSmem<Tin, DK> &sm = *reinterpret_cast<CkptSmem<Tin, DK> *>(smraw);
     const int tid = threadIdx.x, rg = (tid & 31) >> 1;
     const long long nh = blockIdx.x / NS;
     const int rank = (int)(blockIdx.x % NS), col0 = rank * kDVC;
@@ -327,12 +350,12 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_ckpt_kernel(BwdParams p) 
                          : Tin(0.f);
     for (long long t0 = bos; t0 < eos; t0 += kCB) {
         const int cnt = (int)min((long long)kCB, eos - t0);
-        float4 *ck = ckb + (((c0 + (t0 - bos) / kCB) * p.H + h) * NS + rank) * (RP * kBwdThreads);
+        float4 *ck = ckb + (((c0 + (t0 - bos) / kCB) * p.H + h) * NS + rank) * (RP * kGrp);
 #pragma unroll
-        for (int r = 0; r < RP; ++r) ck[r * kBwdThreads + tid] = s[r];
-        take_stretch<Tin, DK, false>(p, sm, cnt, braw);
+        for (int r = 0; r < RP; ++r) ck[r * kGrp + tid] = s[r];
+        take_stretch<Tin, DK, false>(p, sm.st, sm.tv, cnt, braw, 0);
         if (t0 + kCB < eos) braw = issue_stretch<Tin, DK, DV, false>(p, sm.st, t0 + kCB, (int)min((long long)kCB, eos - t0 - kCB), h, col0);
-        for (int i = 0; i < cnt; ++i) fwd_step<Tin, DK, DV>(sm, i, s);
+        for (int i = 0; i < cnt; ++i) fwd_step<Tin, DK, DV>(sm.tv, i, s);
     }
 }
 
@@ -340,23 +363,32 @@ __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 // Reverse sweep: one cluster of NS CTAs per (sequence, head), CTA rank r owning
-// value columns 32 r .. 32 r + 31, warp w of it columns 32 r + 8 w .. 32 r + 8 w + 7.
-// Per stretch: take the staged tokens, start the copy of the stretch before,
-// rerun the stretch forward from its checkpoint keeping every token's decayed
-// state S' (in this CTA's scratch, thread-major) and u = S'^T k^, walk it back,
-// then the cluster adds the slice terms. The cluster barrier that frees the
-// slice-term buffers for the next stretch is split: arrive after the adding,
-// wait just before the next walk writes them.
-template <typename Tin, int DK, int DV>
-__global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
+// value columns 32 r .. 32 r + 31. A CTA has two groups of 4 warps. The preparing
+// group (warps 4..7) takes in the next stretch to walk and reruns it forward from
+// its checkpoint, keeping every token's decayed state S' (a scratch buffer) and
+// u = S'^T k^ (its token vectors); meanwhile the walking group (warps 0..3) walks
+// the previous stretch back from the other buffer set. Iteration it prepares
+// stretch nst-1-it and walks stretch nst-it; the walking group then adds, with the
+// cluster, the slice terms of the stretch it walked at the start of the next
+// iteration. Cluster barriers: B (arrive and wait, all threads) at the start of an
+// iteration, after those adds, frees the slice-term buffers and the token vectors
+// that the adds read; A at the end, after a block barrier, publishes every rank's
+// terms of the walked stretch.
+// With kSplit false the CTA is one group of 128 threads that does both jobs in
+// turn (same order, same buffers): the form for grids of more than one CTA per SM,
+// where two such CTAs share an SM.
+template <typename Tin, int DK, int DV, bool kSplit>
+__global__ void __launch_bounds__(kSplit ? kRevThreads : kGrp) kda_bwd_kernel(BwdParams p) {
     using Tl = BwdTile<DK, DV>;
     constexpr int RP = Tl::RP, NS = Tl::NS, RH = RP / 2;
+    constexpr int kWalkBar = 1, kPrepBar = 2;
     extern __shared__ __align__(16) uint8_t smraw[];
-    BwdSmem<Tin, DK> &sm = *reinterpret_cast<BwdSmem<Tin, DK> *>(smraw);
+    RevSmem<Tin, DK> &sm = *reinterpret_cast<RevSmem<Tin, DK> *>(smraw);
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, rg = lane >> 1, cgp = lane & 1;
-    const int cs0 = 8 * warp + 4 * cgp;  // this lane's first column within the CTA slice
+    const bool walker = !kSplit || threadIdx.x < kGrp, preparer = !kSplit || threadIdx.x >= kGrp;
+    const int ltid = gtid(), lane = threadIdx.x & 31, lwarp = gwarp(), rg = lane >> 1, cgp = lane & 1;
+    const int cs0 = 8 * lwarp + 4 * cgp;  // this lane's first column within the CTA slice
     const long long nh = blockIdx.x / NS;
     const int col0 = rank * kDVC;
     const int n = (int)(nh / p.H), h = (int)(nh % p.H);
@@ -364,53 +396,110 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
     const long long bos = seq_begin(p, n), eos = seq_end(p, n);
     const long long c0 = first_ckpt(p, n);
     const float4 *ckb = reinterpret_cast<const float4 *>(p.ckpt);
-    // slot i, row part r of thread t at scr[(i RP + r) 128 + t]
-    float4 *scr = reinterpret_cast<float4 *>(p.scratch) + (long long)blockIdx.x * kCB * RP * kBwdThreads + tid;
-
-    float4 ds[RP], s[RP];
-#pragma unroll
-    for (int r = 0; r < RP; ++r)
-        ds[r] = p.dSf ? *state_ptr<DV>(const_cast<float *>(p.dSf) + nh * DK * DV, rg * RP + r, col0)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-    int ph = 0;
+    // two scratch buffers per CTA; slot i, row part r of group thread t at ((i RP + r) 128 + t)
+    float4 *scr = reinterpret_cast<float4 *>(p.scratch) + (long long)blockIdx.x * 2 * kCB * RP * kGrp + ltid;
     const long long len = eos - bos;
     const long long nst = (len + kCB - 1) / kCB;
-    Tin braw = nst > 0 ? issue_stretch<Tin, DK, DV, true>(p, sm.st, bos + (nst - 1) * kCB, (int)(len - (nst - 1) * kCB),
-                                                          h, col0)
-                       : Tin(0.f);
-    for (long long cs = nst - 1; cs >= 0; --cs) {
+
+    float4 ds[RP], s[RP];
+    if (walker) {
+#pragma unroll
+        for (int r = 0; r < RP; ++r)
+            ds[r] = p.dSf ? *state_ptr<DV>(const_cast<float *>(p.dSf) + nh * DK * DV, rg * RP + r, col0)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    Tin braw = Tin(0.f);
+    if (preparer && nst > 0)
+        braw = issue_stretch<Tin, DK, DV, true>(p, sm.st, bos + (nst - 1) * kCB, (int)(len - (nst - 1) * kCB), h, col0);
+
+    // the cluster's terms of the stretch walked last (buffer b): rank r finishes tokens
+    // r, r + NS, ... (group warp w takes every kGW-th of them)
+    auto finish_stretch = [&](long long cs, int b) {
+        const RevVec<DK> &tv = sm.tv[b];
         const long long t0 = bos + cs * kCB;
         const int cnt = (int)min((long long)kCB, eos - t0);
-        const float4 *ck = ckb + (((c0 + cs) * H + h) * NS + rank) * (RP * kBwdThreads);
-        take_stretch<Tin, DK, true>(p, sm, cnt, braw);
-        if (cs > 0) braw = issue_stretch<Tin, DK, DV, true>(p, sm.st, t0 - kCB, kCB, h, col0);
-        // forward from the checkpoint, keeping S' and u of every token
+        for (int i = rank + NS * lwarp; i < cnt; i += NS * kGW) {
+            constexpr int CP = DK / 32;  // channels per lane, contiguous: c0 .. c0 + CP - 1
+            const int cb = CP * lane;
+            float sq[CP], sk[CP], sg[CP], qv[CP], kv[CP];
 #pragma unroll
-        for (int r = 0; r < RP; ++r) s[r] = ck[r * kBwdThreads + tid];
-        for (int i = 0; i < cnt; ++i) fwd_step<Tin, DK, DV>(sm, i, s, scr + i * RP * kBwdThreads, &sm.u[i][8 * warp]);
-        __syncwarp();  // u of the lane's columns, written by lanes 0 and 1, is read by all lanes
-        if (cs != nst - 1) cluster_wait();  // every rank has added the previous stretch's terms
+            for (int j = 0; j < CP; ++j) { sq[j] = 0.f; sk[j] = 0.f; sg[j] = 0.f; }
+#pragma unroll
+            for (int q = 0; q < NS; ++q) {
+                const RevSmem<Tin, DK> *rs = cluster.map_shared_rank(&sm, q);
+                float x[CP], y[CP], z[CP];
+                load_rows<CP>(&rs->pd[0][i][cb], x);
+                load_rows<CP>(&rs->pd[1][i][cb], y);
+                load_rows<CP>(&rs->pd[2][i][cb], z);
+#pragma unroll
+                for (int j = 0; j < CP; ++j) { sq[j] += x[j]; sk[j] += y[j]; sg[j] += z[j]; }
+            }
+            load_rows<CP>(&tv.qh[i][cb], qv);
+            load_rows<CP>(&tv.kh[i][cb], kv);
+            float qd = 0.f, kd = 0.f;
+#pragma unroll
+            for (int j = 0; j < CP; ++j) { qd = fmaf(qv[j], sq[j], qd); kd = fmaf(kv[j], sk[j], kd); }
+            qd = p.use_l2 ? warp_sum(qd) : 0.f;
+            kd = p.use_l2 ? warp_sum(kd) : 0.f;
+            const float rq = tv.rq[i], rk = tv.rk[i];
+            const long long gi = ((t0 + i) * H + h) * DK + cb;
+#pragma unroll
+            for (int j = 0; j < CP; ++j) {
+                static_cast<Tin *>(p.dq)[gi + j] = from_f32<Tin>(rq * fmaf(-qv[j], qd, sq[j]));
+                static_cast<Tin *>(p.dk)[gi + j] = from_f32<Tin>(rk * fmaf(-kv[j], kd, sk[j]));
+                static_cast<Tin *>(p.dg)[gi + j] = from_f32<Tin>(sg[j]);
+            }
+            if (lane == 0) {
+                float db = 0.f;
+#pragma unroll
+                for (int q = 0; q < NS; ++q) db += cluster.map_shared_rank(&sm, q)->pdb[i];
+                const float b = tv.b[i];
+                static_cast<Tin *>(p.dbeta)[(t0 + i) * H + h] = from_f32<Tin>(p.beta_prob ? db : db * b * (1.f - b));
+            }
+        }
+    };
+
+    // prepare stretch cs into buffer b: intake, then the forward from its checkpoint
+    auto prepare = [&](long long cs, int b) {
+        const long long t0 = bos + cs * kCB;
+        const int cnt = (int)min((long long)kCB, eos - t0);
+        take_stretch<Tin, DK, true>(p, sm.st, sm.tv[b], cnt, braw, kPrepBar);
+        if (cs > 0) braw = issue_stretch<Tin, DK, DV, true>(p, sm.st, t0 - kCB, kCB, h, col0);
+        const float4 *ck = ckb + (((c0 + cs) * H + h) * NS + rank) * (RP * kGrp);
+#pragma unroll
+        for (int r = 0; r < RP; ++r) s[r] = ck[r * kGrp + ltid];
+        float4 *sb = scr + b * kCB * RP * kGrp;
+        for (int i = 0; i < cnt; ++i) fwd_step<Tin, DK, DV>(sm.tv[b], i, s, sb + i * RP * kGrp, &sm.tv[b].u[i][8 * lwarp]);
+    };
+
+    int ph = 0;  // alternates between the per-warp term buffers token by token
+    // walk stretch cs back from buffer b (the walking threads)
+    auto walk = [&](long long cs, int b) {
+        const RevVec<DK> &tv = sm.tv[b];
+        const long long t0 = bos + cs * kCB;
+        const int cnt = (int)min((long long)kCB, eos - t0);
+        const float4 *sb = scr + b * kCB * RP * kGrp;
         float4 sp[RP];  // S' of the current token, fetched one token ahead
 #pragma unroll
-        for (int r = 0; r < RP; ++r) sp[r] = scr[((cnt - 1) * RP + r) * kBwdThreads];
+        for (int r = 0; r < RP; ++r) sp[r] = sb[((cnt - 1) * RP + r) * kGrp];
         for (int i = cnt - 1; i >= 0; --i, ph ^= 1) {
 #pragma unroll
             for (int r = 0; r < RP; ++r) s[r] = sp[r];
             if (i > 0) {
 #pragma unroll
-                for (int r = 0; r < RP; ++r) sp[r] = scr[((i - 1) * RP + r) * kBwdThreads];
+                for (int r = 0; r < RP; ++r) sp[r] = sb[((i - 1) * RP + r) * kGrp];
             }
             float kr[RP], ar[RP], qr[RP];
-            load_rows<RP>(&sm.kh[i][rg * RP], kr);
-            load_rows<RP>(&sm.al[i][rg * RP], ar);
-            load_rows<RP>(&sm.qh[i][rg * RP], qr);
-            const float b = sm.b[i];
-            const float4 dov = *reinterpret_cast<const float4 *>(&sm.dout[i][cs0]);
-            const float4 vv = *reinterpret_cast<const float4 *>(&sm.v[i][cs0]);
-            const float4 u = *reinterpret_cast<const float4 *>(&sm.u[i][cs0]);
+            load_rows<RP>(&tv.kh[i][rg * RP], kr);
+            load_rows<RP>(&tv.al[i][rg * RP], ar);
+            load_rows<RP>(&tv.qh[i][rg * RP], qr);
+            const float bt = tv.b[i];
+            const float4 dov = *reinterpret_cast<const float4 *>(&tv.dout[i][cs0]);
+            const float4 vv = *reinterpret_cast<const float4 *>(&tv.v[i][cs0]);
+            const float4 u = *reinterpret_cast<const float4 *>(&tv.u[i][cs0]);
 
-            // ---- dS += scale q^ do^T, then ddelta = dS^T k^ (column sums); column pairs on
-            // the paired fp32 FMA pipe, two chains
+            // ---- dS += scale q^ do^T, then ddelta = dS^T k^ (column sums); column
+            // pairs on the paired fp32 FMA pipe, two chains
             const float2 do01 = make_float2(dov.x, dov.y), do23 = make_float2(dov.z, dov.w);
             const float2 z2 = make_float2(0.f, 0.f);
             float2 pd[2][2] = {{z2, z2}, {z2, z2}};
@@ -427,11 +516,11 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
             const float2 e01 = __fadd2_rn(pd[0][0], pd[1][0]), e23 = __fadd2_rn(pd[0][1], pd[1][1]);
             const float4 dd = colsum4(make_float4(e01.x, e01.y, e23.x, e23.y));
             const float4 vu = make_float4(vv.x - u.x, vv.y - u.y, vv.z - u.z, vv.w - u.w);
-            const float4 dl = make_float4(b * vu.x, b * vu.y, b * vu.z, b * vu.w);
+            const float4 dl = make_float4(bt * vu.x, bt * vu.y, bt * vu.z, bt * vu.w);
             if (lane < 2) {  // dv = b ddelta for this lane's columns
                 Tin *dv = static_cast<Tin *>(p.dv) + ((t0 + i) * H + h) * DV + col0 + cs0;
-                dv[0] = from_f32<Tin>(b * dd.x); dv[1] = from_f32<Tin>(b * dd.y);
-                dv[2] = from_f32<Tin>(b * dd.z); dv[3] = from_f32<Tin>(b * dd.w);
+                dv[0] = from_f32<Tin>(bt * dd.x); dv[1] = from_f32<Tin>(bt * dd.y);
+                dv[2] = from_f32<Tin>(bt * dd.z); dv[3] = from_f32<Tin>(bt * dd.w);
             }
             // this lane's terms of delta . do and ddelta . (v - u) (its 4 columns)
             const float ddo = dot4(dl, dov);
@@ -451,11 +540,11 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
                 const float2 xh = __ffma2_rn(g23, s23, __fmul2_rn(g01, s01));
                 const float ra = xa.x + xa.y, rb = xb.x + xb.y, re = xe.x + xe.y, rh = xh.x + xh.y;
                 tq[r] = p.scale * fmaf(kr[r], ddo, ra);
-                tk[r] = fmaf(-b, re, rb);
-                tg[r] = ar[r] > 0.f ? fmaf(-b * kr[r], re, rh) : 0.f;
+                tk[r] = fmaf(-bt, re, rb);
+                tg[r] = ar[r] > 0.f ? fmaf(-bt * kr[r], re, rh) : 0.f;
             }
-            // ---- the warp's terms: add the two column groups (lane bit 0), each lane keeping
-            // half of its rows (cg 0 the first RH, cg 1 the last RH)
+            // ---- the warp's terms: add the two column groups (lane bit 0), each lane
+            // keeping half of its rows (cg 0 the first RH, cg 1 the last RH)
             float wq[RH], wk[RH], wg[RH];
 #pragma unroll
             for (int j = 0; j < RH; ++j) {
@@ -468,86 +557,75 @@ __global__ void __launch_bounds__(kBwdThreads) kda_bwd_kernel(BwdParams p) {
             }
             db += __shfl_xor_sync(0xffffffffu, db, 1);
             const int row0 = rg * RP + cgp * RH;
-            store_rows<RH>(&sm.wp[ph][warp][0][row0], wq);
-            store_rows<RH>(&sm.wp[ph][warp][1][row0], wk);
-            store_rows<RH>(&sm.wp[ph][warp][2][row0], wg);
-            if (lane == 0) sm.wdb[ph][warp] = db;
+            store_rows<RH>(&sm.wp[ph][lwarp][0][row0], wq);
+            store_rows<RH>(&sm.wp[ph][lwarp][1][row0], wk);
+            store_rows<RH>(&sm.wp[ph][lwarp][2][row0], wg);
+            if (lane == 0) sm.wdb[ph][lwarp] = db;
             // ---- dS <- diag(a) (dS - b k^ ddelta^T), the cotangent of the entering state
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
-                const float nbk = -b * kr[r], a = fabsf(ar[r]);
+                const float nbk = -bt * kr[r], a = fabsf(ar[r]);
                 const float2 nbk2 = make_float2(nbk, nbk), a2 = make_float2(a, a);
                 const float2 lo = __fmul2_rn(a2, __ffma2_rn(nbk2, dd01, make_float2(ds[r].x, ds[r].y)));
                 const float2 hi = __fmul2_rn(a2, __ffma2_rn(nbk2, dd23, make_float2(ds[r].z, ds[r].w)));
                 ds[r] = make_float4(lo.x, lo.y, hi.x, hi.y);
             }
             // ---- the CTA's terms of token i: the 4 warps' terms added in a fixed order
-            __syncthreads();
+            grp_sync(kWalkBar);
             constexpr int Q4 = DK / 4;  // float4 per quantity row
-            if (tid < 3 * Q4) {
-                const int qn = tid / Q4, c = (tid % Q4) * 4;
+            if (ltid < 3 * Q4) {
+                const int qn = ltid / Q4, c = (ltid % Q4) * 4;
                 float4 acc = *reinterpret_cast<const float4 *>(&sm.wp[ph][0][qn][c]);
 #pragma unroll
-                for (int w = 1; w < kWarps; ++w) {
+                for (int w = 1; w < kGW; ++w) {
                     const float4 x = *reinterpret_cast<const float4 *>(&sm.wp[ph][w][qn][c]);
                     acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
                 }
                 *reinterpret_cast<float4 *>(&sm.pd[qn][i][c]) = acc;
-            } else if (tid == kBwdThreads - 1) {
+            } else if (ltid == kGrp - 1) {
                 float acc = sm.wdb[ph][0];
 #pragma unroll
-                for (int w = 1; w < kWarps; ++w) acc += sm.wdb[ph][w];
+                for (int w = 1; w < kGW; ++w) acc += sm.wdb[ph][w];
                 sm.pdb[i] = acc;
             }
         }
-        // ---- the stretch's slice terms are complete in every CTA of the cluster:
-        // rank r finishes tokens r, r + NS, ... (warp w takes every kWarps-th of them)
-        cluster_arrive();
-        cluster_wait();
-        for (int i = rank + NS * warp; i < cnt; i += NS * kWarps) {
-            constexpr int CP = DK / 32;  // channels per lane, contiguous: c0 .. c0 + CP - 1
-            const int c0 = CP * lane;
-            float sq[CP], sk[CP], sg[CP], qv[CP], kv[CP];
-#pragma unroll
-            for (int j = 0; j < CP; ++j) { sq[j] = 0.f; sk[j] = 0.f; sg[j] = 0.f; }
-#pragma unroll
-            for (int q = 0; q < NS; ++q) {
-                const BwdSmem<Tin, DK> *rs = cluster.map_shared_rank(&sm, q);
-                float x[CP], y[CP], z[CP];
-                load_rows<CP>(&rs->pd[0][i][c0], x);
-                load_rows<CP>(&rs->pd[1][i][c0], y);
-                load_rows<CP>(&rs->pd[2][i][c0], z);
-#pragma unroll
-                for (int j = 0; j < CP; ++j) { sq[j] += x[j]; sk[j] += y[j]; sg[j] += z[j]; }
+    };
+
+    if constexpr (kSplit) {
+        // iteration it prepares stretch nst-1-it and walks stretch nst-it
+        for (long long it = 0; it <= nst; ++it) {
+            if (walker) {
+                if (it >= 2) finish_stretch(nst - it + 1, (int)((it - 2) & 1));
+                cluster_arrive();  // B
+                cluster_wait();
+                if (it >= 1) walk(nst - it, (int)((it - 1) & 1));
+            } else {
+                cluster_arrive();  // B: the walking group's adds have read the token vectors
+                cluster_wait();
+                if (it < nst) prepare(nst - 1 - it, (int)(it & 1));
             }
-            load_rows<CP>(&sm.qh[i][c0], qv);
-            load_rows<CP>(&sm.kh[i][c0], kv);
-            float qd = 0.f, kd = 0.f;
-#pragma unroll
-            for (int j = 0; j < CP; ++j) { qd = fmaf(qv[j], sq[j], qd); kd = fmaf(kv[j], sk[j], kd); }
-            qd = p.use_l2 ? warp_sum(qd) : 0.f;
-            kd = p.use_l2 ? warp_sum(kd) : 0.f;
-            const float rq = sm.rq[i], rk = sm.rk[i];
-            const long long gi = ((t0 + i) * H + h) * DK + c0;
-#pragma unroll
-            for (int j = 0; j < CP; ++j) {
-                static_cast<Tin *>(p.dq)[gi + j] = from_f32<Tin>(rq * fmaf(-qv[j], qd, sq[j]));
-                static_cast<Tin *>(p.dk)[gi + j] = from_f32<Tin>(rk * fmaf(-kv[j], kd, sk[j]));
-                static_cast<Tin *>(p.dg)[gi + j] = from_f32<Tin>(sg[j]);
-            }
-            if (lane == 0) {
-                float db = 0.f;
-#pragma unroll
-                for (int q = 0; q < NS; ++q) db += cluster.map_shared_rank(&sm, q)->pdb[i];
-                const float b = sm.b[i];
-                static_cast<Tin *>(p.dbeta)[(t0 + i) * H + h] = from_f32<Tin>(p.beta_prob ? db : db * b * (1.f - b));
-            }
+            __syncthreads();
+            cluster_arrive();  // A: every rank's terms of the stretch walked in this iteration are complete
+            cluster_wait();
         }
-        cluster_arrive();  // this rank has read every rank's terms of the stretch
+        if (walker && nst >= 1) finish_stretch(0, (int)((nst - 1) & 1));
+    } else {
+        // one buffer set: prepare a stretch (overlapping the B wait), walk it, add its terms
+        for (long long cs = nst - 1; cs >= 0; --cs) {
+            prepare(cs, 0);
+            if (cs != nst - 1) cluster_wait();  // B: every rank has added the previous stretch's terms
+            walk(cs, 0);
+            cluster_arrive();  // A
+            cluster_wait();
+            finish_stretch(cs, 0);
+            cluster_arrive();  // B
+        }
+        if (nst > 0) cluster_wait();
     }
-    // no CTA leaves while another rank may still read its shared memory
-    if (nst > 0) cluster_wait();
-    if (p.dS0) {
+    // no CTA leaves while another may still read its shared memory
+    cluster_arrive();
+    cluster_wait();
+    if (walker && p.dS0) {
 #pragma unroll
         for (int r = 0; r < RP; ++r) *state_ptr<DV>(p.dS0 + nh * DK * DV, rg * RP + r, col0) = ds[r];
     }
@@ -570,22 +648,29 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st) {
     constexpr int NS = BwdTile<DK, DV>::NS;
     const long long heads = (long long)p.N * p.H;
     if (heads == 0) return cudaSuccess;
-    const int smem_f = (int)sizeof(FwdSmem<Tin, DK>), smem_b = (int)sizeof(BwdSmem<Tin, DK>);
-    static_assert(sizeof(BwdSmem<Tin, DK>) <= 232448, "shared memory of the reverse sweep");
+    const int smem_f = (int)sizeof(CkptSmem<Tin, DK>), smem_b = (int)sizeof(RevSmem<Tin, DK>);
+    static_assert(sizeof(RevSmem<Tin, DK>) <= 232448, "shared memory of the reverse sweep");
     cudaError_t e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    // one CTA per SM or fewer: walking and preparing groups side by side; more: one
+    // group doing both, two CTAs per SM
+    const bool split = heads * NS <= (long long)sms;
+    auto rev = split ? kda_bwd_kernel<Tin, DK, DV, true> : kda_bwd_kernel<Tin, DK, DV, false>;
     if ((e = cudaFuncSetAttribute(kda_bwd_ckpt_kernel<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_f)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(kda_bwd_kernel<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_b)) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(rev, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_b)) != cudaSuccess)
         return e;
     if (p.cu_seqlens) {
         kda_bwd_offsets<<<1, 32, 0, st>>>(p.cu_seqlens, p.N, p.ckpt_off);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    kda_bwd_ckpt_kernel<Tin, DK, DV><<<(unsigned)(heads * NS), kBwdThreads, smem_f, st>>>(p);
+    kda_bwd_ckpt_kernel<Tin, DK, DV><<<(unsigned)(heads * NS), kGrp, smem_f, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(heads * NS));
-    cfg.blockDim = dim3(kBwdThreads);
+    cfg.blockDim = dim3(split ? kRevThreads : kGrp);
     cfg.dynamicSmemBytes = (size_t)smem_b;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -595,7 +680,7 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kda_bwd_kernel<Tin, DK, DV>, p);
+    return cudaLaunchKernelEx(&cfg, rev, p);
 }
 
 template <typename Tin>
@@ -611,18 +696,18 @@ cudaError_t launch_bwd_dt(const BwdParams &p, int Dk, int Dv, cudaStream_t st) {
 
 }  // namespace
 
-// Workspace: [ckpt_off: N+1 ints, 256-byte block][per-CTA scratch: kCB states per head][checkpoints]
+// Workspace: [ckpt_off: N+1 ints, 256-byte block][per-CTA scratch: two stretches of states][checkpoints]
 size_t bwd_workspace_bytes(bool varlen, long long T, int N, int H, int Dk, int Dv) {
     const long long nck = varlen ? (T + kCB - 1) / kCB + N : (long long)N * ((T + kCB - 1) / kCB);
     const size_t head = (((size_t)(N + 1) * 4 + 255) / 256) * 256;
-    return head + (size_t)N * H * kCB * Dk * Dv * 4 + (size_t)nck * H * Dk * Dv * 4;
+    return head + 2 * (size_t)N * H * kCB * Dk * Dv * 4 + (size_t)nck * H * Dk * Dv * 4;
 }
 
 cudaError_t launch_bwd(BwdParams p, bool bf16, int Dk, int Dv, void *workspace, cudaStream_t st) {
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     p.ckpt_off = reinterpret_cast<int *>(ws);
     p.scratch = reinterpret_cast<float *>(ws + (((size_t)(p.N + 1) * 4 + 255) / 256) * 256);
-    p.ckpt = p.scratch + (size_t)p.N * p.H * kCB * Dk * Dv;
+    p.ckpt = p.scratch + 2 * (size_t)p.N * p.H * kCB * Dk * Dv;
     return bf16 ? launch_bwd_dt<__nv_bfloat16>(p, Dk, Dv, st) : launch_bwd_dt<float>(p, Dk, Dv, st);
 }
 

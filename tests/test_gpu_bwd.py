@@ -53,6 +53,15 @@ def test_backward_matches_oracle(dims, dtype):
     run_and_compare(inp, dtype, lower_bound=-5.0, tag=f"{dims}")
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_backward_many_heads(dtype):
+    """More CTAs than SMs (5 sequences x 8 heads x 4 column slices at d 128): the
+    reverse sweep then runs one warp group per CTA doing both of its jobs in turn;
+    fewer (the other tests) run the two groups side by side."""
+    inp = draw((33, 17, 1, 16, 40), 8, 128, 128, dtype, seed=97)
+    run_and_compare(inp, dtype, lower_bound=-5.0, tag="many heads")
+
+
 @pytest.mark.parametrize("case", ["no_final", "no_l2", "prob", "clamp_active", "empty_seqs"])
 def test_backward_options(case):
     dtype = torch.float32
