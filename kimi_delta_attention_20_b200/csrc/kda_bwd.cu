@@ -96,7 +96,7 @@ struct RevVec : FwdVec<DK> {
 template <typename Tin, int DK>
 struct CkptSmem {
     Stage<Tin, DK> st;
-    FwdVec<DK> tv;
+    FwdVec<DK> tv[2];
 };
 
 // Reverse sweep: two sets of token vectors (the walked stretch and the one being
@@ -327,35 +327,54 @@ __device__ __forceinline__ float4 *state_ptr(float *base, int row, int col0) {
 
 // Recompute of the forward, storing the entering state of tokens 0, kCB, 2 kCB, ...
 // (thread-major: checkpoint j of CTA slice r at ((j H + h) NS + r) RP 128 float4).
-// One CTA of 128 threads per (sequence, head, 32-column slice); no cross-CTA traffic.
+// One CTA of two warp groups per (sequence, head, 32-column slice), no cross-CTA
+// traffic: warps 0..3 step stretch j - 1 forward from one token-vector buffer while
+// warps 4..7 take stretch j into the other (and start the copy of stretch j + 1).
 template <typename Tin, int DK, int DV>
-__global__ void __launch_bounds__(kGrp) kda_bwd_ckpt_kernel(BwdParams p) {
+__global__ void __launch_bounds__(2 * kGrp) kda_bwd_ckpt_kernel(BwdParams p) {
     using Tl = BwdTile<DK, DV>;
     constexpr int RP = Tl::RP, NS = Tl::NS;
+    constexpr int kIntakeBar = 1;
     extern __shared__ __align__(16) uint8_t smraw[];
     CkptSmem<Tin, DK> &sm = *reinterpret_cast<CkptSmem<Tin, DK> *>(smraw);
-    const int tid = threadIdx.x, rg = (tid & 31) >> 1;
+    const bool stepper = threadIdx.x < kGrp;
+    const int ltid = gtid(), rg = (threadIdx.x & 31) >> 1;
     const long long nh = blockIdx.x / NS;
     const int rank = (int)(blockIdx.x % NS), col0 = rank * kDVC;
     const int n = (int)(nh / p.H), h = (int)(nh % p.H);
     const long long bos = seq_begin(p, n), eos = seq_end(p, n);
+    const long long nst = (eos - bos + kCB - 1) / kCB;
     float4 s[RP];
+    if (stepper) {
 #pragma unroll
-    for (int r = 0; r < RP; ++r)
-        s[r] = p.S0 ? *state_ptr<DV>(const_cast<float *>(p.S0) + nh * DK * DV, rg * RP + r, col0)
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = 0; r < RP; ++r)
+            s[r] = p.S0 ? *state_ptr<DV>(const_cast<float *>(p.S0) + nh * DK * DV, rg * RP + r, col0)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     const long long c0 = first_ckpt(p, n);
     float4 *ckb = reinterpret_cast<float4 *>(p.ckpt);
-    Tin braw = bos < eos ? issue_stretch<Tin, DK, DV, false>(p, sm.st, bos, (int)min((long long)kCB, eos - bos), h, col0)
-                         : Tin(0.f);
-    for (long long t0 = bos; t0 < eos; t0 += kCB) {
-        const int cnt = (int)min((long long)kCB, eos - t0);
-        float4 *ck = ckb + (((c0 + (t0 - bos) / kCB) * p.H + h) * NS + rank) * (RP * kGrp);
+    Tin braw = Tin(0.f);
+    if (!stepper && nst > 0)
+        braw = issue_stretch<Tin, DK, DV, false>(p, sm.st, bos, (int)min((long long)kCB, eos - bos), h, col0);
+    for (long long j = 0; j <= nst; ++j) {
+        if (stepper) {
+            if (j >= 1) {
+                const long long t0 = bos + (j - 1) * kCB;
+                const int cnt = (int)min((long long)kCB, eos - t0);
+                float4 *ck = ckb + (((c0 + j - 1) * p.H + h) * NS + rank) * (RP * kGrp);
 #pragma unroll
-        for (int r = 0; r < RP; ++r) ck[r * kGrp + tid] = s[r];
-        take_stretch<Tin, DK, false>(p, sm.st, sm.tv, cnt, braw, 0);
-        if (t0 + kCB < eos) braw = issue_stretch<Tin, DK, DV, false>(p, sm.st, t0 + kCB, (int)min((long long)kCB, eos - t0 - kCB), h, col0);
-        for (int i = 0; i < cnt; ++i) fwd_step<Tin, DK, DV>(sm.tv, i, s);
+                for (int r = 0; r < RP; ++r) ck[r * kGrp + ltid] = s[r];
+                const FwdVec<DK> &tv = sm.tv[(j - 1) & 1];
+                for (int i = 0; i < cnt; ++i) fwd_step<Tin, DK, DV>(tv, i, s);
+            }
+        } else if (j < nst) {
+            const long long t0 = bos + j * kCB;
+            const int cnt = (int)min((long long)kCB, eos - t0);
+            take_stretch<Tin, DK, false>(p, sm.st, sm.tv[j & 1], cnt, braw, kIntakeBar);
+            if (t0 + kCB < eos)
+                braw = issue_stretch<Tin, DK, DV, false>(p, sm.st, t0 + kCB, (int)min((long long)kCB, eos - t0 - kCB), h, col0);
+        }
+        __syncthreads();
     }
 }
 
@@ -666,7 +685,7 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st) {
         kda_bwd_offsets<<<1, 32, 0, st>>>(p.cu_seqlens, p.N, p.ckpt_off);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    kda_bwd_ckpt_kernel<Tin, DK, DV><<<(unsigned)(heads * NS), kGrp, smem_f, st>>>(p);
+    kda_bwd_ckpt_kernel<Tin, DK, DV><<<(unsigned)(heads * NS), 2 * kGrp, smem_f, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(heads * NS));
