@@ -34,12 +34,16 @@
 // and applies the L2-norm and sigmoid chain rules once per token.
 //
 // The entering state of every token comes from a checkpoint written every kCB
-// tokens by a recompute of the forward (`kda_bwd_ckpt_kernel`): per stretch of kCB
-// tokens the reverse sweep (`kda_bwd_kernel`) runs the forward once from the
-// checkpoint, keeping each token's decayed state S' = diag(a) S in a per-CTA
-// scratch (each thread stores and later reloads only its own tile; it stays in
-// L2) and u = S'^T k^ in shared memory, then walks the tokens back. Checkpoints
-// and scratch are thread-major per CTA (coalesced).
+// tokens by a recompute of the forward (`kda_bwd_ckpt_kernel`, one warp group
+// stepping while another takes in the next stretch). Per stretch of kCB tokens the
+// reverse sweep (`kda_bwd_kernel`) prepares the stretch (intake, then the forward
+// once from its checkpoint, keeping each token's decayed state S' = diag(a) S in
+// a per-CTA scratch that stays in L2 and u = S'^T k^ in shared memory), walks the
+// tokens back, and lets the cluster add the slice terms. When the grid has at most
+// one CTA per SM a CTA has two warp groups, one preparing the next stretch into a
+// second buffer set while the other walks the current one; otherwise one group
+// does both in turn and two CTAs share an SM. Checkpoints and scratch are
+// thread-major per CTA (coalesced).
 #include <cooperative_groups.h>
 
 #include "kda_common.cuh"
