@@ -56,7 +56,7 @@ namespace {
 
 namespace cg = cooperative_groups;
 
-constexpr int kGrp = 128;              // threads of one warp group; the checkpoint kernel is one group
+constexpr int kGrp = 128;              // threads of one warp group
 constexpr int kGW = kGrp / 32;         // warps per group
 constexpr int kRevThreads = 2 * kGrp;  // reverse sweep: a walking group and a preparing group
 constexpr int kCB = 16;                // tokens per checkpoint (one stretch)
