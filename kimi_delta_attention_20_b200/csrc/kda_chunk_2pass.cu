@@ -43,6 +43,7 @@
 #include "kda_common.cuh"
 #include "kda_sm100.cuh"
 #include "kda_tc_util.cuh"
+#include "kda_stage.cuh"
 
 namespace kda {
 namespace tp {
@@ -1252,18 +1253,18 @@ size_t queue_bytes(const ChunkParams &p) { return round1k((size_t)max_chunks(p) 
 
 }  // namespace tp
 
-size_t chunk_2pass_workspace_bytes(const ChunkParams &p) {
-    using namespace tp;
+namespace tp {
+
+size_t base_workspace_bytes(const ChunkParams &p) {
     return 1024 + 16384 + offsets_bytes(p) + table_bytes(p) + queue_bytes(p) + (size_t)max_chunks(p) * p.H * REC_BYTES;
 }
 
-cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int32_t *cu_host, cudaStream_t st) {
-    using namespace tp;
+// prep, pass 1 and the exact records of p into the workspace ws (its layout follows p)
+cudaError_t run_pass1(const ChunkParams &p, uint8_t *ws, cudaStream_t st) {
     const long long total = p.cu_seqlens ? (long long)p.T : (long long)p.N * p.T;
     if (total <= 0) return cudaErrorInvalidValue;
     const long long n_items = max_chunks(p) * p.H;
     if (n_items >= (1LL << 31) || total >= (1LL << 31)) return cudaErrorInvalidValue;
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *status = reinterpret_cast<int *>(ws);
     int *fix_count = reinterpret_cast<int *>(ws + 64);
     uint8_t *consts = ws + 1024;
@@ -1272,7 +1273,6 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     int2 *chunk_tok = reinterpret_cast<int2 *>(ws + base + offsets_bytes(p));
     int *fix_list = reinterpret_cast<int *>(ws + base + offsets_bytes(p) + table_bytes(p));
     uint8_t *rec = ws + base + offsets_bytes(p) + table_bytes(p) + queue_bytes(p);
-    const int cpr = (int)(((long long)p.T + C - 1) / C);
 
     static_assert(sizeof(IntraParams) <= 4096 && sizeof(StateParams) <= 4096, "kernel parameter blocks");
     IntraParams A;
@@ -1281,7 +1281,7 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     A.rec = rec;
     A.chunk_tok = p.cu_seqlens ? chunk_tok : nullptr;
     A.n_chunks = p.cu_seqlens ? chunk_off + p.N : nullptr;
-    A.cpr = cpr;
+    A.cpr = (int)(((long long)p.T + C - 1) / C);
     A.n_items = n_items;
     A.split_gate = (p.gate_mode == kGateLog && p.has_lb &&
                     __bfloat162float(__float2bfloat16_rn(p.lb)) != p.lb) ? 1 : 0;
@@ -1292,25 +1292,6 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     if (!make_map(&A.tq, p.q, total, p.H) || !make_map(&A.tk, p.k, total, p.H) ||
         !make_map(&A.tg, p.g, total, p.H))
         return cudaErrorInvalidValue;
-
-    StateParams B;
-    memset(&B, 0, sizeof(B));
-    B.p = p;
-    B.rec = rec;
-    B.chunk_off = p.cu_seqlens ? chunk_off : nullptr;
-    B.cpr = cpr;
-    B.status = status;
-    if (!make_map(&B.tv, p.v, total, p.H)) return cudaErrorInvalidValue;
-    B.nperm = 0;
-    if (cu_host && p.N <= kMaxPerm) {  // longest sequences first
-        std::vector<int> idx(p.N);
-        for (int i = 0; i < p.N; ++i) idx[i] = i;
-        std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) {
-            return (cu_host[a + 1] - cu_host[a]) > (cu_host[b + 1] - cu_host[b]);
-        });
-        for (int i = 0; i < p.N; ++i) B.perm[i] = idx[i];
-        B.nperm = p.N;
-    }
 
     cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
     if (e != cudaSuccess) return e;
@@ -1327,11 +1308,224 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     e = cudaFuncSetAttribute(kda_tp_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEMX_BYTES);
     if (e != cudaSuccess) return e;
     kda_tp_exact_kernel<<<(unsigned)std::min<long long>(n_items, nsm), NTX, SMEMX_BYTES, st>>>(A);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kda_tp_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2_ALLOC);
+    return cudaGetLastError();
+}
+
+// pass 2 of p (v, S0, S_out and o as p gives them) over the records in ws
+cudaError_t run_pass2(const ChunkParams &p, uint8_t *ws, const int32_t *cu_host, cudaStream_t st) {
+    const long long total = p.cu_seqlens ? (long long)p.T : (long long)p.N * p.T;
+    int *status = reinterpret_cast<int *>(ws);
+    const size_t base = 1024 + 16384;
+    int *chunk_off = reinterpret_cast<int *>(ws + base);
+    uint8_t *rec = ws + base + offsets_bytes(p) + table_bytes(p) + queue_bytes(p);
+    StateParams B;
+    memset(&B, 0, sizeof(B));
+    B.p = p;
+    B.rec = rec;
+    B.chunk_off = p.cu_seqlens ? chunk_off : nullptr;
+    B.cpr = (int)(((long long)p.T + C - 1) / C);
+    B.status = status;
+    if (!make_map(&B.tv, p.v, total, p.H)) return cudaErrorInvalidValue;
+    B.nperm = 0;
+    if (cu_host && p.N <= kMaxPerm) {  // longest sequences first
+        std::vector<int> idx(p.N);
+        for (int i = 0; i < p.N; ++i) idx[i] = i;
+        std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) {
+            return (cu_host[a + 1] - cu_host[a]) > (cu_host[b + 1] - cu_host[b]);
+        });
+        for (int i = 0; i < p.N; ++i) B.perm[i] = idx[i];
+        B.nperm = p.N;
+    }
+    cudaError_t e = cudaFuncSetAttribute(kda_tp_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2_ALLOC);
     if (e != cudaSuccess) return e;
     kda_tp_state_kernel<<<(unsigned)((long long)p.N * p.H), NT2, SMEM2_ALLOC, st>>>(B);
     return cudaGetLastError();
+}
+
+// ---- segments: with few (sequence, head) state chains, every sequence is cut into
+// P chunk-aligned segments whose chains run side by side. The state after a segment
+// is affine in the state before it, S_end = M S_start + N (the chunk update
+// S <- diag(e^{G_last}) S + Khat^T (U - W S) is affine in S), so pass 2 runs three
+// times over the segments: with v = 0 and S_start = I (its final states are the
+// M), with S_start = 0 (the N), and, once `kda_seg_chain` has walked the segments
+// of each sequence to their true entering states, with those states for the
+// outputs. Pass 1's records do not depend on the state and serve all three runs.
+constexpr int kMaxSeg = 16;
+constexpr int kChainSms = 148;  // chains wanted in flight: the SM count of the part
+
+int seg_count(const ChunkParams &p) {
+    const long long chains = (long long)p.N * p.H;
+    if (chains >= kChainSms) return 1;
+    const long long avg = p.cu_seqlens ? (long long)p.T / (p.N > 0 ? p.N : 1) : (long long)p.T;
+    long long P = std::min<long long>(kMaxSeg, kChainSms / chains);  // one wave of pass-2 CTAs (one per SM)
+    P = std::min<long long>(P, avg / (4 * C));  // at least four chunks per segment on average
+    return P < 2 ? 1 : (int)P;
+}
+
+// The segment view of p: P segments per sequence as a varlen batch.
+ChunkParams seg_view(const ChunkParams &p, int P, const int32_t *cu_v) {
+    ChunkParams q = p;
+    q.T = p.cu_seqlens ? p.T : p.N * p.T;  // total tokens (varlen convention)
+    q.N = p.N * P;
+    q.cu_seqlens = cu_v;
+    return q;
+}
+
+size_t seg_state_bytes(const ChunkParams &p, int P) { return round1k((size_t)p.N * P * p.H * 128 * 128 * 4); }
+size_t seg_tok_bytes(const ChunkParams &p, size_t esz) {
+    const long long total = p.cu_seqlens ? (long long)p.T : (long long)p.N * p.T;
+    return round1k((size_t)total * p.H * 128 * esz);
+}
+
+// cu_v[n P + s] = first token of segment s of sequence n (segment length: the
+// sequence's length / P rounded up to whole chunks; trailing segments may be empty)
+__global__ void kda_seg_setup(const int32_t *cu, int T, int N, int P, int32_t *cu_v) {
+    for (int n = blockIdx.x * blockDim.x + threadIdx.x; n < N; n += gridDim.x * blockDim.x) {
+        const long long bos = cu ? cu[n] : (long long)n * T, len = cu ? (long long)cu[n + 1] - cu[n] : T;
+        const long long L = ((len + P - 1) / P + C - 1) / C * C;
+        for (int sg = 0; sg < P; ++sg) cu_v[(long long)n * P + sg] = (int32_t)(bos + std::min<long long>(sg * L, len));
+        if (n == N - 1) cu_v[(long long)N * P] = (int32_t)(bos + len);
+    }
+}
+
+// count identity states [128][128]
+__global__ void kda_seg_identity(float *S, long long count) {
+    const long long total = count * 128 * 128;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
+        const int r = (int)((i >> 7) & 127), c = (int)(i & 127);
+        S[i] = r == c ? 1.f : 0.f;
+    }
+}
+
+// One CTA of 256 threads per (sequence, head, 16-column slice): walk the P segments of
+// the sequence, S_start(s) = S, S <- M_s S + N_s, from the caller's initial state
+// (or zero); the last S is the final state. M_s is staged in shared memory by
+// cp.async while the previous segment is applied (rows padded to 132 floats: 16-byte
+// aligned, and the 16 rows a warp reads at one k fall in 2-way shared banks).
+constexpr int kChainCols = 16, kChainSlices = 128 / kChainCols, kMLd = 132;
+struct SegChainSmem {
+    float4 sc[2][128][kChainCols / 4];  // the state slice (a warp reads one row at a time)
+    float m[2][128][kMLd];
+};
+
+__global__ void __launch_bounds__(256) kda_seg_chain(const float *S0, const float *M, const float *Nst, float *S_start,
+                                                     float *S_out, int N, int H, int P) {
+    extern __shared__ __align__(16) uint8_t smraw[];
+    SegChainSmem &sm = *reinterpret_cast<SegChainSmem *>(smraw);
+    const int tid = threadIdx.x;
+    const int slice = blockIdx.x % kChainSlices, nh = blockIdx.x / kChainSlices;
+    const int n = nh / H, h = nh % H, j0 = kChainCols * slice;
+    const int r = tid >> 1, c4 = (tid & 1) * 2;  // this thread: row r, slice columns 4 c4 .. 4 c4 + 7
+    auto stage_m = [&](int sg, int b) {  // start the copy of M_sg into buffer b
+        const float *src = M + (((long long)n * P + sg) * H + h) * 128 * 128;
+        for (int e = tid; e < 128 * 32; e += 256) cp_async16(&sm.m[b][e >> 5][(e & 31) * 4], src + (long long)e * 4);
+        cp_async_commit();
+    };
+    for (int e = tid; e < 128 * (kChainCols / 4); e += 256) {
+        const int rr = e / (kChainCols / 4), q = e % (kChainCols / 4);
+        sm.sc[0][rr][q] = S0 ? *reinterpret_cast<const float4 *>(S0 + ((long long)nh * 128 + rr) * 128 + j0 + 4 * q)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (P > 0) stage_m(0, 0);
+    int cur = 0;
+    for (int sg = 0; sg < P; ++sg) {
+        const long long vs = ((long long)n * P + sg) * H + h;  // virtual (segment, head) state index
+        cp_async_wait_all();
+        __syncthreads();  // M_sg and the current state are in shared memory; the other M buffer is free
+        if (sg + 1 < P) stage_m(sg + 1, (sg + 1) & 1);
+        const float (*m)[kMLd] = sm.m[sg & 1];
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+            *reinterpret_cast<float4 *>(S_start + (vs * 128 + r) * 128 + j0 + 4 * (c4 + q)) = sm.sc[cur][r][c4 + q];
+        float2 acc[4];
+        const float4 *nrow = reinterpret_cast<const float4 *>(Nst + (vs * 128 + r) * 128 + j0 + 4 * c4);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const float4 x = nrow[q];
+            acc[2 * q] = make_float2(x.x, x.y);
+            acc[2 * q + 1] = make_float2(x.z, x.w);
+        }
+#pragma unroll 8
+        for (int k = 0; k < 128; ++k) {
+            const float mv = m[r][k];
+            const float2 m2 = make_float2(mv, mv);
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const float4 x = sm.sc[cur][k][c4 + q];
+                acc[2 * q] = __ffma2_rn(m2, make_float2(x.x, x.y), acc[2 * q]);
+                acc[2 * q + 1] = __ffma2_rn(m2, make_float2(x.z, x.w), acc[2 * q + 1]);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+            sm.sc[cur ^ 1][r][c4 + q] = make_float4(acc[2 * q].x, acc[2 * q].y, acc[2 * q + 1].x, acc[2 * q + 1].y);
+        cur ^= 1;
+    }
+    __syncthreads();
+    if (S_out) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+            *reinterpret_cast<float4 *>(S_out + ((long long)nh * 128 + r) * 128 + j0 + 4 * (c4 + q)) = sm.sc[cur][r][c4 + q];
+    }
+}
+
+}  // namespace tp
+
+size_t chunk_2pass_workspace_bytes(const ChunkParams &p) {
+    using namespace tp;
+    const int P = seg_count(p);
+    if (P == 1) return base_workspace_bytes(p);
+    const ChunkParams q = seg_view(p, P, reinterpret_cast<const int32_t *>(16));  // only its presence is read
+    const size_t esz = 2;  // the two-pass path takes bf16 inputs
+    return base_workspace_bytes(q) + round1k(((size_t)p.N * P + 1) * 4) + 2 * seg_tok_bytes(p, esz) +
+           4 * seg_state_bytes(p, P);
+}
+
+cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int32_t *cu_host, cudaStream_t st) {
+    using namespace tp;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const int P = seg_count(p);
+    cudaError_t e;
+    if (P == 1) {
+        if ((e = run_pass1(p, ws, st)) != cudaSuccess) return e;
+        return run_pass2(p, ws, cu_host, st);
+    }
+    // workspace: [two-pass workspace of the segment view][cu_v][zero v][o scratch][I][M][N][S_start]
+    int32_t *cu_v = reinterpret_cast<int32_t *>(ws + base_workspace_bytes(seg_view(p, P, reinterpret_cast<const int32_t *>(16))));
+    const ChunkParams q = seg_view(p, P, cu_v);
+    uint8_t *cursor = reinterpret_cast<uint8_t *>(cu_v) + round1k(((size_t)p.N * P + 1) * 4);
+    void *zero_v = cursor;
+    cursor += seg_tok_bytes(p, 2);
+    void *o_scr = cursor;
+    cursor += seg_tok_bytes(p, 2);
+    float *Ibuf = reinterpret_cast<float *>(cursor);
+    cursor += seg_state_bytes(p, P);
+    float *Mbuf = reinterpret_cast<float *>(cursor);
+    cursor += seg_state_bytes(p, P);
+    float *Nbuf = reinterpret_cast<float *>(cursor);
+    cursor += seg_state_bytes(p, P);
+    float *Sbuf = reinterpret_cast<float *>(cursor);
+
+    kda_seg_setup<<<(p.N + 255) / 256, 256, 0, st>>>(p.cu_seqlens, p.T, p.N, P, cu_v);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(zero_v, 0, seg_tok_bytes(p, 2), st)) != cudaSuccess) return e;
+    kda_seg_identity<<<1024, 256, 0, st>>>(Ibuf, (long long)q.N * p.H);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = run_pass1(q, ws, st)) != cudaSuccess) return e;
+    ChunkParams pm = q;  // the transitions: v = 0 from the identity
+    pm.v = zero_v; pm.S0 = Ibuf; pm.S_out = Mbuf; pm.o = o_scr;
+    if ((e = run_pass2(pm, ws, nullptr, st)) != cudaSuccess) return e;
+    ChunkParams pn = q;  // the offsets: from zero
+    pn.S0 = nullptr; pn.S_out = Nbuf; pn.o = o_scr;
+    if ((e = run_pass2(pn, ws, nullptr, st)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(kda_seg_chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SegChainSmem))) != cudaSuccess)
+        return e;
+    kda_seg_chain<<<(unsigned)((long long)p.N * p.H * kChainSlices), 256, sizeof(SegChainSmem), st>>>(
+        p.S0, Mbuf, Nbuf, Sbuf, p.S_out, p.N, p.H, P);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ChunkParams pf = q;  // the outputs, from the true entering states
+    pf.S0 = Sbuf; pf.S_out = nullptr;
+    return run_pass2(pf, ws, nullptr, st);
 }
 
 }  // namespace kda

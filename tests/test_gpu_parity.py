@@ -87,6 +87,37 @@ def test_workload_varlen_H96():
     assert torch.isfinite(o).all() and torch.isfinite(S).all()
 
 
+@pytest.mark.parametrize("case", ["batch", "varlen", "gate_forms"])
+def test_segmented_state_chains(case):
+    """Few (sequence, head) chains and long sequences: the two-pass forward cuts every
+    sequence into chunk-aligned segments, runs pass 2 over them three times (transitions,
+    offsets, outputs) and chains the segment states in between. Ragged last segments,
+    an empty sequence and a one-chunk sequence (its trailing segments empty), initial
+    and final states."""
+    kw = dict(dtype=torch.bfloat16, init_state=True)
+    if case == "batch":
+        inp = KI.draw_chunk(2, 1100, 2, 128, 128, seed=120, **kw)
+        okw, lb = {}, -5.0
+    elif case == "varlen":
+        inp = KI.draw_chunk(1, 2264, 3, 128, 128, seed=121, seqlens=(700, 1500, 64, 0), **kw)
+        okw, lb = {}, None
+    else:
+        inp = KI.draw_chunk(1, 1400, 2, 128, 128, seed=122, gate="input", **kw)
+        inp.update(KI.draw_gate_params(2, 128, seed=122))
+        okw, lb = dict(gate_form="safe", A_log=inp["A_log"], dt_bias=inp["dt_bias"]), -5.0
+    if case == "gate_forms":
+        kda = kda_mod()
+        d = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        o, S = kda.chunk_kda(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=d["initial_state"],
+                             output_final_state=True, use_qk_l2norm_in_kernel=True, use_gate_in_kernel=True,
+                             safe_gate=True, lower_bound=lb, A_log=d["A_log"], dt_bias=d["dt_bias"])
+        sub = {k: v for k, v in inp.items() if k not in ("A_log", "dt_bias")}
+        compare_chunk(sub, o, S, torch.bfloat16, lower_bound=lb, tag="seg-gate", **okw)
+    else:
+        o, S = run_chunk(inp, lower_bound=lb)
+        compare_chunk(inp, o, S, torch.bfloat16, lower_bound=lb, tag=f"seg-{case}")
+
+
 def test_workload_300m_layer():
     """One layer of the 300M pure-KDA model (d_k 32, d_v 64, in-kernel gate, beta as a
     probability), full size; 6 of the 128 sequences checked on all 8 heads."""
