@@ -127,7 +127,14 @@ typedef struct {
  * tensor-core kernel, whose workspace holds one 65 KiB record per (chunk, head)
  * (about 1.04 bytes per input byte of q, k, g and v); a smaller workspace of at
  * least 256 bytes runs the single-pass tensor-core kernel instead (same result
- * up to rounding), and less than that returns KDA_ERR_WORKSPACE. */
+ * up to rounding), and less than that returns KDA_ERR_WORKSPACE.
+ * When there are few (sequence, head) pairs and the sequences are long, the size
+ * also covers cutting each sequence into segments whose states are chained
+ * afterwards (a few d_k x d_v fp32 states per segment and head, plus two
+ * scratch copies of the v rows); this applies to the two-pass kernel and, for
+ * d_k = d_v, to the token-recurrent kernel that the other shapes run, and a
+ * workspace too small for it runs the unsegmented kernel (same result up to
+ * rounding). */
 KDA_API kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args *args, size_t *bytes);
 
 /* Queue the chunkwise forward on `stream`. Returns KDA_OK once queued. */

@@ -10,7 +10,9 @@
 namespace kda {
 cudaError_t launch_decode(const StepParams &p, bool bf16, int Dk, int Dv, cudaStream_t st);
 cudaError_t launch_chunk_simt(const ChunkParams &p, bool bf16, int Dk, int Dv, int chunk, cudaStream_t st);
-cudaError_t launch_chunk_rec(const ChunkParams &p, bool bf16, int Dk, int Dv, cudaStream_t st);
+cudaError_t launch_chunk_rec(const ChunkParams &p, bool bf16, int Dk, int Dv, void *workspace, size_t workspace_bytes,
+                             cudaStream_t st);
+size_t chunk_rec_workspace_bytes(const ChunkParams &p, bool bf16, int Dk, int Dv);
 bool chunk_tc_supported(bool bf16, int Dk, int Dv, int chunk_size);
 size_t chunk_tc_workspace_bytes(int N, int H, int Dk, int Dv);
 cudaError_t launch_chunk_tc(const ChunkParams &p, int Dk, int Dv, void *workspace,
@@ -145,6 +147,11 @@ kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args *a, size_t *bytes) 
         p.cu_seqlens = a->cu_seqlens;  // only its presence is read
         p.T = a->T; p.N = N; p.H = a->H;
         *bytes = kda::chunk_2pass_workspace_bytes(p);
+    } else if (a->chunk_size != 32 && (long long)a->B * a->T > 0) {
+        kda::ChunkParams p{};
+        p.cu_seqlens = a->cu_seqlens;  // only its presence is read
+        p.T = a->T; p.N = N; p.H = a->H;
+        *bytes = kda::chunk_rec_workspace_bytes(p, a->dtype == KDA_DTYPE_BF16, a->Dk, a->Dv);
     }
     return KDA_OK;
 }
@@ -203,7 +210,7 @@ kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
     // other shapes: the register-resident recurrence; an explicit 32-token chunk
     // request runs the chunked CUDA-core kernel with C = 32 (same result)
     if (a->chunk_size == 32) return cuda_status(kda::launch_chunk_simt(p, bf16, a->Dk, a->Dv, 32, st));
-    return cuda_status(kda::launch_chunk_rec(p, bf16, a->Dk, a->Dv, st));
+    return cuda_status(kda::launch_chunk_rec(p, bf16, a->Dk, a->Dv, a->workspace, a->workspace_bytes, st));
 }
 
 kda_status kda_recurrent_step(const kda_step_args *a, void *stream) {

@@ -44,6 +44,7 @@
 #include "kda_sm100.cuh"
 #include "kda_tc_util.cuh"
 #include "kda_stage.cuh"
+#include "kda_seg.cuh"
 
 namespace kda {
 namespace tp {
@@ -1377,98 +1378,6 @@ size_t seg_tok_bytes(const ChunkParams &p, size_t esz) {
     return round1k((size_t)total * p.H * 128 * esz);
 }
 
-// cu_v[n P + s] = first token of segment s of sequence n (segment length: the
-// sequence's length / P rounded up to whole chunks; trailing segments may be empty)
-__global__ void kda_seg_setup(const int32_t *cu, int T, int N, int P, int32_t *cu_v) {
-    for (int n = blockIdx.x * blockDim.x + threadIdx.x; n < N; n += gridDim.x * blockDim.x) {
-        const long long bos = cu ? cu[n] : (long long)n * T, len = cu ? (long long)cu[n + 1] - cu[n] : T;
-        const long long L = ((len + P - 1) / P + C - 1) / C * C;
-        for (int sg = 0; sg < P; ++sg) cu_v[(long long)n * P + sg] = (int32_t)(bos + std::min<long long>(sg * L, len));
-        if (n == N - 1) cu_v[(long long)N * P] = (int32_t)(bos + len);
-    }
-}
-
-// count identity states [128][128]
-__global__ void kda_seg_identity(float *S, long long count) {
-    const long long total = count * 128 * 128;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
-        const int r = (int)((i >> 7) & 127), c = (int)(i & 127);
-        S[i] = r == c ? 1.f : 0.f;
-    }
-}
-
-// One CTA of 256 threads per (sequence, head, 16-column slice): walk the P segments of
-// the sequence, S_start(s) = S, S <- M_s S + N_s, from the caller's initial state
-// (or zero); the last S is the final state. M_s is staged in shared memory by
-// cp.async while the previous segment is applied (rows padded to 132 floats: 16-byte
-// aligned, and the 16 rows a warp reads at one k fall in 2-way shared banks).
-constexpr int kChainCols = 16, kChainSlices = 128 / kChainCols, kMLd = 132;
-struct SegChainSmem {
-    float4 sc[2][128][kChainCols / 4];  // the state slice (a warp reads one row at a time)
-    float m[2][128][kMLd];
-};
-
-__global__ void __launch_bounds__(256) kda_seg_chain(const float *S0, const float *M, const float *Nst, float *S_start,
-                                                     float *S_out, int N, int H, int P) {
-    extern __shared__ __align__(16) uint8_t smraw[];
-    SegChainSmem &sm = *reinterpret_cast<SegChainSmem *>(smraw);
-    const int tid = threadIdx.x;
-    const int slice = blockIdx.x % kChainSlices, nh = blockIdx.x / kChainSlices;
-    const int n = nh / H, h = nh % H, j0 = kChainCols * slice;
-    const int r = tid >> 1, c4 = (tid & 1) * 2;  // this thread: row r, slice columns 4 c4 .. 4 c4 + 7
-    auto stage_m = [&](int sg, int b) {  // start the copy of M_sg into buffer b
-        const float *src = M + (((long long)n * P + sg) * H + h) * 128 * 128;
-        for (int e = tid; e < 128 * 32; e += 256) cp_async16(&sm.m[b][e >> 5][(e & 31) * 4], src + (long long)e * 4);
-        cp_async_commit();
-    };
-    for (int e = tid; e < 128 * (kChainCols / 4); e += 256) {
-        const int rr = e / (kChainCols / 4), q = e % (kChainCols / 4);
-        sm.sc[0][rr][q] = S0 ? *reinterpret_cast<const float4 *>(S0 + ((long long)nh * 128 + rr) * 128 + j0 + 4 * q)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    if (P > 0) stage_m(0, 0);
-    int cur = 0;
-    for (int sg = 0; sg < P; ++sg) {
-        const long long vs = ((long long)n * P + sg) * H + h;  // virtual (segment, head) state index
-        cp_async_wait_all();
-        __syncthreads();  // M_sg and the current state are in shared memory; the other M buffer is free
-        if (sg + 1 < P) stage_m(sg + 1, (sg + 1) & 1);
-        const float (*m)[kMLd] = sm.m[sg & 1];
-#pragma unroll
-        for (int q = 0; q < 2; ++q)
-            *reinterpret_cast<float4 *>(S_start + (vs * 128 + r) * 128 + j0 + 4 * (c4 + q)) = sm.sc[cur][r][c4 + q];
-        float2 acc[4];
-        const float4 *nrow = reinterpret_cast<const float4 *>(Nst + (vs * 128 + r) * 128 + j0 + 4 * c4);
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const float4 x = nrow[q];
-            acc[2 * q] = make_float2(x.x, x.y);
-            acc[2 * q + 1] = make_float2(x.z, x.w);
-        }
-#pragma unroll 8
-        for (int k = 0; k < 128; ++k) {
-            const float mv = m[r][k];
-            const float2 m2 = make_float2(mv, mv);
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const float4 x = sm.sc[cur][k][c4 + q];
-                acc[2 * q] = __ffma2_rn(m2, make_float2(x.x, x.y), acc[2 * q]);
-                acc[2 * q + 1] = __ffma2_rn(m2, make_float2(x.z, x.w), acc[2 * q + 1]);
-            }
-        }
-#pragma unroll
-        for (int q = 0; q < 2; ++q)
-            sm.sc[cur ^ 1][r][c4 + q] = make_float4(acc[2 * q].x, acc[2 * q].y, acc[2 * q + 1].x, acc[2 * q + 1].y);
-        cur ^= 1;
-    }
-    __syncthreads();
-    if (S_out) {
-#pragma unroll
-        for (int q = 0; q < 2; ++q)
-            *reinterpret_cast<float4 *>(S_out + ((long long)nh * 128 + r) * 128 + j0 + 4 * (c4 + q)) = sm.sc[cur][r][c4 + q];
-    }
-}
-
 }  // namespace tp
 
 size_t chunk_2pass_workspace_bytes(const ChunkParams &p) {
@@ -1506,10 +1415,10 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     cursor += seg_state_bytes(p, P);
     float *Sbuf = reinterpret_cast<float *>(cursor);
 
-    kda_seg_setup<<<(p.N + 255) / 256, 256, 0, st>>>(p.cu_seqlens, p.T, p.N, P, cu_v);
+    kda_seg_setup<<<(p.N + 255) / 256, 256, 0, st>>>(p.cu_seqlens, p.T, p.N, P, C, cu_v);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaMemsetAsync(zero_v, 0, seg_tok_bytes(p, 2), st)) != cudaSuccess) return e;
-    kda_seg_identity<<<1024, 256, 0, st>>>(Ibuf, (long long)q.N * p.H);
+    kda_seg_identity<<<1024, 256, 0, st>>>(Ibuf, (long long)q.N * p.H, 128);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = run_pass1(q, ws, st)) != cudaSuccess) return e;
     ChunkParams pm = q;  // the transitions: v = 0 from the identity
@@ -1518,10 +1427,7 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     ChunkParams pn = q;  // the offsets: from zero
     pn.S0 = nullptr; pn.S_out = Nbuf; pn.o = o_scr;
     if ((e = run_pass2(pn, ws, nullptr, st)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(kda_seg_chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SegChainSmem))) != cudaSuccess)
-        return e;
-    kda_seg_chain<<<(unsigned)((long long)p.N * p.H * kChainSlices), 256, sizeof(SegChainSmem), st>>>(
-        p.S0, Mbuf, Nbuf, Sbuf, p.S_out, p.N, p.H, P);
+    if ((e = seg_chain_launch<128>(p.S0, Mbuf, Nbuf, Sbuf, p.S_out, p.N, p.H, P, st)) != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ChunkParams pf = q;  // the outputs, from the true entering states
     pf.S0 = Sbuf; pf.S_out = nullptr;

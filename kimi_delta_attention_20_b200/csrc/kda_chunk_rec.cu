@@ -19,8 +19,11 @@
 // stretch are copied by cp.async while the current one runs, turned into fp32
 // (L2 norms, gate, sigmoid) once per stretch, and the stretch's outputs leave
 // from shared memory as whole rows.
+#include <algorithm>
+
 #include "kda_common.cuh"
 #include "kda_stage.cuh"
+#include "kda_seg.cuh"
 
 namespace kda {
 
@@ -298,9 +301,92 @@ cudaError_t launch_rec_dt(const ChunkParams &p, int Dk, int Dv, cudaStream_t st)
     return cudaErrorInvalidValue;
 }
 
+// ---- segments (kda_seg.cuh): with few (sequence, head) chains, square states (the
+// transition M is d_k x d_k and is obtained as the final state from the identity)
+constexpr int kRecMaxSeg = 16;
+constexpr int kRecChains = 8 * 148;  // chains wanted in flight: several small CTAs per SM
+
+int rec_seg_count(const ChunkParams &p, int Dk, int Dv) {
+    if (Dk != Dv) return 1;
+    const long long chains = (long long)p.N * p.H;
+    if (chains <= 0 || chains * 2 > kRecChains) return 1;
+    const long long avg = p.cu_seqlens ? (long long)p.T / (p.N > 0 ? p.N : 1) : (long long)p.T;
+    long long P = std::min<long long>(kRecMaxSeg, kRecChains / chains);
+    P = std::min<long long>(P, avg / 64);  // at least 64 tokens per segment on average
+    return P < 2 ? 1 : (int)P;
+}
+
+size_t rk1(size_t b) { return (b + 1023) / 1024 * 1024; }
+
+struct RecSegLayout {
+    size_t cu, tok, state, total;
+};
+RecSegLayout rec_seg_layout(const ChunkParams &p, int P, int D, size_t esz) {
+    const long long total = p.cu_seqlens ? (long long)p.T : (long long)p.N * p.T;
+    RecSegLayout L;
+    L.cu = rk1(((size_t)p.N * P + 1) * 4);
+    L.tok = rk1((size_t)total * p.H * D * esz);
+    L.state = rk1((size_t)p.N * P * p.H * D * D * 4);
+    L.total = L.cu + 2 * L.tok + 4 * L.state;
+    return L;
+}
+
+template <typename Tin, int D>
+cudaError_t launch_rec_seg(const ChunkParams &p, int P, uint8_t *ws, cudaStream_t st) {
+    const RecSegLayout L = rec_seg_layout(p, P, D, sizeof(Tin));
+    int32_t *cu_v = reinterpret_cast<int32_t *>(ws);
+    void *zero_v = ws + L.cu;
+    void *o_scr = ws + L.cu + L.tok;
+    float *Ibuf = reinterpret_cast<float *>(ws + L.cu + 2 * L.tok);
+    float *Mbuf = Ibuf + L.state / 4;
+    float *Nbuf = Mbuf + L.state / 4;
+    float *Sbuf = Nbuf + L.state / 4;
+    ChunkParams q = p;  // the segment view: P segments per sequence as a varlen batch
+    q.T = p.cu_seqlens ? p.T : p.N * p.T;
+    q.N = p.N * P;
+    q.cu_seqlens = cu_v;
+    cudaError_t e;
+    kda_seg_setup<<<(p.N + 255) / 256, 256, 0, st>>>(p.cu_seqlens, p.T, p.N, P, 16, cu_v);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(zero_v, 0, L.tok, st)) != cudaSuccess) return e;
+    kda_seg_identity<<<512, 256, 0, st>>>(Ibuf, (long long)q.N * p.H, D);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ChunkParams pm = q;  // the transitions: v = 0 from the identity
+    pm.v = zero_v; pm.S0 = Ibuf; pm.S_out = Mbuf; pm.o = o_scr;
+    if ((e = launch_rec_t<Tin, D, D>(pm, st)) != cudaSuccess) return e;
+    ChunkParams pn = q;  // the offsets: from zero
+    pn.S0 = nullptr; pn.S_out = Nbuf; pn.o = o_scr;
+    if ((e = launch_rec_t<Tin, D, D>(pn, st)) != cudaSuccess) return e;
+    if ((e = seg_chain_launch<D>(p.S0, Mbuf, Nbuf, Sbuf, p.S_out, p.N, p.H, P, st)) != cudaSuccess) return e;
+    ChunkParams pf = q;  // the outputs, from the true entering states
+    pf.S0 = Sbuf; pf.S_out = nullptr;
+    return launch_rec_t<Tin, D, D>(pf, st);
+}
+
+template <typename Tin>
+cudaError_t launch_rec_seg_dt(const ChunkParams &p, int P, int D, uint8_t *ws, cudaStream_t st) {
+    if (D == 32) return launch_rec_seg<Tin, 32>(p, P, ws, st);
+    if (D == 64) return launch_rec_seg<Tin, 64>(p, P, ws, st);
+    if (D == 128) return launch_rec_seg<Tin, 128>(p, P, ws, st);
+    return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
-cudaError_t launch_chunk_rec(const ChunkParams &p, bool bf16, int Dk, int Dv, cudaStream_t st) {
+// Workspace the recurrent forward can use (0: it needs none).
+size_t chunk_rec_workspace_bytes(const ChunkParams &p, bool bf16, int Dk, int Dv) {
+    const int P = rec_seg_count(p, Dk, Dv);
+    return P < 2 ? 0 : rec_seg_layout(p, P, Dk, bf16 ? 2 : 4).total;
+}
+
+cudaError_t launch_chunk_rec(const ChunkParams &p, bool bf16, int Dk, int Dv, void *workspace, size_t workspace_bytes,
+                             cudaStream_t st) {
+    const int P = rec_seg_count(p, Dk, Dv);
+    if (P >= 2 && workspace && (reinterpret_cast<uintptr_t>(workspace) & 255) == 0 &&
+        workspace_bytes >= rec_seg_layout(p, P, Dk, bf16 ? 2 : 4).total) {
+        uint8_t *ws = static_cast<uint8_t *>(workspace);
+        return bf16 ? launch_rec_seg_dt<__nv_bfloat16>(p, P, Dk, ws, st) : launch_rec_seg_dt<float>(p, P, Dk, ws, st);
+    }
     return bf16 ? launch_rec_dt<__nv_bfloat16>(p, Dk, Dv, st) : launch_rec_dt<float>(p, Dk, Dv, st);
 }
 

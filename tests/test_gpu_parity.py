@@ -118,6 +118,26 @@ def test_segmented_state_chains(case):
         compare_chunk(inp, o, S, torch.bfloat16, lower_bound=lb, tag=f"seg-{case}")
 
 
+@pytest.mark.parametrize("case", ["d32_batch", "d64_varlen", "d32_fp32"])
+def test_segmented_recurrent(case):
+    """The recurrent forward (shapes without the tensor-core path) with few chains: every
+    sequence is cut into segments, the token recurrence runs over them three times
+    (transitions from the identity with v = 0, offsets from zero, outputs from the chained
+    entering states). Empty trailing segments, an empty sequence, initial states."""
+    if case == "d32_batch":
+        inp = KI.draw_chunk(2, 1100, 2, 32, 32, seed=130, dtype=torch.bfloat16, init_state=True)
+        lb, dt = -5.0, torch.bfloat16
+    elif case == "d64_varlen":
+        inp = KI.draw_chunk(1, 2264, 3, 64, 64, seed=131, dtype=torch.bfloat16, init_state=True,
+                            seqlens=(700, 1500, 64, 0))
+        lb, dt = None, torch.bfloat16
+    else:
+        inp = KI.draw_chunk(1, 3000, 1, 32, 32, seed=132, dtype=torch.float32, init_state=False)
+        lb, dt = None, torch.float32
+    o, S = run_chunk(inp, lower_bound=lb)
+    compare_chunk(inp, o, S, dt, lower_bound=lb, tag=f"rseg-{case}")
+
+
 def test_workload_300m_layer():
     """One layer of the 300M pure-KDA model (d_k 32, d_v 64, in-kernel gate, beta as a
     probability), full size; 6 of the 128 sequences checked on all 8 heads."""
