@@ -251,6 +251,8 @@ def run_kda(args, rank, world, local_rank):
     hbm_peak, tc_peak, peak_kind = load_peaks()
 
     wl = KI.CHUNK_WORKLOADS[args.workload if (args.only and args.workload is not None) else CHUNK_WL]
+    if args.only == "chunk" and args.chunk_heads:  # fewer heads for profiler captures
+        wl = dataclasses.replace(wl, H=args.chunk_heads, name=f"{wl.name} (H{args.chunk_heads})")
     if args.only in (None, "chunk"):  # the single-leg profiler runs allocate only their own leg
         inp = KI.chunk_inputs(wl, device=dev)
         q, k, v, g, beta = (inp[n] for n in ("q", "k", "v", "g", "beta"))
@@ -596,6 +598,8 @@ def main():
                     help="with --only bwd: sequence length of the backward workload (default 8192)")
     ap.add_argument("--workload", type=int, default=None,
                     help="with --only chunk: chunk workload index (default: the varlen H=96 one)")
+    ap.add_argument("--chunk-heads", type=int, default=None,
+                    help="with --only chunk: number of heads of the chunk workload (default: its own)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "kda":
         ap.error("--warmup must be >= 3")

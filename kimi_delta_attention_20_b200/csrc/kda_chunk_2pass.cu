@@ -1427,7 +1427,7 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     ChunkParams pn = q;  // the offsets: from zero
     pn.S0 = nullptr; pn.S_out = Nbuf; pn.o = o_scr;
     if ((e = run_pass2(pn, ws, nullptr, st)) != cudaSuccess) return e;
-    if ((e = seg_chain_launch<128>(p.S0, Mbuf, Nbuf, Sbuf, p.S_out, p.N, p.H, P, st)) != cudaSuccess) return e;
+    if ((e = seg_chain_launch<128>(p.S0, Mbuf, Nbuf, 128, 128LL * 128, Sbuf, p.S_out, p.N, p.H, P, st)) != cudaSuccess) return e;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ChunkParams pf = q;  // the outputs, from the true entering states
     pf.S0 = Sbuf; pf.S_out = nullptr;

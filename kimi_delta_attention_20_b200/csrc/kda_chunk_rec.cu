@@ -57,10 +57,11 @@ struct RecSmem {
 // Start the copy of tokens [t0, t0 + cnt) of head h; returns this thread's raw
 // beta (thread i < cnt holds token i's), left unconverted so that the load
 // completes in the background.
-template <typename Tin, int DK, int DV>
+template <typename Tin, int DK, int DV, bool AUG>
 __device__ __forceinline__ Tin rec_issue(const ChunkParams &p, RecSmem<Tin, DK, DV> &sm, long long t0, int cnt, int h) {
     constexpr int NT = RecCfg<DK, DV>::NT, EP = 16 / (int)sizeof(Tin);
-    constexpr int RK = DK / EP, RV = DV / EP;
+    constexpr int VOFF = AUG ? DK : 0, DVR = DV - VOFF;  // augmented: v occupies columns DK .. DV - 1
+    constexpr int RK = DK / EP, RV = DVR / EP;
     const int tid = threadIdx.x, H = p.H;
     for (int e = tid; e < cnt * RK; e += NT) {
         const int i = e / RK, c = (e % RK) * EP;
@@ -71,7 +72,7 @@ __device__ __forceinline__ Tin rec_issue(const ChunkParams &p, RecSmem<Tin, DK, 
     }
     for (int e = tid; e < cnt * RV; e += NT) {
         const int i = e / RV, c = (e % RV) * EP;
-        cp_async16(&sm.rv[i][c], static_cast<const Tin *>(p.v) + ((t0 + i) * H + h) * DV + c);
+        cp_async16(&sm.rv[i][VOFF + c], static_cast<const Tin *>(p.v) + ((t0 + i) * H + h) * DVR + c);
     }
     cp_async_commit();
     return tid < cnt ? static_cast<const Tin *>(p.beta)[(t0 + tid) * H + h] : Tin(0.f);
@@ -80,7 +81,7 @@ __device__ __forceinline__ Tin rec_issue(const ChunkParams &p, RecSmem<Tin, DK, 
 // The staged stretch as fp32 token vectors. Each key row is taken by TPR
 // threads that form its squared norms with shuffles (uniform trip count: rows
 // past cnt read row 0 and store nothing). Barriers on both sides.
-template <typename Tin, int DK, int DV>
+template <typename Tin, int DK, int DV, bool AUG>
 __device__ void rec_take(const ChunkParams &p, RecSmem<Tin, DK, DV> &sm, int cnt, Tin beta_raw, float rate) {
     using Cfg = RecCfg<DK, DV>;
     constexpr int NT = Cfg::NT, TPR = Cfg::TPR, E = Cfg::E;
@@ -119,7 +120,7 @@ __device__ void rec_take(const ChunkParams &p, RecSmem<Tin, DK, DV> &sm, int cnt
     }
     for (int e = tid; e < cnt * DV; e += NT) {
         const int i = e / DV, cc = e % DV;
-        sm.vo[i][cc] = to_f32(sm.rv[i][cc]);
+        sm.vo[i][cc] = (AUG && cc < DK) ? 0.f : to_f32(sm.rv[i][cc]);
     }
     if (tid < cnt) sm.b[tid] = beta_value(to_f32(beta_raw), p.beta_prob);
     __syncthreads();
@@ -158,7 +159,11 @@ __device__ __forceinline__ float rowgroup_scatter(const float (&x)[CG]) {
     return a[0];
 }
 
-template <typename Tin, int DK, int DV>
+// AUG: the augmented run of the segment form. Its state is [M | N] (d_k x (d_k + d_v)):
+// the first d_k columns start from the identity and see v = 0, the others start from
+// zero and see v; the outputs [scale M^T q^ | scale N^T q^] go out in fp32, rows of
+// d_k + d_v, and the final state as [d_k][d_k + d_v].
+template <typename Tin, int DK, int DV, bool AUG>
 __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(ChunkParams p) {
     using Cfg = RecCfg<DK, DV>;
     constexpr int RP = Cfg::RP, CT = Cfg::CT, NT = Cfg::NT, CG = Cfg::CG, CP = CG / 2;
@@ -184,17 +189,19 @@ __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(Chunk
     for (int r = 0; r < RP; ++r)
 #pragma unroll
         for (int j = 0; j < CP; j += 2) {
-            const float4 x = p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + (nh * DK + rg * RP + r) * DV + col + 2 * j)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            const int row = rg * RP + r, c0 = col + 2 * j;
+            const float4 x = AUG ? make_float4(row == c0, row == c0 + 1, row == c0 + 2, row == c0 + 3)
+                             : p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + (nh * DK + row) * DV + c0)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
             s[r][j] = make_float2(x.x, x.y);
             s[r][j + 1] = make_float2(x.z, x.w);
         }
 
-    Tin braw = bos < eos ? rec_issue<Tin, DK, DV>(p, sm, bos, (int)min((long long)CT, eos - bos), h) : Tin(0.f);
+    Tin braw = bos < eos ? rec_issue<Tin, DK, DV, AUG>(p, sm, bos, (int)min((long long)CT, eos - bos), h) : Tin(0.f);
     for (long long t0 = bos; t0 < eos; t0 += CT) {
         const int cnt = (int)min((long long)CT, eos - t0);
-        rec_take<Tin, DK, DV>(p, sm, cnt, braw, rate);
-        if (t0 + CT < eos) braw = rec_issue<Tin, DK, DV>(p, sm, t0 + CT, (int)min((long long)CT, eos - t0 - CT), h);
+        rec_take<Tin, DK, DV, AUG>(p, sm, cnt, braw, rate);
+        if (t0 + CT < eos) braw = rec_issue<Tin, DK, DV, AUG>(p, sm, t0 + CT, (int)min((long long)CT, eos - t0 - CT), h);
 #pragma unroll 2
         for (int i = 0; i < cnt; ++i) {
             float kr[RP], ar[RP], qr[RP];
@@ -264,9 +271,13 @@ __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(Chunk
         for (int e = 4 * tid; e < cnt * DV; e += 4 * NT) {
             const int i = e / DV, c = e % DV;
             const float4 x = *reinterpret_cast<const float4 *>(&sm.vo[i][c]);
-            Tin *dst = static_cast<Tin *>(p.o) + ((t0 + i) * H + h) * DV + c;
-            dst[0] = from_f32<Tin>(x.x); dst[1] = from_f32<Tin>(x.y);
-            dst[2] = from_f32<Tin>(x.z); dst[3] = from_f32<Tin>(x.w);
+            if constexpr (AUG) {
+                *reinterpret_cast<float4 *>(static_cast<float *>(p.o) + ((t0 + i) * H + h) * DV + c) = x;
+            } else {
+                Tin *dst = static_cast<Tin *>(p.o) + ((t0 + i) * H + h) * DV + c;
+                dst[0] = from_f32<Tin>(x.x); dst[1] = from_f32<Tin>(x.y);
+                dst[2] = from_f32<Tin>(x.z); dst[3] = from_f32<Tin>(x.w);
+            }
         }
     }
     if (p.S_out) {
@@ -279,14 +290,14 @@ __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(Chunk
     }
 }
 
-template <typename Tin, int DK, int DV>
+template <typename Tin, int DK, int DV, bool AUG = false>
 cudaError_t launch_rec_t(const ChunkParams &p, cudaStream_t st) {
     const long long blocks = (long long)p.N * p.H;
     if (blocks == 0) return cudaSuccess;
     const int smem = (int)sizeof(RecSmem<Tin, DK, DV>);
-    cudaError_t e = cudaFuncSetAttribute(kda_chunk_rec_kernel<Tin, DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(kda_chunk_rec_kernel<Tin, DK, DV, AUG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kda_chunk_rec_kernel<Tin, DK, DV><<<(unsigned)blocks, RecCfg<DK, DV>::NT, smem, st>>>(p);
+    kda_chunk_rec_kernel<Tin, DK, DV, AUG><<<(unsigned)blocks, RecCfg<DK, DV>::NT, smem, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -301,73 +312,152 @@ cudaError_t launch_rec_dt(const ChunkParams &p, int Dk, int Dv, cudaStream_t st)
     return cudaErrorInvalidValue;
 }
 
-// ---- segments (kda_seg.cuh): with few (sequence, head) chains, square states (the
-// transition M is d_k x d_k and is obtained as the final state from the identity)
+// ---- segments (kda_seg.cuh): with few (sequence, head) chains and square states, each
+// sequence is cut into P segments. One augmented launch runs every segment with the
+// state [M | N] (columns of S evolve independently, so the transition M, from the
+// identity with v = 0, and the offset N, from zero with v, are extra columns of one
+// state); it also writes w_t = scale M_t^T q^_t and scale N_t^T q^_t per token, M_t, N_t
+// being the maps up to token t within the segment. `kda_seg_chain` then walks the
+// segments to their entering states S_s, and since S_t = M_t S_s + N_t the outputs are
+// o_t = S_s^T w_t + scale N_t^T q^_t, a product per token with no sequential dependence.
 constexpr int kRecMaxSeg = 16;
 constexpr int kRecChains = 8 * 148;  // chains wanted in flight: several small CTAs per SM
 
 int rec_seg_count(const ChunkParams &p, int Dk, int Dv) {
-    if (Dk != Dv) return 1;
+    if (Dk != Dv || (Dk != 32 && Dk != 64)) return 1;
     const long long chains = (long long)p.N * p.H;
     if (chains <= 0 || chains * 2 > kRecChains) return 1;
     const long long avg = p.cu_seqlens ? (long long)p.T / (p.N > 0 ? p.N : 1) : (long long)p.T;
     long long P = std::min<long long>(kRecMaxSeg, kRecChains / chains);
     P = std::min<long long>(P, avg / 64);  // at least 64 tokens per segment on average
-    return P < 2 ? 1 : (int)P;
+    if (P < 2) return 1;
+    const long long seg_max = (((long long)p.T + P - 1) / P + 15) / 16 * 16;
+    return (seg_max + 31) / 32 > 65535 ? 1 : (int)P;  // the fixup grid's second dimension (32-token tiles)
 }
 
 size_t rk1(size_t b) { return (b + 1023) / 1024 * 1024; }
 
+// Tiles of kFixTok tokens in the longest segment: ceil(len / P) rounded up to 16 tokens,
+// len <= T (T is the tokens of a batch row, or the total of a varlen call)
+constexpr int kFixTok = 32;
+long long rec_fix_tiles(const ChunkParams &p, int P) {
+    const long long seg_max = (((long long)p.T + P - 1) / P + 15) / 16 * 16;
+    return (seg_max + kFixTok - 1) / kFixTok;
+}
+
 struct RecSegLayout {
-    size_t cu, tok, state, total;
+    size_t cu, oaug, saug, sstart, total;
 };
-RecSegLayout rec_seg_layout(const ChunkParams &p, int P, int D, size_t esz) {
+RecSegLayout rec_seg_layout(const ChunkParams &p, int P, int D) {
     const long long total = p.cu_seqlens ? (long long)p.T : (long long)p.N * p.T;
+    const size_t states = (size_t)p.N * P * p.H;
     RecSegLayout L;
-    L.cu = rk1(((size_t)p.N * P + 1) * 4);
-    L.tok = rk1((size_t)total * p.H * D * esz);
-    L.state = rk1((size_t)p.N * P * p.H * D * D * 4);
-    L.total = L.cu + 2 * L.tok + 4 * L.state;
+    L.cu = rk1((states / p.H + 1) * 4);
+    L.oaug = rk1((size_t)total * p.H * 2 * D * 4);
+    L.saug = rk1(states * D * 2 * D * 4);
+    L.sstart = rk1(states * D * D * 4);
+    L.total = L.cu + L.oaug + L.saug + L.sstart;
     return L;
+}
+
+__device__ __forceinline__ void store_o4(float *dst, float4 x) { *reinterpret_cast<float4 *>(dst) = x; }
+__device__ __forceinline__ void store_o4(__nv_bfloat16 *dst, float4 x) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y), b = __floats2bfloat162_rn(x.z, x.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t *>(&a);
+    u.y = *reinterpret_cast<uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(dst) = u;
+}
+
+// One CTA of 128 threads per (segment, head, 32-token tile): o_t = S_s^T w_t +
+// (scale N_t^T q^_t) for the tile's tokens, from the augmented outputs (rows
+// [w_t | scale N_t^T q^_t], fp32) and the entering state S_s (packed D x D). S_s and the
+// tile's w rows are copied into shared memory by cp.async while each thread loads its
+// offset terms; thread t then takes tokens t / (D / 4) + (128 / (D / 4)) i and 4 output
+// columns. Tiles past the segment's end exit at once (the grid covers the longest
+// segment any sequence can have).
+template <typename To, int D>
+__global__ void __launch_bounds__(128) kda_rec_seg_fixup(const float *oaug, const float *S_start, const int32_t *cu_v,
+                                                         To *o, int H) {
+    constexpr int NT = 128, Q = D / 4, TT = kFixTok, TPP = NT / Q, NTOK = TT / TPP, LW = D + 4;
+    __shared__ __align__(16) float S[D][D];
+    __shared__ __align__(16) float w[TT][LW];
+    const int v = blockIdx.x / H, h = blockIdx.x % H, tid = threadIdx.x;
+    const long long eos = cu_v[v + 1], t0 = cu_v[v] + (long long)blockIdx.y * TT;
+    if (t0 >= eos) return;
+    const int cnt = (int)min((long long)TT, eos - t0);
+    const float *Ss = S_start + (long long)blockIdx.x * D * D;  // state index v H + h
+    for (int e = tid; e < D * Q; e += NT) cp_async16(&S[e / Q][(e % Q) * 4], Ss + (long long)e * 4);
+    for (int e = tid; e < cnt * Q; e += NT) {
+        const int i = e / Q, k4 = (e % Q) * 4;
+        cp_async16(&w[i][k4], oaug + ((t0 + i) * H + h) * (2 * D) + k4);
+    }
+    cp_async_commit();
+    const int tb = tid / Q, c = (tid % Q) * 4;
+    float4 acc[NTOK];
+#pragma unroll
+    for (int i = 0; i < NTOK; ++i) {
+        const int ti = tb + TPP * i;
+        acc[i] = ti < cnt ? *reinterpret_cast<const float4 *>(oaug + ((t0 + ti) * H + h) * (2 * D) + D + c)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+#pragma unroll 2
+    for (int k = 0; k < D; k += 4) {
+        float4 sv[4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) sv[kk] = *reinterpret_cast<const float4 *>(&S[k + kk][c]);
+#pragma unroll
+        for (int i = 0; i < NTOK; ++i) {
+            const float4 wv = *reinterpret_cast<const float4 *>(&w[tb + TPP * i][k]);
+            const float wk[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                acc[i].x = fmaf(wk[kk], sv[kk].x, acc[i].x);
+                acc[i].y = fmaf(wk[kk], sv[kk].y, acc[i].y);
+                acc[i].z = fmaf(wk[kk], sv[kk].z, acc[i].z);
+                acc[i].w = fmaf(wk[kk], sv[kk].w, acc[i].w);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < NTOK; ++i) {
+        const int ti = tb + TPP * i;
+        if (ti < cnt) store_o4(o + ((t0 + ti) * H + h) * D + c, acc[i]);
+    }
 }
 
 template <typename Tin, int D>
 cudaError_t launch_rec_seg(const ChunkParams &p, int P, uint8_t *ws, cudaStream_t st) {
-    const RecSegLayout L = rec_seg_layout(p, P, D, sizeof(Tin));
+    const RecSegLayout L = rec_seg_layout(p, P, D);
     int32_t *cu_v = reinterpret_cast<int32_t *>(ws);
-    void *zero_v = ws + L.cu;
-    void *o_scr = ws + L.cu + L.tok;
-    float *Ibuf = reinterpret_cast<float *>(ws + L.cu + 2 * L.tok);
-    float *Mbuf = Ibuf + L.state / 4;
-    float *Nbuf = Mbuf + L.state / 4;
-    float *Sbuf = Nbuf + L.state / 4;
+    float *oaug = reinterpret_cast<float *>(ws + L.cu);
+    float *saug = reinterpret_cast<float *>(ws + L.cu + L.oaug);
+    float *sstart = reinterpret_cast<float *>(ws + L.cu + L.oaug + L.saug);
     ChunkParams q = p;  // the segment view: P segments per sequence as a varlen batch
     q.T = p.cu_seqlens ? p.T : p.N * p.T;
     q.N = p.N * P;
     q.cu_seqlens = cu_v;
+    q.S0 = nullptr;
+    q.S_out = saug;
+    q.o = oaug;
     cudaError_t e;
     kda_seg_setup<<<(p.N + 255) / 256, 256, 0, st>>>(p.cu_seqlens, p.T, p.N, P, 16, cu_v);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(zero_v, 0, L.tok, st)) != cudaSuccess) return e;
-    kda_seg_identity<<<512, 256, 0, st>>>(Ibuf, (long long)q.N * p.H, D);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    ChunkParams pm = q;  // the transitions: v = 0 from the identity
-    pm.v = zero_v; pm.S0 = Ibuf; pm.S_out = Mbuf; pm.o = o_scr;
-    if ((e = launch_rec_t<Tin, D, D>(pm, st)) != cudaSuccess) return e;
-    ChunkParams pn = q;  // the offsets: from zero
-    pn.S0 = nullptr; pn.S_out = Nbuf; pn.o = o_scr;
-    if ((e = launch_rec_t<Tin, D, D>(pn, st)) != cudaSuccess) return e;
-    if ((e = seg_chain_launch<D>(p.S0, Mbuf, Nbuf, Sbuf, p.S_out, p.N, p.H, P, st)) != cudaSuccess) return e;
-    ChunkParams pf = q;  // the outputs, from the true entering states
-    pf.S0 = Sbuf; pf.S_out = nullptr;
-    return launch_rec_t<Tin, D, D>(pf, st);
+    if ((e = launch_rec_t<Tin, D, 2 * D, true>(q, st)) != cudaSuccess) return e;
+    if ((e = seg_chain_launch<D>(p.S0, saug, saug + D, 2 * D, 2LL * D * D, sstart, p.S_out, p.N, p.H, P, st)) !=
+        cudaSuccess)
+        return e;
+    const dim3 fgrid((unsigned)((long long)q.N * p.H), (unsigned)rec_fix_tiles(p, P));
+    kda_rec_seg_fixup<Tin, D><<<fgrid, 128, 0, st>>>(oaug, sstart, cu_v, static_cast<Tin *>(p.o), p.H);
+    return cudaGetLastError();
 }
 
 template <typename Tin>
 cudaError_t launch_rec_seg_dt(const ChunkParams &p, int P, int D, uint8_t *ws, cudaStream_t st) {
     if (D == 32) return launch_rec_seg<Tin, 32>(p, P, ws, st);
     if (D == 64) return launch_rec_seg<Tin, 64>(p, P, ws, st);
-    if (D == 128) return launch_rec_seg<Tin, 128>(p, P, ws, st);
     return cudaErrorInvalidValue;
 }
 
@@ -376,14 +466,15 @@ cudaError_t launch_rec_seg_dt(const ChunkParams &p, int P, int D, uint8_t *ws, c
 // Workspace the recurrent forward can use (0: it needs none).
 size_t chunk_rec_workspace_bytes(const ChunkParams &p, bool bf16, int Dk, int Dv) {
     const int P = rec_seg_count(p, Dk, Dv);
-    return P < 2 ? 0 : rec_seg_layout(p, P, Dk, bf16 ? 2 : 4).total;
+    (void)bf16;
+    return P < 2 ? 0 : rec_seg_layout(p, P, Dk).total;
 }
 
 cudaError_t launch_chunk_rec(const ChunkParams &p, bool bf16, int Dk, int Dv, void *workspace, size_t workspace_bytes,
                              cudaStream_t st) {
     const int P = rec_seg_count(p, Dk, Dv);
     if (P >= 2 && workspace && (reinterpret_cast<uintptr_t>(workspace) & 255) == 0 &&
-        workspace_bytes >= rec_seg_layout(p, P, Dk, bf16 ? 2 : 4).total) {
+        workspace_bytes >= rec_seg_layout(p, P, Dk).total) {
         uint8_t *ws = static_cast<uint8_t *>(workspace);
         return bf16 ? launch_rec_seg_dt<__nv_bfloat16>(p, P, Dk, ws, st) : launch_rec_seg_dt<float>(p, P, Dk, ws, st);
     }

@@ -121,9 +121,10 @@ def test_segmented_state_chains(case):
 @pytest.mark.parametrize("case", ["d32_batch", "d64_varlen", "d32_fp32"])
 def test_segmented_recurrent(case):
     """The recurrent forward (shapes without the tensor-core path) with few chains: every
-    sequence is cut into segments, the token recurrence runs over them three times
-    (transitions from the identity with v = 0, offsets from zero, outputs from the chained
-    entering states). Empty trailing segments, an empty sequence, initial states."""
+    sequence is cut into segments, one run of the token recurrence over them carries the
+    transition (from the identity, v = 0) and the offset (from zero) as one widened state,
+    the segment states are chained, and the outputs are fixed up from the entering states.
+    Empty trailing segments, an empty sequence, initial states."""
     if case == "d32_batch":
         inp = KI.draw_chunk(2, 1100, 2, 32, 32, seed=130, dtype=torch.bfloat16, init_state=True)
         lb, dt = -5.0, torch.bfloat16
