@@ -942,6 +942,8 @@ struct StateParams {
     const int *chunk_off;
     int cpr;
     int *status;
+    int s0_identity;  // start every chain from the identity (S0 is not read)
+    int v_zero;       // v = 0: no v tiles are copied (tv is not read) and the stage's v area stays zero
     int nperm;
     int perm[kMaxPerm];
 };
@@ -973,7 +975,12 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
         for (int i = 0; i < 6; ++i) mbar_init(bar_full + i, 1);
         mbar_init(bar_of, kGroup); mbar_init(bar_of + 1, kGroup);
         fence_mbar_init();
-        tma_prefetch_desc(&P.tv);
+        if (!P.v_zero) tma_prefetch_desc(&P.tv);
+    }
+    if (P.v_zero) {  // the v areas of both stages, read by the products as zeros
+        for (int e = tid; e < 2 * 1024; e += NT2)
+            sts128(sm, (e >> 10) * STAGE_BYTES + S_V + (e & 1023) * 16, make_uint4(0u, 0u, 0u, 0u));
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -996,10 +1003,11 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
         const int s = ci & 1;
         uint8_t *dst = sm + s * STAGE_BYTES;
         const uint8_t *src = P.rec + ((c_first + ci) * H + h) * (long long)REC_BYTES;
-        mbar_arrive_expect_tx(bar_full + s, STAGE_BYTES);
+        mbar_arrive_expect_tx(bar_full + s, P.v_zero ? REC_BYTES : STAGE_BYTES);
         bulk_load(dst, src, REC_BYTES, bar_full + s);
         const int t = (int)(bos + (long long)ci * C);
-        for (int hf = 0; hf < 2; ++hf) tma_load_3d(dst + S_V + hf * 8192, &P.tv, bar_full + s, hf * 64, h, t);
+        if (!P.v_zero)
+            for (int hf = 0; hf < 2; ++hf) tma_load_3d(dst + S_V + hf * 8192, &P.tv, bar_full + s, hf * 64, h, t);
         full_out |= 1u << s;
     };
     if (tid == kTma) {
@@ -1033,7 +1041,9 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
                 float x[32];
                 if (ci == 0) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) x[j] = p.S0 ? p.S0[sbase_state + (long long)(c0 + j) * D + v] : 0.f;
+                    for (int j = 0; j < 32; ++j)
+                        x[j] = P.s0_identity ? (c0 + j == v ? 1.f : 0.f)
+                                             : p.S0 ? p.S0[sbase_state + (long long)(c0 + j) * D + v] : 0.f;
                 } else {
                     tmem_ld32(tb + TM2_S + lane_sel + c0, x);
                     tmem_ld_wait();
@@ -1120,7 +1130,9 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
                     float x[32];
                     if (nchunks == 0) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) x[j] = p.S0 ? p.S0[sbase_state + (long long)(c0 + j) * D + v] : 0.f;
+                        for (int j = 0; j < 32; ++j)
+                            x[j] = P.s0_identity ? (c0 + j == v ? 1.f : 0.f)
+                                                 : p.S0 ? p.S0[sbase_state + (long long)(c0 + j) * D + v] : 0.f;
                     } else {
                         tmem_ld32(tb + TM2_S + lane_sel + c0, x);
                         tmem_ld_wait();
@@ -1168,7 +1180,7 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int r = r0 + j;
-                if (r < L) O[((t0 + r) * H + h) * D + v] = __float2bfloat16_rn(p.scale * iq[j] * x[j]);
+                if (r < L && O) O[((t0 + r) * H + h) * D + v] = __float2bfloat16_rn(p.scale * iq[j] * x[j]);
             }
         }
         if (aborted && tid == kTma) {  // copies still in flight finish before exit
@@ -1312,8 +1324,10 @@ cudaError_t run_pass1(const ChunkParams &p, uint8_t *ws, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-// pass 2 of p (v, S0, S_out and o as p gives them) over the records in ws
-cudaError_t run_pass2(const ChunkParams &p, uint8_t *ws, const int32_t *cu_host, cudaStream_t st) {
+// pass 2 of p (v, S0, S_out and o as p gives them; o may be null) over the records in ws;
+// s0_identity starts every chain from the identity, v_zero takes v = 0 (p.v is not read)
+cudaError_t run_pass2(const ChunkParams &p, uint8_t *ws, const int32_t *cu_host, cudaStream_t st, int s0_identity = 0,
+                      int v_zero = 0) {
     const long long total = p.cu_seqlens ? (long long)p.T : (long long)p.N * p.T;
     int *status = reinterpret_cast<int *>(ws);
     const size_t base = 1024 + 16384;
@@ -1326,7 +1340,9 @@ cudaError_t run_pass2(const ChunkParams &p, uint8_t *ws, const int32_t *cu_host,
     B.chunk_off = p.cu_seqlens ? chunk_off : nullptr;
     B.cpr = (int)(((long long)p.T + C - 1) / C);
     B.status = status;
-    if (!make_map(&B.tv, p.v, total, p.H)) return cudaErrorInvalidValue;
+    B.s0_identity = s0_identity;
+    B.v_zero = v_zero;
+    if (!v_zero && !make_map(&B.tv, p.v, total, p.H)) return cudaErrorInvalidValue;
     B.nperm = 0;
     if (cu_host && p.N <= kMaxPerm) {  // longest sequences first
         std::vector<int> idx(p.N);
@@ -1348,7 +1364,8 @@ cudaError_t run_pass2(const ChunkParams &p, uint8_t *ws, const int32_t *cu_host,
 // is affine in the state before it, S_end = M S_start + N (the chunk update
 // S <- diag(e^{G_last}) S + Khat^T (U - W S) is affine in S), so pass 2 runs three
 // times over the segments: with v = 0 and S_start = I (its final states are the
-// M), with S_start = 0 (the N), and, once `kda_seg_chain` has walked the segments
+// M; the identity is formed in the kernel and no v is read), with S_start = 0 (the N;
+// neither run writes outputs), and, once `kda_seg_chain` has walked the segments
 // of each sequence to their true entering states, with those states for the
 // outputs. Pass 1's records do not depend on the state and serve all three runs.
 constexpr int kMaxSeg = 16;
@@ -1373,10 +1390,6 @@ ChunkParams seg_view(const ChunkParams &p, int P, const int32_t *cu_v) {
 }
 
 size_t seg_state_bytes(const ChunkParams &p, int P) { return round1k((size_t)p.N * P * p.H * 128 * 128 * 4); }
-size_t seg_tok_bytes(const ChunkParams &p, size_t esz) {
-    const long long total = p.cu_seqlens ? (long long)p.T : (long long)p.N * p.T;
-    return round1k((size_t)total * p.H * 128 * esz);
-}
 
 }  // namespace tp
 
@@ -1385,9 +1398,7 @@ size_t chunk_2pass_workspace_bytes(const ChunkParams &p) {
     const int P = seg_count(p);
     if (P == 1) return base_workspace_bytes(p);
     const ChunkParams q = seg_view(p, P, reinterpret_cast<const int32_t *>(16));  // only its presence is read
-    const size_t esz = 2;  // the two-pass path takes bf16 inputs
-    return base_workspace_bytes(q) + round1k(((size_t)p.N * P + 1) * 4) + 2 * seg_tok_bytes(p, esz) +
-           4 * seg_state_bytes(p, P);
+    return base_workspace_bytes(q) + round1k(((size_t)p.N * P + 1) * 4) + 3 * seg_state_bytes(p, P);
 }
 
 cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int32_t *cu_host, cudaStream_t st) {
@@ -1399,16 +1410,10 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
         if ((e = run_pass1(p, ws, st)) != cudaSuccess) return e;
         return run_pass2(p, ws, cu_host, st);
     }
-    // workspace: [two-pass workspace of the segment view][cu_v][zero v][o scratch][I][M][N][S_start]
+    // workspace: [two-pass workspace of the segment view][cu_v][M][N][S_start]
     int32_t *cu_v = reinterpret_cast<int32_t *>(ws + base_workspace_bytes(seg_view(p, P, reinterpret_cast<const int32_t *>(16))));
     const ChunkParams q = seg_view(p, P, cu_v);
     uint8_t *cursor = reinterpret_cast<uint8_t *>(cu_v) + round1k(((size_t)p.N * P + 1) * 4);
-    void *zero_v = cursor;
-    cursor += seg_tok_bytes(p, 2);
-    void *o_scr = cursor;
-    cursor += seg_tok_bytes(p, 2);
-    float *Ibuf = reinterpret_cast<float *>(cursor);
-    cursor += seg_state_bytes(p, P);
     float *Mbuf = reinterpret_cast<float *>(cursor);
     cursor += seg_state_bytes(p, P);
     float *Nbuf = reinterpret_cast<float *>(cursor);
@@ -1417,18 +1422,14 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
 
     kda_seg_setup<<<(p.N + 255) / 256, 256, 0, st>>>(p.cu_seqlens, p.T, p.N, P, C, cu_v);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(zero_v, 0, seg_tok_bytes(p, 2), st)) != cudaSuccess) return e;
-    kda_seg_identity<<<1024, 256, 0, st>>>(Ibuf, (long long)q.N * p.H, 128);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = run_pass1(q, ws, st)) != cudaSuccess) return e;
-    ChunkParams pm = q;  // the transitions: v = 0 from the identity
-    pm.v = zero_v; pm.S0 = Ibuf; pm.S_out = Mbuf; pm.o = o_scr;
-    if ((e = run_pass2(pm, ws, nullptr, st)) != cudaSuccess) return e;
-    ChunkParams pn = q;  // the offsets: from zero
-    pn.S0 = nullptr; pn.S_out = Nbuf; pn.o = o_scr;
+    ChunkParams pm = q;  // the transitions: v = 0 from the identity, no outputs
+    pm.v = nullptr; pm.S0 = nullptr; pm.S_out = Mbuf; pm.o = nullptr;
+    if ((e = run_pass2(pm, ws, nullptr, st, 1, 1)) != cudaSuccess) return e;
+    ChunkParams pn = q;  // the offsets: from zero, no outputs
+    pn.S0 = nullptr; pn.S_out = Nbuf; pn.o = nullptr;
     if ((e = run_pass2(pn, ws, nullptr, st)) != cudaSuccess) return e;
     if ((e = seg_chain_launch<128>(p.S0, Mbuf, Nbuf, 128, 128LL * 128, Sbuf, p.S_out, p.N, p.H, P, st)) != cudaSuccess) return e;
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ChunkParams pf = q;  // the outputs, from the true entering states
     pf.S0 = Sbuf; pf.S_out = nullptr;
     return run_pass2(pf, ws, nullptr, st);

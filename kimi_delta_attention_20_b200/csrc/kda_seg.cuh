@@ -1,11 +1,11 @@
 // Segments of long sequences, for the chunk forward when there are too few
 // (sequence, head) state chains to fill the GPU. Every sequence is cut into P
 // segments aligned to `align` tokens; the state after a segment is affine in the
-// state before it, S_end = M S_start + N (each token's update is affine in S), so
-// the forward runs over the segments with v = 0 from the identity (the final
-// states are the M), from zero (the N), and, once `kda_seg_chain` has walked each
-// sequence's segments to their true entering states, from those states for the
-// outputs. Internal linkage: every file that includes this has its own copies.
+// state before it, S_end = M S_start + N (each token's update is affine in S). The
+// caller obtains every segment's transition M and offset N (runs of its forward over
+// the segments), `kda_seg_chain` walks each sequence's segments to their true
+// entering states, and the caller forms the outputs from those. Internal linkage:
+// every file that includes this has its own copies.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -25,15 +25,6 @@ __global__ void kda_seg_setup(const int32_t *cu, int T, int N, int P, int align,
         const long long L = ((len + P - 1) / P + align - 1) / align * align;
         for (int sg = 0; sg < P; ++sg) cu_v[(long long)n * P + sg] = (int32_t)(bos + (sg * L < len ? sg * L : len));
         if (n == N - 1) cu_v[(long long)N * P] = (int32_t)(bos + len);
-    }
-}
-
-// count identity states [D][D]
-__global__ void kda_seg_identity(float *S, long long count, int D) {
-    const long long total = count * D * D;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
-        const long long e = i % ((long long)D * D);
-        S[i] = (e / D) == (e % D) ? 1.f : 0.f;
     }
 }
 
