@@ -239,13 +239,20 @@ typedef struct {
     int has_lower_bound;
     float lower_bound;
     int beta_is_prob;           /* 1: beta is a probability (dbeta is then d/dprob) */
-    void *workspace;            /* device scratch of kda_chunk_bwd_workspace_size() bytes, 16-byte aligned */
+    void *workspace;            /* device scratch of kda_chunk_bwd_workspace_size() bytes, 16-byte aligned
+                                   (256-byte aligned for the segment form) */
     size_t workspace_bytes;
 } kda_chunk_bwd_args;
 
-/* Bytes of workspace kda_chunk_bwd needs: the state checkpoints (one d_k x d_v fp32
- * state per 16 tokens per head), a scratch of 16 states per (sequence, head) and a
- * small header. Only shapes are read. */
+/* Bytes of workspace with which kda_chunk_bwd runs its fastest form: the state
+ * checkpoints (one d_k x d_v fp32 state per 16 tokens per head), a scratch of 16
+ * states per (sequence, head) and a small header; when there are few (sequence, head)
+ * pairs of long sequences and d_k = d_v, also the buffers of the segment form (each
+ * sequence cut into up to 16 segments that are swept side by side: per segment and
+ * head a widened d_k x 2 d_v state and two d_k x d_v states, and the checkpoints and
+ * scratch of the segments). A workspace of at least the plain form's size (the same
+ * sum without the segment buffers) runs the plain form (same result up to rounding);
+ * less returns KDA_ERR_WORKSPACE. Only shapes are read. */
 KDA_API kda_status kda_chunk_bwd_workspace_size(const kda_chunk_bwd_args *args, size_t *bytes);
 
 KDA_API kda_status kda_chunk_bwd(const kda_chunk_bwd_args *args, void *stream);

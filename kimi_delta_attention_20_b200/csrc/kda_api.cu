@@ -21,7 +21,8 @@ size_t chunk_2pass_workspace_bytes(const ChunkParams &p);
 cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int32_t *cu_host, cudaStream_t st);
 bool token_conv_supported(int K);
 size_t bwd_workspace_bytes(bool varlen, long long T, int N, int H, int Dk, int Dv);
-cudaError_t launch_bwd(BwdParams p, bool bf16, int Dk, int Dv, void *workspace, cudaStream_t st);
+size_t bwd_workspace_bytes_min(bool varlen, long long T, int N, int H, int Dk, int Dv);
+cudaError_t launch_bwd(BwdParams p, bool bf16, int Dk, int Dv, void *workspace, size_t workspace_bytes, cudaStream_t st);
 cudaError_t launch_token(const TokenParams &tp, bool bf16, int Dk, int Dv, cudaStream_t st);
 }  // namespace kda
 
@@ -321,7 +322,7 @@ kda_status kda_chunk_bwd(const kda_chunk_bwd_args *a, void *stream) {
             if (cu[n + 1] < cu[n]) return KDA_ERR_INVALID_ARGUMENT;
     }
     if (!a->cu_seqlens && a->cu_seqlens_host) return KDA_ERR_INVALID_ARGUMENT;
-    const size_t need_ws = kda::bwd_workspace_bytes(a->cu_seqlens != nullptr, a->T, N, a->H, a->Dk, a->Dv);
+    const size_t need_ws = kda::bwd_workspace_bytes_min(a->cu_seqlens != nullptr, a->T, N, a->H, a->Dk, a->Dv);
     if (!a->workspace || a->workspace_bytes < need_ws || !aligned(a->workspace, 16)) return KDA_ERR_WORKSPACE;
     kda::BwdParams p{};
     p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta; p.dout = a->dout;
@@ -333,7 +334,8 @@ kda_status kda_chunk_bwd(const kda_chunk_bwd_args *a, void *stream) {
     p.has_lb = a->has_lower_bound ? 1 : 0;
     p.lb = a->lower_bound;
     p.beta_prob = a->beta_is_prob ? 1 : 0;
-    return cuda_status(kda::launch_bwd(p, bf16, a->Dk, a->Dv, a->workspace, static_cast<cudaStream_t>(stream)));
+    return cuda_status(
+        kda::launch_bwd(p, bf16, a->Dk, a->Dv, a->workspace, a->workspace_bytes, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -46,9 +46,12 @@
 // thread-major per CTA (coalesced).
 #include <cooperative_groups.h>
 
+#include <algorithm>
+
 #include "kda_common.cuh"
 #include "kda_bwd.cuh"
 #include "kda_stage.cuh"
+#include "kda_seg.cuh"
 
 namespace kda {
 
@@ -720,18 +723,154 @@ cudaError_t launch_bwd_dt(const BwdParams &p, int Dk, int Dv, cudaStream_t st) {
 }  // namespace
 
 // Workspace: [ckpt_off: N+1 ints, 256-byte block][per-CTA scratch: two stretches of states][checkpoints]
-size_t bwd_workspace_bytes(bool varlen, long long T, int N, int H, int Dk, int Dv) {
+size_t bwd_workspace_bytes_min(bool varlen, long long T, int N, int H, int Dk, int Dv) {
     const long long nck = varlen ? (T + kCB - 1) / kCB + N : (long long)N * ((T + kCB - 1) / kCB);
     const size_t head = (((size_t)(N + 1) * 4 + 255) / 256) * 256;
     return head + 2 * (size_t)N * H * kCB * Dk * Dv * 4 + (size_t)nck * H * Dk * Dv * 4;
 }
 
-cudaError_t launch_bwd(BwdParams p, bool bf16, int Dk, int Dv, void *workspace, cudaStream_t st) {
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
+// Segments: with few (sequence, head) chains the sweeps would leave most SMs idle, so
+// every sequence is cut into P segments that run as a varlen batch of N P sequences.
+// The forward state after a segment is affine in the one before it (S_end = M S_start +
+// N) and so is the state cotangent before a segment in the one after it (dS_start =
+// M' dS_end + N'): the maps come from the two-pass tensor-core kernel's auxiliary
+// passes (bf16, d = 128) or from a widened run of the recurrence (the forward's, and
+// the cotangent walk's, in kda_chunk_rec.cu), `kda_seg_chain` walks them forwards to
+// each segment's entering state and backwards to each segment's leaving cotangent (and
+// the initial-state gradient), and the two sweeps then run over the segments. P fills
+// about two waves of the reverse sweep at two CTAs per SM, with at least 64 tokens per
+// segment on average; square heads only.
+constexpr int kBwdMaxSeg = 16;
+constexpr int kBwdSms = 148;
+
+int bwd_seg_count(bool varlen, long long T, int N, int H, int Dk, int Dv) {
+    if (Dk != Dv || (Dk != 32 && Dk != 64 && Dk != 128)) return 1;
+    const long long ctas = (long long)N * H * (Dv / kDVC);
+    if (ctas <= 0 || ctas * 2 > 4 * kBwdSms) return 1;
+    const long long avg = varlen ? T / (N > 0 ? N : 1) : T;
+    long long P = std::min<long long>(kBwdMaxSeg, 4 * kBwdSms / ctas);
+    P = std::min<long long>(P, avg / 64);
+    return P < 2 ? 1 : (int)P;
+}
+
+size_t chunk_2pass_base_bytes(const ChunkParams &q);
+cudaError_t chunk_2pass_transitions(const ChunkParams &q, void *workspace, float *M, float *Nst, cudaStream_t st);
+cudaError_t rec_widened_run(const ChunkParams &q, bool bf16, int D, bool rev, cudaStream_t st);
+
+// The segment view of a backward call as forward parameters (cu_v: the segment offsets).
+ChunkParams bwd_seg_view(const BwdParams &b, int P, const int32_t *cu_v) {
+    ChunkParams q{};
+    q.q = b.q; q.k = b.k; q.v = b.v; q.g = b.g; q.beta = b.beta;
+    q.cu_seqlens = cu_v;
+    q.T = b.cu_seqlens ? b.T : b.N * b.T;
+    q.N = b.N * P; q.H = b.H;
+    q.scale = b.scale; q.use_l2 = b.use_l2; q.has_lb = b.has_lb; q.lb = b.lb;
+    q.gate_mode = kGateLog; q.beta_prob = b.beta_prob;
+    return q;
+}
+
+// Workspace: [cu_v][widened states (or M, N)][entering states][leaving cotangents][shared]
+// where "shared" holds first the two-pass kernel's records (when it gives the maps),
+// then the sweeps' own workspace.
+struct BwdSegLayout {
+    size_t cu, saug, states, shared, total;
+};
+BwdSegLayout bwd_seg_layout(bool varlen, long long T, int N, int H, int D, int P, bool tc) {
+    auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
+    const long long total = varlen ? T : (long long)N * T;
+    const size_t nv = (size_t)N * P;
+    BwdSegLayout L;
+    L.cu = r256((nv + 1) * 4);
+    L.saug = r256(nv * H * D * 2 * D * 4);
+    L.states = r256(nv * H * D * D * 4);
+    L.shared = bwd_workspace_bytes_min(true, total, (int)nv, H, D, D);
+    if (tc) {
+        ChunkParams q{};
+        q.cu_seqlens = reinterpret_cast<const int32_t *>(16);  // only its presence is read
+        q.T = (int)total; q.N = (int)nv; q.H = H;
+        L.shared = std::max(L.shared, chunk_2pass_base_bytes(q));
+    }
+    L.total = L.cu + L.saug + 2 * L.states + L.shared;
+    return L;
+}
+
+cudaError_t launch_bwd_ws(BwdParams p, bool bf16, int Dk, int Dv, uint8_t *ws, cudaStream_t st) {
     p.ckpt_off = reinterpret_cast<int *>(ws);
     p.scratch = reinterpret_cast<float *>(ws + (((size_t)(p.N + 1) * 4 + 255) / 256) * 256);
     p.ckpt = p.scratch + 2 * (size_t)p.N * p.H * kCB * Dk * Dv;
     return bf16 ? launch_bwd_dt<__nv_bfloat16>(p, Dk, Dv, st) : launch_bwd_dt<float>(p, Dk, Dv, st);
+}
+
+template <int D>
+cudaError_t bwd_segments(const BwdParams &p, bool bf16, int P, const BwdSegLayout &L, uint8_t *ws, bool tc,
+                         cudaStream_t st) {
+    int32_t *cu_v = reinterpret_cast<int32_t *>(ws);
+    float *saug = reinterpret_cast<float *>(ws + L.cu);
+    float *S_start = reinterpret_cast<float *>(ws + L.cu + L.saug);
+    float *dS_end = reinterpret_cast<float *>(ws + L.cu + L.saug + L.states);
+    uint8_t *shared = ws + L.cu + L.saug + 2 * L.states;
+    const ChunkParams q = bwd_seg_view(p, P, cu_v);
+    cudaError_t e;
+    // segments of whole 64-token chunks for the two-pass kernel, of 16-token stretches otherwise
+    kda_seg_setup<<<(p.N + 255) / 256, 256, 0, st>>>(p.cu_seqlens, p.T, p.N, P, tc ? 64 : 16, cu_v);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // the forward maps, then the entering states
+    if (tc) {
+        const size_t half = (size_t)q.N * q.H * D * D;
+        if ((e = chunk_2pass_transitions(q, shared, saug, saug + half, st)) != cudaSuccess) return e;
+        if ((e = seg_chain_launch<D>(p.S0, saug, saug + half, D, (long long)D * D, S_start, nullptr, p.N, p.H, P, st)) !=
+            cudaSuccess)
+            return e;
+    } else {
+        ChunkParams w = q;
+        w.S_out = saug;
+        if ((e = rec_widened_run(w, bf16, D, false, st)) != cudaSuccess) return e;
+        if ((e = seg_chain_launch<D>(p.S0, saug, saug + D, 2 * D, 2LL * D * D, S_start, nullptr, p.N, p.H, P, st)) !=
+            cudaSuccess)
+            return e;
+    }
+    // the cotangent maps, then the leaving cotangents and the initial-state gradient
+    ChunkParams r = q;
+    r.v = p.dout;
+    r.S_out = saug;
+    if ((e = rec_widened_run(r, bf16, D, true, st)) != cudaSuccess) return e;
+    if ((e = seg_chain_launch<D>(p.dSf, saug, saug + D, 2 * D, 2LL * D * D, dS_end, p.dS0, p.N, p.H, P, st, 1)) !=
+        cudaSuccess)
+        return e;
+    BwdParams b = p;  // the sweeps over the segments; dS0 came from the cotangent chain
+    b.cu_seqlens = cu_v;
+    b.T = q.T;
+    b.N = q.N;
+    b.S0 = S_start;
+    b.dSf = dS_end;
+    b.dS0 = nullptr;
+    return launch_bwd_ws(b, bf16, D, D, shared, st);
+}
+
+// The workspace with which kda_chunk_bwd runs its fastest form (the segments when they apply).
+size_t bwd_workspace_bytes(bool varlen, long long T, int N, int H, int Dk, int Dv) {
+    const size_t plain = bwd_workspace_bytes_min(varlen, T, N, H, Dk, Dv);
+    const int P = bwd_seg_count(varlen, T, N, H, Dk, Dv);
+    if (P < 2) return plain;
+    // the larger of the two map sources, so that either dtype fits
+    return std::max({plain, bwd_seg_layout(varlen, T, N, H, Dk, P, false).total,
+                     Dk == 128 ? bwd_seg_layout(varlen, T, N, H, Dk, P, true).total : (size_t)0});
+}
+
+cudaError_t launch_bwd(BwdParams p, bool bf16, int Dk, int Dv, void *workspace, size_t workspace_bytes, cudaStream_t st) {
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const bool varlen = p.cu_seqlens != nullptr;
+    const int P = bwd_seg_count(varlen, p.T, p.N, p.H, Dk, Dv);
+    if (P >= 2 && (reinterpret_cast<uintptr_t>(ws) & 255) == 0) {
+        const bool tc = bf16 && Dk == 128;
+        const BwdSegLayout L = bwd_seg_layout(varlen, p.T, p.N, p.H, Dk, P, tc);
+        if (workspace_bytes >= L.total) {
+            if (Dk == 32) return bwd_segments<32>(p, bf16, P, L, ws, tc, st);
+            if (Dk == 64) return bwd_segments<64>(p, bf16, P, L, ws, tc, st);
+            return bwd_segments<128>(p, bf16, P, L, ws, tc, st);
+        }
+    }
+    return launch_bwd_ws(p, bf16, Dk, Dv, ws, st);
 }
 
 }  // namespace kda

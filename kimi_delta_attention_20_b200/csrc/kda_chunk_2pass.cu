@@ -1401,6 +1401,24 @@ size_t chunk_2pass_workspace_bytes(const ChunkParams &p) {
     return base_workspace_bytes(q) + round1k(((size_t)p.N * P + 1) * 4) + 3 * seg_state_bytes(p, P);
 }
 
+// For kda_bwd.cu's segment form: the transitions and offsets of every sequence of the
+// (segment) view q, from pass 1 over q and pass 2 from the identity with v = 0 (final
+// states to M) and from zero (to Nst), neither writing outputs. ws: chunk_2pass_base_bytes(q).
+size_t chunk_2pass_base_bytes(const ChunkParams &q) { return tp::base_workspace_bytes(q); }
+
+cudaError_t chunk_2pass_transitions(const ChunkParams &q, void *workspace, float *M, float *Nst, cudaStream_t st) {
+    using namespace tp;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    cudaError_t e;
+    if ((e = run_pass1(q, ws, st)) != cudaSuccess) return e;
+    ChunkParams pm = q;
+    pm.v = nullptr; pm.S0 = nullptr; pm.S_out = M; pm.o = nullptr;
+    if ((e = run_pass2(pm, ws, nullptr, st, 1, 1)) != cudaSuccess) return e;
+    ChunkParams pn = q;
+    pn.S0 = nullptr; pn.S_out = Nst; pn.o = nullptr;
+    return run_pass2(pn, ws, nullptr, st);
+}
+
 cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int32_t *cu_host, cudaStream_t st) {
     using namespace tp;
     uint8_t *ws = static_cast<uint8_t *>(workspace);

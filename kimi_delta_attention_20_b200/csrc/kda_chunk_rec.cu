@@ -57,11 +57,13 @@ struct RecSmem {
 // Start the copy of tokens [t0, t0 + cnt) of head h; returns this thread's raw
 // beta (thread i < cnt holds token i's), left unconverted so that the load
 // completes in the background.
-template <typename Tin, int DK, int DV, bool AUG>
-__device__ __forceinline__ Tin rec_issue(const ChunkParams &p, RecSmem<Tin, DK, DV> &sm, long long t0, int cnt, int h) {
-    constexpr int NT = RecCfg<DK, DV>::NT, EP = 16 / (int)sizeof(Tin);
+// (The CTA holds state columns c0 .. c0 + CB - 1 of DV.)
+template <typename Tin, int DK, int DV, bool AUG, int CB>
+__device__ __forceinline__ Tin rec_issue(const ChunkParams &p, RecSmem<Tin, DK, CB> &sm, long long t0, int cnt, int h,
+                                         int c0) {
+    constexpr int NT = RecCfg<DK, CB>::NT, EP = 16 / (int)sizeof(Tin);
     constexpr int VOFF = AUG ? DK : 0, DVR = DV - VOFF;  // augmented: v occupies columns DK .. DV - 1
-    constexpr int RK = DK / EP, RV = DVR / EP;
+    constexpr int RK = DK / EP;
     const int tid = threadIdx.x, H = p.H;
     for (int e = tid; e < cnt * RK; e += NT) {
         const int i = e / RK, c = (e % RK) * EP;
@@ -70,9 +72,11 @@ __device__ __forceinline__ Tin rec_issue(const ChunkParams &p, RecSmem<Tin, DK, 
         cp_async16(&sm.rq[i][c], static_cast<const Tin *>(p.q) + gi);
         cp_async16(&sm.rg[i][c], static_cast<const Tin *>(p.g) + gi);
     }
-    for (int e = tid; e < cnt * RV; e += NT) {
-        const int i = e / RV, c = (e % RV) * EP;
-        cp_async16(&sm.rv[i][VOFF + c], static_cast<const Tin *>(p.v) + ((t0 + i) * H + h) * DVR + c);
+    // the CTA's columns that see v: local vlo .. CB - 1 (none for a block of M columns)
+    const int vlo = max(c0, VOFF) - c0, rv = (CB - vlo) / EP;
+    for (int e = tid; e < cnt * rv; e += NT) {
+        const int i = e / rv, c = (e % rv) * EP;
+        cp_async16(&sm.rv[i][vlo + c], static_cast<const Tin *>(p.v) + ((t0 + i) * H + h) * DVR + (c0 + vlo - VOFF) + c);
     }
     cp_async_commit();
     return tid < cnt ? static_cast<const Tin *>(p.beta)[(t0 + tid) * H + h] : Tin(0.f);
@@ -81,9 +85,9 @@ __device__ __forceinline__ Tin rec_issue(const ChunkParams &p, RecSmem<Tin, DK, 
 // The staged stretch as fp32 token vectors. Each key row is taken by TPR
 // threads that form its squared norms with shuffles (uniform trip count: rows
 // past cnt read row 0 and store nothing). Barriers on both sides.
-template <typename Tin, int DK, int DV, bool AUG>
-__device__ void rec_take(const ChunkParams &p, RecSmem<Tin, DK, DV> &sm, int cnt, Tin beta_raw, float rate) {
-    using Cfg = RecCfg<DK, DV>;
+template <typename Tin, int DK, bool AUG, int CB>
+__device__ void rec_take(const ChunkParams &p, RecSmem<Tin, DK, CB> &sm, int cnt, Tin beta_raw, float rate, int c0) {
+    using Cfg = RecCfg<DK, CB>;
     constexpr int NT = Cfg::NT, TPR = Cfg::TPR, E = Cfg::E;
     const int tid = threadIdx.x;
     cp_async_wait_all();
@@ -118,9 +122,9 @@ __device__ void rec_take(const ChunkParams &p, RecSmem<Tin, DK, DV> &sm, int cnt
             store_vec<E>(&sm.al[i][c], gx);
         }
     }
-    for (int e = tid; e < cnt * DV; e += NT) {
-        const int i = e / DV, cc = e % DV;
-        sm.vo[i][cc] = (AUG && cc < DK) ? 0.f : to_f32(sm.rv[i][cc]);
+    for (int e = tid; e < cnt * CB; e += NT) {
+        const int i = e / CB, cc = e % CB;
+        sm.vo[i][cc] = (AUG && c0 + cc < DK) ? 0.f : to_f32(sm.rv[i][cc]);
     }
     if (tid < cnt) sm.b[tid] = beta_value(to_f32(beta_raw), p.beta_prob);
     __syncthreads();
@@ -163,16 +167,25 @@ __device__ __forceinline__ float rowgroup_scatter(const float (&x)[CG]) {
 // the first d_k columns start from the identity and see v = 0, the others start from
 // zero and see v; the outputs [scale M^T q^ | scale N^T q^] go out in fp32, rows of
 // d_k + d_v, and the final state as [d_k][d_k + d_v].
-template <typename Tin, int DK, int DV, bool AUG>
-__global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(ChunkParams p) {
-    using Cfg = RecCfg<DK, DV>;
+// REV (with AUG): the cotangent walk of the backward's segment form. Tokens are taken
+// from the segment's end back to its start, and per token (v holding the output
+// cotangent do) dS += scale q^ do^T, ddelta = dS^T k^, dS <- diag(a) (dS - b k^ ddelta^T):
+// the cotangent of the state before the token. From [I | 0] the final state is
+// [M | N] with dS_start = M dS_end + N over the segment. No outputs.
+// CB: state columns per CTA; the DV / CB CTAs of one (sequence, head) (blockIdx.y) need
+// nothing from one another, since the columns of S evolve independently.
+template <typename Tin, int DK, int DV, bool AUG, bool REV = false, int CB = DV>
+__global__ void __launch_bounds__(RecCfg<DK, CB>::NT) kda_chunk_rec_kernel(ChunkParams p) {
+    using Cfg = RecCfg<DK, CB>;
     constexpr int RP = Cfg::RP, CT = Cfg::CT, NT = Cfg::NT, CG = Cfg::CG, CP = CG / 2;
     constexpr int VS = 32 / CG;  // lanes between the holders of consecutive reduced values
     extern __shared__ __align__(16) uint8_t smraw[];
-    RecSmem<Tin, DK, DV> &sm = *reinterpret_cast<RecSmem<Tin, DK, DV> *>(smraw);
+    RecSmem<Tin, DK, CB> &sm = *reinterpret_cast<RecSmem<Tin, DK, CB> *>(smraw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int rg = lane >> 2, cg = lane & 3;
-    const int col = Cfg::WC * warp + CG * cg;  // this lane's first value column
+    const int c0 = blockIdx.y * CB;            // the CTA's first state column
+    const int col = Cfg::WC * warp + CG * cg;  // this lane's first value column within the CTA's
+    const int gcol = c0 + col;
     const long long nh = blockIdx.x;
     const int n = (int)(nh / p.H), h = (int)(nh % p.H), H = p.H;
     long long bos, eos;
@@ -189,115 +202,180 @@ __global__ void __launch_bounds__(RecCfg<DK, DV>::NT) kda_chunk_rec_kernel(Chunk
     for (int r = 0; r < RP; ++r)
 #pragma unroll
         for (int j = 0; j < CP; j += 2) {
-            const int row = rg * RP + r, c0 = col + 2 * j;
-            const float4 x = AUG ? make_float4(row == c0, row == c0 + 1, row == c0 + 2, row == c0 + 3)
-                             : p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + (nh * DK + row) * DV + c0)
+            const int row = rg * RP + r, cj = gcol + 2 * j;
+            const float4 x = AUG ? make_float4(row == cj, row == cj + 1, row == cj + 2, row == cj + 3)
+                             : p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + (nh * DK + row) * DV + cj)
                                     : make_float4(0.f, 0.f, 0.f, 0.f);
             s[r][j] = make_float2(x.x, x.y);
             s[r][j + 1] = make_float2(x.z, x.w);
         }
 
-    Tin braw = bos < eos ? rec_issue<Tin, DK, DV, AUG>(p, sm, bos, (int)min((long long)CT, eos - bos), h) : Tin(0.f);
-    for (long long t0 = bos; t0 < eos; t0 += CT) {
-        const int cnt = (int)min((long long)CT, eos - t0);
-        rec_take<Tin, DK, DV, AUG>(p, sm, cnt, braw, rate);
-        if (t0 + CT < eos) braw = rec_issue<Tin, DK, DV, AUG>(p, sm, t0 + CT, (int)min((long long)CT, eos - t0 - CT), h);
+    // stretches of CT tokens, in order (forward) or from the end (REV: the cotangent walk)
+    long long t0 = REV ? max(bos, eos - CT) : bos;
+    int cnt = (int)(REV ? eos - t0 : min((long long)CT, eos - bos));
+    Tin braw = cnt > 0 ? rec_issue<Tin, DK, DV, AUG, CB>(p, sm, t0, cnt, h, c0) : Tin(0.f);
+    while (cnt > 0) {
+        rec_take<Tin, DK, AUG, CB>(p, sm, cnt, braw, rate, c0);
+        long long t0n;
+        int cntn;
+        if (REV) { t0n = max(bos, t0 - CT); cntn = (int)(t0 - t0n); }
+        else { t0n = t0 + CT; cntn = (int)max(0LL, min((long long)CT, eos - t0n)); }
+        if (cntn > 0) braw = rec_issue<Tin, DK, DV, AUG, CB>(p, sm, t0n, cntn, h, c0);
+        if constexpr (REV) {
 #pragma unroll 2
-        for (int i = 0; i < cnt; ++i) {
-            float kr[RP], ar[RP], qr[RP];
-            rows_in<RP>(&sm.kh[i][rg * RP], kr);
-            rows_in<RP>(&sm.al[i][rg * RP], ar);
-            rows_in<RP>(&sm.qh[i][rg * RP], qr);
-            const float b = sm.b[i];
-            float2 vv[CP];
+            for (int i = cnt - 1; i >= 0; --i) {
+                float kr[RP], ar[RP], qr[RP];
+                rows_in<RP>(&sm.kh[i][rg * RP], kr);
+                rows_in<RP>(&sm.al[i][rg * RP], ar);
+                rows_in<RP>(&sm.qh[i][rg * RP], qr);
+                const float b = sm.b[i];
+                float2 dov[CP];  // scale do of the lane's columns (zero in the M block)
 #pragma unroll
-            for (int j = 0; j < CP; j += 2) {
-                const float4 x = *reinterpret_cast<const float4 *>(&sm.vo[i][col + 2 * j]);
-                vv[j] = make_float2(x.x, x.y);
-                vv[j + 1] = make_float2(x.z, x.w);
-            }
-            // S' = diag(a) S and this lane's part of u = S'^T k^ (two chains per pair)
-            const float2 z2 = make_float2(0.f, 0.f);
-            float2 acc[2][CP];
+                for (int j = 0; j < CP; j += 2) {
+                    const float4 x = *reinterpret_cast<const float4 *>(&sm.vo[i][col + 2 * j]);
+                    dov[j] = make_float2(p.scale * x.x, p.scale * x.y);
+                    dov[j + 1] = make_float2(p.scale * x.z, p.scale * x.w);
+                }
+                // dS += scale q^ do^T and this lane's part of ddelta = dS^T k^
+                const float2 z2 = make_float2(0.f, 0.f);
+                float2 acc[2][CP];
 #pragma unroll
-            for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
+                for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
 #pragma unroll
-            for (int r = 0; r < RP; ++r) {
-                const float2 a2 = make_float2(ar[r], ar[r]), k2 = make_float2(kr[r], kr[r]);
+                for (int r = 0; r < RP; ++r) {
+                    const float2 q2 = make_float2(qr[r], qr[r]), k2 = make_float2(kr[r], kr[r]);
+#pragma unroll
+                    for (int j = 0; j < CP; ++j) {
+                        s[r][j] = __ffma2_rn(q2, dov[j], s[r][j]);
+                        acc[r & 1][j] = __ffma2_rn(s[r][j], k2, acc[r & 1][j]);
+                    }
+                }
+                float part[CG];
 #pragma unroll
                 for (int j = 0; j < CP; ++j) {
-                    s[r][j] = __fmul2_rn(s[r][j], a2);
-                    acc[r & 1][j] = __ffma2_rn(s[r][j], k2, acc[r & 1][j]);
+                    const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
+                    part[2 * j] = t.x; part[2 * j + 1] = t.y;
+                }
+                const float m = rowgroup_scatter<CG>(part);
+                float2 nd[CP];  // -b ddelta of the lane's columns
+#pragma unroll
+                for (int j = 0; j < CP; ++j)
+                    nd[j] = make_float2(-b * __shfl_sync(0xffffffffu, m, (2 * j) * VS + cg),
+                                        -b * __shfl_sync(0xffffffffu, m, (2 * j + 1) * VS + cg));
+                // dS <- diag(a) (dS - b k^ ddelta^T): the cotangent of the previous state
+#pragma unroll
+                for (int r = 0; r < RP; ++r) {
+                    const float2 k2 = make_float2(kr[r], kr[r]), a2 = make_float2(ar[r], ar[r]);
+#pragma unroll
+                    for (int j = 0; j < CP; ++j) s[r][j] = __fmul2_rn(__ffma2_rn(k2, nd[j], s[r][j]), a2);
                 }
             }
-            float part[CG];
+        } else {
+#pragma unroll 2
+            for (int i = 0; i < cnt; ++i) {
+                float kr[RP], ar[RP], qr[RP];
+                rows_in<RP>(&sm.kh[i][rg * RP], kr);
+                rows_in<RP>(&sm.al[i][rg * RP], ar);
+                rows_in<RP>(&sm.qh[i][rg * RP], qr);
+                const float b = sm.b[i];
+                float2 vv[CP];
 #pragma unroll
-            for (int j = 0; j < CP; ++j) {
-                const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
-                part[2 * j] = t.x; part[2 * j + 1] = t.y;
-            }
-            const float m = rowgroup_scatter<CG>(part);
-            // gather u of the lane's columns from the lanes that hold them
-            float2 d[CP];
-            const float2 b2 = make_float2(b, b);
+                for (int j = 0; j < CP; j += 2) {
+                    const float4 x = *reinterpret_cast<const float4 *>(&sm.vo[i][col + 2 * j]);
+                    vv[j] = make_float2(x.x, x.y);
+                    vv[j + 1] = make_float2(x.z, x.w);
+                }
+                // S' = diag(a) S and this lane's part of u = S'^T k^ (two chains per pair)
+                const float2 z2 = make_float2(0.f, 0.f);
+                float2 acc[2][CP];
 #pragma unroll
-            for (int j = 0; j < CP; ++j) {
-                const float2 u = make_float2(__shfl_sync(0xffffffffu, m, (2 * j) * VS + cg),
-                                             __shfl_sync(0xffffffffu, m, (2 * j + 1) * VS + cg));
-                d[j] = __fmul2_rn(b2, __fadd2_rn(vv[j], make_float2(-u.x, -u.y)));
-            }
-            // S = S' + k^ d^T and this lane's part of S^T q^
+                for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
 #pragma unroll
-            for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
+                for (int r = 0; r < RP; ++r) {
+                    const float2 a2 = make_float2(ar[r], ar[r]), k2 = make_float2(kr[r], kr[r]);
 #pragma unroll
-            for (int r = 0; r < RP; ++r) {
-                const float2 k2 = make_float2(kr[r], kr[r]), q2 = make_float2(qr[r], qr[r]);
+                    for (int j = 0; j < CP; ++j) {
+                        s[r][j] = __fmul2_rn(s[r][j], a2);
+                        acc[r & 1][j] = __ffma2_rn(s[r][j], k2, acc[r & 1][j]);
+                    }
+                }
+                float part[CG];
 #pragma unroll
                 for (int j = 0; j < CP; ++j) {
-                    s[r][j] = __ffma2_rn(k2, d[j], s[r][j]);
-                    acc[r & 1][j] = __ffma2_rn(s[r][j], q2, acc[r & 1][j]);
+                    const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
+                    part[2 * j] = t.x; part[2 * j + 1] = t.y;
+                }
+                const float m = rowgroup_scatter<CG>(part);
+                // gather u of the lane's columns from the lanes that hold them
+                float2 d[CP];
+                const float2 b2 = make_float2(b, b);
+#pragma unroll
+                for (int j = 0; j < CP; ++j) {
+                    const float2 u = make_float2(__shfl_sync(0xffffffffu, m, (2 * j) * VS + cg),
+                                                 __shfl_sync(0xffffffffu, m, (2 * j + 1) * VS + cg));
+                    d[j] = __fmul2_rn(b2, __fadd2_rn(vv[j], make_float2(-u.x, -u.y)));
+                }
+                // S = S' + k^ d^T and this lane's part of S^T q^
+#pragma unroll
+                for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
+#pragma unroll
+                for (int r = 0; r < RP; ++r) {
+                    const float2 k2 = make_float2(kr[r], kr[r]), q2 = make_float2(qr[r], qr[r]);
+#pragma unroll
+                    for (int j = 0; j < CP; ++j) {
+                        s[r][j] = __ffma2_rn(k2, d[j], s[r][j]);
+                        acc[r & 1][j] = __ffma2_rn(s[r][j], q2, acc[r & 1][j]);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < CP; ++j) {
+                    const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
+                    part[2 * j] = t.x; part[2 * j + 1] = t.y;
+                }
+                const float ov = rowgroup_scatter<CG>(part);
+                if (CG == 8 || (lane & 4) == 0) sm.vo[i][col + lane / VS] = p.scale * ov;
+            }
+        }
+        if (p.o) {
+            // the stretch's output rows, from shared memory
+            __syncthreads();
+            for (int e = 4 * tid; e < cnt * CB; e += 4 * NT) {
+                const int i = e / CB, c = e % CB;
+                const float4 x = *reinterpret_cast<const float4 *>(&sm.vo[i][c]);
+                if constexpr (AUG) {
+                    *reinterpret_cast<float4 *>(static_cast<float *>(p.o) + ((t0 + i) * H + h) * DV + c0 + c) = x;
+                } else {
+                    Tin *dst = static_cast<Tin *>(p.o) + ((t0 + i) * H + h) * DV + c0 + c;
+                    dst[0] = from_f32<Tin>(x.x); dst[1] = from_f32<Tin>(x.y);
+                    dst[2] = from_f32<Tin>(x.z); dst[3] = from_f32<Tin>(x.w);
                 }
             }
-#pragma unroll
-            for (int j = 0; j < CP; ++j) {
-                const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
-                part[2 * j] = t.x; part[2 * j + 1] = t.y;
-            }
-            const float ov = rowgroup_scatter<CG>(part);
-            if (CG == 8 || (lane & 4) == 0) sm.vo[i][col + lane / VS] = p.scale * ov;
+    
         }
-        // the stretch's output rows, from shared memory
-        __syncthreads();
-        for (int e = 4 * tid; e < cnt * DV; e += 4 * NT) {
-            const int i = e / DV, c = e % DV;
-            const float4 x = *reinterpret_cast<const float4 *>(&sm.vo[i][c]);
-            if constexpr (AUG) {
-                *reinterpret_cast<float4 *>(static_cast<float *>(p.o) + ((t0 + i) * H + h) * DV + c) = x;
-            } else {
-                Tin *dst = static_cast<Tin *>(p.o) + ((t0 + i) * H + h) * DV + c;
-                dst[0] = from_f32<Tin>(x.x); dst[1] = from_f32<Tin>(x.y);
-                dst[2] = from_f32<Tin>(x.z); dst[3] = from_f32<Tin>(x.w);
-            }
-        }
+        t0 = t0n;
+        cnt = cntn;
     }
     if (p.S_out) {
 #pragma unroll
         for (int r = 0; r < RP; ++r)
 #pragma unroll
             for (int j = 0; j < CP; j += 2)
-                *reinterpret_cast<float4 *>(p.S_out + (nh * DK + rg * RP + r) * DV + col + 2 * j) =
+                *reinterpret_cast<float4 *>(p.S_out + (nh * DK + rg * RP + r) * DV + gcol + 2 * j) =
                     make_float4(s[r][j].x, s[r][j].y, s[r][j + 1].x, s[r][j + 1].y);
     }
 }
 
-template <typename Tin, int DK, int DV, bool AUG = false>
+template <typename Tin, int DK, int DV, bool AUG = false, bool REV = false, int CB = DV>
 cudaError_t launch_rec_t(const ChunkParams &p, cudaStream_t st) {
+    static_assert(!REV || AUG, "the cotangent walk runs in the widened form");
+    static_assert(DV % CB == 0 && (!AUG || DK % CB == 0 || CB == DV), "a column block lies inside the M or the N block, or holds both");
     const long long blocks = (long long)p.N * p.H;
     if (blocks == 0) return cudaSuccess;
-    const int smem = (int)sizeof(RecSmem<Tin, DK, DV>);
-    cudaError_t e = cudaFuncSetAttribute(kda_chunk_rec_kernel<Tin, DK, DV, AUG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem = (int)sizeof(RecSmem<Tin, DK, CB>);
+    auto kern = kda_chunk_rec_kernel<Tin, DK, DV, AUG, REV, CB>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kda_chunk_rec_kernel<Tin, DK, DV, AUG><<<(unsigned)blocks, RecCfg<DK, DV>::NT, smem, st>>>(p);
+    kern<<<dim3((unsigned)blocks, DV / CB), RecCfg<DK, CB>::NT, smem, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -462,6 +540,21 @@ cudaError_t launch_rec_seg_dt(const ChunkParams &p, int P, int D, uint8_t *ws, c
 }
 
 }  // namespace
+
+// One widened run over a segment view q (kda_bwd.cu's segment form): the forward's
+// [M | N] (rev = false: v from q.v) or the cotangent walk's (rev = true: the output
+// cotangent in q.v), final states to q.S_out as [d][2d]; q.o is not written.
+cudaError_t rec_widened_run(const ChunkParams &q, bool bf16, int D, bool rev, cudaStream_t st) {
+#define KDA_WIDE(D_)                                                                                        \
+    if (D == D_) {                                                                                          \
+        if (bf16) return rev ? launch_rec_t<__nv_bfloat16, D_, 2 * D_, true, true>(q, st)                   \
+                             : launch_rec_t<__nv_bfloat16, D_, 2 * D_, true, false>(q, st);                 \
+        return rev ? launch_rec_t<float, D_, 2 * D_, true, true>(q, st) : launch_rec_t<float, D_, 2 * D_, true, false>(q, st); \
+    }
+    KDA_WIDE(32) KDA_WIDE(64) KDA_WIDE(128)
+#undef KDA_WIDE
+    return cudaErrorInvalidValue;
+}
 
 // Workspace the recurrent forward can use (0: it needs none).
 size_t chunk_rec_workspace_bytes(const ChunkParams &p, bool bf16, int Dk, int Dv) {

@@ -55,10 +55,14 @@ struct SegChainSmem {
 };
 
 // M_s and N_s are read at M + vs pitch and Nst + vs pitch (vs = (n P + s) H + h), rows
-// ld floats apart; S_start is written as packed D x D states.
+// ld floats apart; S_start is written as packed D x D states. rev walks the segments
+// from the last to the first (the backward's cotangent, entering at each segment's end:
+// S0 is then the final-state cotangent, S_start(s) the cotangent at the end of segment
+// s, and S_out the cotangent of the initial state).
 template <int D>
 __global__ void __launch_bounds__(SegChainCfg<D>::NT) kda_seg_chain(const float *S0, const float *M, const float *Nst, int ld,
-                                                    long long pitch, float *S_start, float *S_out, int N, int H, int P) {
+                                                    long long pitch, float *S_start, float *S_out, int N, int H, int P,
+                                                    int rev) {
     using Cfg = SegChainCfg<D>;
     constexpr int NT = Cfg::NT, R = Cfg::R, NB = Cfg::NB, SL = D / 16;
     extern __shared__ __align__(16) uint8_t smraw[];
@@ -70,7 +74,7 @@ __global__ void __launch_bounds__(SegChainCfg<D>::NT) kda_seg_chain(const float 
     auto stage = [&](int sg) {  // start the copies of M_sg and N_sg's slice into buffer sg % NB
         if (sg < P) {
             const int b = sg % NB;
-            const long long vs = ((long long)n * P + sg) * H + h;
+            const long long vs = ((long long)n * P + (rev ? P - 1 - sg : sg)) * H + h;
             const float *src = M + vs * pitch;
             for (int e = tid; e < D * (D / 4); e += NT)
                 cp_async16(&sm.m[b][e / (D / 4)][(e % (D / 4)) * 4], src + (long long)(e / (D / 4)) * ld + (e % (D / 4)) * 4);
@@ -89,7 +93,7 @@ __global__ void __launch_bounds__(SegChainCfg<D>::NT) kda_seg_chain(const float 
     int cur = 0;
 #pragma unroll 1
     for (int sg = 0; sg < P; ++sg) {
-        const long long vs = ((long long)n * P + sg) * H + h;  // virtual (segment, head) state index
+        const long long vs = ((long long)n * P + (rev ? P - 1 - sg : sg)) * H + h;  // virtual (segment, head) state index
         cp_async_wait_group<NB - 2>();
         __syncthreads();  // M_sg, N_sg and the current state are in place; buffer (sg - 1) % NB is free
         stage(sg + NB - 1);
@@ -142,12 +146,12 @@ __global__ void __launch_bounds__(SegChainCfg<D>::NT) kda_seg_chain(const float 
 // Launch the chain for N sequences x H heads of D x D states.
 template <int D>
 cudaError_t seg_chain_launch(const float *S0, const float *M, const float *Nst, int ld, long long pitch, float *S_start,
-                             float *S_out, int N, int H, int P, cudaStream_t st) {
+                             float *S_out, int N, int H, int P, cudaStream_t st, int rev = 0) {
     cudaError_t e = cudaFuncSetAttribute(kda_seg_chain<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(SegChainSmem<D>));
     if (e != cudaSuccess) return e;
     kda_seg_chain<D><<<(unsigned)((long long)N * H * (D / 16)), SegChainCfg<D>::NT, sizeof(SegChainSmem<D>), st>>>(
-        S0, M, Nst, ld, pitch, S_start, S_out, N, H, P);
+        S0, M, Nst, ld, pitch, S_start, S_out, N, H, P, rev);
     return cudaGetLastError();
 }
 

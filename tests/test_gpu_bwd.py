@@ -82,6 +82,28 @@ def test_backward_options(case):
     run_and_compare(inp, dtype, tag=case, **kw)
 
 
+@pytest.mark.parametrize("case", ["d32_fp32_varlen", "d64_bf16", "d128_bf16", "d64_fp32_options"])
+def test_backward_segments(case):
+    """Few (sequence, head) chains of long sequences: the backward cuts every sequence
+    into segments, gets each segment's entering state and leaving state cotangent from
+    two widened runs and two chain walks, and sweeps the segments side by side. An
+    empty sequence, a short one (trailing segments empty), initial states, the
+    final-state cotangent and the initial-state gradient through the chains."""
+    if case == "d32_fp32_varlen":
+        inp = draw((700, 1500, 64, 0), 1, 32, 32, torch.float32, seed=140)
+        run_and_compare(inp, torch.float32, lower_bound=-5.0, tag=case)
+    elif case == "d64_bf16":
+        inp = draw((300, 900), 2, 64, 64, torch.bfloat16, seed=141)
+        run_and_compare(inp, torch.bfloat16, lower_bound=-5.0, tag=case)
+    elif case == "d128_bf16":
+        inp = draw((1000,), 2, 128, 128, torch.bfloat16, seed=142)
+        run_and_compare(inp, torch.bfloat16, lower_bound=-5.0, tag=case)
+    else:
+        inp = draw((500, 260), 1, 64, 64, torch.float32, seed=143)
+        inp["beta"] = torch.sigmoid(inp["beta"].float())
+        run_and_compare(inp, torch.float32, final=False, prob=True, tag=case)
+
+
 def test_autograd_through_chunk_kda():
     """loss.backward() through chunk_kda gives kda_chunk_bwd's gradients, which match the oracle."""
     import kimi_delta_attention_20_b200 as kda
