@@ -731,15 +731,17 @@ size_t bwd_workspace_bytes_min(bool varlen, long long T, int N, int H, int Dk, i
 
 // Segments: with few (sequence, head) chains the sweeps would leave most SMs idle, so
 // every sequence is cut into P segments that run as a varlen batch of N P sequences.
-// The forward state after a segment is affine in the one before it (S_end = M S_start +
-// N) and so is the state cotangent before a segment in the one after it (dS_start =
-// M' dS_end + N'): the maps come from the two-pass tensor-core kernel's auxiliary
-// passes (bf16, d = 128) or from a widened run of the recurrence (the forward's, and
-// the cotangent walk's, in kda_chunk_rec.cu), `kda_seg_chain` walks them forwards to
-// each segment's entering state and backwards to each segment's leaving cotangent (and
-// the initial-state gradient), and the two sweeps then run over the segments. P fills
-// about two waves of the reverse sweep at two CTAs per SM, with at least 64 tokens per
-// segment on average; square heads only.
+// Per token the forward map is S -> A S + b k^ v^T with A = (I - b k^ k^T) diag(a), and
+// the cotangent map is dS -> A^T (dS + scale q^ do^T): A^T = diag(a) (I - b k^ k^T). So
+// over a segment S_end = M S_start + N and dS_start = M^T dS_end + N', where M = A_last
+// ... A_first, N' = sum_t w_t do_t^T and w_t = scale M_t^T q^_t (M_t = A_t ... A_first,
+// the map up to token t) is the output of the run that gives M. M, N and w come from
+// the two-pass tensor-core kernel's auxiliary passes (bf16, d = 128) or from a widened
+// run of the recurrence (kda_chunk_rec.cu); `kda_seg_chain` walks them forwards to each
+// segment's entering state and, with M^T and N', backwards to each segment's leaving
+// cotangent (and the initial-state gradient); the two sweeps then run over the
+// segments. P fills about two waves of the reverse sweep at two CTAs per SM, with at
+// least 64 tokens per segment on average; square heads only.
 constexpr int kBwdMaxSeg = 16;
 constexpr int kBwdSms = 148;
 
@@ -754,8 +756,88 @@ int bwd_seg_count(bool varlen, long long T, int N, int H, int Dk, int Dv) {
 }
 
 size_t chunk_2pass_base_bytes(const ChunkParams &q);
-cudaError_t chunk_2pass_transitions(const ChunkParams &q, void *workspace, float *M, float *Nst, cudaStream_t st);
-cudaError_t rec_widened_run(const ChunkParams &q, bool bf16, int D, bool rev, cudaStream_t st);
+cudaError_t chunk_2pass_transitions(const ChunkParams &q, void *workspace, float *M, float *Nst, float *w,
+                                    cudaStream_t st);
+cudaError_t rec_widened_run(const ChunkParams &q, bool bf16, int D, cudaStream_t st);
+
+namespace {
+
+// MT[s] = M[s]^T (packed D x D) for the states at M + s pitch, rows ld floats apart; one
+// 32 x 32 tile per CTA through shared memory.
+template <int D>
+__global__ void __launch_bounds__(256) kda_seg_transpose(const float *M, int ld, long long pitch, float *MT) {
+    constexpr int TB = D / 32;
+    __shared__ float tile[32][33];
+    const long long b = blockIdx.x, s = b / (TB * TB);
+    const int tr = (int)(b % (TB * TB)) / TB, tc = (int)(b % TB);
+    const float *src = M + s * pitch;
+    float *dst = MT + s * (long long)D * D;
+    const int x = threadIdx.x & 31, y = threadIdx.x >> 5;
+    for (int i = y; i < 32; i += 8) tile[i][x] = src[(long long)(32 * tr + i) * ld + 32 * tc + x];
+    __syncthreads();
+    for (int i = y; i < 32; i += 8) dst[(long long)(32 * tc + i) * D + 32 * tr + x] = tile[x][i];
+}
+
+__device__ __forceinline__ float4 load4_f32(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4_f32(const __nv_bfloat16 *p) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+// N'[v H + h] = sum over the tokens t of segment v of w_t do_t^T, w_t = row t H + h of w
+// (wstride floats apart), do_t = row t H + h of dout. One CTA per (segment, head, 32
+// rows k of N'); tokens in tiles of 32 staged in shared memory; thread (kr, cc) = (warp,
+// lane) sums rows 4 kr .. of its block and columns CC cc .. (CC = D / 32).
+template <typename Tin, int D>
+__global__ void __launch_bounds__(256) kda_seg_cot_offset(const float *w, int wstride, const Tin *dout,
+                                                          const int32_t *cu_v, float *Nrev, int H) {
+    constexpr int TT = 32, CC = D / 32;
+    __shared__ __align__(16) float wsm[TT][36];
+    __shared__ __align__(16) float dsm[TT][D + 4];
+    const int v = blockIdx.x / H, h = blockIdx.x % H, kb = blockIdx.y;
+    const int tid = threadIdx.x, kr = tid >> 5, cc = tid & 31;
+    const long long bos = cu_v[v], eos = cu_v[v + 1];
+    float acc[4][CC];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int j = 0; j < CC; ++j) acc[r][j] = 0.f;
+    for (long long t0 = bos; t0 < eos; t0 += TT) {
+        const int cnt = (int)min((long long)TT, eos - t0);
+        __syncthreads();  // the previous tile is consumed
+        for (int e = tid; e < TT * 8; e += 256) {
+            const int i = e >> 3, q4 = (e & 7) * 4;
+            *reinterpret_cast<float4 *>(&wsm[i][q4]) =
+                i < cnt ? load4_f32(w + ((t0 + i) * H + h) * wstride + 32 * kb + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        for (int e = tid; e < TT * (D / 4); e += 256) {
+            const int i = e / (D / 4), c4 = (e % (D / 4)) * 4;
+            *reinterpret_cast<float4 *>(&dsm[i][c4]) =
+                i < cnt ? load4_f32(dout + ((t0 + i) * H + h) * D + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        __syncthreads();
+        for (int i = 0; i < cnt; ++i) {
+            const float4 wk = *reinterpret_cast<const float4 *>(&wsm[i][4 * kr]);
+            const float wv[4] = {wk.x, wk.y, wk.z, wk.w};
+            float dc[CC];
+#pragma unroll
+            for (int j = 0; j < CC; ++j) dc[j] = dsm[i][CC * cc + j];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int j = 0; j < CC; ++j) acc[r][j] = fmaf(wv[r], dc[j], acc[r][j]);
+        }
+    }
+    float *dst = Nrev + ((long long)blockIdx.x * D + 32 * kb + 4 * kr) * D + CC * cc;
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int j = 0; j < CC; ++j) dst[(long long)r * D + j] = acc[r][j];
+}
+
+}  // namespace
 
 // The segment view of a backward call as forward parameters (cu_v: the segment offsets).
 ChunkParams bwd_seg_view(const BwdParams &b, int P, const int32_t *cu_v) {
@@ -769,11 +851,11 @@ ChunkParams bwd_seg_view(const BwdParams &b, int P, const int32_t *cu_v) {
     return q;
 }
 
-// Workspace: [cu_v][widened states (or M, N)][entering states][leaving cotangents][shared]
-// where "shared" holds first the two-pass kernel's records (when it gives the maps),
-// then the sweeps' own workspace.
+// Workspace: [cu_v][M, N (or [M | N] rows)][entering states][leaving cotangents]
+// [M^T, N'][w rows][shared] where "shared" holds first the two-pass kernel's records
+// (when it gives the maps), then the sweeps' own workspace.
 struct BwdSegLayout {
-    size_t cu, saug, states, shared, total;
+    size_t cu, maps, states, w, shared, total;
 };
 BwdSegLayout bwd_seg_layout(bool varlen, long long T, int N, int H, int D, int P, bool tc) {
     auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
@@ -781,8 +863,9 @@ BwdSegLayout bwd_seg_layout(bool varlen, long long T, int N, int H, int D, int P
     const size_t nv = (size_t)N * P;
     BwdSegLayout L;
     L.cu = r256((nv + 1) * 4);
-    L.saug = r256(nv * H * D * 2 * D * 4);
+    L.maps = r256(nv * H * D * 2 * D * 4);
     L.states = r256(nv * H * D * D * 4);
+    L.w = r256((size_t)total * H * D * (tc ? 1 : 2) * 4);
     L.shared = bwd_workspace_bytes_min(true, total, (int)nv, H, D, D);
     if (tc) {
         ChunkParams q{};
@@ -790,7 +873,7 @@ BwdSegLayout bwd_seg_layout(bool varlen, long long T, int N, int H, int D, int P
         q.T = (int)total; q.N = (int)nv; q.H = H;
         L.shared = std::max(L.shared, chunk_2pass_base_bytes(q));
     }
-    L.total = L.cu + L.saug + 2 * L.states + L.shared;
+    L.total = L.cu + L.maps + 4 * L.states + L.w + L.shared;
     return L;
 }
 
@@ -804,38 +887,47 @@ cudaError_t launch_bwd_ws(BwdParams p, bool bf16, int Dk, int Dv, uint8_t *ws, c
 template <int D>
 cudaError_t bwd_segments(const BwdParams &p, bool bf16, int P, const BwdSegLayout &L, uint8_t *ws, bool tc,
                          cudaStream_t st) {
-    int32_t *cu_v = reinterpret_cast<int32_t *>(ws);
-    float *saug = reinterpret_cast<float *>(ws + L.cu);
-    float *S_start = reinterpret_cast<float *>(ws + L.cu + L.saug);
-    float *dS_end = reinterpret_cast<float *>(ws + L.cu + L.saug + L.states);
-    uint8_t *shared = ws + L.cu + L.saug + 2 * L.states;
+    uint8_t *cur = ws;
+    int32_t *cu_v = reinterpret_cast<int32_t *>(cur); cur += L.cu;
+    float *maps = reinterpret_cast<float *>(cur); cur += L.maps;
+    float *S_start = reinterpret_cast<float *>(cur); cur += L.states;
+    float *dS_end = reinterpret_cast<float *>(cur); cur += L.states;
+    float *MT = reinterpret_cast<float *>(cur); cur += L.states;
+    float *Nrev = reinterpret_cast<float *>(cur); cur += L.states;
+    float *w = reinterpret_cast<float *>(cur); cur += L.w;
+    uint8_t *shared = cur;
     const ChunkParams q = bwd_seg_view(p, P, cu_v);
+    const long long nst = (long long)q.N * q.H;
     cudaError_t e;
     // segments of whole 64-token chunks for the two-pass kernel, of 16-token stretches otherwise
     kda_seg_setup<<<(p.N + 255) / 256, 256, 0, st>>>(p.cu_seqlens, p.T, p.N, P, tc ? 64 : 16, cu_v);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // the forward maps, then the entering states
+    // the forward maps and w, then the entering states
+    const float *M, *Nf;
+    int ld, wstride;
+    long long pitch;
     if (tc) {
-        const size_t half = (size_t)q.N * q.H * D * D;
-        if ((e = chunk_2pass_transitions(q, shared, saug, saug + half, st)) != cudaSuccess) return e;
-        if ((e = seg_chain_launch<D>(p.S0, saug, saug + half, D, (long long)D * D, S_start, nullptr, p.N, p.H, P, st)) !=
-            cudaSuccess)
-            return e;
+        M = maps; Nf = maps + nst * D * D; ld = D; pitch = (long long)D * D; wstride = D;
+        if ((e = chunk_2pass_transitions(q, shared, maps, maps + nst * D * D, w, st)) != cudaSuccess) return e;
     } else {
-        ChunkParams w = q;
-        w.S_out = saug;
-        if ((e = rec_widened_run(w, bf16, D, false, st)) != cudaSuccess) return e;
-        if ((e = seg_chain_launch<D>(p.S0, saug, saug + D, 2 * D, 2LL * D * D, S_start, nullptr, p.N, p.H, P, st)) !=
-            cudaSuccess)
-            return e;
+        M = maps; Nf = maps + D; ld = 2 * D; pitch = 2LL * D * D; wstride = 2 * D;
+        ChunkParams r = q;
+        r.S_out = maps;
+        r.o = w;
+        if ((e = rec_widened_run(r, bf16, D, st)) != cudaSuccess) return e;
     }
-    // the cotangent maps, then the leaving cotangents and the initial-state gradient
-    ChunkParams r = q;
-    r.v = p.dout;
-    r.S_out = saug;
-    if ((e = rec_widened_run(r, bf16, D, true, st)) != cudaSuccess) return e;
-    if ((e = seg_chain_launch<D>(p.dSf, saug, saug + D, 2 * D, 2LL * D * D, dS_end, p.dS0, p.N, p.H, P, st, 1)) !=
-        cudaSuccess)
+    if ((e = seg_chain_launch<D>(p.S0, M, Nf, ld, pitch, S_start, nullptr, p.N, p.H, P, st)) != cudaSuccess) return e;
+    // the cotangent maps M^T and N', then the leaving cotangents and the initial-state gradient
+    kda_seg_transpose<D><<<(unsigned)(nst * (D / 32) * (D / 32)), 256, 0, st>>>(M, ld, pitch, MT);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (bf16)
+        kda_seg_cot_offset<__nv_bfloat16, D><<<dim3((unsigned)nst, D / 32), 256, 0, st>>>(
+            w, wstride, static_cast<const __nv_bfloat16 *>(p.dout), cu_v, Nrev, p.H);
+    else
+        kda_seg_cot_offset<float, D><<<dim3((unsigned)nst, D / 32), 256, 0, st>>>(
+            w, wstride, static_cast<const float *>(p.dout), cu_v, Nrev, p.H);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = seg_chain_launch<D>(p.dSf, MT, Nrev, D, (long long)D * D, dS_end, p.dS0, p.N, p.H, P, st, 1)) != cudaSuccess)
         return e;
     BwdParams b = p;  // the sweeps over the segments; dS0 came from the cotangent chain
     b.cu_seqlens = cu_v;

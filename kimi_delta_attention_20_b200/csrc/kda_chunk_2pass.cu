@@ -943,6 +943,7 @@ struct StateParams {
     int cpr;
     int *status;
     int s0_identity;  // start every chain from the identity (S0 is not read)
+    int o_f32;        // outputs in fp32 (rows of D floats) instead of bf16
     int v_zero;       // v = 0: no v tiles are copied (tv is not read) and the stage's v area stays zero
     int nperm;
     int perm[kMaxPerm];
@@ -1149,6 +1150,7 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
     } else {
         // ================= output rows, one chunk behind
         __nv_bfloat16 *O = static_cast<__nv_bfloat16 *>(p.o);
+        float *Of = P.o_f32 ? static_cast<float *>(p.o) : nullptr;
         for (int ci = 0; ci < nchunks; ++ci) {
             const int s = ci & 1, b = ci & 1;
             const uint8_t *stg = sm + s * STAGE_BYTES;
@@ -1180,7 +1182,11 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int r = r0 + j;
-                if (r < L && O) O[((t0 + r) * H + h) * D + v] = __float2bfloat16_rn(p.scale * iq[j] * x[j]);
+                if (r < L && O) {
+                    const float ov = p.scale * iq[j] * x[j];
+                    if (Of) Of[((t0 + r) * H + h) * D + v] = ov;
+                    else O[((t0 + r) * H + h) * D + v] = __float2bfloat16_rn(ov);
+                }
             }
         }
         if (aborted && tid == kTma) {  // copies still in flight finish before exit
@@ -1327,7 +1333,7 @@ cudaError_t run_pass1(const ChunkParams &p, uint8_t *ws, cudaStream_t st) {
 // pass 2 of p (v, S0, S_out and o as p gives them; o may be null) over the records in ws;
 // s0_identity starts every chain from the identity, v_zero takes v = 0 (p.v is not read)
 cudaError_t run_pass2(const ChunkParams &p, uint8_t *ws, const int32_t *cu_host, cudaStream_t st, int s0_identity = 0,
-                      int v_zero = 0) {
+                      int v_zero = 0, int o_f32 = 0) {
     const long long total = p.cu_seqlens ? (long long)p.T : (long long)p.N * p.T;
     int *status = reinterpret_cast<int *>(ws);
     const size_t base = 1024 + 16384;
@@ -1342,6 +1348,7 @@ cudaError_t run_pass2(const ChunkParams &p, uint8_t *ws, const int32_t *cu_host,
     B.status = status;
     B.s0_identity = s0_identity;
     B.v_zero = v_zero;
+    B.o_f32 = o_f32;
     if (!v_zero && !make_map(&B.tv, p.v, total, p.H)) return cudaErrorInvalidValue;
     B.nperm = 0;
     if (cu_host && p.N <= kMaxPerm) {  // longest sequences first
@@ -1403,17 +1410,20 @@ size_t chunk_2pass_workspace_bytes(const ChunkParams &p) {
 
 // For kda_bwd.cu's segment form: the transitions and offsets of every sequence of the
 // (segment) view q, from pass 1 over q and pass 2 from the identity with v = 0 (final
-// states to M) and from zero (to Nst), neither writing outputs. ws: chunk_2pass_base_bytes(q).
+// states to M; per token, w_t = scale M_t^T q^_t to w in fp32 rows of D when w is given,
+// M_t the map up to token t) and from zero (final states to Nst, no outputs).
+// ws: chunk_2pass_base_bytes(q).
 size_t chunk_2pass_base_bytes(const ChunkParams &q) { return tp::base_workspace_bytes(q); }
 
-cudaError_t chunk_2pass_transitions(const ChunkParams &q, void *workspace, float *M, float *Nst, cudaStream_t st) {
+cudaError_t chunk_2pass_transitions(const ChunkParams &q, void *workspace, float *M, float *Nst, float *w,
+                                    cudaStream_t st) {
     using namespace tp;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     cudaError_t e;
     if ((e = run_pass1(q, ws, st)) != cudaSuccess) return e;
     ChunkParams pm = q;
-    pm.v = nullptr; pm.S0 = nullptr; pm.S_out = M; pm.o = nullptr;
-    if ((e = run_pass2(pm, ws, nullptr, st, 1, 1)) != cudaSuccess) return e;
+    pm.v = nullptr; pm.S0 = nullptr; pm.S_out = M; pm.o = w;
+    if ((e = run_pass2(pm, ws, nullptr, st, 1, 1, 1)) != cudaSuccess) return e;
     ChunkParams pn = q;
     pn.S0 = nullptr; pn.S_out = Nst; pn.o = nullptr;
     return run_pass2(pn, ws, nullptr, st);

@@ -167,14 +167,9 @@ __device__ __forceinline__ float rowgroup_scatter(const float (&x)[CG]) {
 // the first d_k columns start from the identity and see v = 0, the others start from
 // zero and see v; the outputs [scale M^T q^ | scale N^T q^] go out in fp32, rows of
 // d_k + d_v, and the final state as [d_k][d_k + d_v].
-// REV (with AUG): the cotangent walk of the backward's segment form. Tokens are taken
-// from the segment's end back to its start, and per token (v holding the output
-// cotangent do) dS += scale q^ do^T, ddelta = dS^T k^, dS <- diag(a) (dS - b k^ ddelta^T):
-// the cotangent of the state before the token. From [I | 0] the final state is
-// [M | N] with dS_start = M dS_end + N over the segment. No outputs.
 // CB: state columns per CTA; the DV / CB CTAs of one (sequence, head) (blockIdx.y) need
 // nothing from one another, since the columns of S evolve independently.
-template <typename Tin, int DK, int DV, bool AUG, bool REV = false, int CB = DV>
+template <typename Tin, int DK, int DV, bool AUG, int CB = DV>
 __global__ void __launch_bounds__(RecCfg<DK, CB>::NT) kda_chunk_rec_kernel(ChunkParams p) {
     using Cfg = RecCfg<DK, CB>;
     constexpr int RP = Cfg::RP, CT = Cfg::CT, NT = Cfg::NT, CG = Cfg::CG, CP = CG / 2;
@@ -210,131 +205,77 @@ __global__ void __launch_bounds__(RecCfg<DK, CB>::NT) kda_chunk_rec_kernel(Chunk
             s[r][j + 1] = make_float2(x.z, x.w);
         }
 
-    // stretches of CT tokens, in order (forward) or from the end (REV: the cotangent walk)
-    long long t0 = REV ? max(bos, eos - CT) : bos;
-    int cnt = (int)(REV ? eos - t0 : min((long long)CT, eos - bos));
+    long long t0 = bos;  // stretches of CT tokens
+    int cnt = (int)min((long long)CT, eos - bos);
     Tin braw = cnt > 0 ? rec_issue<Tin, DK, DV, AUG, CB>(p, sm, t0, cnt, h, c0) : Tin(0.f);
     while (cnt > 0) {
         rec_take<Tin, DK, AUG, CB>(p, sm, cnt, braw, rate, c0);
-        long long t0n;
-        int cntn;
-        if (REV) { t0n = max(bos, t0 - CT); cntn = (int)(t0 - t0n); }
-        else { t0n = t0 + CT; cntn = (int)max(0LL, min((long long)CT, eos - t0n)); }
+        const long long t0n = t0 + CT;
+        const int cntn = (int)max(0LL, min((long long)CT, eos - t0n));
         if (cntn > 0) braw = rec_issue<Tin, DK, DV, AUG, CB>(p, sm, t0n, cntn, h, c0);
-        if constexpr (REV) {
 #pragma unroll 2
-            for (int i = cnt - 1; i >= 0; --i) {
-                float kr[RP], ar[RP], qr[RP];
-                rows_in<RP>(&sm.kh[i][rg * RP], kr);
-                rows_in<RP>(&sm.al[i][rg * RP], ar);
-                rows_in<RP>(&sm.qh[i][rg * RP], qr);
-                const float b = sm.b[i];
-                float2 dov[CP];  // scale do of the lane's columns (zero in the M block)
+        for (int i = 0; i < cnt; ++i) {
+            float kr[RP], ar[RP], qr[RP];
+            rows_in<RP>(&sm.kh[i][rg * RP], kr);
+            rows_in<RP>(&sm.al[i][rg * RP], ar);
+            rows_in<RP>(&sm.qh[i][rg * RP], qr);
+            const float b = sm.b[i];
+            float2 vv[CP];
 #pragma unroll
-                for (int j = 0; j < CP; j += 2) {
-                    const float4 x = *reinterpret_cast<const float4 *>(&sm.vo[i][col + 2 * j]);
-                    dov[j] = make_float2(p.scale * x.x, p.scale * x.y);
-                    dov[j + 1] = make_float2(p.scale * x.z, p.scale * x.w);
-                }
-                // dS += scale q^ do^T and this lane's part of ddelta = dS^T k^
-                const float2 z2 = make_float2(0.f, 0.f);
-                float2 acc[2][CP];
+            for (int j = 0; j < CP; j += 2) {
+                const float4 x = *reinterpret_cast<const float4 *>(&sm.vo[i][col + 2 * j]);
+                vv[j] = make_float2(x.x, x.y);
+                vv[j + 1] = make_float2(x.z, x.w);
+            }
+            // S' = diag(a) S and this lane's part of u = S'^T k^ (two chains per pair)
+            const float2 z2 = make_float2(0.f, 0.f);
+            float2 acc[2][CP];
 #pragma unroll
-                for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
+            for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
 #pragma unroll
-                for (int r = 0; r < RP; ++r) {
-                    const float2 q2 = make_float2(qr[r], qr[r]), k2 = make_float2(kr[r], kr[r]);
-#pragma unroll
-                    for (int j = 0; j < CP; ++j) {
-                        s[r][j] = __ffma2_rn(q2, dov[j], s[r][j]);
-                        acc[r & 1][j] = __ffma2_rn(s[r][j], k2, acc[r & 1][j]);
-                    }
-                }
-                float part[CG];
+            for (int r = 0; r < RP; ++r) {
+                const float2 a2 = make_float2(ar[r], ar[r]), k2 = make_float2(kr[r], kr[r]);
 #pragma unroll
                 for (int j = 0; j < CP; ++j) {
-                    const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
-                    part[2 * j] = t.x; part[2 * j + 1] = t.y;
-                }
-                const float m = rowgroup_scatter<CG>(part);
-                float2 nd[CP];  // -b ddelta of the lane's columns
-#pragma unroll
-                for (int j = 0; j < CP; ++j)
-                    nd[j] = make_float2(-b * __shfl_sync(0xffffffffu, m, (2 * j) * VS + cg),
-                                        -b * __shfl_sync(0xffffffffu, m, (2 * j + 1) * VS + cg));
-                // dS <- diag(a) (dS - b k^ ddelta^T): the cotangent of the previous state
-#pragma unroll
-                for (int r = 0; r < RP; ++r) {
-                    const float2 k2 = make_float2(kr[r], kr[r]), a2 = make_float2(ar[r], ar[r]);
-#pragma unroll
-                    for (int j = 0; j < CP; ++j) s[r][j] = __fmul2_rn(__ffma2_rn(k2, nd[j], s[r][j]), a2);
+                    s[r][j] = __fmul2_rn(s[r][j], a2);
+                    acc[r & 1][j] = __ffma2_rn(s[r][j], k2, acc[r & 1][j]);
                 }
             }
-        } else {
-#pragma unroll 2
-            for (int i = 0; i < cnt; ++i) {
-                float kr[RP], ar[RP], qr[RP];
-                rows_in<RP>(&sm.kh[i][rg * RP], kr);
-                rows_in<RP>(&sm.al[i][rg * RP], ar);
-                rows_in<RP>(&sm.qh[i][rg * RP], qr);
-                const float b = sm.b[i];
-                float2 vv[CP];
+            float part[CG];
 #pragma unroll
-                for (int j = 0; j < CP; j += 2) {
-                    const float4 x = *reinterpret_cast<const float4 *>(&sm.vo[i][col + 2 * j]);
-                    vv[j] = make_float2(x.x, x.y);
-                    vv[j + 1] = make_float2(x.z, x.w);
-                }
-                // S' = diag(a) S and this lane's part of u = S'^T k^ (two chains per pair)
-                const float2 z2 = make_float2(0.f, 0.f);
-                float2 acc[2][CP];
-#pragma unroll
-                for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
-#pragma unroll
-                for (int r = 0; r < RP; ++r) {
-                    const float2 a2 = make_float2(ar[r], ar[r]), k2 = make_float2(kr[r], kr[r]);
-#pragma unroll
-                    for (int j = 0; j < CP; ++j) {
-                        s[r][j] = __fmul2_rn(s[r][j], a2);
-                        acc[r & 1][j] = __ffma2_rn(s[r][j], k2, acc[r & 1][j]);
-                    }
-                }
-                float part[CG];
-#pragma unroll
-                for (int j = 0; j < CP; ++j) {
-                    const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
-                    part[2 * j] = t.x; part[2 * j + 1] = t.y;
-                }
-                const float m = rowgroup_scatter<CG>(part);
-                // gather u of the lane's columns from the lanes that hold them
-                float2 d[CP];
-                const float2 b2 = make_float2(b, b);
-#pragma unroll
-                for (int j = 0; j < CP; ++j) {
-                    const float2 u = make_float2(__shfl_sync(0xffffffffu, m, (2 * j) * VS + cg),
-                                                 __shfl_sync(0xffffffffu, m, (2 * j + 1) * VS + cg));
-                    d[j] = __fmul2_rn(b2, __fadd2_rn(vv[j], make_float2(-u.x, -u.y)));
-                }
-                // S = S' + k^ d^T and this lane's part of S^T q^
-#pragma unroll
-                for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
-#pragma unroll
-                for (int r = 0; r < RP; ++r) {
-                    const float2 k2 = make_float2(kr[r], kr[r]), q2 = make_float2(qr[r], qr[r]);
-#pragma unroll
-                    for (int j = 0; j < CP; ++j) {
-                        s[r][j] = __ffma2_rn(k2, d[j], s[r][j]);
-                        acc[r & 1][j] = __ffma2_rn(s[r][j], q2, acc[r & 1][j]);
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < CP; ++j) {
-                    const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
-                    part[2 * j] = t.x; part[2 * j + 1] = t.y;
-                }
-                const float ov = rowgroup_scatter<CG>(part);
-                if (CG == 8 || (lane & 4) == 0) sm.vo[i][col + lane / VS] = p.scale * ov;
+            for (int j = 0; j < CP; ++j) {
+                const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
+                part[2 * j] = t.x; part[2 * j + 1] = t.y;
             }
+            const float m = rowgroup_scatter<CG>(part);
+            // gather u of the lane's columns from the lanes that hold them
+            float2 d[CP];
+            const float2 b2 = make_float2(b, b);
+#pragma unroll
+            for (int j = 0; j < CP; ++j) {
+                const float2 u = make_float2(__shfl_sync(0xffffffffu, m, (2 * j) * VS + cg),
+                                             __shfl_sync(0xffffffffu, m, (2 * j + 1) * VS + cg));
+                d[j] = __fmul2_rn(b2, __fadd2_rn(vv[j], make_float2(-u.x, -u.y)));
+            }
+            // S = S' + k^ d^T and this lane's part of S^T q^
+#pragma unroll
+            for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
+#pragma unroll
+            for (int r = 0; r < RP; ++r) {
+                const float2 k2 = make_float2(kr[r], kr[r]), q2 = make_float2(qr[r], qr[r]);
+#pragma unroll
+                for (int j = 0; j < CP; ++j) {
+                    s[r][j] = __ffma2_rn(k2, d[j], s[r][j]);
+                    acc[r & 1][j] = __ffma2_rn(s[r][j], q2, acc[r & 1][j]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < CP; ++j) {
+                const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
+                part[2 * j] = t.x; part[2 * j + 1] = t.y;
+            }
+            const float ov = rowgroup_scatter<CG>(part);
+            if (CG == 8 || (lane & 4) == 0) sm.vo[i][col + lane / VS] = p.scale * ov;
         }
         if (p.o) {
             // the stretch's output rows, from shared memory
@@ -365,14 +306,13 @@ __global__ void __launch_bounds__(RecCfg<DK, CB>::NT) kda_chunk_rec_kernel(Chunk
     }
 }
 
-template <typename Tin, int DK, int DV, bool AUG = false, bool REV = false, int CB = DV>
+template <typename Tin, int DK, int DV, bool AUG = false, int CB = DV>
 cudaError_t launch_rec_t(const ChunkParams &p, cudaStream_t st) {
-    static_assert(!REV || AUG, "the cotangent walk runs in the widened form");
     static_assert(DV % CB == 0 && (!AUG || DK % CB == 0 || CB == DV), "a column block lies inside the M or the N block, or holds both");
     const long long blocks = (long long)p.N * p.H;
     if (blocks == 0) return cudaSuccess;
     const int smem = (int)sizeof(RecSmem<Tin, DK, CB>);
-    auto kern = kda_chunk_rec_kernel<Tin, DK, DV, AUG, REV, CB>;
+    auto kern = kda_chunk_rec_kernel<Tin, DK, DV, AUG, CB>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     kern<<<dim3((unsigned)blocks, DV / CB), RecCfg<DK, CB>::NT, smem, st>>>(p);
@@ -541,16 +481,12 @@ cudaError_t launch_rec_seg_dt(const ChunkParams &p, int P, int D, uint8_t *ws, c
 
 }  // namespace
 
-// One widened run over a segment view q (kda_bwd.cu's segment form): the forward's
-// [M | N] (rev = false: v from q.v) or the cotangent walk's (rev = true: the output
-// cotangent in q.v), final states to q.S_out as [d][2d]; q.o is not written.
-cudaError_t rec_widened_run(const ChunkParams &q, bool bf16, int D, bool rev, cudaStream_t st) {
-#define KDA_WIDE(D_)                                                                                        \
-    if (D == D_) {                                                                                          \
-        if (bf16) return rev ? launch_rec_t<__nv_bfloat16, D_, 2 * D_, true, true>(q, st)                   \
-                             : launch_rec_t<__nv_bfloat16, D_, 2 * D_, true, false>(q, st);                 \
-        return rev ? launch_rec_t<float, D_, 2 * D_, true, true>(q, st) : launch_rec_t<float, D_, 2 * D_, true, false>(q, st); \
-    }
+// One widened run over a segment view q (kda_bwd.cu's segment form): final states
+// [M | N] to q.S_out as [d][2d] and, when q.o is given, the fp32 outputs
+// [scale M_t^T q^_t | scale N_t^T q^_t] as rows of 2d.
+cudaError_t rec_widened_run(const ChunkParams &q, bool bf16, int D, cudaStream_t st) {
+#define KDA_WIDE(D_) \
+    if (D == D_) return bf16 ? launch_rec_t<__nv_bfloat16, D_, 2 * D_, true>(q, st) : launch_rec_t<float, D_, 2 * D_, true>(q, st);
     KDA_WIDE(32) KDA_WIDE(64) KDA_WIDE(128)
 #undef KDA_WIDE
     return cudaErrorInvalidValue;
