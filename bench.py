@@ -107,9 +107,12 @@ def token_algorithmic(N, H, D, K):
 
 
 # chunk_kda backward: the B1 T8192 H16 d128 lb-5 chunk workload with an output and a
-# final-state cotangent; two kernels per call (checkpoints, reverse sweep)
+# final-state cotangent. Its 16 (sequence, head) chains run in segment form, 13 kernels
+# per call: segment offsets; pass 1 (prep, intra, exact) and two state passes of the
+# two-pass forward for the segment maps; the forward chain; the transpose and the
+# cotangent offsets; the reverse chain; checkpoint offsets, checkpoints, reverse sweep
 BWD_WL = 2
-BWD_LAUNCHES = 2
+BWD_LAUNCHES = 13
 # FP32 FMA peak of the part: 148 SMs x 128 FP32 lanes x 2 flops x 1965 MHz
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
