@@ -40,8 +40,29 @@ __global__ void __launch_bounds__(256) kda_decode_kernel(StepParams p) {
     const int rg = tid >> 3;                         // first key row of this thread
 
     float *S = p.state + nh * (long long)(DK * DV) + slab * Cfg::kCols + cg * 4;
+    const int h = nh % p.H;
 
-    // Issue the state reads first so their latency hides the vector work.
+    // The token's vectors first: they are few bytes, but every step after the state
+    // read waits on them, and a new token's vectors come from HBM. Raw values now,
+    // converted once the state reads are in flight.
+    static_assert(DK <= Cfg::kThreads, "one key channel per thread");
+    Tin q_raw = Tin(0.f), k_raw = Tin(0.f), g_raw = Tin(0.f), b_raw = Tin(0.f), v_raw = Tin(0.f);
+    float bias = 0.f, rate = 0.f;
+    if (tid < DK) {
+        q_raw = static_cast<const Tin *>(p.q)[nh * DK + tid];
+        k_raw = static_cast<const Tin *>(p.k)[nh * DK + tid];
+        g_raw = static_cast<const Tin *>(p.g)[nh * DK + tid];
+        if (p.gate_mode != kGateLog) {
+            rate = expf(p.A_log[h]);
+            if (p.dt_bias) bias = p.dt_bias[h * DK + tid];
+        }
+    }
+    if (warp == 0) {
+        b_raw = static_cast<const Tin *>(p.beta)[nh];
+        v_raw = static_cast<const Tin *>(p.v)[nh * DV + slab * Cfg::kCols + lane];
+    }
+
+    // then the state reads, held in registers until the write-back
     float4 s[NP];
 #pragma unroll
     for (int i = 0; i < NP; ++i) {
@@ -55,16 +76,10 @@ __global__ void __launch_bounds__(256) kda_decode_kernel(StepParams p) {
     __shared__ float rk_part[NW][32], rq_part[NW][32];
     __shared__ float sdelta[32];
 
-    const Tin *qp = static_cast<const Tin *>(p.q) + nh * DK;
-    const Tin *kp = static_cast<const Tin *>(p.k) + nh * DK;
-    const Tin *gp = static_cast<const Tin *>(p.g) + nh * DK;
-    const int h = nh % p.H;
-    const float rate = p.gate_mode != kGateLog ? expf(p.A_log[h]) : 0.f;
-    for (int c = tid; c < DK; c += Cfg::kThreads) {
-        sq[c] = to_f32(qp[c]);
-        sk[c] = to_f32(kp[c]);
-        const float bias = p.gate_mode != kGateLog && p.dt_bias ? p.dt_bias[h * DK + c] : 0.f;
-        sa[c] = expf(gate_value(to_f32(gp[c]), bias, rate, p.gate_mode, p.has_lb, p.lb));
+    if (tid < DK) {
+        sq[tid] = to_f32(q_raw);
+        sk[tid] = to_f32(k_raw);
+        sa[tid] = expf(gate_value(to_f32(g_raw), bias, rate, p.gate_mode, p.has_lb, p.lb));
     }
     __syncthreads();
     if (warp == 0) {
@@ -112,8 +127,8 @@ __global__ void __launch_bounds__(256) kda_decode_kernel(StepParams p) {
 #pragma unroll
         for (int w = 0; w < NW; ++w) { a += rk_part[w][lane]; b += rq_part[w][lane]; }
         const int col = slab * Cfg::kCols + lane;
-        const float bsig = beta_value(to_f32(static_cast<const Tin *>(p.beta)[nh]), p.beta_prob);
-        const float vj = to_f32(static_cast<const Tin *>(p.v)[nh * DV + col]);
+        const float bsig = beta_value(to_f32(b_raw), p.beta_prob);
+        const float vj = to_f32(v_raw);
         const float delta = bsig * (vj - inv_k * a);
         sdelta[lane] = delta;
         const float kq = inv_k * inv_q * sred[2];
