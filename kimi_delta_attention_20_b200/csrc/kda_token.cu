@@ -35,7 +35,17 @@ __global__ void __launch_bounds__(kTokThreads) kda_token_kernel(TokenParams tp) 
     const long long n = nh / H;
 
     float *S = p.state + nh * (long long)(DK * DV) + 4 * vg;
-    // the state reads go first so that their latency hides the conv and vector work
+    // the token's gate, beta and output-gate values first (a few bytes each, but the
+    // steps after the state read wait on them), raw until used
+    const Tin *gop = static_cast<const Tin *>(tp.g_out);
+    Tin g_raw = Tin(0.f), b_raw = Tin(0.f), go_raw = Tin(0.f);
+    if (tid < DK) g_raw = static_cast<const Tin *>(p.g)[nh * DK + tid];
+    if (tid < DV) {
+        b_raw = static_cast<const Tin *>(p.beta)[nh];
+        if (gop) go_raw = gop[nh * DV + tid];
+    }
+    static_assert(DK <= kTokThreads && DV <= kTokThreads, "one channel per thread");
+    // then the state reads, whose latency hides the conv and vector work
     float4 s[RP];
 #pragma unroll
     for (int i = 0; i < RP; ++i) s[i] = ld_stream(reinterpret_cast<const float4 *>(S + (long long)(kg * RP + i) * DV));
@@ -75,11 +85,10 @@ __global__ void __launch_bounds__(kTokThreads) kda_token_kernel(TokenParams tp) 
         }
         *dst = acc / (1.f + expf(-acc));  // SiLU
     }
-    const Tin *gp = static_cast<const Tin *>(p.g) + nh * DK;
     const float rate = p.gate_mode != kGateLog ? expf(p.A_log[h]) : 0.f;
-    for (int c = tid; c < DK; c += NT) {
-        const float bias = p.gate_mode != kGateLog && p.dt_bias ? p.dt_bias[h * DK + c] : 0.f;
-        sa[c] = expf(gate_value(to_f32(gp[c]), bias, rate, p.gate_mode, p.has_lb, p.lb));
+    if (tid < DK) {
+        const float bias = p.gate_mode != kGateLog && p.dt_bias ? p.dt_bias[h * DK + tid] : 0.f;
+        sa[tid] = expf(gate_value(to_f32(g_raw), bias, rate, p.gate_mode, p.has_lb, p.lb));
     }
     __syncthreads();
     if (warp == 0) {
@@ -117,13 +126,12 @@ __global__ void __launch_bounds__(kTokThreads) kda_token_kernel(TokenParams tp) 
         float a = 0.f, b = 0.f;
 #pragma unroll 8
         for (int g = 0; g < KG; ++g) { a += rk_part[g][tid]; b += rq_part[g][tid]; }
-        const float bsig = beta_value(to_f32(static_cast<const Tin *>(p.beta)[nh]), p.beta_prob);
+        const float bsig = beta_value(to_f32(b_raw), p.beta_prob);
         const float delta = bsig * (sv[tid] - inv_k * a);
         sdelta[tid] = delta;
         core = p.scale * (inv_q * b + delta * inv_k * inv_q * sred[2]);
     }
     // ---- output gate: RMS of the head's core output (threads tid < DV hold it)
-    const Tin *gop = static_cast<const Tin *>(tp.g_out);
     if (gop) {
         float ss = warp_sum(tid < DV ? core * core : 0.f);
         if (lane == 0) swarp[warp] = ss;
@@ -136,7 +144,7 @@ __global__ void __launch_bounds__(kTokThreads) kda_token_kernel(TokenParams tp) 
 #pragma unroll
             for (int w = 0; w < NW; ++w) tot += swarp[w];
             const float inv = rsqrtf(tot / DV + tp.norm_eps);
-            const float gv = to_f32(gop[nh * DV + tid]);
+            const float gv = to_f32(go_raw);
             out = core * inv / (1.f + expf(-gv));
         }
         static_cast<Tin *>(p.o)[nh * DV + tid] = from_f32<Tin>(out);
