@@ -821,9 +821,16 @@ __global__ void __launch_bounds__(256) kda_seg_cot_offset(const float *w, int ws
         for (int i = 0; i < cnt; ++i) {
             const float4 wk = *reinterpret_cast<const float4 *>(&wsm[i][4 * kr]);
             const float wv[4] = {wk.x, wk.y, wk.z, wk.w};
-            float dc[CC];
-#pragma unroll
-            for (int j = 0; j < CC; ++j) dc[j] = dsm[i][CC * cc + j];
+            float dc[CC];  // one vector load of the lane's CC consecutive columns (no bank conflicts)
+            if constexpr (CC == 4) {
+                const float4 x = *reinterpret_cast<const float4 *>(&dsm[i][4 * cc]);
+                dc[0] = x.x; dc[1] = x.y; dc[2] = x.z; dc[3] = x.w;
+            } else if constexpr (CC == 2) {
+                const float2 x = *reinterpret_cast<const float2 *>(&dsm[i][2 * cc]);
+                dc[0] = x.x; dc[1] = x.y;
+            } else {
+                dc[0] = dsm[i][cc];
+            }
 #pragma unroll
             for (int r = 0; r < 4; ++r)
 #pragma unroll
