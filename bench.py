@@ -37,6 +37,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -149,10 +150,10 @@ class ClockSampler:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, log_dir=None):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.path = os.path.join(log_dir or tempfile.gettempdir(), f"kda_clocks_rank{gpu_index}.csv")
 
     def __enter__(self):
         try:
@@ -369,7 +370,7 @@ def run_kda(args, rank, world, local_rank):
     tok_graph.replay()
     torch.cuda.synchronize(dev)
 
-    with ClockSampler(gpu_index) as clocks:
+    with ClockSampler(gpu_index, args.clocks_log) as clocks:
         # chunk forward: K timed steps
         barrier(); torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -616,6 +617,8 @@ def main():
                     help="with --only chunk: chunk workload index (default: the varlen H=96 one)")
     ap.add_argument("--chunk-heads", type=int, default=None,
                     help="with --only chunk: number of heads of the chunk workload (default: its own)")
+    ap.add_argument("--clocks-log", default=None,
+                    help="directory for the nvidia-smi clock samples (default: the temp directory)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "kda":
         ap.error("--warmup must be >= 3")
