@@ -219,11 +219,13 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
 
     uint32_t ph_in = 0, ph_mma = 0;
     bool in_out = false, mma_out = false, aborted = false;
+    // the phase advances only when it completed, so an abort waits on the pending one
     auto wait_all = [&](uint64_t *bar, uint32_t &ph) -> bool {
         bool ok = true;
         if (warp == 0) ok = mbar_wait(bar, ph, kWaitLimitNs);
-        ph ^= 1;
-        return __syncthreads_or(!ok) != 0;
+        const bool stop = __syncthreads_or(!ok) != 0;
+        if (!stop) ph ^= 1;
+        return stop;
     };
     auto issue_in = [&](const Item &it) {
         mbar_arrive_expect_tx(bar_in, 4 * 16384);

@@ -170,11 +170,13 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     };
     // a bounded wait on an mbarrier phase: one warp polls, the others park in the
     // CTA barrier (no issue slots spent polling); true if the CTA must stop
+    // (the phase advances only when it completed, so an abort waits on the pending one)
     auto wait_all = [&](uint64_t *bar, uint32_t &ph) -> bool {
         bool ok = true;
         if (warp == 0) ok = mbar_wait(bar, ph, kWaitLimitNs);
-        ph ^= 1;
-        return __syncthreads_or(!ok) != 0;
+        const bool stop = __syncthreads_or(!ok) != 0;
+        if (!stop) ph ^= 1;
+        return stop;
     };
 
     // thread kMma issues the MMAs, thread kTma (another warp) the TMA loads
@@ -212,9 +214,9 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
         {
             bool ok = true;
             if (warp == 0) ok = mbar_wait(bar_qkg, ph_qkg, kWaitLimitNs) && mbar_wait(bar_v, ph_v, kWaitLimitNs);
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
             ph_qkg ^= 1; ph_v ^= 1;
             if (tid == kTma) qkg_out = v_out = false;
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
         }
 
         // ---------------- P1: gate cumsum, in-warp scan over the 64 rows
