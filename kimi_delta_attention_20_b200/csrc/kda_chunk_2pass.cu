@@ -38,6 +38,8 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <functional>
+#include <queue>
 #include <vector>
 
 #include "kda_common.cuh"
@@ -1332,6 +1334,64 @@ cudaError_t run_pass1(const ChunkParams &p, uint8_t *ws, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// Finish time of pass 2 when its CTAs -- the sequences in the order `ord`, all heads of
+// a sequence in a row -- go in that order to whichever of `slots` SMs frees first (one
+// CTA per SM), a CTA taking one unit per chunk of its sequence (at least one).
+long long dispatch_makespan(const std::vector<int> &ord, const std::vector<long long> &units, int H, int slots) {
+    std::priority_queue<long long, std::vector<long long>, std::greater<long long>> free_at;
+    for (int i = 0; i < slots; ++i) free_at.push(0);
+    long long end = 0;
+    for (int n : ord)
+        for (int h = 0; h < H; ++h) {
+            const long long t = free_at.top() + units[n];
+            free_at.pop();
+            free_at.push(t);
+            end = std::max(end, t);
+        }
+    return end;
+}
+
+// The launch order of pass 2's sequences: longest first, then pairwise swaps that
+// shorten the simulated finish time (few sequences of a few lengths leave a ragged
+// last wave under longest-first: lengths 4096/8192/12288/7168 at H = 96 finish at 368
+// chunk units longest-first and at 352 with 7168 moved ahead of 8192).
+std::vector<int> pass2_order(const int32_t *cu_host, int N, int H, int slots) {
+    std::vector<int> ord(N);
+    std::vector<long long> units(N);
+    for (int i = 0; i < N; ++i) {
+        ord[i] = i;
+        units[i] = std::max<long long>(1, ((long long)cu_host[i + 1] - cu_host[i] + C - 1) / C);
+    }
+    std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return units[a] > units[b]; });
+    if (N < 2 || N > 16 || (long long)N * H <= slots || (long long)N * H > 16384) return ord;
+    // the search (tens of microseconds) runs once per set of lengths on this thread
+    thread_local std::vector<long long> last_units;
+    thread_local std::vector<int> last_ord;
+    thread_local int last_H = -1, last_slots = -1;
+    if (H == last_H && slots == last_slots && units == last_units) return last_ord;
+    long long best = dispatch_makespan(ord, units, H, slots);
+    long long total = 0;
+    for (int i = 0; i < N; ++i) total += units[i] * H;
+    const long long lower = std::max(units[ord[0]], (total + slots - 1) / slots);
+    for (int round = 0; round < 4 && best * 50 > lower * 51; ++round) {  // more than 2 % above the bound
+        bool better = false;
+        for (int i = 0; i < N; ++i)
+            for (int j = i + 1; j < N; ++j) {
+                if (units[ord[i]] == units[ord[j]]) continue;
+                std::swap(ord[i], ord[j]);
+                const long long m = dispatch_makespan(ord, units, H, slots);
+                if (m < best) { best = m; better = true; }
+                else std::swap(ord[i], ord[j]);
+            }
+        if (!better) break;
+    }
+    last_H = H;
+    last_slots = slots;
+    last_units = units;
+    last_ord = ord;
+    return ord;
+}
+
 // pass 2 of p (v, S0, S_out and o as p gives them; o may be null) over the records in ws;
 // s0_identity starts every chain from the identity, v_zero takes v = 0 (p.v is not read)
 cudaError_t run_pass2(const ChunkParams &p, uint8_t *ws, const int32_t *cu_host, cudaStream_t st, int s0_identity = 0,
@@ -1353,16 +1413,16 @@ cudaError_t run_pass2(const ChunkParams &p, uint8_t *ws, const int32_t *cu_host,
     B.o_f32 = o_f32;
     if (!v_zero && !make_map(&B.tv, p.v, total, p.H)) return cudaErrorInvalidValue;
     B.nperm = 0;
-    if (cu_host && p.N <= kMaxPerm) {  // longest sequences first
-        std::vector<int> idx(p.N);
-        for (int i = 0; i < p.N; ++i) idx[i] = i;
-        std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) {
-            return (cu_host[a + 1] - cu_host[a]) > (cu_host[b + 1] - cu_host[b]);
-        });
-        for (int i = 0; i < p.N; ++i) B.perm[i] = idx[i];
+    cudaError_t e;
+    if (cu_host && p.N <= kMaxPerm) {  // the launch order of the sequences (longest first, tail balanced)
+        int dev = 0, nsm = 148;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        const std::vector<int> ord = pass2_order(cu_host, p.N, p.H, nsm);
+        for (int i = 0; i < p.N; ++i) B.perm[i] = ord[i];
         B.nperm = p.N;
     }
-    cudaError_t e = cudaFuncSetAttribute(kda_tp_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2_ALLOC);
+    e = cudaFuncSetAttribute(kda_tp_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2_ALLOC);
     if (e != cudaSuccess) return e;
     kda_tp_state_kernel<<<(unsigned)((long long)p.N * p.H), NT2, SMEM2_ALLOC, st>>>(B);
     return cudaGetLastError();
