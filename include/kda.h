@@ -144,7 +144,10 @@ KDA_API kda_status kda_chunk_fwd(const kda_chunk_args *args, void *stream);
  * One recurrent decode step for N sequences at once: the recurrence above
  * applied to one token per sequence (page "atlas_core/kimi_k3/kda.rs",
  * `kda_recurrent_step`), with the state read, updated and written back IN
- * PLACE (a read-modify-write of [N,H,Dk,Dv] fp32).
+ * PLACE (a read-modify-write of [N,H,Dk,Dv] fp32), or written to `state_out`
+ * when that is given. The out-of-place form serves callers that keep two state
+ * buffers and swap them each step, so the previous state stays intact (page
+ * "memra-engine tests/kda_fixture_gpu.rs", the decode with `state` / `state_alt`).
  */
 typedef struct {
     kda_dtype dtype;      /* dtype of q, k, v, g, beta and o */
@@ -163,6 +166,9 @@ typedef struct {
     const float *A_log;        /* [H] fp32 */
     const float *dt_bias;      /* [H,Dk] fp32 or NULL */
     int beta_is_prob;
+    float *state_out;          /* NULL: state updated in place. Else [N,H,Dk,Dv] fp32 out, 16-byte
+                                * aligned, equal to state or not overlapping it; state is then
+                                * only read */
 } kda_step_args;
 
 KDA_API kda_status kda_recurrent_step(const kda_step_args *args, void *stream);
@@ -202,6 +208,8 @@ typedef struct {
     const float *A_log;   /* [H] fp32, in-kernel gate forms only */
     const float *dt_bias; /* [H,Dk] fp32 or NULL */
     int beta_is_prob;
+    float *state_out;     /* NULL: state updated in place; else as in kda_step_args (the conv
+                           * windows are always updated in place) */
 } kda_token_args;
 
 KDA_API kda_status kda_decode_token(const kda_token_args *args, void *stream);

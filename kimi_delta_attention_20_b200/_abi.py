@@ -61,6 +61,7 @@ class StepArgs(ctypes.Structure):
         ("has_lower_bound", ctypes.c_int), ("lower_bound", ctypes.c_float),
         ("gate_mode", ctypes.c_int), ("A_log", _vp), ("dt_bias", _vp),
         ("beta_is_prob", ctypes.c_int),
+        ("state_out", _vp),
     ]
 
 
@@ -76,6 +77,7 @@ class TokenArgs(ctypes.Structure):
         ("has_lower_bound", ctypes.c_int), ("lower_bound", ctypes.c_float),
         ("gate_mode", ctypes.c_int), ("A_log", _vp), ("dt_bias", _vp),
         ("beta_is_prob", ctypes.c_int),
+        ("state_out", _vp),
     ]
 
 

@@ -8,7 +8,7 @@
 #include "kda_bwd.cuh"
 
 namespace kda {
-cudaError_t launch_decode(const StepParams &p, bool bf16, int Dk, int Dv, cudaStream_t st);
+cudaError_t launch_decode(const StepParams &p, float *state_out, bool bf16, int Dk, int Dv, cudaStream_t st);
 cudaError_t launch_chunk_simt(const ChunkParams &p, bool bf16, int Dk, int Dv, int chunk, cudaStream_t st);
 cudaError_t launch_chunk_rec(const ChunkParams &p, bool bf16, int Dk, int Dv, void *workspace, size_t workspace_bytes,
                              cudaStream_t st);
@@ -23,7 +23,7 @@ bool token_conv_supported(int K);
 size_t bwd_workspace_bytes(bool varlen, long long T, int N, int H, int Dk, int Dv);
 size_t bwd_workspace_bytes_min(bool varlen, long long T, int N, int H, int Dk, int Dv);
 cudaError_t launch_bwd(BwdParams p, bool bf16, int Dk, int Dv, void *workspace, size_t workspace_bytes, cudaStream_t st);
-cudaError_t launch_token(const TokenParams &tp, bool bf16, int Dk, int Dv, cudaStream_t st);
+cudaError_t launch_token(const TokenParams &tp, float *state_out, bool bf16, int Dk, int Dv, cudaStream_t st);
 }  // namespace kda
 
 namespace {
@@ -37,6 +37,16 @@ kda_status cuda_status(cudaError_t e) {
 }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// An out-of-place decode state: 16-byte aligned and either the state itself or
+// disjoint from it (a partial overlap would let one CTA read what another wrote).
+bool state_out_ok(const float *state, const float *out, long long N, int H, int Dk, int Dv) {
+    if (!out || out == state) return true;
+    if (!aligned(out, 16)) return false;
+    const uintptr_t bytes = (uintptr_t)(N * H * (long long)Dk * Dv) * sizeof(float);
+    const uintptr_t a = reinterpret_cast<uintptr_t>(state), b = reinterpret_cast<uintptr_t>(out);
+    return a + bytes <= b || b + bytes <= a;
+}
 
 bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
 
@@ -231,6 +241,7 @@ kda_status kda_recurrent_step(const kda_step_args *a, void *stream) {
         !aligned(a->o, 16) || !aligned(a->state, 16) || !aligned(a->beta, esz))
         return KDA_ERR_INVALID_ARGUMENT;
     if (check_gate_ptrs(a->gate_mode, a->A_log, a->dt_bias) != KDA_OK) return KDA_ERR_INVALID_ARGUMENT;
+    if (!state_out_ok(a->state, a->state_out, a->N, a->H, a->Dk, a->Dv)) return KDA_ERR_INVALID_ARGUMENT;
     kda::StepParams p;
     p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
     p.state = a->state; p.o = a->o; p.N = a->N; p.H = a->H;
@@ -242,7 +253,7 @@ kda_status kda_recurrent_step(const kda_step_args *a, void *stream) {
     p.A_log = a->A_log;
     p.dt_bias = a->dt_bias;
     p.beta_prob = a->beta_is_prob ? 1 : 0;
-    return cuda_status(kda::launch_decode(p, bf16, a->Dk, a->Dv, static_cast<cudaStream_t>(stream)));
+    return cuda_status(kda::launch_decode(p, a->state_out, bf16, a->Dk, a->Dv, static_cast<cudaStream_t>(stream)));
 }
 
 kda_status kda_decode_token(const kda_token_args *a, void *stream) {
@@ -265,6 +276,7 @@ kda_status kda_decode_token(const kda_token_args *a, void *stream) {
         !aligned(a->state, 16))
         return KDA_ERR_INVALID_ARGUMENT;
     if (check_gate_ptrs(a->gate_mode, a->A_log, a->dt_bias) != KDA_OK) return KDA_ERR_INVALID_ARGUMENT;
+    if (!state_out_ok(a->state, a->state_out, a->N, a->H, a->Dk, a->Dv)) return KDA_ERR_INVALID_ARGUMENT;
     kda::TokenParams tp;
     kda::StepParams &p = tp.step;
     p.q = p.k = p.v = nullptr;
@@ -284,7 +296,7 @@ kda_status kda_decode_token(const kda_token_args *a, void *stream) {
     tp.K = a->conv_kernel;
     tp.g_out = a->g_out;
     tp.norm_eps = a->norm_eps;
-    return cuda_status(kda::launch_token(tp, bf16, a->Dk, a->Dv, static_cast<cudaStream_t>(stream)));
+    return cuda_status(kda::launch_token(tp, a->state_out, bf16, a->Dk, a->Dv, static_cast<cudaStream_t>(stream)));
 }
 
 kda_status kda_chunk_bwd_workspace_size(const kda_chunk_bwd_args *a, size_t *bytes) {

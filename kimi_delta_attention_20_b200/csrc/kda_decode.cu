@@ -5,7 +5,8 @@
 // head at 128x128) against ~1 KiB of per-token vectors, so it is bound by HBM
 // bandwidth. Each CTA owns a 32-column slab of one head's state: 128 bytes of
 // every key row, read and written back as float4 with streaming cache hints,
-// kept in registers between the read and the write (one pass over HBM).
+// kept in registers between the read and the write (one pass over HBM). The
+// write goes back in place, or to `state_out` when the caller keeps the old state.
 //
 // g is the log-decay as given (clamped) or formed from the gate input in the
 // kernel; beta a logit or a given probability. Per head, with S' = diag(exp g) S, the two column reductions over the key
@@ -30,7 +31,7 @@ struct DecodeCfg {
 };
 
 template <typename Tin, int DK, int DV>
-__global__ void __launch_bounds__(256) kda_decode_kernel(StepParams p) {
+__global__ void __launch_bounds__(256) kda_decode_kernel(StepParams p, float *state_out) {
     using Cfg = DecodeCfg<Tin, DK, DV>;
     constexpr int NP = Cfg::kPasses, RP = Cfg::kRowsPerPass, NW = Cfg::kWarps;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -39,7 +40,9 @@ __global__ void __launch_bounds__(256) kda_decode_kernel(StepParams p) {
     const int cg = tid & 7;                          // float4 column group in the slab
     const int rg = tid >> 3;                         // first key row of this thread
 
-    float *S = p.state + nh * (long long)(DK * DV) + slab * Cfg::kCols + cg * 4;
+    const long long tile = nh * (long long)(DK * DV) + slab * Cfg::kCols + cg * 4;
+    const float *S = p.state + tile;
+    float *So = (state_out ? state_out : p.state) + tile;
     const int h = nh % p.H;
 
     // The token's vectors first: they are few bytes, but every step after the state
@@ -147,25 +150,25 @@ __global__ void __launch_bounds__(256) kda_decode_kernel(StepParams p) {
             float4 u;
             u.x = fmaf(kc, d0, s[i].x); u.y = fmaf(kc, d1, s[i].y);
             u.z = fmaf(kc, d2, s[i].z); u.w = fmaf(kc, d3, s[i].w);
-            st_stream(reinterpret_cast<float4 *>(S + (long long)c * DV), u);
+            st_stream(reinterpret_cast<float4 *>(So + (long long)c * DV), u);
         }
     }
 }
 
 template <typename Tin, int DK, int DV>
-cudaError_t launch_decode_t(const StepParams &p, cudaStream_t st) {
+cudaError_t launch_decode_t(const StepParams &p, float *state_out, cudaStream_t st) {
     using Cfg = DecodeCfg<Tin, DK, DV>;
     const long long blocks = (long long)p.N * p.H * Cfg::kSlabs;
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    kda_decode_kernel<Tin, DK, DV><<<(unsigned)blocks, Cfg::kThreads, 0, st>>>(p);
+    kda_decode_kernel<Tin, DK, DV><<<(unsigned)blocks, Cfg::kThreads, 0, st>>>(p, state_out);
     return cudaGetLastError();
 }
 
 template <typename Tin>
-cudaError_t launch_decode_dt(const StepParams &p, int Dk, int Dv, cudaStream_t st) {
+cudaError_t launch_decode_dt(const StepParams &p, float *state_out, int Dk, int Dv, cudaStream_t st) {
 #define KDA_DEC_CASE(DK_, DV_) \
-    if (Dk == DK_ && Dv == DV_) return launch_decode_t<Tin, DK_, DV_>(p, st);
+    if (Dk == DK_ && Dv == DV_) return launch_decode_t<Tin, DK_, DV_>(p, state_out, st);
     KDA_DEC_CASE(32, 32) KDA_DEC_CASE(32, 64) KDA_DEC_CASE(32, 128)
     KDA_DEC_CASE(64, 32) KDA_DEC_CASE(64, 64) KDA_DEC_CASE(64, 128)
     KDA_DEC_CASE(128, 32) KDA_DEC_CASE(128, 64) KDA_DEC_CASE(128, 128)
@@ -173,9 +176,9 @@ cudaError_t launch_decode_dt(const StepParams &p, int Dk, int Dv, cudaStream_t s
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_decode(const StepParams &p, bool bf16, int Dk, int Dv, cudaStream_t st) {
-    return bf16 ? launch_decode_dt<__nv_bfloat16>(p, Dk, Dv, st)
-                : launch_decode_dt<float>(p, Dk, Dv, st);
+cudaError_t launch_decode(const StepParams &p, float *state_out, bool bf16, int Dk, int Dv, cudaStream_t st) {
+    return bf16 ? launch_decode_dt<__nv_bfloat16>(p, state_out, Dk, Dv, st)
+                : launch_decode_dt<float>(p, state_out, Dk, Dv, st);
 }
 
 }  // namespace kda

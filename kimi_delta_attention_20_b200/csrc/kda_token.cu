@@ -8,7 +8,8 @@
 // by HBM bandwidth; the conv windows of the head's 2 Dk + Dv channels (6 KiB at
 // K = 4) and the token vectors add about 10 %. Thread (kg, vg) holds rows
 // kg*RP .. kg*RP+RP-1 and columns 4 vg .. 4 vg + 3 of the state as float4 in
-// registers between the read and the write. The per-head steps:
+// registers between the read and the write, which goes back in place or to
+// `state_out` when the caller keeps the old state. The per-head steps:
 //   conv:   window <- (window[1:], x), y = silu(w . window) for q, k, v channels
 //   step:   S' = diag(exp g) S, r_k = S'^T k, r_q = S'^T q (one pass),
 //           delta = sigmoid(beta) (v - r_k / |k|), S = S' + (k/|k|) delta^T,
@@ -24,7 +25,7 @@ constexpr int kTokThreads = 256;
 constexpr int kMaxConv = 8;
 
 template <typename Tin, int DK, int DV>
-__global__ void __launch_bounds__(kTokThreads) kda_token_kernel(TokenParams tp) {
+__global__ void __launch_bounds__(kTokThreads) kda_token_kernel(TokenParams tp, float *state_out) {
     constexpr int NT = kTokThreads, VG = DV / 4, KG = NT / VG, RP = DK / KG, NW = NT / 32;
     static_assert(VG * KG == NT && RP * KG == DK && RP >= 1, "state tiling");
     const StepParams &p = tp.step;
@@ -34,7 +35,9 @@ __global__ void __launch_bounds__(kTokThreads) kda_token_kernel(TokenParams tp) 
     const int H = p.H, h = (int)(nh % H);
     const long long n = nh / H;
 
-    float *S = p.state + nh * (long long)(DK * DV) + 4 * vg;
+    const long long tile = nh * (long long)(DK * DV) + 4 * vg;
+    const float *S = p.state + tile;
+    float *So = (state_out ? state_out : p.state) + tile;
     // the token's gate, beta and output-gate values first (a few bytes each, but the
     // steps after the state read wait on them), raw until used
     const Tin *gop = static_cast<const Tin *>(tp.g_out);
@@ -160,23 +163,23 @@ __global__ void __launch_bounds__(kTokThreads) kda_token_kernel(TokenParams tp) 
         float4 u;
         u.x = fmaf(kc, d0, s[i].x); u.y = fmaf(kc, d1, s[i].y);
         u.z = fmaf(kc, d2, s[i].z); u.w = fmaf(kc, d3, s[i].w);
-        st_stream(reinterpret_cast<float4 *>(S + (long long)c * DV), u);
+        st_stream(reinterpret_cast<float4 *>(So + (long long)c * DV), u);
     }
 }
 
 template <typename Tin, int DK, int DV>
-cudaError_t launch_token_t(const TokenParams &tp, cudaStream_t st) {
+cudaError_t launch_token_t(const TokenParams &tp, float *state_out, cudaStream_t st) {
     const long long blocks = (long long)tp.step.N * tp.step.H;
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    kda_token_kernel<Tin, DK, DV><<<(unsigned)blocks, kTokThreads, 0, st>>>(tp);
+    kda_token_kernel<Tin, DK, DV><<<(unsigned)blocks, kTokThreads, 0, st>>>(tp, state_out);
     return cudaGetLastError();
 }
 
 template <typename Tin>
-cudaError_t launch_token_dt(const TokenParams &tp, int Dk, int Dv, cudaStream_t st) {
+cudaError_t launch_token_dt(const TokenParams &tp, float *state_out, int Dk, int Dv, cudaStream_t st) {
 #define KDA_TOK_CASE(DK_, DV_) \
-    if (Dk == DK_ && Dv == DV_) return launch_token_t<Tin, DK_, DV_>(tp, st);
+    if (Dk == DK_ && Dv == DV_) return launch_token_t<Tin, DK_, DV_>(tp, state_out, st);
     KDA_TOK_CASE(32, 32) KDA_TOK_CASE(32, 64) KDA_TOK_CASE(32, 128)
     KDA_TOK_CASE(64, 32) KDA_TOK_CASE(64, 64) KDA_TOK_CASE(64, 128)
     KDA_TOK_CASE(128, 32) KDA_TOK_CASE(128, 64) KDA_TOK_CASE(128, 128)
@@ -188,8 +191,9 @@ cudaError_t launch_token_dt(const TokenParams &tp, int Dk, int Dv, cudaStream_t 
 
 bool token_conv_supported(int K) { return K >= 1 && K <= kMaxConv; }
 
-cudaError_t launch_token(const TokenParams &tp, bool bf16, int Dk, int Dv, cudaStream_t st) {
-    return bf16 ? launch_token_dt<__nv_bfloat16>(tp, Dk, Dv, st) : launch_token_dt<float>(tp, Dk, Dv, st);
+cudaError_t launch_token(const TokenParams &tp, float *state_out, bool bf16, int Dk, int Dv, cudaStream_t st) {
+    return bf16 ? launch_token_dt<__nv_bfloat16>(tp, state_out, Dk, Dv, st)
+                : launch_token_dt<float>(tp, state_out, Dk, Dv, st);
 }
 
 }  // namespace kda

@@ -196,19 +196,30 @@ def chunk_bwd_workspace_bytes(B, T, H, Dk, Dv, *, dtype=torch.bfloat16, N=None, 
     return nbytes.value
 
 
+def _check_state_out(state: torch.Tensor, state_out: Optional[torch.Tensor]):
+    if state_out is None:
+        return
+    _need_cuda("state_out", state_out)
+    if state_out.dtype != torch.float32 or state_out.shape != state.shape or not state_out.is_contiguous():
+        raise ValueError(f"state_out must be a contiguous float32 tensor of shape {tuple(state.shape)}")
+
+
 def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                    beta: torch.Tensor, state: torch.Tensor, *, A_log: Optional[torch.Tensor] = None,
                    dt_bias: Optional[torch.Tensor] = None, scale: Optional[float] = None,
                    use_qk_l2norm_in_kernel: bool = True, use_gate_in_kernel: bool = False,
                    use_beta_sigmoid_in_kernel: bool = True, safe_gate: bool = False,
                    lower_bound: Optional[float] = None,
-                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                   out: Optional[torch.Tensor] = None,
+                   state_out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """One decode token per sequence (page "atlas_core/kimi_k3/kda.rs",
     `kda_recurrent_step`, which always normalises q and k).
 
     q, k, g: [N, H, Dk]; v: [N, H, Dv]; beta: [N, H] logits (or probabilities
     with use_beta_sigmoid_in_kernel=False); state: [N, H, Dk, Dv] fp32, updated
-    IN PLACE. Gate arguments as in ``chunk_kda``. Returns o [N, H, Dv].
+    IN PLACE, or only read when ``state_out`` (a second fp32 [N, H, Dk, Dv]
+    buffer, disjoint from ``state``) receives the new state. Gate arguments as in
+    ``chunk_kda``. Returns o [N, H, Dv].
     """
     lib = _abi.load()
     for name, t in (("q", q), ("k", k), ("v", v), ("g", g), ("beta", beta), ("state", state)):
@@ -221,11 +232,13 @@ def recurrent_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
         raise ValueError("shape mismatch among q, k, v, g, beta")
     if state.dtype != torch.float32 or state.shape != (N, H, Dk, Dv):
         raise ValueError(f"state must be float32 [{N}, {H}, {Dk}, {Dv}]")
+    _check_state_out(state, state_out)
     o = out if out is not None else torch.empty(N, H, Dv, dtype=q.dtype, device=q.device)
     a = _abi.StepArgs()
     a.dtype = _DTYPES[q.dtype]
     a.N, a.H, a.Dk, a.Dv = N, H, Dk, Dv
     a.q, a.k, a.v, a.g, a.beta, a.state, a.o = (_ptr(t) for t in (q, k, v, g, beta, state, o))
+    a.state_out = _ptr(state_out)
     a.scale = float("nan") if scale is None else float(scale)
     a.use_qk_l2norm = int(bool(use_qk_l2norm_in_kernel))
     _gate_fields(a, q.device, H, Dk, A_log, dt_bias, use_gate_in_kernel, safe_gate, lower_bound,
@@ -242,15 +255,16 @@ def decode_token(x: torch.Tensor, conv_w: torch.Tensor, conv_state: torch.Tensor
                  use_qk_l2norm_in_kernel: bool = True, use_gate_in_kernel: bool = False,
                  use_beta_sigmoid_in_kernel: bool = True, safe_gate: bool = False,
                  lower_bound: Optional[float] = None,
-                 out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                 out: Optional[torch.Tensor] = None,
+                 state_out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """One serving decode token per sequence in one launch (page
     "atlas_core/kimi_k3/kda.rs": `conv_update` + SiLU, `kda_recurrent_step`, and
     `full_rank_output_gate` when ``g_out`` is given).
 
     x: [N, H*(2 Dk + Dv)] pre-conv projections q | k | v; conv_w: [H*(2 Dk + Dv), K]
     fp32; conv_state: [N, H*(2 Dk + Dv), K] fp32, oldest input first, updated IN
-    PLACE; g: [N, H, Dk]; beta: [N, H]; state: [N, H, Dk, Dv] fp32, updated IN PLACE;
-    g_out: [N, H, Dv] or None. ``norm_eps`` is the RMSNorm epsilon of the output
+    PLACE; g: [N, H, Dk]; beta: [N, H]; state: [N, H, Dk, Dv] fp32, updated IN PLACE
+    unless ``state_out`` is given (as in ``recurrent_step``); g_out: [N, H, Dv] or None. ``norm_eps`` is the RMSNorm epsilon of the output
     gate (1e-6 by default, the norm epsilon of the KDA model configs). Gate and beta
     arguments as in ``recurrent_step``. Returns o [N, H, Dv]: the gated, normalised
     output with ``g_out``, else the recurrent step's output.
@@ -280,6 +294,7 @@ def decode_token(x: torch.Tensor, conv_w: torch.Tensor, conv_state: torch.Tensor
         raise ValueError("g must be [N, H, Dk] and beta [N, H]")
     if g_out is not None and g_out.shape != (N, H, Dv):
         raise ValueError(f"g_out must be [{N}, {H}, {Dv}]")
+    _check_state_out(state, state_out)
     for name, t in (("x", x), ("conv_w", conv_w), ("conv_state", conv_state), ("g", g), ("beta", beta),
                     ("state", state)) + ((("g_out", g_out),) if g_out is not None else ()):
         if not t.is_contiguous():
@@ -291,6 +306,7 @@ def decode_token(x: torch.Tensor, conv_w: torch.Tensor, conv_state: torch.Tensor
     a.x, a.conv_w, a.conv_state, a.g, a.beta, a.state, a.o = (
         _ptr(t) for t in (x, conv_w, conv_state, g, beta, state, o))
     a.g_out = _ptr(g_out) if g_out is not None else None
+    a.state_out = _ptr(state_out)
     a.norm_eps = float(norm_eps)
     a.scale = float("nan") if scale is None else float(scale)
     a.use_qk_l2norm = int(bool(use_qk_l2norm_in_kernel))

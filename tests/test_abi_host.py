@@ -141,6 +141,9 @@ def test_workspace_query_reads_shapes_only():
     (dict(state=FAKE + 4), _abi.KDA_ERR_INVALID_ARGUMENT),
     (dict(q=FAKE + 2), _abi.KDA_ERR_INVALID_ARGUMENT),
     (dict(has_lower_bound=1, lower_bound=1.0), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(state_out=FAKE + 0x40000 + 4), _abi.KDA_ERR_INVALID_ARGUMENT),   # misaligned
+    (dict(state_out=FAKE + 1024), _abi.KDA_ERR_INVALID_ARGUMENT),          # overlaps state
+    (dict(state=FAKE + 0x3fc00, state_out=FAKE), _abi.KDA_ERR_INVALID_ARGUMENT),  # state starts inside it
 ])
 def test_recurrent_step_rejects(over, want):
     lib = _abi.load()
@@ -183,6 +186,8 @@ def token_args(**over):
     (dict(g_out=FAKE + 1), _abi.KDA_ERR_INVALID_ARGUMENT),
     (dict(has_lower_bound=1, lower_bound=0.5), _abi.KDA_ERR_INVALID_ARGUMENT),
     (dict(gate_mode=_abi.KDA_GATE_SOFTPLUS), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(state_out=FAKE + 0x40000 + 4), _abi.KDA_ERR_INVALID_ARGUMENT),
+    (dict(state_out=FAKE + 0x3fff0), _abi.KDA_ERR_INVALID_ARGUMENT),
 ])
 def test_decode_token_rejects(over, want):
     lib = _abi.load()

@@ -403,3 +403,32 @@ def test_two_pass_and_single_pass_agree():
     o1, S1 = run_chunk(inp, lower_bound=-5.0, workspace=ws)
     check("2pass vs 1pass o", o2, o1.double().cpu().numpy(), torch.bfloat16)
     check("2pass vs 1pass S", S2, S1.double().cpu().numpy(), torch.bfloat16)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_state_out_ping_pong(dtype):
+    """The out-of-place step (two state buffers swapped each step, page "memra-engine
+    tests/kda_fixture_gpu.rs", `state` / `state_alt`) leaves the old state intact and
+    gives bit for bit the in-place result; both match the oracle."""
+    kda = kda_mod()
+    N, H, Dk, Dv, steps = 4, 3, 128, 64, 5
+    inp = KI.draw_decode(N, H, Dk, Dv, steps, dtype=dtype, seed=21)
+    S_in = inp["state"].to(DEV)
+    S_a, S_b = S_in.clone(), torch.empty_like(S_in)
+    o_in, o_pp = [], []
+    for t in range(steps):
+        args = [inp[n][t].to(DEV) for n in ("q", "k", "v", "g", "beta")]
+        o_in.append(kda.recurrent_step(*args, S_in, lower_bound=-5.0))
+        before = S_a.clone()
+        o_pp.append(kda.recurrent_step(*args, S_a, lower_bound=-5.0, state_out=S_b))
+        torch.cuda.synchronize()
+        assert torch.equal(S_a, before), "the read-only state was written"
+        S_a, S_b = S_b, S_a
+    assert torch.equal(torch.stack(o_in), torch.stack(o_pp))
+    assert torch.equal(S_in, S_a)
+    o = torch.stack(o_pp)
+    for n in range(N):
+        o_ref, S_ref = oracle.recurrent(inp["q"][:, n], inp["k"][:, n], inp["v"][:, n], inp["g"][:, n],
+                                        inp["beta"][:, n], lower_bound=-5.0, initial_state=inp["state"][n:n + 1])
+        check(f"pp o n{n}", o[:, n], o_ref, dtype)
+        check(f"pp S n{n}", S_a[n], S_ref[0], dtype)

@@ -129,3 +129,28 @@ def test_decode_token_production_geometry_sampled():
         check(f"prod o n{n}", o[n:n + 1], o_ref, torch.bfloat16)
         check(f"prod S n{n}", S[n:n + 1], S_ref, torch.bfloat16)
         np.testing.assert_array_equal(cs[n:n + 1].cpu().double().numpy(), cs_ref)
+
+
+def test_decode_token_state_out_ping_pong():
+    """The serving token with the new state written to a second buffer: the old state
+    stays intact and the result is bit for bit the in-place one (conv windows are
+    updated in place either way)."""
+    import kimi_delta_attention_20_b200 as kda
+    N, H, Dk, Dv, K, steps = 3, 2, 128, 128, 4, 4
+    inp = draw(N, H, Dk, Dv, K, steps, torch.bfloat16, seed=9)
+    w_d = inp["w"].to(DEV)
+    cs_in, cs_pp = inp["cs"].clone().to(DEV), inp["cs"].clone().to(DEV)
+    S_in = inp["S0"].clone().to(DEV)
+    S_a, S_b = S_in.clone(), torch.empty_like(S_in)
+    for t in range(steps):
+        args = dict(g_out=inp["g_out"][t].to(DEV), norm_eps=1e-6)
+        x, g, b = inp["x"][t].to(DEV), inp["g"][t].to(DEV), inp["beta"][t].to(DEV)
+        o_in = kda.decode_token(x, w_d, cs_in, g, b, S_in, **args)
+        before = S_a.clone()
+        o_pp = kda.decode_token(x, w_d, cs_pp, g, b, S_a, state_out=S_b, **args)
+        torch.cuda.synchronize()
+        assert torch.equal(S_a, before), "the read-only state was written"
+        assert torch.equal(o_in, o_pp)
+        S_a, S_b = S_b, S_a
+    assert torch.equal(S_in, S_a)
+    assert torch.equal(cs_in, cs_pp)
