@@ -33,6 +33,10 @@
 #ifndef KDA_H_
 #define KDA_H_
 
+/* 0.2.0: kda_step_args and kda_token_args end with `state_out` (0.1.0 had no
+ * such field). */
+#define KDA_VERSION 200
+
 #include <stddef.h>
 #include <stdint.h>
 
@@ -295,7 +299,9 @@ KDA_API const char *kda_status_string(kda_status status);
  * this host thread, 0 if none. */
 KDA_API int kda_last_cuda_error(void);
 
-/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH; equal to KDA_VERSION of
+ * the header the library was built with. A caller built against an older header
+ * passes shorter argument structs, so compare the two before calling. */
 KDA_API int kda_version(void);
 
 #ifdef __cplusplus

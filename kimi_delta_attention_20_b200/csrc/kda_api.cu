@@ -144,7 +144,7 @@ const char *kda_status_string(kda_status s) {
 
 int kda_last_cuda_error(void) { return g_last_cuda_error; }
 
-int kda_version(void) { return 100; }
+int kda_version(void) { return KDA_VERSION; }
 
 kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args *a, size_t *bytes) {
     if (!bytes) return KDA_ERR_INVALID_ARGUMENT;

@@ -26,7 +26,9 @@ def test_library_exports_every_declared_symbol():
     lib = _abi.load()
     for name in declared_symbols():
         assert hasattr(lib, name), name
-    assert lib.kda_version() >= 100
+    with open(os.path.join(ROOT, "include", "kda.h")) as f:
+        header = int(re.search(r"#define KDA_VERSION (\d+)", f.read()).group(1))
+    assert lib.kda_version() == header >= 200
 
 
 def test_status_strings():
