@@ -10,8 +10,11 @@ states out). The decode step workload (64 sequences x 96 heads x 128 x 128
 fp32 state, bf16 token vectors, one fresh token per step) is timed in the
 same run, K' = 256 steps per timed pass, and reported under "decode"; so is the
 serving decode token (conv window 4 + SiLU, the recurrent step and the output
-gate fused, same geometry) under "decode_token", and the chunk_kda backward on the
-B1 T8192 H16 d128 chunk workload under "backward".
+gate fused, same geometry) under "decode_token", the chunk_kda backward on the
+B1 T8192 H16 d128 chunk workload under "backward", and the other chunk workloads
+(twin B4 T2048 H8 d32 with states, B1 T8192 H16 d128 lb -5, one layer of the
+300M model: B128 T2048 H8 d_k 32 d_v 64 with the in-kernel gate) under
+"chunk_workloads", each timed launch by launch with L2 flushed in between.
 Inputs are resident in HBM and larger than L2 (3.9 GB chunk inputs, 384 MiB
 decode state), so no L2 flush runs between iterations.
 
@@ -24,7 +27,8 @@ Multi-GPU (torchrun, one rank per GPU): every rank runs its own replica of
 the workload (no data-path collective; weak scaling); the timed region is
 bracketed by barriers and the slowest rank's device time is reported.
 `--impl reference` times the fp64 CPU oracle on a bounded sample of the same
-workload on the host cores (rank 0 only).
+workload on the host cores (rank 0 only); the main arm's `cpu_baseline` times the
+same sample once, with the chunkwise oracle (form C) timed beside it.
 """
 from __future__ import annotations
 
@@ -49,8 +53,12 @@ DECODE_WL = 3
 DECODE_STEPS_PER_PASS = 256
 # kernels one chunk forward launches on the bench workload (set-up, intra-chunk
 # records, exact records, state pass) and the sources they are built from
-CHUNK_LAUNCHES = 4
 CHUNK_SOURCES = ("kda_chunk_2pass.cu", "kda_tc_util.cuh", "kda_sm100.cuh", "kda_common.cuh")
+# the other chunk workloads, timed one launch at a time with L2 flushed in between
+EXTRA_CHUNK_WLS = (1, 2, 5)
+L2_FLUSH_BYTES = 256 << 20
+# heads of the varlen workload in the CPU oracle's sample (all four sequences)
+CPU_SAMPLE_HEADS = 16
 
 
 def load_peaks():
@@ -108,12 +116,8 @@ def token_algorithmic(N, H, D, K):
 
 
 # chunk_kda backward: the B1 T8192 H16 d128 lb-5 chunk workload with an output and a
-# final-state cotangent. Its 16 (sequence, head) chains run in segment form, 13 kernels
-# per call: segment offsets; pass 1 (prep, intra, exact) and two state passes of the
-# two-pass forward for the segment maps; the forward chain; the transpose and the
-# cotangent offsets; the reverse chain; checkpoint offsets, checkpoints, reverse sweep
+# final-state cotangent (its 16 (sequence, head) chains run in segment form)
 BWD_WL = 2
-BWD_LAUNCHES = 13
 # FP32 FMA peak of the part: 148 SMs x 128 FP32 lanes x 2 flops x 1965 MHz
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
@@ -214,6 +218,25 @@ def ncu_traffic(key, sha):
         return None
 
 
+def launches():
+    """Kernel launches libkda.so has queued so far (its own counter)."""
+    from kimi_delta_attention_20_b200 import _abi
+    return int(_abi.load().kda_launch_count())
+
+
+def bench_config(world):
+    """The `config` object of the JSON line (both arms)."""
+    return {
+        "workload": "chunk_kda fwd: varlen 4096/8192/12288/7168 (T=31744), H=96, d_k=d_v=128, "
+                    "bf16, lower_bound=-5, chunk 64, initial+final states; decode: N=64, H=96, "
+                    "d=128, fp32 state, 256 steps per pass",
+        "tokens_per_step": 31744, "heads": 96, "d_k": 128, "d_v": 128,
+        "chunk_size": 64, "parallelism": f"replica per GPU x{world} (no collective)",
+        "l2": "inputs larger than L2 (3.9 GB chunk inputs, 384 MiB decode state); no flush "
+              "(the smaller chunk workloads flush L2 before every timed launch)",
+    }
+
+
 # --------------------------------------------------------------------------- ranks
 
 def rank_barrier(world):
@@ -261,6 +284,7 @@ def run_kda(args, rank, world, local_rank):
         inp = KI.chunk_inputs(wl, device=dev)
         q, k, v, g, beta = (inp[n] for n in ("q", "k", "v", "g", "beta"))
         S0, cu = inp["initial_state"], inp["cu_seqlens"]
+        cu_cpu = cu.cpu() if cu is not None else None  # host copy: no blocking read per call
         o = torch.empty_like(v)
         S_out = torch.empty(wl.n_seqs, wl.H, wl.Dk, wl.Dv, dtype=torch.float32, device=dev) \
             if wl.final_state else None
@@ -271,7 +295,8 @@ def run_kda(args, rank, world, local_rank):
 
     def chunk_step():
         kda.chunk_kda(q, k, v, g, beta, initial_state=S0, output_final_state=wl.final_state,
-                      cu_seqlens=cu, out=o, final_state_out=S_out, workspace=ws, **opts)
+                      cu_seqlens=cu, cu_seqlens_cpu=cu_cpu, out=o, final_state_out=S_out,
+                      workspace=ws, **opts)
 
     dwl = KI.DECODE_WORKLOADS[DECODE_WL]
     if args.only in (None, "token"):
@@ -346,26 +371,80 @@ def run_kda(args, rank, world, local_rank):
 
     def capture_pass(step_fn):
         """One pass of DECODE_STEPS_PER_PASS decode steps as a CUDA graph, the way a serving
-        engine launches its decode steps: the same kernels, without the launch gaps."""
+        engine launches its decode steps: the same kernels, without the launch gaps.
+        Returns the graph and the number of library kernels it holds."""
         side = torch.cuda.Stream(dev)
         side.wait_stream(torch.cuda.current_stream(dev))
         with torch.cuda.stream(side):
             step_fn(0)
         torch.cuda.current_stream(dev).wait_stream(side)
         graph = torch.cuda.CUDAGraph()
+        n0 = launches()
         with torch.cuda.graph(graph):
             for t in range(DECODE_STEPS_PER_PASS):
                 step_fn(t)
         torch.cuda.synchronize(dev)
-        return graph
+        return graph, launches() - n0
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev) if args.only is None else None
+
+    def time_chunk_workload(idx):
+        """One of the smaller chunk workloads: K launches, each timed by its own events
+        with L2 flushed (a 256 MiB write) before it, the flush outside the events."""
+        xwl = KI.CHUNK_WORKLOADS[idx]
+        xin = KI.chunk_inputs(xwl, device=dev)
+        xo = torch.empty_like(xin["v"])
+        xS = torch.empty(xwl.n_seqs, xwl.H, xwl.Dk, xwl.Dv, dtype=torch.float32, device=dev) \
+            if xwl.final_state else None
+        xopts = chunk_options(xwl, xin)
+        xcu = xin["cu_seqlens"]
+        xcu_cpu = xcu.cpu() if xcu is not None else None
+        xws = torch.empty(max(kda.chunk_workspace_bytes(xwl.B, xwl.T, xwl.H, xwl.Dk, xwl.Dv, N=xwl.n_seqs,
+                                                        varlen=xwl.seqlens is not None), 1),
+                          dtype=torch.uint8, device=dev)
+
+        def step():
+            kda.chunk_kda(xin["q"], xin["k"], xin["v"], xin["g"], xin["beta"], initial_state=xin["initial_state"],
+                          output_final_state=xwl.final_state, cu_seqlens=xcu, cu_seqlens_cpu=xcu_cpu, out=xo,
+                          final_state_out=xS, workspace=xws, **xopts)
+
+        for _ in range(args.warmup):
+            step()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier(); torch.cuda.synchronize(dev)
+        n0 = launches()
+        for a0, a1 in evs:
+            flush.zero_()
+            a0.record(stream)
+            step()
+            a1.record(stream)
+        torch.cuda.synchronize(dev); barrier()
+        n_launch = launches() - n0
+        ms = max_over_ranks(sum(a0.elapsed_time(a1) for a0, a1 in evs)) / args.steps
+        nbytes, nflops = chunk_algorithmic(xwl)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        tflops = nflops / (ms * 1e-3) / 1e12
+        leg = {
+            "workload": xwl.name, "value": whole_job_rate(world, xwl.tokens, ms), "unit": "tokens/s",
+            "ms_per_step": ms, "steps_timed": args.steps, "launches_per_step": n_launch / args.steps,
+            "l2": "flushed before every timed launch",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": gbs / hbm_peak, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": nbytes,
+                         "tensor": {"achieved_tflops": tflops, "peak_tflops": tc_peak,
+                                    "frac": tflops / tc_peak}},
+        }
+        del xin, xo, xS, xws
+        return leg, n_launch
 
     # warm-up (untimed)
     for _ in range(args.warmup):
         chunk_step()
     for t in range(min(args.warmup, dwl.steps)):
         decode_step(t)
-    dec_graph = capture_pass(lambda t: decode_step(t % dwl.steps))
-    tok_graph = capture_pass(token_step)
+    dec_graph, dec_graph_launches = capture_pass(lambda t: decode_step(t % dwl.steps))
+    tok_graph, tok_graph_launches = capture_pass(token_step)
     dec_graph.replay()
     tok_graph.replay()
     torch.cuda.synchronize(dev)
@@ -373,12 +452,14 @@ def run_kda(args, rank, world, local_rank):
     with ClockSampler(gpu_index, args.clocks_log) as clocks:
         # chunk forward: K timed steps
         barrier(); torch.cuda.synchronize(dev)
+        n0 = launches()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.steps):
             chunk_step()
         e1.record(stream)
         torch.cuda.synchronize(dev); barrier()
+        chunk_launches = launches() - n0
         chunk_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
 
         # decode: K passes of 256 steps each
@@ -406,13 +487,21 @@ def run_kda(args, rank, world, local_rank):
         for _ in range(args.warmup):
             bwd_step()
         barrier(); torch.cuda.synchronize(dev)
+        n0 = launches()
         b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         b0.record(stream)
         for _ in range(args.steps):
             bwd_step()
         b1.record(stream)
         torch.cuda.synchronize(dev); barrier()
+        bwd_launches = launches() - n0
         bwd_ms = max_over_ranks(b0.elapsed_time(b1)) / args.steps
+        # the smaller chunk workloads
+        extra_legs, extra_launches = {}, 0
+        for idx in EXTRA_CHUNK_WLS:
+            leg, n_launch = time_chunk_workload(idx)
+            extra_legs[str(idx)] = leg
+            extra_launches += n_launch
     clk = clocks.summary()
 
     # end to end through the public API with host buffers: every step copies its inputs
@@ -446,7 +535,8 @@ def run_kda(args, rank, world, local_rank):
                 s_c.wait_event(ev_read[b])  # step i - 2's outputs have been copied back
             kda.chunk_kda(dbuf[b]["q"], dbuf[b]["k"], dbuf[b]["v"], dbuf[b]["g"], dbuf[b]["beta"],
                           initial_state=dbuf[b]["initial_state"], output_final_state=True,
-                          cu_seqlens=cu_dev[b], out=dout[b][0], final_state_out=dout[b][1], workspace=ws, **opts)
+                          cu_seqlens=cu_dev[b], cu_seqlens_cpu=cu_host, out=dout[b][0],
+                          final_state_out=dout[b][1], workspace=ws, **opts)
             ev_done[b].record(s_c)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_done[b])
@@ -491,14 +581,7 @@ def run_kda(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; shapes and distributions of the varlen chunk and decode workloads)",
-        "config": {
-            "workload": "chunk_kda fwd: varlen 4096/8192/12288/7168 (T=31744), H=96, d_k=d_v=128, "
-                        "bf16, lower_bound=-5, chunk 64, initial+final states; decode: N=64, H=96, "
-                        "d=128, fp32 state, 256 steps per pass",
-            "tokens_per_step": wl.tokens, "heads": wl.H, "d_k": wl.Dk, "d_v": wl.Dv,
-            "chunk_size": wl.chunk_size, "parallelism": f"replica per GPU x{world} (no collective)",
-            "l2": "inputs larger than L2 (3.9 GB chunk inputs, 384 MiB decode state); no flush",
-        },
+        "config": bench_config(world),
         "roofline": {
             "bound": "hbm", "achieved": chunk_gbs, "peak": hbm_peak, "unit": "GB/s",
             "frac": chunk_gbs / hbm_peak, "peak_kind": peak_kind,
@@ -543,61 +626,88 @@ def run_kda(args, rank, world, local_rank):
         "e2e": {"value": whole_job_rate(world, wl.tokens, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "pipelined": "copy-in, compute and copy-back of consecutive steps on three streams"},
-        "gpu_launches": args.steps * (CHUNK_LAUNCHES + 2 * DECODE_STEPS_PER_PASS + BWD_LAUNCHES),
+        "chunk_workloads": extra_legs,
+        "gpu_launches": chunk_launches + args.steps * (dec_graph_launches + tok_graph_launches)
+        + bwd_launches + extra_launches,
+        "gpu_launches_by_leg": {"chunk": chunk_launches, "decode": args.steps * dec_graph_launches,
+                                "decode_token": args.steps * tok_graph_launches, "backward": bwd_launches,
+                                "chunk_workloads": extra_launches,
+                                "counted_by": "libkda.so's own launch counter (kda_launch_count); graph "
+                                              "replays count the kernels captured in the graph"},
         "clocks": clk,
         "library": os.path.relpath(_abi.LIB_PATH, ROOT),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(inp, wl)
+        result["cpu_baseline"] = cpu_baseline(wl)
     return result
 
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def cpu_baseline(inp, wl, heads=24):
-    """Time the fp64 oracle (form R, as it stands) on a bounded sample of the
-    chunk workload: all four sequences, the first `heads` heads."""
+def cpu_sample(wl, heads=CPU_SAMPLE_HEADS):
+    """The CPU oracle's sample of the varlen chunk workload: the same recipe (lengths,
+    dims, dtype, distributions, seed) drawn on the host for the first `heads` heads."""
+    import kda_inputs as KI
+    return KI.draw_chunk(1, wl.T, heads, wl.Dk, wl.Dv, dtype=wl.dtype, seed=wl.seed,
+                         seqlens=wl.seqlens, init_state=wl.init_state)
+
+
+def time_oracle(inp, wl, form):
+    """Seconds the fp64 oracle (as it stands) takes for the sample, on all host cores."""
     import oracle
-    nthreads = os.cpu_count() or 1
-    sl = lambda x: x[0][:, :heads].cpu()
-    q, k, v, g, beta = (sl(inp[n]) for n in ("q", "k", "v", "g", "beta"))
-    S0 = inp["initial_state"][:, :heads].cpu()
-    cu = inp["cu_seqlens"].cpu()
+    fn = {"R": oracle.recurrent, "C": oracle.chunkwise}[form]
     t0 = time.perf_counter()
-    oracle.recurrent(q, k, v, g, beta, initial_state=S0, cu_seqlens=cu,
-                     lower_bound=wl.lower_bound, nthreads=nthreads)
-    dt = time.perf_counter() - t0
-    tok_heads = wl.tokens * heads
-    return {"value": tok_heads / wl.H / dt, "unit": "tokens/s", "cores": nthreads,
+    fn(inp["q"][0], inp["k"][0], inp["v"][0], inp["g"][0], inp["beta"][0],
+       initial_state=inp["initial_state"], cu_seqlens=inp["cu_seqlens"], lower_bound=wl.lower_bound,
+       nthreads=os.cpu_count() or 1)
+    return time.perf_counter() - t0
+
+
+def sample_rate(wl, heads, seconds):
+    """tokens/s of the whole workload implied by the sample: it holds `heads` of wl.H heads."""
+    return wl.tokens * heads / wl.H / seconds
+
+
+def cpu_baseline(wl, heads=CPU_SAMPLE_HEADS):
+    """The oracle timed on the sample: form R (the definition, the baseline) and form C
+    (the chunkwise oracle) beside it."""
+    inp = cpu_sample(wl, heads)
+    tR = time_oracle(inp, wl, "R")
+    tC = time_oracle(inp, wl, "C")
+    return {"value": sample_rate(wl, heads, tR), "unit": "tokens/s", "cores": os.cpu_count() or 1,
             "kind": "oracle",
-            "sample": f"fp64 form R on all {wl.n_seqs} sequences ({wl.tokens} tokens) x {heads} of "
-                      f"{wl.H} heads; {tok_heads} token-heads in {dt:.1f} s, scaled to tokens of "
-                      f"all {wl.H} heads"}
+            "sample": f"fp64 form R (token recurrence) on all {wl.n_seqs} sequences ({wl.tokens} tokens) x "
+                      f"{heads} of {wl.H} heads in {tR:.2f} s, scaled to tokens of all {wl.H} heads",
+            "form_c": {"value": sample_rate(wl, heads, tC), "unit": "tokens/s", "seconds": tC,
+                       "kind": "oracle (chunkwise form, chunk 64)"}}
 
 
 def run_reference(args):
+    """The reference arm: the fp64 CPU oracle, each step one run of form R over the
+    sample. ms_per_step is the measured wall time of that run; `value` is the rate of
+    the whole workload that it implies."""
     import kda_inputs as KI
     wl = KI.CHUNK_WORKLOADS[CHUNK_WL]
-    heads = 4
-    # the same recipe (lengths, dims, dtype, distributions) drawn for `heads` heads only,
-    # so the host does not materialise the 96-head tensors
-    inp = KI.draw_chunk(1, wl.T, heads, wl.Dk, wl.Dv, dtype=wl.dtype, seed=wl.seed,
-                        seqlens=wl.seqlens, init_state=True)
+    heads = CPU_SAMPLE_HEADS
+    inp = cpu_sample(wl, heads)
     for _ in range(args.warmup):
-        pass  # the oracle has no warm-up state; warm-up steps are no-ops
-    vals = []
-    for _ in range(args.steps):
-        vals.append(cpu_baseline(inp, wl, heads=heads))
-    v = statistics.median(x["value"] for x in vals)
+        pass  # the oracle keeps no state between runs: warm-up steps are no-ops
+    secs = [time_oracle(inp, wl, "R") for _ in range(args.steps)]
+    per_step = statistics.mean(secs)
+    v = sample_rate(wl, heads, per_step)
+    tC = time_oracle(inp, wl, "C")
     return {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": wl.tokens / v * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "chunk_kda fwd: varlen 4096/8192/12288/7168, H=96, d=128, "
-                               "lower_bound=-5 (CPU oracle on a 4-head sample per step)"},
-        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["cores"],
-                         "kind": "oracle", "sample": vals[0]["sample"]},
+        "ms_per_step": per_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": bench_config(1),
+        "step": f"form R over all {wl.n_seqs} sequences x {heads} of {wl.H} heads; the whole workload "
+                f"would take {per_step * wl.H / heads * 1e3:.0f} ms",
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": os.cpu_count() or 1, "kind": "oracle",
+                         "sample": f"fp64 form R on all {wl.n_seqs} sequences ({wl.tokens} tokens) x {heads} "
+                                   f"of {wl.H} heads per step, {per_step:.2f} s per step",
+                         "form_c": {"value": sample_rate(wl, heads, tC), "unit": "tokens/s", "seconds": tC,
+                                    "kind": "oracle (chunkwise form, chunk 64)"}},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

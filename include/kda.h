@@ -18,8 +18,9 @@
  * Conventions shared by every entry point:
  *  - Every buffer is caller-owned DEVICE memory, except the fields whose
  *    names end in `_host`. The library allocates nothing, frees nothing and
- *    never synchronises; work is queued on the caller's stream (a
- *    cudaStream_t passed as `void *`; NULL is the legacy default stream).
+ *    never synchronises (except the two *_status queries, which exist to
+ *    wait); work is queued on the caller's stream (a cudaStream_t passed as
+ *    `void *`; NULL is the legacy default stream).
  *  - Tensors are dense, row-major, in the layouts given per field. Data
  *    pointers must be 16-byte aligned (beta: 2-byte aligned for bf16,
  *    4-byte for fp32). Outputs must not alias inputs (except where stated).
@@ -33,9 +34,10 @@
 #ifndef KDA_H_
 #define KDA_H_
 
-/* 0.2.0: kda_step_args and kda_token_args end with `state_out` (0.1.0 had no
- * such field). */
-#define KDA_VERSION 200
+/* 0.3.0: kda_chunk_args ends with `debug_flags`; kda_chunk_fwd_status,
+ * kda_chunk_fwd_noalloc_status and kda_launch_count added. 0.2.0: kda_step_args and kda_token_args
+ * end with `state_out` (0.1.0 had no such field). */
+#define KDA_VERSION 300
 
 #include <stddef.h>
 #include <stdint.h>
@@ -123,7 +125,16 @@ typedef struct {
     const float *A_log;        /* [H] fp32, in-kernel gate forms only */
     const float *dt_bias;      /* [H,Dk] fp32 or NULL, in-kernel gate forms only */
     int beta_is_prob;          /* 1: beta is used as given (no sigmoid) */
+    unsigned int debug_flags;  /* 0 in normal use; KDA_DEBUG_* bits exercise failure paths */
 } kda_chunk_args;
+
+/* debug_flags bit for tests of the bounded device waits: the tensor-core forward
+ * (bf16, Dk = Dv = 128, 64-token chunks) does not issue the first input copy of
+ * its first kernel, so that kernel's first wait gives up after its 2 s limit, its
+ * CTAs leave cleanly and the status word reads KDA_ERR_TIMEOUT (see
+ * kda_chunk_fwd_status). The outputs of such a call are undefined. Other shapes
+ * ignore the bit. */
+#define KDA_DEBUG_STALL_FIRST_WAIT 1u
 
 /* Bytes of device workspace with which kda_chunk_fwd runs its fastest kernel
  * for these arguments (may be 0). Only shapes, dtype and flags are read;
@@ -141,8 +152,26 @@ typedef struct {
  * rounding). */
 KDA_API kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args *args, size_t *bytes);
 
-/* Queue the chunkwise forward on `stream`. Returns KDA_OK once queued. */
+/* Queue the chunkwise forward on `stream`. Returns KDA_OK once queued.
+ *
+ * Device-side failure: the tensor-core kernels (bf16, Dk = Dv = 128, 64-token
+ * chunks) wait on their own copies and products with a 2 s limit per wait. A wait
+ * that gives up makes its CTA drain what it has in flight, free its tensor memory
+ * and leave, and sets the first int32 of the workspace to 1 (it is cleared to 0 at
+ * the start of every call); o and final_state are then partly written. Because
+ * kda_chunk_fwd never synchronises it cannot return KDA_ERR_TIMEOUT itself: call
+ * kda_chunk_fwd_status with the same arguments to read the word. Other shapes run
+ * kernels without device waits. */
 KDA_API kda_status kda_chunk_fwd(const kda_chunk_args *args, void *stream);
+
+/* Outcome of the last kda_chunk_fwd queued with these arguments on `stream`:
+ * waits for the stream to drain (cudaStreamSynchronize), then returns
+ * KDA_ERR_TIMEOUT if a bounded device wait gave up (the status word, the first
+ * int32 of args->workspace, is non-zero), KDA_OK if it is zero or the arguments
+ * select a kernel without device waits, KDA_ERR_CUDA if the copy or the
+ * synchronisation failed. The one entry point that synchronises; it reads 4 bytes
+ * and launches nothing. */
+KDA_API kda_status kda_chunk_fwd_status(const kda_chunk_args *args, void *stream);
 
 /*
  * One recurrent decode step for N sequences at once: the recurrence above
@@ -289,8 +318,20 @@ KDA_API kda_status kda_chunk_bwd(const kda_chunk_bwd_args *args, void *stream);
  *  - Every call on a device shares the one array, which keeps the last call's
  *    contents; the library clears what must start at zero. Calls whose work
  *    overlaps on the GPU (different streams, no ordering) race on it: order them.
+ *  - The array's address is looked up on every call, so a device reset (which
+ *    reloads the library's device code) does not leave a stale address behind.
+ *  - The status word of the bounded device waits (see kda_chunk_fwd) lives in
+ *    that array, out of the caller's reach: read it with
+ *    kda_chunk_fwd_noalloc_status.
  */
 KDA_API kda_status kda_chunk_fwd_noalloc(const kda_chunk_args *args, void *stream);
+
+/* kda_chunk_fwd_status for the allocation-free entry point: synchronises
+ * `stream`, then reports whether a bounded device wait of the last
+ * kda_chunk_fwd_noalloc with these arguments on this device gave up
+ * (KDA_ERR_TIMEOUT), or KDA_OK. Calls on other streams since then may have
+ * overwritten the word. */
+KDA_API kda_status kda_chunk_fwd_noalloc_status(const kda_chunk_args *args, void *stream);
 
 /* Static, human-readable name of a status. */
 KDA_API const char *kda_status_string(kda_status status);
@@ -298,6 +339,12 @@ KDA_API const char *kda_status_string(kda_status status);
 /* CUDA error code (cudaError_t as int) of the last KDA_ERR_CUDA returned on
  * this host thread, 0 if none. */
 KDA_API int kda_last_cuda_error(void);
+
+/* Kernel launches the library has queued since it was loaded, over all host
+ * threads and devices: a diagnostic for benchmarks, which read it before and
+ * after a timed region. A launch recorded into a CUDA graph counts once, when it
+ * is captured, not when the graph is replayed. */
+KDA_API unsigned long long kda_launch_count(void);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH; equal to KDA_VERSION of
  * the header the library was built with. A caller built against an older header

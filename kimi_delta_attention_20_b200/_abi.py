@@ -25,6 +25,8 @@ KDA_GATE_LOG = 0
 KDA_GATE_SOFTPLUS = 1
 KDA_GATE_SAFE = 2
 
+KDA_DEBUG_STALL_FIRST_WAIT = 1
+
 _vp = ctypes.c_void_p
 _fp = ctypes.POINTER(ctypes.c_float)
 _i32p = ctypes.POINTER(ctypes.c_int32)
@@ -47,6 +49,7 @@ class ChunkArgs(ctypes.Structure):
         ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t),
         ("gate_mode", ctypes.c_int), ("A_log", _vp), ("dt_bias", _vp),
         ("beta_is_prob", ctypes.c_int),
+        ("debug_flags", ctypes.c_uint),
     ]
 
 
@@ -102,9 +105,10 @@ class BwdArgs(ctypes.Structure):
 
 
 # every symbol include/kda.h declares
-EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_noalloc",
+EXPORTS = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_status",
+           "kda_chunk_fwd_noalloc", "kda_chunk_fwd_noalloc_status",
            "kda_recurrent_step", "kda_decode_token", "kda_chunk_bwd_workspace_size", "kda_chunk_bwd",
-           "kda_status_string", "kda_last_cuda_error", "kda_version")
+           "kda_status_string", "kda_last_cuda_error", "kda_launch_count", "kda_version")
 
 _lib = None
 
@@ -125,6 +129,9 @@ def load():
     lib.kda_chunk_fwd.restype = ctypes.c_int
     lib.kda_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(ChunkArgs), _vp]
     lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
+    for name in ("kda_chunk_fwd_status", "kda_chunk_fwd_noalloc_status"):
+        getattr(lib, name).argtypes = [ctypes.POINTER(ChunkArgs), _vp]
+        getattr(lib, name).restype = ctypes.c_int
     lib.kda_recurrent_step.argtypes = [ctypes.POINTER(StepArgs), _vp]
     lib.kda_recurrent_step.restype = ctypes.c_int
     lib.kda_decode_token.argtypes = [ctypes.POINTER(TokenArgs), _vp]
@@ -137,6 +144,8 @@ def load():
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_last_cuda_error.argtypes = []
     lib.kda_last_cuda_error.restype = ctypes.c_int
+    lib.kda_launch_count.argtypes = []
+    lib.kda_launch_count.restype = ctypes.c_ulonglong
     lib.kda_version.argtypes = []
     lib.kda_version.restype = ctypes.c_int
     _lib = lib

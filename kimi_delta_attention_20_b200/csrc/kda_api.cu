@@ -3,6 +3,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/kda.h"
 #include "kda_common.cuh"
 #include "kda_bwd.cuh"
@@ -98,6 +100,19 @@ kda_status check_chunk_shape(const kda_chunk_args *a, int *N_out) {
 
 namespace kda {
 void record_cuda_error(int e) { g_last_cuda_error = e; }
+
+std::atomic<unsigned long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+// The status word at `word` (device memory) once `st` has drained: non-zero means a
+// bounded device wait gave up.
+kda_status read_status_word(const void *word, cudaStream_t st) {
+    int v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, word, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_status(e);
+    return v ? KDA_ERR_TIMEOUT : KDA_OK;
+}
 }  // namespace kda
 
 namespace {
@@ -146,6 +161,8 @@ int kda_last_cuda_error(void) { return g_last_cuda_error; }
 
 int kda_version(void) { return KDA_VERSION; }
 
+unsigned long long kda_launch_count(void) { return kda::g_launches.load(std::memory_order_relaxed); }
+
 kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args *a, size_t *bytes) {
     if (!bytes) return KDA_ERR_INVALID_ARGUMENT;
     int N = 0;
@@ -193,7 +210,7 @@ kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
     }
     if (!a->cu_seqlens && a->cu_seqlens_host) return KDA_ERR_INVALID_ARGUMENT;
 
-    kda::ChunkParams p;
+    kda::ChunkParams p{};
     p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta; p.o = a->o;
     p.S0 = a->initial_state; p.S_out = a->final_state;
     p.cu_seqlens = a->cu_seqlens; p.T = a->T; p.N = N; p.H = a->H;
@@ -205,6 +222,7 @@ kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
     p.A_log = a->A_log;
     p.dt_bias = a->dt_bias;
     p.beta_prob = a->beta_is_prob ? 1 : 0;
+    p.stall_first_wait = (a->debug_flags & KDA_DEBUG_STALL_FIRST_WAIT) ? 1 : 0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     if (ntok > 0 && kda::chunk_tc_supported(bf16, a->Dk, a->Dv, a->chunk_size)) {
@@ -222,6 +240,16 @@ kda_status kda_chunk_fwd(const kda_chunk_args *a, void *stream) {
     // request runs the chunked CUDA-core kernel with C = 32 (same result)
     if (a->chunk_size == 32) return cuda_status(kda::launch_chunk_simt(p, bf16, a->Dk, a->Dv, 32, st));
     return cuda_status(kda::launch_chunk_rec(p, bf16, a->Dk, a->Dv, a->workspace, a->workspace_bytes, st));
+}
+
+kda_status kda_chunk_fwd_status(const kda_chunk_args *a, void *stream) {
+    if (!a) return KDA_ERR_INVALID_ARGUMENT;
+    size_t need = 0;
+    kda_status s = kda::chunk_workspace_min_bytes(a, &need);
+    if (s != KDA_OK) return s;
+    if (need == 0) return KDA_OK;  // a kernel without device waits
+    if (!a->workspace) return KDA_ERR_WORKSPACE;
+    return kda::read_status_word(a->workspace, static_cast<cudaStream_t>(stream));
 }
 
 kda_status kda_recurrent_step(const kda_step_args *a, void *stream) {

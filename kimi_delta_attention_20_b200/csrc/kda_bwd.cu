@@ -689,9 +689,11 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st) {
     if ((e = cudaFuncSetAttribute(rev, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_b)) != cudaSuccess)
         return e;
     if (p.cu_seqlens) {
+        count_launch();
         kda_bwd_offsets<<<1, 32, 0, st>>>(p.cu_seqlens, p.N, p.ckpt_off);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
+    count_launch();
     kda_bwd_ckpt_kernel<Tin, DK, DV><<<(unsigned)(heads * NS), 2 * kGrp, smem_f, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -706,6 +708,7 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    count_launch();
     return cudaLaunchKernelEx(&cfg, rev, p);
 }
 
@@ -907,6 +910,7 @@ cudaError_t bwd_segments(const BwdParams &p, bool bf16, int P, const BwdSegLayou
     const long long nst = (long long)q.N * q.H;
     cudaError_t e;
     // segments of whole 64-token chunks for the two-pass kernel, of 16-token stretches otherwise
+    count_launch();
     kda_seg_setup<<<(p.N + 255) / 256, 256, 0, st>>>(p.cu_seqlens, p.T, p.N, P, tc ? 64 : 16, cu_v);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // the forward maps and w, then the entering states
@@ -925,8 +929,10 @@ cudaError_t bwd_segments(const BwdParams &p, bool bf16, int P, const BwdSegLayou
     }
     if ((e = seg_chain_launch<D>(p.S0, M, Nf, ld, pitch, S_start, nullptr, p.N, p.H, P, st)) != cudaSuccess) return e;
     // the cotangent maps M^T and N', then the leaving cotangents and the initial-state gradient
+    count_launch();
     kda_seg_transpose<D><<<(unsigned)(nst * (D / 32) * (D / 32)), 256, 0, st>>>(M, ld, pitch, MT);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    count_launch();
     if (bf16)
         kda_seg_cot_offset<__nv_bfloat16, D><<<dim3((unsigned)nst, D / 32), 256, 0, st>>>(
             w, wstride, static_cast<const __nv_bfloat16 *>(p.dout), cu_v, Nrev, p.H);

@@ -251,7 +251,8 @@ __global__ void __launch_bounds__(NT1, 2) kda_tp_intra_kernel(const __grid_const
     long long item = blockIdx.x;
     Item cur;
     bool have = decode_item(P, item, nch, cur);
-    if (have && tid == kTma) { issue_in(cur); in_out = true; }
+    // (a test of the bounded waits leaves the first copy unissued: the first wait gives up)
+    if (have && tid == kTma && !p.stall_first_wait) { issue_in(cur); in_out = true; }
     unsigned short beta_raw = (have && tid < C) ? load_beta(cur) : (unsigned short)0;
 
     while (have) {
@@ -1318,6 +1319,7 @@ cudaError_t run_pass1(const ChunkParams &p, uint8_t *ws, cudaStream_t st) {
 
     cudaError_t e = cudaMemsetAsync(ws, 0, 256, st);
     if (e != cudaSuccess) return e;
+    count_launch();
     kda_tp_prep<<<1, 1024, 0, st>>>(consts, p.cu_seqlens, p.N, chunk_off, chunk_tok);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     int dev = 0, nsm = 148;
@@ -1326,10 +1328,12 @@ cudaError_t run_pass1(const ChunkParams &p, uint8_t *ws, cudaStream_t st) {
     e = cudaFuncSetAttribute(kda_tp_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM1_ALLOC);
     if (e != cudaSuccess) return e;
     const long long grid1 = std::min<long long>(n_items, 2LL * nsm);
+    count_launch();
     kda_tp_intra_kernel<<<(unsigned)grid1, NT1, SMEM1_ALLOC, st>>>(A);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_tp_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEMX_BYTES);
     if (e != cudaSuccess) return e;
+    count_launch();
     kda_tp_exact_kernel<<<(unsigned)std::min<long long>(n_items, nsm), NTX, SMEMX_BYTES, st>>>(A);
     return cudaGetLastError();
 }
@@ -1424,6 +1428,7 @@ cudaError_t run_pass2(const ChunkParams &p, uint8_t *ws, const int32_t *cu_host,
     }
     e = cudaFuncSetAttribute(kda_tp_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM2_ALLOC);
     if (e != cudaSuccess) return e;
+    count_launch();
     kda_tp_state_kernel<<<(unsigned)((long long)p.N * p.H), NT2, SMEM2_ALLOC, st>>>(B);
     return cudaGetLastError();
 }
@@ -1510,6 +1515,7 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     cursor += seg_state_bytes(p, P);
     float *Sbuf = reinterpret_cast<float *>(cursor);
 
+    count_launch();
     kda_seg_setup<<<(p.N + 255) / 256, 256, 0, st>>>(p.cu_seqlens, p.T, p.N, P, C, cu_v);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = run_pass1(q, ws, st)) != cudaSuccess) return e;

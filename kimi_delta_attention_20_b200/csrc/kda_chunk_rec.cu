@@ -315,6 +315,7 @@ cudaError_t launch_rec_t(const ChunkParams &p, cudaStream_t st) {
     auto kern = kda_chunk_rec_kernel<Tin, DK, DV, AUG, CB>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    count_launch();
     kern<<<dim3((unsigned)blocks, DV / CB), RecCfg<DK, CB>::NT, smem, st>>>(p);
     return cudaGetLastError();
 }
@@ -461,6 +462,7 @@ cudaError_t launch_rec_seg(const ChunkParams &p, int P, uint8_t *ws, cudaStream_
     q.S_out = saug;
     q.o = oaug;
     cudaError_t e;
+    count_launch();
     kda_seg_setup<<<(p.N + 255) / 256, 256, 0, st>>>(p.cu_seqlens, p.T, p.N, P, 16, cu_v);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_rec_t<Tin, D, 2 * D, true>(q, st)) != cudaSuccess) return e;
@@ -468,6 +470,7 @@ cudaError_t launch_rec_seg(const ChunkParams &p, int P, uint8_t *ws, cudaStream_
         cudaSuccess)
         return e;
     const dim3 fgrid((unsigned)((long long)q.N * p.H), (unsigned)rec_fix_tiles(p, P));
+    count_launch();
     kda_rec_seg_fixup<Tin, D><<<fgrid, 128, 0, st>>>(oaug, sstart, cu_v, static_cast<Tin *>(p.o), p.H);
     return cudaGetLastError();
 }

@@ -221,6 +221,7 @@ cudaError_t launch_simt_t(const ChunkParams &p, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
+    count_launch();
     kern<<<(unsigned)blocks, Cfg::kThreads, Cfg::kSmemBytes, st>>>(p);
     return cudaGetLastError();
 }

@@ -184,7 +184,8 @@ __global__ void __launch_bounds__(NT, 1) kda_chunk_tc_kernel(const __grid_consta
     uint32_t ph_qkg = 0, ph_v = 0, ph_mma = 0;
     bool qkg_out = false, v_out = false, mma_out = false;  // outstanding async work of this thread
     bool aborted = false;
-    if (tid == kTma && nchunks > 0) { issue_qkg(bos); issue_v(bos); qkg_out = v_out = true; }
+    // (a test of the bounded waits leaves the first copies unissued: the first wait gives up)
+    if (tid == kTma && nchunks > 0 && !p.stall_first_wait) { issue_qkg(bos); issue_v(bos); qkg_out = v_out = true; }
 
     const long long sbase_state = ((long long)n * H + h) * D * D;
     const __nv_bfloat16 *bt = static_cast<const __nv_bfloat16 *>(p.beta);
@@ -814,6 +815,7 @@ cudaError_t launch_chunk_tc(const ChunkParams &p, int, int, void *workspace, siz
     e = cudaFuncSetAttribute(kda_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     const long long blocks = (long long)p.N * p.H;
+    count_launch();
     kda_chunk_tc_kernel<<<(unsigned)blocks, NT, SMEM_ALLOC, st>>>(P);
     return cudaGetLastError();
 }

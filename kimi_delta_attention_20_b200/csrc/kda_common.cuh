@@ -7,6 +7,9 @@
 
 namespace kda {
 
+// Counts one kernel launch queued by the library (kda_launch_count of the C ABI).
+void count_launch();
+
 constexpr float kL2Eps = 1e-6f;  // x / sqrt(sum x^2 + 1e-6), "atlas_core/kimi_k3/kda.rs" l2norm_rows
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
@@ -68,6 +71,7 @@ struct ChunkParams {
     const float *A_log;         // [H], in-kernel gate forms
     const float *dt_bias;       // [H, Dk] or null
     int beta_prob;              // 1: beta is a probability
+    int stall_first_wait;       // test of the bounded waits: the first input copy is not issued
 };
 
 // Launch parameters of the recurrent decode step.

@@ -161,6 +161,7 @@ cudaError_t launch_decode_t(const StepParams &p, float *state_out, cudaStream_t 
     const long long blocks = (long long)p.N * p.H * Cfg::kSlabs;
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    count_launch();
     kda_decode_kernel<Tin, DK, DV><<<(unsigned)blocks, Cfg::kThreads, 0, st>>>(p, state_out);
     return cudaGetLastError();
 }

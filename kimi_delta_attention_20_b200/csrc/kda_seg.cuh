@@ -150,6 +150,7 @@ cudaError_t seg_chain_launch(const float *S0, const float *M, const float *Nst, 
     cudaError_t e = cudaFuncSetAttribute(kda_seg_chain<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sizeof(SegChainSmem<D>));
     if (e != cudaSuccess) return e;
+    count_launch();
     kda_seg_chain<D><<<(unsigned)((long long)N * H * (D / 16)), SegChainCfg<D>::NT, sizeof(SegChainSmem<D>), st>>>(
         S0, M, Nst, ld, pitch, S_start, S_out, N, H, P, rev);
     return cudaGetLastError();

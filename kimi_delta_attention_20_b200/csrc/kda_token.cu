@@ -172,6 +172,7 @@ cudaError_t launch_token_t(const TokenParams &tp, float *state_out, cudaStream_t
     const long long blocks = (long long)tp.step.N * tp.step.H;
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    count_launch();
     kda_token_kernel<Tin, DK, DV><<<(unsigned)blocks, kTokThreads, 0, st>>>(tp, state_out);
     return cudaGetLastError();
 }

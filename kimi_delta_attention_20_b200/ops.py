@@ -33,6 +33,39 @@ def _stream(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+def _seqlens(cu_seqlens, cu_seqlens_cpu, device):
+    """Device and host copies of the varlen offsets (int32, [N + 1]).
+
+    The library validates the offsets and orders its work from the host copy
+    during the call, and its kernels read the device copy. A CPU ``cu_seqlens``
+    is that host copy and goes to the device by an asynchronous copy from pinned
+    memory; a CUDA ``cu_seqlens`` with ``cu_seqlens_cpu`` (its host copy) costs no
+    copy at all. Only a CUDA ``cu_seqlens`` without a host copy needs a blocking
+    device-to-host read, which stalls the host until the stream reaches it.
+    """
+    if cu_seqlens is None:
+        if cu_seqlens_cpu is not None:
+            raise ValueError("cu_seqlens_cpu needs cu_seqlens")
+        return None, None
+    if cu_seqlens_cpu is not None:
+        if cu_seqlens_cpu.is_cuda:
+            raise ValueError("cu_seqlens_cpu must be a CPU tensor")
+        if cu_seqlens_cpu.shape != cu_seqlens.shape:
+            raise ValueError("cu_seqlens_cpu must have the shape of cu_seqlens")
+        host = cu_seqlens_cpu.to(torch.int32).contiguous()
+    elif not cu_seqlens.is_cuda:
+        host = cu_seqlens.to(torch.int32).contiguous()
+    else:
+        host = cu_seqlens.detach().to("cpu", torch.int32).contiguous()  # blocking
+    if cu_seqlens.is_cuda:
+        if cu_seqlens.device != device:
+            raise ValueError(f"cu_seqlens must be on {device}")
+        dev = cu_seqlens.to(torch.int32).contiguous()
+    else:
+        dev = host.pin_memory().to(device, non_blocking=True)
+    return dev, host
+
+
 def _gate_fields(a, device, H, Dk, A_log, dt_bias, use_gate_in_kernel, safe_gate,
                  lower_bound, use_beta_sigmoid_in_kernel):
     """Gate and beta fields of the C argument struct (page "K3/kda/ops/api.py",
@@ -76,6 +109,7 @@ def _chunk_kda_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
               use_beta_sigmoid_in_kernel: bool = True, safe_gate: bool = False,
               lower_bound: Optional[float] = None,
               chunk_size: int = 64, cu_seqlens: Optional[torch.Tensor] = None,
+              cu_seqlens_cpu: Optional[torch.Tensor] = None,
               out: Optional[torch.Tensor] = None, final_state_out: Optional[torch.Tensor] = None,
               workspace: Optional[torch.Tensor] = None
               ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
@@ -91,7 +125,10 @@ def _chunk_kda_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
     -exp(A_log) softplus(g + dt_bias), or with safe_gate
     lower_bound * sigmoid(exp(A_log) (g + dt_bias)) (A_log: [H] fp32,
     dt_bias: [H, Dk] fp32 or None; the unbounded form ignores lower_bound).
-    ``cu_seqlens`` (int32, [N+1], B == 1) packs N sequences. ``chunk_size``
+    ``cu_seqlens`` (int32, [N+1], B == 1) packs N sequences; it may be a CPU
+    tensor (uploaded asynchronously) or a CUDA tensor, and a CUDA one should come
+    with ``cu_seqlens_cpu``, its host copy: without it every call reads the
+    offsets back with a blocking device-to-host copy. ``chunk_size``
     <= 32 selects 32-token chunks (CUDA-core kernel), anything else 64.
     Returns (o [B, T, H, Dv], final_state [N, H, Dk, Dv] fp32 or None).
 
@@ -118,16 +155,10 @@ def _chunk_kda_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
     if not isinstance(chunk_size, int) or chunk_size < 0:
         raise ValueError("chunk_size must be a non-negative int")
     chunk_size = 32 if 0 < chunk_size <= 32 else 64  # api.py's 32-or-64 rule
-    cu_host = None
-    if cu_seqlens is not None:
-        if B != 1:
-            raise ValueError("cu_seqlens requires B == 1")
-        cu_host = cu_seqlens.detach().to("cpu", torch.int32).contiguous()
-        cu_dev = cu_seqlens.to(q.device, torch.int32).contiguous()
-        N = cu_host.numel() - 1
-    else:
-        cu_dev = None
-        N = B
+    if cu_seqlens is not None and B != 1:
+        raise ValueError("cu_seqlens requires B == 1")
+    cu_dev, cu_host = _seqlens(cu_seqlens, cu_seqlens_cpu, q.device)
+    N = B if cu_host is None else cu_host.numel() - 1
     if initial_state is not None:
         _need_cuda("initial_state", initial_state)
         if initial_state.dtype != torch.float32 or initial_state.shape != (N, H, Dk, Dv):
@@ -322,6 +353,7 @@ def chunk_kda_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
                   initial_state: Optional[torch.Tensor] = None, scale: Optional[float] = None,
                   use_qk_l2norm_in_kernel: bool = False, use_beta_sigmoid_in_kernel: bool = True,
                   lower_bound: Optional[float] = None, cu_seqlens: Optional[torch.Tensor] = None,
+                  cu_seqlens_cpu: Optional[torch.Tensor] = None,
                   want_dinitial_state: bool = True, workspace: Optional[torch.Tensor] = None):
     """Gradients of ``chunk_kda`` (log-decay gate, the derivatives of the token
     recurrence of page "atlas_core/kimi_k3/kda.rs"; the pages give no backward
@@ -343,14 +375,10 @@ def chunk_kda_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
     dout = dout.to(q.dtype).contiguous()
     if dout.shape != v.shape:
         raise ValueError("dout must have the shape of v")
-    cu_host = cu_dev = None
-    N = B
-    if cu_seqlens is not None:
-        if B != 1:
-            raise ValueError("cu_seqlens requires B == 1")
-        cu_host = cu_seqlens.detach().to("cpu", torch.int32).contiguous()
-        cu_dev = cu_seqlens.to(q.device, torch.int32).contiguous()
-        N = cu_host.numel() - 1
+    if cu_seqlens is not None and B != 1:
+        raise ValueError("cu_seqlens requires B == 1")
+    cu_dev, cu_host = _seqlens(cu_seqlens, cu_seqlens_cpu, q.device)
+    N = B if cu_host is None else cu_host.numel() - 1
     for name, t in (("initial_state", initial_state), ("dfinal_state", dfinal_state)):
         if t is not None:
             _need_cuda(name, t)
@@ -404,6 +432,7 @@ class _ChunkKDA(torch.autograd.Function):
             use_qk_l2norm_in_kernel=kw.get("use_qk_l2norm_in_kernel", False),
             use_beta_sigmoid_in_kernel=kw.get("use_beta_sigmoid_in_kernel", True),
             lower_bound=kw.get("lower_bound"), cu_seqlens=kw.get("cu_seqlens"),
+            cu_seqlens_cpu=kw.get("cu_seqlens_cpu"),
             want_dinitial_state=S0 is not None and ctx.needs_input_grad[5])
         return dq, dk, dv, dg, db, dS0, None
 

@@ -31,6 +31,19 @@ def test_library_exports_every_declared_symbol():
     assert lib.kda_version() == header >= 200
 
 
+def test_status_queries_on_the_host():
+    """The status queries validate like the forward, need a workspace where the
+    tensor-core kernels would run, and read nothing for shapes whose kernels have
+    no device waits (fp32, or head dims other than 128) -- no GPU needed."""
+    lib = _abi.load()
+    for fn in (lib.kda_chunk_fwd_status, lib.kda_chunk_fwd_noalloc_status):
+        assert fn(None, None) == _abi.KDA_ERR_INVALID_ARGUMENT
+        assert fn(ctypes.byref(chunk_args(Dk=48)), None) == _abi.KDA_ERR_UNSUPPORTED
+        assert fn(ctypes.byref(chunk_args(dtype=_abi.KDA_DTYPE_F32)), None) == _abi.KDA_OK
+        assert fn(ctypes.byref(chunk_args(Dk=64, Dv=64)), None) == _abi.KDA_OK
+    assert lib.kda_chunk_fwd_status(ctypes.byref(chunk_args()), None) == _abi.KDA_ERR_WORKSPACE
+
+
 def test_status_strings():
     lib = _abi.load()
     for s in range(6):

@@ -38,7 +38,9 @@ def run_chunk(inp, wl=None, *, scale=None, lower_bound=None, final=True, l2=True
 
 
 def compare_chunk(inp, o, S, dtype, *, heads=None, seqs=None, scale=None, lower_bound=None,
-                  l2=True, tag="", **okw):
+                  l2=True, tag="", per_head=False, **okw):
+    """o and the final states against form R, per sequence over the chosen heads, or
+    with ``per_head`` per (sequence, head) so that no head hides under the others."""
     ref = oracle_chunk({k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()},
                        heads=heads, seqs=seqs, scale=scale, lower_bound=lower_bound, l2=l2, **okw)
     H = inp["q"].shape[2]
@@ -46,11 +48,14 @@ def compare_chunk(inp, o, S, dtype, *, heads=None, seqs=None, scale=None, lower_
     ns = list(range(len(ref))) if seqs is None else list(seqs)
     B, T = inp["q"].shape[:2]
     o_flat = o.reshape(B * T, H, -1)
+    groups = [([h], [j]) for j, h in enumerate(hs)] if per_head else [(hs, list(range(len(hs))))]
     for (a, b, o_ref, S_ref), n in zip(ref, ns):
-        if b > a:
-            check(f"{tag} o seq{n}", o_flat[a:b][:, hs], o_ref, dtype)
-        if S is not None:
-            check(f"{tag} S seq{n}", S[n, hs], S_ref, dtype)
+        for hg, jg in groups:
+            name = f"seq{n} h{hg[0]}" if per_head else f"seq{n}"
+            if b > a:
+                check(f"{tag} o {name}", o_flat[a:b][:, hg], o_ref[:, jg], dtype)
+            if S is not None:
+                check(f"{tag} S {name}", S[n, hg], S_ref[jg], dtype)
 
 
 # --- the named workloads, full size ------------------------------------------
@@ -74,16 +79,18 @@ def test_workload_d128_T8192_clamped():
     inp = KI.chunk_inputs(wl, device=DEV)
     o, S = run_chunk(inp, lower_bound=wl.lower_bound)
     compare_chunk(inp, o, S, wl.dtype, heads=[0, 5, 11, 15], lower_bound=wl.lower_bound,
-                  tag="d128")
+                  tag="d128", per_head=True)
 
 
 def test_workload_varlen_H96():
     wl = KI.CHUNK_WORKLOADS[4]
     inp = KI.chunk_inputs(wl, device=DEV)
     o, S = run_chunk(inp, lower_bound=wl.lower_bound)
+    # the first and the last head and eight drawn ones, each (sequence, head) on its own
     rng = np.random.default_rng(0)
-    heads = sorted(rng.choice(96, size=3, replace=False).tolist())
-    compare_chunk(inp, o, S, wl.dtype, heads=heads, lower_bound=wl.lower_bound, tag="varlen")
+    heads = sorted({0, 95} | set(rng.choice(np.arange(1, 95), size=8, replace=False).tolist()))
+    compare_chunk(inp, o, S, wl.dtype, heads=heads, lower_bound=wl.lower_bound, tag="varlen",
+                  per_head=True)
     assert torch.isfinite(o).all() and torch.isfinite(S).all()
 
 
@@ -165,14 +172,19 @@ def test_workload_decode_256_steps():
     for t in range(wl.steps):
         outs.append(kda.recurrent_step(inp["q"][t], inp["k"][t], inp["v"][t], inp["g"][t],
                                        inp["beta"][t], state))
-    o = torch.stack(outs)  # [steps, N, H, Dv]
+    o = torch.stack(outs).cpu()  # [steps, N, H, Dv]
+    # 16 (sequence, head) pairs, the first and the last among them; every step's output
+    # of each pair is checked on its own, and the pair's state after the 256 steps
     rng = np.random.default_rng(1)
-    for n, h in zip(rng.choice(wl.N, 4, replace=False), rng.choice(wl.H, 4, replace=False)):
+    pairs = [(0, 0), (wl.N - 1, wl.H - 1)] + list(zip(rng.choice(wl.N, 14).tolist(),
+                                                       rng.choice(wl.H, 14).tolist()))
+    for n, h in pairs:
         sl = lambda x: x[:, n, h:h + 1].cpu()
         o_ref, S_ref = oracle.recurrent(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["g"]),
                                         inp["beta"][:, n, h:h + 1].cpu(),
                                         initial_state=inp["state"][n:n + 1, h:h + 1].cpu())
-        check(f"decode o n{n} h{h}", o[:, n, h:h + 1], o_ref, wl.dtype)
+        for t in range(wl.steps):
+            check(f"decode o n{n} h{h} step{t}", o[t, n, h], o_ref[t, 0], wl.dtype)
         check(f"decode S n{n} h{h}", state[n, h], S_ref[0, 0], wl.dtype)
 
 
