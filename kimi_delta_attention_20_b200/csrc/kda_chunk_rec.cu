@@ -10,12 +10,15 @@
 // arithmetic, not its value. For small head dims the recurrence also takes
 // fewer operations than the chunked form (no C x C blocks, no inverse).
 //
-// One CTA per (sequence, head), one warp per 4 CG value columns (CG = 4). Lane (rg, cg) = (lane / 4, lane % 4) keeps rows
-// rg*RP .. rg*RP+RP-1 (RP = d_k / 8) of columns CG cg .. CG cg + CG - 1 of its
-// warp's block in registers, as column pairs for the paired fp32 FMA pipe. The
-// key-axis sums u and o are reductions over the 8 row groups of a warp (a
-// reduce-scatter, then a gather for u); nothing else crosses lanes, and no barrier
-// is taken per token. Tokens arrive in stretches of CT: the raw rows of the next
+// One CTA per (sequence, head). A warp holds WC value columns of the state over all
+// d_k rows: lane (rg, cg) = (lane / CGN, lane % CGN) keeps the RP = 16 key rows
+// rg*RP .. rg*RP+15 of columns CG cg .. CG cg + CG - 1 of its warp's block in registers,
+// as column pairs for the paired fp32 FMA pipe. For d_k <= 64 the warp has d_k / 16
+// row groups and CG = 2, so the key-axis sums u and o are a butterfly of one or two
+// shuffle levels that leaves every lane with the totals of its own columns; for
+// d_k = 128 there are 8 row groups and CG = 4, and the sums are a reduce-scatter
+// followed by a gather for u. Nothing else crosses lanes, and no barrier is taken
+// per token. Tokens arrive in stretches of CT: the raw rows of the next
 // stretch are copied by cp.async while the current one runs, turned into fp32
 // (L2 norms, gate, sigmoid) once per stretch, and the stretch's outputs leave
 // from shared memory as whole rows.
@@ -31,16 +34,19 @@ namespace {
 
 template <int DK, int DV>
 struct RecCfg {
-    // value columns per lane: 4. Eight halve the shuffles and loads per state element
-    // but also the warps per CTA; on the 300M layer (1024 CTAs, one wave) that was
-    // slower (1.59 ms against 1.44 ms), the kernel leaning on warps to hide latency.
-    static constexpr int CG = 4;
-    static constexpr int WC = 4 * CG;               // value columns per warp
+    // 16 key rows per lane. Small key dims take the butterfly layout (d_k / 16 row groups,
+    // 2 value columns per lane); d_k = 128 keeps 8 row groups of 4 value columns, where
+    // a butterfly would need three levels and twice the warps' columns.
+    static constexpr bool BFLY = DK <= 64;
+    static constexpr int RGN = BFLY ? DK / 16 : 8;  // row groups per warp
+    static constexpr int CGN = 32 / RGN;            // column groups per warp (lanes per row group)
+    static constexpr int CG = BFLY ? 2 : 4;         // value columns per lane
+    static constexpr int WC = CGN * CG;             // value columns per warp
     static constexpr int NW = DV / WC, NT = NW * 32;
-    static constexpr int RP = DK / 8;               // rows per lane
+    static constexpr int RP = DK / RGN;             // rows per lane
     static constexpr int CT = DK >= 128 ? 16 : 32;  // tokens per stretch
     static constexpr int TPR = 8, E = DK / TPR;     // intake: threads per key row, elements each
-    static_assert(NW >= 1 && NW * WC == DV && RP * 8 == DK && NT >= CT && NT >= 64, "recurrent tiling");
+    static_assert(NW >= 1 && NW * WC == DV && RP == 16 && NT >= CT, "recurrent tiling");
 };
 
 template <typename Tin, int DK, int DV>
@@ -172,12 +178,14 @@ __device__ __forceinline__ float rowgroup_scatter(const float (&x)[CG]) {
 template <typename Tin, int DK, int DV, bool AUG, int CB = DV>
 __global__ void __launch_bounds__(RecCfg<DK, CB>::NT) kda_chunk_rec_kernel(ChunkParams p) {
     using Cfg = RecCfg<DK, CB>;
-    constexpr int RP = Cfg::RP, CT = Cfg::CT, NT = Cfg::NT, CG = Cfg::CG, CP = CG / 2;
-    constexpr int VS = 32 / CG;  // lanes between the holders of consecutive reduced values
+    constexpr int RP = Cfg::RP, CT = Cfg::CT, NT = Cfg::NT, CG = Cfg::CG, CP = CG / 2, CGN = Cfg::CGN;
+    constexpr bool BFLY = Cfg::BFLY;
+    constexpr int NACC = BFLY ? 4 : 2;  // independent accumulation chains per column pair
+    constexpr int VS = 32 / CG;  // lanes between the holders of consecutive reduced values (reduce-scatter)
     extern __shared__ __align__(16) uint8_t smraw[];
     RecSmem<Tin, DK, CB> &sm = *reinterpret_cast<RecSmem<Tin, DK, CB> *>(smraw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int rg = lane >> 2, cg = lane & 3;
+    const int rg = lane / CGN, cg = lane % CGN;
     const int c0 = blockIdx.y * CB;            // the CTA's first state column
     const int col = Cfg::WC * warp + CG * cg;  // this lane's first value column within the CTA's
     const int gcol = c0 + col;
@@ -194,16 +202,24 @@ __global__ void __launch_bounds__(RecCfg<DK, CB>::NT) kda_chunk_rec_kernel(Chunk
     // the state as column pairs (col + 2 j, col + 2 j + 1), for the paired fp32 FMA pipe
     float2 s[RP][CP];
 #pragma unroll
-    for (int r = 0; r < RP; ++r)
+    for (int r = 0; r < RP; ++r) {
+        const int row = rg * RP + r;
+        if constexpr (CP == 1) {
+            s[r][0] = AUG ? make_float2(row == gcol, row == gcol + 1)
+                    : p.S0 ? *reinterpret_cast<const float2 *>(p.S0 + (nh * DK + row) * DV + gcol)
+                           : make_float2(0.f, 0.f);
+        } else {
 #pragma unroll
-        for (int j = 0; j < CP; j += 2) {
-            const int row = rg * RP + r, cj = gcol + 2 * j;
-            const float4 x = AUG ? make_float4(row == cj, row == cj + 1, row == cj + 2, row == cj + 3)
-                             : p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + (nh * DK + row) * DV + cj)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-            s[r][j] = make_float2(x.x, x.y);
-            s[r][j + 1] = make_float2(x.z, x.w);
+            for (int j = 0; j < CP; j += 2) {
+                const int cj = gcol + 2 * j;
+                const float4 x = AUG ? make_float4(row == cj, row == cj + 1, row == cj + 2, row == cj + 3)
+                                 : p.S0 ? *reinterpret_cast<const float4 *>(p.S0 + (nh * DK + row) * DV + cj)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                s[r][j] = make_float2(x.x, x.y);
+                s[r][j + 1] = make_float2(x.z, x.w);
+            }
         }
+    }
 
     long long t0 = bos;  // stretches of CT tokens
     int cnt = (int)min((long long)CT, eos - bos);
@@ -221,61 +237,93 @@ __global__ void __launch_bounds__(RecCfg<DK, CB>::NT) kda_chunk_rec_kernel(Chunk
             rows_in<RP>(&sm.qh[i][rg * RP], qr);
             const float b = sm.b[i];
             float2 vv[CP];
+            if constexpr (CP == 1) {
+                vv[0] = *reinterpret_cast<const float2 *>(&sm.vo[i][col]);
+            } else {
 #pragma unroll
-            for (int j = 0; j < CP; j += 2) {
-                const float4 x = *reinterpret_cast<const float4 *>(&sm.vo[i][col + 2 * j]);
-                vv[j] = make_float2(x.x, x.y);
-                vv[j + 1] = make_float2(x.z, x.w);
+                for (int j = 0; j < CP; j += 2) {
+                    const float4 x = *reinterpret_cast<const float4 *>(&sm.vo[i][col + 2 * j]);
+                    vv[j] = make_float2(x.x, x.y);
+                    vv[j + 1] = make_float2(x.z, x.w);
+                }
             }
-            // S' = diag(a) S and this lane's part of u = S'^T k^ (two chains per pair)
+            // S' = diag(a) S and this lane's part of u = S'^T k^ (NACC chains per pair)
             const float2 z2 = make_float2(0.f, 0.f);
-            float2 acc[2][CP];
+            float2 acc[NACC][CP];
 #pragma unroll
-            for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
+            for (int a = 0; a < NACC; ++a)
+#pragma unroll
+                for (int j = 0; j < CP; ++j) acc[a][j] = z2;
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
                 const float2 a2 = make_float2(ar[r], ar[r]), k2 = make_float2(kr[r], kr[r]);
 #pragma unroll
                 for (int j = 0; j < CP; ++j) {
                     s[r][j] = __fmul2_rn(s[r][j], a2);
-                    acc[r & 1][j] = __ffma2_rn(s[r][j], k2, acc[r & 1][j]);
+                    acc[r % NACC][j] = __ffma2_rn(s[r][j], k2, acc[r % NACC][j]);
                 }
             }
-            float part[CG];
-#pragma unroll
-            for (int j = 0; j < CP; ++j) {
-                const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
-                part[2 * j] = t.x; part[2 * j + 1] = t.y;
-            }
-            const float m = rowgroup_scatter<CG>(part);
-            // gather u of the lane's columns from the lanes that hold them
             float2 d[CP];
             const float2 b2 = make_float2(b, b);
+            if constexpr (BFLY) {
+                // u of the lane's two columns: its chains, then the other row groups
+                float2 u = __fadd2_rn(acc[0][0], acc[1][0]);
 #pragma unroll
-            for (int j = 0; j < CP; ++j) {
-                const float2 u = make_float2(__shfl_sync(0xffffffffu, m, (2 * j) * VS + cg),
-                                             __shfl_sync(0xffffffffu, m, (2 * j + 1) * VS + cg));
-                d[j] = __fmul2_rn(b2, __fadd2_rn(vv[j], make_float2(-u.x, -u.y)));
+                for (int a = 2; a < NACC; ++a) u = __fadd2_rn(u, acc[a][0]);
+#pragma unroll
+                for (int bit = 16; bit >= CGN; bit >>= 1)
+                    u = __fadd2_rn(u, make_float2(__shfl_xor_sync(0xffffffffu, u.x, bit),
+                                                  __shfl_xor_sync(0xffffffffu, u.y, bit)));
+                d[0] = __fmul2_rn(b2, __fadd2_rn(vv[0], make_float2(-u.x, -u.y)));
+            } else {
+                float part[CG];
+#pragma unroll
+                for (int j = 0; j < CP; ++j) {
+                    const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
+                    part[2 * j] = t.x; part[2 * j + 1] = t.y;
+                }
+                const float m = rowgroup_scatter<CG>(part);
+                // gather u of the lane's columns from the lanes that hold them
+#pragma unroll
+                for (int j = 0; j < CP; ++j) {
+                    const float2 u = make_float2(__shfl_sync(0xffffffffu, m, (2 * j) * VS + cg),
+                                                 __shfl_sync(0xffffffffu, m, (2 * j + 1) * VS + cg));
+                    d[j] = __fmul2_rn(b2, __fadd2_rn(vv[j], make_float2(-u.x, -u.y)));
+                }
             }
             // S = S' + k^ d^T and this lane's part of S^T q^
 #pragma unroll
-            for (int j = 0; j < CP; ++j) { acc[0][j] = z2; acc[1][j] = z2; }
+            for (int a = 0; a < NACC; ++a)
+#pragma unroll
+                for (int j = 0; j < CP; ++j) acc[a][j] = z2;
 #pragma unroll
             for (int r = 0; r < RP; ++r) {
                 const float2 k2 = make_float2(kr[r], kr[r]), q2 = make_float2(qr[r], qr[r]);
 #pragma unroll
                 for (int j = 0; j < CP; ++j) {
                     s[r][j] = __ffma2_rn(k2, d[j], s[r][j]);
-                    acc[r & 1][j] = __ffma2_rn(s[r][j], q2, acc[r & 1][j]);
+                    acc[r % NACC][j] = __ffma2_rn(s[r][j], q2, acc[r % NACC][j]);
                 }
             }
+            if constexpr (BFLY) {
+                float2 ov = __fadd2_rn(acc[0][0], acc[1][0]);
 #pragma unroll
-            for (int j = 0; j < CP; ++j) {
-                const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
-                part[2 * j] = t.x; part[2 * j + 1] = t.y;
+                for (int a = 2; a < NACC; ++a) ov = __fadd2_rn(ov, acc[a][0]);
+#pragma unroll
+                for (int bit = 16; bit >= CGN; bit >>= 1)
+                    ov = __fadd2_rn(ov, make_float2(__shfl_xor_sync(0xffffffffu, ov.x, bit),
+                                                    __shfl_xor_sync(0xffffffffu, ov.y, bit)));
+                if (rg == 0) *reinterpret_cast<float2 *>(&sm.vo[i][col]) = make_float2(p.scale * ov.x, p.scale * ov.y);
+            } else {
+                float part[CG];
+#pragma unroll
+                for (int j = 0; j < CP; ++j) {
+                    const float2 t = __fadd2_rn(acc[0][j], acc[1][j]);
+                    part[2 * j] = t.x; part[2 * j + 1] = t.y;
+                }
+                const float ov = rowgroup_scatter<CG>(part);
+                if (CG == 8 || (lane & 4) == 0) sm.vo[i][col + lane / VS] = p.scale * ov;
             }
-            const float ov = rowgroup_scatter<CG>(part);
-            if (CG == 8 || (lane & 4) == 0) sm.vo[i][col + lane / VS] = p.scale * ov;
         }
         if (p.o) {
             // the stretch's output rows, from shared memory
@@ -298,11 +346,16 @@ __global__ void __launch_bounds__(RecCfg<DK, CB>::NT) kda_chunk_rec_kernel(Chunk
     }
     if (p.S_out) {
 #pragma unroll
-        for (int r = 0; r < RP; ++r)
+        for (int r = 0; r < RP; ++r) {
+            float *dst = p.S_out + (nh * DK + rg * RP + r) * DV + gcol;
+            if constexpr (CP == 1) {
+                *reinterpret_cast<float2 *>(dst) = s[r][0];
+            } else {
 #pragma unroll
-            for (int j = 0; j < CP; j += 2)
-                *reinterpret_cast<float4 *>(p.S_out + (nh * DK + rg * RP + r) * DV + gcol + 2 * j) =
-                    make_float4(s[r][j].x, s[r][j].y, s[r][j + 1].x, s[r][j + 1].y);
+                for (int j = 0; j < CP; j += 2)
+                    *reinterpret_cast<float4 *>(dst + 2 * j) = make_float4(s[r][j].x, s[r][j].y, s[r][j + 1].x, s[r][j + 1].y);
+            }
+        }
     }
 }
 
