@@ -24,9 +24,12 @@
 // from shared memory as whole rows.
 #include <algorithm>
 
+#include <type_traits>
+
 #include "kda_common.cuh"
 #include "kda_stage.cuh"
 #include "kda_seg.cuh"
+#include "kda_tc_util.cuh"
 
 namespace kda {
 
@@ -120,7 +123,16 @@ __device__ void rec_take(const ChunkParams &p, RecSmem<Tin, DK, CB> &sm, int cnt
         for (int e = 0; e < E; ++e) {
             kx[e] *= rk;
             qx[e] *= rq;
-            gx[e] = expf(gate_value(gx[e], sm.dtb[c + e], rate, p.gate_mode, p.has_lb, p.lb));
+            if constexpr (std::is_same<Tin, __nv_bfloat16>::value) {
+                // bf16 inputs: the gate and the decay on the special-function unit (the
+                // forms of the tensor-core path; their error is far below bf16 rounding)
+                constexpr float kL2e = 1.4426950408889634f;
+                const float gv = p.gate_mode == kGateLog ? (p.has_lb ? fmaxf(gx[e], p.lb) : gx[e])
+                                                         : tcu::gate_fast(gx[e], sm.dtb[c + e], rate, p.gate_mode, p.lb);
+                gx[e] = tcu::ex2a(gv * kL2e);
+            } else {
+                gx[e] = expf(gate_value(gx[e], sm.dtb[c + e], rate, p.gate_mode, p.has_lb, p.lb));
+            }
         }
         if (live) {
             store_vec<E>(&sm.kh[i][c], kx);
