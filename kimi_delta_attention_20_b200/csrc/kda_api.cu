@@ -22,7 +22,7 @@ cudaError_t launch_chunk_tc(const ChunkParams &p, int Dk, int Dv, void *workspac
 size_t chunk_2pass_workspace_bytes(const ChunkParams &p);
 cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int32_t *cu_host, cudaStream_t st);
 bool token_conv_supported(int K);
-size_t bwd_workspace_bytes(bool varlen, long long T, int N, int H, int Dk, int Dv);
+size_t bwd_workspace_bytes(const BwdParams &p, bool bf16, int Dk, int Dv);
 size_t bwd_workspace_bytes_min(bool varlen, long long T, int N, int H, int Dk, int Dv);
 cudaError_t launch_bwd(BwdParams p, bool bf16, int Dk, int Dv, void *workspace, size_t workspace_bytes, cudaStream_t st);
 cudaError_t launch_token(const TokenParams &tp, float *state_out, bool bf16, int Dk, int Dv, cudaStream_t st);
@@ -327,13 +327,29 @@ kda_status kda_decode_token(const kda_token_args *a, void *stream) {
     return cuda_status(kda::launch_token(tp, a->state_out, bf16, a->Dk, a->Dv, static_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+kda::BwdParams bwd_params(const kda_chunk_bwd_args *a, int N) {
+    kda::BwdParams p{};
+    p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta; p.dout = a->dout;
+    p.S0 = a->initial_state; p.dSf = a->dfinal_state;
+    p.dq = a->dq; p.dk = a->dk; p.dv = a->dv; p.dg = a->dg; p.dbeta = a->dbeta; p.dS0 = a->dinitial_state;
+    p.cu_seqlens = a->cu_seqlens; p.T = a->T; p.N = N; p.H = a->H;
+    p.scale = resolve_scale(a->scale, a->Dk);
+    p.use_l2 = a->use_qk_l2norm ? 1 : 0;
+    p.has_lb = a->has_lower_bound ? 1 : 0;
+    p.lb = a->lower_bound;
+    p.beta_prob = a->beta_is_prob ? 1 : 0;
+    return p;
+}
+}  // namespace
+
 kda_status kda_chunk_bwd_workspace_size(const kda_chunk_bwd_args *a, size_t *bytes) {
     if (!a || !bytes) return KDA_ERR_INVALID_ARGUMENT;
     const kda_chunk_args f = fwd_view(a);
     int N = 0;
     kda_status s = check_chunk_shape(&f, &N);
     if (s != KDA_OK) return s;
-    *bytes = kda::bwd_workspace_bytes(a->cu_seqlens != nullptr, a->T, N, a->H, a->Dk, a->Dv);
+    *bytes = kda::bwd_workspace_bytes(bwd_params(a, N), a->dtype == KDA_DTYPE_BF16, a->Dk, a->Dv);
     return KDA_OK;
 }
 
@@ -364,16 +380,7 @@ kda_status kda_chunk_bwd(const kda_chunk_bwd_args *a, void *stream) {
     if (!a->cu_seqlens && a->cu_seqlens_host) return KDA_ERR_INVALID_ARGUMENT;
     const size_t need_ws = kda::bwd_workspace_bytes_min(a->cu_seqlens != nullptr, a->T, N, a->H, a->Dk, a->Dv);
     if (!a->workspace || a->workspace_bytes < need_ws || !aligned(a->workspace, 16)) return KDA_ERR_WORKSPACE;
-    kda::BwdParams p{};
-    p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta; p.dout = a->dout;
-    p.S0 = a->initial_state; p.dSf = a->dfinal_state;
-    p.dq = a->dq; p.dk = a->dk; p.dv = a->dv; p.dg = a->dg; p.dbeta = a->dbeta; p.dS0 = a->dinitial_state;
-    p.cu_seqlens = a->cu_seqlens; p.T = a->T; p.N = N; p.H = a->H;
-    p.scale = resolve_scale(a->scale, a->Dk);
-    p.use_l2 = a->use_qk_l2norm ? 1 : 0;
-    p.has_lb = a->has_lower_bound ? 1 : 0;
-    p.lb = a->lower_bound;
-    p.beta_prob = a->beta_is_prob ? 1 : 0;
+    const kda::BwdParams p = bwd_params(a, N);
     return cuda_status(
         kda::launch_bwd(p, bf16, a->Dk, a->Dv, a->workspace, a->workspace_bytes, static_cast<cudaStream_t>(stream)));
 }

@@ -952,7 +952,20 @@ cudaError_t bwd_segments(const BwdParams &p, bool bf16, int P, const BwdSegLayou
     return launch_bwd_ws(b, bf16, D, D, shared, st);
 }
 
-// The workspace with which kda_chunk_bwd runs its fastest form (the segments when they apply).
+size_t bwd_chunked_workspace_bytes(const BwdParams &p, bool bf16, int Dk, int Dv);
+cudaError_t launch_bwd_chunked(const BwdParams &p, void *workspace, cudaStream_t st);
+size_t bwd_workspace_bytes(bool varlen, long long T, int N, int H, int Dk, int Dv);
+
+// The workspace with which kda_chunk_bwd runs its fastest form: the chunked form
+// (kda_bwd_chunk.cu) where it applies, else the segments when they apply.
+size_t bwd_workspace_bytes(const BwdParams &p, bool bf16, int Dk, int Dv) {
+    const bool varlen = p.cu_seqlens != nullptr;
+    const size_t chunked = bwd_chunked_workspace_bytes(p, bf16, Dk, Dv);
+    if (chunked) return std::max(chunked, bwd_workspace_bytes_min(varlen, p.T, p.N, p.H, Dk, Dv));
+    return bwd_workspace_bytes(varlen, p.T, p.N, p.H, Dk, Dv);
+}
+
+// The workspace of the token-recurrence form (the segments when they apply).
 size_t bwd_workspace_bytes(bool varlen, long long T, int N, int H, int Dk, int Dv) {
     const size_t plain = bwd_workspace_bytes_min(varlen, T, N, H, Dk, Dv);
     const int P = bwd_seg_count(varlen, T, N, H, Dk, Dv);
@@ -965,6 +978,9 @@ size_t bwd_workspace_bytes(bool varlen, long long T, int N, int H, int Dk, int D
 cudaError_t launch_bwd(BwdParams p, bool bf16, int Dk, int Dv, void *workspace, size_t workspace_bytes, cudaStream_t st) {
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const bool varlen = p.cu_seqlens != nullptr;
+    const size_t chunked = bwd_chunked_workspace_bytes(p, bf16, Dk, Dv);
+    if (chunked && workspace_bytes >= chunked && (reinterpret_cast<uintptr_t>(ws) & 255) == 0)
+        return launch_bwd_chunked(p, ws, st);
     const int P = bwd_seg_count(varlen, p.T, p.N, p.H, Dk, Dv);
     if (P >= 2 && (reinterpret_cast<uintptr_t>(ws) & 255) == 0) {
         const bool tc = bf16 && Dk == 128;

@@ -47,6 +47,7 @@
 #include "kda_tc_util.cuh"
 #include "kda_stage.cuh"
 #include "kda_seg.cuh"
+#include "kda_record.cuh"
 
 namespace kda {
 namespace tp {
@@ -59,20 +60,7 @@ constexpr int D = 128;
 constexpr float kSpanMax = 80.f;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded waits: 2 s
 
-// ---- record of one (chunk, head), bytes; every tile is a shared-memory image
-// with the 128-byte swizzle (16-byte chunk index XOR row % 8, rows of 128 B)
-// Pass 2 reads [Qtil^T | -W^T] as one N = 128 operand and [Khat^T ; A_qk] as one
-// N = 192 operand, so those tiles are adjacent.
-constexpr uint32_t R_QT = 0;        // Qtil^T [128 c][64 r]: B of S^T Qtil^T, N = r contiguous (MN-major)
-constexpr uint32_t R_WT = 16384;    // -W^T   [128 c][64 r]: B of S^T (-W^T), MN-major
-constexpr uint32_t R_KH = 32768;    // Khat^T [128 c][64 s]: B of D~^T Khat, K = s contiguous (K-major)
-constexpr uint32_t R_AQK = 49152;   // A_qk (raw rows) [64 r][64 s], K-major B
-constexpr uint32_t R_TPU = 57344;   // T' = T diag(beta) [64 r][64 s], K-major B
-static_assert(R_WT - R_QT == 16384 && R_AQK == R_KH + 16384, "operand groups of pass 2 are adjacent");
-constexpr uint32_t R_MISC = 65536;  // f32: e^{G_last}[128], 1/|q_r|[64], 1/|k_s|[64]
-constexpr uint32_t R_GAM = R_MISC, R_INVQ = R_MISC + 512, R_INVK = R_MISC + 768;
-constexpr uint32_t REC_BYTES = R_MISC + 1024;
-static_assert(REC_BYTES % 1024 == 0, "records stay 1024-byte aligned");
+// the record of one (chunk, head): kda_record.cuh
 
 // ============================================================== pass 1
 constexpr int NT1 = 256;  // 8 warps, two CTAs per SM
@@ -950,6 +938,7 @@ struct StateParams {
     int s0_identity;  // start every chain from the identity (S0 is not read)
     int o_f32;        // outputs in fp32 (rows of D floats) instead of bf16
     int v_zero;       // v = 0: no v tiles are copied (tv is not read) and the stage's v area stays zero
+    uint8_t *save;    // or null: per (chunk, head) backward record, the S^T and D~^T images go there
     int nperm;
     int perm[kMaxPerm];
 };
@@ -968,6 +957,7 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
     else { bos = (long long)n * p.T; eos = bos + p.T; c_first = (long long)n * P.cpr; }
     const int nchunks = (int)((eos - bos + C - 1) / C);
     constexpr int kTma = kGroup;  // first thread of the output group issues the stage copies
+    constexpr int kSave = 32;     // stores the chain's images to the backward record
 
     uint64_t *bar_full = reinterpret_cast<uint64_t *>(sm + M2_BAR);  // [2] stage s loaded
     uint64_t *bar_m1 = bar_full + 2;                                 // first products done
@@ -1029,6 +1019,7 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
             const int s = ci & 1, b = ci & 1;
             uint8_t *stg = sm + s * STAGE_BYTES;
             const uint32_t so = s * STAGE_BYTES;
+            if (tid == kSave && P.save) bulk_wait_read_all();  // the previous chunk's images were copied out
             {
                 bool ok = true;
                 if (warp == 0) {
@@ -1069,6 +1060,8 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
             tc_fence_before();
             bar_sync(1, kGroup);
             tc_fence_after();
+            uint8_t *bsave = P.save ? P.save + ((c_first + ci) * H + h) * (long long)BR_BYTES : nullptr;
+            if (tid == kSave && bsave) { bulk_store(bsave + BR_S0, sm + ST2, 32768); bulk_commit(); }
 
             // [O^T | D^T] = S^T [Qtil^T | -W^T], then D^T += V^T T'^T
             if (warp == 0) {
@@ -1108,6 +1101,7 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
             tc_fence_before();
             bar_sync(1, kGroup);
             tc_fence_after();
+            if (tid == kSave && bsave) { bulk_store(bsave + BR_DL, sm + DT2, 16384); bulk_commit(); }
 
             // S^T += D~^T Khat (committed on its own: the next chunk waits for it), then
             // O^T += D~^T A_qk^T (the output group waits for that one)
@@ -1152,6 +1146,7 @@ __global__ void __launch_bounds__(NT2, 1) kda_tp_state_kernel(const __grid_const
             mbar_wait(bar_o + (issued & 1), (issued >> 1) & 1, kWaitLimitNs);
             if (P.status && lane == 0) atomicOr(P.status, 1);
         }
+        if (tid == kSave && P.save) bulk_wait_all();
     } else {
         // ================= output rows, one chunk behind
         __nv_bfloat16 *O = static_cast<__nv_bfloat16 *>(p.o);
@@ -1399,7 +1394,7 @@ std::vector<int> pass2_order(const int32_t *cu_host, int N, int H, int slots) {
 // pass 2 of p (v, S0, S_out and o as p gives them; o may be null) over the records in ws;
 // s0_identity starts every chain from the identity, v_zero takes v = 0 (p.v is not read)
 cudaError_t run_pass2(const ChunkParams &p, uint8_t *ws, const int32_t *cu_host, cudaStream_t st, int s0_identity = 0,
-                      int v_zero = 0, int o_f32 = 0) {
+                      int v_zero = 0, int o_f32 = 0, uint8_t *save = nullptr) {
     const long long total = p.cu_seqlens ? (long long)p.T : (long long)p.N * p.T;
     int *status = reinterpret_cast<int *>(ws);
     const size_t base = 1024 + 16384;
@@ -1415,6 +1410,7 @@ cudaError_t run_pass2(const ChunkParams &p, uint8_t *ws, const int32_t *cu_host,
     B.s0_identity = s0_identity;
     B.v_zero = v_zero;
     B.o_f32 = o_f32;
+    B.save = save;
     if (!v_zero && !make_map(&B.tv, p.v, total, p.H)) return cudaErrorInvalidValue;
     B.nperm = 0;
     cudaError_t e;
@@ -1496,14 +1492,27 @@ cudaError_t chunk_2pass_transitions(const ChunkParams &q, void *workspace, float
     return run_pass2(pn, ws, nullptr, st);
 }
 
-cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int32_t *cu_host, cudaStream_t st) {
+// The records of the forward run in ws (its layout follows the segment view when p is
+// segmented); chunk numbering is the same either way, as segments are chunk-aligned.
+uint8_t *chunk_2pass_records(const ChunkParams &p, void *workspace) {
+    using namespace tp;
+    const int P = seg_count(p);
+    const ChunkParams q = P == 1 ? p : seg_view(p, P, reinterpret_cast<const int32_t *>(16));
+    return static_cast<uint8_t *>(workspace) + 1024 + 16384 + offsets_bytes(q) + table_bytes(q) + queue_bytes(q);
+}
+
+// The forward of p; with save non-null, the pass that forms the outputs also writes
+// every (chunk, head)'s S^T and D~^T images to its backward record (save + (chunk * H
+// + head) * BR_BYTES, global chunk numbering).
+cudaError_t launch_chunk_2pass_save(const ChunkParams &p, void *workspace, const int32_t *cu_host, uint8_t *save,
+                                    cudaStream_t st) {
     using namespace tp;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const int P = seg_count(p);
     cudaError_t e;
     if (P == 1) {
         if ((e = run_pass1(p, ws, st)) != cudaSuccess) return e;
-        return run_pass2(p, ws, cu_host, st);
+        return run_pass2(p, ws, cu_host, st, 0, 0, 0, save);
     }
     // workspace: [two-pass workspace of the segment view][cu_v][M][N][S_start]
     int32_t *cu_v = reinterpret_cast<int32_t *>(ws + base_workspace_bytes(seg_view(p, P, reinterpret_cast<const int32_t *>(16))));
@@ -1528,7 +1537,20 @@ cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int3
     if ((e = seg_chain_launch<128>(p.S0, Mbuf, Nbuf, 128, 128LL * 128, Sbuf, p.S_out, p.N, p.H, P, st)) != cudaSuccess) return e;
     ChunkParams pf = q;  // the outputs, from the true entering states
     pf.S0 = Sbuf; pf.S_out = nullptr;
-    return run_pass2(pf, ws, nullptr, st);
+    return run_pass2(pf, ws, nullptr, st, 0, 0, 0, save);
+}
+
+// The chunk offsets and table of a varlen batch (the prep kernel also writes the constant
+// tiles to consts, 16 KB).
+cudaError_t chunk_2pass_chunk_table(const int32_t *cu, int N, int *chunk_off, int2 *chunk_tok, uint8_t *consts,
+                                    cudaStream_t st) {
+    count_launch();
+    tp::kda_tp_prep<<<1, 1024, 0, st>>>(consts, cu, N, chunk_off, chunk_tok);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_2pass(const ChunkParams &p, void *workspace, const int32_t *cu_host, cudaStream_t st) {
+    return launch_chunk_2pass_save(p, workspace, cu_host, nullptr, st);
 }
 
 }  // namespace kda
