@@ -303,15 +303,15 @@ __global__ void __launch_bounds__(NTC, 1) kda_cb_dstate_kernel(const __grid_cons
 }
 
 // ============================================================== chunk-local gradients
-// One item = one (chunk, head); persistent CTAs of 256 threads (8 warps) walk the
+// One item = one (chunk, head); persistent CTAs of 512 threads (16 warps) walk the
 // items. Products are warp-level bf16 tensor-core MMAs (m16n8k16, fp32 accumulate)
 // on tiles in shared memory: the backward record's images (128-byte swizzle) and the
 // raw rows (padded to 136 elements, 272-byte rows, so the eight rows of a fragment
 // load fall on distinct banks); the three 64 x 64 x 64 products of the inverse run as
 // tf32 MMAs on fp32 tiles. Every [64][128] result uses one warp layout -- warp w
-// owns rows 16 (w % 4) .. and columns 64 (w / 4) .. -- so the contributions to dq^,
+// owns rows 16 (w % 4) .. and columns 32 (w / 4) .. -- so the contributions to dq^,
 // dk^ and dG of an element stay in the registers of one thread until the end.
-constexpr int NTI = 256;
+constexpr int NTI = 512;
 constexpr int LP = 136;                  // padded row of a bf16 [64][128] tile (elements)
 constexpr uint32_t PT = 64 * LP * 2;     // bytes of such a tile: 17,408
 constexpr int LG = 136;                  // fp32 row of G / dG (floats)
@@ -324,8 +324,8 @@ constexpr uint32_t X_MISC = X_DAQ + 64 * LA * 2;
 constexpr uint32_t XM_RK = X_MISC, XM_RQ = X_MISC + 256, XM_B = X_MISC + 512, XM_DB = X_MISC + 768,
                    XM_DGC = X_MISC + 1024,   // [4][128] column partials of sum_s dKhat Khat
                    XM_DGAM = X_MISC + 3072,  // [128] gamma_c sum_v S dS_C
-                   XM_RED = X_MISC + 3584,   // [8][128] f32 reduction scratch
-                   XM_BAR = XM_RED + 4096;
+                   XM_RED = X_MISC + 3584,   // [16][128] f32 reduction scratch
+                   XM_BAR = XM_RED + 8192;
 constexpr uint32_t X_R = (XM_BAR + 64 + 1023) / 1024 * 1024;      // phase region
 // phase A/B
 constexpr uint32_t Y_SV = X_R, Y_S0 = Y_SV + BR_S0, Y_DL = Y_SV + BR_DL, Y_DS = Y_SV + BR_DS, Y_DD = Y_SV + BR_DD;
@@ -422,15 +422,15 @@ __device__ __forceinline__ void zero(float (&acc)[NT][4]) {
 #pragma unroll
     for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
 }
-// 64 x 64 x 64 tf32 product, warp tile rows m0.., columns n0.. (4 n-tiles)
-template <class FA, class FB>
-__device__ __forceinline__ void tgemm(float (&acc)[4][4], FA a, FB b, int m0, int n0, int g, int t) {
+// 64 x 64 x 64 tf32 product, warp tile rows m0.., columns n0.. (NT n-tiles)
+template <int NT, class FA, class FB>
+__device__ __forceinline__ void tgemm(float (&acc)[NT][4], FA a, FB b, int m0, int n0, int g, int t) {
 #pragma unroll 2
     for (int k0 = 0; k0 < 64; k0 += 8) {
         const uint32_t af[4] = {to_tf32(a(m0 + g, k0 + t)), to_tf32(a(m0 + g + 8, k0 + t)), to_tf32(a(m0 + g, k0 + t + 4)),
                                 to_tf32(a(m0 + g + 8, k0 + t + 4))};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < NT; ++j) {
             const uint32_t bf[2] = {to_tf32(b(k0 + t, n0 + 8 * j + g)), to_tf32(b(k0 + t + 4, n0 + 8 * j + g))};
             mma_tf32_16x8x8(acc[j], af, bf);
         }
@@ -452,22 +452,22 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
     const int tid = threadIdx.x, lane = tid & 31;
     const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
     const int g8 = lane >> 2, t4 = lane & 3;
-    const int mt = warp & 3, nh = warp >> 2;
-    const int m0 = 16 * mt, n0 = 64 * nh, n0s = 32 * nh;  // [64][128] and [64][64] warp tiles
+    const int mt = warp & 3, nq = warp >> 2;
+    const int m0 = 16 * mt, n0 = 32 * nq, n0s = 16 * nq;  // [64][128] and [64][64] warp tiles
     const int H = P.H;
     const uint32_t sb = smem_u32(sm);
     float *rk = reinterpret_cast<float *>(sm + XM_RK), *rq = reinterpret_cast<float *>(sm + XM_RQ);
     float *bb = reinterpret_cast<float *>(sm + XM_B), *dbs = reinterpret_cast<float *>(sm + XM_DB);
     float *dgc = reinterpret_cast<float *>(sm + XM_DGC), *dgam = reinterpret_cast<float *>(sm + XM_DGAM);
     float *red = reinterpret_cast<float *>(sm + XM_RED);
+    float *Gs = reinterpret_cast<float *>(sm + X_G);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + XM_BAR);
     if (tid == 0) { mbar_init(bar, 1); fence_mbar_init(); }
     __syncthreads();
     uint32_t phase = 0;
     const float lb = P.lb;
-    const Pad pq{sb + X_Q}, pk{sb + X_K};
-
     const long long n_items = P.n_items >= 0 ? P.n_items : (long long)P.chunk_off[P.N] * H;
+
     for (long long item = blockIdx.x; item < n_items; item += gridDim.x) {
         const long long gc = item / H;
         const int h = (int)(item % H);
@@ -512,34 +512,38 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
         }
         cp_async_wait_all();
         __syncthreads();
-        // ---------------- norms (4 threads per row), G (a thread per channel)
+        // ---------------- norms (8 threads per row); G: 4 threads per channel, 16 rows each
         {
-            const int r = tid >> 2, part = tid & 3;
+            const int r = tid >> 3, part = tid & 7;
             float sk = 0.f, sq = 0.f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
+            for (int j = 0; j < 2; ++j) {
                 float fk[8], fq[8];
-                unpack8(lds128(sm, X_K + r * (2 * LP) + (part * 4 + j) * 16), fk);
-                unpack8(lds128(sm, X_Q + r * (2 * LP) + (part * 4 + j) * 16), fq);
+                unpack8(lds128(sm, X_K + r * (2 * LP) + (part * 2 + j) * 16), fk);
+                unpack8(lds128(sm, X_Q + r * (2 * LP) + (part * 2 + j) * 16), fq);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) { sk = fmaf(fk[e], fk[e], sk); sq = fmaf(fq[e], fq[e], sq); }
             }
-            sk += __shfl_xor_sync(0xffffffffu, sk, 1);
-            sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-            sk += __shfl_xor_sync(0xffffffffu, sk, 2);
-            sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) {
+                sk += __shfl_xor_sync(0xffffffffu, sk, o);
+                sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            }
             if (part == 0) {
                 rk[r] = r < L ? (P.use_l2 ? rsqrtf(sk + 1e-6f) : 1.f) : 0.f;
                 rq[r] = r < L ? (P.use_l2 ? rsqrtf(sq + 1e-6f) : 1.f) : 0.f;
             }
         }
-        if (tid < D) {
+        {
+            const int c = tid & 127, part = tid >> 7;
             float run = 0.f;
-            for (int r = 0; r < C; ++r) {
-                const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + Y_DW + r * (2 * LP) + 2 * tid));
+#pragma unroll 4
+            for (int r = 16 * part; r < 16 * part + 16; ++r) {
+                const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + Y_DW + r * (2 * LP) + 2 * c));
                 run += r < L ? fmaxf(x, lb) : 0.f;
-                *reinterpret_cast<float *>(sm + X_G + (r * LG + tid) * 4) = run;
+                Gs[r * LG + c] = run;
             }
+            red[part * 128 + c] = run;
         }
         const bool ok = mbar_wait(bar, phase, kWaitLimitNs);
         phase ^= 1;
@@ -549,6 +553,13 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
                 if (P.status) atomicOr(P.status, 1);
             }
             return;
+        }
+        {   // carries of the G parts
+            const int c = tid & 127, part = tid >> 7;
+            float carry = 0.f;
+            for (int p2 = 0; p2 < part; ++p2) carry += red[p2 * 128 + c];
+            if (part > 0)
+                for (int r = 16 * part; r < 16 * part + 16; ++r) Gs[r * LG + c] += carry;
         }
         // D~^T -> D^T (times |k_s|, zero for rows past the chunk)
         for (int e = tid; e < 128 * 8; e += NTI) {
@@ -564,53 +575,52 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
             sts128(sm, off, pack8(y));
         }
 
-        float dq_[32], dk_[32], dG_[32];
+        float dq_[16], dk_[16], dG_[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) dq_[e] = dk_[e] = dG_[e] = 0.f;
-        // element (j, hi) pair of the [64][128] warp tile: row m0 + g8 + 8 hi, columns c, c + 1
+        for (int e = 0; e < 16; ++e) dq_[e] = dk_[e] = dG_[e] = 0.f;
+        // element pair (j, hi) of the [64][128] warp tile: row m0 + g8 + 8 hi, columns c, c + 1
         auto erow = [&](int hi) { return m0 + g8 + 8 * hi; };
         auto ecol = [&](int j) { return n0 + 8 * j + 2 * t4; };
-        auto G2 = [&](int r, int c) { return ldf2(sm, X_G + (r * LG + c) * 4); };
+        auto G2 = [&](int r, int c) { return *reinterpret_cast<const float2 *>(Gs + r * LG + c); };
         auto kh2 = [&](int r, int c) { const float2 x = ldb2(sm, X_K + r * (2 * LP) + 2 * c); const float s = rk[r]; return make_float2(x.x * s, x.y * s); };
         auto qh2 = [&](int r, int c) { const float2 x = ldb2(sm, X_Q + r * (2 * LP) + 2 * c); const float s = rq[r]; return make_float2(x.x * s, x.y * s); };
 
         __syncthreads();
         // ---------------- P1: dQtil = scale dO S^T;  P2: dW = -dD S^T -> bf16 tile
         {
-            float acc[8][4];
+            float acc[4][4];
             zero(acc);
-            wgemm<8, false, true>(acc, Pad{sb + Y_DO}, Img{sb + Y_S0, 128}, m0, n0, 0, 128, lane);
+            wgemm<4, false, true>(acc, Pad{sb + Y_DO}, Img{sb + Y_S0, 128}, m0, n0, 0, 128, lane);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
                     const int r = erow(hi), c = ecol(j), e = 4 * j + 2 * hi;
                     const float2 G = G2(r, c), q = qh2(r, c);
-                    const float ea = e2(G.x), eb = e2(G.y);
-                    const float va = P.scale * acc[j][2 * hi] * ea, vb = P.scale * acc[j][2 * hi + 1] * eb;
+                    const float va = P.scale * acc[j][2 * hi] * e2(G.x), vb = P.scale * acc[j][2 * hi + 1] * e2(G.y);
                     dq_[e] += va; dq_[e + 1] += vb;
                     dG_[e] += va * q.x; dG_[e + 1] += vb * q.y;
                 }
         }
         {
-            float acc[8][4];
+            float acc[4][4];
             zero(acc);
-            wgemm<8, true, true>(acc, Img{sb + Y_DD, 128}, Img{sb + Y_S0, 128}, m0, n0, 0, 128, lane);
+            wgemm<4, true, true>(acc, Img{sb + Y_DD, 128}, Img{sb + Y_S0, 128}, m0, n0, 0, 128, lane);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi)
                     stb2(sm, Y_DW + erow(hi) * (2 * LP) + 2 * ecol(j), -acc[j][2 * hi], -acc[j][2 * hi + 1]);
         }
-        // ---------------- gamma_c sum_v S[c][v] dS_C[c][v]: thread (8 channels, 8 values)
+        // ---------------- gamma_c sum_v S[c][v] dS_C[c][v]: thread (8 channels, 4 values)
         {
             const int cs = tid & 15, vg = tid >> 4;
             float a8[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) a8[j] = 0.f;
-#pragma unroll 2
-            for (int u = 0; u < 8; ++u) {
-                const int vv = 8 * vg + u;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int vv = 4 * vg + u;
                 float s8[8], d8[8];
                 unpack8(lds128(sm, Y_S0 + sw128_chunk(vv, 8 * cs, 128)), s8);
                 unpack8(lds128(sm, Y_DS + sw128_chunk(vv, 8 * cs, 128)), d8);
@@ -627,18 +637,17 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
         if (tid < D) {
             float s = 0.f;
 #pragma unroll
-            for (int w = 0; w < 8; ++w) s += red[w * 128 + tid];
-            const float G63 = *reinterpret_cast<const float *>(sm + X_G + (63 * LG + tid) * 4);
-            dgam[tid] = s * e2(G63);
+            for (int w = 0; w < NTI / 32; ++w) s += red[w * 128 + tid];
+            dgam[tid] = s * e2(Gs[63 * LG + tid]);
         }
         // ---------------- P4: dKhat = D dS_C^T
         {
-            float acc[8][4];
+            float acc[4][4];
             zero(acc);
-            wgemm<8, true, true>(acc, Img{sb + Y_DL, 128}, Img{sb + Y_DS, 128}, m0, n0, 0, 128, lane);
-            float cs_[16];
+            wgemm<4, true, true>(acc, Img{sb + Y_DL, 128}, Img{sb + Y_DS, 128}, m0, n0, 0, 128, lane);
+            float cs_[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 4; ++j) {
                 const int c = ecol(j);
                 const float2 GC = G2(63, c);
                 cs_[2 * j] = cs_[2 * j + 1] = 0.f;
@@ -655,7 +664,7 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
                 }
             }
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < 8; ++j) {
                 float x = cs_[j];
                 x += __shfl_xor_sync(0xffffffffu, x, 4);
                 x += __shfl_xor_sync(0xffffffffu, x, 8);
@@ -664,7 +673,7 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
             }
             if (g8 == 0)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < 4; ++j) {
                     dgc[mt * 128 + ecol(j)] = cs_[2 * j];
                     dgc[mt * 128 + ecol(j) + 1] = cs_[2 * j + 1];
                 }
@@ -688,11 +697,11 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
         }
         // ---------------- P3: dA_qk = scale dO D^T (s <= r) -> bf16
         {
-            float acc[4][4];
+            float acc[2][4];
             zero(acc);
-            wgemm<4, false, true>(acc, Pad{sb + Y_DO}, Img{sb + Y_DL, 128}, m0, n0s, 0, 128, lane);
+            wgemm<2, false, true>(acc, Pad{sb + Y_DO}, Img{sb + Y_DL, 128}, m0, n0s, 0, 128, lane);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
                     const int r = erow(hi), c = n0s + 8 * j + 2 * t4;
@@ -710,14 +719,14 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
         }
         __syncthreads();
         // ---------------- P5: dT' = dD V^T + dW Ktil^T -> fp32
+        float *dtp = reinterpret_cast<float *>(sm + Y_DTP);
         {
-            float acc[4][4];
+            float acc[2][4];
             zero(acc);
-            wgemm<4, true, false>(acc, Img{sb + Y_DD, 128}, Pad{sb + Y_V}, m0, n0s, 0, 128, lane);
-            wgemm<4, false, false>(acc, Pad{sb + Y_DW}, Pad{sb + Y_KT}, m0, n0s, 0, 128, lane);
-            float *dtp = reinterpret_cast<float *>(sm + Y_DTP);
+            wgemm<2, true, false>(acc, Img{sb + Y_DD, 128}, Pad{sb + Y_V}, m0, n0s, 0, 128, lane);
+            wgemm<2, false, false>(acc, Pad{sb + Y_DW}, Pad{sb + Y_KT}, m0, n0s, 0, 128, lane);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
                     const int r = erow(hi), c = n0s + 8 * j + 2 * t4;
@@ -726,11 +735,11 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
         }
         // ---------------- P6: dV = T'^T dD (out); dKtil = T'^T dW
         {
-            float acc[8][4];
+            float acc[4][4];
             zero(acc);
-            wgemm<8, true, false>(acc, Img{sb + Y_TP, 64}, Img{sb + Y_DD, 128}, m0, n0, 0, 64, lane);
+            wgemm<4, true, false>(acc, Img{sb + Y_TP, 64}, Img{sb + Y_DD, 128}, m0, n0, 0, 64, lane);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
                     const int r = erow(hi);
@@ -740,17 +749,16 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
                 }
         }
         {
-            float acc[8][4];
+            float acc[4][4];
             zero(acc);
-            wgemm<8, true, true>(acc, Img{sb + Y_TP, 64}, Pad{sb + Y_DW}, m0, n0, 0, 64, lane);
+            wgemm<4, true, true>(acc, Img{sb + Y_TP, 64}, Pad{sb + Y_DW}, m0, n0, 0, 64, lane);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
                     const int r = erow(hi), c = ecol(j), e = 4 * j + 2 * hi;
                     const float2 G = G2(r, c), k = kh2(r, c);
-                    const float ea = e2(G.x), eb = e2(G.y);
-                    const float xa = acc[j][2 * hi] * ea, xb = acc[j][2 * hi + 1] * eb;
+                    const float xa = acc[j][2 * hi] * e2(G.x), xb = acc[j][2 * hi + 1] * e2(G.y);
                     dk_[e] += xa; dk_[e + 1] += xb;
                     dG_[e] += xa * k.x; dG_[e + 1] += xb * k.y;
                 }
@@ -759,6 +767,7 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
         // ---------------- the k tiles of the block-referenced products
         // B_j (j = 1..3): rows s < 16 j hold k^_s e^{E_j - G_s}, rows r >= 16 j hold
         // k^_r e^{G_r - E_j} (E_j = G_{16 j - 1}); XD / YD: k^ e^{+-(G - M_b)}, M_b = G_{16 b + 7}.
+        // The q side (q_side) writes only XD and the rows r >= 16 j of the B_j, from q^.
         auto build_k = [&](uint32_t yd, uint32_t xd, uint32_t b1, uint32_t b2, uint32_t b3, bool q_side) {
             for (int e = tid; e < 64 * 64; e += NTI) {
                 const int r = e >> 6, c = 2 * (e & 63), blk = r >> 4;
@@ -779,43 +788,38 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
         };
         build_k(Y_KYD, Y_KXD, Y_KB1, Y_KB2, Y_KB3, false);
         __syncthreads();
-        // ---------------- A_kk (strict lower) -> fp32: warp (mt, nh), column blocks 2 nh, 2 nh + 1
+        // ---------------- A_kk (strict lower) -> fp32: warp (mt, nq) forms block (mt, nq)
+        float *af = reinterpret_cast<float *>(sm + Y_AF);
         {
-            float *af = reinterpret_cast<float *>(sm + Y_AF);
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                const int cbk = 2 * nh + p;
-                float acc[2][4];
-                zero(acc);
-                if (cbk < mt) {
-                    const uint32_t bt = mt == 1 ? Y_KB1 : mt == 2 ? Y_KB2 : Y_KB3;
-                    wgemm<2, false, false>(acc, Pad{sb + bt}, Pad{sb + bt}, m0, 16 * cbk, 0, 128, lane);
-                } else if (cbk == mt) {
-                    wgemm<2, false, false>(acc, Pad{sb + Y_KXD}, Pad{sb + Y_KYD}, m0, 16 * cbk, 0, 128, lane);
-                }
-#pragma unroll
-                for (int j = 0; j < 2; ++j)
-#pragma unroll
-                    for (int hi = 0; hi < 2; ++hi) {
-                        const int r = erow(hi), c = 16 * cbk + 8 * j + 2 * t4;
-                        *reinterpret_cast<float2 *>(af + r * LF + c) =
-                            make_float2(c < r ? acc[j][2 * hi] : 0.f, c + 1 < r ? acc[j][2 * hi + 1] : 0.f);
-                    }
+            const int cbk = nq;
+            float acc[2][4];
+            zero(acc);
+            if (cbk < mt) {
+                const uint32_t bt = mt == 1 ? Y_KB1 : mt == 2 ? Y_KB2 : Y_KB3;
+                wgemm<2, false, false>(acc, Pad{sb + bt}, Pad{sb + bt}, m0, 16 * cbk, 0, 128, lane);
+            } else if (cbk == mt) {
+                wgemm<2, false, false>(acc, Pad{sb + Y_KXD}, Pad{sb + Y_KYD}, m0, 16 * cbk, 0, 128, lane);
             }
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi) {
+                    const int r = erow(hi), c = 16 * cbk + 8 * j + 2 * t4;
+                    *reinterpret_cast<float2 *>(af + r * LF + c) =
+                        make_float2(c < r ? acc[j][2 * hi] : 0.f, c + 1 < r ? acc[j][2 * hi + 1] : 0.f);
+                }
         }
         __syncthreads();  // the k tiles are free
         // ---------------- T = I - T' A_kk (tf32)
-        const float *af = reinterpret_cast<const float *>(sm + Y_AF);
         float *tf = reinterpret_cast<float *>(sm + Y_TF);
         float *x1 = reinterpret_cast<float *>(sm + Y_X1);
-        float *dtp = reinterpret_cast<float *>(sm + Y_DTP);
         {
-            float acc[4][4];
+            float acc[2][4];
             zero(acc);
             tgemm(acc, [&](int m, int k) { return bf(sm, Y_TP + sw128(m, k, 64)); },
                   [&](int k, int n) { return af[k * LF + n]; }, m0, n0s, g8, t4);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
                     const int r = erow(hi), c = n0s + 8 * j + 2 * t4;
@@ -824,14 +828,15 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
                 }
         }
         __syncthreads();
-        // db_s = sum_r dT'_rs T_rs (four threads per column); dT' <- dT' diag(b)
+        // db_s = sum_r dT'_rs T_rs (eight threads per column); dT' <- dT' diag(b)
         {
-            const int c = tid >> 2, part = tid & 3;
+            const int c = tid >> 3, part = tid & 7;
             float s = 0.f;
-#pragma unroll 4
-            for (int r = 16 * part; r < 16 * part + 16; ++r) s = fmaf(dtp[r * LF + c], tf[r * LT + c], s);
+#pragma unroll
+            for (int r = 8 * part; r < 8 * part + 8; ++r) s = fmaf(dtp[r * LF + c], tf[r * LT + c], s);
             s += __shfl_xor_sync(0xffffffffu, s, 1);
             s += __shfl_xor_sync(0xffffffffu, s, 2);
+            s += __shfl_xor_sync(0xffffffffu, s, 4);
             if (part == 0) dbs[c] = s;
         }
         __syncthreads();
@@ -839,12 +844,12 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
         __syncthreads();
         // X1 = (dT' diag(b)) T^T
         {
-            float acc[4][4];
+            float acc[2][4];
             zero(acc);
             tgemm(acc, [&](int m, int k) { return dtp[m * LF + k]; }, [&](int k, int n) { return tf[n * LT + k]; }, m0, n0s,
                   g8, t4);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
                     const int r = erow(hi), c = n0s + 8 * j + 2 * t4;
@@ -854,13 +859,13 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
         __syncthreads();
         // dM = -T^T X1;  dA = diag(b) dM (s < r) -> bf16;  db_r += sum_{s<r} dM_rs A_rs
         {
-            float acc[4][4];
+            float acc[2][4];
             zero(acc);
             tgemm(acc, [&](int m, int k) { return tf[k * LT + m]; }, [&](int k, int n) { return x1[k * LF + n]; }, m0, n0s,
                   g8, t4);
             float rs[2] = {0.f, 0.f};
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
                     const int r = erow(hi), c = n0s + 8 * j + 2 * t4;
@@ -872,11 +877,11 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
             for (int hi = 0; hi < 2; ++hi) {
                 rs[hi] += __shfl_xor_sync(0xffffffffu, rs[hi], 1);
                 rs[hi] += __shfl_xor_sync(0xffffffffu, rs[hi], 2);
-                if (t4 == 0) red[nh * 64 + erow(hi)] = rs[hi];
+                if (t4 == 0) red[nq * 64 + erow(hi)] = rs[hi];
             }
         }
         __syncthreads();
-        if (tid < C) dbs[tid] += red[tid] + red[64 + tid];
+        if (tid < C) dbs[tid] += red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid];
         // ---------------- the k tiles again (A_kk's area is reused), then the gated gradients
         build_k(Z_YD, Z_XD, Z_B1, Z_B2, Z_B3, false);
         __syncthreads();
@@ -885,15 +890,17 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
 #pragma unroll 1
         for (int which = 0; which < 2; ++which) {
             const PadA dA = which ? pdaq : pda;
-            float acc[8][4];
-            if (mt > 0) {
+            float acc[4][4];
+#pragma unroll 1
+            for (int part = mt > 0 ? 0 : 1; part < 2; ++part) {  // 0: columns below the block, 1: the block
                 zero(acc);
-                const uint32_t bt = mt == 1 ? Z_B1 : mt == 2 ? Z_B2 : Z_B3;
-                wgemm<8, false, true>(acc, dA, Pad{sb + bt}, m0, n0, 0, 16 * mt, lane);
+                const uint32_t bt = part ? Z_YD : mt == 1 ? Z_B1 : mt == 2 ? Z_B2 : Z_B3;
+                wgemm<4, false, true>(acc, dA, Pad{sb + bt}, m0, n0, part ? 16 * mt : 0, part ? 16 * mt + 16 : 16 * mt, lane);
+                const int refrow = part ? 16 * mt + 7 : 16 * mt - 1;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < 4; ++j) {
                     const int c = ecol(j);
-                    const float2 E = G2(16 * mt - 1, c);
+                    const float2 E = G2(refrow, c);
 #pragma unroll
                     for (int hi = 0; hi < 2; ++hi) {
                         const int r = erow(hi), e = 4 * j + 2 * hi;
@@ -902,21 +909,6 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
                         if (which) { dq_[e] += za; dq_[e + 1] += zb; } else { dk_[e] += za; dk_[e + 1] += zb; }
                         dG_[e] += za * x.x; dG_[e + 1] += zb * x.y;
                     }
-                }
-            }
-            zero(acc);
-            wgemm<8, false, true>(acc, dA, Pad{sb + Z_YD}, m0, n0, 16 * mt, 16 * mt + 16, lane);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int c = ecol(j);
-                const float2 M = G2(16 * mt + 7, c);
-#pragma unroll
-                for (int hi = 0; hi < 2; ++hi) {
-                    const int r = erow(hi), e = 4 * j + 2 * hi;
-                    const float2 G = G2(r, c), x = which ? qh2(r, c) : kh2(r, c);
-                    const float za = acc[j][2 * hi] * e2(G.x - M.x), zb = acc[j][2 * hi + 1] * e2(G.y - M.y);
-                    if (which) { dq_[e] += za; dq_[e + 1] += zb; } else { dk_[e] += za; dk_[e + 1] += zb; }
-                    dG_[e] += za * x.x; dG_[e + 1] += zb * x.y;
                 }
             }
         }
@@ -929,15 +921,18 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
                 __syncthreads();
             }
             const PadA dA = which ? pdaq : pda;
-            float acc[8][4];
-            if (mt < 3) {
+            float acc[4][4];
+#pragma unroll 1
+            for (int part = mt < 3 ? 0 : 1; part < 2; ++part) {  // 0: rows above the block, 1: the block
                 zero(acc);
-                const uint32_t bt = mt == 0 ? Z_B1 : mt == 1 ? Z_B2 : Z_B3;
-                wgemm<8, true, true>(acc, dA, Pad{sb + bt}, m0, n0, 16 * mt + 16, 64, lane);
+                const uint32_t bt = part ? Z_XD : mt == 0 ? Z_B1 : mt == 1 ? Z_B2 : Z_B3;
+                wgemm<4, true, true>(acc, dA, Pad{sb + bt}, m0, n0, part ? 16 * mt : 16 * mt + 16, part ? 16 * mt + 16 : 64,
+                                     lane);
+                const int refrow = part ? 16 * mt + 7 : 16 * mt + 15;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
+                for (int j = 0; j < 4; ++j) {
                     const int c = ecol(j);
-                    const float2 E = G2(16 * mt + 15, c);
+                    const float2 E = G2(refrow, c);
 #pragma unroll
                     for (int hi = 0; hi < 2; ++hi) {
                         const int r = erow(hi), e = 4 * j + 2 * hi;
@@ -948,28 +943,13 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
                     }
                 }
             }
-            zero(acc);
-            wgemm<8, true, true>(acc, dA, Pad{sb + Z_XD}, m0, n0, 16 * mt, 16 * mt + 16, lane);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int c = ecol(j);
-                const float2 M = G2(16 * mt + 7, c);
-#pragma unroll
-                for (int hi = 0; hi < 2; ++hi) {
-                    const int r = erow(hi), e = 4 * j + 2 * hi;
-                    const float2 G = G2(r, c), k = kh2(r, c);
-                    const float za = acc[j][2 * hi] * e2(M.x - G.x), zb = acc[j][2 * hi + 1] * e2(M.y - G.y);
-                    dk_[e] += za; dk_[e + 1] += zb;
-                    dG_[e] -= za * k.x; dG_[e + 1] -= zb * k.y;
-                }
-            }
         }
         // ---------------- outputs
-        // row dots k^ . dk^ and q^ . dq^ (quad sums, then the two column halves)
+        // row dots k^ . dk^ and q^ . dq^ (quad sums, then the four column quarters)
         {
             float sk2[2] = {0.f, 0.f}, sq2[2] = {0.f, 0.f};
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
                     const int r = erow(hi), c = ecol(j), e = 4 * j + 2 * hi;
@@ -988,50 +968,50 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
             if (t4 == 0)
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
-                    red[nh * 64 + erow(hi)] = sk2[hi];
-                    red[128 + nh * 64 + erow(hi)] = sq2[hi];
+                    red[nq * 64 + erow(hi)] = sk2[hi];
+                    red[256 + nq * 64 + erow(hi)] = sq2[hi];
                 }
             // dG into G's area (every read of G is behind the barrier above)
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+            for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
                     const int e = 4 * j + 2 * hi;
-                    *reinterpret_cast<float2 *>(sm + X_G + (erow(hi) * LG + ecol(j)) * 4) = make_float2(dG_[e], dG_[e + 1]);
+                    *reinterpret_cast<float2 *>(Gs + erow(hi) * LG + ecol(j)) = make_float2(dG_[e], dG_[e + 1]);
                 }
         }
         __syncthreads();
-        {
-            const float *rdot = red;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 4; ++j)
 #pragma unroll
-                for (int hi = 0; hi < 2; ++hi) {
-                    const int r = erow(hi), c = ecol(j), e = 4 * j + 2 * hi;
-                    if (r >= L) continue;
-                    const float dotk = rdot[r] + rdot[64 + r], dotq = rdot[128 + r] + rdot[192 + r];
-                    const float2 k = kh2(r, c), q = qh2(r, c);
-                    float ka = dk_[e], kb = dk_[e + 1], qa = dq_[e], qb = dq_[e + 1];
-                    if (P.use_l2) {
-                        ka = rk[r] * (ka - k.x * dotk); kb = rk[r] * (kb - k.y * dotk);
-                        qa = rq[r] * (qa - q.x * dotq); qb = rq[r] * (qb - q.y * dotq);
-                    }
-                    const long long o = (t0 + r) * rowstride + (long long)h * D + c;
-                    *reinterpret_cast<__nv_bfloat162 *>(P.dk + o) = __floats2bfloat162_rn(ka, kb);
-                    *reinterpret_cast<__nv_bfloat162 *>(P.dq + o) = __floats2bfloat162_rn(qa, qb);
+            for (int hi = 0; hi < 2; ++hi) {
+                const int r = erow(hi), c = ecol(j), e = 4 * j + 2 * hi;
+                if (r >= L) continue;
+                const float dotk = red[r] + red[64 + r] + red[128 + r] + red[192 + r];
+                const float dotq = red[256 + r] + red[320 + r] + red[384 + r] + red[448 + r];
+                const float2 k = kh2(r, c), q = qh2(r, c);
+                float ka = dk_[e], kb = dk_[e + 1], qa = dq_[e], qb = dq_[e + 1];
+                if (P.use_l2) {
+                    ka = rk[r] * (ka - k.x * dotk); kb = rk[r] * (kb - k.y * dotk);
+                    qa = rq[r] * (qa - q.x * dotq); qb = rq[r] * (qb - q.y * dotq);
                 }
-        }
-        // dg: reverse in-chunk cumsum of dG (with dG_C on the last row), clamp mask
+                const long long o = (t0 + r) * rowstride + (long long)h * D + c;
+                *reinterpret_cast<__nv_bfloat162 *>(P.dk + o) = __floats2bfloat162_rn(ka, kb);
+                *reinterpret_cast<__nv_bfloat162 *>(P.dq + o) = __floats2bfloat162_rn(qa, qb);
+            }
+        // dg: reverse in-chunk cumsum of dG (with dG_C on the last row), clamp mask; four
+        // threads per channel, 16 rows each
         {
-            const int c = tid & 127, part = tid >> 7;  // part 1: rows 32..63, part 0: rows 0..31
-            float *gcol = reinterpret_cast<float *>(sm + X_G) + c;
+            const int c = tid & 127, part = tid >> 7;
+            float *gcol = Gs + c;
             float run = 0.f;
-            if (part == 1) run = dgc[c] + dgc[128 + c] + dgc[256 + c] + dgc[384 + c] + dgam[c];
-            for (int r = 32 * part + 31; r >= 32 * part; --r) { run += gcol[r * LG]; gcol[r * LG] = run; }
-            if (part == 1) red[512 + c] = run;
+            if (part == 3) run = dgc[c] + dgc[128 + c] + dgc[256 + c] + dgc[384 + c] + dgam[c];
+            for (int r = 16 * part + 15; r >= 16 * part; --r) { run += gcol[r * LG]; gcol[r * LG] = run; }
+            red[512 + part * 128 + c] = run;
             __syncthreads();
-            const float carry = part == 0 ? red[512 + c] : 0.f;
-            for (int r = 32 * part; r < 32 * part + 32; ++r) {
+            float carry = 0.f;
+            for (int p2 = part + 1; p2 < 4; ++p2) carry += red[512 + p2 * 128 + c];
+            for (int r = 16 * part; r < 16 * part + 16; ++r) {
                 if (r >= L) break;
                 const long long o = (t0 + r) * rowstride + (long long)h * D + c;
                 const float graw = __bfloat162float(P.g[o]);
