@@ -42,6 +42,7 @@
 #include "kda_tc_util.cuh"
 #include "kda_stage.cuh"
 #include "kda_record.cuh"
+#include "kda_seg.cuh"
 
 namespace kda {
 
@@ -50,6 +51,9 @@ size_t chunk_2pass_workspace_bytes(const ChunkParams &p);
 uint8_t *chunk_2pass_records(const ChunkParams &p, void *workspace);
 cudaError_t launch_chunk_2pass_save(const ChunkParams &p, void *workspace, const int32_t *cu_host, uint8_t *save,
                                     cudaStream_t st);
+int chunk_2pass_seg_info(const ChunkParams &p, void *workspace, const int32_t **cu_v, const int **chunk_off_v,
+                         const float **M);
+int chunk_2pass_seg_count(const ChunkParams &p);
 
 namespace cb {
 
@@ -161,7 +165,7 @@ __global__ void __launch_bounds__(NTC, 1) kda_cb_dstate_kernel(const __grid_cons
         const int s = i & 1, ci = nchunks - 1 - i;
         const uint32_t so = s * C_STAGE;
         uint8_t *stg = sm + so;
-        if (tid == kSave) bulk_wait_read_all();  // the previous chunk's images were copied out
+        if (tid == kSave && P.bsave) bulk_wait_read_all();  // the previous chunk's images were copied out
         {
             bool ok = true;
             if (warp == 0) {
@@ -215,8 +219,8 @@ __global__ void __launch_bounds__(NTC, 1) kda_cb_dstate_kernel(const __grid_cons
         tc_fence_before();
         bar_sync(1, NTC);
         tc_fence_after();
-        uint8_t *bsave = P.bsave + ((c_first + ci) * H + h) * (long long)BR_BYTES;
-        if (tid == kSave) { bulk_store(bsave + BR_DS, sm + C_DST, 32768); bulk_commit(); }
+        uint8_t *bsave = P.bsave ? P.bsave + ((c_first + ci) * H + h) * (long long)BR_BYTES : nullptr;
+        if (tid == kSave && bsave) { bulk_store(bsave + BR_DS, sm + C_DST, 32768); bulk_commit(); }
         if (warp == 0) {
             const uint32_t ld = elect_one();
 #pragma unroll
@@ -250,7 +254,7 @@ __global__ void __launch_bounds__(NTC, 1) kda_cb_dstate_kernel(const __grid_cons
         tc_fence_before();
         bar_sync(1, NTC);
         tc_fence_after();
-        if (tid == kSave) { bulk_store(bsave + BR_DD, sm + C_DDT, 16384); bulk_commit(); }
+        if (tid == kSave && bsave) { bulk_store(bsave + BR_DD, sm + C_DDT, 16384); bulk_commit(); }
         if (warp == 0) {
             const uint32_t ld = elect_one();
 #pragma unroll
@@ -293,13 +297,26 @@ __global__ void __launch_bounds__(NTC, 1) kda_cb_dstate_kernel(const __grid_cons
             if (P.status) atomicOr(P.status, 1);
         }
     }
-    if (tid == kSave) bulk_wait_all();
+    if (tid == kSave && P.bsave) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tb, TMC_COLS);
     }
+}
+
+// MT[s] = M[s]^T for packed 128 x 128 states; one 32 x 32 tile per CTA.
+__global__ void __launch_bounds__(256) kda_cb_transpose(const float *M, float *MT) {
+    __shared__ float tile[32][33];
+    const long long b = blockIdx.x, s = b >> 4;
+    const int tr = (int)(b & 15) >> 2, tc = (int)(b & 3);
+    const float *src = M + s * D * D;
+    float *dst = MT + s * D * D;
+    const int x = threadIdx.x & 31, y = threadIdx.x >> 5;
+    for (int i = y; i < 32; i += 8) tile[i][x] = src[(32 * tr + i) * D + 32 * tc + x];
+    __syncthreads();
+    for (int i = y; i < 32; i += 8) dst[(32 * tc + i) * D + 32 * tr + x] = tile[x][i];
 }
 
 // ============================================================== chunk-local gradients
@@ -325,8 +342,9 @@ constexpr uint32_t XM_RK = X_MISC, XM_RQ = X_MISC + 256, XM_B = X_MISC + 512, XM
                    XM_DGC = X_MISC + 1024,   // [4][128] column partials of sum_s dKhat Khat
                    XM_DGAM = X_MISC + 3072,  // [128] gamma_c sum_v S dS_C
                    XM_RED = X_MISC + 3584,   // [16][128] f32 reduction scratch
-                   XM_BAR = XM_RED + 8192;
-constexpr uint32_t X_R = (XM_BAR + 64 + 1023) / 1024 * 1024;      // phase region
+                   XM_BAR = XM_RED + 8192,
+                   XM_DAD = XM_BAR + 64;      // [64] the diagonal of dA_qk
+constexpr uint32_t X_R = (XM_DAD + 256 + 1023) / 1024 * 1024;     // phase region
 // phase A/B
 constexpr uint32_t Y_SV = X_R, Y_S0 = Y_SV + BR_S0, Y_DL = Y_SV + BR_DL, Y_DS = Y_SV + BR_DS, Y_DD = Y_SV + BR_DD;
 constexpr uint32_t Y_DO = X_R + BR_BYTES, Y_DW = Y_DO + PT;       // raw dO; dW (bf16) -- raw g before it
@@ -460,6 +478,7 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
     float *bb = reinterpret_cast<float *>(sm + XM_B), *dbs = reinterpret_cast<float *>(sm + XM_DB);
     float *dgc = reinterpret_cast<float *>(sm + XM_DGC), *dgam = reinterpret_cast<float *>(sm + XM_DGAM);
     float *red = reinterpret_cast<float *>(sm + XM_RED);
+    float *dad = reinterpret_cast<float *>(sm + XM_DAD);
     float *Gs = reinterpret_cast<float *>(sm + X_G);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + XM_BAR);
     if (tid == 0) { mbar_init(bar, 1); fence_mbar_init(); }
@@ -695,7 +714,9 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
             }
             cp_async_commit();
         }
-        // ---------------- P3: dA_qk = scale dO D^T (s <= r) -> bf16
+        // ---------------- P3: dA_qk = scale dO D^T: the part below the diagonal -> bf16, the
+        // diagonal apart (A_qk[r,r] = q^_r . k^_r has no gate factor, so its cotangent goes to
+        // q^ and k^ directly and to no dG: the gated split would leave a rounding residue)
         {
             float acc[2][4];
             zero(acc);
@@ -705,8 +726,10 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
                     const int r = erow(hi), c = n0s + 8 * j + 2 * t4;
-                    stb2(sm, X_DAQ + (r * LA + c) * 2, c <= r ? P.scale * acc[j][2 * hi] : 0.f,
-                         c + 1 <= r ? P.scale * acc[j][2 * hi + 1] : 0.f);
+                    const float va = P.scale * acc[j][2 * hi], vb = P.scale * acc[j][2 * hi + 1];
+                    stb2(sm, X_DAQ + (r * LA + c) * 2, c < r ? va : 0.f, c + 1 < r ? vb : 0.f);
+                    if (c == r) dad[r] = va;
+                    if (c + 1 == r) dad[r] = vb;
                 }
         }
         cp_async_wait_all();
@@ -944,6 +967,17 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
                 }
             }
         }
+        // the diagonal of dA_qk: dq^_r += dA_qk[r,r] k^_r, dk^_r += dA_qk[r,r] q^_r
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int hi = 0; hi < 2; ++hi) {
+                const int r = erow(hi), c = ecol(j), e = 4 * j + 2 * hi;
+                const float2 k = kh2(r, c), q = qh2(r, c);
+                const float d = dad[r];
+                dq_[e] += d * k.x; dq_[e + 1] += d * k.y;
+                dk_[e] += d * q.x; dk_[e + 1] += d * q.y;
+            }
         // ---------------- outputs
         // row dots k^ . dk^ and q^ . dq^ (quad sums, then the four column quarters)
         {
@@ -1056,17 +1090,22 @@ long long cb_max_chunks(const BwdParams &p) {
     return p.cu_seqlens ? ((long long)p.T + C - 1) / C + p.N : (long long)p.N * (((long long)p.T + C - 1) / C);
 }
 
-// Workspace: [the forward's two-pass workspace][backward records][chunk offsets][chunk table]
+// Workspace: [the forward's two-pass workspace][backward records][chunk offsets][chunk
+// table][segment form: per (segment, head) the cotangent offsets N', M^T and the
+// leaving cotangents]
 struct CbLayout {
-    size_t fwd, save, offs, table, total;
+    size_t fwd, save, offs, table, seg, total;
 };
+int cb_seg_count(const BwdParams &p) { return chunk_2pass_seg_count(cb_fwd_params(p)); }
 CbLayout cb_layout(const BwdParams &p) {
     CbLayout L;
     L.fwd = round1k(chunk_2pass_workspace_bytes(cb_fwd_params(p)));
     L.save = (size_t)cb_max_chunks(p) * p.H * BR_BYTES;
     L.offs = p.cu_seqlens ? round1k((size_t)(p.N + 1) * 4) : 0;
     L.table = p.cu_seqlens ? round1k((size_t)cb_max_chunks(p) * 8) + 16384 : 0;
-    L.total = L.fwd + L.save + L.offs + L.table;
+    const int P = cb_seg_count(p);
+    L.seg = P > 1 ? 3 * round1k((size_t)p.N * P * p.H * D * D * 4) : 0;
+    L.total = L.fwd + L.save + L.offs + L.table + L.seg;
     return L;
 }
 
@@ -1117,9 +1156,48 @@ cudaError_t launch_bwd_chunked(const BwdParams &p, void *workspace, cudaStream_t
     if ((e = cudaFuncSetAttribute(kda_cb_dstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEMC_ALLOC)) !=
         cudaSuccess)
         return e;
-    count_launch();
-    kda_cb_dstate_kernel<<<(unsigned)((long long)p.N * p.H), NTC, SMEMC_ALLOC, st>>>(B);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int32_t *cu_v = nullptr;
+    const int *chunk_off_v = nullptr;
+    const float *Mseg = nullptr;
+    const int P = chunk_2pass_seg_info(f, ws, &cu_v, &chunk_off_v, &Mseg);
+    if (P == 1) {
+        count_launch();
+        kda_cb_dstate_kernel<<<(unsigned)((long long)p.N * p.H), NTC, SMEMC_ALLOC, st>>>(B);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    } else {
+        // the segments of the forward's view: the cotangent over a segment is affine in the
+        // cotangent leaving it, dS_start = M^T dS_end + N', so the chain runs once over all
+        // segments from zero (the N'), the segments are walked back with M^T to their
+        // leaving cotangents, and the chain runs again from those (writing the records)
+        const size_t sb = round1k((size_t)p.N * P * p.H * D * D * 4);
+        float *Nrev = reinterpret_cast<float *>(save + Lo.save + Lo.offs + Lo.table);
+        float *MT = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(Nrev) + sb);
+        float *dSend = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(Nrev) + 2 * sb);
+        const long long nv = (long long)p.N * P * p.H;
+        DStateParams Bv = B;
+        Bv.cu_seqlens = cu_v;
+        Bv.chunk_off = chunk_off_v;
+        Bv.T = p.cu_seqlens ? p.T : p.N * p.T;
+        Bv.N = p.N * P;
+        Bv.bsave = nullptr;
+        Bv.dSf = nullptr;
+        Bv.dS0 = Nrev;
+        count_launch();
+        kda_cb_dstate_kernel<<<(unsigned)nv, NTC, SMEMC_ALLOC, st>>>(Bv);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        count_launch();
+        kda_cb_transpose<<<(unsigned)(nv * 16), 256, 0, st>>>(Mseg, MT);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = seg_chain_launch<D>(p.dSf, MT, Nrev, D, (long long)D * D, dSend, p.dS0, p.N, p.H, P, st, 1)) !=
+            cudaSuccess)
+            return e;
+        Bv.bsave = save;
+        Bv.dSf = dSend;
+        Bv.dS0 = nullptr;
+        count_launch();
+        kda_cb_dstate_kernel<<<(unsigned)nv, NTC, SMEMC_ALLOC, st>>>(Bv);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     // the chunk-local gradients: every (chunk, head) of the chunk numbering (varlen: the
     // table's count; slots past it belong to no sequence and are skipped by count)
     IntraBwdParams I;

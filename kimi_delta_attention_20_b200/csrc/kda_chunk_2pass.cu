@@ -1540,6 +1540,25 @@ cudaError_t launch_chunk_2pass_save(const ChunkParams &p, void *workspace, const
     return run_pass2(pf, ws, nullptr, st, 0, 0, 0, save);
 }
 
+int chunk_2pass_seg_count(const ChunkParams &p) { return tp::seg_count(p); }
+
+// Where a segmented forward of p keeps its segment view in ws: returns P (1 when p is not
+// segmented, and nothing is set), the view's cu_seqlens and chunk offsets, and the
+// segment transitions M ([N P, H, 128, 128], S_end = M S_start + N).
+int chunk_2pass_seg_info(const ChunkParams &p, void *workspace, const int32_t **cu_v, const int **chunk_off_v,
+                         const float **M) {
+    using namespace tp;
+    const int P = seg_count(p);
+    if (P == 1) return 1;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const ChunkParams q = seg_view(p, P, reinterpret_cast<const int32_t *>(16));
+    uint8_t *cv = ws + base_workspace_bytes(q);
+    *cu_v = reinterpret_cast<const int32_t *>(cv);
+    *chunk_off_v = reinterpret_cast<const int *>(ws + 1024 + 16384);
+    *M = reinterpret_cast<const float *>(cv + round1k(((size_t)p.N * P + 1) * 4));
+    return P;
+}
+
 // The chunk offsets and table of a varlen batch (the prep kernel also writes the constant
 // tiles to consts, 16 KB).
 cudaError_t chunk_2pass_chunk_table(const int32_t *cu, int N, int *chunk_off, int2 *chunk_tok, uint8_t *consts,
