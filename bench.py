@@ -53,7 +53,7 @@ DECODE_WL = 3
 DECODE_STEPS_PER_PASS = 256
 # kernels one chunk forward launches on the bench workload (set-up, intra-chunk
 # records, exact records, state pass) and the sources they are built from
-CHUNK_SOURCES = ("kda_chunk_2pass.cu", "kda_tc_util.cuh", "kda_sm100.cuh", "kda_common.cuh")
+CHUNK_SOURCES = ("kda_chunk_2pass.cu", "kda_tc_util.cuh", "kda_sm100.cuh", "kda_common.cuh", "kda_record.cuh")
 # the other chunk workloads, timed one launch at a time with L2 flushed in between
 EXTRA_CHUNK_WLS = (1, 2, 5)
 L2_FLUSH_BYTES = 256 << 20
@@ -118,25 +118,28 @@ def token_algorithmic(N, H, D, K):
 # chunk_kda backward: the B1 T8192 H16 d128 lb-5 chunk workload with an output and a
 # final-state cotangent (its 16 (sequence, head) chains run in segment form)
 BWD_WL = 2
-# FP32 FMA peak of the part: 148 SMs x 128 FP32 lanes x 2 flops x 1965 MHz
-FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def bwd_algorithmic(wl):
-    """Flops and bytes of one chunk_kda backward call on workload wl.
+    """Flops and bytes of one chunk_kda backward call on workload wl (d_k = d_v = d),
+    in the chunk form the library runs for it (bf16, d = 128, lower bound >= -5).
 
-    Flops per token-head (fp32, the token recurrence): one forward step to rebuild
-    the entering state (S' = a S, u = S'^T k, S += k delta^T: 5 d_k d_v) and the
-    reverse step (S', u, dS += q do^T, ddelta = dS^T k, the four row sums S' do,
-    dS delta, S' ddelta, dS . S', dS - b k ddelta^T and the decay of dS:
-    18 d_k d_v). Bytes: q, k, v, g, do, beta read, dq, dk, dv, dg, dbeta written,
-    the final-state cotangent read and the initial-state gradient written.
+    Flops per token-head, as for the forward (2 per multiply-add, triangles
+    exploited, C the chunk): the recompute of what the backward needs from the
+    forward (A_kk, A_qk, W, U: 4 C d; W S and Khat^T D: 4 d^2), the cotangent chain
+    (A_qk^T dO: C d; Khat dS, Qtil^T dO, W^T dD: 6 d^2) and the chunk-local terms
+    (dO S^T, dD S^T, D dS^T: 6 d^2; dA_qk, dT' (two), dV, dKtil, A_kk again and the
+    four gated products: 10 C d; the inverse's three C x C x C products, C^2) --
+    15 C d + 16 d^2 + C^2 in all. Bytes: q, k, v, g, do, beta read, dq, dk, dv, dg,
+    dbeta written, the final-state cotangent read and the initial-state gradient
+    written.
     """
     th = wl.tokens * wl.H
     esz = 2
     per_th = 2 * (3 * wl.Dk + 2 * wl.Dv) * esz + 2 * esz
     states = 2 * wl.n_seqs * wl.H * wl.Dk * wl.Dv * 4
-    return th * 23 * wl.Dk * wl.Dv, th * per_th + states
+    C, d = wl.chunk_size, wl.Dk
+    return th * (15 * C * d + 16 * d * d + C * C), th * per_th + states
 
 
 def decode_algorithmic(wl):
@@ -615,10 +618,12 @@ def run_kda(args, rank, world, local_rank):
             "steps_timed": args.steps,
             "workload": "chunk_kda backward: B1 T8192 H16 d128, bf16, lower_bound=-5, output and "
                         "final-state cotangents, initial-state gradient out",
-            "roofline": {"bound": "alu", "achieved": bwd_flops / (bwd_ms * 1e-3) / 1e12,
-                         "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
-                         "frac": bwd_flops / (bwd_ms * 1e-3) / 1e12 / FP32_PEAK_TFLOPS,
-                         "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 x 1965 MHz",
+            "form": "chunked: forward with state saves, cotangent chain on tcgen05 over segments, "
+                    "chunk-local gradients on warp-level MMAs",
+            "roofline": {"bound": "tensor", "achieved": bwd_flops / (bwd_ms * 1e-3) / 1e12,
+                         "peak": tc_peak, "unit": "TFLOP/s",
+                         "frac": bwd_flops / (bwd_ms * 1e-3) / 1e12 / tc_peak,
+                         "peak_kind": peak_kind,
                          "algorithmic_flops_per_launch": bwd_flops,
                          "hbm": {"algorithmic_bytes_per_launch": bwd_bytes,
                                  "achieved_gbs": bwd_bytes / (bwd_ms * 1e-3) / 1e9}},
