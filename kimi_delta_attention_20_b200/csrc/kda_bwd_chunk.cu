@@ -343,8 +343,10 @@ constexpr uint32_t XM_RK = X_MISC, XM_RQ = X_MISC + 256, XM_B = X_MISC + 512, XM
                    XM_DGAM = X_MISC + 3072,  // [128] gamma_c sum_v S dS_C
                    XM_RED = X_MISC + 3584,   // [16][128] f32 reduction scratch
                    XM_BAR = XM_RED + 8192,
-                   XM_DAD = XM_BAR + 64;      // [64] the diagonal of dA_qk
-constexpr uint32_t X_R = (XM_DAD + 256 + 1023) / 1024 * 1024;     // phase region
+                   XM_DAD = XM_BAR + 64,      // [64] the diagonal of dA_qk
+                   XM_MSK = XM_DAD + 256,     // [64][4] u32: g >= lower bound (the clamp passes the gradient)
+                   XM_KN = XM_MSK + 1024;     // [64] |k_r| (with the norm's eps; 1 without the norm, 0 past L)
+constexpr uint32_t X_R = (XM_KN + 256 + 1023) / 1024 * 1024;      // phase region
 // phase A/B
 constexpr uint32_t Y_SV = X_R, Y_S0 = Y_SV + BR_S0, Y_DL = Y_SV + BR_DL, Y_DS = Y_SV + BR_DS, Y_DD = Y_SV + BR_DD;
 constexpr uint32_t Y_DO = X_R + BR_BYTES, Y_DW = Y_DO + PT;       // raw dO; dW (bf16) -- raw g before it
@@ -479,6 +481,8 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
     float *dgc = reinterpret_cast<float *>(sm + XM_DGC), *dgam = reinterpret_cast<float *>(sm + XM_DGAM);
     float *red = reinterpret_cast<float *>(sm + XM_RED);
     float *dad = reinterpret_cast<float *>(sm + XM_DAD);
+    float *knorm = reinterpret_cast<float *>(sm + XM_KN);
+    uint32_t *gmask = reinterpret_cast<uint32_t *>(sm + XM_MSK);
     float *Gs = reinterpret_cast<float *>(sm + X_G);
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + XM_BAR);
     if (tid == 0) { mbar_init(bar, 1); fence_mbar_init(); }
@@ -487,38 +491,54 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
     const float lb = P.lb;
     const long long n_items = P.n_items >= 0 ? P.n_items : (long long)P.chunk_off[P.N] * H;
 
-    for (long long item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const long long gc = item / H;
-        const int h = (int)(item % H);
-        long long t0;
-        int L;
-        if (P.cu_seqlens) {  // the sequence holding global chunk gc
+    const long long rowstride = (long long)H * D;  // elements between token rows
+    // first token and rows of an item's chunk
+    auto locate = [&](long long it, long long &t0_, int &L_) {  // item counts are below 2^31
+        const int gc_ = (int)it / H;
+        if (P.cu_seqlens) {  // the sequence holding global chunk gc_
             int lo = 0, hi = P.N - 1;
-            while (lo < hi) { const int mid = (lo + hi + 1) >> 1; if (P.chunk_off[mid] <= gc) lo = mid; else hi = mid - 1; }
-            const long long ci = gc - P.chunk_off[lo];
-            t0 = P.cu_seqlens[lo] + ci * C;
-            L = (int)min((long long)C, (long long)P.cu_seqlens[lo + 1] - t0);
+            while (lo < hi) { const int mid = (lo + hi + 1) >> 1; if (P.chunk_off[mid] <= gc_) lo = mid; else hi = mid - 1; }
+            const int ci = gc_ - P.chunk_off[lo];
+            t0_ = P.cu_seqlens[lo] + ci * C;
+            L_ = (int)min((long long)C, (long long)P.cu_seqlens[lo + 1] - t0_);
         } else {
-            const long long n = gc / P.cpr, ci = gc % P.cpr;
-            t0 = n * P.T + ci * C;
-            L = (int)min((long long)C, (long long)P.T - ci * C);
+            const int n = gc_ / P.cpr, ci = gc_ - n * P.cpr;
+            t0_ = (long long)n * P.T + ci * C;
+            L_ = min(C, P.T - ci * C);
         }
-        const long long rowstride = (long long)H * D;  // elements between token rows
-        auto grow = [&](const __nv_bfloat16 *base, int r) { return base + (t0 + r) * rowstride + (long long)h * D; };
-
-        // ---------------- loads: the backward record (bulk), raw q, k, dO, g (cp.async)
-        if (tid == 0) {
+    };
+    // an item's inputs: the backward record (bulk), then raw rows (cp.async, one group);
+    // which: 0 = record, dO and g;  1 = q and k
+    auto issue_loads = [&](long long it, int which) {
+        long long t0_;
+        int L_;
+        locate(it, t0_, L_);
+        const int h_ = (int)it % H;
+        if (which == 0 && tid == 0) {
             mbar_arrive_expect_tx(bar, BR_BYTES);
-            bulk_load(sm + Y_SV, P.bsave + item * (long long)BR_BYTES, BR_BYTES, bar);
+            bulk_load(sm + Y_SV, P.bsave + it * (long long)BR_BYTES, BR_BYTES, bar);
         }
-        for (int e = tid; e < 4 * 64 * 16; e += NTI) {
-            const int which = e >> 10, r = (e >> 4) & 63, ch = e & 15;
-            const uint32_t dst = (which == 0 ? X_Q : which == 1 ? X_K : which == 2 ? Y_DO : Y_DW) + r * (2 * LP) + ch * 16;
-            const __nv_bfloat16 *src = which == 0 ? P.q : which == 1 ? P.k : which == 2 ? P.dout : P.g;
-            if (r < L) cp_async16(sm + dst, grow(src, r) + ch * 8);
+        for (int e = tid; e < 2 * 64 * 16; e += NTI) {
+            const int sel = e >> 10, r = (e >> 4) & 63, ch = e & 15;
+            const uint32_t base = which ? (sel ? X_K : X_Q) : (sel ? Y_DW : Y_DO);
+            const __nv_bfloat16 *src = which ? (sel ? P.k : P.q) : (sel ? P.g : P.dout);
+            const uint32_t dst = base + r * (2 * LP) + ch * 16;
+            if (r < L_) cp_async16(sm + dst, src + (t0_ + r) * rowstride + (long long)h_ * D + ch * 8);
             else *reinterpret_cast<uint4 *>(sm + dst) = make_uint4(0u, 0u, 0u, 0u);
         }
         cp_async_commit();
+    };
+    if (blockIdx.x < n_items) { issue_loads(blockIdx.x, 0); issue_loads(blockIdx.x, 1); }
+
+    for (long long item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int h = (int)item % H;
+        long long t0;
+        int L;
+        locate(item, t0, L);
+        const long long next = item + gridDim.x;
+        auto grow = [&](const __nv_bfloat16 *base, int r) { return base + (t0 + r) * rowstride + (long long)h * D; };
+
+        // ---------------- this item's inputs were issued before (the previous item's tail)
         if (tid < C) {
             float b = 0.f;
             if (tid < L) {
@@ -551,9 +571,10 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
             if (part == 0) {
                 rk[r] = r < L ? (P.use_l2 ? rsqrtf(sk + 1e-6f) : 1.f) : 0.f;
                 rq[r] = r < L ? (P.use_l2 ? rsqrtf(sq + 1e-6f) : 1.f) : 0.f;
+                knorm[r] = r < L ? (P.use_l2 ? sqrtf(sk + 1e-6f) : 1.f) : 0.f;
             }
         }
-        {
+        {   // a warp: 32 channels of one 16-row part; the clamp mask by ballot
             const int c = tid & 127, part = tid >> 7;
             float run = 0.f;
 #pragma unroll 4
@@ -561,6 +582,8 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
                 const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + Y_DW + r * (2 * LP) + 2 * c));
                 run += r < L ? fmaxf(x, lb) : 0.f;
                 Gs[r * LG + c] = run;
+                const uint32_t m = __ballot_sync(0xffffffffu, x >= lb);
+                if (lane == 0) gmask[r * 4 + (c >> 5)] = m;
             }
             red[part * 128 + c] = run;
         }
@@ -587,10 +610,7 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
             float y[8];
             unpack8(lds128(sm, off), y);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float r_ = rk[8 * cs + j];
-                y[j] = r_ > 0.f ? y[j] / r_ : 0.f;
-            }
+            for (int j = 0; j < 8; ++j) y[j] *= knorm[8 * cs + j];
             sts128(sm, off, pack8(y));
         }
 
@@ -862,15 +882,12 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
             s += __shfl_xor_sync(0xffffffffu, s, 4);
             if (part == 0) dbs[c] = s;
         }
-        __syncthreads();
-        for (int e = tid; e < 64 * 64; e += NTI) { const int r = e >> 6, c = e & 63; dtp[r * LF + c] *= bb[c]; }
-        __syncthreads();
         // X1 = (dT' diag(b)) T^T
         {
             float acc[2][4];
             zero(acc);
-            tgemm(acc, [&](int m, int k) { return dtp[m * LF + k]; }, [&](int k, int n) { return tf[n * LT + k]; }, m0, n0s,
-                  g8, t4);
+            tgemm(acc, [&](int m, int k) { return dtp[m * LF + k] * bb[k]; }, [&](int k, int n) { return tf[n * LT + k]; },
+                  m0, n0s, g8, t4);
 #pragma unroll
             for (int j = 0; j < 2; ++j)
 #pragma unroll
@@ -967,6 +984,8 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
                 }
             }
         }
+        __syncthreads();  // the tile areas (record, dO, dW) are free: the next item's record, dO and g
+        if (next < n_items) issue_loads(next, 0);
         // the diagonal of dA_qk: dq^_r += dA_qk[r,r] k^_r, dk^_r += dA_qk[r,r] q^_r
 #pragma unroll
         for (int j = 0; j < 4; ++j)
@@ -1033,23 +1052,27 @@ __global__ void __launch_bounds__(NTI, 1) kda_cb_intra_kernel(const __grid_const
                 *reinterpret_cast<__nv_bfloat162 *>(P.dk + o) = __floats2bfloat162_rn(ka, kb);
                 *reinterpret_cast<__nv_bfloat162 *>(P.dq + o) = __floats2bfloat162_rn(qa, qb);
             }
+        __syncthreads();  // raw q and k are no longer read: the next item's
+        if (next < n_items) issue_loads(next, 1);
         // dg: reverse in-chunk cumsum of dG (with dG_C on the last row), clamp mask; four
         // threads per channel, 16 rows each
         {
             const int c = tid & 127, part = tid >> 7;
-            float *gcol = Gs + c;
-            float run = 0.f;
-            if (part == 3) run = dgc[c] + dgc[128 + c] + dgc[256 + c] + dgc[384 + c] + dgam[c];
-            for (int r = 16 * part + 15; r >= 16 * part; --r) { run += gcol[r * LG]; gcol[r * LG] = run; }
+            const float *gcol = Gs + c;
+            float sfx[16];
+            float run = part == 3 ? dgc[c] + dgc[128 + c] + dgc[256 + c] + dgc[384 + c] + dgam[c] : 0.f;
+#pragma unroll
+            for (int i = 15; i >= 0; --i) { run += gcol[(16 * part + i) * LG]; sfx[i] = run; }
             red[512 + part * 128 + c] = run;
             __syncthreads();
             float carry = 0.f;
             for (int p2 = part + 1; p2 < 4; ++p2) carry += red[512 + p2 * 128 + c];
-            for (int r = 16 * part; r < 16 * part + 16; ++r) {
-                if (r >= L) break;
-                const long long o = (t0 + r) * rowstride + (long long)h * D + c;
-                const float graw = __bfloat162float(P.g[o]);
-                P.dg[o] = __float2bfloat16_rn(graw >= lb ? gcol[r * LG] + carry : 0.f);
+            __nv_bfloat16 *dgp = P.dg + (t0 + 16 * part) * rowstride + (long long)h * D + c;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int r = 16 * part + i;
+                const bool pass = (gmask[r * 4 + (c >> 5)] >> (c & 31)) & 1u;
+                if (r < L) dgp[i * rowstride] = __float2bfloat16_rn(pass ? sfx[i] + carry : 0.f);
             }
         }
         if (tid < L) {
