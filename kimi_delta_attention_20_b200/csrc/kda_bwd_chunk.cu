@@ -398,20 +398,29 @@ __device__ __forceinline__ void ldsm4t(uint32_t addr, uint32_t (&r)[4]) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
 }
+// Operand tiles: at(row, col) is the shared address of the 16-byte piece at (row, col),
+// col % 8 == 0; kRow16 / kCol16 the address step of 16 rows / 16 columns where that step
+// is a constant (kColLinear: along the columns too).
 // A padded bf16 tile: element (row, col) at base + row * 2 LP + 2 col.
 struct Pad {
     uint32_t base;
+    static constexpr uint32_t kRow16 = 16 * 2 * LP, kCol16 = 32;
+    static constexpr bool kColLinear = true;
     __device__ __forceinline__ uint32_t at(int row, int col) const { return base + (uint32_t)(row * (2 * LP) + 2 * col); }
 };
 // A padded bf16 64 x 64 tile with rows of LA elements.
 struct PadA {
     uint32_t base;
+    static constexpr uint32_t kRow16 = 16 * 2 * LA, kCol16 = 32;
+    static constexpr bool kColLinear = true;
     __device__ __forceinline__ uint32_t at(int row, int col) const { return base + (uint32_t)(row * (2 * LA) + 2 * col); }
 };
-// A swizzled image with `rows` rows (64-column halves).
+// A swizzled image with `rows` rows (64-column halves): linear along the rows only.
 struct Img {
     uint32_t base;
     int rows;
+    static constexpr uint32_t kRow16 = 16 * 128, kCol16 = 0;
+    static constexpr bool kColLinear = false;
     __device__ __forceinline__ uint32_t at(int row, int col) const { return base + sw128_chunk(row, col, rows); }
 };
 
@@ -421,17 +430,28 @@ template <int NT, bool AT, bool BT, class OA, class OB>
 __device__ __forceinline__ void wgemm(float (&acc)[NT][4], const OA &A, const OB &B, int m0, int n0, int k0, int k1,
                                       int lane) {
     const int li = lane & 7, l3 = (lane >> 3) & 1, l4 = lane >> 4;
-#pragma unroll 1
-    for (int k = k0; k < k1; k += 16) {
+    static_assert(AT || OA::kColLinear, "A read along its columns needs a column-linear tile");
+    // this lane's fragment addresses at k0 and their step per 16 of k
+    const uint32_t a0 = AT ? A.at(k0 + li + 8 * l4, m0 + 8 * l3) : A.at(m0 + li + 8 * l3, k0 + 8 * l4);
+    constexpr uint32_t da = AT ? OA::kRow16 : OA::kCol16;
+    constexpr bool b_lin = BT || OB::kColLinear;
+    constexpr uint32_t db = BT ? OB::kRow16 : OB::kCol16;
+    uint32_t b0[NT / 2];
+#pragma unroll
+    for (int p = 0; p < NT / 2; ++p)
+        b0[p] = BT ? B.at(k0 + li + 8 * l3, n0 + 16 * p + 8 * l4) : B.at(n0 + 16 * p + li + 8 * l4, k0 + 8 * l3);
+    const int nk = (k1 - k0) >> 4;
+#pragma unroll 2
+    for (int i = 0; i < nk; ++i) {
         uint32_t a[4];
-        if (!AT) ldsm4(A.at(m0 + li + 8 * l3, k + 8 * l4), a);
-        else ldsm4t(A.at(k + li + 8 * l4, m0 + 8 * l3), a);
+        if (!AT) ldsm4(a0 + i * da, a);
+        else ldsm4t(a0 + i * da, a);
 #pragma unroll
         for (int p = 0; p < NT / 2; ++p) {
-            const int n = n0 + 16 * p;
             uint32_t b[4];
-            if (!BT) ldsm4(B.at(n + li + 8 * l4, k + 8 * l3), b);
-            else ldsm4t(B.at(k + li + 8 * l3, n + 8 * l4), b);
+            const uint32_t ba = b_lin ? b0[p] + i * db : B.at(n0 + 16 * p + li + 8 * l4, k0 + 16 * i + 8 * l3);
+            if (!BT) ldsm4(ba, b);
+            else ldsm4t(ba, b);
             mma16816(acc[2 * p], a, b[0], b[1]);
             mma16816(acc[2 * p + 1], a, b[2], b[3]);
         }
