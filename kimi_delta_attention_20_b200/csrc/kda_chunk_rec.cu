@@ -567,6 +567,12 @@ size_t chunk_rec_workspace_bytes(const ChunkParams &p, bool bf16, int Dk, int Dv
     return P < 2 ? 0 : rec_seg_layout(p, P, Dk).total;
 }
 
+bool chunk_warp_supported(bool bf16, int Dk, int Dv);
+cudaError_t launch_chunk_warp(const ChunkParams &p, int Dv, cudaStream_t st);
+
+// Few chains of long sequences: the segment form of the recurrence; otherwise, for bf16
+// with d_k = 32, the tensor-core micro-chunk form (one warp per chain, kda_chunk_warp.cu);
+// otherwise the recurrence.
 cudaError_t launch_chunk_rec(const ChunkParams &p, bool bf16, int Dk, int Dv, void *workspace, size_t workspace_bytes,
                              cudaStream_t st) {
     const int P = rec_seg_count(p, Dk, Dv);
@@ -575,6 +581,7 @@ cudaError_t launch_chunk_rec(const ChunkParams &p, bool bf16, int Dk, int Dv, vo
         uint8_t *ws = static_cast<uint8_t *>(workspace);
         return bf16 ? launch_rec_seg_dt<__nv_bfloat16>(p, P, Dk, ws, st) : launch_rec_seg_dt<float>(p, P, Dk, ws, st);
     }
+    if (P < 2 && chunk_warp_supported(bf16, Dk, Dv)) return launch_chunk_warp(p, Dv, st);
     return bf16 ? launch_rec_dt<__nv_bfloat16>(p, Dk, Dv, st) : launch_rec_dt<float>(p, Dk, Dv, st);
 }
 

@@ -1,0 +1,464 @@
+// Chunk forward for bf16 inputs with d_k = 32 (d_v = 32 or 64) when there are many
+// (sequence, head) chains: one warp per chain, the WY/UT chunk form on 16-token
+// micro-chunks, every product a warp-level tensor-core MMA (m16n8k16, bf16 operands,
+// fp32 accumulate) and the fp32 state in the warp's accumulator registers.
+//
+// The operator is the `chunk_kda` boundary of page "K3/kda/ops/api.py" (the token
+// recurrence of page "atlas_core/kimi_k3/kda.rs"). The chunk form is exact for any
+// chunk size -- grouping tokens changes the order of the arithmetic, not its value --
+// and with 16 tokens the UT inverse is a 16 x 16 unit-triangular solve inside one
+// warp, every product is one MMA tile high, and a 32 x d_v state fits in 64 registers
+// per lane, so a chain needs no block barrier and no record. Per micro-chunk (G the
+// in-chunk cumsum of the gate, k^, q^ the normalised rows, b the write strengths):
+//   A_kk[r,s] = sum_c k^_rc k^_sc e^{G_rc - G_sc} (s < r),  A_qk likewise with q^ (s <= r)
+//   T' = (I + diag(b) A_kk)^-1 diag(b),  U = T' V,  W = T' (k^ e^G)
+//   D = U - W S,  O = scale ((q^ e^G) S + A_qk D),  S <- diag(e^{G_last}) S + (k^ e^{G_last - G})^T D.
+// The gated products split e^{G_r - G_s} at the micro-chunk's middle row (both parts
+// <= e^80 while the gate moves by at most 80 over half a micro-chunk); a micro-chunk
+// whose gate moves further takes A_kk and A_qk from exponent differences on the CUDA
+// cores. Lane = key channel for the gate, its cumsum and the operand tiles.
+#include <algorithm>
+
+#include "kda_common.cuh"
+#include "kda_stage.cuh"
+#include "kda_tc_util.cuh"
+#include "kda_sm100.cuh"
+
+namespace kda {
+namespace cw {
+
+using namespace tcu;
+
+constexpr int CW = 16;      // tokens per micro-chunk
+constexpr int DK = 32;      // key dim (lane = key channel)
+constexpr int LK = DK + 8;  // padded row of a [16][32] bf16 tile (elements): 80 B, conflict-free fragments
+constexpr int LT = 24;      // padded row of a [16][16] bf16 tile: 48 B
+constexpr int LL = 17;      // row of the fp32 L tile
+constexpr int NWARP = 4;    // chains per CTA
+constexpr float kL2e = 1.4426950408889634f;
+constexpr float kSpan = 80.f;  // largest |G - G_mid| of the split products
+
+template <int DV>
+struct Lay {
+    static constexpr int LV = DV + 8;                      // padded row of [*][DV] bf16 tiles
+    static constexpr uint32_t Q = 0, K = Q + CW * LK * 2, G = K + CW * LK * 2, V = G + CW * LK * 2;
+    static constexpr uint32_t B = V + CW * LV * 2;          // raw beta [16] (f32)
+    static constexpr uint32_t X = B + 64;                    // k^ e^{G-M}; later -W
+    static constexpr uint32_t Y = X + CW * LK * 2;           // k^ e^{M-G}
+    static constexpr uint32_t XQ = Y + CW * LK * 2;          // q^ e^{G-M}
+    static constexpr uint32_t D = Y;                         // D (bf16 [16][LV]) over Y and XQ
+    static constexpr uint32_t KT = XQ + CW * LK * 2;         // k^ e^G
+    static constexpr uint32_t QT = KT + CW * LK * 2;         // q^ e^G
+    static constexpr uint32_t KH = QT + CW * LK * 2;         // k^ e^{G_last - G}
+    static constexpr uint32_t TP = KH + CW * LK * 2;         // T' [16][LT]
+    static constexpr uint32_t AQ = TP + CW * LT * 2;         // A_qk [16][LT]
+    static constexpr uint32_t S = AQ + CW * LT * 2;          // S (bf16 [32][LV]); exponent scratch G [16][33] f32
+    static constexpr uint32_t L = S + DK * LV * 2;           // L = diag(b) A_kk, f32 [16][LL]
+    static constexpr uint32_t RK = L + CW * LL * 4, RQ = RK + 64, BB = RQ + 64, GAM = BB + 64;
+    static constexpr uint32_t BYTES = (GAM + DK * 4 + 127) / 128 * 128;
+    static_assert(D + CW * LV * 2 <= KT && CW * 33 * 4 <= DK * LV * 2, "aliases");
+};
+
+// ---- warp-level MMA
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+// Fragment loads of a row-major bf16 tile with rows of `ld` elements at shared address
+// `base`. A (16 x 16 at (m0, k0)) from [M][K] storage, or from [K][M] storage (trans).
+__device__ __forceinline__ void frag_a(uint32_t base, int ld, int m0, int k0, int lane, uint32_t (&a)[4]) {
+    ldsm4(base + 2 * ((m0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ld + k0 + 8 * (lane >> 4)), a);
+}
+__device__ __forceinline__ void frag_at(uint32_t base, int ld, int m0, int k0, int lane, uint32_t (&a)[4]) {
+    ldsm4t(base + 2 * ((k0 + (lane & 7) + 8 * (lane >> 4)) * ld + m0 + 8 * ((lane >> 3) & 1)), a);
+}
+// B for two n-tiles (n0 .. n0 + 15) x k0 .. k0 + 15: from [N][K] storage, or [K][N] (trans).
+// b[0], b[1]: n-tile n0; b[2], b[3]: n-tile n0 + 8.
+__device__ __forceinline__ void frag_b(uint32_t base, int ld, int n0, int k0, int lane, uint32_t (&b)[4]) {
+    ldsm4(base + 2 * ((n0 + (lane & 7) + 8 * (lane >> 4)) * ld + k0 + 8 * ((lane >> 3) & 1)), b);
+}
+__device__ __forceinline__ void frag_bt(uint32_t base, int ld, int n0, int k0, int lane, uint32_t (&b)[4]) {
+    ldsm4t(base + 2 * ((k0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ld + n0 + 8 * (lane >> 4)), b);
+}
+// 16-byte cp.async that zero-fills the destination when `valid` is false (no bytes read;
+// the source address is still a valid one)
+__device__ __forceinline__ void cp16z(void *sdst, const void *gsrc, bool valid) {
+    const uint32_t d = sm100::smem_u32(sdst);
+    const int n = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gsrc), "r"(n) : "memory");
+}
+__device__ __forceinline__ void stb2(uint8_t *p, float a, float b) {
+    *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(a, b);
+}
+__device__ __forceinline__ float e2(float x) { return ex2a(x * kL2e); }
+
+template <int DV>
+__global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const ChunkParams p) {
+    using Ly = Lay<DV>;
+    constexpr int LV = Ly::LV, NVT = DV / 8;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const long long chain = (long long)blockIdx.x * NWARP + warp;
+    if (chain >= (long long)p.N * p.H) return;  // no block barriers below: the warps are independent
+    const int n = (int)(chain / p.H), h = (int)(chain % p.H);
+    uint8_t *sm = smem_raw + warp * Ly::BYTES;
+    const uint32_t sb = sm100::smem_u32(sm);
+    float *rk = reinterpret_cast<float *>(sm + Ly::RK), *rq = reinterpret_cast<float *>(sm + Ly::RQ);
+    float *bb = reinterpret_cast<float *>(sm + Ly::BB), *gam = reinterpret_cast<float *>(sm + Ly::GAM);
+    float *Lf = reinterpret_cast<float *>(sm + Ly::L);
+    const int H = p.H, g8 = lane >> 2, t4 = lane & 3;
+    long long bos, eos;
+    if (p.cu_seqlens) { bos = p.cu_seqlens[n]; eos = p.cu_seqlens[n + 1]; }
+    else { bos = (long long)n * p.T; eos = bos + p.T; }
+    const int nmc = (int)((eos - bos + CW - 1) / CW);
+    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q), *kg = static_cast<const __nv_bfloat16 *>(p.k);
+    const __nv_bfloat16 *gg = static_cast<const __nv_bfloat16 *>(p.g), *vg = static_cast<const __nv_bfloat16 *>(p.v);
+    const __nv_bfloat16 *betag = static_cast<const __nv_bfloat16 *>(p.beta);
+    __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(p.o);
+    // in-kernel gate: rate and this lane's channel bias
+    const float rate = p.gate_mode != kGateLog ? expf(p.A_log[h]) : 0.f;
+    const float bias = (p.gate_mode != kGateLog && p.dt_bias) ? p.dt_bias[(long long)h * DK + lane] : 0.f;
+
+    // raw rows of micro-chunk mc (rows past the sequence zero-filled): q, k, g, v by
+    // cp.async; lane r < 16 also loads token r's beta into braw (stored to shared memory
+    // after the copies are waited for, so the load does not stall the warp here)
+    float braw = 0.f;
+    // lane (row r = lane / 2, half hf = lane % 2): pieces hf*2, hf*2+1 of its q, k, g rows
+    // and hf*DV/16 .. of its v row (16-byte pieces)
+    auto issue = [&](int mc) {
+        const long long t0 = bos + (long long)mc * CW;
+        const int L = (int)min((long long)CW, eos - t0);
+        const int r = lane >> 1, hf = lane & 1;
+        const bool ok = r < L;
+        const long long row = (t0 + (ok ? r : 0)) * H + h;
+        const __nv_bfloat16 *qs = qg + row * DK + 16 * hf, *ks = kg + row * DK + 16 * hf, *gs = gg + row * DK + 16 * hf;
+        const __nv_bfloat16 *vs = vg + row * DV + (DV / 2) * hf;
+        const uint32_t o = (r * LK + 16 * hf) * 2, ov = (r * LV + (DV / 2) * hf) * 2;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            cp16z(sm + Ly::Q + o + 16 * c, qs + 8 * c, ok);
+            cp16z(sm + Ly::K + o + 16 * c, ks + 8 * c, ok);
+            cp16z(sm + Ly::G + o + 16 * c, gs + 8 * c, ok);
+        }
+#pragma unroll
+        for (int c = 0; c < DV / 16; ++c) cp16z(sm + Ly::V + ov + 16 * c, vs + 8 * c, ok);
+        braw = lane < L ? __bfloat162float(betag[(t0 + lane) * H + h]) : 0.f;
+        cp_async_commit();
+    };
+
+    // the state: rows c = 16 mk + g8 (+ 8), columns 8 j + 2 t4 (+ 1), in MMA accumulator layout
+    float S[2][NVT][4];
+    const long long sbase = ((long long)n * H + h) * DK * DV;
+#pragma unroll
+    for (int mk = 0; mk < 2; ++mk)
+#pragma unroll
+        for (int j = 0; j < NVT; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int c = 16 * mk + g8 + 8 * (i >> 1), v = 8 * j + 2 * t4 + (i & 1);
+                S[mk][j][i] = p.S0 ? p.S0[sbase + (long long)c * DV + v] : 0.f;
+            }
+
+    if (nmc > 0) issue(0);
+    for (int mc = 0; mc < nmc; ++mc) {
+        const long long t0 = bos + (long long)mc * CW;
+        const int L = (int)min((long long)CW, eos - t0);
+        if (lane < CW) reinterpret_cast<float *>(sm + Ly::B)[lane] = braw;
+        cp_async_wait_all();
+        __syncwarp();
+        // ---- gate and its in-chunk cumsum: lane = channel, G[r] for the 16 rows (the 16
+        // gate values first, independently, then the running sum)
+        float G[CW];
+        {
+#pragma unroll
+            for (int r = 0; r < CW; ++r) {
+                const float x = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(sm + Ly::G)[r * LK + lane]);
+                const float gv = p.gate_mode == kGateLog ? (p.has_lb ? fmaxf(x, p.lb) : x)
+                                                         : gate_fast(x, bias, rate, p.gate_mode, p.lb);
+                G[r] = r < L ? gv : 0.f;
+            }
+#pragma unroll
+            for (int r = 1; r < CW; ++r) G[r] += G[r - 1];
+        }
+        // ---- row norms (lanes 0..15: k rows, 16..31: q rows) and write strengths
+        {
+            const int r = lane & 15;
+            const uint32_t row = (lane < 16 ? Ly::K : Ly::Q) + r * LK * 2;
+            float s = 0.f;
+#pragma unroll
+            for (int c8 = 0; c8 < DK / 8; ++c8) {
+                float f[8];
+                unpack8(lds128(sm, row + 16 * c8), f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) s = fmaf(f[e], f[e], s);
+            }
+            const float inv = r < L ? (p.use_l2 ? rsqrtf(s + 1e-6f) : 1.f) : 0.f;
+            if (lane < 16) {
+                rk[r] = inv;
+                const float bx = reinterpret_cast<const float *>(sm + Ly::B)[r];
+                bb[r] = r < L ? beta_value(bx, p.beta_prob) : 0.f;
+            } else {
+                rq[r] = inv;
+            }
+        }
+        __syncwarp();
+        // ---- operand tiles, column `lane` of each: X = k^ e^{G-M}, Y = k^ e^{M-G},
+        // XQ = q^ e^{G-M}, KT = k^ e^G, QT = q^ e^G, KH = k^ e^{G_last-G}
+        const float Gm = G[7], GC = G[CW - 1];
+        bool steep = false;
+        {
+            const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(sm + Ly::K);
+            const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(sm + Ly::Q);
+#pragma unroll
+            for (int r = 0; r < CW; ++r) {
+                const float kh = __bfloat162float(kr[r * LK + lane]) * rk[r];
+                const float qh = __bfloat162float(qr[r * LK + lane]) * rq[r];
+                const float dm = G[r] - Gm;
+                steep |= fabsf(dm) > kSpan;
+                const float em = e2(dm), en = e2(-dm), eg = e2(G[r]), ec = e2(GC - G[r]);
+                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::X)[r * LK + lane] = __float2bfloat16_rn(kh * em);
+                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::Y)[r * LK + lane] = __float2bfloat16_rn(kh * en);
+                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::XQ)[r * LK + lane] = __float2bfloat16_rn(qh * em);
+                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::KT)[r * LK + lane] = __float2bfloat16_rn(kh * eg);
+                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::QT)[r * LK + lane] = __float2bfloat16_rn(qh * eg);
+                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::KH)[r * LK + lane] = __float2bfloat16_rn(kh * ec);
+            }
+            gam[lane] = e2(GC);
+        }
+        steep = __any_sync(0xffffffffu, steep);
+        __syncwarp();
+        // ---- A_kk (s < r) -> L = diag(b) A_kk (fp32), A_qk (s <= r) -> bf16 tile
+        {
+            float akk[2][4] = {}, aqk[2][4] = {};
+#pragma unroll
+            for (int k0 = 0; k0 < DK; k0 += 16) {
+                uint32_t a[4], aq[4], b[4];
+                frag_a(sb + Ly::X, LK, 0, k0, lane, a);
+                frag_a(sb + Ly::XQ, LK, 0, k0, lane, aq);
+                frag_b(sb + Ly::Y, LK, 0, k0, lane, b);
+                mma16816(akk[0], a, b[0], b[1]);
+                mma16816(akk[1], a, b[2], b[3]);
+                mma16816(aqk[0], aq, b[0], b[1]);
+                mma16816(aqk[1], aq, b[2], b[3]);
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi) {
+                    const int r = g8 + 8 * hi, s = 8 * j + 2 * t4;
+                    const float br = bb[r];
+                    Lf[r * LL + s] = s < r ? br * akk[j][2 * hi] : 0.f;
+                    Lf[r * LL + s + 1] = s + 1 < r ? br * akk[j][2 * hi + 1] : 0.f;
+                    stb2(sm + Ly::AQ + (r * LT + s) * 2, s <= r ? aqk[j][2 * hi] : 0.f,
+                         s + 1 <= r ? aqk[j][2 * hi + 1] : 0.f);
+                }
+        }
+        if (steep) {  // exponent differences (never positive) on the CUDA cores
+            float *Gs = reinterpret_cast<float *>(sm + Ly::S);
+#pragma unroll
+            for (int r = 0; r < CW; ++r) Gs[r * 33 + lane] = G[r];
+            __syncwarp();
+            const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(sm + Ly::K);
+            const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(sm + Ly::Q);
+            for (int e = lane; e < CW * CW; e += 32) {
+                const int r = e >> 4, s = e & 15;
+                if (s > r) continue;
+                float akk = 0.f, aqk = 0.f;
+                for (int c = 0; c < DK; ++c) {
+                    const float ed = expf(Gs[r * 33 + c] - Gs[s * 33 + c]);
+                    const float ks = __bfloat162float(kr[s * LK + c]) * ed;
+                    akk = fmaf(__bfloat162float(kr[r * LK + c]), ks, akk);
+                    aqk = fmaf(__bfloat162float(qr[r * LK + c]), ks, aqk);
+                }
+                akk *= rk[r] * rk[s];
+                aqk *= rq[r] * rk[s];
+                if (s < r) Lf[r * LL + s] = bb[r] * akk;
+                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::AQ)[r * LT + s] = __float2bfloat16_rn(aqk);
+            }
+        }
+        __syncwarp();
+        // ---- T = (I + L)^-1 by forward substitution (lane j < 16: column j), T' = T diag(b)
+        if (lane < CW) {
+            const int j = lane;
+            float t[CW];
+#pragma unroll
+            for (int i = 0; i < CW; ++i) {
+                float acc = i == j ? 1.f : 0.f;
+#pragma unroll
+                for (int k = 0; k < i; ++k) acc = fmaf(-Lf[i * LL + k], t[k], acc);
+                t[i] = acc;
+            }
+            const float bj = bb[j];
+#pragma unroll
+            for (int i = 0; i < CW; ++i)
+                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::TP)[i * LT + j] = __float2bfloat16_rn(t[i] * bj);
+        }
+        __syncwarp();
+        // ---- U = T' V (registers), -W = -T' Ktil (bf16 tile over X)
+        float U[NVT][4];
+        {
+            uint32_t a[4];
+            frag_a(sb + Ly::TP, LT, 0, 0, lane, a);
+#pragma unroll
+            for (int j = 0; j < NVT; j += 2) {
+                uint32_t b[4];
+                frag_bt(sb + Ly::V, LV, 8 * j, 0, lane, b);
+                U[j][0] = U[j][1] = U[j][2] = U[j][3] = 0.f;
+                U[j + 1][0] = U[j + 1][1] = U[j + 1][2] = U[j + 1][3] = 0.f;
+                mma16816(U[j], a, b[0], b[1]);
+                mma16816(U[j + 1], a, b[2], b[3]);
+            }
+            float w[4][4] = {};
+#pragma unroll
+            for (int j = 0; j < 4; j += 2) {
+                uint32_t b[4];
+                frag_bt(sb + Ly::KT, LK, 8 * j, 0, lane, b);
+                mma16816(w[j], a, b[0], b[1]);
+                mma16816(w[j + 1], a, b[2], b[3]);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi)
+                    stb2(sm + Ly::X + ((g8 + 8 * hi) * LK + 8 * j + 2 * t4) * 2, -w[j][2 * hi], -w[j][2 * hi + 1]);
+        }
+        // the state as a bf16 operand
+#pragma unroll
+        for (int mk = 0; mk < 2; ++mk)
+#pragma unroll
+            for (int j = 0; j < NVT; ++j)
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi)
+                    stb2(sm + Ly::S + ((16 * mk + g8 + 8 * hi) * LV + 8 * j + 2 * t4) * 2, S[mk][j][2 * hi],
+                         S[mk][j][2 * hi + 1]);
+        __syncwarp();  // the raw rows are consumed: the next micro-chunk's copies start
+        if (mc + 1 < nmc) issue(mc + 1);
+        // ---- D = U - W S (in U's registers) -> bf16 tile
+#pragma unroll
+        for (int k0 = 0; k0 < DK; k0 += 16) {
+            uint32_t a[4];
+            frag_a(sb + Ly::X, LK, 0, k0, lane, a);
+#pragma unroll
+            for (int j = 0; j < NVT; j += 2) {
+                uint32_t b[4];
+                frag_bt(sb + Ly::S, LV, 8 * j, k0, lane, b);
+                mma16816(U[j], a, b[0], b[1]);
+                mma16816(U[j + 1], a, b[2], b[3]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < NVT; ++j)
+#pragma unroll
+            for (int hi = 0; hi < 2; ++hi)
+                stb2(sm + Ly::D + ((g8 + 8 * hi) * LV + 8 * j + 2 * t4) * 2, U[j][2 * hi], U[j][2 * hi + 1]);
+        __syncwarp();
+        // ---- O = scale ((q^ e^G) S + A_qk D), rows < L to o
+        {
+            float O[NVT][4];
+#pragma unroll
+            for (int j = 0; j < NVT; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
+#pragma unroll
+            for (int k0 = 0; k0 < DK; k0 += 16) {
+                uint32_t a[4];
+                frag_a(sb + Ly::QT, LK, 0, k0, lane, a);
+#pragma unroll
+                for (int j = 0; j < NVT; j += 2) {
+                    uint32_t b[4];
+                    frag_bt(sb + Ly::S, LV, 8 * j, k0, lane, b);
+                    mma16816(O[j], a, b[0], b[1]);
+                    mma16816(O[j + 1], a, b[2], b[3]);
+                }
+            }
+            {
+                uint32_t a[4];
+                frag_a(sb + Ly::AQ, LT, 0, 0, lane, a);
+#pragma unroll
+                for (int j = 0; j < NVT; j += 2) {
+                    uint32_t b[4];
+                    frag_bt(sb + Ly::D, LV, 8 * j, 0, lane, b);
+                    mma16816(O[j], a, b[0], b[1]);
+                    mma16816(O[j + 1], a, b[2], b[3]);
+                }
+            }
+            if (og) {
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi) {
+                    const int r = g8 + 8 * hi;
+                    if (r < L) {
+                        const float f = p.scale;  // Qtil and A_qk are built from q^
+                        __nv_bfloat16 *orow = og + ((t0 + r) * H + h) * DV + 2 * t4;
+#pragma unroll
+                        for (int j = 0; j < NVT; ++j)
+                            *reinterpret_cast<__nv_bfloat162 *>(orow + 8 * j) =
+                                __floats2bfloat162_rn(f * O[j][2 * hi], f * O[j][2 * hi + 1]);
+                    }
+                }
+            }
+        }
+        // ---- S <- diag(e^{G_last}) S + Khat^T D
+#pragma unroll
+        for (int mk = 0; mk < 2; ++mk) {
+            const float ga = gam[16 * mk + g8], gb = gam[16 * mk + g8 + 8];
+#pragma unroll
+            for (int j = 0; j < NVT; ++j) {
+                S[mk][j][0] *= ga; S[mk][j][1] *= ga;
+                S[mk][j][2] *= gb; S[mk][j][3] *= gb;
+            }
+            uint32_t a[4];
+            frag_at(sb + Ly::KH, LK, 16 * mk, 0, lane, a);
+#pragma unroll
+            for (int j = 0; j < NVT; j += 2) {
+                uint32_t b[4];
+                frag_bt(sb + Ly::D, LV, 8 * j, 0, lane, b);
+                mma16816(S[mk][j], a, b[0], b[1]);
+                mma16816(S[mk][j + 1], a, b[2], b[3]);
+            }
+        }
+        __syncwarp();  // every tile of this micro-chunk is read
+    }
+    cp_async_wait_all();
+    if (p.S_out) {
+#pragma unroll
+        for (int mk = 0; mk < 2; ++mk)
+#pragma unroll
+            for (int j = 0; j < NVT; ++j)
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi) {
+                    const int c = 16 * mk + g8 + 8 * hi, v = 8 * j + 2 * t4;
+                    *reinterpret_cast<float2 *>(p.S_out + sbase + (long long)c * DV + v) =
+                        make_float2(S[mk][j][2 * hi], S[mk][j][2 * hi + 1]);
+                }
+    }
+}
+
+template <int DV>
+cudaError_t launch_t(const ChunkParams &p, cudaStream_t st) {
+    const long long chains = (long long)p.N * p.H;
+    if (chains <= 0) return cudaSuccess;
+    const uint32_t smem = NWARP * Lay<DV>::BYTES;
+    cudaError_t e = cudaFuncSetAttribute(kda_chunk_warp_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    count_launch();
+    kda_chunk_warp_kernel<DV><<<(unsigned)((chains + NWARP - 1) / NWARP), NWARP * 32, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace cw
+
+bool chunk_warp_supported(bool bf16, int Dk, int Dv) { return bf16 && Dk == 32 && (Dv == 32 || Dv == 64); }
+
+cudaError_t launch_chunk_warp(const ChunkParams &p, int Dv, cudaStream_t st) {
+    return Dv == 32 ? cw::launch_t<32>(p, st) : cw::launch_t<64>(p, st);
+}
+
+}  // namespace kda

@@ -1,0 +1,95 @@
+"""GPU parity of the micro-chunk tensor-core forward (bf16, d_k = 32, d_v 32 or 64: one
+warp per (sequence, head), 16-token micro-chunks) against form R, the token recurrence
+of page "atlas_core/kimi_k3/kda.rs" (`chunk_kda` of page "K3/kda/ops/api.py"). This
+form takes bf16 d_k = 32 calls that the segment form of the recurrence does not:
+many chains, short sequences, or d_k != d_v."""
+import pytest
+import torch
+
+import kda_inputs as KI
+from kda_check import check, oracle_chunk
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+DT = torch.bfloat16
+
+
+def kda_mod():
+    import kimi_delta_attention_20_b200 as kda
+    return kda
+
+
+def run(inp, **kw):
+    kda = kda_mod()
+    d = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    return kda.chunk_kda(d["q"], d["k"], d["v"], d["g"], d["beta"], initial_state=d.get("initial_state"),
+                         output_final_state=True, cu_seqlens=d.get("cu_seqlens"), **kw)
+
+
+def compare(inp, o, S, tag, **okw):
+    ref = oracle_chunk({k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}, **okw)
+    H = inp["q"].shape[2]
+    B, T = inp["q"].shape[:2]
+    o_flat = o.reshape(B * T, H, -1)
+    for n, (a, b, o_ref, S_ref) in enumerate(ref):
+        for h in range(H):
+            if b > a:
+                check(f"{tag} o seq{n} h{h}", o_flat[a:b][:, [h]], o_ref[:, [h]], DT)
+            check(f"{tag} S seq{n} h{h}", S[n, [h]], S_ref[[h]], DT)
+
+
+@pytest.mark.parametrize("dv", [32, 64])
+def test_warp_ragged_varlen(dv):
+    """Micro-chunk tails of every kind and empty sequences in a varlen batch."""
+    lens = [0, 1, 15, 16, 17, 33, 100, 0, 257, 64]
+    inp = KI.draw_chunk(1, sum(lens), 3, 32, dv, dtype=DT, seed=500 + dv, seqlens=lens, init_state=True)
+    o, S = run(inp, use_qk_l2norm_in_kernel=True)
+    compare(inp, o, S, f"ragged d_v{dv}")
+
+
+@pytest.mark.parametrize("dv", [32, 64])
+def test_warp_steep_gates(dv):
+    """Gates that drop by up to ~100 per token: the middle-row split would leave the fp32
+    range, so those micro-chunks take the exponent-difference products; others keep the
+    tensor-core split."""
+    inp = KI.draw_chunk(2, 120, 2, 32, dv, dtype=DT, seed=510 + dv, init_state=True)
+    g = inp["g"].float()
+    g[:, 20:50] = g[:, 20:50] * 40.0
+    inp["g"] = g.to(DT)
+    o, S = run(inp, use_qk_l2norm_in_kernel=True)
+    compare(inp, o, S, f"steep d_v{dv}")
+
+
+@pytest.mark.parametrize("form", ["softplus", "safe"])
+def test_warp_in_kernel_gate(form):
+    """The in-kernel gate forms (page "atlas_core/kimi_k3/kda.rs" `bounded_gate`)."""
+    inp = KI.draw_chunk(2, 150, 4, 32, 64, dtype=DT, seed=520 + len(form), init_state=True, gate="input")
+    gen = torch.Generator().manual_seed(521)
+    A_log = torch.empty(4).uniform_(-2.0, 0.5, generator=gen)
+    dt_bias = torch.randn(4, 32, generator=gen) * 0.5
+    kw = dict(use_gate_in_kernel=True, A_log=A_log.to(DEV), dt_bias=dt_bias.to(DEV), use_qk_l2norm_in_kernel=True)
+    okw = dict(gate_form=form, A_log=A_log, dt_bias=dt_bias)
+    if form == "safe":
+        kw.update(safe_gate=True, lower_bound=-5.0)
+        okw["lower_bound"] = -5.0
+    o, S = run(inp, **kw)
+    compare(inp, o, S, f"gate {form}", **okw)
+
+
+def test_warp_options():
+    """beta as a probability, no in-kernel L2 norm, an explicit scale, no initial state."""
+    inp = KI.draw_chunk(2, 90, 2, 32, 32, dtype=DT, seed=530, beta="prob")
+    inp["k"] = (inp["k"].float() / 6.0).to(DT)
+    with pytest.warns(RuntimeWarning):
+        o, S = run(inp, use_qk_l2norm_in_kernel=False, use_beta_sigmoid_in_kernel=False, scale=0.37)
+    compare(inp, o, S, "options", l2=False, beta_is_logit=False, scale=0.37)
+
+
+def test_warp_many_chains():
+    """1,024 chains (one wave of warps), a sample of sequences checked on every head."""
+    inp = KI.draw_chunk(64, 96, 16, 32, 64, dtype=DT, seed=540, init_state=True)
+    o, S = run(inp, use_qk_l2norm_in_kernel=True, lower_bound=-5.0)
+    sub = {n: inp[n][[0, 31, 63]] for n in ("q", "k", "v", "g", "beta")}
+    sub["initial_state"] = inp["initial_state"][[0, 31, 63]]
+    compare(sub, o[[0, 31, 63]], S[[0, 31, 63]], "many", lower_bound=-5.0)
