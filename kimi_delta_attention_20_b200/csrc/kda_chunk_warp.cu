@@ -43,20 +43,24 @@ struct Lay {
     static constexpr int LV = DV + 8;                      // padded row of [*][DV] bf16 tiles
     static constexpr uint32_t Q = 0, K = Q + CW * LK * 2, G = K + CW * LK * 2, V = G + CW * LK * 2;
     static constexpr uint32_t B = V + CW * LV * 2;          // raw beta [16] (f32)
-    static constexpr uint32_t X = B + 64;                    // k^ e^{G-M}; later -W
-    static constexpr uint32_t Y = X + CW * LK * 2;           // k^ e^{M-G}
-    static constexpr uint32_t XQ = Y + CW * LK * 2;          // q^ e^{G-M}
+    // the operand tiles, stored transposed ([32 channels][16 rows], rows of LT): X^T of
+    // k^ e^{G-M} (later the -W tile, [16][LK]), Y^T of k^ e^{M-G}, XQ^T of q^ e^{G-M},
+    // KT^T of k^ e^G, QT^T of q^ e^G, KH^T of k^ e^{G_last-G}
+    static constexpr uint32_t TT = DK * LT * 2;
+    static constexpr uint32_t X = B + 64;
+    static constexpr uint32_t Y = X + TT;
+    static constexpr uint32_t XQ = Y + TT;
     static constexpr uint32_t D = Y;                         // D (bf16 [16][LV]) over Y and XQ
-    static constexpr uint32_t KT = XQ + CW * LK * 2;         // k^ e^G
-    static constexpr uint32_t QT = KT + CW * LK * 2;         // q^ e^G
-    static constexpr uint32_t KH = QT + CW * LK * 2;         // k^ e^{G_last - G}
-    static constexpr uint32_t TP = KH + CW * LK * 2;         // T' [16][LT]
+    static constexpr uint32_t KT = XQ + TT;
+    static constexpr uint32_t QT = KT + TT;
+    static constexpr uint32_t KH = QT + TT;
+    static constexpr uint32_t TP = KH + TT;                  // T' [16][LT]
     static constexpr uint32_t AQ = TP + CW * LT * 2;         // A_qk [16][LT]
     static constexpr uint32_t S = AQ + CW * LT * 2;          // S (bf16 [32][LV]); exponent scratch G [16][33] f32
     static constexpr uint32_t L = S + DK * LV * 2;           // L = diag(b) A_kk, f32 [16][LL]
     static constexpr uint32_t RK = L + CW * LL * 4, RQ = RK + 64, BB = RQ + 64, GAM = BB + 64;
     static constexpr uint32_t BYTES = (GAM + DK * 4 + 127) / 128 * 128;
-    static_assert(D + CW * LV * 2 <= KT && CW * 33 * 4 <= DK * LV * 2, "aliases");
+    static_assert(D + CW * LV * 2 <= KT && CW * LK * 2 <= TT && CW * 33 * 4 <= DK * LV * 2, "aliases");
 };
 
 // ---- warp-level MMA
@@ -212,26 +216,35 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
             }
         }
         __syncwarp();
-        // ---- operand tiles, column `lane` of each: X = k^ e^{G-M}, Y = k^ e^{M-G},
-        // XQ = q^ e^{G-M}, KT = k^ e^G, QT = q^ e^G, KH = k^ e^{G_last-G}
+        // ---- operand tiles, row `lane` of each transposed tile (16 values = two 16-byte
+        // stores): X = k^ e^{G-M}, Y = k^ e^{M-G}, XQ = q^ e^{G-M}, KT = k^ e^G,
+        // QT = q^ e^G, KH = k^ e^{G_last-G}
         const float Gm = G[7], GC = G[CW - 1];
         bool steep = false;
         {
             const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(sm + Ly::K);
             const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(sm + Ly::Q);
 #pragma unroll
-            for (int r = 0; r < CW; ++r) {
-                const float kh = __bfloat162float(kr[r * LK + lane]) * rk[r];
-                const float qh = __bfloat162float(qr[r * LK + lane]) * rq[r];
-                const float dm = G[r] - Gm;
-                steep |= fabsf(dm) > kSpan;
-                const float em = e2(dm), en = e2(-dm), eg = e2(G[r]), ec = e2(GC - G[r]);
-                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::X)[r * LK + lane] = __float2bfloat16_rn(kh * em);
-                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::Y)[r * LK + lane] = __float2bfloat16_rn(kh * en);
-                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::XQ)[r * LK + lane] = __float2bfloat16_rn(qh * em);
-                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::KT)[r * LK + lane] = __float2bfloat16_rn(kh * eg);
-                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::QT)[r * LK + lane] = __float2bfloat16_rn(qh * eg);
-                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::KH)[r * LK + lane] = __float2bfloat16_rn(kh * ec);
+            for (int h8 = 0; h8 < 2; ++h8) {
+                float x[8], y[8], xq[8], kt[8], qt[8], kc[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int r = 8 * h8 + u;
+                    const float kh = __bfloat162float(kr[r * LK + lane]) * rk[r];
+                    const float qh = __bfloat162float(qr[r * LK + lane]) * rq[r];
+                    const float dm = G[r] - Gm;
+                    steep |= fabsf(dm) > kSpan;
+                    const float em = e2(dm), en = e2(-dm), eg = e2(G[r]), ec = e2(GC - G[r]);
+                    x[u] = kh * em; y[u] = kh * en; xq[u] = qh * em;
+                    kt[u] = kh * eg; qt[u] = qh * eg; kc[u] = kh * ec;
+                }
+                const uint32_t o = (lane * LT + 8 * h8) * 2;
+                sts128(sm, Ly::X + o, pack8(x));
+                sts128(sm, Ly::Y + o, pack8(y));
+                sts128(sm, Ly::XQ + o, pack8(xq));
+                sts128(sm, Ly::KT + o, pack8(kt));
+                sts128(sm, Ly::QT + o, pack8(qt));
+                sts128(sm, Ly::KH + o, pack8(kc));
             }
             gam[lane] = e2(GC);
         }
@@ -243,9 +256,9 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
 #pragma unroll
             for (int k0 = 0; k0 < DK; k0 += 16) {
                 uint32_t a[4], aq[4], b[4];
-                frag_a(sb + Ly::X, LK, 0, k0, lane, a);
-                frag_a(sb + Ly::XQ, LK, 0, k0, lane, aq);
-                frag_b(sb + Ly::Y, LK, 0, k0, lane, b);
+                frag_at(sb + Ly::X, LT, 0, k0, lane, a);
+                frag_at(sb + Ly::XQ, LT, 0, k0, lane, aq);
+                frag_bt(sb + Ly::Y, LT, 0, k0, lane, b);
                 mma16816(akk[0], a, b[0], b[1]);
                 mma16816(akk[1], a, b[2], b[3]);
                 mma16816(aqk[0], aq, b[0], b[1]);
@@ -322,7 +335,7 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
 #pragma unroll
             for (int j = 0; j < 4; j += 2) {
                 uint32_t b[4];
-                frag_bt(sb + Ly::KT, LK, 8 * j, 0, lane, b);
+                frag_b(sb + Ly::KT, LT, 8 * j, 0, lane, b);
                 mma16816(w[j], a, b[0], b[1]);
                 mma16816(w[j + 1], a, b[2], b[3]);
             }
@@ -370,7 +383,7 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
 #pragma unroll
             for (int k0 = 0; k0 < DK; k0 += 16) {
                 uint32_t a[4];
-                frag_a(sb + Ly::QT, LK, 0, k0, lane, a);
+                frag_at(sb + Ly::QT, LT, 0, k0, lane, a);
 #pragma unroll
                 for (int j = 0; j < NVT; j += 2) {
                     uint32_t b[4];
@@ -415,7 +428,7 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
                 S[mk][j][2] *= gb; S[mk][j][3] *= gb;
             }
             uint32_t a[4];
-            frag_at(sb + Ly::KH, LK, 16 * mk, 0, lane, a);
+            frag_a(sb + Ly::KH, LT, 16 * mk, 0, lane, a);
 #pragma unroll
             for (int j = 0; j < NVT; j += 2) {
                 uint32_t b[4];
