@@ -512,6 +512,10 @@ __global__ void __launch_bounds__(128) kda_rec_seg_fixup(const float *oaug, cons
     }
 }
 
+}  // namespace
+cudaError_t launch_chunk_warp_widened(const ChunkParams &q, cudaStream_t st);
+namespace {
+
 template <typename Tin, int D>
 cudaError_t launch_rec_seg(const ChunkParams &p, int P, uint8_t *ws, cudaStream_t st) {
     const RecSegLayout L = rec_seg_layout(p, P, D);
@@ -530,7 +534,11 @@ cudaError_t launch_rec_seg(const ChunkParams &p, int P, uint8_t *ws, cudaStream_
     count_launch();
     kda_seg_setup<<<(p.N + 255) / 256, 256, 0, st>>>(p.cu_seqlens, p.T, p.N, P, 16, cu_v);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = launch_rec_t<Tin, D, 2 * D, true>(q, st)) != cudaSuccess) return e;
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value && D == 32)  // the widened run on tensor cores
+        e = launch_chunk_warp_widened(q, st);
+    else
+        e = launch_rec_t<Tin, D, 2 * D, true>(q, st);
+    if (e != cudaSuccess) return e;
     if ((e = seg_chain_launch<D>(p.S0, saug, saug + D, 2 * D, 2LL * D * D, sstart, p.S_out, p.N, p.H, P, st)) !=
         cudaSuccess)
         return e;

@@ -106,10 +106,15 @@ __device__ __forceinline__ void stb2(uint8_t *p, float a, float b) {
 }
 __device__ __forceinline__ float e2(float x) { return ex2a(x * kL2e); }
 
-template <int DV>
+// AUG: the widened run of the segment form (kda_chunk_rec.cu): the state is [M | N]
+// (32 x DV, DV = 32 + d_v), the first 32 columns start from the identity and see v = 0,
+// the others start from zero and see v; the outputs [scale M^T q^ | scale N^T q^] go
+// out in fp32 as rows of DV and the final state as [32][DV].
+template <int DV, bool AUG>
 __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const ChunkParams p) {
     using Ly = Lay<DV>;
     constexpr int LV = Ly::LV, NVT = DV / 8;
+    constexpr int VOFF = AUG ? DK : 0, DVR = DV - VOFF;  // v's columns in the state, and its width
     extern __shared__ __align__(16) uint8_t smem_raw[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const long long chain = (long long)blockIdx.x * NWARP + warp;
@@ -146,8 +151,8 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
         const bool ok = r < L;
         const long long row = (t0 + (ok ? r : 0)) * H + h;
         const __nv_bfloat16 *qs = qg + row * DK + 16 * hf, *ks = kg + row * DK + 16 * hf, *gs = gg + row * DK + 16 * hf;
-        const __nv_bfloat16 *vs = vg + row * DV + (DV / 2) * hf;
-        const uint32_t o = (r * LK + 16 * hf) * 2, ov = (r * LV + (DV / 2) * hf) * 2;
+        const __nv_bfloat16 *vs = vg + row * DVR + (DVR / 2) * hf;
+        const uint32_t o = (r * LK + 16 * hf) * 2, ov = (r * LV + VOFF + (DVR / 2) * hf) * 2;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
             cp16z(sm + Ly::Q + o + 16 * c, qs + 8 * c, ok);
@@ -155,7 +160,7 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
             cp16z(sm + Ly::G + o + 16 * c, gs + 8 * c, ok);
         }
 #pragma unroll
-        for (int c = 0; c < DV / 16; ++c) cp16z(sm + Ly::V + ov + 16 * c, vs + 8 * c, ok);
+        for (int c = 0; c < DVR / 16; ++c) cp16z(sm + Ly::V + ov + 16 * c, vs + 8 * c, ok);
         braw = lane < L ? __bfloat162float(betag[(t0 + lane) * H + h]) : 0.f;
         cp_async_commit();
     };
@@ -170,8 +175,13 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int c = 16 * mk + g8 + 8 * (i >> 1), v = 8 * j + 2 * t4 + (i & 1);
-                S[mk][j][i] = p.S0 ? p.S0[sbase + (long long)c * DV + v] : 0.f;
+                S[mk][j][i] = AUG ? (c == v ? 1.f : 0.f) : p.S0 ? p.S0[sbase + (long long)c * DV + v] : 0.f;
             }
+    if constexpr (AUG) {  // the identity block sees v = 0: its columns of the v tile stay zero
+        const uint32_t z = ((lane >> 1) * LV + 16 * (lane & 1)) * 2;
+        sts128(sm, Ly::V + z, make_uint4(0u, 0u, 0u, 0u));
+        sts128(sm, Ly::V + z + 16, make_uint4(0u, 0u, 0u, 0u));
+    }
 
     if (nmc > 0) issue(0);
     for (int mc = 0; mc < nmc; ++mc) {
@@ -403,17 +413,22 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
                     mma16816(O[j + 1], a, b[2], b[3]);
                 }
             }
-            if (og) {
+            if (p.o) {
+                const float f = p.scale;  // Qtil and A_qk are built from q^
 #pragma unroll
                 for (int hi = 0; hi < 2; ++hi) {
                     const int r = g8 + 8 * hi;
                     if (r < L) {
-                        const float f = p.scale;  // Qtil and A_qk are built from q^
-                        __nv_bfloat16 *orow = og + ((t0 + r) * H + h) * DV + 2 * t4;
+                        const long long ob = ((t0 + r) * H + h) * DV + 2 * t4;
 #pragma unroll
-                        for (int j = 0; j < NVT; ++j)
-                            *reinterpret_cast<__nv_bfloat162 *>(orow + 8 * j) =
-                                __floats2bfloat162_rn(f * O[j][2 * hi], f * O[j][2 * hi + 1]);
+                        for (int j = 0; j < NVT; ++j) {
+                            if constexpr (AUG)
+                                *reinterpret_cast<float2 *>(static_cast<float *>(p.o) + ob + 8 * j) =
+                                    make_float2(f * O[j][2 * hi], f * O[j][2 * hi + 1]);
+                            else
+                                *reinterpret_cast<__nv_bfloat162 *>(og + ob + 8 * j) =
+                                    __floats2bfloat162_rn(f * O[j][2 * hi], f * O[j][2 * hi + 1]);
+                        }
                     }
                 }
             }
@@ -454,15 +469,16 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
     }
 }
 
-template <int DV>
+template <int DV, bool AUG = false>
 cudaError_t launch_t(const ChunkParams &p, cudaStream_t st) {
     const long long chains = (long long)p.N * p.H;
     if (chains <= 0) return cudaSuccess;
     const uint32_t smem = NWARP * Lay<DV>::BYTES;
-    cudaError_t e = cudaFuncSetAttribute(kda_chunk_warp_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(kda_chunk_warp_kernel<DV, AUG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    kda_chunk_warp_kernel<DV><<<(unsigned)((chains + NWARP - 1) / NWARP), NWARP * 32, smem, st>>>(p);
+    kda_chunk_warp_kernel<DV, AUG><<<(unsigned)((chains + NWARP - 1) / NWARP), NWARP * 32, smem, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -473,5 +489,9 @@ bool chunk_warp_supported(bool bf16, int Dk, int Dv) { return bf16 && Dk == 32 &
 cudaError_t launch_chunk_warp(const ChunkParams &p, int Dv, cudaStream_t st) {
     return Dv == 32 ? cw::launch_t<32>(p, st) : cw::launch_t<64>(p, st);
 }
+
+// The widened run of the segment form for bf16 d_k = d_v = 32 (outputs fp32 rows of 64,
+// final states [32][64]); q is the segment view.
+cudaError_t launch_chunk_warp_widened(const ChunkParams &q, cudaStream_t st) { return cw::launch_t<64, true>(q, st); }
 
 }  // namespace kda
