@@ -41,13 +41,16 @@ constexpr float kSpan = 80.f;  // largest |G - G_mid| of the split products
 template <int DV>
 struct Lay {
     static constexpr int LV = DV + 8;                      // padded row of [*][DV] bf16 tiles
-    static constexpr uint32_t Q = 0, K = Q + CW * LK * 2, G = K + CW * LK * 2, V = G + CW * LK * 2;
-    static constexpr uint32_t B = V + CW * LV * 2;          // raw beta [16] (f32)
+    // two input stages (micro-chunk parity): raw q, k, g rows [16][32] (read by column or
+    // whole rows: no padding) and v [16][LV]
+    static constexpr uint32_t Q = 0, K = Q + CW * DK * 2, G = K + CW * DK * 2, V = G + CW * DK * 2;
+    static constexpr uint32_t IN = (V + CW * LV * 2 + 127) / 128 * 128;
+    static constexpr uint32_t B = 2 * IN;
     // the operand tiles, stored transposed ([32 channels][16 rows], rows of LT): X^T of
     // k^ e^{G-M} (later the -W tile, [16][LK]), Y^T of k^ e^{M-G}, XQ^T of q^ e^{G-M},
     // KT^T of k^ e^G, QT^T of q^ e^G, KH^T of k^ e^{G_last-G}
     static constexpr uint32_t TT = DK * LT * 2;
-    static constexpr uint32_t X = B + 64;
+    static constexpr uint32_t X = B;
     static constexpr uint32_t Y = X + TT;
     static constexpr uint32_t XQ = Y + TT;
     static constexpr uint32_t D = Y;                         // D (bf16 [16][LV]) over Y and XQ
@@ -138,9 +141,9 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
     const float rate = p.gate_mode != kGateLog ? expf(p.A_log[h]) : 0.f;
     const float bias = (p.gate_mode != kGateLog && p.dt_bias) ? p.dt_bias[(long long)h * DK + lane] : 0.f;
 
-    // raw rows of micro-chunk mc (rows past the sequence zero-filled): q, k, g, v by
-    // cp.async; lane r < 16 also loads token r's beta into braw (stored to shared memory
-    // after the copies are waited for, so the load does not stall the warp here)
+    // raw rows of micro-chunk mc (rows past the sequence zero-filled) into input stage
+    // mc % 2: q, k, g, v by cp.async; lane r < 16 also loads token r's beta into braw
+    // (a register, used one micro-chunk later, so the load does not stall the warp)
     float braw = 0.f;
     // lane (row r = lane / 2, half hf = lane % 2): pieces hf*2, hf*2+1 of its q, k, g rows
     // and hf*DV/16 .. of its v row (16-byte pieces)
@@ -152,7 +155,8 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
         const long long row = (t0 + (ok ? r : 0)) * H + h;
         const __nv_bfloat16 *qs = qg + row * DK + 16 * hf, *ks = kg + row * DK + 16 * hf, *gs = gg + row * DK + 16 * hf;
         const __nv_bfloat16 *vs = vg + row * DVR + (DVR / 2) * hf;
-        const uint32_t o = (r * LK + 16 * hf) * 2, ov = (r * LV + VOFF + (DVR / 2) * hf) * 2;
+        const uint32_t in = (mc & 1) * Ly::IN;
+        const uint32_t o = in + (r * DK + 16 * hf) * 2, ov = in + (r * LV + VOFF + (DVR / 2) * hf) * 2;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
             cp16z(sm + Ly::Q + o + 16 * c, qs + 8 * c, ok);
@@ -177,18 +181,27 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
                 const int c = 16 * mk + g8 + 8 * (i >> 1), v = 8 * j + 2 * t4 + (i & 1);
                 S[mk][j][i] = AUG ? (c == v ? 1.f : 0.f) : p.S0 ? p.S0[sbase + (long long)c * DV + v] : 0.f;
             }
-    if constexpr (AUG) {  // the identity block sees v = 0: its columns of the v tile stay zero
+    if constexpr (AUG) {  // the identity block sees v = 0: its columns of both v tiles stay zero
         const uint32_t z = ((lane >> 1) * LV + 16 * (lane & 1)) * 2;
-        sts128(sm, Ly::V + z, make_uint4(0u, 0u, 0u, 0u));
-        sts128(sm, Ly::V + z + 16, make_uint4(0u, 0u, 0u, 0u));
+#pragma unroll
+        for (int st2 = 0; st2 < 2; ++st2) {
+            sts128(sm, st2 * Ly::IN + Ly::V + z, make_uint4(0u, 0u, 0u, 0u));
+            sts128(sm, st2 * Ly::IN + Ly::V + z + 16, make_uint4(0u, 0u, 0u, 0u));
+        }
     }
 
     if (nmc > 0) issue(0);
     for (int mc = 0; mc < nmc; ++mc) {
         const long long t0 = bos + (long long)mc * CW;
         const int L = (int)min((long long)CW, eos - t0);
-        if (lane < CW) reinterpret_cast<float *>(sm + Ly::B)[lane] = braw;
-        cp_async_wait_all();
+        const float bcur = braw;  // beta of this micro-chunk's row `lane` (lane < 16)
+        const uint32_t in = (mc & 1) * Ly::IN;
+        if (mc + 1 < nmc) {  // the next micro-chunk's rows into the other stage, then wait for ours
+            issue(mc + 1);
+            cp_async_wait_group<1>();
+        } else {
+            cp_async_wait_all();
+        }
         __syncwarp();
         // ---- gate and its in-chunk cumsum: lane = channel, G[r] for the 16 rows (the 16
         // gate values first, independently, then the running sum)
@@ -196,7 +209,7 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
         {
 #pragma unroll
             for (int r = 0; r < CW; ++r) {
-                const float x = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(sm + Ly::G)[r * LK + lane]);
+                const float x = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::G)[r * DK + lane]);
                 const float gv = p.gate_mode == kGateLog ? (p.has_lb ? fmaxf(x, p.lb) : x)
                                                          : gate_fast(x, bias, rate, p.gate_mode, p.lb);
                 G[r] = r < L ? gv : 0.f;
@@ -207,7 +220,7 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
         // ---- row norms (lanes 0..15: k rows, 16..31: q rows) and write strengths
         {
             const int r = lane & 15;
-            const uint32_t row = (lane < 16 ? Ly::K : Ly::Q) + r * LK * 2;
+            const uint32_t row = in + (lane < 16 ? Ly::K : Ly::Q) + r * DK * 2;
             float s = 0.f;
 #pragma unroll
             for (int c8 = 0; c8 < DK / 8; ++c8) {
@@ -219,8 +232,7 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
             const float inv = r < L ? (p.use_l2 ? rsqrtf(s + 1e-6f) : 1.f) : 0.f;
             if (lane < 16) {
                 rk[r] = inv;
-                const float bx = reinterpret_cast<const float *>(sm + Ly::B)[r];
-                bb[r] = r < L ? beta_value(bx, p.beta_prob) : 0.f;
+                bb[r] = r < L ? beta_value(bcur, p.beta_prob) : 0.f;
             } else {
                 rq[r] = inv;
             }
@@ -232,16 +244,16 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
         const float Gm = G[7], GC = G[CW - 1];
         bool steep = false;
         {
-            const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(sm + Ly::K);
-            const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(sm + Ly::Q);
+            const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::K);
+            const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::Q);
 #pragma unroll
             for (int h8 = 0; h8 < 2; ++h8) {
                 float x[8], y[8], xq[8], kt[8], qt[8], kc[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int r = 8 * h8 + u;
-                    const float kh = __bfloat162float(kr[r * LK + lane]) * rk[r];
-                    const float qh = __bfloat162float(qr[r * LK + lane]) * rq[r];
+                    const float kh = __bfloat162float(kr[r * DK + lane]) * rk[r];
+                    const float qh = __bfloat162float(qr[r * DK + lane]) * rq[r];
                     const float dm = G[r] - Gm;
                     steep |= fabsf(dm) > kSpan;
                     const float em = e2(dm), en = e2(-dm), eg = e2(G[r]), ec = e2(GC - G[r]);
@@ -291,17 +303,17 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
 #pragma unroll
             for (int r = 0; r < CW; ++r) Gs[r * 33 + lane] = G[r];
             __syncwarp();
-            const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(sm + Ly::K);
-            const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(sm + Ly::Q);
+            const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::K);
+            const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::Q);
             for (int e = lane; e < CW * CW; e += 32) {
                 const int r = e >> 4, s = e & 15;
                 if (s > r) continue;
                 float akk = 0.f, aqk = 0.f;
                 for (int c = 0; c < DK; ++c) {
                     const float ed = expf(Gs[r * 33 + c] - Gs[s * 33 + c]);
-                    const float ks = __bfloat162float(kr[s * LK + c]) * ed;
-                    akk = fmaf(__bfloat162float(kr[r * LK + c]), ks, akk);
-                    aqk = fmaf(__bfloat162float(qr[r * LK + c]), ks, aqk);
+                    const float ks = __bfloat162float(kr[s * DK + c]) * ed;
+                    akk = fmaf(__bfloat162float(kr[r * DK + c]), ks, akk);
+                    aqk = fmaf(__bfloat162float(qr[r * DK + c]), ks, aqk);
                 }
                 akk *= rk[r] * rk[s];
                 aqk *= rq[r] * rk[s];
@@ -335,7 +347,7 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
 #pragma unroll
             for (int j = 0; j < NVT; j += 2) {
                 uint32_t b[4];
-                frag_bt(sb + Ly::V, LV, 8 * j, 0, lane, b);
+                frag_bt(sb + in + Ly::V, LV, 8 * j, 0, lane, b);
                 U[j][0] = U[j][1] = U[j][2] = U[j][3] = 0.f;
                 U[j + 1][0] = U[j + 1][1] = U[j + 1][2] = U[j + 1][3] = 0.f;
                 mma16816(U[j], a, b[0], b[1]);
@@ -364,8 +376,7 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
                 for (int hi = 0; hi < 2; ++hi)
                     stb2(sm + Ly::S + ((16 * mk + g8 + 8 * hi) * LV + 8 * j + 2 * t4) * 2, S[mk][j][2 * hi],
                          S[mk][j][2 * hi + 1]);
-        __syncwarp();  // the raw rows are consumed: the next micro-chunk's copies start
-        if (mc + 1 < nmc) issue(mc + 1);
+        __syncwarp();
         // ---- D = U - W S (in U's registers) -> bf16 tile
 #pragma unroll
         for (int k0 = 0; k0 < DK; k0 += 16) {
