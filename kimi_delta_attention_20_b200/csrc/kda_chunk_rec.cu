@@ -407,10 +407,15 @@ cudaError_t launch_rec_dt(const ChunkParams &p, int Dk, int Dv, cudaStream_t st)
 constexpr int kRecMaxSeg = 16;
 constexpr int kRecChains = 8 * 148;  // chains wanted in flight: several small CTAs per SM
 
-int rec_seg_count(const ChunkParams &p, int Dk, int Dv) {
+int rec_seg_count(const ChunkParams &p, int Dk, int Dv, bool bf16) {
     if (Dk != Dv || (Dk != 32 && Dk != 64)) return 1;
     const long long chains = (long long)p.N * p.H;
     if (chains <= 0 || chains * 2 > kRecChains) return 1;
+    // bf16 d = 64: from 128 chains on, the micro-chunk form (kda_chunk_warp.cu) beats the
+    // segments, whose widened run is the recurrence at twice the width (B T2048 H8:
+    // 128 chains 0.41 against 0.64 ms, 512 chains 0.52 against 2.13 ms; 64 chains 0.37
+    // against 0.34 ms)
+    if (bf16 && Dk == 64 && chains >= 128) return 1;
     const long long avg = p.cu_seqlens ? (long long)p.T / (p.N > 0 ? p.N : 1) : (long long)p.T;
     long long P = std::min<long long>(kRecMaxSeg, kRecChains / chains);
     P = std::min<long long>(P, avg / 64);  // at least 64 tokens per segment on average
@@ -570,26 +575,25 @@ cudaError_t rec_widened_run(const ChunkParams &q, bool bf16, int D, cudaStream_t
 
 // Workspace the recurrent forward can use (0: it needs none).
 size_t chunk_rec_workspace_bytes(const ChunkParams &p, bool bf16, int Dk, int Dv) {
-    const int P = rec_seg_count(p, Dk, Dv);
-    (void)bf16;
+    const int P = rec_seg_count(p, Dk, Dv, bf16);
     return P < 2 ? 0 : rec_seg_layout(p, P, Dk).total;
 }
 
 bool chunk_warp_supported(bool bf16, int Dk, int Dv);
-cudaError_t launch_chunk_warp(const ChunkParams &p, int Dv, cudaStream_t st);
+cudaError_t launch_chunk_warp(const ChunkParams &p, int Dk, int Dv, cudaStream_t st);
 
 // Few chains of long sequences: the segment form of the recurrence; otherwise, for bf16
-// with d_k = 32, the tensor-core micro-chunk form (one warp per chain, kda_chunk_warp.cu);
+// with d_k 32 or 64 and d_v 32 or 64, the tensor-core micro-chunk form (kda_chunk_warp.cu);
 // otherwise the recurrence.
 cudaError_t launch_chunk_rec(const ChunkParams &p, bool bf16, int Dk, int Dv, void *workspace, size_t workspace_bytes,
                              cudaStream_t st) {
-    const int P = rec_seg_count(p, Dk, Dv);
+    const int P = rec_seg_count(p, Dk, Dv, bf16);
     if (P >= 2 && workspace && (reinterpret_cast<uintptr_t>(workspace) & 255) == 0 &&
         workspace_bytes >= rec_seg_layout(p, P, Dk).total) {
         uint8_t *ws = static_cast<uint8_t *>(workspace);
         return bf16 ? launch_rec_seg_dt<__nv_bfloat16>(p, P, Dk, ws, st) : launch_rec_seg_dt<float>(p, P, Dk, ws, st);
     }
-    if (P < 2 && chunk_warp_supported(bf16, Dk, Dv)) return launch_chunk_warp(p, Dv, st);
+    if (P < 2 && chunk_warp_supported(bf16, Dk, Dv)) return launch_chunk_warp(p, Dk, Dv, st);
     return bf16 ? launch_rec_dt<__nv_bfloat16>(p, Dk, Dv, st) : launch_rec_dt<float>(p, Dk, Dv, st);
 }
 

@@ -493,11 +493,403 @@ cudaError_t launch_t(const ChunkParams &p, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+
+// ---- d_k = 64: one CTA of two warps per chain. Warp w owns the value columns
+// [VW w, VW w + VW) of the 64 x d_v state (VW = d_v / 2, registers) and the key channels
+// [32 w, 32 w + 32) of the gate and of the transposed operand tiles; the 16 x 16 blocks
+// are split between the warps (warp 0 A_kk and the inverse, warp 1 A_qk), and block
+// barriers separate the phases that read the other warp's half.
+namespace w64 {
+constexpr int DK2 = 64;
+constexpr int LKR = DK2 + 8;  // padded raw row (elements): 144 B, conflict-free row reads
+constexpr int LW = DK2 + 8;   // the -W tile [16][LW]
+template <int DV>
+struct Lay {
+    static constexpr int LV = DV + 8;
+    static constexpr uint32_t Q = 0, K = Q + CW * LKR * 2, G = K + CW * LKR * 2, V = G + CW * LKR * 2;
+    static constexpr uint32_t IN = (V + CW * LV * 2 + 127) / 128 * 128;
+    static constexpr uint32_t TT = DK2 * LT * 2;             // a transposed tile [64][LT]
+    static constexpr uint32_t X = 2 * IN, Y = X + TT, XQ = Y + TT, KT = XQ + TT, QT = KT + TT, KH = QT + TT;
+    static constexpr uint32_t W = X;                          // -W [16][LW] over X^T
+    static constexpr uint32_t D = Y;                          // D [16][LV] over Y^T
+    static constexpr uint32_t TP = KH + TT, AQ = TP + CW * LT * 2;
+    static constexpr uint32_t S = AQ + CW * LT * 2;           // S bf16 [64][LV]; exponent scratch [16][65] f32
+    static constexpr uint32_t L = S + DK2 * LV * 2;
+    static constexpr uint32_t RK = L + CW * LL * 4, RQ = RK + 64, BB = RQ + 64, PART = BB + 64, GAM = PART + 256;
+    static constexpr uint32_t BYTES = (GAM + DK2 * 4 + 127) / 128 * 128;
+    static_assert(CW * LW * 2 <= TT && CW * LV * 2 <= TT && CW * 65 * 4 <= DK2 * LV * 2, "aliases");
+};
+
+template <int DV>
+__global__ void __launch_bounds__(64, 4) kda_chunk_warp64_kernel(const ChunkParams p) {
+    using Ly = Lay<DV>;
+    constexpr int LV = Ly::LV, VW = DV / 2, NVT = VW / 8;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const long long chain = blockIdx.x;
+    const int n = (int)(chain / p.H), h = (int)(chain % p.H);
+    uint8_t *sm = smem_raw;
+    const uint32_t sb = sm100::smem_u32(sm);
+    float *rk = reinterpret_cast<float *>(sm + Ly::RK), *rq = reinterpret_cast<float *>(sm + Ly::RQ);
+    float *bb = reinterpret_cast<float *>(sm + Ly::BB), *gam = reinterpret_cast<float *>(sm + Ly::GAM);
+    float *part = reinterpret_cast<float *>(sm + Ly::PART);
+    float *Lf = reinterpret_cast<float *>(sm + Ly::L);
+    const int H = p.H, g8 = lane >> 2, t4 = lane & 3, c = 32 * w + lane;  // this thread's key channel
+    long long bos, eos;
+    if (p.cu_seqlens) { bos = p.cu_seqlens[n]; eos = p.cu_seqlens[n + 1]; }
+    else { bos = (long long)n * p.T; eos = bos + p.T; }
+    const int nmc = (int)((eos - bos + CW - 1) / CW);
+    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(p.q), *kg = static_cast<const __nv_bfloat16 *>(p.k);
+    const __nv_bfloat16 *gg = static_cast<const __nv_bfloat16 *>(p.g), *vg = static_cast<const __nv_bfloat16 *>(p.v);
+    const __nv_bfloat16 *betag = static_cast<const __nv_bfloat16 *>(p.beta);
+    __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(p.o);
+    const float rate = p.gate_mode != kGateLog ? expf(p.A_log[h]) : 0.f;
+    const float bias = (p.gate_mode != kGateLog && p.dt_bias) ? p.dt_bias[(long long)h * DK2 + c] : 0.f;
+
+    // thread (row r = tid / 4, quarter qq = tid % 4): q, k, g pieces 2 qq, 2 qq + 1 and its
+    // share of the v row; thread r < 16 also loads token r's beta into braw
+    float braw = 0.f;
+    auto issue = [&](int mc) {
+        const long long t0 = bos + (long long)mc * CW;
+        const int L = (int)min((long long)CW, eos - t0);
+        const int r = tid >> 2, qq = tid & 3;
+        const bool ok = r < L;
+        const long long row = (t0 + (ok ? r : 0)) * H + h;
+        const uint32_t in = (mc & 1) * Ly::IN, o = in + (r * LKR + 16 * qq) * 2;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            cp16z(sm + Ly::Q + o + 16 * cc, qg + row * DK2 + 16 * qq + 8 * cc, ok);
+            cp16z(sm + Ly::K + o + 16 * cc, kg + row * DK2 + 16 * qq + 8 * cc, ok);
+            cp16z(sm + Ly::G + o + 16 * cc, gg + row * DK2 + 16 * qq + 8 * cc, ok);
+        }
+        constexpr int VP = DV / 32;  // 16-byte v pieces per thread
+#pragma unroll
+        for (int cc = 0; cc < VP; ++cc) {
+            const int piece = VP * qq + cc;
+            cp16z(sm + in + Ly::V + (r * LV + 8 * piece) * 2, vg + row * DV + 8 * piece, ok);
+        }
+        braw = tid < L ? __bfloat162float(betag[(t0 + tid) * H + h]) : 0.f;
+        cp_async_commit();
+    };
+
+    float S[4][NVT][4];  // rows 16 mk + g8 (+ 8), columns VW w + 8 j + 2 t4 (+ 1)
+    const long long sbase = ((long long)n * H + h) * DK2 * DV;
+#pragma unroll
+    for (int mk = 0; mk < 4; ++mk)
+#pragma unroll
+        for (int j = 0; j < NVT; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int cr = 16 * mk + g8 + 8 * (i >> 1), v = VW * w + 8 * j + 2 * t4 + (i & 1);
+                S[mk][j][i] = p.S0 ? p.S0[sbase + (long long)cr * DV + v] : 0.f;
+            }
+
+    if (nmc > 0) issue(0);
+    for (int mc = 0; mc < nmc; ++mc) {
+        const long long t0 = bos + (long long)mc * CW;
+        const int L = (int)min((long long)CW, eos - t0);
+        const float bcur = braw;
+        const uint32_t in = (mc & 1) * Ly::IN;
+        if (mc + 1 < nmc) {
+            issue(mc + 1);
+            cp_async_wait_group<1>();
+        } else {
+            cp_async_wait_all();
+        }
+        __syncthreads();
+        // gate and cumsum for channel c
+        float G[CW];
+#pragma unroll
+        for (int r = 0; r < CW; ++r) {
+            const float x = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::G)[r * LKR + c]);
+            const float gv = p.gate_mode == kGateLog ? (p.has_lb ? fmaxf(x, p.lb) : x)
+                                                     : gate_fast(x, bias, rate, p.gate_mode, p.lb);
+            G[r] = r < L ? gv : 0.f;
+        }
+#pragma unroll
+        for (int r = 1; r < CW; ++r) G[r] += G[r - 1];
+        // row norms: each warp sums its 32 channels (lanes 0..15 k rows, 16..31 q rows)
+        {
+            const int r = lane & 15;
+            const uint32_t row = in + (lane < 16 ? Ly::K : Ly::Q) + (r * LKR + 32 * w) * 2;
+            float sacc = 0.f;
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8) {
+                float f[8];
+                unpack8(lds128(sm, row + 16 * c8), f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) sacc = fmaf(f[e], f[e], sacc);
+            }
+            part[w * 32 + lane] = sacc;
+        }
+        __syncthreads();
+        if (tid < 32) {
+            const int r = tid & 15;
+            const float ssum = part[tid] + part[32 + tid];
+            const float inv = r < L ? (p.use_l2 ? rsqrtf(ssum + 1e-6f) : 1.f) : 0.f;
+            if (tid < 16) {
+                rk[r] = inv;
+                bb[r] = r < L ? beta_value(bcur, p.beta_prob) : 0.f;
+            } else {
+                rq[r] = inv;
+            }
+        }
+        __syncthreads();
+        // operand tiles, row c of each transposed tile
+        const float Gm = G[7], GC = G[CW - 1];
+        bool steep = false;
+        {
+            const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::K);
+            const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::Q);
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+                float x[8], y[8], xq[8], kt[8], qt[8], kc[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int r = 8 * h8 + u;
+                    const float kh = __bfloat162float(kr[r * LKR + c]) * rk[r];
+                    const float qh = __bfloat162float(qr[r * LKR + c]) * rq[r];
+                    const float dm = G[r] - Gm;
+                    steep |= fabsf(dm) > kSpan;
+                    const float em = e2(dm), en = e2(-dm), eg = e2(G[r]), ec = e2(GC - G[r]);
+                    x[u] = kh * em; y[u] = kh * en; xq[u] = qh * em;
+                    kt[u] = kh * eg; qt[u] = qh * eg; kc[u] = kh * ec;
+                }
+                const uint32_t o = (c * LT + 8 * h8) * 2;
+                sts128(sm, Ly::X + o, pack8(x));
+                sts128(sm, Ly::Y + o, pack8(y));
+                sts128(sm, Ly::XQ + o, pack8(xq));
+                sts128(sm, Ly::KT + o, pack8(kt));
+                sts128(sm, Ly::QT + o, pack8(qt));
+                sts128(sm, Ly::KH + o, pack8(kc));
+            }
+            gam[c] = e2(GC);
+        }
+        steep = __syncthreads_or(steep) != 0;
+        // A_kk (warp 0) -> L = diag(b) A_kk; A_qk (warp 1) -> bf16 tile
+        {
+            float acc[2][4] = {};
+            const uint32_t xa = w == 0 ? Ly::X : Ly::XQ;
+#pragma unroll
+            for (int k0 = 0; k0 < DK2; k0 += 16) {
+                uint32_t a[4], b[4];
+                frag_at(sb + xa, LT, 0, k0, lane, a);
+                frag_bt(sb + Ly::Y, LT, 0, k0, lane, b);
+                mma16816(acc[0], a, b[0], b[1]);
+                mma16816(acc[1], a, b[2], b[3]);
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi) {
+                    const int r = g8 + 8 * hi, s_ = 8 * j + 2 * t4;
+                    if (w == 0) {
+                        const float br = bb[r];
+                        Lf[r * LL + s_] = s_ < r ? br * acc[j][2 * hi] : 0.f;
+                        Lf[r * LL + s_ + 1] = s_ + 1 < r ? br * acc[j][2 * hi + 1] : 0.f;
+                    } else {
+                        stb2(sm + Ly::AQ + (r * LT + s_) * 2, s_ <= r ? acc[j][2 * hi] : 0.f,
+                             s_ + 1 <= r ? acc[j][2 * hi + 1] : 0.f);
+                    }
+                }
+        }
+        if (steep) {  // exponent differences (never positive) on the CUDA cores
+            float *Gs = reinterpret_cast<float *>(sm + Ly::S);
+#pragma unroll
+            for (int r = 0; r < CW; ++r) Gs[r * 65 + c] = G[r];
+            __syncthreads();
+            const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::K);
+            const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::Q);
+            for (int e = tid; e < CW * CW; e += 64) {
+                const int r = e >> 4, s_ = e & 15;
+                if (s_ > r) continue;
+                float akk = 0.f, aqk = 0.f;
+                for (int cc = 0; cc < DK2; ++cc) {
+                    const float ed = expf(Gs[r * 65 + cc] - Gs[s_ * 65 + cc]);
+                    const float ks = __bfloat162float(kr[s_ * LKR + cc]) * ed;
+                    akk = fmaf(__bfloat162float(kr[r * LKR + cc]), ks, akk);
+                    aqk = fmaf(__bfloat162float(qr[r * LKR + cc]), ks, aqk);
+                }
+                akk *= rk[r] * rk[s_];
+                aqk *= rq[r] * rk[s_];
+                if (s_ < r) Lf[r * LL + s_] = bb[r] * akk;
+                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::AQ)[r * LT + s_] = __float2bfloat16_rn(aqk);
+            }
+        }
+        __syncthreads();
+        // T' by forward substitution (warp 0, lane j < 16: column j)
+        if (w == 0 && lane < CW) {
+            const int j = lane;
+            float t[CW];
+#pragma unroll
+            for (int i = 0; i < CW; ++i) {
+                float acc = i == j ? 1.f : 0.f;
+#pragma unroll
+                for (int k = 0; k < i; ++k) acc = fmaf(-Lf[i * LL + k], t[k], acc);
+                t[i] = acc;
+            }
+            const float bj = bb[j];
+#pragma unroll
+            for (int i = 0; i < CW; ++i)
+                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::TP)[i * LT + j] = __float2bfloat16_rn(t[i] * bj);
+        }
+        __syncthreads();
+        // U (own value columns, registers); -W for own key channels into the shared tile
+        float U[NVT][4];
+        {
+            uint32_t a[4];
+            frag_a(sb + Ly::TP, LT, 0, 0, lane, a);
+#pragma unroll
+            for (int j = 0; j < NVT; j += 2) {
+                uint32_t b[4];
+                frag_bt(sb + in + Ly::V, LV, VW * w + 8 * j, 0, lane, b);
+                U[j][0] = U[j][1] = U[j][2] = U[j][3] = 0.f;
+                U[j + 1][0] = U[j + 1][1] = U[j + 1][2] = U[j + 1][3] = 0.f;
+                mma16816(U[j], a, b[0], b[1]);
+                mma16816(U[j + 1], a, b[2], b[3]);
+            }
+            float wv[4][4] = {};
+#pragma unroll
+            for (int j = 0; j < 4; j += 2) {
+                uint32_t b[4];
+                frag_b(sb + Ly::KT, LT, 32 * w + 8 * j, 0, lane, b);
+                mma16816(wv[j], a, b[0], b[1]);
+                mma16816(wv[j + 1], a, b[2], b[3]);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi)
+                    stb2(sm + Ly::W + ((g8 + 8 * hi) * LW + 32 * w + 8 * j + 2 * t4) * 2, -wv[j][2 * hi],
+                         -wv[j][2 * hi + 1]);
+        }
+        // own columns of the state as a bf16 operand
+#pragma unroll
+        for (int mk = 0; mk < 4; ++mk)
+#pragma unroll
+            for (int j = 0; j < NVT; ++j)
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi)
+                    stb2(sm + Ly::S + ((16 * mk + g8 + 8 * hi) * LV + VW * w + 8 * j + 2 * t4) * 2, S[mk][j][2 * hi],
+                         S[mk][j][2 * hi + 1]);
+        __syncthreads();  // -W complete
+        // D = U - W S (own columns) -> bf16 tile
+#pragma unroll
+        for (int k0 = 0; k0 < DK2; k0 += 16) {
+            uint32_t a[4];
+            frag_a(sb + Ly::W, LW, 0, k0, lane, a);
+#pragma unroll
+            for (int j = 0; j < NVT; j += 2) {
+                uint32_t b[4];
+                frag_bt(sb + Ly::S, LV, VW * w + 8 * j, k0, lane, b);
+                mma16816(U[j], a, b[0], b[1]);
+                mma16816(U[j + 1], a, b[2], b[3]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < NVT; ++j)
+#pragma unroll
+            for (int hi = 0; hi < 2; ++hi)
+                stb2(sm + Ly::D + ((g8 + 8 * hi) * LV + VW * w + 8 * j + 2 * t4) * 2, U[j][2 * hi], U[j][2 * hi + 1]);
+        __syncwarp();
+        // O = scale (Qtil S + A_qk D), own columns
+        {
+            float O[NVT][4];
+#pragma unroll
+            for (int j = 0; j < NVT; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
+#pragma unroll
+            for (int k0 = 0; k0 < DK2; k0 += 16) {
+                uint32_t a[4];
+                frag_at(sb + Ly::QT, LT, 0, k0, lane, a);
+#pragma unroll
+                for (int j = 0; j < NVT; j += 2) {
+                    uint32_t b[4];
+                    frag_bt(sb + Ly::S, LV, VW * w + 8 * j, k0, lane, b);
+                    mma16816(O[j], a, b[0], b[1]);
+                    mma16816(O[j + 1], a, b[2], b[3]);
+                }
+            }
+            {
+                uint32_t a[4];
+                frag_a(sb + Ly::AQ, LT, 0, 0, lane, a);
+#pragma unroll
+                for (int j = 0; j < NVT; j += 2) {
+                    uint32_t b[4];
+                    frag_bt(sb + Ly::D, LV, VW * w + 8 * j, 0, lane, b);
+                    mma16816(O[j], a, b[0], b[1]);
+                    mma16816(O[j + 1], a, b[2], b[3]);
+                }
+            }
+            if (og) {
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi) {
+                    const int r = g8 + 8 * hi;
+                    if (r < L) {
+                        __nv_bfloat16 *orow = og + ((t0 + r) * H + h) * DV + VW * w + 2 * t4;
+#pragma unroll
+                        for (int j = 0; j < NVT; ++j)
+                            *reinterpret_cast<__nv_bfloat162 *>(orow + 8 * j) =
+                                __floats2bfloat162_rn(p.scale * O[j][2 * hi], p.scale * O[j][2 * hi + 1]);
+                    }
+                }
+            }
+        }
+        // S <- diag(e^{G_last}) S + Khat^T D (own columns)
+#pragma unroll
+        for (int mk = 0; mk < 4; ++mk) {
+            const float ga = gam[16 * mk + g8], gb = gam[16 * mk + g8 + 8];
+#pragma unroll
+            for (int j = 0; j < NVT; ++j) {
+                S[mk][j][0] *= ga; S[mk][j][1] *= ga;
+                S[mk][j][2] *= gb; S[mk][j][3] *= gb;
+            }
+            uint32_t a[4];
+            frag_a(sb + Ly::KH, LT, 16 * mk, 0, lane, a);
+#pragma unroll
+            for (int j = 0; j < NVT; j += 2) {
+                uint32_t b[4];
+                frag_bt(sb + Ly::D, LV, VW * w + 8 * j, 0, lane, b);
+                mma16816(S[mk][j], a, b[0], b[1]);
+                mma16816(S[mk][j + 1], a, b[2], b[3]);
+            }
+        }
+        __syncthreads();  // every tile of this micro-chunk is read
+    }
+    cp_async_wait_all();
+    if (p.S_out) {
+#pragma unroll
+        for (int mk = 0; mk < 4; ++mk)
+#pragma unroll
+            for (int j = 0; j < NVT; ++j)
+#pragma unroll
+                for (int hi = 0; hi < 2; ++hi) {
+                    const int cr = 16 * mk + g8 + 8 * hi, v = VW * w + 8 * j + 2 * t4;
+                    *reinterpret_cast<float2 *>(p.S_out + sbase + (long long)cr * DV + v) =
+                        make_float2(S[mk][j][2 * hi], S[mk][j][2 * hi + 1]);
+                }
+    }
+}
+
+template <int DV>
+cudaError_t launch_t(const ChunkParams &p, cudaStream_t st) {
+    const long long chains = (long long)p.N * p.H;
+    if (chains <= 0) return cudaSuccess;
+    const uint32_t smem = Lay<DV>::BYTES;
+    cudaError_t e = cudaFuncSetAttribute(kda_chunk_warp64_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    count_launch();
+    kda_chunk_warp64_kernel<DV><<<(unsigned)chains, 64, smem, st>>>(p);
+    return cudaGetLastError();
+}
+}  // namespace w64
+
 }  // namespace cw
 
-bool chunk_warp_supported(bool bf16, int Dk, int Dv) { return bf16 && Dk == 32 && (Dv == 32 || Dv == 64); }
+bool chunk_warp_supported(bool bf16, int Dk, int Dv) { return bf16 && (Dk == 32 || Dk == 64) && (Dv == 32 || Dv == 64); }
 
-cudaError_t launch_chunk_warp(const ChunkParams &p, int Dv, cudaStream_t st) {
+cudaError_t launch_chunk_warp(const ChunkParams &p, int Dk, int Dv, cudaStream_t st) {
+    if (Dk == 64) return Dv == 32 ? cw::w64::launch_t<32>(p, st) : cw::w64::launch_t<64>(p, st);
     return Dv == 32 ? cw::launch_t<32>(p, st) : cw::launch_t<64>(p, st);
 }
 

@@ -1,8 +1,9 @@
-"""GPU parity of the micro-chunk tensor-core forward (bf16, d_k = 32, d_v 32 or 64: one
-warp per (sequence, head), 16-token micro-chunks) against form R, the token recurrence
-of page "atlas_core/kimi_k3/kda.rs" (`chunk_kda` of page "K3/kda/ops/api.py"). This
-form takes bf16 d_k = 32 calls that the segment form of the recurrence does not:
-many chains, short sequences, or d_k != d_v."""
+"""GPU parity of the micro-chunk tensor-core forward (bf16, d_k 32 or 64, d_v 32 or 64:
+16-token micro-chunks, one warp per (sequence, head) at d_k = 32, a CTA of two warps at
+d_k = 64) against form R, the token recurrence of page "atlas_core/kimi_k3/kda.rs"
+(`chunk_kda` of page "K3/kda/ops/api.py"). This form takes the bf16 calls of those
+shapes that the segment form of the recurrence does not: many chains, short sequences,
+or d_k != d_v."""
 import pytest
 import torch
 
@@ -39,35 +40,41 @@ def compare(inp, o, S, tag, **okw):
             check(f"{tag} S seq{n} h{h}", S[n, [h]], S_ref[[h]], DT)
 
 
-@pytest.mark.parametrize("dv", [32, 64])
-def test_warp_ragged_varlen(dv):
+DIMS = [(32, 32), (32, 64), (64, 32), (64, 64)]
+
+
+@pytest.mark.parametrize("dims", DIMS)
+def test_warp_ragged_varlen(dims):
     """Micro-chunk tails of every kind and empty sequences in a varlen batch."""
+    dk, dv = dims
     lens = [0, 1, 15, 16, 17, 33, 100, 0, 257, 64]
-    inp = KI.draw_chunk(1, sum(lens), 3, 32, dv, dtype=DT, seed=500 + dv, seqlens=lens, init_state=True)
+    inp = KI.draw_chunk(1, sum(lens), 3, dk, dv, dtype=DT, seed=500 + dk + dv, seqlens=lens, init_state=True)
     o, S = run(inp, use_qk_l2norm_in_kernel=True)
-    compare(inp, o, S, f"ragged d_v{dv}")
+    compare(inp, o, S, f"ragged {dims}")
 
 
-@pytest.mark.parametrize("dv", [32, 64])
-def test_warp_steep_gates(dv):
+@pytest.mark.parametrize("dims", DIMS)
+def test_warp_steep_gates(dims):
     """Gates that drop by up to ~100 per token: the middle-row split would leave the fp32
     range, so those micro-chunks take the exponent-difference products; others keep the
     tensor-core split."""
-    inp = KI.draw_chunk(2, 120, 2, 32, dv, dtype=DT, seed=510 + dv, init_state=True)
+    dk, dv = dims
+    inp = KI.draw_chunk(2, 120, 2, dk, dv, dtype=DT, seed=510 + dk + dv, init_state=True)
     g = inp["g"].float()
     g[:, 20:50] = g[:, 20:50] * 40.0
     inp["g"] = g.to(DT)
     o, S = run(inp, use_qk_l2norm_in_kernel=True)
-    compare(inp, o, S, f"steep d_v{dv}")
+    compare(inp, o, S, f"steep {dims}")
 
 
+@pytest.mark.parametrize("dk", [32, 64])
 @pytest.mark.parametrize("form", ["softplus", "safe"])
-def test_warp_in_kernel_gate(form):
+def test_warp_in_kernel_gate(form, dk):
     """The in-kernel gate forms (page "atlas_core/kimi_k3/kda.rs" `bounded_gate`)."""
-    inp = KI.draw_chunk(2, 150, 4, 32, 64, dtype=DT, seed=520 + len(form), init_state=True, gate="input")
+    inp = KI.draw_chunk(2, 150, 4, dk, 64, dtype=DT, seed=520 + len(form) + dk, init_state=True, gate="input")
     gen = torch.Generator().manual_seed(521)
     A_log = torch.empty(4).uniform_(-2.0, 0.5, generator=gen)
-    dt_bias = torch.randn(4, 32, generator=gen) * 0.5
+    dt_bias = torch.randn(4, dk, generator=gen) * 0.5
     kw = dict(use_gate_in_kernel=True, A_log=A_log.to(DEV), dt_bias=dt_bias.to(DEV), use_qk_l2norm_in_kernel=True)
     okw = dict(gate_form=form, A_log=A_log, dt_bias=dt_bias)
     if form == "safe":
@@ -77,18 +84,20 @@ def test_warp_in_kernel_gate(form):
     compare(inp, o, S, f"gate {form}", **okw)
 
 
-def test_warp_options():
+@pytest.mark.parametrize("dk", [32, 64])
+def test_warp_options(dk):
     """beta as a probability, no in-kernel L2 norm, an explicit scale, no initial state."""
-    inp = KI.draw_chunk(2, 90, 2, 32, 32, dtype=DT, seed=530, beta="prob")
+    inp = KI.draw_chunk(2, 90, 2, dk, 32, dtype=DT, seed=530 + dk, beta="prob")
     inp["k"] = (inp["k"].float() / 6.0).to(DT)
     with pytest.warns(RuntimeWarning):
         o, S = run(inp, use_qk_l2norm_in_kernel=False, use_beta_sigmoid_in_kernel=False, scale=0.37)
     compare(inp, o, S, "options", l2=False, beta_is_logit=False, scale=0.37)
 
 
-def test_warp_many_chains():
-    """1,024 chains (one wave of warps), a sample of sequences checked on every head."""
-    inp = KI.draw_chunk(64, 96, 16, 32, 64, dtype=DT, seed=540, init_state=True)
+@pytest.mark.parametrize("dk", [32, 64])
+def test_warp_many_chains(dk):
+    """1,024 chains (one wave), a sample of sequences checked on every head."""
+    inp = KI.draw_chunk(64, 96, 16, dk, 64, dtype=DT, seed=540 + dk, init_state=True)
     o, S = run(inp, use_qk_l2norm_in_kernel=True, lower_bound=-5.0)
     sub = {n: inp[n][[0, 31, 63]] for n in ("q", "k", "v", "g", "beta")}
     sub["initial_state"] = inp["initial_state"][[0, 31, 63]]
