@@ -954,14 +954,20 @@ cudaError_t bwd_segments(const BwdParams &p, bool bf16, int P, const BwdSegLayou
 
 size_t bwd_chunked_workspace_bytes(const BwdParams &p, bool bf16, int Dk, int Dv);
 cudaError_t launch_bwd_chunked(const BwdParams &p, void *workspace, cudaStream_t st);
+bool bwd_warp_supported(const BwdParams &p, bool bf16, int Dk, int Dv);
+size_t bwd_warp_workspace_bytes(const BwdParams &p, int Dv);
+cudaError_t launch_bwd_warp(const BwdParams &p, int Dv, void *workspace, cudaStream_t st);
 size_t bwd_workspace_bytes(bool varlen, long long T, int N, int H, int Dk, int Dv);
 
 // The workspace with which kda_chunk_bwd runs its fastest form: the chunked form
-// (kda_bwd_chunk.cu) where it applies, else the segments when they apply.
+// (kda_bwd_chunk.cu, d = 128) or the micro-chunk form (kda_bwd_warp.cu, d_k = 32) where
+// they apply, else the segments when they apply.
 size_t bwd_workspace_bytes(const BwdParams &p, bool bf16, int Dk, int Dv) {
     const bool varlen = p.cu_seqlens != nullptr;
     const size_t chunked = bwd_chunked_workspace_bytes(p, bf16, Dk, Dv);
     if (chunked) return std::max(chunked, bwd_workspace_bytes_min(varlen, p.T, p.N, p.H, Dk, Dv));
+    if (bwd_warp_supported(p, bf16, Dk, Dv))
+        return std::max(bwd_warp_workspace_bytes(p, Dv), bwd_workspace_bytes_min(varlen, p.T, p.N, p.H, Dk, Dv));
     return bwd_workspace_bytes(varlen, p.T, p.N, p.H, Dk, Dv);
 }
 
@@ -981,6 +987,9 @@ cudaError_t launch_bwd(BwdParams p, bool bf16, int Dk, int Dv, void *workspace, 
     const size_t chunked = bwd_chunked_workspace_bytes(p, bf16, Dk, Dv);
     if (chunked && workspace_bytes >= chunked && (reinterpret_cast<uintptr_t>(ws) & 255) == 0)
         return launch_bwd_chunked(p, ws, st);
+    if (bwd_warp_supported(p, bf16, Dk, Dv) && workspace_bytes >= bwd_warp_workspace_bytes(p, Dv) &&
+        (reinterpret_cast<uintptr_t>(ws) & 255) == 0)
+        return launch_bwd_warp(p, Dv, ws, st);
     const int P = bwd_seg_count(varlen, p.T, p.N, p.H, Dk, Dv);
     if (P >= 2 && (reinterpret_cast<uintptr_t>(ws) & 255) == 0) {
         const bool tc = bf16 && Dk == 128;

@@ -23,6 +23,7 @@
 #include "kda_stage.cuh"
 #include "kda_tc_util.cuh"
 #include "kda_sm100.cuh"
+#include "kda_warp_mma.cuh"
 
 namespace kda {
 namespace cw {
@@ -35,7 +36,6 @@ constexpr int LK = DK + 8;  // padded row of a [16][32] bf16 tile (elements): 80
 constexpr int LT = 24;      // padded row of a [16][16] bf16 tile: 48 B
 constexpr int LL = 17;      // row of the fp32 L tile
 constexpr int NWARP = 4;    // chains per CTA
-constexpr float kL2e = 1.4426950408889634f;
 constexpr float kSpan = 80.f;  // largest |G - G_mid| of the split products
 
 template <int DV>
@@ -66,55 +66,17 @@ struct Lay {
     static_assert(D + CW * LV * 2 <= KT && CW * LK * 2 <= TT && CW * 33 * 4 <= DK * LV * 2, "aliases");
 };
 
-// ---- warp-level MMA
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t (&r)[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-__device__ __forceinline__ void ldsm4t(uint32_t addr, uint32_t (&r)[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-// Fragment loads of a row-major bf16 tile with rows of `ld` elements at shared address
-// `base`. A (16 x 16 at (m0, k0)) from [M][K] storage, or from [K][M] storage (trans).
-__device__ __forceinline__ void frag_a(uint32_t base, int ld, int m0, int k0, int lane, uint32_t (&a)[4]) {
-    ldsm4(base + 2 * ((m0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ld + k0 + 8 * (lane >> 4)), a);
-}
-__device__ __forceinline__ void frag_at(uint32_t base, int ld, int m0, int k0, int lane, uint32_t (&a)[4]) {
-    ldsm4t(base + 2 * ((k0 + (lane & 7) + 8 * (lane >> 4)) * ld + m0 + 8 * ((lane >> 3) & 1)), a);
-}
-// B for two n-tiles (n0 .. n0 + 15) x k0 .. k0 + 15: from [N][K] storage, or [K][N] (trans).
-// b[0], b[1]: n-tile n0; b[2], b[3]: n-tile n0 + 8.
-__device__ __forceinline__ void frag_b(uint32_t base, int ld, int n0, int k0, int lane, uint32_t (&b)[4]) {
-    ldsm4(base + 2 * ((n0 + (lane & 7) + 8 * (lane >> 4)) * ld + k0 + 8 * ((lane >> 3) & 1)), b);
-}
-__device__ __forceinline__ void frag_bt(uint32_t base, int ld, int n0, int k0, int lane, uint32_t (&b)[4]) {
-    ldsm4t(base + 2 * ((k0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ld + n0 + 8 * (lane >> 4)), b);
-}
-// 16-byte cp.async that zero-fills the destination when `valid` is false (no bytes read;
-// the source address is still a valid one)
-__device__ __forceinline__ void cp16z(void *sdst, const void *gsrc, bool valid) {
-    const uint32_t d = sm100::smem_u32(sdst);
-    const int n = valid ? 16 : 0;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gsrc), "r"(n) : "memory");
-}
-__device__ __forceinline__ void stb2(uint8_t *p, float a, float b) {
-    *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(a, b);
-}
-__device__ __forceinline__ float e2(float x) { return ex2a(x * kL2e); }
 
 // AUG: the widened run of the segment form (kda_chunk_rec.cu): the state is [M | N]
 // (32 x DV, DV = 32 + d_v), the first 32 columns start from the identity and see v = 0,
 // the others start from zero and see v; the outputs [scale M^T q^ | scale N^T q^] go
 // out in fp32 as rows of DV and the final state as [32][DV].
+// save (or null): the state entering every micro-chunk, bf16 [32][DV], at
+// save + ((slot * H + h) * 32 + row) * DV with slot = bos / 16 + n + micro-chunk (distinct
+// across sequences: sequence n's slots end before bos_{n+1} / 16 + n + 1); read by the
+// micro-chunk backward.
 template <int DV, bool AUG>
-__global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const ChunkParams p) {
+__global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const ChunkParams p, __nv_bfloat16 *save) {
     using Ly = Lay<DV>;
     constexpr int LV = Ly::LV, NVT = DV / 8;
     constexpr int VOFF = AUG ? DK : 0, DVR = DV - VOFF;  // v's columns in the state, and its width
@@ -377,6 +339,12 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
                     stb2(sm + Ly::S + ((16 * mk + g8 + 8 * hi) * LV + 8 * j + 2 * t4) * 2, S[mk][j][2 * hi],
                          S[mk][j][2 * hi + 1]);
         __syncwarp();
+        if (save) {  // row `lane` of the entering state
+            const long long slot = (bos >> 4) + n + mc;
+            uint4 *dst = reinterpret_cast<uint4 *>(save + ((slot * H + h) * DK + lane) * DV);
+#pragma unroll
+            for (int q8 = 0; q8 < DV / 8; ++q8) dst[q8] = lds128(sm, Ly::S + (lane * LV + 8 * q8) * 2);
+        }
         // ---- D = U - W S (in U's registers) -> bf16 tile
 #pragma unroll
         for (int k0 = 0; k0 < DK; k0 += 16) {
@@ -481,7 +449,7 @@ __global__ void __launch_bounds__(NWARP * 32, 2) kda_chunk_warp_kernel(const Chu
 }
 
 template <int DV, bool AUG = false>
-cudaError_t launch_t(const ChunkParams &p, cudaStream_t st) {
+cudaError_t launch_t(const ChunkParams &p, cudaStream_t st, __nv_bfloat16 *save = nullptr) {
     const long long chains = (long long)p.N * p.H;
     if (chains <= 0) return cudaSuccess;
     const uint32_t smem = NWARP * Lay<DV>::BYTES;
@@ -489,7 +457,7 @@ cudaError_t launch_t(const ChunkParams &p, cudaStream_t st) {
                                          (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    kda_chunk_warp_kernel<DV, AUG><<<(unsigned)((chains + NWARP - 1) / NWARP), NWARP * 32, smem, st>>>(p);
+    kda_chunk_warp_kernel<DV, AUG><<<(unsigned)((chains + NWARP - 1) / NWARP), NWARP * 32, smem, st>>>(p, save);
     return cudaGetLastError();
 }
 
@@ -891,6 +859,11 @@ bool chunk_warp_supported(bool bf16, int Dk, int Dv) { return bf16 && (Dk == 32 
 cudaError_t launch_chunk_warp(const ChunkParams &p, int Dk, int Dv, cudaStream_t st) {
     if (Dk == 64) return Dv == 32 ? cw::w64::launch_t<32>(p, st) : cw::w64::launch_t<64>(p, st);
     return Dv == 32 ? cw::launch_t<32>(p, st) : cw::launch_t<64>(p, st);
+}
+
+// The d_k = 32 forward saving every micro-chunk's entering state for the backward.
+cudaError_t launch_chunk_warp_save(const ChunkParams &p, int Dv, __nv_bfloat16 *save, cudaStream_t st) {
+    return Dv == 32 ? cw::launch_t<32>(p, st, save) : cw::launch_t<64>(p, st, save);
 }
 
 // The widened run of the segment form for bf16 d_k = d_v = 32 (outputs fp32 rows of 64,
