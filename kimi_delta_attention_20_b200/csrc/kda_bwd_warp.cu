@@ -112,22 +112,18 @@ __global__ void __launch_bounds__(32) kda_bwd_warp_kernel(const BwdParams p, con
                 dS[mk][j][i] = p.dSf ? p.dSf[sbase + (long long)c * DV + v] : 0.f;
             }
 
-    for (int mc = nmc - 1; mc >= 0; --mc) {
+    // the inputs of micro-chunk mc, lane (row r = lane / 2, half hf): part 0 the v and dO rows
+    // and the saved state's row `lane` (last read by dV), part 1 the raw q, k, g rows (last
+    // read by the dq, dk outputs); each part is copied in for the next micro-chunk as soon as
+    // this one is done with it
+    auto issue = [&](int mc, int part) {
         const long long t0 = bos + (long long)mc * CW;
         const int L = (int)min((long long)CW, eos - t0);
-        // ---- inputs: lane (row r = lane / 2, half hf): raw q, k, g, v and dO rows; the
-        // saved state's row `lane`; lane r < 16 also token r's beta
-        {
-            const int r = lane >> 1, hf = lane & 1;
-            const bool ok = r < L;
-            const long long row = (t0 + (ok ? r : 0)) * H + h;
-            const uint32_t o = (r * DK + 16 * hf) * 2, ov = (r * LV + (DV / 2) * hf) * 2;
-#pragma unroll
-            for (int c2 = 0; c2 < 2; ++c2) {
-                cp16z(sm + Ly::Q + o + 16 * c2, qg + row * DK + 16 * hf + 8 * c2, ok);
-                cp16z(sm + Ly::K + o + 16 * c2, kg + row * DK + 16 * hf + 8 * c2, ok);
-                cp16z(sm + Ly::G + o + 16 * c2, gg + row * DK + 16 * hf + 8 * c2, ok);
-            }
+        const int r = lane >> 1, hf = lane & 1;
+        const bool ok = r < L;
+        const long long row = (t0 + (ok ? r : 0)) * H + h;
+        if (part == 0) {
+            const uint32_t ov = (r * LV + (DV / 2) * hf) * 2;
 #pragma unroll
             for (int c2 = 0; c2 < DV / 16; ++c2) {
                 cp16z(sm + Ly::V + ov + 16 * c2, vg + row * DV + (DV / 2) * hf + 8 * c2, ok);
@@ -137,8 +133,22 @@ __global__ void __launch_bounds__(32) kda_bwd_warp_kernel(const BwdParams p, con
             const __nv_bfloat16 *srow = save + ((slot * H + h) * DK + lane) * DV;
 #pragma unroll
             for (int c2 = 0; c2 < DV / 8; ++c2) cp16z(sm + Ly::S + (lane * LV + 8 * c2) * 2, srow + 8 * c2, true);
-            cp_async_commit();
+        } else {
+            const uint32_t o = (r * DK + 16 * hf) * 2;
+#pragma unroll
+            for (int c2 = 0; c2 < 2; ++c2) {
+                cp16z(sm + Ly::Q + o + 16 * c2, qg + row * DK + 16 * hf + 8 * c2, ok);
+                cp16z(sm + Ly::K + o + 16 * c2, kg + row * DK + 16 * hf + 8 * c2, ok);
+                cp16z(sm + Ly::G + o + 16 * c2, gg + row * DK + 16 * hf + 8 * c2, ok);
+            }
         }
+        cp_async_commit();
+    };
+    if (nmc > 0) { issue(nmc - 1, 0); issue(nmc - 1, 1); }
+
+    for (int mc = nmc - 1; mc >= 0; --mc) {
+        const long long t0 = bos + (long long)mc * CW;
+        const int L = (int)min((long long)CW, eos - t0);
         const float braw = lane < L ? __bfloat162float(betag[(t0 + lane) * H + h]) : 0.f;
         cp_async_wait_all();
         __syncwarp();
@@ -544,6 +554,8 @@ __global__ void __launch_bounds__(32) kda_bwd_warp_kernel(const BwdParams p, con
                 }
             }
         }
+        __syncwarp();  // v, dO and the saved state are read: the previous micro-chunk's come in
+        if (mc > 0) issue(mc - 1, 0);
         // dKtil = T'^T dW: dk^ += dKtil e^G, dG += dKtil Ktil
         prod32(acc, Ly::TP, LT, true, Ly::DW, LK, true, CW);
 #pragma unroll
@@ -557,32 +569,55 @@ __global__ void __launch_bounds__(32) kda_bwd_warp_kernel(const BwdParams p, con
                 dG_[e] += xa * k.x; dG_[e + 1] += xb * k.y;
             }
         __syncwarp();
-        // ---- the inverse's backward (lane n < 16 owns column n), fp32
+        // ---- the inverse's backward: db_s = sum_r dT'_rs T_rs (lane s < 16), then the two
+        // 16 x 16 x 16 products X1 = (dT' diag(b)) T^T and dM = -T^T X1 as tf32 warp MMAs
         if (lane < CW) {
-            const int cn = lane;
             float s = 0.f;
 #pragma unroll
-            for (int r = 0; r < CW; ++r) s = fmaf(DTP[r * LF + cn], TF[r * LF + cn], s);
-            dbs[cn] = s;  // db_s = sum_r dT'_rs T_rs
-            // X1[r][n] = sum_k dT'[r][k] b_k T[n][k]
-#pragma unroll 4
-            for (int r = 0; r < CW; ++r) {
-                float x = 0.f;
+            for (int r = 0; r < CW; ++r) s = fmaf(DTP[r * LF + lane], TF[r * LF + lane], s);
+            dbs[lane] = s;
+        }
+        {
+            float x1[2][4] = {};
 #pragma unroll
-                for (int k = 0; k < CW; ++k) x = fmaf(DTP[r * LF + k] * bb[k], TF[cn * LF + k], x);
-                X1[r * LF + cn] = x;
+            for (int k0 = 0; k0 < CW; k0 += 8) {
+                const uint32_t a[4] = {to_tf32(DTP[g8 * LF + k0 + t4] * bb[k0 + t4]),
+                                       to_tf32(DTP[(g8 + 8) * LF + k0 + t4] * bb[k0 + t4]),
+                                       to_tf32(DTP[g8 * LF + k0 + t4 + 4] * bb[k0 + t4 + 4]),
+                                       to_tf32(DTP[(g8 + 8) * LF + k0 + t4 + 4] * bb[k0 + t4 + 4])};
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const uint32_t b[2] = {to_tf32(TF[(8 * j + g8) * LF + k0 + t4]), to_tf32(TF[(8 * j + g8) * LF + k0 + t4 + 4])};
+                    mma_tf32_16x8x8(x1[j], a, b);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                X1[g8 * LF + 8 * j + 2 * t4] = x1[j][0];
+                X1[g8 * LF + 8 * j + 2 * t4 + 1] = x1[j][1];
+                X1[(g8 + 8) * LF + 8 * j + 2 * t4] = x1[j][2];
+                X1[(g8 + 8) * LF + 8 * j + 2 * t4 + 1] = x1[j][3];
             }
         }
         __syncwarp();
-        if (lane < CW) {
-            const int cn = lane;
-            // dM[m][n] = -sum_k T[k][m] X1[k][n]
-#pragma unroll 4
-            for (int m = 0; m < CW; ++m) {
-                float x = 0.f;
+        {
+            float dm[2][4] = {};
 #pragma unroll
-                for (int k = 0; k < CW; ++k) x = fmaf(TF[k * LF + m], X1[k * LF + cn], x);
-                DMf[m * LF + cn] = -x;
+            for (int k0 = 0; k0 < CW; k0 += 8) {
+                const uint32_t a[4] = {to_tf32(TF[(k0 + t4) * LF + g8]), to_tf32(TF[(k0 + t4) * LF + g8 + 8]),
+                                       to_tf32(TF[(k0 + t4 + 4) * LF + g8]), to_tf32(TF[(k0 + t4 + 4) * LF + g8 + 8])};
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const uint32_t b[2] = {to_tf32(X1[(k0 + t4) * LF + 8 * j + g8]), to_tf32(X1[(k0 + t4 + 4) * LF + 8 * j + g8])};
+                    mma_tf32_16x8x8(dm[j], a, b);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                DMf[g8 * LF + 8 * j + 2 * t4] = -dm[j][0];
+                DMf[g8 * LF + 8 * j + 2 * t4 + 1] = -dm[j][1];
+                DMf[(g8 + 8) * LF + 8 * j + 2 * t4] = -dm[j][2];
+                DMf[(g8 + 8) * LF + 8 * j + 2 * t4 + 1] = -dm[j][3];
             }
         }
         __syncwarp();
@@ -672,7 +707,8 @@ __global__ void __launch_bounds__(32) kda_bwd_warp_kernel(const BwdParams p, con
                     *reinterpret_cast<__nv_bfloat162 *>(dqg + o + 8 * j) = __floats2bfloat162_rn(qa, qb);
                 }
             }
-            __syncwarp();  // every read of G is done: dG in its place
+            __syncwarp();  // every read of G and of the raw rows is done: dG in its place
+            if (mc > 0) issue(mc - 1, 1);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
