@@ -11,7 +11,8 @@ fp32 state, bf16 token vectors, one fresh token per step) is timed in the
 same run, K' = 256 steps per timed pass, and reported under "decode"; so is the
 serving decode token (conv window 4 + SiLU, the recurrent step and the output
 gate fused, same geometry) under "decode_token", the chunk_kda backward on the
-B1 T8192 H16 d128 chunk workload under "backward", and the other chunk workloads
+B1 T8192 H16 d128 chunk workload under "backward" (and at the 300M layer's geometry under
+"backward_small"), and the other chunk workloads
 (twin B4 T2048 H8 d32 with states, B1 T8192 H16 d128 lb -5, one layer of the
 300M model: B128 T2048 H8 d_k 32 d_v 64 with the in-kernel gate) under
 "chunk_workloads", each timed launch by launch with L2 flushed in between.
@@ -118,6 +119,14 @@ def token_algorithmic(N, H, D, K):
 # chunk_kda backward: the B1 T8192 H16 d128 lb-5 chunk workload with an output and a
 # final-state cotangent (its 16 (sequence, head) chains run in segment form)
 BWD_WL = 2
+
+
+def bwd_small_workload(KI):
+    """The backward at the 300M layer's geometry (B128 T2048 H8, d_k 32, d_v 64) with the
+    log-decay gate and a lower bound of -5 (the autograd route takes the log gate): the
+    micro-chunk backward."""
+    return dataclasses.replace(KI.CHUNK_WORKLOADS[5], name="300M layer geometry B128 T2048 H8 dk32 dv64 lb-5",
+                               gate_in_kernel=False, beta_prob=False, lower_bound=-5.0, seed=55)
 
 
 def bwd_algorithmic(wl):
@@ -313,6 +322,7 @@ def run_kda(args, rank, world, local_rank):
                          g_out=tk["g_out"][i], lower_bound=-5.0, out=tk_o)
 
     bwl = KI.CHUNK_WORKLOADS[BWD_WL]
+    BWD_SMALL = bwd_small_workload(KI)
     if args.only == "bwd" and args.bwd_tokens:  # shorter sequence for profiler captures
         bwl = dataclasses.replace(bwl, T=args.bwd_tokens, name=f"{bwl.name} T{args.bwd_tokens}")
     if args.only in (None, "bwd"):
@@ -323,6 +333,16 @@ def run_kda(args, rank, world, local_rank):
         b_dSf = torch.randn(bwl.n_seqs, bwl.H, bwl.Dk, bwl.Dv, generator=bgen, device=dev) * 0.5
         b_ws = torch.empty(kda.chunk_bwd_workspace_bytes(bwl.B, bwl.T, bwl.H, bwl.Dk, bwl.Dv, N=bwl.n_seqs),
                            dtype=torch.uint8, device=dev)
+
+    if args.only is None:
+        sinp = KI.chunk_inputs(BWD_SMALL, device=dev)
+        sgen = torch.Generator(device=dev)
+        sgen.manual_seed(BWD_SMALL.seed + 1000)
+        s_do = torch.randn(sinp["v"].shape, generator=sgen, device=dev).to(BWD_SMALL.dtype)
+
+    def bwd_small_step():
+        return kda.chunk_kda_bwd(sinp["q"], sinp["k"], sinp["v"], sinp["g"], sinp["beta"], s_do,
+                                 use_qk_l2norm_in_kernel=True, lower_bound=BWD_SMALL.lower_bound)
 
     def bwd_step():
         return kda.chunk_kda_bwd(binp["q"], binp["k"], binp["v"], binp["g"], binp["beta"], b_do,
@@ -499,6 +519,18 @@ def run_kda(args, rank, world, local_rank):
         torch.cuda.synchronize(dev); barrier()
         bwd_launches = launches() - n0
         bwd_ms = max_over_ranks(b0.elapsed_time(b1)) / args.steps
+        # the small-head backward: K timed calls
+        for _ in range(args.warmup):
+            bwd_small_step()
+        barrier(); torch.cuda.synchronize(dev)
+        n0 = launches()
+        b0.record(stream)
+        for _ in range(args.steps):
+            bwd_small_step()
+        b1.record(stream)
+        torch.cuda.synchronize(dev); barrier()
+        bwd_small_launches = launches() - n0
+        bwd_small_ms = max_over_ranks(b0.elapsed_time(b1)) / args.steps
         # the smaller chunk workloads
         extra_legs, extra_launches = {}, 0
         for idx in EXTRA_CHUNK_WLS:
@@ -570,6 +602,9 @@ def run_kda(args, rank, world, local_rank):
     tok_bytes = token_algorithmic(TOKEN_WL["N"], TOKEN_WL["H"], TOKEN_WL["D"], TOKEN_WL["K"])
     tok_gbs = tok_bytes / (tok_ms * 1e-3) / 1e9
     bwd_flops, bwd_bytes = bwd_algorithmic(bwl)
+    # bytes of the small-head backward (no final-state cotangent, no initial state), all bf16:
+    # q, k, g, v, do, beta in; dq, dk, dg, dv, dbeta out
+    bwd_small_bytes = BWD_SMALL.tokens * BWD_SMALL.H * ((6 * BWD_SMALL.Dk + 3 * BWD_SMALL.Dv) * 2 + 2 * 2)
     chunk_sha = source_sha(*CHUNK_SOURCES)
     result = {
         "metric": METRIC,
@@ -628,14 +663,27 @@ def run_kda(args, rank, world, local_rank):
                          "hbm": {"algorithmic_bytes_per_launch": bwd_bytes,
                                  "achieved_gbs": bwd_bytes / (bwd_ms * 1e-3) / 1e9}},
         },
+        "backward_small": {
+            "value": whole_job_rate(world, BWD_SMALL.tokens, bwd_small_ms), "unit": "tokens/s",
+            "ms_per_step": bwd_small_ms, "steps_timed": args.steps,
+            "workload": "chunk_kda backward at the 300M layer's geometry: B128 T2048 H8, d_k 32, d_v 64, "
+                        "bf16, log-decay gate with lower_bound=-5, output cotangent",
+            "form": "micro-chunk: the d_k = 32 forward saving each 16-token micro-chunk's state, then one "
+                    "warp per (sequence, head) on warp-level MMAs",
+            "roofline": {"bound": "hbm", "achieved": bwd_small_bytes / (bwd_small_ms * 1e-3) / 1e9,
+                         "peak": hbm_peak, "unit": "GB/s",
+                         "frac": bwd_small_bytes / (bwd_small_ms * 1e-3) / 1e9 / hbm_peak,
+                         "peak_kind": peak_kind, "algorithmic_bytes_per_launch": bwd_small_bytes},
+        },
         "e2e": {"value": whole_job_rate(world, wl.tokens, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "pipelined": "copy-in, compute and copy-back of consecutive steps on three streams"},
         "chunk_workloads": extra_legs,
         "gpu_launches": chunk_launches + args.steps * (dec_graph_launches + tok_graph_launches)
-        + bwd_launches + extra_launches,
+        + bwd_launches + bwd_small_launches + extra_launches,
         "gpu_launches_by_leg": {"chunk": chunk_launches, "decode": args.steps * dec_graph_launches,
                                 "decode_token": args.steps * tok_graph_launches, "backward": bwd_launches,
+                                "backward_small": bwd_small_launches,
                                 "chunk_workloads": extra_launches,
                                 "counted_by": "libkda.so's own launch counter (kda_launch_count); graph "
                                               "replays count the kernels captured in the graph"},
