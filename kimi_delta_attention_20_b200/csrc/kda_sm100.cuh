@@ -110,6 +110,11 @@ __device__ __forceinline__ void tc_fence_after() {
 __device__ __forceinline__ void bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+// Arrive on barrier `id` without waiting (the producer side of a hand-off whose
+// consumer waits with bar_sync on the same id and count).
+__device__ __forceinline__ void bar_arrive(int id, int nthreads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 // The same barrier, returning whether `pred` holds in any participating thread.
 __device__ __forceinline__ bool bar_or(int id, int nthreads, bool pred) {
     uint32_t r;

@@ -30,6 +30,19 @@ __device__ __forceinline__ void ldsm4t(uint32_t addr, uint32_t (&r)[4]) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
 }
+// Four 8 x 8 bf16 matrices from the MMA accumulator layout (lane: row lane / 4, columns
+// 2 (lane % 4), + 1; register i = matrix i) to shared memory; lane l gives the address of
+// stored row l % 8 of matrix l / 8. The .trans form stores each matrix transposed.
+__device__ __forceinline__ void stsm4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r0), "r"(r1),
+                 "r"(r2), "r"(r3)
+                 : "memory");
+}
+__device__ __forceinline__ void stsm4t(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r0),
+                 "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
 // Fragment loads of a row-major bf16 tile with rows of `ld` elements at shared address
 // `base`. A (16 x 16 at (m0, k0)) from [M][K] storage, or from [K][M] storage (trans).
 __device__ __forceinline__ void frag_a(uint32_t base, int ld, int m0, int k0, int lane, uint32_t (&a)[4]) {

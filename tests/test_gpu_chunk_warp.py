@@ -102,3 +102,27 @@ def test_warp_many_chains(dk):
     sub = {n: inp[n][[0, 31, 63]] for n in ("q", "k", "v", "g", "beta")}
     sub["initial_state"] = inp["initial_state"][[0, 31, 63]]
     compare(sub, o[[0, 31, 63]], S[[0, 31, 63]], "many", lower_bound=-5.0)
+
+
+@pytest.mark.parametrize("B", [37, 38])
+def test_warp_forms_at_four_chains_per_sm(B):
+    """The two d_k = 32 forms on either side of their switch: 592 chains (four per SM) take
+    the producer/consumer form, 608 the split form; a sample of sequences on every head."""
+    inp = KI.draw_chunk(B, 48, 16, 32, 64, dtype=DT, seed=550 + B, init_state=True)
+    o, S = run(inp, use_qk_l2norm_in_kernel=True, lower_bound=-5.0)
+    pick = [0, B // 2, B - 1]
+    sub = {n: inp[n][pick] for n in ("q", "k", "v", "g", "beta")}
+    sub["initial_state"] = inp["initial_state"][pick]
+    compare(sub, o[pick], S[pick], f"B{B}", lower_bound=-5.0)
+
+
+def test_warp_widened_run_split_form():
+    """d_k = d_v = 32 with 296 chains of 256 tokens: the segment form cuts each sequence into
+    four segments, so its widened run has 1,184 segment chains and takes the split form's
+    widened variant (the [M | N] state, fp32 outputs); entering states cross every segment."""
+    inp = KI.draw_chunk(37, 256, 8, 32, 32, dtype=DT, seed=560, init_state=True)
+    o, S = run(inp, use_qk_l2norm_in_kernel=True)
+    pick = [0, 18, 36]
+    sub = {n: inp[n][pick] for n in ("q", "k", "v", "g", "beta")}
+    sub["initial_state"] = inp["initial_state"][pick]
+    compare(sub, o[pick], S[pick], "widened split")
