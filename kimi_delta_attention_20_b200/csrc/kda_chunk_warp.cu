@@ -438,10 +438,12 @@ cudaError_t launch_t(const ChunkParams &p, cudaStream_t st) {
 
 
 // ---- d_k = 32 on a pair of warps per chain (one 64-thread CTA): warp w owns the value
-// columns [VW w, VW w + VW) of the 32 x d_v state (registers) and rows [8 w, 8 w + 8) of
-// the gate values and of the transposed operand tiles; warp 0 forms A_kk and the inverse,
-// warp 1 A_qk, then its share of the state operand and of (q^ e^G) S while the inverse
-// runs. AUG: the widened run of the segment form (kda_chunk_rec.cu): the state is [M | N]
+// columns [VW w, VW w + VW) of the state, held transposed (S^T, registers) as in the
+// consumer of the pc form below, and rows [8 w, 8 w + 8) of the gate values and of the
+// transposed operand tiles (the warps exchange one running gate sum per channel); warp 0
+// forms A_kk and the inverse, warp 1 A_qk and then its (q^ e^G) S while the inverse runs.
+// S^T and D^T never pass through shared memory, and O^T leaves through transposing matrix
+// stores into this step's v stage (each warp its own columns). AUG: the widened run of the segment form (kda_chunk_rec.cu): the state is [M | N]
 // (32 x DV, DV = 32 + d_v; warp 0 owns M, warp 1 N), M starts from the identity and sees
 // v = 0, N starts from zero and sees v; the outputs [scale M^T q^ | scale N^T q^] go out
 // in fp32 rows of DV and the final state as [32][DV].
@@ -450,26 +452,24 @@ constexpr int LL2 = 20;  // row of the fp32 L tile: 80 B, so a row is read four 
 template <int DV>
 struct Lay {
     static constexpr int LV = DV + 8;
+    // two input stages: raw q, k, g [16][32] and v [16][LV] (v's stage then stages O)
     static constexpr uint32_t Q = 0, K = Q + CW * DK * 2, G = K + CW * DK * 2, V = G + CW * DK * 2;
     static constexpr uint32_t IN = (V + CW * LV * 2 + 127) / 128 * 128;
     static constexpr uint32_t TT = DK * LT * 2;
     static constexpr uint32_t X = 2 * IN, Y = X + TT, XQ = Y + TT, KT = XQ + TT, QT = KT + TT, KH = QT + TT;
-    static constexpr uint32_t W = X;  // -W [16][LK] over X^T
-    static constexpr uint32_t D = Y;  // D [16][LV] over Y^T and XQ^T
-    static constexpr uint32_t TP = KH + TT, AQ = TP + CW * LT * 2;
-    static constexpr uint32_t S = AQ + CW * LT * 2;  // S bf16 [32][LV]; exponent scratch [16][33] f32
-    static constexpr uint32_t GV = S + DK * LV * 2;  // gate values f32 [16][33]
-    static constexpr uint32_t L = GV + CW * 33 * 4;  // L = diag(b) A_kk, f32 [16][LL2]
-    static constexpr uint32_t RK = L + CW * LL2 * 4, RQ = RK + 64, BB = RQ + 64, GAM = BB + 64;
-    static constexpr uint32_t BYTES = (GAM + DK * 4 + 127) / 128 * 128;
-    static_assert(D + CW * LV * 2 <= KT && CW * LK * 2 <= TT && CW * 33 * 4 <= DK * LV * 2, "aliases");
-    static_assert(L % 16 == 0, "L rows are read 16 bytes at a time");
+    static constexpr uint32_t W = X;  // -W [16][LK] over X^T (after the A products)
+    static constexpr uint32_t TP = KH + TT, AQ = TP + CW * LT * 2;  // T'^T [16][LT], A_qk [16][LT]
+    static constexpr uint32_t L = AQ + CW * LT * 2;                  // L = diag(b) A_kk, f32 [16][LL2]
+    static constexpr uint32_t RK = L + CW * LL2 * 4, RQ = RK + 64, BB = RQ + 64, GAM = BB + 64, XG = GAM + DK * 4;
+    static constexpr uint32_t BYTES = (XG + 2 * DK * 4 + 127) / 128 * 128;
+    static_assert(CW * LK * 2 <= TT && CW * 33 * 4 <= 2 * TT, "aliases over X^T (and Y^T)");
+    static_assert(L % 16 == 0 && RK % 16 == 0 && RQ % 16 == 0, "rows read 16 bytes at a time");
 };
 
 template <int DV, bool AUG>
 __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams p) {
     using Ly = Lay<DV>;
-    constexpr int LV = Ly::LV, VW = DV / 2, NVT = VW / 8;
+    constexpr int LV = Ly::LV, VW = DV / 2, MT = VW / 16;  // own value columns and their m-tiles
     constexpr int VOFF = AUG ? DK : 0, DVR = DV - VOFF;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -479,8 +479,8 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
     const uint32_t sb = sm100::smem_u32(sm);
     float *rk = reinterpret_cast<float *>(sm + Ly::RK), *rq = reinterpret_cast<float *>(sm + Ly::RQ);
     float *bb = reinterpret_cast<float *>(sm + Ly::BB), *gam = reinterpret_cast<float *>(sm + Ly::GAM);
-    float *Lf = reinterpret_cast<float *>(sm + Ly::L), *GV = reinterpret_cast<float *>(sm + Ly::GV);
-    const int H = p.H, g8 = lane >> 2, t4 = lane & 3;
+    float *Lf = reinterpret_cast<float *>(sm + Ly::L), *XG = reinterpret_cast<float *>(sm + Ly::XG);
+    const int H = p.H, g8 = lane >> 2, t4 = lane & 3, mi = lane >> 3, mr = lane & 7;
     long long bos, eos;
     if (p.cu_seqlens) { bos = p.cu_seqlens[n]; eos = p.cu_seqlens[n + 1]; }
     else { bos = (long long)n * p.T; eos = bos + p.T; }
@@ -515,22 +515,30 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
         cp_async_commit();
     };
 
-    float S[2][NVT][4];  // rows 16 mk + g8 (+ 8), columns VW w + 8 j + 2 t4 (+ 1)
+    // S^T, own value columns: rows (values) VW w + 16 mt + g8 (+ 8), columns (keys) 8 nk + 2 t4 (+ 1)
+    float ST[MT][4][4];
     const long long sbase = ((long long)n * H + h) * DK * DV;
 #pragma unroll
-    for (int mk = 0; mk < 2; ++mk)
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int j = 0; j < NVT; ++j)
+        for (int nk = 0; nk < 4; ++nk)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int c = 16 * mk + g8 + 8 * (i >> 1), v = VW * w + 8 * j + 2 * t4 + (i & 1);
-                S[mk][j][i] = AUG ? (c == v ? 1.f : 0.f) : p.S0 ? p.S0[sbase + (long long)c * DV + v] : 0.f;
+                const int v = VW * w + 16 * mt + g8 + 8 * (i >> 1), c = 8 * nk + 2 * t4 + (i & 1);
+                ST[mt][nk][i] = AUG ? (c == v ? 1.f : 0.f) : p.S0 ? p.S0[sbase + (long long)c * DV + v] : 0.f;
             }
     if constexpr (AUG) {  // the identity block sees v = 0: its columns of both v tiles stay zero
         const uint32_t z = ((tid >> 2) * LV + 8 * (tid & 3)) * 2;
         sts128(sm, Ly::V + z, make_uint4(0u, 0u, 0u, 0u));
         sts128(sm, Ly::IN + Ly::V + z, make_uint4(0u, 0u, 0u, 0u));
     }
+    // A fragment of S^T (bf16) for own value m-tile mt and key step kk
+    auto sfrag = [&](int mt, int kk, uint32_t (&a)[4]) {
+        a[0] = pack_bf16x2(ST[mt][2 * kk][0], ST[mt][2 * kk][1]);
+        a[1] = pack_bf16x2(ST[mt][2 * kk][2], ST[mt][2 * kk][3]);
+        a[2] = pack_bf16x2(ST[mt][2 * kk + 1][0], ST[mt][2 * kk + 1][1]);
+        a[3] = pack_bf16x2(ST[mt][2 * kk + 1][2], ST[mt][2 * kk + 1][3]);
+    };
 
     if (nmc > 0) issue(0);
     for (int mc = 0; mc < nmc; ++mc) {
@@ -540,16 +548,21 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
         const uint32_t in = (mc & 1) * Ly::IN;
         cp_async_wait_all();
         __syncthreads();  // this micro-chunk's rows, from both warps' copies
-        // ---- gate values of rows 8 w .. 8 w + 7 for channel `lane`; row norms (thread pair
-        // per row: rows 0..15 of k, then of q; 16 channels each) and write strengths
+        // ---- gate values of rows 8 w .. 8 w + 7 for channel `lane` and their running sum
+        // (this warp's total to XG); row norms (thread pair per row: rows 0..15 of k, then
+        // of q; 16 channels each) and write strengths
+        float G8[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             const int r = 8 * w + u;
             const float x = __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::G)[r * DK + lane]);
             const float gv = p.gate_mode == kGateLog ? (p.has_lb ? fmaxf(x, p.lb) : x)
                                                      : gate_fast(x, bias, rate, p.gate_mode, p.lb);
-            GV[r * 33 + lane] = r < L ? gv : 0.f;
+            G8[u] = r < L ? gv : 0.f;
         }
+#pragma unroll
+        for (int u = 1; u < 8; ++u) G8[u] += G8[u - 1];
+        XG[w * DK + lane] = G8[7];
         {
             const int rr = tid >> 1, half = tid & 1, r = rr & 15;
             const uint32_t row = in + (rr < 16 ? Ly::K : Ly::Q) + r * DK * 2 + 32 * half;
@@ -567,28 +580,31 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
             if (tid < CW) bb[tid] = tid < L ? beta_value(bcur, p.beta_prob) : 0.f;
         }
         __syncthreads();
-        // ---- the cumsum of channel `lane` (all 16 rows); operand tiles, rows 8 w .. 8 w + 7
-        // of row `lane` of each transposed tile (one 16-byte store per tile)
-        float G[CW];
+        // ---- the in-chunk cumsum of channel `lane` on rows 8 w .. 8 w + 7 (warp 1 adds warp
+        // 0's total G_7); operand tiles, those rows of row `lane` of each transposed tile
+        const float Gm = XG[lane];
+        if (w) {
 #pragma unroll
-        for (int r = 0; r < CW; ++r) G[r] = GV[r * 33 + lane];
-#pragma unroll
-        for (int r = 1; r < CW; ++r) G[r] += G[r - 1];
-        const float Gm = G[7], GC = G[CW - 1];
+            for (int u = 0; u < 8; ++u) G8[u] += Gm;
+        }
+        const float GC = w ? G8[7] : Gm + XG[DK + lane];
         bool steep = false;
         {
             const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::K);
             const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::Q);
+            const float4 rka = *reinterpret_cast<const float4 *>(rk + 8 * w), rkb = *reinterpret_cast<const float4 *>(rk + 8 * w + 4);
+            const float4 rqa = *reinterpret_cast<const float4 *>(rq + 8 * w), rqb = *reinterpret_cast<const float4 *>(rq + 8 * w + 4);
+            const float rkv[8] = {rka.x, rka.y, rka.z, rka.w, rkb.x, rkb.y, rkb.z, rkb.w};
+            const float rqv[8] = {rqa.x, rqa.y, rqa.z, rqa.w, rqb.x, rqb.y, rqb.z, rqb.w};
             float x[8], y[8], xq[8], kt[8], qt[8], kc[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int r = 8 * w + u;
-                const float Gr = w ? G[8 + u] : G[u];
-                const float kh = __bfloat162float(kr[r * DK + lane]) * rk[r];
-                const float qh = __bfloat162float(qr[r * DK + lane]) * rq[r];
-                const float dm = Gr - Gm;
+                const float kh = __bfloat162float(kr[r * DK + lane]) * rkv[u];
+                const float qh = __bfloat162float(qr[r * DK + lane]) * rqv[u];
+                const float dm = G8[u] - Gm;
                 steep |= fabsf(dm) > kSpan;
-                const float em = e2(dm), en = e2(-dm), eg = e2(Gr), ec = e2(GC - Gr);
+                const float em = e2(dm), en = e2(-dm), eg = e2(G8[u]), ec = e2(GC - G8[u]);
                 x[u] = kh * em; y[u] = kh * en; xq[u] = qh * em;
                 kt[u] = kh * eg; qt[u] = qh * eg; kc[u] = kh * ec;
             }
@@ -603,8 +619,9 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
         }
         steep = __syncthreads_or(steep) != 0;
         // the next micro-chunk's rows into the other stage (last read before the previous
-        // micro-chunk's sixth barrier); issued here rather than at the top of the step,
-        // where they would queue ahead of this step's first shared-memory reads
+        // micro-chunk's sixth barrier, its O staging copied out before this one's first);
+        // issued here rather than at the top of the step, where they would queue ahead of
+        // this step's first shared-memory reads
         if (mc + 1 < nmc) issue(mc + 1);
         // ---- A_kk (warp 0) -> L = diag(b) A_kk (s < r); A_qk (warp 1) -> bf16 tile (s <= r)
         {
@@ -612,11 +629,11 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
             const uint32_t xa = w == 0 ? Ly::X : Ly::XQ;
 #pragma unroll
             for (int k0 = 0; k0 < DK; k0 += 16) {
-                uint32_t a[4], b[4];
+                uint32_t a[4], bf[4];
                 frag_at(sb + xa, LT, 0, k0, lane, a);
-                frag_bt(sb + Ly::Y, LT, 0, k0, lane, b);
-                mma16816(acc[0], a, b[0], b[1]);
-                mma16816(acc[1], a, b[2], b[3]);
+                frag_bt(sb + Ly::Y, LT, 0, k0, lane, bf);
+                mma16816(acc[0], a, bf[0], bf[1]);
+                mma16816(acc[1], a, bf[2], bf[3]);
             }
 #pragma unroll
             for (int j = 0; j < 2; ++j)
@@ -625,8 +642,8 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
                     const int r = g8 + 8 * hi, s_ = 8 * j + 2 * t4;
                     if (w == 0) {
                         const float br = bb[r];
-                        Lf[r * LL2 + s_] = s_ < r ? br * acc[j][2 * hi] : 0.f;
-                        Lf[r * LL2 + s_ + 1] = s_ + 1 < r ? br * acc[j][2 * hi + 1] : 0.f;
+                        *reinterpret_cast<float2 *>(Lf + r * LL2 + s_) = make_float2(
+                            s_ < r ? br * acc[j][2 * hi] : 0.f, s_ + 1 < r ? br * acc[j][2 * hi + 1] : 0.f);
                     } else {
                         stb2(sm + Ly::AQ + (r * LT + s_) * 2, s_ <= r ? acc[j][2 * hi] : 0.f,
                              s_ + 1 <= r ? acc[j][2 * hi + 1] : 0.f);
@@ -634,9 +651,10 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
                 }
         }
         if (steep) {  // exponent differences (never positive) on the CUDA cores
-            float *Gs = reinterpret_cast<float *>(sm + Ly::S);
+            __syncthreads();  // X^T and Y^T are read by both warps: the scratch goes over them
+            float *Gs = reinterpret_cast<float *>(sm + Ly::X);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) Gs[(8 * w + u) * 33 + lane] = w ? G[8 + u] : G[u];
+            for (int u = 0; u < 8; ++u) Gs[(8 * w + u) * 33 + lane] = G8[u];
             __syncthreads();
             const __nv_bfloat16 *kr = reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::K);
             const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::Q);
@@ -657,8 +675,8 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
             }
         }
         __syncthreads();
-        // ---- T = (I + L)^-1 by forward substitution (warp 0, lane j < 16: column j; the
-        // row of L four values at a time), T' = T diag(b)
+        // ---- T = (I + L)^-1 by forward substitution (warp 0, lane j < 16: column j, a row of
+        // L four values at a time); row j of T'^T = column j of T diag(b) (two 16-byte stores)
         if (w == 0 && lane < CW) {
             const int j = lane;
             float t[CW];
@@ -677,147 +695,148 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
             }
             const float bj = bb[j];
 #pragma unroll
-            for (int i = 0; i < CW; ++i)
-                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::TP)[i * LT + j] = __float2bfloat16_rn(t[i] * bj);
+            for (int i = 0; i < CW; ++i) t[i] *= bj;
+            sts128(sm, Ly::TP + (j * LT) * 2, pack8(t));
+            sts128(sm, Ly::TP + (j * LT + 8) * 2, pack8(t + 8));
         }
-        // ---- own columns of the entering state as a bf16 operand (warp 1 while the inverse
-        // runs), then (q^ e^G) S into O
-#pragma unroll
-        for (int mk = 0; mk < 2; ++mk)
-#pragma unroll
-            for (int j = 0; j < NVT; ++j)
-#pragma unroll
-                for (int hi = 0; hi < 2; ++hi)
-                    stb2(sm + Ly::S + ((16 * mk + g8 + 8 * hi) * LV + VW * w + 8 * j + 2 * t4) * 2, S[mk][j][2 * hi],
-                         S[mk][j][2 * hi + 1]);
-        __syncwarp();
-        float O[NVT][4];
-#pragma unroll
-        for (int j = 0; j < NVT; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
-#pragma unroll
-        for (int k0 = 0; k0 < DK; k0 += 16) {
-            uint32_t a[4];
-            frag_at(sb + Ly::QT, LT, 0, k0, lane, a);
-#pragma unroll
-            for (int j = 0; j < NVT; j += 2) {
-                uint32_t b[4];
-                frag_bt(sb + Ly::S, LV, VW * w + 8 * j, k0, lane, b);
-                mma16816(O[j], a, b[0], b[1]);
-                mma16816(O[j + 1], a, b[2], b[3]);
-            }
-        }
-        __syncthreads();  // T'
-        // ---- U = T' V (own columns, registers); -W = -T' Ktil for key channels
-        // [16 w, 16 w + 16) into the shared tile
-        float U[NVT][4];
+        // ---- O^T = S^T Qtil^T for own value columns (warp 1 while the inverse runs)
+        float OT[MT][2][4];
         {
-            uint32_t a[4];
-            frag_a(sb + Ly::TP, LT, 0, 0, lane, a);
+            uint32_t bq[2][4];
+            frag_bt(sb + Ly::QT, LT, 0, 0, lane, bq[0]);
+            frag_bt(sb + Ly::QT, LT, 0, 16, lane, bq[1]);
 #pragma unroll
-            for (int j = 0; j < NVT; j += 2) {
-                uint32_t b[4];
-                frag_bt(sb + in + Ly::V, LV, VW * w + 8 * j, 0, lane, b);
-                U[j][0] = U[j][1] = U[j][2] = U[j][3] = 0.f;
-                U[j + 1][0] = U[j + 1][1] = U[j + 1][2] = U[j + 1][3] = 0.f;
-                mma16816(U[j], a, b[0], b[1]);
-                mma16816(U[j + 1], a, b[2], b[3]);
-            }
-            float wv[2][4] = {};
-            uint32_t b[4];
-            frag_b(sb + Ly::KT, LT, 16 * w, 0, lane, b);
-            mma16816(wv[0], a, b[0], b[1]);
-            mma16816(wv[1], a, b[2], b[3]);
+            for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
-            for (int j = 0; j < 2; ++j)
+                for (int i = 0; i < 4; ++i) OT[mt][0][i] = OT[mt][1][i] = 0.f;
 #pragma unroll
-                for (int hi = 0; hi < 2; ++hi)
-                    stb2(sm + Ly::W + ((g8 + 8 * hi) * LK + 16 * w + 8 * j + 2 * t4) * 2, -wv[j][2 * hi],
-                         -wv[j][2 * hi + 1]);
-        }
-        __syncthreads();  // -W complete
-        // ---- D = U - W S (own columns) -> bf16 tile
-#pragma unroll
-        for (int k0 = 0; k0 < DK; k0 += 16) {
-            uint32_t a[4];
-            frag_a(sb + Ly::W, LK, 0, k0, lane, a);
-#pragma unroll
-            for (int j = 0; j < NVT; j += 2) {
-                uint32_t b[4];
-                frag_bt(sb + Ly::S, LV, VW * w + 8 * j, k0, lane, b);
-                mma16816(U[j], a, b[0], b[1]);
-                mma16816(U[j + 1], a, b[2], b[3]);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < NVT; ++j)
-#pragma unroll
-            for (int hi = 0; hi < 2; ++hi)
-                stb2(sm + Ly::D + ((g8 + 8 * hi) * LV + VW * w + 8 * j + 2 * t4) * 2, U[j][2 * hi], U[j][2 * hi + 1]);
-        __syncwarp();
-        // ---- O += A_qk D (own columns); rows < L to o
-        {
-            uint32_t a[4];
-            frag_a(sb + Ly::AQ, LT, 0, 0, lane, a);
-#pragma unroll
-            for (int j = 0; j < NVT; j += 2) {
-                uint32_t b[4];
-                frag_bt(sb + Ly::D, LV, VW * w + 8 * j, 0, lane, b);
-                mma16816(O[j], a, b[0], b[1]);
-                mma16816(O[j + 1], a, b[2], b[3]);
-            }
-        }
-        if (p.o) {
-            const float f = p.scale;
-#pragma unroll
-            for (int hi = 0; hi < 2; ++hi) {
-                const int r = g8 + 8 * hi;
-                if (r < L) {
-                    const long long ob = ((t0 + r) * H + h) * DV + VW * w + 2 * t4;
-#pragma unroll
-                    for (int j = 0; j < NVT; ++j) {
-                        if constexpr (AUG)
-                            *reinterpret_cast<float2 *>(static_cast<float *>(p.o) + ob + 8 * j) =
-                                make_float2(f * O[j][2 * hi], f * O[j][2 * hi + 1]);
-                        else
-                            *reinterpret_cast<__nv_bfloat162 *>(og + ob + 8 * j) =
-                                __floats2bfloat162_rn(f * O[j][2 * hi], f * O[j][2 * hi + 1]);
-                    }
+                for (int kk = 0; kk < 2; ++kk) {
+                    uint32_t a[4];
+                    sfrag(mt, kk, a);
+                    mma16816(OT[mt][0], a, bq[kk][0], bq[kk][1]);
+                    mma16816(OT[mt][1], a, bq[kk][2], bq[kk][3]);
                 }
             }
         }
-        // ---- S <- diag(e^{G_last}) S + Khat^T D (own columns)
+        __syncthreads();  // T'
+        // ---- U^T = V^T T'^T (own value columns); -W = -T' Ktil for key channels [16 w, 16 w + 16)
+        float UT[MT][2][4];
+        {
+            uint32_t bt[4];
+            frag_bt(sb + Ly::TP, LT, 0, 0, lane, bt);
 #pragma unroll
-        for (int mk = 0; mk < 2; ++mk) {
-            const float ga = gam[16 * mk + g8], gb = gam[16 * mk + g8 + 8];
+            for (int mt = 0; mt < MT; ++mt) {
+                uint32_t a[4];
+                frag_at(sb + in + Ly::V, LV, VW * w + 16 * mt, 0, lane, a);
 #pragma unroll
-            for (int j = 0; j < NVT; ++j) {
-                S[mk][j][0] *= ga; S[mk][j][1] *= ga;
-                S[mk][j][2] *= gb; S[mk][j][3] *= gb;
+                for (int i = 0; i < 4; ++i) UT[mt][0][i] = UT[mt][1][i] = 0.f;
+                mma16816(UT[mt][0], a, bt[0], bt[1]);
+                mma16816(UT[mt][1], a, bt[2], bt[3]);
             }
-            uint32_t a[4];
-            frag_a(sb + Ly::KH, LT, 16 * mk, 0, lane, a);
+            uint32_t a[4], bf[4];
+            frag_at(sb + Ly::TP, LT, 0, 0, lane, a);
+            frag_b(sb + Ly::KT, LT, 16 * w, 0, lane, bf);
+            float wv[2][4] = {};
+            mma16816(wv[0], a, bf[0], bf[1]);
+            mma16816(wv[1], a, bf[2], bf[3]);
+            // matrix mi: row half mi % 2, key n-tile 2 w + mi / 2
+            stsm4(sb + Ly::W + ((8 * (mi & 1) + mr) * LK + 16 * w + 8 * (mi >> 1)) * 2,
+                  pack_bf16x2(-wv[0][0], -wv[0][1]), pack_bf16x2(-wv[0][2], -wv[0][3]),
+                  pack_bf16x2(-wv[1][0], -wv[1][1]), pack_bf16x2(-wv[1][2], -wv[1][3]));
+        }
+        __syncthreads();  // -W complete
+        // ---- D^T = U^T + S^T (-W)^T (own value columns), as bf16 A fragments over the tokens
 #pragma unroll
-            for (int j = 0; j < NVT; j += 2) {
-                uint32_t b[4];
-                frag_bt(sb + Ly::D, LV, VW * w + 8 * j, 0, lane, b);
-                mma16816(S[mk][j], a, b[0], b[1]);
-                mma16816(S[mk][j + 1], a, b[2], b[3]);
+        for (int kk = 0; kk < 2; ++kk) {
+            uint32_t bw[4];
+            frag_b(sb + Ly::W, LK, 0, 16 * kk, lane, bw);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                uint32_t a[4];
+                sfrag(mt, kk, a);
+                mma16816(UT[mt][0], a, bw[0], bw[1]);
+                mma16816(UT[mt][1], a, bw[2], bw[3]);
+            }
+        }
+        uint32_t DA[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            DA[mt][0] = pack_bf16x2(UT[mt][0][0], UT[mt][0][1]);
+            DA[mt][1] = pack_bf16x2(UT[mt][0][2], UT[mt][0][3]);
+            DA[mt][2] = pack_bf16x2(UT[mt][1][0], UT[mt][1][1]);
+            DA[mt][3] = pack_bf16x2(UT[mt][1][2], UT[mt][1][3]);
+        }
+        // ---- O^T += D^T A_qk^T; out through the staging tile over this stage's own v columns
+        // (rows = tokens), or in fp32 rows of DV (AUG)
+        {
+            uint32_t baq[4];
+            frag_b(sb + Ly::AQ, LT, 0, 0, lane, baq);
+            const float f = p.scale;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                mma16816(OT[mt][0], DA[mt], baq[0], baq[1]);
+                mma16816(OT[mt][1], DA[mt], baq[2], baq[3]);
+                if constexpr (AUG) {
+                    if (p.o) {
+#pragma unroll
+                        for (int nr = 0; nr < 2; ++nr)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int r = 8 * nr + 2 * t4 + (i & 1), v = VW * w + 16 * mt + g8 + 8 * (i >> 1);
+                                if (r < L) static_cast<float *>(p.o)[((t0 + r) * H + h) * DV + v] = f * OT[mt][nr][i];
+                            }
+                    }
+                } else {  // matrix mi: token rows 8 (mi / 2) + mr, value columns VW w + 16 mt + 8 (mi % 2)
+                    stsm4t(sb + in + Ly::V + ((8 * (mi >> 1) + mr) * LV + VW * w + 16 * mt + 8 * (mi & 1)) * 2,
+                           pack_bf16x2(f * OT[mt][0][0], f * OT[mt][0][1]), pack_bf16x2(f * OT[mt][0][2], f * OT[mt][0][3]),
+                           pack_bf16x2(f * OT[mt][1][0], f * OT[mt][1][1]), pack_bf16x2(f * OT[mt][1][2], f * OT[mt][1][3]));
+                }
+            }
+        }
+        // ---- S^T <- S^T diag(e^{G_last}) + D^T Khat (own value columns)
+#pragma unroll
+        for (int nk = 0; nk < 4; ++nk) {
+            const float2 gk = *reinterpret_cast<const float2 *>(gam + 8 * nk + 2 * t4);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                ST[mt][nk][0] *= gk.x; ST[mt][nk][1] *= gk.y;
+                ST[mt][nk][2] *= gk.x; ST[mt][nk][3] *= gk.y;
+            }
+        }
+#pragma unroll
+        for (int nk = 0; nk < 4; nk += 2) {
+            uint32_t bk[4];
+            frag_b(sb + Ly::KH, LT, 8 * nk, 0, lane, bk);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                mma16816(ST[mt][nk], DA[mt], bk[0], bk[1]);
+                mma16816(ST[mt][nk + 1], DA[mt], bk[2], bk[3]);
+            }
+        }
+        if (!AUG && p.o) {  // rows < L of the staged O, own columns, 16 bytes per lane and step
+            __syncwarp();
+            constexpr int PR = VW / 8;
+#pragma unroll
+            for (int q = lane; q < CW * PR; q += 32) {
+                const int r = q / PR, c = q % PR;
+                if (r < L)
+                    *reinterpret_cast<uint4 *>(og + ((t0 + r) * H + h) * DV + VW * w + 8 * c) =
+                        lds128(sm, in + Ly::V + (r * LV + VW * w + 8 * c) * 2);
             }
         }
         // no barrier here: every shared tile the next micro-chunk writes before its third
-        // barrier was last read before this one's sixth
+        // barrier was last read before this one's sixth (the O staging is this warp's own)
     }
     cp_async_wait_all();
     if (p.S_out) {
 #pragma unroll
-        for (int mk = 0; mk < 2; ++mk)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int j = 0; j < NVT; ++j)
+            for (int nk = 0; nk < 4; ++nk)
 #pragma unroll
-                for (int hi = 0; hi < 2; ++hi) {
-                    const int c = 16 * mk + g8 + 8 * hi, v = VW * w + 8 * j + 2 * t4;
-                    *reinterpret_cast<float2 *>(p.S_out + sbase + (long long)c * DV + v) =
-                        make_float2(S[mk][j][2 * hi], S[mk][j][2 * hi + 1]);
+                for (int i = 0; i < 4; ++i) {
+                    const int v = VW * w + 16 * mt + g8 + 8 * (i >> 1), c = 8 * nk + 2 * t4 + (i & 1);
+                    p.S_out[sbase + (long long)c * DV + v] = ST[mt][nk][i];
                 }
     }
 }
@@ -1322,9 +1341,9 @@ bool chunk_warp_supported(bool bf16, int Dk, int Dv) { return bf16 && (Dk == 32 
 // four chains (latency per chain decides), the split form otherwise: with more chains, or
 // with an in-kernel gate form (16 gate evaluations per lane and micro-chunk on the
 // producer), the producer warp's serial key-side work would set the pace. B T2048 H8 d_k 32
-// d_v 64, 10 calls, L2 flushed: log gate 128 chains 0.25 against 0.31 ms, 512 chains 0.29
-// against 0.37 ms, 1,024 chains 0.57 against 0.53 ms; softplus gate 256 chains 0.34 against
-// 0.33 ms, 1,024 chains 0.75 against 0.53 ms.
+// d_v 64, 10 calls, L2 flushed: log gate 128 chains 0.25 against 0.29 ms, 512 chains 0.30
+// against 0.34 ms, 1,024 chains 0.57 against 0.47 ms; softplus gate 128 chains 0.35 against
+// 0.31 ms, 1,024 chains 0.75 against 0.48 ms.
 static bool pc_form(const ChunkParams &p) { return p.gate_mode == kGateLog && (long long)p.N * p.H <= 4LL * 148; }
 
 cudaError_t launch_chunk_warp(const ChunkParams &p, int Dk, int Dv, cudaStream_t st) {
