@@ -254,13 +254,25 @@ KDA_API kda_status kda_decode_token(const kda_token_args *args, void *stream);
  * pages give no backward formulas: these are the derivatives of the token
  * recurrence of page "atlas_core/kimi_k3/kda.rs" (through the L2 norm, the clamp
  * g <- max(g, lower_bound), whose gradient is zero where the bound is taken, and
- * the sigmoid of beta). A recompute of the forward stores the state every 16
- * tokens; a reverse sweep then reruns each 16-token stretch forward from its
- * checkpoint (keeping the decayed states in an L2-resident scratch) and walks it
- * back, each (sequence, head) split by value columns over a cluster of Dv/32
- * CTAs; CUDA cores, fp32. Validation as kda_chunk_fwd (q, k, v, g, dout and dq, dk, dv, dg
- * 16-byte aligned; beta and dbeta aligned to their element); g is the log-decay
- * (the in-kernel gate forms are not covered).
+ * the sigmoid of beta), taken in one of three forms, the first that applies:
+ *   - chunked, on tensor cores: bf16, Dk = Dv = 128, has_lower_bound with
+ *     lower_bound >= -5. The forward is rerun in its two-pass chunk form, saving
+ *     each 64-token chunk's entering state; the state cotangent is carried back
+ *     over the chunks with tcgen05 products (over the forward's segments when the
+ *     (sequence, head) pairs are few), and the chunk-local gradients are formed on
+ *     warp-level MMAs;
+ *   - micro-chunk: bf16, Dk = 32, Dv in {32, 64}, has_lower_bound with lower_bound
+ *     >= -10, at least 256 (sequence, head) pairs. The 16-token micro-chunk forward
+ *     saves each micro-chunk's entering state (bf16); then one warp per (sequence,
+ *     head) walks its micro-chunks from the last with the state cotangent in
+ *     registers, every product a warp-level MMA;
+ *   - otherwise the token recurrence: a recompute of the forward stores the state
+ *     every 16 tokens; a reverse sweep reruns each 16-token stretch forward from
+ *     its checkpoint and walks it back, each (sequence, head) split by value
+ *     columns over a cluster of Dv/32 CTAs; CUDA cores, fp32.
+ * Every form gives the same gradients up to rounding. Validation as kda_chunk_fwd
+ * (q, k, v, g, dout and dq, dk, dv, dg 16-byte aligned; beta and dbeta aligned to
+ * their element); g is the log-decay (the in-kernel gate forms are not covered).
  */
 typedef struct {
     kda_dtype dtype;            /* of q, k, v, g, beta, dout and dq, dk, dv, dg, dbeta */
@@ -285,15 +297,20 @@ typedef struct {
     size_t workspace_bytes;
 } kda_chunk_bwd_args;
 
-/* Bytes of workspace with which kda_chunk_bwd runs its fastest form: the state
+/* Bytes of workspace with which kda_chunk_bwd runs its fastest form for these
+ * shapes: for the chunked form, the forward's records and chunk table, a 96 KB
+ * record per 64-token chunk and head (the chunk's entering state, D and the
+ * cotangent chain's output) and, when the (sequence, head) pairs are few, three
+ * d x d fp32 maps per segment and head; for the
+ * micro-chunk form, the saved bf16 states (one d_k x d_v tile per 16 tokens and
+ * head, plus one slot per sequence); for the token recurrence, the state
  * checkpoints (one d_k x d_v fp32 state per 16 tokens per head), a scratch of 16
- * states per (sequence, head) and a small header; when there are few (sequence, head)
- * pairs of long sequences and d_k = d_v, also the buffers of the segment form (each
- * sequence cut into up to 16 segments that are swept side by side: per segment and
- * head a widened d_k x 2 d_v state and two d_k x d_v states, and the checkpoints and
- * scratch of the segments). A workspace of at least the plain form's size (the same
- * sum without the segment buffers) runs the plain form (same result up to rounding);
- * less returns KDA_ERR_WORKSPACE. Only shapes are read. */
+ * states per (sequence, head) and a small header, and, when there are few
+ * (sequence, head) pairs of long sequences and d_k = d_v, the buffers of its
+ * segment form. Each figure is at least the plain token form's. A smaller
+ * workspace (but at least the plain token form's, 256-byte aligned for the other
+ * forms) runs the next form that fits (same result up to rounding); less than the
+ * plain token form's returns KDA_ERR_WORKSPACE. Only shapes are read. */
 KDA_API kda_status kda_chunk_bwd_workspace_size(const kda_chunk_bwd_args *args, size_t *bytes);
 
 KDA_API kda_status kda_chunk_bwd(const kda_chunk_bwd_args *args, void *stream);

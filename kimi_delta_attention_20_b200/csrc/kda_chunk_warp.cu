@@ -22,9 +22,9 @@
 // time is set by per-chain latency while every chain is in flight):
 //   d_k = 32 by default: w2 -- the warps split the value columns and the rows of the
 //     key-side work, meeting at block barriers;
-//   d_k = 32 with the log-decay gate and up to four chains per SM (and every call that
-//     saves the states for the backward): pc -- a producer warp forms the key side of the
-//     next micro-chunk while a consumer warp runs the state chain of the current one;
+//   d_k = 32 with the log-decay gate and up to four chains per SM: pc -- a producer warp
+//     forms the key side of the next micro-chunk while a consumer warp runs the state chain
+//     of the current one;
 //   d_k = 64: w64 -- as w2, over 64 key channels.
 #include <algorithm>
 
@@ -443,7 +443,7 @@ cudaError_t launch_t(const ChunkParams &p, cudaStream_t st) {
 // transposed operand tiles (the warps exchange one running gate sum per channel); warp 0
 // forms A_kk and the inverse, warp 1 A_qk and then its (q^ e^G) S while the inverse runs.
 // S^T and D^T never pass through shared memory, and O^T leaves through transposing matrix
-// stores into this step's v stage (each warp its own columns). AUG: the widened run of the segment form (kda_chunk_rec.cu): the state is [M | N]
+// stores into this step's v stage (each warp its own columns); save as in the pc form. AUG: the widened run of the segment form (kda_chunk_rec.cu): the state is [M | N]
 // (32 x DV, DV = 32 + d_v; warp 0 owns M, warp 1 N), M starts from the identity and sees
 // v = 0, N starts from zero and sees v; the outputs [scale M^T q^ | scale N^T q^] go out
 // in fp32 rows of DV and the final state as [32][DV].
@@ -466,8 +466,8 @@ struct Lay {
     static_assert(L % 16 == 0 && RK % 16 == 0 && RQ % 16 == 0, "rows read 16 bytes at a time");
 };
 
-template <int DV, bool AUG>
-__global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams p) {
+template <int DV, bool AUG, bool SAVE>
+__global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams p, __nv_bfloat16 *save) {
     using Ly = Lay<DV>;
     constexpr int LV = Ly::LV, VW = DV / 2, MT = VW / 16;  // own value columns and their m-tiles
     constexpr int VOFF = AUG ? DK : 0, DVR = DV - VOFF;
@@ -733,6 +733,29 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
                 mma16816(UT[mt][0], a, bt[0], bt[1]);
                 mma16816(UT[mt][1], a, bt[2], bt[3]);
             }
+            if constexpr (SAVE) {  // own columns of the entering state S (bf16 [32][DV]), 16 key rows at a time
+                __syncwarp();  // own v columns are read: they stage the rows
+                const long long slot = (bos >> 4) + n + mc;
+#pragma unroll
+                for (int kh = 0; kh < 2; ++kh) {
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)  // matrix mi: key n-tile 2 kh + mi / 2, value half mi % 2
+                        stsm4t(sb + in + Ly::V + ((8 * (mi >> 1) + mr) * LV + VW * w + 16 * mt + 8 * (mi & 1)) * 2,
+                               pack_bf16x2(ST[mt][2 * kh][0], ST[mt][2 * kh][1]),
+                               pack_bf16x2(ST[mt][2 * kh][2], ST[mt][2 * kh][3]),
+                               pack_bf16x2(ST[mt][2 * kh + 1][0], ST[mt][2 * kh + 1][1]),
+                               pack_bf16x2(ST[mt][2 * kh + 1][2], ST[mt][2 * kh + 1][3]));
+                    __syncwarp();
+                    constexpr int PR = VW / 8;
+#pragma unroll
+                    for (int q = lane; q < CW * PR; q += 32) {
+                        const int r = q / PR, c = q % PR;
+                        *reinterpret_cast<uint4 *>(save + ((slot * H + h) * DK + 16 * kh + r) * DV + VW * w + 8 * c) =
+                            lds128(sm, in + Ly::V + (r * LV + VW * w + 8 * c) * 2);
+                    }
+                    __syncwarp();
+                }
+            }
             uint32_t a[4], bf[4];
             frag_at(sb + Ly::TP, LT, 0, 0, lane, a);
             frag_b(sb + Ly::KT, LT, 16 * w, 0, lane, bf);
@@ -841,16 +864,16 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
     }
 }
 
-template <int DV, bool AUG = false>
-cudaError_t launch_t(const ChunkParams &p, cudaStream_t st) {
+template <int DV, bool AUG = false, bool SAVE = false>
+cudaError_t launch_t(const ChunkParams &p, cudaStream_t st, __nv_bfloat16 *save = nullptr) {
     const long long chains = (long long)p.N * p.H;
     if (chains <= 0) return cudaSuccess;
     const uint32_t smem = Lay<DV>::BYTES;
-    cudaError_t e = cudaFuncSetAttribute(kda_chunk_pair_kernel<DV, AUG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(kda_chunk_pair_kernel<DV, AUG, SAVE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    kda_chunk_pair_kernel<DV, AUG><<<(unsigned)chains, 64, smem, st>>>(p);
+    kda_chunk_pair_kernel<DV, AUG, SAVE><<<(unsigned)chains, 64, smem, st>>>(p, save);
     return cudaGetLastError();
 }
 }  // namespace w2
@@ -1354,7 +1377,8 @@ cudaError_t launch_chunk_warp(const ChunkParams &p, int Dk, int Dv, cudaStream_t
 
 // The d_k = 32 forward saving every micro-chunk's entering state for the backward.
 cudaError_t launch_chunk_warp_save(const ChunkParams &p, int Dv, __nv_bfloat16 *save, cudaStream_t st) {
-    return Dv == 32 ? cw::pc::launch_t<32>(p, st, save) : cw::pc::launch_t<64>(p, st, save);
+    if (pc_form(p)) return Dv == 32 ? cw::pc::launch_t<32>(p, st, save) : cw::pc::launch_t<64>(p, st, save);
+    return Dv == 32 ? cw::w2::launch_t<32, false, true>(p, st, save) : cw::w2::launch_t<64, false, true>(p, st, save);
 }
 
 // The widened run of the segment form for bf16 d_k = d_v = 32 (outputs fp32 rows of 64,

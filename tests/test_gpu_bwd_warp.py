@@ -85,3 +85,11 @@ def test_warp_bwd_options(case):
         inp["g"] = torch.full_like(inp["g"], -10.0)
         kw["lower_bound"] = -10.0
     run_and_compare(inp, tag=case, **kw)
+
+
+@pytest.mark.parametrize("dv", [32, 64])
+def test_warp_bwd_many_chains(dv):
+    """600 chains (75 ragged sequences x 8 heads): more than four per SM, so the saving forward
+    is the split form (the entering states leave through its own transposing stores)."""
+    lens = tuple((7 * i) % 41 + (i % 3) for i in range(75))
+    run_and_compare(draw(dv, seed=640 + dv, lens=lens), tag=f"many d_v{dv}")
