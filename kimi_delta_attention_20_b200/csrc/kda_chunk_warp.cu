@@ -47,35 +47,38 @@ constexpr int LL = 17;      // row of the fp32 L tile
 constexpr float kSpan = 80.f;  // largest |G - G_mid| of the split products
 
 // ---- d_k = 64: one CTA of two warps per chain. Warp w owns the value columns
-// [VW w, VW w + VW) of the 64 x d_v state (VW = d_v / 2, registers) and the key channels
+// [VW w, VW w + VW) of the 64 x d_v state (VW = d_v / 2), held transposed (S^T) in
+// accumulator registers as in the d_k = 32 forms below, and the key channels
 // [32 w, 32 w + 32) of the gate and of the transposed operand tiles; the 16 x 16 blocks
-// are split between the warps (warp 0 A_kk and the inverse, warp 1 A_qk), and block
-// barriers separate the phases that read the other warp's half.
+// are split between the warps (warp 0 A_kk and the inverse, warp 1 A_qk and then its
+// (q^ e^G) S), and block barriers separate the phases that read the other warp's half.
+// O^T leaves through transposing matrix stores into this step's v stage.
 namespace w64 {
 constexpr int DK2 = 64;
 constexpr int LKR = DK2 + 8;  // padded raw row (elements): 144 B, conflict-free row reads
 constexpr int LW = DK2 + 8;   // the -W tile [16][LW]
+constexpr int LLW = 20;       // row of the fp32 L tile: 80 B, a row read four values at a time
 template <int DV>
 struct Lay {
     static constexpr int LV = DV + 8;
+    // two input stages: raw q, k, g [16][LKR] and v [16][LV] (v's stage then stages O)
     static constexpr uint32_t Q = 0, K = Q + CW * LKR * 2, G = K + CW * LKR * 2, V = G + CW * LKR * 2;
     static constexpr uint32_t IN = (V + CW * LV * 2 + 127) / 128 * 128;
-    static constexpr uint32_t TT = DK2 * LT * 2;             // a transposed tile [64][LT]
+    static constexpr uint32_t TT = DK2 * LT * 2;  // a transposed tile [64][LT]
     static constexpr uint32_t X = 2 * IN, Y = X + TT, XQ = Y + TT, KT = XQ + TT, QT = KT + TT, KH = QT + TT;
-    static constexpr uint32_t W = X;                          // -W [16][LW] over X^T
-    static constexpr uint32_t D = Y;                          // D [16][LV] over Y^T
-    static constexpr uint32_t TP = KH + TT, AQ = TP + CW * LT * 2;
-    static constexpr uint32_t S = AQ + CW * LT * 2;           // S bf16 [64][LV]; exponent scratch [16][65] f32
-    static constexpr uint32_t L = S + DK2 * LV * 2;
-    static constexpr uint32_t RK = L + CW * LL * 4, RQ = RK + 64, BB = RQ + 64, PART = BB + 64, GAM = PART + 256;
+    static constexpr uint32_t W = X;                                // -W [16][LW] over X^T
+    static constexpr uint32_t TP = KH + TT, AQ = TP + CW * LT * 2;  // T'^T [16][LT], A_qk [16][LT]
+    static constexpr uint32_t L = AQ + CW * LT * 2;                 // L = diag(b) A_kk, f32 [16][LLW]
+    static constexpr uint32_t RK = L + CW * LLW * 4, RQ = RK + 64, BB = RQ + 64, PART = BB + 64, GAM = PART + 256;
     static constexpr uint32_t BYTES = (GAM + DK2 * 4 + 127) / 128 * 128;
-    static_assert(CW * LW * 2 <= TT && CW * LV * 2 <= TT && CW * 65 * 4 <= DK2 * LV * 2, "aliases");
+    static_assert(CW * LW * 2 <= TT && CW * 65 * 4 <= 2 * TT, "aliases over X^T (and Y^T)");
+    static_assert(L % 16 == 0 && RK % 16 == 0 && RQ % 16 == 0, "rows read 16 bytes at a time");
 };
 
 template <int DV>
-__global__ void __launch_bounds__(64, 4) kda_chunk_warp64_kernel(const ChunkParams p) {
+__global__ void __launch_bounds__(64, 5) kda_chunk_warp64_kernel(const ChunkParams p) {
     using Ly = Lay<DV>;
-    constexpr int LV = Ly::LV, VW = DV / 2, NVT = VW / 8;
+    constexpr int LV = Ly::LV, VW = DV / 2, MT = VW / 16;  // own value columns and their m-tiles
     extern __shared__ __align__(16) uint8_t smem_raw[];
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const long long chain = blockIdx.x;
@@ -86,7 +89,8 @@ __global__ void __launch_bounds__(64, 4) kda_chunk_warp64_kernel(const ChunkPara
     float *bb = reinterpret_cast<float *>(sm + Ly::BB), *gam = reinterpret_cast<float *>(sm + Ly::GAM);
     float *part = reinterpret_cast<float *>(sm + Ly::PART);
     float *Lf = reinterpret_cast<float *>(sm + Ly::L);
-    const int H = p.H, g8 = lane >> 2, t4 = lane & 3, c = 32 * w + lane;  // this thread's key channel
+    const int H = p.H, g8 = lane >> 2, t4 = lane & 3, mi = lane >> 3, mr = lane & 7;
+    const int c = 32 * w + lane;  // this thread's key channel
     long long bos, eos;
     if (p.cu_seqlens) { bos = p.cu_seqlens[n]; eos = p.cu_seqlens[n + 1]; }
     else { bos = (long long)n * p.T; eos = bos + p.T; }
@@ -124,17 +128,25 @@ __global__ void __launch_bounds__(64, 4) kda_chunk_warp64_kernel(const ChunkPara
         cp_async_commit();
     };
 
-    float S[4][NVT][4];  // rows 16 mk + g8 (+ 8), columns VW w + 8 j + 2 t4 (+ 1)
+    // S^T, own value columns: rows (values) VW w + 16 mt + g8 (+ 8), columns (keys) 8 nk + 2 t4 (+ 1)
+    float ST[MT][8][4];
     const long long sbase = ((long long)n * H + h) * DK2 * DV;
 #pragma unroll
-    for (int mk = 0; mk < 4; ++mk)
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-        for (int j = 0; j < NVT; ++j)
+        for (int nk = 0; nk < 8; ++nk)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int cr = 16 * mk + g8 + 8 * (i >> 1), v = VW * w + 8 * j + 2 * t4 + (i & 1);
-                S[mk][j][i] = p.S0 ? p.S0[sbase + (long long)cr * DV + v] : 0.f;
+                const int v = VW * w + 16 * mt + g8 + 8 * (i >> 1), cr = 8 * nk + 2 * t4 + (i & 1);
+                ST[mt][nk][i] = p.S0 ? p.S0[sbase + (long long)cr * DV + v] : 0.f;
             }
+    // A fragment of S^T (bf16) for own value m-tile mt and key step kk
+    auto sfrag = [&](int mt, int kk, uint32_t (&a)[4]) {
+        a[0] = pack_bf16x2(ST[mt][2 * kk][0], ST[mt][2 * kk][1]);
+        a[1] = pack_bf16x2(ST[mt][2 * kk][2], ST[mt][2 * kk][3]);
+        a[2] = pack_bf16x2(ST[mt][2 * kk + 1][0], ST[mt][2 * kk + 1][1]);
+        a[3] = pack_bf16x2(ST[mt][2 * kk + 1][2], ST[mt][2 * kk + 1][3]);
+    };
 
     if (nmc > 0) issue(0);
     for (int mc = 0; mc < nmc; ++mc) {
@@ -142,13 +154,8 @@ __global__ void __launch_bounds__(64, 4) kda_chunk_warp64_kernel(const ChunkPara
         const int L = (int)min((long long)CW, eos - t0);
         const float bcur = braw;
         const uint32_t in = (mc & 1) * Ly::IN;
-        if (mc + 1 < nmc) {
-            issue(mc + 1);
-            cp_async_wait_group<1>();
-        } else {
-            cp_async_wait_all();
-        }
-        __syncthreads();
+        cp_async_wait_all();
+        __syncthreads();  // this micro-chunk's rows, from both warps' copies
         // gate and cumsum for channel c
         float G[CW];
 #pragma unroll
@@ -195,12 +202,18 @@ __global__ void __launch_bounds__(64, 4) kda_chunk_warp64_kernel(const ChunkPara
             const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(sm + in + Ly::Q);
 #pragma unroll
             for (int h8 = 0; h8 < 2; ++h8) {
+                const float4 rka = *reinterpret_cast<const float4 *>(rk + 8 * h8);
+                const float4 rkb = *reinterpret_cast<const float4 *>(rk + 8 * h8 + 4);
+                const float4 rqa = *reinterpret_cast<const float4 *>(rq + 8 * h8);
+                const float4 rqb = *reinterpret_cast<const float4 *>(rq + 8 * h8 + 4);
+                const float rkv[8] = {rka.x, rka.y, rka.z, rka.w, rkb.x, rkb.y, rkb.z, rkb.w};
+                const float rqv[8] = {rqa.x, rqa.y, rqa.z, rqa.w, rqb.x, rqb.y, rqb.z, rqb.w};
                 float x[8], y[8], xq[8], kt[8], qt[8], kc[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int r = 8 * h8 + u;
-                    const float kh = __bfloat162float(kr[r * LKR + c]) * rk[r];
-                    const float qh = __bfloat162float(qr[r * LKR + c]) * rq[r];
+                    const float kh = __bfloat162float(kr[r * LKR + c]) * rkv[u];
+                    const float qh = __bfloat162float(qr[r * LKR + c]) * rqv[u];
                     const float dm = G[r] - Gm;
                     steep |= fabsf(dm) > kSpan;
                     const float em = e2(dm), en = e2(-dm), eg = e2(G[r]), ec = e2(GC - G[r]);
@@ -218,17 +231,21 @@ __global__ void __launch_bounds__(64, 4) kda_chunk_warp64_kernel(const ChunkPara
             gam[c] = e2(GC);
         }
         steep = __syncthreads_or(steep) != 0;
+        // the next micro-chunk's rows into the other stage (read, and its O staging copied
+        // out, in the previous micro-chunk, which both warps finished before this one's
+        // first barrier)
+        if (mc + 1 < nmc) issue(mc + 1);
         // A_kk (warp 0) -> L = diag(b) A_kk; A_qk (warp 1) -> bf16 tile
         {
             float acc[2][4] = {};
             const uint32_t xa = w == 0 ? Ly::X : Ly::XQ;
 #pragma unroll
             for (int k0 = 0; k0 < DK2; k0 += 16) {
-                uint32_t a[4], b[4];
+                uint32_t a[4], bf[4];
                 frag_at(sb + xa, LT, 0, k0, lane, a);
-                frag_bt(sb + Ly::Y, LT, 0, k0, lane, b);
-                mma16816(acc[0], a, b[0], b[1]);
-                mma16816(acc[1], a, b[2], b[3]);
+                frag_bt(sb + Ly::Y, LT, 0, k0, lane, bf);
+                mma16816(acc[0], a, bf[0], bf[1]);
+                mma16816(acc[1], a, bf[2], bf[3]);
             }
 #pragma unroll
             for (int j = 0; j < 2; ++j)
@@ -237,8 +254,8 @@ __global__ void __launch_bounds__(64, 4) kda_chunk_warp64_kernel(const ChunkPara
                     const int r = g8 + 8 * hi, s_ = 8 * j + 2 * t4;
                     if (w == 0) {
                         const float br = bb[r];
-                        Lf[r * LL + s_] = s_ < r ? br * acc[j][2 * hi] : 0.f;
-                        Lf[r * LL + s_ + 1] = s_ + 1 < r ? br * acc[j][2 * hi + 1] : 0.f;
+                        *reinterpret_cast<float2 *>(Lf + r * LLW + s_) = make_float2(
+                            s_ < r ? br * acc[j][2 * hi] : 0.f, s_ + 1 < r ? br * acc[j][2 * hi + 1] : 0.f);
                     } else {
                         stb2(sm + Ly::AQ + (r * LT + s_) * 2, s_ <= r ? acc[j][2 * hi] : 0.f,
                              s_ + 1 <= r ? acc[j][2 * hi + 1] : 0.f);
@@ -246,7 +263,8 @@ __global__ void __launch_bounds__(64, 4) kda_chunk_warp64_kernel(const ChunkPara
                 }
         }
         if (steep) {  // exponent differences (never positive) on the CUDA cores
-            float *Gs = reinterpret_cast<float *>(sm + Ly::S);
+            __syncthreads();  // X^T and Y^T are read by both warps: the scratch goes over them
+            float *Gs = reinterpret_cast<float *>(sm + Ly::X);
 #pragma unroll
             for (int r = 0; r < CW; ++r) Gs[r * 65 + c] = G[r];
             __syncthreads();
@@ -264,12 +282,13 @@ __global__ void __launch_bounds__(64, 4) kda_chunk_warp64_kernel(const ChunkPara
                 }
                 akk *= rk[r] * rk[s_];
                 aqk *= rq[r] * rk[s_];
-                if (s_ < r) Lf[r * LL + s_] = bb[r] * akk;
+                if (s_ < r) Lf[r * LLW + s_] = bb[r] * akk;
                 reinterpret_cast<__nv_bfloat16 *>(sm + Ly::AQ)[r * LT + s_] = __float2bfloat16_rn(aqk);
             }
         }
         __syncthreads();
-        // T' by forward substitution (warp 0, lane j < 16: column j)
+        // T' by forward substitution (warp 0, lane j < 16: column j, a row of L four values at
+        // a time); row j of T'^T = column j of T diag(b) (two 16-byte stores)
         if (w == 0 && lane < CW) {
             const int j = lane;
             float t[CW];
@@ -277,147 +296,151 @@ __global__ void __launch_bounds__(64, 4) kda_chunk_warp64_kernel(const ChunkPara
             for (int i = 0; i < CW; ++i) {
                 float acc = i == j ? 1.f : 0.f;
 #pragma unroll
-                for (int k = 0; k < i; ++k) acc = fmaf(-Lf[i * LL + k], t[k], acc);
+                for (int k4 = 0; k4 < i; k4 += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4 *>(Lf + i * LLW + k4);
+                    acc = fmaf(-l4.x, t[k4], acc);
+                    if (k4 + 1 < i) acc = fmaf(-l4.y, t[k4 + 1], acc);
+                    if (k4 + 2 < i) acc = fmaf(-l4.z, t[k4 + 2], acc);
+                    if (k4 + 3 < i) acc = fmaf(-l4.w, t[k4 + 3], acc);
+                }
                 t[i] = acc;
             }
             const float bj = bb[j];
 #pragma unroll
-            for (int i = 0; i < CW; ++i)
-                reinterpret_cast<__nv_bfloat16 *>(sm + Ly::TP)[i * LT + j] = __float2bfloat16_rn(t[i] * bj);
+            for (int i = 0; i < CW; ++i) t[i] *= bj;
+            sts128(sm, Ly::TP + (j * LT) * 2, pack8(t));
+            sts128(sm, Ly::TP + (j * LT + 8) * 2, pack8(t + 8));
         }
-        __syncthreads();
-        // U (own value columns, registers); -W for own key channels into the shared tile
-        float U[NVT][4];
+        // O^T = S^T Qtil^T for own value columns (warp 1 while the inverse runs)
+        float OT[MT][2][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) OT[mt][0][i] = OT[mt][1][i] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t bq[4];
+            frag_bt(sb + Ly::QT, LT, 0, 16 * kk, lane, bq);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                uint32_t a[4];
+                sfrag(mt, kk, a);
+                mma16816(OT[mt][0], a, bq[0], bq[1]);
+                mma16816(OT[mt][1], a, bq[2], bq[3]);
+            }
+        }
+        __syncthreads();  // T'
+        // U^T = V^T T'^T (own value columns); -W = -T' Ktil for key channels [32 w, 32 w + 32)
+        float UT[MT][2][4];
         {
+            uint32_t bt[4];
+            frag_bt(sb + Ly::TP, LT, 0, 0, lane, bt);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                uint32_t a[4];
+                frag_at(sb + in + Ly::V, LV, VW * w + 16 * mt, 0, lane, a);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) UT[mt][0][i] = UT[mt][1][i] = 0.f;
+                mma16816(UT[mt][0], a, bt[0], bt[1]);
+                mma16816(UT[mt][1], a, bt[2], bt[3]);
+            }
             uint32_t a[4];
-            frag_a(sb + Ly::TP, LT, 0, 0, lane, a);
+            frag_at(sb + Ly::TP, LT, 0, 0, lane, a);
 #pragma unroll
-            for (int j = 0; j < NVT; j += 2) {
-                uint32_t b[4];
-                frag_bt(sb + in + Ly::V, LV, VW * w + 8 * j, 0, lane, b);
-                U[j][0] = U[j][1] = U[j][2] = U[j][3] = 0.f;
-                U[j + 1][0] = U[j + 1][1] = U[j + 1][2] = U[j + 1][3] = 0.f;
-                mma16816(U[j], a, b[0], b[1]);
-                mma16816(U[j + 1], a, b[2], b[3]);
+            for (int jb = 0; jb < 4; jb += 2) {
+                uint32_t bf[4];
+                frag_b(sb + Ly::KT, LT, 32 * w + 8 * jb, 0, lane, bf);
+                float wv[2][4] = {};
+                mma16816(wv[0], a, bf[0], bf[1]);
+                mma16816(wv[1], a, bf[2], bf[3]);
+                // matrix mi: row half mi % 2, key n-tile 4 w + jb + mi / 2
+                stsm4(sb + Ly::W + ((8 * (mi & 1) + mr) * LW + 32 * w + 8 * (jb + (mi >> 1))) * 2,
+                      pack_bf16x2(-wv[0][0], -wv[0][1]), pack_bf16x2(-wv[0][2], -wv[0][3]),
+                      pack_bf16x2(-wv[1][0], -wv[1][1]), pack_bf16x2(-wv[1][2], -wv[1][3]));
             }
-            float wv[4][4] = {};
-#pragma unroll
-            for (int j = 0; j < 4; j += 2) {
-                uint32_t b[4];
-                frag_b(sb + Ly::KT, LT, 32 * w + 8 * j, 0, lane, b);
-                mma16816(wv[j], a, b[0], b[1]);
-                mma16816(wv[j + 1], a, b[2], b[3]);
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int hi = 0; hi < 2; ++hi)
-                    stb2(sm + Ly::W + ((g8 + 8 * hi) * LW + 32 * w + 8 * j + 2 * t4) * 2, -wv[j][2 * hi],
-                         -wv[j][2 * hi + 1]);
         }
-        // own columns of the state as a bf16 operand
-#pragma unroll
-        for (int mk = 0; mk < 4; ++mk)
-#pragma unroll
-            for (int j = 0; j < NVT; ++j)
-#pragma unroll
-                for (int hi = 0; hi < 2; ++hi)
-                    stb2(sm + Ly::S + ((16 * mk + g8 + 8 * hi) * LV + VW * w + 8 * j + 2 * t4) * 2, S[mk][j][2 * hi],
-                         S[mk][j][2 * hi + 1]);
         __syncthreads();  // -W complete
-        // D = U - W S (own columns) -> bf16 tile
+        // D^T = U^T + S^T (-W)^T (own value columns), as bf16 A fragments over the tokens
 #pragma unroll
-        for (int k0 = 0; k0 < DK2; k0 += 16) {
-            uint32_t a[4];
-            frag_a(sb + Ly::W, LW, 0, k0, lane, a);
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t bw[4];
+            frag_b(sb + Ly::W, LW, 0, 16 * kk, lane, bw);
 #pragma unroll
-            for (int j = 0; j < NVT; j += 2) {
-                uint32_t b[4];
-                frag_bt(sb + Ly::S, LV, VW * w + 8 * j, k0, lane, b);
-                mma16816(U[j], a, b[0], b[1]);
-                mma16816(U[j + 1], a, b[2], b[3]);
+            for (int mt = 0; mt < MT; ++mt) {
+                uint32_t a[4];
+                sfrag(mt, kk, a);
+                mma16816(UT[mt][0], a, bw[0], bw[1]);
+                mma16816(UT[mt][1], a, bw[2], bw[3]);
             }
         }
+        uint32_t DA[MT][4];
 #pragma unroll
-        for (int j = 0; j < NVT; ++j)
-#pragma unroll
-            for (int hi = 0; hi < 2; ++hi)
-                stb2(sm + Ly::D + ((g8 + 8 * hi) * LV + VW * w + 8 * j + 2 * t4) * 2, U[j][2 * hi], U[j][2 * hi + 1]);
-        __syncwarp();
-        // O = scale (Qtil S + A_qk D), own columns
+        for (int mt = 0; mt < MT; ++mt) {
+            DA[mt][0] = pack_bf16x2(UT[mt][0][0], UT[mt][0][1]);
+            DA[mt][1] = pack_bf16x2(UT[mt][0][2], UT[mt][0][3]);
+            DA[mt][2] = pack_bf16x2(UT[mt][1][0], UT[mt][1][1]);
+            DA[mt][3] = pack_bf16x2(UT[mt][1][2], UT[mt][1][3]);
+        }
+        // O^T += D^T A_qk^T; out through the staging tile over this stage's own v columns
         {
-            float O[NVT][4];
+            uint32_t baq[4];
+            frag_b(sb + Ly::AQ, LT, 0, 0, lane, baq);
+            const float f = p.scale;
 #pragma unroll
-            for (int j = 0; j < NVT; ++j) O[j][0] = O[j][1] = O[j][2] = O[j][3] = 0.f;
-#pragma unroll
-            for (int k0 = 0; k0 < DK2; k0 += 16) {
-                uint32_t a[4];
-                frag_at(sb + Ly::QT, LT, 0, k0, lane, a);
-#pragma unroll
-                for (int j = 0; j < NVT; j += 2) {
-                    uint32_t b[4];
-                    frag_bt(sb + Ly::S, LV, VW * w + 8 * j, k0, lane, b);
-                    mma16816(O[j], a, b[0], b[1]);
-                    mma16816(O[j + 1], a, b[2], b[3]);
-                }
-            }
-            {
-                uint32_t a[4];
-                frag_a(sb + Ly::AQ, LT, 0, 0, lane, a);
-#pragma unroll
-                for (int j = 0; j < NVT; j += 2) {
-                    uint32_t b[4];
-                    frag_bt(sb + Ly::D, LV, VW * w + 8 * j, 0, lane, b);
-                    mma16816(O[j], a, b[0], b[1]);
-                    mma16816(O[j + 1], a, b[2], b[3]);
-                }
-            }
-            if (og) {
-#pragma unroll
-                for (int hi = 0; hi < 2; ++hi) {
-                    const int r = g8 + 8 * hi;
-                    if (r < L) {
-                        __nv_bfloat16 *orow = og + ((t0 + r) * H + h) * DV + VW * w + 2 * t4;
-#pragma unroll
-                        for (int j = 0; j < NVT; ++j)
-                            *reinterpret_cast<__nv_bfloat162 *>(orow + 8 * j) =
-                                __floats2bfloat162_rn(p.scale * O[j][2 * hi], p.scale * O[j][2 * hi + 1]);
-                    }
-                }
+            for (int mt = 0; mt < MT; ++mt) {
+                mma16816(OT[mt][0], DA[mt], baq[0], baq[1]);
+                mma16816(OT[mt][1], DA[mt], baq[2], baq[3]);
+                // matrix mi: token rows 8 (mi / 2) + mr, value columns VW w + 16 mt + 8 (mi % 2)
+                stsm4t(sb + in + Ly::V + ((8 * (mi >> 1) + mr) * LV + VW * w + 16 * mt + 8 * (mi & 1)) * 2,
+                       pack_bf16x2(f * OT[mt][0][0], f * OT[mt][0][1]), pack_bf16x2(f * OT[mt][0][2], f * OT[mt][0][3]),
+                       pack_bf16x2(f * OT[mt][1][0], f * OT[mt][1][1]), pack_bf16x2(f * OT[mt][1][2], f * OT[mt][1][3]));
             }
         }
-        // S <- diag(e^{G_last}) S + Khat^T D (own columns)
+        // S^T <- S^T diag(e^{G_last}) + D^T Khat (own value columns)
 #pragma unroll
-        for (int mk = 0; mk < 4; ++mk) {
-            const float ga = gam[16 * mk + g8], gb = gam[16 * mk + g8 + 8];
+        for (int nk = 0; nk < 8; ++nk) {
+            const float2 gk = *reinterpret_cast<const float2 *>(gam + 8 * nk + 2 * t4);
 #pragma unroll
-            for (int j = 0; j < NVT; ++j) {
-                S[mk][j][0] *= ga; S[mk][j][1] *= ga;
-                S[mk][j][2] *= gb; S[mk][j][3] *= gb;
-            }
-            uint32_t a[4];
-            frag_a(sb + Ly::KH, LT, 16 * mk, 0, lane, a);
-#pragma unroll
-            for (int j = 0; j < NVT; j += 2) {
-                uint32_t b[4];
-                frag_bt(sb + Ly::D, LV, VW * w + 8 * j, 0, lane, b);
-                mma16816(S[mk][j], a, b[0], b[1]);
-                mma16816(S[mk][j + 1], a, b[2], b[3]);
+            for (int mt = 0; mt < MT; ++mt) {
+                ST[mt][nk][0] *= gk.x; ST[mt][nk][1] *= gk.y;
+                ST[mt][nk][2] *= gk.x; ST[mt][nk][3] *= gk.y;
             }
         }
-        __syncthreads();  // every tile of this micro-chunk is read
+#pragma unroll
+        for (int nk = 0; nk < 8; nk += 2) {
+            uint32_t bk[4];
+            frag_b(sb + Ly::KH, LT, 8 * nk, 0, lane, bk);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                mma16816(ST[mt][nk], DA[mt], bk[0], bk[1]);
+                mma16816(ST[mt][nk + 1], DA[mt], bk[2], bk[3]);
+            }
+        }
+        if (og) {  // rows < L of the staged O, own columns, 16 bytes per lane and step
+            __syncwarp();
+            constexpr int PR = VW / 8;
+#pragma unroll
+            for (int q = lane; q < CW * PR; q += 32) {
+                const int r = q / PR, cq = q % PR;
+                if (r < L)
+                    *reinterpret_cast<uint4 *>(og + ((t0 + r) * H + h) * DV + VW * w + 8 * cq) =
+                        lds128(sm, in + Ly::V + (r * LV + VW * w + 8 * cq) * 2);
+            }
+        }
+        // no barrier here: the next micro-chunk writes shared tiles only after its first
+        // barrier, which both warps reach only when done with this one (the O staging is
+        // this warp's own columns)
     }
     cp_async_wait_all();
     if (p.S_out) {
 #pragma unroll
-        for (int mk = 0; mk < 4; ++mk)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int j = 0; j < NVT; ++j)
+            for (int nk = 0; nk < 8; ++nk)
 #pragma unroll
-                for (int hi = 0; hi < 2; ++hi) {
-                    const int cr = 16 * mk + g8 + 8 * hi, v = VW * w + 8 * j + 2 * t4;
-                    *reinterpret_cast<float2 *>(p.S_out + sbase + (long long)cr * DV + v) =
-                        make_float2(S[mk][j][2 * hi], S[mk][j][2 * hi + 1]);
+                for (int i = 0; i < 4; ++i) {
+                    const int v = VW * w + 16 * mt + g8 + 8 * (i >> 1), cr = 8 * nk + 2 * t4 + (i & 1);
+                    p.S_out[sbase + (long long)cr * DV + v] = ST[mt][nk][i];
                 }
     }
 }
