@@ -43,7 +43,7 @@ constexpr int CW = 16;      // tokens per micro-chunk
 constexpr int DK = 32;      // key dim (lane = key channel)
 constexpr int LK = DK + 8;  // padded row of a [16][32] bf16 tile (elements): 80 B, conflict-free fragments
 constexpr int LT = 24;      // padded row of a [16][16] bf16 tile: 48 B
-constexpr int LL = 17;      // row of the fp32 L tile
+constexpr int LL = 20;      // row of the fp32 L tile: 80 B, so a row is read four values at a time
 constexpr float kSpan = 80.f;  // largest |G - G_mid| of the split products
 
 // ---- d_k = 64: one CTA of two warps per chain. Warp w owns the value columns
@@ -57,7 +57,6 @@ namespace w64 {
 constexpr int DK2 = 64;
 constexpr int LKR = DK2 + 8;  // padded raw row (elements): 144 B, conflict-free row reads
 constexpr int LW = DK2 + 8;   // the -W tile [16][LW]
-constexpr int LLW = 20;       // row of the fp32 L tile: 80 B, a row read four values at a time
 template <int DV>
 struct Lay {
     static constexpr int LV = DV + 8;
@@ -68,8 +67,8 @@ struct Lay {
     static constexpr uint32_t X = 2 * IN, Y = X + TT, XQ = Y + TT, KT = XQ + TT, QT = KT + TT, KH = QT + TT;
     static constexpr uint32_t W = X;                                // -W [16][LW] over X^T
     static constexpr uint32_t TP = KH + TT, AQ = TP + CW * LT * 2;  // T'^T [16][LT], A_qk [16][LT]
-    static constexpr uint32_t L = AQ + CW * LT * 2;                 // L = diag(b) A_kk, f32 [16][LLW]
-    static constexpr uint32_t RK = L + CW * LLW * 4, RQ = RK + 64, BB = RQ + 64, PART = BB + 64, GAM = PART + 256;
+    static constexpr uint32_t L = AQ + CW * LT * 2;                 // L = diag(b) A_kk, f32 [16][LL]
+    static constexpr uint32_t RK = L + CW * LL * 4, RQ = RK + 64, BB = RQ + 64, PART = BB + 64, GAM = PART + 256;
     static constexpr uint32_t BYTES = (GAM + DK2 * 4 + 127) / 128 * 128;
     static_assert(CW * LW * 2 <= TT && CW * 65 * 4 <= 2 * TT, "aliases over X^T (and Y^T)");
     static_assert(L % 16 == 0 && RK % 16 == 0 && RQ % 16 == 0, "rows read 16 bytes at a time");
@@ -254,7 +253,7 @@ __global__ void __launch_bounds__(64, 5) kda_chunk_warp64_kernel(const ChunkPara
                     const int r = g8 + 8 * hi, s_ = 8 * j + 2 * t4;
                     if (w == 0) {
                         const float br = bb[r];
-                        *reinterpret_cast<float2 *>(Lf + r * LLW + s_) = make_float2(
+                        *reinterpret_cast<float2 *>(Lf + r * LL + s_) = make_float2(
                             s_ < r ? br * acc[j][2 * hi] : 0.f, s_ + 1 < r ? br * acc[j][2 * hi + 1] : 0.f);
                     } else {
                         stb2(sm + Ly::AQ + (r * LT + s_) * 2, s_ <= r ? acc[j][2 * hi] : 0.f,
@@ -282,7 +281,7 @@ __global__ void __launch_bounds__(64, 5) kda_chunk_warp64_kernel(const ChunkPara
                 }
                 akk *= rk[r] * rk[s_];
                 aqk *= rq[r] * rk[s_];
-                if (s_ < r) Lf[r * LLW + s_] = bb[r] * akk;
+                if (s_ < r) Lf[r * LL + s_] = bb[r] * akk;
                 reinterpret_cast<__nv_bfloat16 *>(sm + Ly::AQ)[r * LT + s_] = __float2bfloat16_rn(aqk);
             }
         }
@@ -297,7 +296,7 @@ __global__ void __launch_bounds__(64, 5) kda_chunk_warp64_kernel(const ChunkPara
                 float acc = i == j ? 1.f : 0.f;
 #pragma unroll
                 for (int k4 = 0; k4 < i; k4 += 4) {
-                    const float4 l4 = *reinterpret_cast<const float4 *>(Lf + i * LLW + k4);
+                    const float4 l4 = *reinterpret_cast<const float4 *>(Lf + i * LL + k4);
                     acc = fmaf(-l4.x, t[k4], acc);
                     if (k4 + 1 < i) acc = fmaf(-l4.y, t[k4 + 1], acc);
                     if (k4 + 2 < i) acc = fmaf(-l4.z, t[k4 + 2], acc);
@@ -471,7 +470,6 @@ cudaError_t launch_t(const ChunkParams &p, cudaStream_t st) {
 // v = 0, N starts from zero and sees v; the outputs [scale M^T q^ | scale N^T q^] go out
 // in fp32 rows of DV and the final state as [32][DV].
 namespace w2 {
-constexpr int LL2 = 20;  // row of the fp32 L tile: 80 B, so a row is read four values at a time
 template <int DV>
 struct Lay {
     static constexpr int LV = DV + 8;
@@ -482,8 +480,8 @@ struct Lay {
     static constexpr uint32_t X = 2 * IN, Y = X + TT, XQ = Y + TT, KT = XQ + TT, QT = KT + TT, KH = QT + TT;
     static constexpr uint32_t W = X;  // -W [16][LK] over X^T (after the A products)
     static constexpr uint32_t TP = KH + TT, AQ = TP + CW * LT * 2;  // T'^T [16][LT], A_qk [16][LT]
-    static constexpr uint32_t L = AQ + CW * LT * 2;                  // L = diag(b) A_kk, f32 [16][LL2]
-    static constexpr uint32_t RK = L + CW * LL2 * 4, RQ = RK + 64, BB = RQ + 64, GAM = BB + 64, XG = GAM + DK * 4;
+    static constexpr uint32_t L = AQ + CW * LT * 2;                  // L = diag(b) A_kk, f32 [16][LL]
+    static constexpr uint32_t RK = L + CW * LL * 4, RQ = RK + 64, BB = RQ + 64, GAM = BB + 64, XG = GAM + DK * 4;
     static constexpr uint32_t BYTES = (XG + 2 * DK * 4 + 127) / 128 * 128;
     static_assert(CW * LK * 2 <= TT && CW * 33 * 4 <= 2 * TT, "aliases over X^T (and Y^T)");
     static_assert(L % 16 == 0 && RK % 16 == 0 && RQ % 16 == 0, "rows read 16 bytes at a time");
@@ -665,7 +663,7 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
                     const int r = g8 + 8 * hi, s_ = 8 * j + 2 * t4;
                     if (w == 0) {
                         const float br = bb[r];
-                        *reinterpret_cast<float2 *>(Lf + r * LL2 + s_) = make_float2(
+                        *reinterpret_cast<float2 *>(Lf + r * LL + s_) = make_float2(
                             s_ < r ? br * acc[j][2 * hi] : 0.f, s_ + 1 < r ? br * acc[j][2 * hi + 1] : 0.f);
                     } else {
                         stb2(sm + Ly::AQ + (r * LT + s_) * 2, s_ <= r ? acc[j][2 * hi] : 0.f,
@@ -693,7 +691,7 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
                 }
                 akk *= rk[r] * rk[s_];
                 aqk *= rq[r] * rk[s_];
-                if (s_ < r) Lf[r * LL2 + s_] = bb[r] * akk;
+                if (s_ < r) Lf[r * LL + s_] = bb[r] * akk;
                 reinterpret_cast<__nv_bfloat16 *>(sm + Ly::AQ)[r * LT + s_] = __float2bfloat16_rn(aqk);
             }
         }
@@ -708,7 +706,7 @@ __global__ void __launch_bounds__(64, 7) kda_chunk_pair_kernel(const ChunkParams
                 float acc = i == j ? 1.f : 0.f;
 #pragma unroll
                 for (int k4 = 0; k4 < i; k4 += 4) {
-                    const float4 l4 = *reinterpret_cast<const float4 *>(Lf + i * LL2 + k4);
+                    const float4 l4 = *reinterpret_cast<const float4 *>(Lf + i * LL + k4);
                     acc = fmaf(-l4.x, t[k4], acc);
                     if (k4 + 1 < i) acc = fmaf(-l4.y, t[k4 + 1], acc);
                     if (k4 + 2 < i) acc = fmaf(-l4.z, t[k4 + 2], acc);
@@ -927,8 +925,8 @@ struct Lay {
     static constexpr uint32_t VS = 2 * QKG, VSZ = CW * LV * 2;  // two v stages [16][LV]
     static constexpr uint32_t TT = DK * LT * 2;                 // a transposed tile [32][LT]
     static constexpr uint32_t X = VS + 2 * VSZ, Y = X + TT, XQ = Y + TT, KT = XQ + TT;
-    static constexpr uint32_t L = KT + TT;                      // f32 [16][LL2]
-    static constexpr uint32_t RK = L + CW * w2::LL2 * 4, RQ = RK + 64, BB = RQ + 64;
+    static constexpr uint32_t L = KT + TT;                      // f32 [16][LL]
+    static constexpr uint32_t RK = L + CW * LL * 4, RQ = RK + 64, BB = RQ + 64;
     // hand-off buffer b at HB + b HSZ: Qtil^T [32][LT], Khat^T [32][LT], A_qk [16][LT],
     // T'^T [16][LT], -W [16][LK], e^{G_last} [32]
     static constexpr uint32_t HB = BB + 64;
@@ -1038,12 +1036,18 @@ __global__ void __maxnreg__(144) kda_chunk_pc_kernel(const ChunkParams p, __nv_b
                 const __nv_bfloat16 *qr = reinterpret_cast<const __nv_bfloat16 *>(sm + st + Ly::Q);
 #pragma unroll
                 for (int h8 = 0; h8 < 2; ++h8) {
+                    const float4 rka = *reinterpret_cast<const float4 *>(rk + 8 * h8);
+                    const float4 rkb = *reinterpret_cast<const float4 *>(rk + 8 * h8 + 4);
+                    const float4 rqa = *reinterpret_cast<const float4 *>(rq + 8 * h8);
+                    const float4 rqb = *reinterpret_cast<const float4 *>(rq + 8 * h8 + 4);
+                    const float rkv[8] = {rka.x, rka.y, rka.z, rka.w, rkb.x, rkb.y, rkb.z, rkb.w};
+                    const float rqv[8] = {rqa.x, rqa.y, rqa.z, rqa.w, rqb.x, rqb.y, rqb.z, rqb.w};
                     float x[8], y[8], xq[8], kt[8], qt[8], kc[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const int r = 8 * h8 + u;
-                        const float kh = __bfloat162float(kr[r * DK + lane]) * rk[r];
-                        const float qh = __bfloat162float(qr[r * DK + lane]) * rq[r];
+                        const float kh = __bfloat162float(kr[r * DK + lane]) * rkv[u];
+                        const float qh = __bfloat162float(qr[r * DK + lane]) * rqv[u];
                         const float dm = G[r] - Gm;
                         steep |= fabsf(dm) > kSpan;
                         const float em = e2(dm), en = e2(-dm), eg = e2(G[r]), ec = e2(GC - G[r]);
@@ -1083,7 +1087,7 @@ __global__ void __maxnreg__(144) kda_chunk_pc_kernel(const ChunkParams p, __nv_b
                     for (int hi = 0; hi < 2; ++hi) {
                         const int r = g8 + 8 * hi, s_ = 8 * j + 2 * t4;
                         const float br = bb[r];
-                        *reinterpret_cast<float2 *>(Lf + r * w2::LL2 + s_) =
+                        *reinterpret_cast<float2 *>(Lf + r * LL + s_) =
                             make_float2(s_ < r ? br * akk[j][2 * hi] : 0.f, s_ + 1 < r ? br * akk[j][2 * hi + 1] : 0.f);
                         stb2(sm + hb + Ly::HAQ + (r * LT + s_) * 2, s_ <= r ? aqk[j][2 * hi] : 0.f,
                              s_ + 1 <= r ? aqk[j][2 * hi + 1] : 0.f);
@@ -1109,7 +1113,7 @@ __global__ void __maxnreg__(144) kda_chunk_pc_kernel(const ChunkParams p, __nv_b
                     }
                     akk *= rk[r] * rk[s_];
                     aqk *= rq[r] * rk[s_];
-                    if (s_ < r) Lf[r * w2::LL2 + s_] = bb[r] * akk;
+                    if (s_ < r) Lf[r * LL + s_] = bb[r] * akk;
                     reinterpret_cast<__nv_bfloat16 *>(sm + hb + Ly::HAQ)[r * LT + s_] = __float2bfloat16_rn(aqk);
                 }
             }
@@ -1124,7 +1128,7 @@ __global__ void __maxnreg__(144) kda_chunk_pc_kernel(const ChunkParams p, __nv_b
                     float acc = i == j ? 1.f : 0.f;
 #pragma unroll
                     for (int k4 = 0; k4 < i; k4 += 4) {
-                        const float4 l4 = *reinterpret_cast<const float4 *>(Lf + i * w2::LL2 + k4);
+                        const float4 l4 = *reinterpret_cast<const float4 *>(Lf + i * LL + k4);
                         acc = fmaf(-l4.x, t[k4], acc);
                         if (k4 + 1 < i) acc = fmaf(-l4.y, t[k4 + 1], acc);
                         if (k4 + 2 < i) acc = fmaf(-l4.z, t[k4 + 2], acc);
